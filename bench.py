@@ -1,0 +1,475 @@
+#!/usr/bin/env python
+"""Throughput of the pi-attention forward operator on B200, one JSON line.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl reference]
+
+A step is one call of the operator (the whole hot path: gate, window and skip logits, single
+softmax, P.V, epilogue) over one batch of the workload, inputs resident in HBM.  The default
+workload is bf16_n4k (bf16, B=1 H=8 n=4096 d=64, window 128, period 64, 4 skips); the other
+workloads of pi_synth.WORKLOADS can be timed with --workload.  The L2 is flushed (a 256 MiB
+write) before every timed step, outside the step's events.
+
+Multi-GPU (torchrun, one process per GPU): every rank runs its own batch of the same workload
+(weak scaling: (b, h) problems are independent, there is no data exchange); the time is the max
+over ranks and the throughput counts the tokens of all ranks.
+
+--impl reference times the fp64 CPU oracle on the host cores on a bounded sample of the same
+workload (the comparison arm).  bench.py is the only product-side file that runs the oracle, and
+only for that arm and for the cpu_baseline field.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+import pi_synth as ps  # noqa: E402
+
+DEFAULT_WORKLOAD = "bf16_n4k"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+L2_FLUSH_BYTES = 256 << 20
+
+
+# ------------------------------------------------------------------------------------------------
+# algorithmic work (only keys in the index sets count; no tile padding)
+# ------------------------------------------------------------------------------------------------
+
+def index_totals(n: int, k: int, pi: int, S: int):
+    """Sum over i < n of |L(i)| and |P(i)| (closed forms of the index rule)."""
+    sl = n * (n + 1) // 2 if n <= k + 1 else (k + 1) * (k + 2) // 2 + (n - k - 1) * (k + 1)
+    sp = sum(max(0, n - m * pi) for m in range(k // pi + 1, S + 1))
+    return sl, sp
+
+
+def work(w):
+    """(tokens, algorithmic flops, algorithmic HBM bytes) of one step of workload w."""
+    es = 2 if w.dtype == "bf16" else 4
+    if w.kind == "prefill":
+        sl, sp = index_totals(w.n, w.k, w.pi, w.S)
+        units = w.B * w.H
+        flops = units * (4 * w.d * (sl + sp) + 2 * w.d * w.n)
+        bytes_ = units * (4 * w.n * w.d * es + 4 * w.n)
+        return w.B * w.n, flops, bytes_
+    i = w.n - 1
+    nl = min(i, w.k) + 1
+    npk = sum(1 for m in range(w.k // w.pi + 1, w.S + 1) if i - m * w.pi >= 0)
+    units = w.B * w.H
+    flops = units * (4 * w.d * (nl + npk) + 2 * w.d)
+    bytes_ = units * (2 * (nl + npk) * w.d * es + 2 * w.d * es + 4)
+    return w.B, flops, bytes_
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def source_hash() -> str:
+    h = hashlib.sha256()
+    for sub in ("periodic_sparse_attention_b200/csrc", "include"):
+        base = os.path.join(ROOT, sub)
+        for fn in sorted(os.listdir(base)):
+            if fn.endswith((".cu", ".cuh", ".h")):
+                with open(os.path.join(base, fn), "rb") as f:
+                    h.update(fn.encode() + b"\0" + f.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(workload: str):
+    """DRAM bytes per launch of the timed kernel from the committed ncu summaries, if they were
+    taken on the current kernel source (a line `bench-traffic: workload=.. bytes_per_launch=..
+    source_sha=..` in profiles/*.md); otherwise None."""
+    d = os.path.join(ROOT, "profiles")
+    if not os.path.isdir(d):
+        return None
+    want = source_hash()
+    for fn in sorted(os.listdir(d)):
+        if not fn.endswith((".md", ".txt")):
+            continue
+        with open(os.path.join(d, fn)) as f:
+            for line in f:
+                if line.startswith("bench-traffic:"):
+                    kv = dict(x.split("=", 1) for x in line.split()[1:] if "=" in x)
+                    if kv.get("workload") == workload and kv.get("source_sha") == want:
+                        return int(kv["bytes_per_launch"])
+    return None
+
+
+# ------------------------------------------------------------------------------------------------
+# clocks during the timed region (NVML reads only; nothing is set)
+# ------------------------------------------------------------------------------------------------
+
+class ClockSampler:
+    def __init__(self, device_index: int, period_s: float = 0.002):
+        self.samples, self.reasons, self.max_mhz = [], set(), None
+        self._stop = threading.Event()
+        self._period = period_s
+        self._t = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self._nv = pynvml
+            self._h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+        except Exception:  # no NVML: report no samples
+            self._nv = None
+
+    def _reason_names(self, mask):
+        nv = self._nv
+        names = {
+            "hw_slowdown": nv.nvmlClocksEventReasonHwSlowdown,
+            "hw_thermal_slowdown": nv.nvmlClocksEventReasonHwThermalSlowdown,
+            "sw_thermal_slowdown": nv.nvmlClocksEventReasonSwThermalSlowdown,
+            "sw_power_cap": nv.nvmlClocksEventReasonSwPowerCap,
+            "hw_power_brake_slowdown": nv.nvmlClocksEventReasonHwPowerBrakeSlowdown,
+            "applications_clocks_setting": nv.nvmlClocksEventReasonApplicationsClocksSetting,
+        }
+        return {k for k, bit in names.items() if mask & bit}
+
+    def _sample(self):
+        nv = self._nv
+        self.samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
+        self.reasons |= self._reason_names(nv.nvmlDeviceGetCurrentClocksEventReasons(self._h))
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self._sample()
+            except Exception:
+                return
+            time.sleep(self._period)
+
+    def __enter__(self):
+        if self._nv is not None:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self._t is not None:
+            self._stop.set()
+            self._t.join()
+            try:
+                self._sample()
+            except Exception:
+                pass
+
+    def summary(self):
+        med = statistics.median(self.samples) if self.samples else None
+        return {"sm_mhz": med, "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons),
+                "samples": len(self.samples)}
+
+
+# ------------------------------------------------------------------------------------------------
+# the oracle on the host (reference arm and cpu_baseline)
+# ------------------------------------------------------------------------------------------------
+
+def oracle_sample(w, budget_s: float, seed: int = 0):
+    """Time the fp64 oracle on a bounded sample of workload w's query rows, using all host cores.
+    Returns (tokens per second, sample description, threads, seconds)."""
+    import oracle
+    threads = max(1, os.cpu_count() or 1)
+    if w.kind == "prefill":
+        inp = ps.prefill_inputs(w, seed)
+        total = w.B * w.H * w.n
+        rng = np.random.default_rng(seed)
+
+        def run(rows):
+            t0 = time.perf_counter()
+            oracle.fwd_rows(inp["q"], inp["k"], inp["v"], inp["w_g"], inp["b_g"], w.k, w.pi, w.S, rows=rows,
+                            nthreads=threads)
+            return time.perf_counter() - t0
+
+        probe = np.sort(rng.choice(total, size=min(total, 4 * threads), replace=False))
+        tp = max(run(probe), 1e-6) / probe.size
+        count = int(min(total, max(probe.size, budget_s / tp)))
+        rows = np.arange(total) if count == total else np.sort(rng.choice(total, size=count, replace=False))
+        sec = run(rows)
+        rows_per_token = w.H  # a token is one query position of one sequence: H rows
+        desc = f"{count} of {total} query rows ({'all' if count == total else 'uniform sample'})"
+        return count / rows_per_token / sec, desc, threads, sec
+    # decode: every (b, h) reads its own ~1k cache rows
+    inp = ps.decode_inputs(w, seed)
+    n, d = w.n, w.d
+    count = 0
+    t_total = 0.0
+    bh_all = np.random.default_rng(seed).permutation(w.B * w.H)
+    for bh in bh_all:
+        b, h = divmod(int(bh), w.H)
+        ks = np.full((1, 1, n, d), 0xFFFF, dtype=np.uint16)
+        vs = np.full((1, 1, n, d), 0xFFFF, dtype=np.uint16)
+        ks[0, 0, inp["pos"]] = inp["kc"][b, h]
+        vs[0, 0, inp["pos"]] = inp["vc"][b, h]
+        t0 = time.perf_counter()
+        oracle.decode(inp["q"][b, h][None, None], ks, vs, inp["w_g"][h][None], inp["b_g"][h][None], w.k, w.pi, w.S,
+                      nthreads=threads)
+        t_total += time.perf_counter() - t0
+        count += 1
+        if t_total > budget_s:
+            break
+    desc = f"{count} of {w.B * w.H} (b, h) decode queries"
+    return count / w.H / t_total, desc, threads, t_total
+
+
+# ------------------------------------------------------------------------------------------------
+# GPU arm
+# ------------------------------------------------------------------------------------------------
+
+def dist_env():
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", str(rank)))
+    return rank, world, local
+
+
+def max_over_ranks(value: float, world: int, device=None) -> float:
+    if world == 1:
+        return value
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def device_inputs(w, seed, torch, device):
+    def dev(a, dtype):
+        if dtype == "bf16":
+            return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).to(device).view(torch.bfloat16)
+        return torch.from_numpy(np.ascontiguousarray(a)).to(device)
+
+    if w.kind == "prefill":
+        inp = ps.prefill_inputs(w, seed)
+        host = {k: inp[k] for k in ("q", "k", "v", "w_g", "b_g")}
+        t = {k: dev(inp[k], w.dtype) for k in ("q", "k", "v")}
+        t["w_g"] = torch.from_numpy(inp["w_g"]).to(device)
+        t["b_g"] = torch.from_numpy(inp["b_g"]).to(device)
+        return t, host
+    inp = ps.decode_inputs(w, seed)
+    pos = torch.from_numpy(inp["pos"]).to(device)
+    t = {"q": dev(inp["q"], w.dtype), "w_g": torch.from_numpy(inp["w_g"]).to(device),
+         "b_g": torch.from_numpy(inp["b_g"]).to(device)}
+    tdt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
+    for name, rows in (("k", inp["kc"]), ("v", inp["vc"])):
+        c = torch.empty((w.B, w.H, w.n, w.d), dtype=tdt, device=device)
+        c.view(torch.int16 if w.dtype == "bf16" else torch.int32).fill_(-1)
+        c[:, :, pos] = dev(rows, w.dtype)
+        t[name] = c
+    return t, {"q": inp["q"], "w_g": inp["w_g"], "b_g": inp["b_g"]}
+
+
+def run_gpu(args):
+    import torch
+    import periodic_sparse_attention_b200 as pia
+    from periodic_sparse_attention_b200 import build as pbuild
+
+    rank, world, local = dist_env()
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    if rank == 0 or world == 1:
+        pbuild.build()
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    pia.load()
+
+    w = ps.WORKLOADS[args.workload]
+    tokens, flops, bytes_ = work(w)
+    t, host = device_inputs(w, args.seed + rank, torch, device)
+    out = torch.empty_like(t["q"])
+    lse_shape = (w.B, w.H, w.n) if w.kind == "prefill" else (w.B, w.H)
+    lse = torch.empty(lse_shape, dtype=torch.float32, device=device)
+    stream = torch.cuda.current_stream(device)
+
+    if w.kind == "prefill":
+        def step():
+            pia.pi_attn_fwd(t["q"], t["k"], t["v"], t["w_g"], t["b_g"], w.k, w.pi, w.S, out=out, lse=lse,
+                            stream=stream)
+        launches_per_step = 1
+    else:
+        def step():
+            pia.pi_attn_decode(t["q"], t["k"], t["v"], t["w_g"], t["b_g"], w.k, w.pi, w.S, out=out, lse=lse,
+                               stream=stream)
+        launches_per_step = 1  # one kernel when (b, h) fill the GPU (no split)
+
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
+    for _ in range(args.warmup):
+        flush.fill_(1)
+        step()
+    pia.pi_attn_check(stream)
+
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    torch.cuda.synchronize(device)
+    with ClockSampler(local) as clocks:
+        for s in range(args.steps):
+            flush.fill_(s & 0xFF)
+            starts[s].record(stream)
+            step()
+            ends[s].record(stream)
+        torch.cuda.synchronize(device)
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    pia.pi_attn_check(stream)
+    per_step_ms = [a.elapsed_time(b) for a, b in zip(starts, ends)]
+    total_ms = max_over_ranks(sum(per_step_ms), world, device)
+    ms_per_step = total_ms / args.steps
+    value = tokens * world / (total_ms / 1e3 / args.steps)
+
+    # end to end through the public call: pinned host inputs -> device, the call, results -> host
+    e2e = None
+    if w.kind == "prefill":
+        hq = {k: torch.from_numpy(np.ascontiguousarray(host[k]).view(np.int16) if w.dtype == "bf16"
+                                  else np.ascontiguousarray(host[k])).pin_memory() for k in ("q", "k", "v")}
+        hw = {k: torch.from_numpy(host[k]).pin_memory() for k in ("w_g", "b_g")}
+        h_out = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+        h_lse = torch.empty(lse.shape, dtype=torch.float32).pin_memory()
+        dq = {k: t[k].view(torch.int16) if w.dtype == "bf16" else t[k] for k in ("q", "k", "v")}
+        e_steps = max(3, min(args.steps, 50))
+        h2d = sum(x.numel() * x.element_size() for x in hq.values()) + sum(
+            x.numel() * x.element_size() for x in hw.values())
+        d2h = h_out.numel() * h_out.element_size() + h_lse.numel() * 4
+
+        def e2e_step():
+            for k in ("q", "k", "v"):
+                dq[k].copy_(hq[k], non_blocking=True)
+            t["w_g"].copy_(hw["w_g"], non_blocking=True)
+            t["b_g"].copy_(hw["b_g"], non_blocking=True)
+            step()
+            h_out.copy_(out, non_blocking=True)
+            h_lse.copy_(lse, non_blocking=True)
+
+        for _ in range(2):
+            e2e_step()
+        torch.cuda.synchronize(device)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(e_steps):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize(device)
+        e_ms = max_over_ranks(e0.elapsed_time(e1), world, device) / e_steps
+        e2e = {"value": tokens * world / (e_ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": int(h2d),
+               "d2h_bytes_per_step": int(d2h), "ms_per_step": e_ms}
+    pia.pi_attn_check(stream)
+
+    peaks, peak_kind = load_peaks()
+    ai = flops / bytes_
+    ridge = peaks["bf16_tflops"] * 1e12 / (peaks["hbm_gbs"] * 1e9)
+    launch_s = statistics.mean(per_step_ms) / 1e3 / launches_per_step
+    if ai < ridge:
+        achieved = bytes_ / launch_s / 1e9
+        roof = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s"}
+    else:
+        achieved = flops / launch_s / 1e12
+        roof = {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s"}
+    roof["frac"] = roof["achieved"] / roof["peak"]
+    roof["traffic"] = profiled_traffic(w.name)
+    roof["peak_source"] = f"{peak_kind} ({'MEASURED_PEAKS.json' if peak_kind == 'measured' else 'recipe fallback'})"
+    roof["algorithmic_bytes"] = bytes_
+    roof["algorithmic_flops"] = flops
+    roof["kernel_ms"] = launch_s * 1e3
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        v, desc, threads, sec = oracle_sample(w, args.cpu_budget)
+        cpu = {"value": v, "unit": "tokens/s", "cores": threads, "kind": "oracle", "sample": desc,
+               "seconds": round(sec, 3)}
+
+    line = {
+        "metric": "pi-attention fwd tokens/s (and % of roofline), 1xB200" if w.kind == "prefill"
+        else "pi-attention decode tokens/s (HBM GB/s roofline), 1xB200",
+        "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": w.dtype, "data": "synthetic (seeded Philox normals, workload recipe)",
+        "config": dict(w.describe(), l2="flushed before every timed step (256 MiB write)",
+                       parallelism=f"replicas x{world} (independent (b, h) batches)"),
+        "achieved_tflops": flops / launch_s / 1e12, "achieved_gbs": bytes_ / launch_s / 1e9,
+        "roofline": roof, "cpu_baseline": cpu, "e2e": e2e,
+        "gpu_launches": launches_per_step * args.steps, "clocks": clocks.summary(),
+        "kernel_source_sha": source_hash(),
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    del t, flush
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def run_reference(args):
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return
+    w = ps.WORKLOADS[args.workload]
+    tokens, flops, bytes_ = work(w)
+    budget = max(0.2, min(args.cpu_budget, 120.0 / max(1, args.steps + args.warmup)))
+    for _ in range(args.warmup):
+        oracle_sample(w, budget)
+    vals, secs, desc, threads = [], [], "", 0
+    for _ in range(args.steps):
+        v, desc, threads, sec = oracle_sample(w, budget)
+        vals.append(v)
+        secs.append(sec)
+    value = statistics.mean(vals)
+    line = {
+        "impl": "reference",
+        "metric": "pi-attention fwd tokens/s (and % of roofline), 1xB200" if w.kind == "prefill"
+        else "pi-attention decode tokens/s (HBM GB/s roofline), 1xB200",
+        "value": value, "unit": "tokens/s", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": statistics.mean(secs) * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded Philox normals, workload recipe)",
+        "config": dict(w.describe(), l2="n/a (host)", parallelism="host threads"),
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": threads, "kind": "oracle", "sample": desc},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "gpu_launches": 0,
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(ps.WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--cpu-budget", type=float, default=10.0, help="seconds of oracle work for cpu_baseline")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    args.warmup = max(3, args.warmup)  # at least 3 untimed warm-up steps
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_gpu(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,114 @@
+/*
+ * pi_attn.h -- C ABI of the pi-attention forward operator for NVIDIA B200 (sm_100a).
+ *
+ * The operator ("pi-Attention: Periodic Sparse Transformers for Efficient Long-Context Modeling",
+ * gist.science summary, section 2 "Methodology", Core Components): every query row i of every
+ * (batch b, head h) attends, under ONE softmax, to the union of
+ *   - its causal ring-local window  L(i) = { j : max(0, i - k) <= j <= i }  (itself + k before),
+ *   - its periodic backward skips   P(i) = { i - m*pi : 1 <= m <= S, m*pi > k, i - m*pi >= 0 }
+ *     (a skip that lands inside the window is dropped, so every key is counted once),
+ * with a per-token, per-head gate alpha = sigmoid(q_i . w_g[h] + b_g[h]) on the unscaled query,
+ * added as a log-prior: log(alpha) on window logits, log(1 - alpha) on skip logits, before the
+ * softmax (section "Dynamic Adaptive Fusion").  Logits are scaled by tau = 1/sqrt(d); the prior
+ * is not scaled.  Outputs:
+ *   out_i = sum_j softmax_j(s) v_j          lse_i = ln sum_j exp(s_j)   (natural log)
+ *
+ * Conventions shared by every entry point
+ *   - Tensors are contiguous, row-major, innermost dimension d.  q/k/v/out of prefill are
+ *     [B, H, n, d]; decode q/out are [B, H, d] and the caches [B, H, n_cache, d]; lse is [B, H, n]
+ *     (prefill) or [B, H] (decode), fp32.  w_g is [H, d] fp32, b_g is [H] fp32.
+ *   - dtype names the storage type of q, k, v, caches and out: PI_ATTN_F32 (fp32) or PI_ATTN_BF16
+ *     (bfloat16).  Arithmetic is fp32 (bf16 products on tensor cores accumulate in fp32); out is
+ *     rounded once, to nearest even, into dtype.
+ *   - All pointers are DEVICE pointers owned by the caller; the library keeps no reference after
+ *     the call returns and holds no allocation of its own between calls.  Tensor pointers must be
+ *     16-byte aligned and d * sizeof(dtype) a multiple of 16 bytes.
+ *   - `stream` is a cudaStream_t (NULL: the legacy default stream).  Calls only enqueue work: they
+ *     are asynchronous and stream-ordered.  Argument errors are returned synchronously and then
+ *     nothing is enqueued.  Errors that only a kernel can see (a cache length out of range, an
+ *     internal wait that gave up) set a device-side error word that pi_attn_check() reads.
+ *   - Entry points are thread-safe; the device error word is shared by all streams of a device.
+ */
+#ifndef PI_ATTN_H
+#define PI_ATTN_H
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    PI_ATTN_OK = 0,
+    PI_ATTN_EINVAL = 1,        /* invalid argument: null pointer, size out of range, misalignment */
+    PI_ATTN_EUNSUPPORTED = 2,  /* valid request this build does not implement (e.g. head size) */
+    PI_ATTN_ECUDA = 3,         /* a CUDA runtime call or kernel launch failed */
+    PI_ATTN_EDEVICE = 4        /* a kernel reported an error through the device error word */
+} pi_attn_status;
+
+typedef enum { PI_ATTN_F32 = 0, PI_ATTN_BF16 = 1 } pi_attn_dtype;
+
+/* Kernel choice for pi_attn_fwd_ex. */
+typedef enum {
+    PI_ATTN_PATH_AUTO = 0,  /* tensor-core kernel where it applies (bf16, d in {64, 128}), else SIMT */
+    PI_ATTN_PATH_SIMT = 1,  /* CUDA-core kernel: every dtype, d <= 256 */
+    PI_ATTN_PATH_TC = 2     /* tcgen05/TMEM kernel only; PI_ATTN_EUNSUPPORTED where it does not apply */
+} pi_attn_path;
+
+/* Prefill forward.  Cited passage: the Core Components (window, skips, gate as log-prior, one
+ * softmax over the union) and "Execution & Scheduling" (local sweep on tensor cores, periodic
+ * strided gather, fusion) of the pi-Attention method section.
+ *   q, k, v   [B, H, n, d] in dtype                        (read)
+ *   w_g [H, d], b_g [H]  fp32 gate parameters               (read)
+ *   out       [B, H, n, d] in dtype                         (written)
+ *   lse       [B, H, n] fp32, natural log; may be NULL     (written)
+ *   B, H, n >= 1; d: multiple of 4 (fp32) or 8 (bf16), 1..256; k_win >= 0; pi >= 1; S >= 0.
+ * Returns PI_ATTN_OK once the work is enqueued. */
+pi_attn_status pi_attn_fwd(const void* q, const void* k, const void* v, const float* w_g, const float* b_g,
+                           void* out, float* lse, int B, int H, int n, int d, int k_win, int pi, int S,
+                           pi_attn_dtype dtype, void* stream);
+
+/* pi_attn_fwd with an explicit kernel choice (see pi_attn_path).  Same arguments and results. */
+pi_attn_status pi_attn_fwd_ex(const void* q, const void* k, const void* v, const float* w_g, const float* b_g,
+                              void* out, float* lse, int B, int H, int n, int d, int k_win, int pi, int S,
+                              pi_attn_dtype dtype, pi_attn_path path, void* stream);
+
+/* Single-step decode.  Cited passage: "Inference" under "Execution & Scheduling" of the
+ * pi-Attention method section (a new token reads its window and its periodic skips).  For each
+ * (b, h) the query q[b, h] is the token at position len_b - 1 of a cache that already holds it,
+ * with len_b = cache_len[b] (or n_cache when cache_len is NULL); it attends to cache rows by the
+ * prefill rule.  Cache rows outside the window and skips are never read.
+ *   q        [B, H, d] dtype                  kcache, vcache [B, H, n_cache, d] dtype
+ *   w_g, b_g as for prefill                   cache_len: device int32 [B] or NULL
+ *   out      [B, H, d] dtype                  lse: [B, H] fp32 or NULL
+ * A cache_len entry outside [1, n_cache] sets the device error word (read by pi_attn_check) and
+ * that sequence's out/lse are written as NaN. */
+pi_attn_status pi_attn_decode(const void* q, const void* kcache, const void* vcache, const float* w_g,
+                              const float* b_g, const int* cache_len, void* out, float* lse, int B, int H,
+                              int n_cache, int d, int k_win, int pi, int S, pi_attn_dtype dtype, void* stream);
+
+/* Index sets as the kernels see them, for exact comparison.  For query rows i = 0..n-1:
+ *   counts [n, 2] int32: |L(i)|, |P(i)|
+ *   idx    [n, width] int32: L(i) ascending, then P(i) in order of increasing m, then -1.
+ * width must be >= k_win + 1 + S.  Both are device pointers. */
+pi_attn_status pi_attn_debug_index_sets(int n, int k_win, int pi, int S, int* counts, int* idx, int width,
+                                        void* stream);
+
+/* Synchronises `stream`, then reads and clears the device error word of the current device.
+ * Returns PI_ATTN_EDEVICE if any kernel set it since the last check (pi_attn_last_error() then
+ * describes the flags), PI_ATTN_ECUDA if the stream reports a CUDA error, else PI_ATTN_OK. */
+pi_attn_status pi_attn_check(void* stream);
+
+/* Static string naming a status code. */
+const char* pi_attn_status_string(pi_attn_status status);
+
+/* Description of the last error returned on the calling thread (static storage per thread; ""
+ * after a success). */
+const char* pi_attn_last_error(void);
+
+/* Library version as major*10000 + minor*100 + patch. */
+int pi_attn_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PI_ATTN_H */

@@ -1,0 +1,150 @@
+"""Python binding of libpiattn (include/pi_attn.h): argument marshalling only.
+
+Every step of the operator runs in the CUDA library; this module converts torch CUDA tensors to
+device pointers, passes the caller's current stream and turns status codes into exceptions.
+There is no CPU fallback: without the built library (or without a GPU) the calls raise.
+
+    import periodic_sparse_attention_b200 as pia
+    out, lse = pia.pi_attn_fwd(q, k, v, w_g, b_g, k_win=128, pi=64, S=4)
+    out, lse = pia.pi_attn_decode(q, kcache, vcache, w_g, b_g, k_win=1024, pi=2048, S=31)
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libpiattn.so")
+
+PI_ATTN_OK, PI_ATTN_EINVAL, PI_ATTN_EUNSUPPORTED, PI_ATTN_ECUDA, PI_ATTN_EDEVICE = range(5)
+PI_ATTN_F32, PI_ATTN_BF16 = 0, 1
+PATHS = {"auto": 0, "simt": 1, "tc": 2}
+
+# (name, restype, argtypes) of every symbol include/pi_attn.h declares
+_vp, _i32, _cstr = ctypes.c_void_p, ctypes.c_int, ctypes.c_char_p
+SIGNATURES = {
+    # 7 tensor pointers, B H n d k_win pi S, dtype, stream
+    "pi_attn_fwd": (_i32, [_vp] * 7 + [_i32] * 8 + [_vp]),
+    # ... as above plus the path selector
+    "pi_attn_fwd_ex": (_i32, [_vp] * 7 + [_i32] * 9 + [_vp]),
+    # 8 pointers (q kcache vcache w_g b_g cache_len out lse), B H n_cache d k_win pi S, dtype, stream
+    "pi_attn_decode": (_i32, [_vp] * 8 + [_i32] * 8 + [_vp]),
+    "pi_attn_debug_index_sets": (_i32, [_i32, _i32, _i32, _i32, _vp, _vp, _i32, _vp]),
+    "pi_attn_check": (_i32, [_vp]),
+    "pi_attn_status_string": (_cstr, [_i32]),
+    "pi_attn_last_error": (_cstr, []),
+    "pi_attn_version": (_i32, []),
+}
+
+_lib = None
+
+
+class PiAttnError(RuntimeError):
+    def __init__(self, status: int, msg: str):
+        super().__init__(f"{_status_name(status)}: {msg}")
+        self.status = status
+
+
+def _status_name(s):
+    return ["PI_ATTN_OK", "PI_ATTN_EINVAL", "PI_ATTN_EUNSUPPORTED", "PI_ATTN_ECUDA", "PI_ATTN_EDEVICE"][s] \
+        if 0 <= s < 5 else f"status {s}"
+
+
+def load(path: str = LIB_PATH):
+    """Load libpiattn.so (built by `build.build()`), declaring every exported signature."""
+    global _lib
+    if _lib is None or path != LIB_PATH:
+        if not os.path.exists(path):
+            raise ImportError(f"libpiattn.so not built at {path}; run python -m periodic_sparse_attention_b200.build")
+        lib = ctypes.CDLL(path)
+        for name, (res, args) in SIGNATURES.items():
+            fn = getattr(lib, name)
+            fn.restype = res
+            fn.argtypes = args
+        if path != LIB_PATH:
+            return lib
+        _lib = lib
+    return _lib
+
+
+def _raise(st: int):
+    if st != PI_ATTN_OK:
+        raise PiAttnError(st, load().pi_attn_last_error().decode())
+
+
+def _dtype_code(t) -> int:
+    import torch
+    if t.dtype == torch.float32:
+        return PI_ATTN_F32
+    if t.dtype == torch.bfloat16:
+        return PI_ATTN_BF16
+    raise TypeError(f"pi-attention tensors must be float32 or bfloat16, got {t.dtype}")
+
+
+def _stream(stream):
+    import torch
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("pi-attention tensors must be CUDA tensors")
+    if not t.is_contiguous():
+        raise ValueError("pi-attention tensors must be contiguous")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def pi_attn_fwd(q, k, v, w_g, b_g, k_win: int, pi: int, S: int, out=None, lse=None, *, path: str = "auto",
+                stream=None, want_lse: bool = True):
+    """Prefill forward on torch CUDA tensors q, k, v [B, H, n, d] (fp32 or bf16), w_g [H, d] and
+    b_g [H] (fp32).  Allocates out (q's dtype) and lse (fp32 [B, H, n]) when not given."""
+    import torch
+    B, H, n, d = q.shape
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None and want_lse:
+        lse = torch.empty((B, H, n), dtype=torch.float32, device=q.device)
+    st = load().pi_attn_fwd_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(w_g), _ptr(b_g), _ptr(out), _ptr(lse), B, H, n, d,
+                               k_win, pi, S, _dtype_code(q), PATHS[path], _stream(stream))
+    _raise(st)
+    return out, lse
+
+
+def pi_attn_decode(q, kcache, vcache, w_g, b_g, k_win: int, pi: int, S: int, cache_len=None, out=None, lse=None, *,
+                   stream=None, want_lse: bool = True):
+    """Decode step: q [B, H, d], caches [B, H, n_cache, d], optional cache_len int32 [B] (device)."""
+    import torch
+    B, H, d = q.shape
+    n_cache = kcache.shape[2]
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None and want_lse:
+        lse = torch.empty((B, H), dtype=torch.float32, device=q.device)
+    st = load().pi_attn_decode(_ptr(q), _ptr(kcache), _ptr(vcache), _ptr(w_g), _ptr(b_g), _ptr(cache_len), _ptr(out),
+                               _ptr(lse), B, H, n_cache, d, k_win, pi, S, _dtype_code(q), _stream(stream))
+    _raise(st)
+    return out, lse
+
+
+def pi_attn_debug_index_sets(n: int, k_win: int, pi: int, S: int, width: int | None = None, device="cuda",
+                             stream=None):
+    """Index sets as the kernels enumerate them: counts [n, 2] and idx [n, width] int32 tensors."""
+    import torch
+    width = k_win + 1 + S if width is None else width
+    counts = torch.empty((n, 2), dtype=torch.int32, device=device)
+    idx = torch.empty((n, width), dtype=torch.int32, device=device)
+    st = load().pi_attn_debug_index_sets(n, k_win, pi, S, _ptr(counts), _ptr(idx), width, _stream(stream))
+    _raise(st)
+    return counts, idx
+
+
+def pi_attn_check(stream=None):
+    """Synchronise the stream and raise if a kernel set the device error word."""
+    _raise(load().pi_attn_check(_stream(stream)))
+
+
+def pi_attn_version() -> int:
+    return load().pi_attn_version()

@@ -1,0 +1,228 @@
+// pi_attn.cu -- the C ABI (include/pi_attn.h): argument checks, kernel choice and launches.
+//
+// One translation unit holds every kernel so that they share the device error word.
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/pi_attn.h"
+#include "common.cuh"
+#include "decode.cuh"
+#include "fwd_simt.cuh"
+#include "fwd_tc.cuh"
+
+namespace {
+
+thread_local char g_msg[512] = "";
+
+pi_attn_status fail(pi_attn_status st, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_msg, sizeof g_msg, fmt, ap);
+  va_end(ap);
+  return st;
+}
+
+pi_attn_status ok() {
+  g_msg[0] = 0;
+  return PI_ATTN_OK;
+}
+
+pi_attn_status cuda_fail(cudaError_t e, const char* what) {
+  return fail(PI_ATTN_ECUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+size_t elem_size(pi_attn_dtype dt) { return dt == PI_ATTN_BF16 ? 2 : 4; }
+
+// Checks shared by prefill and decode.  n_kv is the sequence (prefill) or cache (decode) length.
+pi_attn_status check_common(const void* q, const void* k, const void* v, const float* w_g, const float* b_g,
+                            const void* out, int B, int H, int n_kv, int d, int k_win, int pi, int S,
+                            pi_attn_dtype dtype) {
+  if (!q || !k || !v || !w_g || !b_g || !out) return fail(PI_ATTN_EINVAL, "null tensor pointer");
+  if (dtype != PI_ATTN_F32 && dtype != PI_ATTN_BF16) return fail(PI_ATTN_EINVAL, "unknown dtype %d", (int)dtype);
+  if (B < 1 || H < 1 || n_kv < 1) return fail(PI_ATTN_EINVAL, "B, H and n must be >= 1 (got %d, %d, %d)", B, H, n_kv);
+  if (d < 1 || d > 256) return fail(PI_ATTN_EINVAL, "d must be in [1, 256] (got %d)", d);
+  if ((d * (int)elem_size(dtype)) % 16 != 0)
+    return fail(PI_ATTN_EINVAL, "d * sizeof(dtype) must be a multiple of 16 bytes (d = %d)", d);
+  if (k_win < 0 || pi < 1 || S < 0) return fail(PI_ATTN_EINVAL, "need k_win >= 0, pi >= 1, S >= 0");
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out))
+    return fail(PI_ATTN_EINVAL, "q, k, v and out must be 16-byte aligned");
+  const long long total = (long long)B * H * n_kv * d;
+  if (total / d / n_kv / H != B) return fail(PI_ATTN_EINVAL, "tensor size overflows");
+  return PI_ATTN_OK;
+}
+
+cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s); }
+
+int num_sms() {
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  return sms;
+}
+
+template <typename T, bool DECODE>
+pi_attn_status launch_simt(const void* q, const void* k, const void* v, const float* w_g, const float* b_g,
+                           const int* cache_len, void* out, float* lse, int B, int H, int n_q, int n_kv, int d,
+                           int k_win, int pi, int S, cudaStream_t st) {
+  const long long tasks = DECODE ? (long long)B * H : (long long)B * H * n_q;
+  const int warps_per_block = 8;
+  const long long blocks = (tasks + warps_per_block - 1) / warps_per_block;
+  if (blocks > 0x7fffffffLL) return fail(PI_ATTN_EINVAL, "too many query rows");
+  const float scale_log2 = (float)(1.0 / std::sqrt((double)d)) * pia::kLog2e;
+  pia::simt_attn_kernel<T, DECODE><<<(unsigned)blocks, warps_per_block * 32, 0, st>>>(
+      (const T*)q, (const T*)k, (const T*)v, w_g, b_g, cache_len, (T*)out, lse, B, H, n_q, n_kv, d, k_win, pi, S,
+      scale_log2);
+  cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? ok() : cuda_fail(e, "simt kernel launch");
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* pi_attn_status_string(pi_attn_status s) {
+  switch (s) {
+    case PI_ATTN_OK: return "PI_ATTN_OK";
+    case PI_ATTN_EINVAL: return "PI_ATTN_EINVAL";
+    case PI_ATTN_EUNSUPPORTED: return "PI_ATTN_EUNSUPPORTED";
+    case PI_ATTN_ECUDA: return "PI_ATTN_ECUDA";
+    case PI_ATTN_EDEVICE: return "PI_ATTN_EDEVICE";
+  }
+  return "PI_ATTN_<unknown>";
+}
+
+const char* pi_attn_last_error(void) { return g_msg; }
+
+int pi_attn_version(void) { return 100; }
+
+pi_attn_status pi_attn_fwd_ex(const void* q, const void* k, const void* v, const float* w_g, const float* b_g,
+                              void* out, float* lse, int B, int H, int n, int d, int k_win, int pi, int S,
+                              pi_attn_dtype dtype, pi_attn_path path, void* stream) {
+  pi_attn_status st = check_common(q, k, v, w_g, b_g, out, B, H, n, d, k_win, pi, S, dtype);
+  if (st != PI_ATTN_OK) return st;
+  if (path != PI_ATTN_PATH_AUTO && path != PI_ATTN_PATH_SIMT && path != PI_ATTN_PATH_TC)
+    return fail(PI_ATTN_EINVAL, "unknown path %d", (int)path);
+  const bool tc_ok = pia::tc_supported(dtype == PI_ATTN_BF16, d, n);
+  if (path == PI_ATTN_PATH_TC && !tc_ok)
+    return fail(PI_ATTN_EUNSUPPORTED, "tensor-core path covers bf16 with d in {64, 128} (got dtype %d, d %d)",
+                (int)dtype, d);
+  cudaStream_t s = as_stream(stream);
+  if (path != PI_ATTN_PATH_SIMT && tc_ok) {
+    const char* why = nullptr;
+    cudaError_t e = pia::launch_fwd_tc(q, k, v, w_g, b_g, out, lse, B, H, n, d, k_win, pi, S, s, &why);
+    if (e != cudaSuccess) return cuda_fail(e, why ? why : "tensor-core kernel launch");
+    return ok();
+  }
+  if (dtype == PI_ATTN_F32)
+    return launch_simt<float, false>(q, k, v, w_g, b_g, nullptr, out, lse, B, H, n, n, d, k_win, pi, S, s);
+  return launch_simt<__nv_bfloat16, false>(q, k, v, w_g, b_g, nullptr, out, lse, B, H, n, n, d, k_win, pi, S, s);
+}
+
+pi_attn_status pi_attn_fwd(const void* q, const void* k, const void* v, const float* w_g, const float* b_g,
+                           void* out, float* lse, int B, int H, int n, int d, int k_win, int pi, int S,
+                           pi_attn_dtype dtype, void* stream) {
+  return pi_attn_fwd_ex(q, k, v, w_g, b_g, out, lse, B, H, n, d, k_win, pi, S, dtype, PI_ATTN_PATH_AUTO, stream);
+}
+
+pi_attn_status pi_attn_decode(const void* q, const void* kcache, const void* vcache, const float* w_g,
+                              const float* b_g, const int* cache_len, void* out, float* lse, int B, int H,
+                              int n_cache, int d, int k_win, int pi, int S, pi_attn_dtype dtype, void* stream) {
+  pi_attn_status st = check_common(q, kcache, vcache, w_g, b_g, out, B, H, n_cache, d, k_win, pi, S, dtype);
+  if (st != PI_ATTN_OK) return st;
+  cudaStream_t s = as_stream(stream);
+  if (dtype == PI_ATTN_BF16 && (d == 64 || d == 128)) {
+    const long long bh = (long long)B * H;
+    if (bh > 0x7fffffffLL) return fail(PI_ATTN_EINVAL, "B * H too large");
+    // Split each (b, h) across CTAs only when there are too few (b, h) to fill the GPU.
+    const long long rows = (long long)k_win + 1 + S;
+    const long long want = 4LL * num_sms() * 14;  // ~14 two-warp CTAs per SM, four waves' worth
+    int nsplit = 1;
+    if (bh * 4 < want) {
+      long long ns = (want + bh - 1) / bh;
+      const long long max_ns = (rows + 127) / 128;  // keep >= 128 rows per split
+      if (ns > max_ns) ns = max_ns;
+      if (ns > 64) ns = 64;
+      nsplit = ns < 1 ? 1 : (int)ns;
+    }
+    pia::DecodeArgs a;
+    a.q = (const __nv_bfloat16*)q;
+    a.kc = (const __nv_bfloat16*)kcache;
+    a.vc = (const __nv_bfloat16*)vcache;
+    a.w_g = w_g;
+    a.b_g = b_g;
+    a.cache_len = cache_len;
+    a.out = (__nv_bfloat16*)out;
+    a.lse = lse;
+    a.part = nullptr;
+    a.H = H;
+    a.n_cache = n_cache;
+    a.kwin = k_win;
+    a.pi = pi;
+    a.S = S;
+    a.nsplit = nsplit;
+    a.scale_log2 = (float)(1.0 / std::sqrt((double)d)) * pia::kLog2e;
+    if (nsplit > 1) {
+      const size_t bytes = (size_t)bh * nsplit * (d + 2) * sizeof(float);
+      cudaError_t e = cudaMallocAsync((void**)&a.part, bytes, s);
+      if (e != cudaSuccess) return cuda_fail(e, "decode workspace allocation");
+    }
+    dim3 grid((unsigned)bh, (unsigned)nsplit);
+    if (d == 128) pia::decode_bf16_kernel<128><<<grid, 64, 0, s>>>(a);
+    else pia::decode_bf16_kernel<64><<<grid, 64, 0, s>>>(a);
+    cudaError_t e = cudaGetLastError();
+    if (e == cudaSuccess && nsplit > 1) {
+      if (d == 128)
+        pia::decode_combine_kernel<128><<<(unsigned)bh, 128, 0, s>>>(a.part, nsplit, cache_len, H, n_cache, a.out, lse);
+      else
+        pia::decode_combine_kernel<64><<<(unsigned)bh, 64, 0, s>>>(a.part, nsplit, cache_len, H, n_cache, a.out, lse);
+      e = cudaGetLastError();
+    }
+    if (a.part) {
+      cudaError_t e2 = cudaFreeAsync(a.part, s);
+      if (e == cudaSuccess) e = e2;
+    }
+    return e == cudaSuccess ? ok() : cuda_fail(e, "decode kernel launch");
+  }
+  if (dtype == PI_ATTN_F32)
+    return launch_simt<float, true>(q, kcache, vcache, w_g, b_g, cache_len, out, lse, B, H, 1, n_cache, d, k_win, pi,
+                                    S, s);
+  return launch_simt<__nv_bfloat16, true>(q, kcache, vcache, w_g, b_g, cache_len, out, lse, B, H, 1, n_cache, d, k_win,
+                                          pi, S, s);
+}
+
+pi_attn_status pi_attn_debug_index_sets(int n, int k_win, int pi, int S, int* counts, int* idx, int width,
+                                        void* stream) {
+  if (!counts || !idx) return fail(PI_ATTN_EINVAL, "null pointer");
+  if (n < 1 || k_win < 0 || pi < 1 || S < 0) return fail(PI_ATTN_EINVAL, "need n >= 1, k_win >= 0, pi >= 1, S >= 0");
+  if ((long long)width < (long long)k_win + 1 + S) return fail(PI_ATTN_EINVAL, "width < k_win + 1 + S");
+  const int threads = 256;
+  pia::index_sets_kernel<<<(n + threads - 1) / threads, threads, 0, as_stream(stream)>>>(n, k_win, pi, S, width,
+                                                                                          counts, idx);
+  cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? ok() : cuda_fail(e, "index-set kernel launch");
+}
+
+pi_attn_status pi_attn_check(void* stream) {
+  cudaError_t e = cudaStreamSynchronize(as_stream(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "stream synchronize");
+  unsigned word = 0;
+  e = cudaMemcpyFromSymbol(&word, pia::g_error_word, sizeof word);
+  if (e != cudaSuccess) return cuda_fail(e, "read device error word");
+  if (word) {
+    const unsigned zero = 0;
+    cudaMemcpyToSymbol(pia::g_error_word, &zero, sizeof zero);
+    return fail(PI_ATTN_EDEVICE, "device error flags 0x%x:%s%s%s", word,
+                (word & pia::kErrWaitTimeout) ? " pipeline-wait-timeout" : "",
+                (word & pia::kErrCacheLen) ? " cache_len-out-of-range" : "",
+                (word & pia::kErrInternal) ? " internal-check" : "");
+  }
+  return ok();
+}
+
+}  // extern "C"

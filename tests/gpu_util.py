@@ -1,0 +1,79 @@
+"""Helpers shared by the GPU parity tests: moving generator output to the device and back, and
+the comparison metrics with the operator's tolerances."""
+import math
+
+import numpy as np
+import torch
+
+import pi_synth as ps
+
+# Tolerances of the CUDA path against the fp64 oracle, on the same stored inputs.
+#   fp32 storage: max-abs 1e-5 on out and on lse.
+#   bf16 storage (fp32 accumulation): max-abs 2e-2 and relative L2 5e-3 on out; lse max-abs 1e-3
+#   (fp32 logits and sums; the bf16 rounding of the probabilities fed to the P.V product does not
+#   enter lse).
+TOL = {
+    "f32": dict(out_abs=1e-5, out_rel_l2=1e-5, lse_abs=1e-5),
+    "bf16": dict(out_abs=2e-2, out_rel_l2=5e-3, lse_abs=1e-3),
+}
+
+
+def to_dev(a: np.ndarray, dtype: str, device="cuda"):
+    if dtype == "bf16":
+        return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).to(device).view(torch.bfloat16)
+    return torch.from_numpy(np.ascontiguousarray(a, dtype=np.float32)).to(device)
+
+
+def from_dev(t) -> np.ndarray:
+    """Device tensor -> float64 numpy (bf16 widened exactly)."""
+    if t.dtype == torch.bfloat16:
+        return ps.bf16_bits_to_f32(t.view(torch.int16).cpu().numpy().view(np.uint16)).astype(np.float64)
+    return t.float().cpu().numpy().astype(np.float64)
+
+
+def metrics(got_out, ref_out, got_lse=None, ref_lse=None):
+    d = got_out - ref_out
+    m = {
+        "out_abs": float(np.max(np.abs(d))) if d.size else 0.0,
+        "out_rel_l2": float(np.linalg.norm(d) / max(np.linalg.norm(ref_out), 1e-300)) if d.size else 0.0,
+        "finite": bool(np.all(np.isfinite(got_out))),
+    }
+    if got_lse is not None:
+        m["lse_abs"] = float(np.max(np.abs(got_lse - ref_lse))) if got_lse.size else 0.0
+        m["finite"] = m["finite"] and bool(np.all(np.isfinite(got_lse)))
+    return m
+
+
+def assert_close(m: dict, dtype: str, what: str = ""):
+    tol = TOL[dtype]
+    assert m["finite"], f"{what}: non-finite output {m}"
+    assert m["out_abs"] <= tol["out_abs"], f"{what}: out max-abs {m['out_abs']:.3g} > {tol['out_abs']} {m}"
+    assert m["out_rel_l2"] <= tol["out_rel_l2"], f"{what}: out rel-L2 {m['out_rel_l2']:.3g} {m}"
+    if "lse_abs" in m:
+        assert m["lse_abs"] <= tol["lse_abs"], f"{what}: lse max-abs {m['lse_abs']:.3g} > {tol['lse_abs']} {m}"
+
+
+def sampled_rows(w, count: int, seed: int = 0) -> np.ndarray:
+    """`count` flat query rows drawn without replacement, plus for every (b, h) the boundary rows
+    i in {0, k-1, k, k+1, pi, m0*pi, S*pi - 1, S*pi, n-1} (m0 = first skip outside the window)."""
+    rng = np.random.default_rng(seed)
+    total = w.B * w.H * w.n
+    pick = rng.choice(total, size=min(count, total), replace=False)
+    m0 = w.k // w.pi + 1
+    bound = [0, w.k - 1, w.k, w.k + 1, w.pi, m0 * w.pi, w.S * w.pi - 1, w.S * w.pi, w.n - 1]
+    bound = sorted({i for i in bound if 0 <= i < w.n})
+    bh = np.arange(w.B * w.H)
+    extra = (bh[:, None] * w.n + np.array(bound)[None, :]).reshape(-1)
+    return np.unique(np.concatenate([pick, extra]))
+
+
+def rel(a, b):
+    return abs(a - b) / max(abs(b), 1e-300)
+
+
+def tokens(w):
+    return w.B * w.n if w.kind == "prefill" else w.B
+
+
+def isqrt(x):
+    return int(math.isqrt(x))

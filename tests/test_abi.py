@@ -1,0 +1,101 @@
+"""The C ABI library: it builds for sm_100a, loads, exports every declared symbol, and rejects bad
+arguments before touching the GPU (CPU only: no call here launches a kernel)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import periodic_sparse_attention_b200 as pia
+from periodic_sparse_attention_b200 import build as pbuild
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_functions():
+    names = []
+    for fn in os.listdir(os.path.join(ROOT, "include")):
+        if fn.endswith(".h"):
+            text = open(os.path.join(ROOT, "include", fn)).read()
+            text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+            names += re.findall(r"\b(pi_attn_\w+)\s*\(", text)
+    return sorted(set(names))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    pbuild.build()
+    return pia.load()
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for must in ["pi_attn_fwd", "pi_attn_decode", "pi_attn_debug_index_sets", "pi_attn_check",
+                 "pi_attn_status_string"]:
+        assert must in names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), f"{name} declared in include/ but not exported"
+        assert name in pia.SIGNATURES, f"{name} has no Python binding"
+
+
+def test_status_strings_and_version(lib):
+    assert lib.pi_attn_status_string(0) == b"PI_ATTN_OK"
+    assert lib.pi_attn_status_string(4) == b"PI_ATTN_EDEVICE"
+    assert lib.pi_attn_version() >= 100
+
+
+FAKE = ctypes.c_void_p(0x10000)  # aligned, never dereferenced: every call below fails validation first
+
+
+def _fwd(lib, **kw):
+    a = dict(q=FAKE, k=FAKE, v=FAKE, w=FAKE, b=FAKE, out=FAKE, lse=None, B=1, H=1, n=16, d=64, kw=4, pi=4, S=2,
+             dt=pia.PI_ATTN_BF16, path=0)
+    a.update(kw)
+    return lib.pi_attn_fwd_ex(a["q"], a["k"], a["v"], a["w"], a["b"], a["out"], a["lse"], a["B"], a["H"], a["n"],
+                              a["d"], a["kw"], a["pi"], a["S"], a["dt"], a["path"], None)
+
+
+@pytest.mark.parametrize("bad", [
+    dict(q=None), dict(out=None), dict(w=None), dict(B=0), dict(H=0), dict(n=0), dict(d=0), dict(d=300),
+    dict(d=12), dict(kw=-1), dict(pi=0), dict(S=-1), dict(dt=7), dict(path=9), dict(q=ctypes.c_void_p(0x10008)),
+    dict(dt=pia.PI_ATTN_F32, d=6),
+])
+def test_fwd_rejects_bad_arguments(lib, bad):
+    assert _fwd(lib, **bad) == pia.PI_ATTN_EINVAL
+    assert lib.pi_attn_last_error() != b""
+
+
+def test_tensor_core_path_is_explicit_about_coverage(lib):
+    assert _fwd(lib, dt=pia.PI_ATTN_F32, d=32, path=pia.PATHS["tc"]) in (pia.PI_ATTN_EUNSUPPORTED,)
+    assert _fwd(lib, d=96, path=pia.PATHS["tc"]) == pia.PI_ATTN_EUNSUPPORTED
+
+
+def test_decode_and_index_export_reject_bad_arguments(lib):
+    assert lib.pi_attn_decode(FAKE, FAKE, None, FAKE, FAKE, None, FAKE, None, 1, 1, 8, 64, 4, 4, 2, 1, None) == \
+        pia.PI_ATTN_EINVAL
+    assert lib.pi_attn_decode(FAKE, FAKE, FAKE, FAKE, FAKE, None, FAKE, None, 1, 1, 0, 64, 4, 4, 2, 1, None) == \
+        pia.PI_ATTN_EINVAL
+    assert lib.pi_attn_debug_index_sets(16, 4, 4, 2, FAKE, FAKE, 3, None) == pia.PI_ATTN_EINVAL  # width too small
+    assert lib.pi_attn_debug_index_sets(16, 4, 0, 2, FAKE, FAKE, 16, None) == pia.PI_ATTN_EINVAL
+
+
+def test_built_for_sm100a_only():
+    cmd = pbuild.command("x.so")
+    assert "arch=compute_100a,code=sm_100a" in cmd and "-lineinfo" in cmd
+
+
+def test_product_path_never_touches_the_oracle():
+    pkg = os.path.join(ROOT, "periodic_sparse_attention_b200")
+    for dirpath, _, files in os.walk(pkg):
+        for fn in files:
+            if fn.endswith((".py", ".cu", ".cuh", ".h")):
+                text = open(os.path.join(dirpath, fn)).read()
+                assert "import oracle" not in text and "from oracle" not in text and "pi_oracle" not in text, fn
+
+
+def test_binding_fails_loudly_without_the_library(tmp_path):
+    with pytest.raises(ImportError):
+        pia.load(str(tmp_path / "missing.so"))
