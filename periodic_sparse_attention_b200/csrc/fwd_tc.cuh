@@ -1,12 +1,622 @@
-// fwd_tc.cuh -- tensor-core (tcgen05 / TMEM / TMA) prefill kernel.  (placeholder)
+// fwd_tc.cuh -- pi-attention prefill on Blackwell tensor cores (tcgen05 + TMEM + TMA), bf16,
+// head size 64 or 128.
+//
+// Work unit: one CTA per (query tile of 128 rows, b, h).  The keys a tile needs are the union of
+// its window band [i0 - k, i0 + 127] and, for every surviving skip m, the block
+// [i0 - m*pi, i0 + 127 - m*pi]; the CTA walks the 128-key tiles that intersect this union in
+// increasing order ("local sweep" and "periodic gather" of the method's execution schedule, both
+// as tile loads) and evaluates every tile with the tensor cores:
+//
+//   TMA producer warp   Q tile once, then K and V tiles into a 2-stage ring (128B swizzle)
+//   MMA warp            S = Q K^T (128 x 128, fp32 in TMEM), then O += P V (128 x d, fp32 in TMEM)
+//   softmax warpgroup   one thread per query row: reads its S row from TMEM, applies the index
+//                       rule as a mask and the gate as a log-prior (log(alpha) on window keys,
+//                       log(1 - alpha) on skip keys, -inf elsewhere), keeps one running max and
+//                       one running sum for the whole union (a single softmax), writes P (bf16)
+//                       to shared memory in the MMA operand layout; at the end divides O by the
+//                       sum and writes out and lse.
+//
+// Online softmax with a lazy reference: probabilities are taken against a reference max that is
+// only raised when a tile's max exceeds it by more than 2^8, so O (in TMEM) is rescaled rarely;
+// every probability stays <= 2^8 and the final division uses the same reference, so the result
+// is exact up to rounding.
+//
+// Every wait on an mbarrier is bounded (pia::kWaitLimitNs).  A wait that gives up sets the device
+// error word and an abort flag in shared memory; all roles then leave their loops, drain their
+// own asynchronous work (bounded again) and the CTA frees its TMEM and exits.
 #pragma once
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
 #include "common.cuh"
 
 namespace pia {
-inline bool tc_supported(bool bf16, int d, int n) { (void)bf16; (void)d; (void)n; return false; }
-inline cudaError_t launch_fwd_tc(const void*, const void*, const void*, const float*, const float*, void*, float*, int,
-                                 int, int, int, int, int, int, cudaStream_t, const char** why) {
-  *why = "tensor-core path not built";
-  return cudaErrorNotSupported;
+namespace tc {
+
+constexpr int BM = 128;       // query rows per CTA
+constexpr int BN = 128;       // keys per tile
+constexpr int NSTAGE = 2;     // K/V ring depth
+constexpr int NTHREADS = 192; // warp 0 TMA, warp 1 MMA, warps 2-5 softmax
+constexpr float kRescaleThreshold = 8.0f;  // log2 units
+
+// ---- shared memory plan (offsets from a 1024-byte aligned base) ---------------------------------
+template <int D>
+struct Smem {
+  static constexpr int kTileBytes = BM * D * 2;          // one 128-row bf16 tile
+  static constexpr int kQ = 0;
+  static constexpr int kK = kQ + kTileBytes;
+  static constexpr int kV = kK + NSTAGE * kTileBytes;
+  static constexpr int kP = kV + NSTAGE * kTileBytes;
+  static constexpr int kBar = kP + BM * BN * 2;          // P: 128 x 128 bf16
+  // barriers: q_full, k_full[2], k_empty[2], v_full[2], v_empty[2], s_full, s_free, p_full, pv_done, drain
+  static constexpr int kNumBars = 1 + 4 * NSTAGE + 5;
+  static constexpr int kMisc = kBar + kNumBars * 8;      // tmem base (4 B), abort flag (4 B)
+  static constexpr int kTotal = kMisc + 16;
+  static constexpr int kAlloc = kTotal + 1024 - 128;     // slack to align a (>= 128 B aligned) base to 1 KB
+};
+
+// ---- PTX wrappers ------------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+// Bounded wait: false when the limit passed or another thread of the CTA aborted.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = global_ns();
+  while (true) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if (*abort_flag) return false;
+    if (global_ns() - t0 > kWaitLimitNs) {
+      raise_error(kErrWaitTimeout);
+      *abort_flag = 1;
+      return false;
+    }
+  }
+}
+__device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map, uint32_t bar, int c0, int c1,
+                                            int c2) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4, %5}], "
+      "[%2];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(c0), "r"(c1), "r"(c2)
+      : "memory");
+}
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+__device__ __forceinline__ void tc_mma(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                       uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem_d),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+__device__ __forceinline__ void tc_commit(uint32_t bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar) : "memory");
+}
+
+// 32 consecutive TMEM columns of this warp's 32 lanes: lane l gets row (32*(warp%4) + l).  The
+// wait is inside the same asm statement so no use of the results can be scheduled before it.
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float* v) {
+  uint32_t r[32];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+      "%15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];\n\t"
+      "tcgen05.wait::ld.sync.aligned;"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+        "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+        "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr)
+      : "memory");
+#pragma unroll
+  for (int t = 0; t < 32; ++t) v[t] = __uint_as_float(r[t]);
+}
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const float* v) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, "
+      "%14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32};" ::"r"(taddr),
+      "r"(__float_as_uint(v[0])), "r"(__float_as_uint(v[1])), "r"(__float_as_uint(v[2])),
+      "r"(__float_as_uint(v[3])), "r"(__float_as_uint(v[4])), "r"(__float_as_uint(v[5])),
+      "r"(__float_as_uint(v[6])), "r"(__float_as_uint(v[7])), "r"(__float_as_uint(v[8])),
+      "r"(__float_as_uint(v[9])), "r"(__float_as_uint(v[10])), "r"(__float_as_uint(v[11])),
+      "r"(__float_as_uint(v[12])), "r"(__float_as_uint(v[13])), "r"(__float_as_uint(v[14])),
+      "r"(__float_as_uint(v[15])), "r"(__float_as_uint(v[16])), "r"(__float_as_uint(v[17])),
+      "r"(__float_as_uint(v[18])), "r"(__float_as_uint(v[19])), "r"(__float_as_uint(v[20])),
+      "r"(__float_as_uint(v[21])), "r"(__float_as_uint(v[22])), "r"(__float_as_uint(v[23])),
+      "r"(__float_as_uint(v[24])), "r"(__float_as_uint(v[25])), "r"(__float_as_uint(v[26])),
+      "r"(__float_as_uint(v[27])), "r"(__float_as_uint(v[28])), "r"(__float_as_uint(v[29])),
+      "r"(__float_as_uint(v[30])), "r"(__float_as_uint(v[31]))
+      : "memory");
+}
+__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// ---- UMMA descriptors ----------------------------------------------------------------------------
+// Shared-memory matrix descriptor (sm_100): start address >> 4 in bits [0,14), leading byte
+// offset >> 4 in [16,30), stride byte offset >> 4 in [32,46), version 1 in [46,48), layout type
+// in [61,64) (2 = 128-byte swizzle).
+__device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+  return (uint64_t)((saddr & 0x3FFFFu) >> 4) | ((uint64_t)(lbo >> 4) << 16) | ((uint64_t)(sbo >> 4) << 32) |
+         (1ull << 46) | (2ull << 61);
+}
+// Instruction descriptor of kind::f16: fp32 accumulator, bf16 A and B, A K-major, B K-major
+// (b_mn_major = 0) or N-major (1), N >> 3 at bit 17, M >> 4 at bit 24.
+__host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, int b_mn_major) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)b_mn_major << 16) | ((uint32_t)(N >> 3) << 17) |
+         ((uint32_t)(M >> 4) << 24);
+}
+
+// ---- which 128-key tiles a query tile needs ---------------------------------------------------------
+struct TileWalk {
+  long long i0, last, band_lo;  // query rows [i0, last]; window keys start at band_lo
+  int pi, S, m0;
+  // smallest needed key tile index >= t, or -1 when none is left
+  __device__ __forceinline__ int next(int t) const {
+    const long long p = (long long)t * BN;
+    long long cand = -1;
+    if (p <= last) cand = p > band_lo ? p : band_lo;
+    const long long room = last - p;  // a skip range [i0 - m pi, last - m pi] reaches p iff m pi <= room
+    if (room >= 0) {
+      long long mm = room / pi;
+      if (mm > S) mm = S;
+      if (mm >= m0) {
+        long long st = i0 - mm * pi;
+        if (st < p) st = p;
+        if (cand < 0 || st < cand) cand = st;
+      }
+    }
+    return cand < 0 ? -1 : (int)(cand / BN);
+  }
+};
+
+struct Params {
+  const float* w_g;
+  const float* b_g;
+  __nv_bfloat16* out;
+  float* lse;
+  int H, n, kwin, pi, S;
+  float scale_log2;
+};
+
+template <int D>
+__global__ void __launch_bounds__(NTHREADS, D == 64 ? 2 : 1) fwd_tc_kernel(const __grid_constant__ CUtensorMap tmq,
+                                                             const __grid_constant__ CUtensorMap tmk,
+                                                             const __grid_constant__ CUtensorMap tmv, Params prm) {
+  using L = Smem<D>;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  uint8_t* const sbase = smem_raw + (base - raw);
+  if (base - raw + L::kTotal > (uint32_t)L::kAlloc) {  // the plan does not fit: refuse, touch nothing
+    if (threadIdx.x == 0) raise_error(kErrInternal);
+    return;
+  }
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int qt = blockIdx.x;
+  const int bh = blockIdx.y;
+  const int h = bh % prm.H;
+  const long long i0 = (long long)qt * BM;
+
+  TileWalk walk;
+  walk.i0 = i0;
+  walk.last = i0 + BM - 1 < prm.n - 1 ? i0 + BM - 1 : prm.n - 1;
+  walk.band_lo = i0 - prm.kwin > 0 ? i0 - prm.kwin : 0;
+  walk.pi = prm.pi;
+  walk.S = prm.S;
+  walk.m0 = first_skip_m(prm.kwin, prm.pi);
+
+  const uint32_t sQ = base + L::kQ, sK = base + L::kK, sV = base + L::kV, sP = base + L::kP;
+  const uint32_t bar0 = base + L::kBar;
+  const uint32_t bar_q = bar0;
+  auto bar_kfull = [&](int s) { return bar0 + 8u * (1 + s); };
+  auto bar_kempty = [&](int s) { return bar0 + 8u * (1 + NSTAGE + s); };
+  auto bar_vfull = [&](int s) { return bar0 + 8u * (1 + 2 * NSTAGE + s); };
+  auto bar_vempty = [&](int s) { return bar0 + 8u * (1 + 3 * NSTAGE + s); };
+  const uint32_t bar_sfull = bar0 + 8u * (1 + 4 * NSTAGE);
+  const uint32_t bar_sfree = bar_sfull + 8;
+  const uint32_t bar_pfull = bar_sfull + 16;
+  const uint32_t bar_pvdone = bar_sfull + 24;
+  const uint32_t bar_drain = bar_sfull + 32;
+  uint32_t* const tmem_slot = reinterpret_cast<uint32_t*>(sbase + L::kMisc);
+  volatile int* const abort_flag = reinterpret_cast<volatile int*>(sbase + L::kMisc + 4);
+
+  if (threadIdx.x == 0) {
+    mbar_init(bar_q, 1);
+    for (int s = 0; s < NSTAGE; ++s) {
+      mbar_init(bar_kfull(s), 1);
+      mbar_init(bar_kempty(s), 1);
+      mbar_init(bar_vfull(s), 1);
+      mbar_init(bar_vempty(s), 1);
+    }
+    mbar_init(bar_sfull, 1);
+    mbar_init(bar_sfree, BM);
+    mbar_init(bar_pfull, BM);
+    mbar_init(bar_pvdone, 1);
+    mbar_init(bar_drain, 1);
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 1) {  // TMEM: S in columns [0, 128), O in [128, 128 + D)
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], 256;" ::"r"(smem_u32(tmem_slot))
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t tS = tmem, tO = tmem + 128;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      constexpr uint32_t kTile = L::kTileBytes;
+      mbar_expect_tx(bar_q, kTile);
+#pragma unroll
+      for (int c = 0; c < D / 64; ++c) tma_load_3d(sQ + c * BM * 128, &tmq, bar_q, c * 64, (int)i0, bh);
+      int nk = 0, nv = 0;  // K and V tile loads issued
+      for (int t = walk.next(0); t >= 0; t = walk.next(t + 1)) {
+        const int s = nk % NSTAGE, use = nk / NSTAGE;
+        if (use > 0 && !mbar_wait(bar_kempty(s), (use - 1) & 1, abort_flag)) break;
+        mbar_expect_tx(bar_kfull(s), kTile);
+#pragma unroll
+        for (int c = 0; c < D / 64; ++c)
+          tma_load_3d(sK + s * kTile + c * BN * 128, &tmk, bar_kfull(s), c * 64, t * BN, bh);
+        ++nk;
+        if (use > 0 && !mbar_wait(bar_vempty(s), (use - 1) & 1, abort_flag)) break;
+        mbar_expect_tx(bar_vfull(s), kTile);
+#pragma unroll
+        for (int c = 0; c < D / 64; ++c)
+          tma_load_3d(sV + s * kTile + c * BN * 128, &tmv, bar_vfull(s), c * 64, t * BN, bh);
+        ++nv;
+      }
+      if (*abort_flag) {  // let the loads already in flight land before the CTA can exit
+        volatile int never = 0;
+        mbar_wait(bar_q, 0, &never);
+        for (int u = nk > NSTAGE ? nk - NSTAGE : 0; u < nk; ++u)
+          mbar_wait(bar_kfull(u % NSTAGE), (u / NSTAGE) & 1, &never);
+        for (int u = nv > NSTAGE ? nv - NSTAGE : 0; u < nv; ++u)
+          mbar_wait(bar_vfull(u % NSTAGE), (u / NSTAGE) & 1, &never);
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ------------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t kTile = L::kTileBytes;
+      constexpr uint32_t idesc_qk = idesc_bf16(BM, BN, 0);
+      constexpr uint32_t idesc_pv = idesc_bf16(BM, D, 1);
+      bool okw = mbar_wait(bar_q, 0, abort_flag);
+      tc_fence_after();
+      // S = Q K_j^T : K = D, 16 per instruction; 64-column blocks of 16 KB
+      auto issue_qk = [&](int s) {
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * (BM * 128) + (kk & 3) * 32;
+          tc_mma(tS, sw128_desc(sQ + off, 16, 1024), sw128_desc(sK + s * kTile + off, 16, 1024), idesc_qk,
+                 kk > 0 ? 1u : 0u);
+        }
+      };
+      // O += P V_j : K = 128 keys, 16 per instruction; V is N-major (d contiguous)
+      auto issue_pv = [&](int s, bool first) {
+#pragma unroll
+        for (int kk = 0; kk < BN / 16; ++kk) {
+          const uint32_t aoff = (kk >> 2) * (BM * 128) + (kk & 3) * 32;
+          const uint32_t boff = kk * 16 * 128;
+          tc_mma(tO, sw128_desc(sP + aoff, 16, 1024), sw128_desc(sV + s * kTile + boff, BN * 128, 1024), idesc_pv,
+                 (first && kk == 0) ? 0u : 1u);
+        }
+      };
+      int j = 0;
+      int t = walk.next(0);
+      if (okw && t >= 0) {
+        okw = mbar_wait(bar_kfull(0), 0, abort_flag);
+        if (okw) {
+          tc_fence_after();
+          issue_qk(0);
+          tc_commit(bar_sfull);
+          tc_commit(bar_kempty(0));
+        }
+      }
+      while (okw && t >= 0) {
+        const int tn = walk.next(t + 1);
+        const int s = j % NSTAGE;
+        if (tn >= 0) {
+          const int jn = j + 1, sn = jn % NSTAGE;
+          if (!mbar_wait(bar_kfull(sn), (jn / NSTAGE) & 1, abort_flag)) break;
+          if (!mbar_wait(bar_sfree, j & 1, abort_flag)) break;
+          tc_fence_after();
+          issue_qk(sn);
+          tc_commit(bar_sfull);
+          tc_commit(bar_kempty(sn));
+        }
+        if (!mbar_wait(bar_vfull(s), (j / NSTAGE) & 1, abort_flag)) break;
+        if (!mbar_wait(bar_pfull, j & 1, abort_flag)) break;
+        tc_fence_after();
+        issue_pv(s, j == 0);
+        tc_commit(bar_pvdone);
+        tc_commit(bar_vempty(s));
+        ++j;
+        t = tn;
+      }
+      // all MMAs issued by this thread have completed once the drain barrier flips
+      tc_commit(bar_drain);
+      volatile int never = 0;
+      mbar_wait(bar_drain, 0, &never);
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------------ softmax warpgroup
+    const int q4 = warp & 3;                  // TMEM lane quarter this warp may access
+    const int r = q4 * 32 + lane;             // query row within the tile
+    const long long i = i0 + r;
+    const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
+
+    // gate on the unscaled query row (read from the swizzled Q tile)
+    bool ok = mbar_wait(bar_q, 0, abort_flag);
+    float z = prm.b_g[h];
+    {
+      const float* wg = prm.w_g + (long long)h * D;
+#pragma unroll
+      for (int c = 0; c < D / 8; ++c) {
+        const int blk = c >> 3, cc = c & 7;
+        const uint4 u = *reinterpret_cast<const uint4*>(sbase + L::kQ + blk * (BM * 128) + r * 128 +
+                                                        ((cc ^ (r & 7)) << 4));
+        float f[8];
+        bf16x8_to_f32(u, f);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) z = fmaf(f[e], wg[c * 8 + e], z);
+      }
+    }
+    const float bias_l = log_sigmoid(z) * kLog2e;
+    const float bias_p = log_sigmoid(-z) * kLog2e;
+    const float NEG_INF = -INFINITY;
+
+    float m_ref = NEG_INF;  // reference max (log2 units)
+    float l_sum = 0.f;      // running sum of probabilities against m_ref
+    int j = 0;
+    for (int t = walk.next(0); ok && t >= 0; t = walk.next(t + 1), ++j) {
+      if (!mbar_wait(bar_sfull, j & 1, abort_flag)) { ok = false; break; }
+      tc_fence_after();
+      float x[BN];
+#pragma unroll
+      for (int c = 0; c < BN / 32; ++c) tmem_ld32(tS + lane_off + c * 32, x + c * 32);
+      tc_fence_before();
+      mbar_arrive(bar_sfree);
+
+      // the index rule on this tile, for row i: window columns [lc_lo, lc_hi], skip columns bitmask
+      const long long j0 = (long long)t * BN;
+      const long long d0 = i - j0;  // i - j at column 0
+      long long lo = (i - prm.kwin > 0 ? i - prm.kwin : 0) - j0;
+      long long hi = d0;
+      const int lc_lo = lo < 0 ? 0 : (lo > BN ? BN : (int)lo);
+      const int lc_hi = hi > BN - 1 ? BN - 1 : (hi < -1 ? -1 : (int)hi);
+      uint32_t sk[BN / 32] = {0u, 0u, 0u, 0u};
+      if (d0 > prm.kwin && prm.S >= walk.m0) {
+        long long m_hi = d0 / prm.pi;
+        if (m_hi > prm.S) m_hi = prm.S;
+        long long m_lo = d0 - (BN - 1) > 0 ? (d0 - (BN - 1) + prm.pi - 1) / prm.pi : 0;
+        if (m_lo < walk.m0) m_lo = walk.m0;
+        for (long long m = m_lo; m <= m_hi; ++m) {
+          const int c = (int)(d0 - m * prm.pi);
+          sk[c >> 5] |= 1u << (c & 31);
+        }
+      }
+      const bool all_local = lc_lo == 0 && lc_hi == BN - 1 && (sk[0] | sk[1] | sk[2] | sk[3]) == 0u;
+      float mt = NEG_INF;
+      if (all_local) {
+#pragma unroll
+        for (int c = 0; c < BN; ++c) {
+          x[c] = fmaf(x[c], prm.scale_log2, bias_l);
+          mt = fmaxf(mt, x[c]);
+        }
+      } else {
+#pragma unroll
+        for (int c = 0; c < BN; ++c) {
+          const bool loc = c >= lc_lo && c <= lc_hi;
+          const bool skp = (sk[c >> 5] >> (c & 31)) & 1u;
+          const float b = loc ? bias_l : (skp ? bias_p : NEG_INF);
+          x[c] = fmaf(x[c], prm.scale_log2, b);
+          mt = fmaxf(mt, x[c]);
+        }
+      }
+      // lazy reference max
+      float factor = 1.f;
+      bool rescale = false;
+      if (mt > m_ref + kRescaleThreshold || (m_ref == NEG_INF && mt != NEG_INF)) {
+        factor = ex2(m_ref - mt);  // 0 when m_ref = -inf
+        rescale = l_sum > 0.f;
+        l_sum *= factor;
+        m_ref = mt;
+      }
+      const float m_use = m_ref == NEG_INF ? 0.f : m_ref;
+      // probabilities, row sum, bf16 pairs
+      uint32_t pk[BN / 2];
+      float ls = 0.f;
+#pragma unroll
+      for (int c = 0; c < BN; c += 2) {
+        const float p0 = ex2(x[c] - m_use), p1 = ex2(x[c + 1] - m_use);
+        ls += p0 + p1;
+        __nv_bfloat162 b2 = __floats2bfloat162_rn(p0, p1);
+        pk[c / 2] = *reinterpret_cast<uint32_t*>(&b2);
+      }
+      l_sum += ls;
+
+      // P buffer and O are free once the previous P.V has completed
+      if (j > 0) {
+        if (!mbar_wait(bar_pvdone, (j - 1) & 1, abort_flag)) { ok = false; break; }
+        tc_fence_after();
+        if (rescale) {
+#pragma unroll
+          for (int c = 0; c < D / 32; ++c) {
+            float o[32];
+            tmem_ld32(tO + lane_off + c * 32, o);
+#pragma unroll
+            for (int e = 0; e < 32; ++e) o[e] *= factor;
+            tmem_st32(tO + lane_off + c * 32, o);
+          }
+          tmem_wait_st();
+        }
+      }
+      // P row r -> shared memory, K-major with the 128-byte swizzle (16-byte chunk c ^ (r & 7))
+#pragma unroll
+      for (int c = 0; c < BN / 8; ++c) {
+        const int blk = c >> 3, cc = c & 7;
+        uint4 u;
+        u.x = pk[c * 4 + 0];
+        u.y = pk[c * 4 + 1];
+        u.z = pk[c * 4 + 2];
+        u.w = pk[c * 4 + 3];
+        *reinterpret_cast<uint4*>(sbase + L::kP + blk * (BM * 128) + r * 128 + ((cc ^ (r & 7)) << 4)) = u;
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      mbar_arrive(bar_pfull);
+    }
+    // epilogue: O / l_sum -> out (bf16), lse
+    if (ok && j > 0 && mbar_wait(bar_pvdone, (j - 1) & 1, abort_flag)) {
+      tc_fence_after();
+      const float inv = 1.f / l_sum;
+      const bool row_ok = i < prm.n;
+      __nv_bfloat16* orow = prm.out + ((long long)bh * prm.n + i) * D;
+#pragma unroll
+      for (int c = 0; c < D / 32; ++c) {
+        float o[32];
+        tmem_ld32(tO + lane_off + c * 32, o);
+        if (row_ok) {
+#pragma unroll
+          for (int g = 0; g < 4; ++g) {
+            uint4 u;
+            uint32_t w[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              __nv_bfloat162 b2 = __floats2bfloat162_rn(o[g * 8 + 2 * e] * inv, o[g * 8 + 2 * e + 1] * inv);
+              w[e] = *reinterpret_cast<uint32_t*>(&b2);
+            }
+            u.x = w[0];
+            u.y = w[1];
+            u.z = w[2];
+            u.w = w[3];
+            *reinterpret_cast<uint4*>(orow + c * 32 + g * 8) = u;
+          }
+        }
+      }
+      if (row_ok && prm.lse) prm.lse[(long long)bh * prm.n + i] = (m_ref + log2f(l_sum)) * kLn2;
+    }
+    tc_fence_before();
+  }
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) {
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, 256;" ::"r"(tmem) : "memory");
+  }
+}
+
+// ---- host side --------------------------------------------------------------------------------------
+inline PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }
+  return fn;
+}
+
+// [B*H, n, d] bf16 viewed as a 3-D tensor (d innermost); box = 64 elements x 128 rows x 1.
+inline bool make_map(CUtensorMap* m, const void* ptr, int BH, int n, int d) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)n, (cuuint64_t)BH};
+  cuuint64_t strides[2] = {(cuuint64_t)d * 2, (cuuint64_t)n * d * 2};
+  cuuint32_t box[3] = {64, 128, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+}  // namespace tc
+
+inline bool tc_supported(bool bf16, int d, int n) { return bf16 && (d == 64 || d == 128) && n >= 1; }
+
+template <int D>
+cudaError_t launch_fwd_tc_d(const void* q, const void* k, const void* v, const float* w_g, const float* b_g,
+                            void* out, float* lse, int B, int H, int n, int kwin, int pi, int S, cudaStream_t st,
+                            const char** why) {
+  using L = tc::Smem<D>;
+  CUtensorMap mq, mk, mv;
+  const int BH = B * H;
+  if (!tc::make_map(&mq, q, BH, n, D) || !tc::make_map(&mk, k, BH, n, D) || !tc::make_map(&mv, v, BH, n, D)) {
+    *why = "cuTensorMapEncodeTiled failed";
+    return cudaErrorInvalidValue;
+  }
+  static bool attr_done = false;
+  if (!attr_done) {
+    cudaError_t e = cudaFuncSetAttribute(tc::fwd_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc);
+    if (e != cudaSuccess) {
+      *why = "cudaFuncSetAttribute(max dynamic shared memory)";
+      return e;
+    }
+    attr_done = true;
+  }
+  tc::Params p;
+  p.w_g = w_g;
+  p.b_g = b_g;
+  p.out = (__nv_bfloat16*)out;
+  p.lse = lse;
+  p.H = H;
+  p.n = n;
+  p.kwin = kwin;
+  p.pi = pi;
+  p.S = S;
+  p.scale_log2 = (float)(1.0 / std::sqrt((double)D)) * kLog2e;
+  dim3 grid((unsigned)((n + tc::BM - 1) / tc::BM), (unsigned)BH);
+  tc::fwd_tc_kernel<D><<<grid, tc::NTHREADS, L::kAlloc, st>>>(mq, mk, mv, p);
+  *why = "tensor-core kernel launch";
+  return cudaGetLastError();
+}
+
+inline cudaError_t launch_fwd_tc(const void* q, const void* k, const void* v, const float* w_g, const float* b_g,
+                                 void* out, float* lse, int B, int H, int n, int d, int kwin, int pi, int S,
+                                 cudaStream_t st, const char** why) {
+  if (d == 128) return launch_fwd_tc_d<128>(q, k, v, w_g, b_g, out, lse, B, H, n, kwin, pi, S, st, why);
+  return launch_fwd_tc_d<64>(q, k, v, w_g, b_g, out, lse, B, H, n, kwin, pi, S, st, why);
+}
+
 }  // namespace pia

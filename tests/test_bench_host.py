@@ -1,0 +1,93 @@
+"""Host-side logic of bench.py (CPU only): algorithmic work counts, traffic lookup, and the
+multi-rank timing reduction under a 2-rank gloo process group."""
+import json
+import os
+import socket
+import subprocess
+import sys
+
+import torch.multiprocessing as mp
+
+import bench
+import oracle
+import pi_synth as ps
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def test_index_totals_agree_with_oracle_enumeration():
+    for name in ("tiny_f32", "bf16_n4k", "bf16_n32k", "bf16_n128k"):
+        w = ps.WORKLOADS[name]
+        assert bench.index_totals(w.n, w.k, w.pi, w.S) == oracle.counts(w.n, w.k, w.pi, w.S)
+
+
+def test_work_of_the_default_workload():
+    w = ps.WORKLOADS["bf16_n4k"]
+    tokens, flops, bytes_ = bench.work(w)
+    assert tokens == 4096
+    # 8 heads x (520128 window + 7744 skip) pairs x 4 d flops, plus the gate
+    assert flops == 8 * (4 * 64 * (520128 + 7744) + 2 * 64 * 4096)
+    assert bytes_ == 8 * (4 * 4096 * 64 * 2 + 4 * 4096)
+
+
+def test_decode_work():
+    w = ps.WORKLOADS["decode_bf16"]
+    tokens, flops, bytes_ = bench.work(w)
+    assert tokens == 64
+    assert bytes_ == 64 * 32 * (2 * 1056 * 128 * 2 + 2 * 128 * 2 + 4)
+
+
+def test_traffic_line_needs_the_current_source(tmp_path, monkeypatch):
+    sha = bench.source_hash()
+    prof = tmp_path / "profiles"
+    prof.mkdir()
+    (prof / "x.md").write_text(f"bench-traffic: workload=bf16_n4k bytes_per_launch=123 source_sha={sha}\n"
+                               f"bench-traffic: workload=bf16_n32k bytes_per_launch=9 source_sha=stale\n")
+    real_root = bench.ROOT
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    os.symlink(os.path.join(real_root, "include"), tmp_path / "include")
+    os.makedirs(tmp_path / "periodic_sparse_attention_b200")
+    os.symlink(os.path.join(real_root, "periodic_sparse_attention_b200", "csrc"),
+               tmp_path / "periodic_sparse_attention_b200" / "csrc")
+    assert bench.profiled_traffic("bf16_n4k") == 123
+    assert bench.profiled_traffic("bf16_n32k") is None
+
+
+def _free_port():
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    p = s.getsockname()[1]
+    s.close()
+    return p
+
+
+def _rank_main(rank, world, port, out_dir):
+    import torch.distributed as dist
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank), WORLD_SIZE=str(world))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    r, w, _ = bench.dist_env()
+    got = bench.max_over_ranks(10.0 + 5.0 * rank, w)
+    with open(os.path.join(out_dir, f"r{r}.json"), "w") as f:
+        json.dump({"rank": r, "world": w, "max": got}, f)
+    dist.barrier()
+    dist.destroy_process_group()
+
+
+def test_max_over_ranks_two_gloo_ranks(tmp_path):
+    port = _free_port()
+    mp.start_processes(_rank_main, args=(2, port, str(tmp_path)), nprocs=2, start_method="spawn")
+    res = [json.load(open(tmp_path / f"r{i}.json")) for i in range(2)]
+    assert [r["max"] for r in res] == [15.0, 15.0]
+    assert [r["world"] for r in res] == [2, 2]
+
+
+def test_reference_arm_prints_one_line():
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--steps", "1",
+                        "--warmup", "3", "--workload", "tiny_f32", "--cpu-budget", "0.3"],
+                       capture_output=True, text=True, timeout=300)
+    assert r.returncode == 0, r.stderr
+    lines = [ln for ln in r.stdout.splitlines() if ln.strip()]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    assert d["impl"] == "reference" and d["value"] > 0 and d["cpu_baseline"]["cores"] >= 1
+    assert d["e2e"]["h2d_bytes_per_step"] == 0
