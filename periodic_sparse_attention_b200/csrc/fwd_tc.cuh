@@ -29,12 +29,13 @@
 #include <cudaTypedefs.h>
 
 #include "common.cuh"
+#include "tile_rule.cuh"
 
 namespace pia {
 namespace tc {
 
 constexpr int BM = 128;       // query rows per CTA
-constexpr int BN = 128;       // keys per tile
+constexpr int BN = kTileKeys; // keys per tile
 constexpr int NSTAGE = 2;     // K/V ring depth
 constexpr int NTHREADS = 192; // warp 0 TMA, warp 1 MMA, warps 2-5 softmax
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
@@ -177,29 +178,6 @@ __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, int b_mn_major) 
          ((uint32_t)(M >> 4) << 24);
 }
 
-// ---- which 128-key tiles a query tile needs ---------------------------------------------------------
-struct TileWalk {
-  long long i0, last, band_lo;  // query rows [i0, last]; window keys start at band_lo
-  int pi, S, m0;
-  // smallest needed key tile index >= t, or -1 when none is left
-  __device__ __forceinline__ int next(int t) const {
-    const long long p = (long long)t * BN;
-    long long cand = -1;
-    if (p <= last) cand = p > band_lo ? p : band_lo;
-    const long long room = last - p;  // a skip range [i0 - m pi, last - m pi] reaches p iff m pi <= room
-    if (room >= 0) {
-      long long mm = room / pi;
-      if (mm > S) mm = S;
-      if (mm >= m0) {
-        long long st = i0 - mm * pi;
-        if (st < p) st = p;
-        if (cand < 0 || st < cand) cand = st;
-      }
-    }
-    return cand < 0 ? -1 : (int)(cand / BN);
-  }
-};
-
 struct Params {
   const float* w_g;
   const float* b_g;
@@ -230,12 +208,7 @@ __global__ void __launch_bounds__(NTHREADS, D == 64 ? 2 : 1) fwd_tc_kernel(const
   const long long i0 = (long long)qt * BM;
 
   TileWalk walk;
-  walk.i0 = i0;
-  walk.last = i0 + BM - 1 < prm.n - 1 ? i0 + BM - 1 : prm.n - 1;
-  walk.band_lo = i0 - prm.kwin > 0 ? i0 - prm.kwin : 0;
-  walk.pi = prm.pi;
-  walk.S = prm.S;
-  walk.m0 = first_skip_m(prm.kwin, prm.pi);
+  walk.init(i0, prm.n, BM, prm.kwin, prm.pi, prm.S);
 
   const uint32_t sQ = base + L::kQ, sK = base + L::kK, sV = base + L::kV, sP = base + L::kP;
   const uint32_t bar0 = base + L::kBar;
@@ -417,39 +390,45 @@ __global__ void __launch_bounds__(NTHREADS, D == 64 ? 2 : 1) fwd_tc_kernel(const
       mbar_arrive(bar_sfree);
 
       // the index rule on this tile, for row i: window columns [lc_lo, lc_hi], skip columns bitmask
-      const long long j0 = (long long)t * BN;
-      const long long d0 = i - j0;  // i - j at column 0
-      long long lo = (i - prm.kwin > 0 ? i - prm.kwin : 0) - j0;
-      long long hi = d0;
-      const int lc_lo = lo < 0 ? 0 : (lo > BN ? BN : (int)lo);
-      const int lc_hi = hi > BN - 1 ? BN - 1 : (hi < -1 ? -1 : (int)hi);
-      uint32_t sk[BN / 32] = {0u, 0u, 0u, 0u};
-      if (d0 > prm.kwin && prm.S >= walk.m0) {
-        long long m_hi = d0 / prm.pi;
-        if (m_hi > prm.S) m_hi = prm.S;
-        long long m_lo = d0 - (BN - 1) > 0 ? (d0 - (BN - 1) + prm.pi - 1) / prm.pi : 0;
-        if (m_lo < walk.m0) m_lo = walk.m0;
-        for (long long m = m_lo; m <= m_hi; ++m) {
-          const int c = (int)(d0 - m * prm.pi);
-          sk[c >> 5] |= 1u << (c & 31);
-        }
-      }
-      const bool all_local = lc_lo == 0 && lc_hi == BN - 1 && (sk[0] | sk[1] | sk[2] | sk[3]) == 0u;
+      int lc_lo, lc_hi;
+      uint32_t sk[BN / 32];
+      row_tile_mask(i, (long long)t * BN, prm.kwin, prm.pi, prm.S, walk.m0, lc_lo, lc_hi, sk);
+      // per 32-column chunk, the cheapest exact treatment for this row (see chunk_class)
+      int cls[BN / 32];
+      int one_col[BN / 32];
+      float one_x[BN / 32];
       float mt = NEG_INF;
-      if (all_local) {
 #pragma unroll
-        for (int c = 0; c < BN; ++c) {
-          x[c] = fmaf(x[c], prm.scale_log2, bias_l);
-          mt = fmaxf(mt, x[c]);
-        }
-      } else {
+      for (int cb = 0; cb < BN / 32; ++cb) {
+        const int c0 = cb * 32;
+        const uint32_t skb = sk[cb];
+        cls[cb] = chunk_class(cb, lc_lo, lc_hi, skb);
+        one_col[cb] = 0;
+        one_x[cb] = NEG_INF;
+        if (cls[cb] == kFull) {
 #pragma unroll
-        for (int c = 0; c < BN; ++c) {
-          const bool loc = c >= lc_lo && c <= lc_hi;
-          const bool skp = (sk[c >> 5] >> (c & 31)) & 1u;
-          const float b = loc ? bias_l : (skp ? bias_p : NEG_INF);
-          x[c] = fmaf(x[c], prm.scale_log2, b);
-          mt = fmaxf(mt, x[c]);
+          for (int e = 0; e < 32; ++e) {
+            x[c0 + e] = fmaf(x[c0 + e], prm.scale_log2, bias_l);
+            mt = fmaxf(mt, x[c0 + e]);
+          }
+        } else if (cls[cb] == kOne) {
+          const int sc = __ffs(skb) - 1;
+          float xs = 0.f;
+#pragma unroll
+          for (int e = 0; e < 32; ++e) xs = e == sc ? x[c0 + e] : xs;
+          one_col[cb] = sc;
+          one_x[cb] = fmaf(xs, prm.scale_log2, bias_p);
+          mt = fmaxf(mt, one_x[cb]);
+        } else if (cls[cb] == kMixed) {
+#pragma unroll
+          for (int e = 0; e < 32; ++e) {
+            const int c = c0 + e;
+            const bool loc = c >= lc_lo && c <= lc_hi;
+            const bool skp = (skb >> e) & 1u;
+            const float b = loc ? bias_l : (skp ? bias_p : NEG_INF);
+            x[c] = fmaf(x[c], prm.scale_log2, b);
+            mt = fmaxf(mt, x[c]);
+          }
         }
       }
       // lazy reference max
@@ -466,11 +445,28 @@ __global__ void __launch_bounds__(NTHREADS, D == 64 ? 2 : 1) fwd_tc_kernel(const
       uint32_t pk[BN / 2];
       float ls = 0.f;
 #pragma unroll
-      for (int c = 0; c < BN; c += 2) {
-        const float p0 = ex2(x[c] - m_use), p1 = ex2(x[c + 1] - m_use);
-        ls += p0 + p1;
-        __nv_bfloat162 b2 = __floats2bfloat162_rn(p0, p1);
-        pk[c / 2] = *reinterpret_cast<uint32_t*>(&b2);
+      for (int cb = 0; cb < BN / 32; ++cb) {
+        const int c0 = cb * 32;
+        if (cls[cb] == kFull || cls[cb] == kMixed) {
+#pragma unroll
+          for (int e = 0; e < 32; e += 2) {
+            const float p0 = ex2(x[c0 + e] - m_use), p1 = ex2(x[c0 + e + 1] - m_use);
+            ls += p0 + p1;
+            __nv_bfloat162 b2 = __floats2bfloat162_rn(p0, p1);
+            pk[(c0 + e) / 2] = *reinterpret_cast<uint32_t*>(&b2);
+          }
+        } else if (cls[cb] == kOne) {
+          const float p1 = ex2(one_x[cb] - m_use);
+          ls += p1;
+          __nv_bfloat162 b2 = __floats2bfloat162_rn(p1, p1);
+          const uint32_t both = *reinterpret_cast<uint32_t*>(&b2);
+          const uint32_t word = (one_col[cb] & 1) ? (both & 0xFFFF0000u) : (both & 0x0000FFFFu);
+#pragma unroll
+          for (int w = 0; w < 16; ++w) pk[c0 / 2 + w] = (one_col[cb] >> 1) == w ? word : 0u;
+        } else {
+#pragma unroll
+          for (int w = 0; w < 16; ++w) pk[c0 / 2 + w] = 0u;
+        }
       }
       l_sum += ls;
 

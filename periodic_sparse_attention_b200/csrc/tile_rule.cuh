@@ -1,0 +1,91 @@
+// tile_rule.cuh -- the index rule as the tensor-core kernel applies it, in 128-key tiles.
+//
+// Host and device code: the kernel uses it, and a CPU test compiles the same header with g++ to
+// check, for many shapes, that the keys visited and unmasked are exactly L(i) and P(i).
+//   window  L(i) = [max(0, i - k), i]
+//   skips   P(i) = { i - m*pi : m0 <= m <= S, i - m*pi >= 0 },  m0 = floor(k / pi) + 1
+#pragma once
+#include <stdint.h>
+
+#if defined(__CUDACC__)
+#define PIA_HD __host__ __device__ __forceinline__
+#else
+#define PIA_HD inline
+#endif
+
+namespace pia {
+
+constexpr int kTileKeys = 128;  // keys per tile (BN)
+
+// Walks, in increasing order, the 128-key tiles that hold at least one key of the union of L(i)
+// and P(i) over the query rows [i0, last] of one tile.
+struct TileWalk {
+  long long i0, last, band_lo;  // query rows [i0, last]; the window keys of the tile start at band_lo
+  int pi, S, m0;
+  PIA_HD void init(long long i0_, long long n, int rows, int kwin, int pi_, int S_) {
+    i0 = i0_;
+    last = i0_ + rows - 1 < n - 1 ? i0_ + rows - 1 : n - 1;
+    band_lo = i0_ - kwin > 0 ? i0_ - kwin : 0;
+    pi = pi_;
+    S = S_;
+    m0 = kwin / pi_ + 1;
+  }
+  // smallest needed key tile index >= t, or -1 when none is left
+  PIA_HD int next(int t) const {
+    const long long p = (long long)t * kTileKeys;
+    long long cand = -1;
+    if (p <= last) cand = p > band_lo ? p : band_lo;
+    // the skip block of m, [i0 - m pi, last - m pi], reaches row p iff m pi <= last - p;
+    // the largest such m has the leftmost block
+    const long long room = last - p;
+    if (room >= 0) {
+      long long mm = room / pi;
+      if (mm > S) mm = S;
+      if (mm >= m0) {
+        long long st = i0 - mm * pi;
+        if (st < p) st = p;
+        if (cand < 0 || st < cand) cand = st;
+      }
+    }
+    return cand < 0 ? -1 : (int)(cand / kTileKeys);
+  }
+};
+
+// For query row i and the key tile starting at j0: window columns [lc_lo, lc_hi] (empty when
+// lc_lo > lc_hi) and a 128-bit mask of skip columns.  Skip columns never overlap the window.
+PIA_HD void row_tile_mask(long long i, long long j0, int kwin, int pi, int S, int m0, int& lc_lo, int& lc_hi,
+                          uint32_t sk[kTileKeys / 32]) {
+  const long long d0 = i - j0;  // i - j at column 0
+  const long long lo = (i - kwin > 0 ? i - kwin : 0) - j0;
+  lc_lo = lo < 0 ? 0 : (lo > kTileKeys ? kTileKeys : (int)lo);
+  lc_hi = d0 > kTileKeys - 1 ? kTileKeys - 1 : (d0 < -1 ? -1 : (int)d0);
+  for (int w = 0; w < kTileKeys / 32; ++w) sk[w] = 0u;
+  if (d0 > kwin && S >= m0) {
+    long long m_hi = d0 / pi;
+    if (m_hi > S) m_hi = S;
+    long long m_lo = d0 - (kTileKeys - 1) > 0 ? (d0 - (kTileKeys - 1) + pi - 1) / pi : 0;
+    if (m_lo < m0) m_lo = m0;
+    for (long long m = m_lo; m <= m_hi; ++m) {
+      const int c = (int)(d0 - m * pi);
+      sk[c >> 5] |= 1u << (c & 31);
+    }
+  }
+}
+
+// Cheapest exact treatment of a 32-column chunk cb of a tile for one row:
+//   kEmpty  no key of the union: p = 0, no exponential
+//   kFull   every column a window key and no skip: one FMA per logit
+//   kOne    exactly one skip key and no window key: one exponential for the chunk
+//   kMixed  anything else: per-column mask
+enum : int { kEmpty = 0, kFull = 1, kOne = 2, kMixed = 3 };
+PIA_HD int chunk_class(int cb, int lc_lo, int lc_hi, uint32_t skb) {
+  const int c0 = cb * 32;
+  const bool any_loc = lc_lo <= c0 + 31 && lc_hi >= c0 && lc_lo <= lc_hi;
+  const bool all_loc = lc_lo <= c0 && lc_hi >= c0 + 31;
+  if (!any_loc && skb == 0u) return kEmpty;
+  if (all_loc && skb == 0u) return kFull;
+  if (!any_loc && (skb & (skb - 1u)) == 0u) return kOne;
+  return kMixed;
+}
+
+}  // namespace pia
