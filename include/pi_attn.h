@@ -48,9 +48,14 @@ typedef enum { PI_ATTN_F32 = 0, PI_ATTN_BF16 = 1 } pi_attn_dtype;
 
 /* Kernel choice for pi_attn_fwd_ex. */
 typedef enum {
-    PI_ATTN_PATH_AUTO = 0,  /* tensor-core kernel where it applies (bf16, d in {64, 128}), else SIMT */
-    PI_ATTN_PATH_SIMT = 1,  /* CUDA-core kernel: every dtype, d <= 256 */
-    PI_ATTN_PATH_TC = 2     /* tcgen05/TMEM kernel only; PI_ATTN_EUNSUPPORTED where it does not apply */
+    PI_ATTN_PATH_AUTO = 0,      /* tensor-core kernel where it applies (bf16, d in {64, 128}), else SIMT */
+    PI_ATTN_PATH_SIMT = 1,      /* CUDA-core kernel: every dtype, d <= 256 */
+    PI_ATTN_PATH_TC = 2,        /* tcgen05/TMEM kernels only (single pass or split, chosen by shape);
+                                   PI_ATTN_EUNSUPPORTED where they do not apply */
+    PI_ATTN_PATH_TC_FUSED = 3,  /* tensor cores, window and skips in one pass */
+    PI_ATTN_PATH_TC_SPLIT = 4   /* tensor cores, skips in a residue-class pass (scratch of
+                                   B*H*n*(2d + 4) bytes from cudaMallocAsync on `stream`), then the
+                                   window pass merging them; needs n % pi == 0 */
 } pi_attn_path;
 
 /* Prefill forward.  Cited passage: the Core Components (window, skips, gate as log-prior, one

@@ -18,7 +18,7 @@ LIB_PATH = os.path.join(HERE, "libpiattn.so")
 
 PI_ATTN_OK, PI_ATTN_EINVAL, PI_ATTN_EUNSUPPORTED, PI_ATTN_ECUDA, PI_ATTN_EDEVICE = range(5)
 PI_ATTN_F32, PI_ATTN_BF16 = 0, 1
-PATHS = {"auto": 0, "simt": 1, "tc": 2}
+PATHS = {"auto": 0, "simt": 1, "tc": 2, "tc_fused": 3, "tc_split": 4}
 
 # (name, restype, argtypes) of every symbol include/pi_attn.h declares
 _vp, _i32, _cstr = ctypes.c_void_p, ctypes.c_int, ctypes.c_char_p

@@ -108,9 +108,11 @@ __global__ void __launch_bounds__(64) decode_bf16_kernel(DecodeArgs a) {
 #pragma unroll
   for (int e = 0; e < 8; ++e) acc[e] = 0.f;
 
+  // The trip count is the same for every lane of a warp (the loop variable is warp-uniform), so
+  // the full-warp shuffles of the dot-product reduction always see all 32 lanes.
   constexpr int STEP = NW * RPI * UNR;
-  for (int t0 = t_begin + (warp * RPI + slot) * UNR; t0 < t_end; t0 += STEP) {
-    // rows t0 .. t0+UNR-1 belong to this slot
+  for (int base = t_begin + warp * RPI * UNR; base < t_end; base += STEP) {
+    const int t0 = base + slot * UNR;  // rows t0 .. t0+UNR-1 belong to this slot
     uint4 kr[UNR], vr[UNR];
     bool ok[UNR];
     float bias[UNR];
@@ -120,7 +122,7 @@ __global__ void __launch_bounds__(64) decode_bf16_kernel(DecodeArgs a) {
       ok[u] = t < t_end;
       long long j = t < nL ? j0 + t : i - (long long)(m0 + (t - nL)) * a.pi;
       bias[u] = t < nL ? bias_l : bias_p;
-      if (!ok[u]) j = i;
+      if (!ok[u]) j = i;  // a row that exists; its score is discarded below
       kr[u] = __ldg(reinterpret_cast<const uint4*>(kb + j * D));
       vr[u] = __ldg(reinterpret_cast<const uint4*>(vb + j * D));
     }
@@ -139,21 +141,22 @@ __global__ void __launch_bounds__(64) decode_bf16_kernel(DecodeArgs a) {
     float mn = m;
 #pragma unroll
     for (int u = 0; u < UNR; ++u) mn = fmaxf(mn, s[u]);
-    if (mn == -INFINITY) continue;
-    const float corr = exp2f(m - mn);
-    l *= corr;
+    if (mn != -INFINITY) {  // per-slot state update; no warp-collective operation inside
+      const float corr = exp2f(m - mn);
+      l *= corr;
 #pragma unroll
-    for (int e = 0; e < 8; ++e) acc[e] *= corr;
+      for (int e = 0; e < 8; ++e) acc[e] *= corr;
 #pragma unroll
-    for (int u = 0; u < UNR; ++u) {
-      const float p = exp2f(s[u] - mn);
-      l += p;
-      float vf[8];
-      bf16x8_to_f32(vr[u], vf);
+      for (int u = 0; u < UNR; ++u) {
+        const float p = exp2f(s[u] - mn);
+        l += p;
+        float vf[8];
+        bf16x8_to_f32(vr[u], vf);
 #pragma unroll
-      for (int e = 0; e < 8; ++e) acc[e] = fmaf(p, vf[e], acc[e]);
+        for (int e = 0; e < 8; ++e) acc[e] = fmaf(p, vf[e], acc[e]);
+      }
+      m = mn;
     }
-    m = mn;
   }
 
   // merge the slots of this warp (lanes with equal `sub`)

@@ -102,6 +102,14 @@ __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map
       "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(c0), "r"(c1), "r"(c2)
       : "memory");
 }
+__device__ __forceinline__ void tma_load_4d(uint32_t dst, const CUtensorMap* map, uint32_t bar, int c0, int c1,
+                                            int c2, int c3) {
+  asm volatile(
+      "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4, %5, "
+      "%6}], [%2];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(c0), "r"(c1), "r"(c2), "r"(c3)
+      : "memory");
+}
 __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
@@ -178,19 +186,37 @@ __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, int b_mn_major) 
          ((uint32_t)(M >> 4) << 24);
 }
 
+// Three ways to run the kernel:
+//   kFused      window and skips of a 128-row query tile in one pass (the default)
+//   kResidue    the skip part alone, in the residue-class view: for a residue r (mod pi), rows
+//               t*pi + r form their own sequence, and P(i) becomes the band t - S .. t - m0 of it,
+//               a dense band the tensor cores evaluate without the 1/128 diagonal waste of skip
+//               tiles.  Writes the skip partial (normalised output in bf16, lse in fp32) of every
+//               row to scratch, in sequence layout.
+//   kBandMerge  the window part alone; the epilogue merges the skip partial of its rows:
+//               with a = log2 of the window mass, b = log2 of the skip mass, M = max(a, b),
+//               out = (out_L 2^(a-M) + out_P 2^(b-M)) / (2^(a-M) + 2^(b-M)),
+//               lse = (M + log2(2^(a-M) + 2^(b-M))) ln 2 -- the same single softmax, summed in
+//               two pieces.
+enum : int { kFused = 0, kResidue = 1, kBandMerge = 2 };
+
 struct Params {
   const float* w_g;
   const float* b_g;
   __nv_bfloat16* out;
   float* lse;
+  __nv_bfloat16* skip_o;  // [B*H, n, D] skip partial (kResidue writes, kBandMerge reads)
+  float* skip_lse;        // [B*H, n]
   int H, n, kwin, pi, S;
+  int T;                  // kResidue: rows per residue class (n / pi)
   float scale_log2;
 };
 
-template <int D>
+template <int D, int MODE>
 __global__ void __launch_bounds__(NTHREADS, D == 64 ? 2 : 1) fwd_tc_kernel(const __grid_constant__ CUtensorMap tmq,
-                                                             const __grid_constant__ CUtensorMap tmk,
-                                                             const __grid_constant__ CUtensorMap tmv, Params prm) {
+                                                                          const __grid_constant__ CUtensorMap tmk,
+                                                                          const __grid_constant__ CUtensorMap tmv,
+                                                                          Params prm) {
   using L = Smem<D>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
@@ -202,13 +228,28 @@ __global__ void __launch_bounds__(NTHREADS, D == 64 ? 2 : 1) fwd_tc_kernel(const
   }
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int qt = blockIdx.x;
   const int bh = blockIdx.y;
   const int h = bh % prm.H;
-  const long long i0 = (long long)qt * BM;
-
+  const int m0 = first_skip_m(prm.kwin, prm.pi);
+  // query tile: rows q0 .. q0+127 of the view (the sequence, or residue class `res`)
+  int res = 0;
+  long long q0;
   TileWalk walk;
-  walk.init(i0, prm.n, BM, prm.kwin, prm.pi, prm.S);
+  if (MODE == kResidue) {
+    res = blockIdx.x % prm.pi;
+    q0 = (long long)(blockIdx.x / prm.pi) * BM;
+    // keys of row t: t - S .. t - m0 (the skips of sequence row t*pi + res)
+    walk.i0 = q0;
+    walk.last = (q0 + BM - 1 < prm.T - 1 ? q0 + BM - 1 : prm.T - 1) - m0;
+    walk.band_lo = q0 - prm.S > 0 ? q0 - prm.S : 0;
+    walk.pi = 1;
+    walk.S = 0;
+    walk.m0 = 1;
+  } else {
+    q0 = (long long)blockIdx.x * BM;
+    walk.init(q0, prm.n, BM, prm.kwin, prm.pi, MODE == kFused ? prm.S : 0);
+  }
+  const int view_rows = MODE == kResidue ? prm.T : prm.n;
 
   const uint32_t sQ = base + L::kQ, sK = base + L::kK, sV = base + L::kV, sP = base + L::kP;
   const uint32_t bar0 = base + L::kBar;
@@ -252,27 +293,33 @@ __global__ void __launch_bounds__(NTHREADS, D == 64 ? 2 : 1) fwd_tc_kernel(const
   const uint32_t tmem = *tmem_slot;
   const uint32_t tS = tmem, tO = tmem + 128;
 
+  // one 128-row tile of the view (rows r0 .. r0+127) into shared memory, D/64 boxes of 64 columns
+  auto load_tile = [&](uint32_t dst, const CUtensorMap* map, uint32_t bar, long long r0) {
+#pragma unroll
+    for (int c = 0; c < D / 64; ++c) {
+      if (MODE == kResidue)
+        tma_load_4d(dst + c * BM * 128, map, bar, c * 64, res, (int)r0, bh);
+      else
+        tma_load_3d(dst + c * BM * 128, map, bar, c * 64, (int)r0, bh);
+    }
+  };
+
   if (warp == 0) {
     // ------------------------------------------------------------------ TMA producer
     if (lane == 0) {
       constexpr uint32_t kTile = L::kTileBytes;
       mbar_expect_tx(bar_q, kTile);
-#pragma unroll
-      for (int c = 0; c < D / 64; ++c) tma_load_3d(sQ + c * BM * 128, &tmq, bar_q, c * 64, (int)i0, bh);
+      load_tile(sQ, &tmq, bar_q, q0);
       int nk = 0, nv = 0;  // K and V tile loads issued
       for (int t = walk.next(0); t >= 0; t = walk.next(t + 1)) {
         const int s = nk % NSTAGE, use = nk / NSTAGE;
         if (use > 0 && !mbar_wait(bar_kempty(s), (use - 1) & 1, abort_flag)) break;
         mbar_expect_tx(bar_kfull(s), kTile);
-#pragma unroll
-        for (int c = 0; c < D / 64; ++c)
-          tma_load_3d(sK + s * kTile + c * BN * 128, &tmk, bar_kfull(s), c * 64, t * BN, bh);
+        load_tile(sK + s * kTile, &tmk, bar_kfull(s), (long long)t * BN);
         ++nk;
         if (use > 0 && !mbar_wait(bar_vempty(s), (use - 1) & 1, abort_flag)) break;
         mbar_expect_tx(bar_vfull(s), kTile);
-#pragma unroll
-        for (int c = 0; c < D / 64; ++c)
-          tma_load_3d(sV + s * kTile + c * BN * 128, &tmv, bar_vfull(s), c * 64, t * BN, bh);
+        load_tile(sV + s * kTile, &tmv, bar_vfull(s), (long long)t * BN);
         ++nv;
       }
       if (*abort_flag) {  // let the loads already in flight land before the CTA can exit
@@ -354,11 +401,12 @@ __global__ void __launch_bounds__(NTHREADS, D == 64 ? 2 : 1) fwd_tc_kernel(const
     // ------------------------------------------------------------------ softmax warpgroup
     const int q4 = warp & 3;                  // TMEM lane quarter this warp may access
     const int r = q4 * 32 + lane;             // query row within the tile
-    const long long i = i0 + r;
+    const long long qi = q0 + r;              // row in the view
+    const long long i = MODE == kResidue ? qi * prm.pi + res : qi;  // row in the sequence
     const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
 
     // gate on the unscaled query row (read from the swizzled Q tile)
-    bool ok = mbar_wait(bar_q, 0, abort_flag);
+    bool ok = __all_sync(0xffffffffu, mbar_wait(bar_q, 0, abort_flag));
     float z = prm.b_g[h];
     {
       const float* wg = prm.w_g + (long long)h * D;
@@ -373,15 +421,17 @@ __global__ void __launch_bounds__(NTHREADS, D == 64 ? 2 : 1) fwd_tc_kernel(const
         for (int e = 0; e < 8; ++e) z = fmaf(f[e], wg[c * 8 + e], z);
       }
     }
-    const float bias_l = log_sigmoid(z) * kLog2e;
-    const float bias_p = log_sigmoid(-z) * kLog2e;
+    // the prior of the keys this pass unmasks as "window" columns
+    const float bias_l = log_sigmoid(MODE == kResidue ? -z : z) * kLog2e;  // log2(alpha), or log2(1-alpha)
+    const float bias_p = log_sigmoid(-z) * kLog2e;                         // log2(1 - alpha)
     const float NEG_INF = -INFINITY;
 
     float m_ref = NEG_INF;  // reference max (log2 units)
     float l_sum = 0.f;      // running sum of probabilities against m_ref
     int j = 0;
     for (int t = walk.next(0); ok && t >= 0; t = walk.next(t + 1), ++j) {
-      if (!mbar_wait(bar_sfull, j & 1, abort_flag)) { ok = false; break; }
+      // every lane of the warp takes the same branch: the tcgen05.ld below is .sync.aligned
+      if (!__all_sync(0xffffffffu, mbar_wait(bar_sfull, j & 1, abort_flag))) { ok = false; break; }
       tc_fence_after();
       float x[BN];
 #pragma unroll
@@ -389,10 +439,13 @@ __global__ void __launch_bounds__(NTHREADS, D == 64 ? 2 : 1) fwd_tc_kernel(const
       tc_fence_before();
       mbar_arrive(bar_sfree);
 
-      // the index rule on this tile, for row i: window columns [lc_lo, lc_hi], skip columns bitmask
+      // the index rule on this tile, for row qi: window columns [lc_lo, lc_hi], skip columns bitmask
       int lc_lo, lc_hi;
       uint32_t sk[BN / 32];
-      row_tile_mask(i, (long long)t * BN, prm.kwin, prm.pi, prm.S, walk.m0, lc_lo, lc_hi, sk);
+      if (MODE == kResidue)
+        row_tile_mask(qi, (long long)t * BN, prm.S, 1, 0, 1, lc_lo, lc_hi, sk, m0);
+      else
+        row_tile_mask(qi, (long long)t * BN, prm.kwin, prm.pi, MODE == kFused ? prm.S : 0, m0, lc_lo, lc_hi, sk);
       // per 32-column chunk, the cheapest exact treatment for this row (see chunk_class)
       int cls[BN / 32];
       int one_col[BN / 32];
@@ -472,15 +525,18 @@ __global__ void __launch_bounds__(NTHREADS, D == 64 ? 2 : 1) fwd_tc_kernel(const
 
       // P buffer and O are free once the previous P.V has completed
       if (j > 0) {
-        if (!mbar_wait(bar_pvdone, (j - 1) & 1, abort_flag)) { ok = false; break; }
+        if (!__all_sync(0xffffffffu, mbar_wait(bar_pvdone, (j - 1) & 1, abort_flag))) { ok = false; break; }
         tc_fence_after();
-        if (rescale) {
+        // the rescale is per row, but TMEM access is per warp: the warp rescales when any of its
+        // rows needs it, the others multiply by 1
+        if (__any_sync(0xffffffffu, rescale)) {
+          const float f = rescale ? factor : 1.f;
 #pragma unroll
           for (int c = 0; c < D / 32; ++c) {
             float o[32];
             tmem_ld32(tO + lane_off + c * 32, o);
 #pragma unroll
-            for (int e = 0; e < 32; ++e) o[e] *= factor;
+            for (int e = 0; e < 32; ++e) o[e] *= f;
             tmem_st32(tO + lane_off + c * 32, o);
           }
           tmem_wait_st();
@@ -501,12 +557,28 @@ __global__ void __launch_bounds__(NTHREADS, D == 64 ? 2 : 1) fwd_tc_kernel(const
       tc_fence_before();
       mbar_arrive(bar_pfull);
     }
-    // epilogue: O / l_sum -> out (bf16), lse
-    if (ok && j > 0 && mbar_wait(bar_pvdone, (j - 1) & 1, abort_flag)) {
+    // ---- epilogue
+    const bool row_ok = qi < view_rows;
+    const long long orow = (long long)bh * prm.n + i;  // row in [B*H, n] layouts
+    const bool have_o = __all_sync(0xffffffffu, ok && j > 0 && mbar_wait(bar_pvdone, (j - 1) & 1, abort_flag));
+    if (have_o) {
       tc_fence_after();
-      const float inv = 1.f / l_sum;
-      const bool row_ok = i < prm.n;
-      __nv_bfloat16* orow = prm.out + ((long long)bh * prm.n + i) * D;
+      float inv = l_sum > 0.f ? 1.f / l_sum : 0.f;
+      float wl = 1.f, wp = 0.f, lse2 = m_ref + log2f(l_sum);  // log2 of this pass's mass
+      const uint4* so = nullptr;
+      if (MODE == kBandMerge && row_ok) {
+        // merge the skip partial of this row
+        const float b2 = prm.skip_lse[orow] * kLog2e;
+        const float M = fmaxf(lse2, b2);
+        wl = ex2(lse2 - M);
+        wp = ex2(b2 - M);
+        const float den = wl + wp;
+        wl /= den;
+        wp /= den;
+        lse2 = M + log2f(den);
+        so = reinterpret_cast<const uint4*>(prm.skip_o + orow * D);
+      }
+      __nv_bfloat16* orow_ptr = (MODE == kResidue ? prm.skip_o : prm.out) + orow * D;
 #pragma unroll
       for (int c = 0; c < D / 32; ++c) {
         float o[32];
@@ -514,22 +586,37 @@ __global__ void __launch_bounds__(NTHREADS, D == 64 ? 2 : 1) fwd_tc_kernel(const
         if (row_ok) {
 #pragma unroll
           for (int g = 0; g < 4; ++g) {
-            uint4 u;
+            float sp[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+            if (MODE == kBandMerge) bf16x8_to_f32(so[c * 4 + g], sp);
             uint32_t w[4];
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
-              __nv_bfloat162 b2 = __floats2bfloat162_rn(o[g * 8 + 2 * e] * inv, o[g * 8 + 2 * e + 1] * inv);
+              const float a0 = o[g * 8 + 2 * e] * inv * wl + sp[2 * e] * wp;
+              const float a1 = o[g * 8 + 2 * e + 1] * inv * wl + sp[2 * e + 1] * wp;
+              __nv_bfloat162 b2 = __floats2bfloat162_rn(a0, a1);
               w[e] = *reinterpret_cast<uint32_t*>(&b2);
             }
+            uint4 u;
             u.x = w[0];
             u.y = w[1];
             u.z = w[2];
             u.w = w[3];
-            *reinterpret_cast<uint4*>(orow + c * 32 + g * 8) = u;
+            *reinterpret_cast<uint4*>(orow_ptr + c * 32 + g * 8) = u;
           }
         }
       }
-      if (row_ok && prm.lse) prm.lse[(long long)bh * prm.n + i] = (m_ref + log2f(l_sum)) * kLn2;
+      if (row_ok) {
+        // a row with no key in this pass (only possible for kResidue) has lse -inf
+        const float lse_val = l_sum > 0.f ? lse2 * kLn2 : NEG_INF;
+        if (MODE == kResidue) prm.skip_lse[orow] = lse_val;
+        else if (prm.lse) prm.lse[orow] = lse_val;
+      }
+    } else if (MODE == kResidue && ok && j == 0 && row_ok) {
+      // no skip key for any row of this tile: empty partial
+      uint4 zero = make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+      for (int c = 0; c < D / 8; ++c) reinterpret_cast<uint4*>(prm.skip_o + orow * D)[c] = zero;
+      prm.skip_lse[orow] = NEG_INF;
     }
     tc_fence_before();
   }
@@ -553,7 +640,7 @@ inline PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
-// [B*H, n, d] bf16 viewed as a 3-D tensor (d innermost); box = 64 elements x 128 rows x 1.
+// [B*H, n, d] bf16 as a 3-D tensor (d innermost); box = 64 elements x 128 rows x 1.
 inline bool make_map(CUtensorMap* m, const void* ptr, int BH, int n, int d) {
   auto fn = encode_fn();
   if (!fn) return false;
@@ -567,14 +654,57 @@ inline bool make_map(CUtensorMap* m, const void* ptr, int BH, int n, int d) {
   return r == CUDA_SUCCESS;
 }
 
+// The residue-class view of [B*H, n, d] with n = T*pi: a 4-D tensor (d, residue, t, bh) in which
+// row t of residue r is sequence row t*pi + r; box = 64 elements x 1 residue x 128 rows x 1.
+inline bool make_residue_map(CUtensorMap* m, const void* ptr, int BH, int n, int d, int pi) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[4] = {(cuuint64_t)d, (cuuint64_t)pi, (cuuint64_t)(n / pi), (cuuint64_t)BH};
+  cuuint64_t strides[3] = {(cuuint64_t)d * 2, (cuuint64_t)pi * d * 2, (cuuint64_t)n * d * 2};
+  cuuint32_t box[4] = {64, 1, 128, 1};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(ptr), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+template <int D, int MODE>
+cudaError_t set_smem_attr() {
+  static bool done = false;
+  if (done) return cudaSuccess;
+  cudaError_t e = cudaFuncSetAttribute(fwd_tc_kernel<D, MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       Smem<D>::kAlloc);
+  if (e == cudaSuccess) done = true;
+  return e;
+}
+
 }  // namespace tc
 
 inline bool tc_supported(bool bf16, int d, int n) { return bf16 && (d == 64 || d == 128) && n >= 1; }
 
+// The split (residue pass + window pass) applies when the sequence is a whole number of periods
+// (the residue view is a plain 4-D tensor) and the residue sequences fit the int coordinates.
+inline bool tc_split_applies(int n, int kwin, int pi, int S) {
+  const int m0 = first_skip_m(kwin, pi);
+  return S >= m0 && n % pi == 0 && (long long)pi * ((n / pi + tc::BM - 1) / tc::BM) < 0x7fffffffLL;
+}
+
+// Pick the split when the skips would cost more tensor work as diagonal tiles than the extra
+// HBM traffic of the split costs: diagonal skip tiles ~ S' per query tile vs ~(k + 128)/128 window
+// tiles; the split adds ~1.3 KB of traffic per row.
+inline bool tc_split_preferred(int n, int kwin, int pi, int S) {
+  if (!tc_split_applies(n, kwin, pi, S)) return false;
+  const int m0 = first_skip_m(kwin, pi);
+  const int nskip = S - m0 + 1;
+  const int band_tiles = (kwin + 127) / 128 + 1;
+  return pi >= tc::BN && nskip > 2 * band_tiles;
+}
+
 template <int D>
 cudaError_t launch_fwd_tc_d(const void* q, const void* k, const void* v, const float* w_g, const float* b_g,
-                            void* out, float* lse, int B, int H, int n, int kwin, int pi, int S, cudaStream_t st,
-                            const char** why) {
+                            void* out, float* lse, int B, int H, int n, int kwin, int pi, int S, bool split,
+                            cudaStream_t st, const char** why) {
   using L = tc::Smem<D>;
   CUtensorMap mq, mk, mv;
   const int BH = B * H;
@@ -582,37 +712,64 @@ cudaError_t launch_fwd_tc_d(const void* q, const void* k, const void* v, const f
     *why = "cuTensorMapEncodeTiled failed";
     return cudaErrorInvalidValue;
   }
-  static bool attr_done = false;
-  if (!attr_done) {
-    cudaError_t e = cudaFuncSetAttribute(tc::fwd_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc);
-    if (e != cudaSuccess) {
-      *why = "cudaFuncSetAttribute(max dynamic shared memory)";
-      return e;
-    }
-    attr_done = true;
-  }
   tc::Params p;
   p.w_g = w_g;
   p.b_g = b_g;
   p.out = (__nv_bfloat16*)out;
   p.lse = lse;
+  p.skip_o = nullptr;
+  p.skip_lse = nullptr;
   p.H = H;
   p.n = n;
   p.kwin = kwin;
   p.pi = pi;
   p.S = S;
+  p.T = n / pi;
   p.scale_log2 = (float)(1.0 / std::sqrt((double)D)) * kLog2e;
-  dim3 grid((unsigned)((n + tc::BM - 1) / tc::BM), (unsigned)BH);
-  tc::fwd_tc_kernel<D><<<grid, tc::NTHREADS, L::kAlloc, st>>>(mq, mk, mv, p);
-  *why = "tensor-core kernel launch";
-  return cudaGetLastError();
+  const dim3 grid((unsigned)((n + tc::BM - 1) / tc::BM), (unsigned)BH);
+  cudaError_t e;
+  if (!split) {
+    if ((e = tc::set_smem_attr<D, tc::kFused>()) != cudaSuccess) { *why = "cudaFuncSetAttribute"; return e; }
+    tc::fwd_tc_kernel<D, tc::kFused><<<grid, tc::NTHREADS, L::kAlloc, st>>>(mq, mk, mv, p);
+    *why = "tensor-core kernel launch";
+    return cudaGetLastError();
+  }
+  CUtensorMap rq, rk, rv;
+  if (!tc::make_residue_map(&rq, q, BH, n, D, pi) || !tc::make_residue_map(&rk, k, BH, n, D, pi) ||
+      !tc::make_residue_map(&rv, v, BH, n, D, pi)) {
+    *why = "cuTensorMapEncodeTiled (residue view) failed";
+    return cudaErrorInvalidValue;
+  }
+  if ((e = tc::set_smem_attr<D, tc::kResidue>()) != cudaSuccess) { *why = "cudaFuncSetAttribute"; return e; }
+  if ((e = tc::set_smem_attr<D, tc::kBandMerge>()) != cudaSuccess) { *why = "cudaFuncSetAttribute"; return e; }
+  // scratch for the skip partials: [B*H, n, D] bf16 + [B*H, n] fp32, stream-ordered
+  const size_t rows = (size_t)BH * n;
+  void* scratch = nullptr;
+  if ((e = cudaMallocAsync(&scratch, rows * (D * 2 + 4), st)) != cudaSuccess) {
+    *why = "skip-partial scratch allocation";
+    return e;
+  }
+  p.skip_o = (__nv_bfloat16*)scratch;
+  p.skip_lse = (float*)((char*)scratch + rows * D * 2);
+  const dim3 grid_r((unsigned)(pi * ((p.T + tc::BM - 1) / tc::BM)), (unsigned)BH);
+  tc::fwd_tc_kernel<D, tc::kResidue><<<grid_r, tc::NTHREADS, L::kAlloc, st>>>(rq, rk, rv, p);
+  e = cudaGetLastError();
+  if (e == cudaSuccess) {
+    tc::fwd_tc_kernel<D, tc::kBandMerge><<<grid, tc::NTHREADS, L::kAlloc, st>>>(mq, mk, mv, p);
+    e = cudaGetLastError();
+  }
+  cudaError_t e2 = cudaFreeAsync(scratch, st);
+  *why = "tensor-core split kernels";
+  return e != cudaSuccess ? e : e2;
 }
 
+// mode: 0 = choose, 1 = single pass, 2 = split (residue pass + window pass)
 inline cudaError_t launch_fwd_tc(const void* q, const void* k, const void* v, const float* w_g, const float* b_g,
-                                 void* out, float* lse, int B, int H, int n, int d, int kwin, int pi, int S,
+                                 void* out, float* lse, int B, int H, int n, int d, int kwin, int pi, int S, int mode,
                                  cudaStream_t st, const char** why) {
-  if (d == 128) return launch_fwd_tc_d<128>(q, k, v, w_g, b_g, out, lse, B, H, n, kwin, pi, S, st, why);
-  return launch_fwd_tc_d<64>(q, k, v, w_g, b_g, out, lse, B, H, n, kwin, pi, S, st, why);
+  const bool split = mode == 2 || (mode == 0 && tc_split_preferred(n, kwin, pi, S));
+  if (d == 128) return launch_fwd_tc_d<128>(q, k, v, w_g, b_g, out, lse, B, H, n, kwin, pi, S, split, st, why);
+  return launch_fwd_tc_d<64>(q, k, v, w_g, b_g, out, lse, B, H, n, kwin, pi, S, split, st, why);
 }
 
 }  // namespace pia

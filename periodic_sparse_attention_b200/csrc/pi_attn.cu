@@ -106,16 +106,19 @@ pi_attn_status pi_attn_fwd_ex(const void* q, const void* k, const void* v, const
                               pi_attn_dtype dtype, pi_attn_path path, void* stream) {
   pi_attn_status st = check_common(q, k, v, w_g, b_g, out, B, H, n, d, k_win, pi, S, dtype);
   if (st != PI_ATTN_OK) return st;
-  if (path != PI_ATTN_PATH_AUTO && path != PI_ATTN_PATH_SIMT && path != PI_ATTN_PATH_TC)
-    return fail(PI_ATTN_EINVAL, "unknown path %d", (int)path);
+  if (path < PI_ATTN_PATH_AUTO || path > PI_ATTN_PATH_TC_SPLIT) return fail(PI_ATTN_EINVAL, "unknown path %d", (int)path);
   const bool tc_ok = pia::tc_supported(dtype == PI_ATTN_BF16, d, n);
-  if (path == PI_ATTN_PATH_TC && !tc_ok)
+  const bool want_tc = path == PI_ATTN_PATH_TC || path == PI_ATTN_PATH_TC_FUSED || path == PI_ATTN_PATH_TC_SPLIT;
+  if (want_tc && !tc_ok)
     return fail(PI_ATTN_EUNSUPPORTED, "tensor-core path covers bf16 with d in {64, 128} (got dtype %d, d %d)",
                 (int)dtype, d);
+  if (path == PI_ATTN_PATH_TC_SPLIT && !pia::tc_split_applies(n, k_win, pi, S))
+    return fail(PI_ATTN_EUNSUPPORTED, "split path needs n %% pi == 0 and at least one skip outside the window");
   cudaStream_t s = as_stream(stream);
   if (path != PI_ATTN_PATH_SIMT && tc_ok) {
     const char* why = nullptr;
-    cudaError_t e = pia::launch_fwd_tc(q, k, v, w_g, b_g, out, lse, B, H, n, d, k_win, pi, S, s, &why);
+    const int mode = path == PI_ATTN_PATH_TC_FUSED ? 1 : path == PI_ATTN_PATH_TC_SPLIT ? 2 : 0;
+    cudaError_t e = pia::launch_fwd_tc(q, k, v, w_g, b_g, out, lse, B, H, n, d, k_win, pi, S, mode, s, &why);
     if (e != cudaSuccess) return cuda_fail(e, why ? why : "tensor-core kernel launch");
     return ok();
   }
@@ -141,10 +144,10 @@ pi_attn_status pi_attn_decode(const void* q, const void* kcache, const void* vca
     if (bh > 0x7fffffffLL) return fail(PI_ATTN_EINVAL, "B * H too large");
     // Split each (b, h) across CTAs only when there are too few (b, h) to fill the GPU.
     const long long rows = (long long)k_win + 1 + S;
-    const long long want = 4LL * num_sms() * 14;  // ~14 two-warp CTAs per SM, four waves' worth
+    const long long slots = 14LL * num_sms();  // two-warp CTAs resident at once (~14 per SM)
     int nsplit = 1;
-    if (bh * 4 < want) {
-      long long ns = (want + bh - 1) / bh;
+    if (bh * 2 < slots) {
+      long long ns = (slots + bh - 1) / bh;
       const long long max_ns = (rows + 127) / 128;  // keep >= 128 rows per split
       if (ns > max_ns) ns = max_ns;
       if (ns > 64) ns = 64;

@@ -53,12 +53,16 @@ struct TileWalk {
 
 // For query row i and the key tile starting at j0: window columns [lc_lo, lc_hi] (empty when
 // lc_lo > lc_hi) and a 128-bit mask of skip columns.  Skip columns never overlap the window.
+// The window of row i is [max(0, i - kwin), i - lo_off]: lo_off = 0 for pi-attention's window;
+// the residue-class pass uses it for the skip band of a residue sequence (kwin = S, lo_off = m0,
+// no skips).
 PIA_HD void row_tile_mask(long long i, long long j0, int kwin, int pi, int S, int m0, int& lc_lo, int& lc_hi,
-                          uint32_t sk[kTileKeys / 32]) {
+                          uint32_t sk[kTileKeys / 32], int lo_off = 0) {
   const long long d0 = i - j0;  // i - j at column 0
   const long long lo = (i - kwin > 0 ? i - kwin : 0) - j0;
+  const long long hi = d0 - lo_off;
   lc_lo = lo < 0 ? 0 : (lo > kTileKeys ? kTileKeys : (int)lo);
-  lc_hi = d0 > kTileKeys - 1 ? kTileKeys - 1 : (d0 < -1 ? -1 : (int)d0);
+  lc_hi = hi > kTileKeys - 1 ? kTileKeys - 1 : (hi < -1 ? -1 : (int)hi);
   for (int w = 0; w < kTileKeys / 32; ++w) sk[w] = 0u;
   if (d0 > kwin && S >= m0) {
     long long m_hi = d0 / pi;

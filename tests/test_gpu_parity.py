@@ -66,7 +66,7 @@ def test_tiny_f32_every_row():
     assert_close(metrics(out, ro, lse, rl), "f32", "tiny_f32")
 
 
-@pytest.mark.parametrize("path", ["auto", "simt", TC])
+@pytest.mark.parametrize("path", ["auto", "simt", TC, "tc_fused", "tc_split"])
 def test_bf16_n4k_every_row(path):
     w = ps.WORKLOADS["bf16_n4k"]
     inp = ps.prefill_inputs(w)
@@ -75,11 +75,12 @@ def test_bf16_n4k_every_row(path):
     assert_close(metrics(out, ro, lse, rl), "bf16", f"bf16_n4k/{path}")
 
 
+@pytest.mark.parametrize("path", ["auto", "tc_fused", "tc_split"])
 @pytest.mark.parametrize("name", ["bf16_n32k", "bf16_n128k"])
-def test_long_workloads_sampled_rows(name):
+def test_long_workloads_sampled_rows(name, path):
     w = ps.WORKLOADS[name]
     inp = ps.prefill_inputs(w)
-    out, lse = _run_fwd(inp, "bf16", w.k, w.pi, w.S)
+    out, lse = _run_fwd(inp, "bf16", w.k, w.pi, w.S, path)
     rows = sampled_rows(w, 4096)
     ro, rl, _ = oracle.fwd_rows(inp["q"], inp["k"], inp["v"], inp["w_g"], inp["b_g"], w.k, w.pi, w.S, rows=rows)
     m = metrics(out.reshape(-1, w.d)[rows], ro, lse.reshape(-1)[rows], rl)
@@ -136,16 +137,26 @@ EDGE = [  # B, H, n, d, k, pi, S
     (1, 1, 130, 64, 5, 7, 3),       # tiny window, ragged
     (2, 2, 640, 128, 0, 128, 4),    # window of the token alone
     (1, 1, 385, 64, 127, 129, 2),   # window just under a tile, period just over
+    (1, 2, 1024, 128, 64, 256, 3),  # residue sequences of 4 rows
+    (2, 1, 2048, 64, 100, 128, 8),  # residue sequences of 16 rows, first skip m = 1
+    (1, 1, 4096, 128, 300, 256, 12),  # first surviving skip m = 2
+    (1, 1, 2112, 64, 10, 64, 40),   # 33 rows per residue, skips reach the start
 ]
 
 
-@pytest.mark.parametrize("path", ["auto", "simt", TC])
+def _split_applies(n, k, pi, S):
+    return n % pi == 0 and S >= k // pi + 1
+
+
+@pytest.mark.parametrize("path", ["auto", "simt", TC, "tc_fused", "tc_split"])
 @pytest.mark.parametrize("case", EDGE)
 def test_edge_cases_bf16(case, path):
     B, H, n, d, k, pi, S = case
     inp = _inputs(B, H, n, d, "bf16", seed=n + 7 * k)
-    if path == TC and not _tc_applies("bf16", d):
+    if path.startswith("tc") and not _tc_applies("bf16", d):
         pytest.skip("tensor-core path does not cover this head size")
+    if path == "tc_split" and not _split_applies(n, k, pi, S):
+        pytest.skip("split path needs n % pi == 0 and a skip outside the window")
     out, lse = _run_fwd(inp, "bf16", k, pi, S, path)
     ro, rl, _ = oracle.fwd(inp["q"], inp["k"], inp["v"], inp["w_g"], inp["b_g"], k, pi, S)
     assert_close(metrics(out, ro, lse, rl), "bf16", f"{case}/{path}")
@@ -161,10 +172,10 @@ def test_edge_cases_f32(case):
     assert_close(metrics(out, ro, lse, rl), "f32", str(case))
 
 
-@pytest.mark.parametrize("path", ["auto", "simt"])
+@pytest.mark.parametrize("path", ["auto", "simt", "tc_fused", "tc_split"])
 @pytest.mark.parametrize("bias", [60.0, -60.0])
 def test_gate_saturation(bias, path):
-    B, H, n, d, k, pi, S = 1, 2, 700, 128, 64, 96, 6
+    B, H, n, d, k, pi, S = 1, 2, 768, 128, 64, 96, 6
     inp = _inputs(B, H, n, d, "bf16", seed=11)
     inp["w_g"][:] = 0
     inp["b_g"][:] = bias
@@ -173,10 +184,10 @@ def test_gate_saturation(bias, path):
     assert_close(metrics(out, ro, lse, rl), "bf16", f"bias {bias}/{path}")
 
 
-@pytest.mark.parametrize("path", ["auto", "simt"])
+@pytest.mark.parametrize("path", ["auto", "simt", "tc_fused", "tc_split"])
 def test_rows_are_normalised(path):
     # V = 1 everywhere: every output element must be 1 (the weights of each row sum to one)
-    inp = _inputs(1, 4, 1100, 128, "bf16", seed=3)
+    inp = _inputs(1, 4, 1280, 128, "bf16", seed=3)
     inp["v"][:] = 0x3F80  # bf16 1.0
     out, _ = _run_fwd(inp, "bf16", 256, 256, 8, path)
     assert np.max(np.abs(out - 1.0)) <= 4e-3
