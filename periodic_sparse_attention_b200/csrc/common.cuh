@@ -67,7 +67,8 @@ __device__ __forceinline__ uint64_t global_ns() {
   asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
   return t;
 }
-// Upper bound for any wait inside a kernel.  A healthy pipeline waits microseconds.
-constexpr uint64_t kWaitLimitNs = 2000000000ull;
+// Upper bound for any wait inside a kernel, in SM clock cycles (about 2 s at the B200's 1.965 GHz
+// boost clock, longer at lower clocks).  A healthy pipeline waits microseconds.
+constexpr long long kWaitLimitCycles = 4000000000ll;
 
 }  // namespace pia

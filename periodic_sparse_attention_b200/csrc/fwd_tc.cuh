@@ -80,17 +80,24 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
       : "memory");
   return ok != 0;
 }
-// Bounded wait: false when the limit passed or another thread of the CTA aborted.
+// Bounded wait: false when the limit passed or another thread of the CTA aborted.  The loop spins
+// on try_wait alone; the abort flag and the SM clock are looked at only every 64 failed tries, so
+// noticing a completed phase costs one try_wait, not a clock read.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag) {
   if (mbar_try_wait(bar, parity)) return true;
-  const uint64_t t0 = global_ns();
-  while (true) {
+  long long t0 = 0;
+  for (uint32_t it = 1;; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
-    if (*abort_flag) return false;
-    if (global_ns() - t0 > kWaitLimitNs) {
-      raise_error(kErrWaitTimeout);
-      *abort_flag = 1;
-      return false;
+    if ((it & 63u) == 0u) {
+      if (*abort_flag) return false;
+      const long long now = clock64();
+      if (t0 == 0) {
+        t0 = now;
+      } else if (now - t0 > kWaitLimitCycles) {
+        raise_error(kErrWaitTimeout);
+        *abort_flag = 1;
+        return false;
+      }
     }
   }
 }
@@ -459,11 +466,13 @@ __global__ void __launch_bounds__(NTHREADS, D == 64 ? 2 : 1) fwd_tc_kernel(const
         one_col[cb] = 0;
         one_x[cb] = NEG_INF;
         if (cls[cb] == kFull) {
+          float mp[4] = {NEG_INF, NEG_INF, NEG_INF, NEG_INF};  // independent chains
 #pragma unroll
           for (int e = 0; e < 32; ++e) {
             x[c0 + e] = fmaf(x[c0 + e], prm.scale_log2, bias_l);
-            mt = fmaxf(mt, x[c0 + e]);
+            mp[e & 3] = fmaxf(mp[e & 3], x[c0 + e]);
           }
+          mt = fmaxf(mt, fmaxf(fmaxf(mp[0], mp[1]), fmaxf(mp[2], mp[3])));
         } else if (cls[cb] == kOne) {
           const int sc = __ffs(skb) - 1;
           float xs = 0.f;
@@ -473,6 +482,7 @@ __global__ void __launch_bounds__(NTHREADS, D == 64 ? 2 : 1) fwd_tc_kernel(const
           one_x[cb] = fmaf(xs, prm.scale_log2, bias_p);
           mt = fmaxf(mt, one_x[cb]);
         } else if (cls[cb] == kMixed) {
+          float mp[4] = {NEG_INF, NEG_INF, NEG_INF, NEG_INF};
 #pragma unroll
           for (int e = 0; e < 32; ++e) {
             const int c = c0 + e;
@@ -480,8 +490,9 @@ __global__ void __launch_bounds__(NTHREADS, D == 64 ? 2 : 1) fwd_tc_kernel(const
             const bool skp = (skb >> e) & 1u;
             const float b = loc ? bias_l : (skp ? bias_p : NEG_INF);
             x[c] = fmaf(x[c], prm.scale_log2, b);
-            mt = fmaxf(mt, x[c]);
+            mp[e & 3] = fmaxf(mp[e & 3], x[c]);
           }
+          mt = fmaxf(mt, fmaxf(fmaxf(mp[0], mp[1]), fmaxf(mp[2], mp[3])));
         }
       }
       // lazy reference max
@@ -501,13 +512,15 @@ __global__ void __launch_bounds__(NTHREADS, D == 64 ? 2 : 1) fwd_tc_kernel(const
       for (int cb = 0; cb < BN / 32; ++cb) {
         const int c0 = cb * 32;
         if (cls[cb] == kFull || cls[cb] == kMixed) {
+          float sp[4] = {0.f, 0.f, 0.f, 0.f};  // independent chains
 #pragma unroll
           for (int e = 0; e < 32; e += 2) {
             const float p0 = ex2(x[c0 + e] - m_use), p1 = ex2(x[c0 + e + 1] - m_use);
-            ls += p0 + p1;
+            sp[(e >> 1) & 3] += p0 + p1;
             __nv_bfloat162 b2 = __floats2bfloat162_rn(p0, p1);
             pk[(c0 + e) / 2] = *reinterpret_cast<uint32_t*>(&b2);
           }
+          ls += (sp[0] + sp[1]) + (sp[2] + sp[3]);
         } else if (cls[cb] == kOne) {
           const float p1 = ex2(one_x[cb] - m_use);
           ls += p1;
