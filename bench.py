@@ -79,25 +79,36 @@ def load_peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
-def source_hash() -> str:
+KERNEL_FILES = {  # sources of each timed kernel (for matching committed ncu counters to the code)
+    "prefill": ["fwd_tc.cuh", "tile_rule.cuh", "common.cuh"],
+    "decode": ["decode.cuh", "common.cuh"],
+}
+
+
+def source_hash(files=None) -> str:
+    """Hash of kernel sources: the listed csrc files, or every csrc/include source when None."""
     h = hashlib.sha256()
-    for sub in ("periodic_sparse_attention_b200/csrc", "include"):
-        base = os.path.join(ROOT, sub)
-        for fn in sorted(os.listdir(base)):
-            if fn.endswith((".cu", ".cuh", ".h")):
-                with open(os.path.join(base, fn), "rb") as f:
-                    h.update(fn.encode() + b"\0" + f.read())
+    if files is None:
+        paths = []
+        for sub in ("periodic_sparse_attention_b200/csrc", "include"):
+            base = os.path.join(ROOT, sub)
+            paths += [os.path.join(base, fn) for fn in sorted(os.listdir(base)) if fn.endswith((".cu", ".cuh", ".h"))]
+    else:
+        paths = [os.path.join(ROOT, "periodic_sparse_attention_b200", "csrc", fn) for fn in files]
+    for path in paths:
+        with open(path, "rb") as f:
+            h.update(os.path.basename(path).encode() + b"\0" + f.read())
     return h.hexdigest()[:16]
 
 
 def profiled_traffic(workload: str):
     """DRAM bytes per launch of the timed kernel from the committed ncu summaries, if they were
-    taken on the current kernel source (a line `bench-traffic: workload=.. bytes_per_launch=..
-    source_sha=..` in profiles/*.md); otherwise None."""
+    taken on the current kernel source: a line
+      bench-traffic: workload=.. bytes_per_launch=.. files=a.cuh,b.cuh source_sha=..
+    in profiles/*.md whose files still hash to source_sha.  Otherwise None."""
     d = os.path.join(ROOT, "profiles")
     if not os.path.isdir(d):
         return None
-    want = source_hash()
     for fn in sorted(os.listdir(d)):
         if not fn.endswith((".md", ".txt")):
             continue
@@ -105,8 +116,13 @@ def profiled_traffic(workload: str):
             for line in f:
                 if line.startswith("bench-traffic:"):
                     kv = dict(x.split("=", 1) for x in line.split()[1:] if "=" in x)
-                    if kv.get("workload") == workload and kv.get("source_sha") == want:
-                        return int(kv["bytes_per_launch"])
+                    if kv.get("workload") != workload or "files" not in kv:
+                        continue
+                    try:
+                        if kv.get("source_sha") == source_hash(kv["files"].split(",")):
+                            return int(kv["bytes_per_launch"])
+                    except OSError:
+                        continue
     return None
 
 
@@ -305,8 +321,8 @@ def run_gpu(args):
     if w.kind == "prefill":
         def step():
             pia.pi_attn_fwd(t["q"], t["k"], t["v"], t["w_g"], t["b_g"], w.k, w.pi, w.S, out=out, lse=lse,
-                            stream=stream)
-        launches_per_step = 1
+                            stream=stream, path=args.path)
+        launches_per_step, _ = pia.pi_attn_fwd_plan(w.B, w.H, w.n, w.d, w.k, w.pi, w.S, w.dtype, args.path)
     else:
         def step():
             pia.pi_attn_decode(t["q"], t["k"], t["v"], t["w_g"], t["b_g"], w.k, w.pi, w.S, out=out, lse=lse,
@@ -411,8 +427,8 @@ def run_gpu(args):
                        parallelism=f"replicas x{world} (independent (b, h) batches)"),
         "achieved_tflops": flops / launch_s / 1e12, "achieved_gbs": bytes_ / launch_s / 1e9,
         "roofline": roof, "cpu_baseline": cpu, "e2e": e2e,
-        "gpu_launches": launches_per_step * args.steps, "clocks": clocks.summary(),
-        "kernel_source_sha": source_hash(),
+        "gpu_launches": launches_per_step * args.steps, "clocks": clocks.summary(), "path": args.path,
+        "kernel_source_sha": source_hash(KERNEL_FILES[w.kind]),
     }
     if rank == 0:
         print(json.dumps(line), flush=True)
@@ -461,6 +477,8 @@ def main(argv=None):
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(ps.WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--path", default="auto", choices=["auto", "simt", "tc", "tc_fused", "tc_split"],
+                    help="prefill kernel choice (pi_attn_fwd_ex path)")
     ap.add_argument("--cpu-budget", type=float, default=10.0, help="seconds of oracle work for cpu_baseline")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args(argv)

@@ -76,6 +76,13 @@ pi_attn_status pi_attn_fwd_ex(const void* q, const void* k, const void* v, const
                               void* out, float* lse, int B, int H, int n, int d, int k_win, int pi, int S,
                               pi_attn_dtype dtype, pi_attn_path path, void* stream);
 
+/* What a pi_attn_fwd_ex call with these arguments would launch, without launching anything:
+ * *launches = number of kernel launches (1 for a single pass, 2 for the split), *scratch_bytes =
+ * device scratch it takes from cudaMallocAsync on the stream (0 for a single pass).  Returns
+ * PI_ATTN_EUNSUPPORTED / PI_ATTN_EINVAL exactly where pi_attn_fwd_ex would. */
+pi_attn_status pi_attn_fwd_plan(int B, int H, int n, int d, int k_win, int pi, int S, pi_attn_dtype dtype,
+                                pi_attn_path path, int* launches, long long* scratch_bytes);
+
 /* Single-step decode.  Cited passage: "Inference" under "Execution & Scheduling" of the
  * pi-Attention method section (a new token reads its window and its periodic skips).  For each
  * (b, h) the query q[b, h] is the token at position len_b - 1 of a cache that already holds it,

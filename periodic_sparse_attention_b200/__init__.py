@@ -27,6 +27,8 @@ SIGNATURES = {
     "pi_attn_fwd": (_i32, [_vp] * 7 + [_i32] * 8 + [_vp]),
     # ... as above plus the path selector
     "pi_attn_fwd_ex": (_i32, [_vp] * 7 + [_i32] * 9 + [_vp]),
+    # B H n d k_win pi S, dtype, path, out: launches, scratch bytes
+    "pi_attn_fwd_plan": (_i32, [_i32] * 9 + [_vp, _vp]),
     # 8 pointers (q kcache vcache w_g b_g cache_len out lse), B H n_cache d k_win pi S, dtype, stream
     "pi_attn_decode": (_i32, [_vp] * 8 + [_i32] * 8 + [_vp]),
     "pi_attn_debug_index_sets": (_i32, [_i32, _i32, _i32, _i32, _vp, _vp, _i32, _vp]),
@@ -111,6 +113,17 @@ def pi_attn_fwd(q, k, v, w_g, b_g, k_win: int, pi: int, S: int, out=None, lse=No
                                k_win, pi, S, _dtype_code(q), PATHS[path], _stream(stream))
     _raise(st)
     return out, lse
+
+
+def pi_attn_fwd_plan(B: int, H: int, n: int, d: int, k_win: int, pi: int, S: int, dtype: str = "bf16",
+                     path: str = "auto"):
+    """(kernel launches, scratch bytes) a pi_attn_fwd_ex call would use, without launching."""
+    launches = ctypes.c_int(0)
+    scratch = ctypes.c_longlong(0)
+    st = load().pi_attn_fwd_plan(B, H, n, d, k_win, pi, S, PI_ATTN_BF16 if dtype == "bf16" else PI_ATTN_F32,
+                                 PATHS[path], ctypes.byref(launches), ctypes.byref(scratch))
+    _raise(st)
+    return launches.value, scratch.value
 
 
 def pi_attn_decode(q, kcache, vcache, w_g, b_g, k_win: int, pi: int, S: int, cache_len=None, out=None, lse=None, *,

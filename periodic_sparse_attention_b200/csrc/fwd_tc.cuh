@@ -49,8 +49,13 @@ struct Smem {
   static constexpr int kV = kK + NSTAGE * kTileBytes;
   static constexpr int kP = kV + NSTAGE * kTileBytes;
   static constexpr int kBar = kP + BM * BN * 2;          // P: 128 x 128 bf16
-  // barriers: q_full, k_full[2], k_empty[2], v_full[2], v_empty[2], s_full, s_free, p_full, pv_done, drain
-  static constexpr int kNumBars = 1 + 4 * NSTAGE + 5;
+  // S buffers in TMEM: two for d = 128 (one CTA per SM: the next tile's Q.K^T overlaps this
+  // tile's softmax), one for d = 64 (two CTAs per SM overlap each other instead)
+  static constexpr int kSBufs = D == 128 ? 2 : 1;
+  static constexpr int kTmemCols = kSBufs == 2 ? 512 : 256;  // S buffers (128 each) + O (D)
+  // barriers: q_full, k_full[2], k_empty[2], v_full[2], v_empty[2], s_full[NSB], s_free[NSB],
+  // p_full, pv_done, drain
+  static constexpr int kNumBars = 1 + 4 * NSTAGE + 2 * kSBufs + 3;
   static constexpr int kMisc = kBar + kNumBars * 8;      // tmem base (4 B), abort flag (4 B)
   static constexpr int kTotal = kMisc + 16;
   static constexpr int kAlloc = kTotal + 1024 - 128;     // slack to align a (>= 128 B aligned) base to 1 KB
@@ -265,11 +270,12 @@ __global__ void __launch_bounds__(NTHREADS, D == 64 ? 2 : 1) fwd_tc_kernel(const
   auto bar_kempty = [&](int s) { return bar0 + 8u * (1 + NSTAGE + s); };
   auto bar_vfull = [&](int s) { return bar0 + 8u * (1 + 2 * NSTAGE + s); };
   auto bar_vempty = [&](int s) { return bar0 + 8u * (1 + 3 * NSTAGE + s); };
-  const uint32_t bar_sfull = bar0 + 8u * (1 + 4 * NSTAGE);
-  const uint32_t bar_sfree = bar_sfull + 8;
-  const uint32_t bar_pfull = bar_sfull + 16;
-  const uint32_t bar_pvdone = bar_sfull + 24;
-  const uint32_t bar_drain = bar_sfull + 32;
+  constexpr int NSB = L::kSBufs;
+  auto bar_sfull = [&](int b) { return bar0 + 8u * (1 + 4 * NSTAGE + b); };
+  auto bar_sfree = [&](int b) { return bar0 + 8u * (1 + 4 * NSTAGE + NSB + b); };
+  const uint32_t bar_pfull = bar0 + 8u * (1 + 4 * NSTAGE + 2 * NSB);
+  const uint32_t bar_pvdone = bar_pfull + 8;
+  const uint32_t bar_drain = bar_pfull + 16;
   uint32_t* const tmem_slot = reinterpret_cast<uint32_t*>(sbase + L::kMisc);
   volatile int* const abort_flag = reinterpret_cast<volatile int*>(sbase + L::kMisc + 4);
 
@@ -281,16 +287,19 @@ __global__ void __launch_bounds__(NTHREADS, D == 64 ? 2 : 1) fwd_tc_kernel(const
       mbar_init(bar_vfull(s), 1);
       mbar_init(bar_vempty(s), 1);
     }
-    mbar_init(bar_sfull, 1);
-    mbar_init(bar_sfree, BM);
+    for (int b = 0; b < NSB; ++b) {
+      mbar_init(bar_sfull(b), 1);
+      mbar_init(bar_sfree(b), BM);
+    }
     mbar_init(bar_pfull, BM);
     mbar_init(bar_pvdone, 1);
     mbar_init(bar_drain, 1);
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
-  if (warp == 1) {  // TMEM: S in columns [0, 128), O in [128, 128 + D)
-    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], 256;" ::"r"(smem_u32(tmem_slot))
+  if (warp == 1) {  // TMEM: S buffer b in columns [128 b, 128 b + 128), O in [128 NSB, 128 NSB + D)
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
+                 "n"(L::kTmemCols)
                  : "memory");
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
   }
@@ -298,7 +307,7 @@ __global__ void __launch_bounds__(NTHREADS, D == 64 ? 2 : 1) fwd_tc_kernel(const
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const uint32_t tS = tmem, tO = tmem + 128;
+  const uint32_t tS = tmem, tO = tmem + 128 * NSB;  // S buffer b at tS + 128 b
 
   // one 128-row tile of the view (rows r0 .. r0+127) into shared memory, D/64 boxes of 64 columns
   auto load_tile = [&](uint32_t dst, const CUtensorMap* map, uint32_t bar, long long r0) {
@@ -347,12 +356,12 @@ __global__ void __launch_bounds__(NTHREADS, D == 64 ? 2 : 1) fwd_tc_kernel(const
       constexpr uint32_t idesc_pv = idesc_bf16(BM, D, 1);
       bool okw = mbar_wait(bar_q, 0, abort_flag);
       tc_fence_after();
-      // S = Q K_j^T : K = D, 16 per instruction; 64-column blocks of 16 KB
-      auto issue_qk = [&](int s) {
+      // S_j = Q K_j^T into S buffer j % NSB : K = D, 16 per instruction; 64-column blocks of 16 KB
+      auto issue_qk = [&](int s, int b) {
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk >> 2) * (BM * 128) + (kk & 3) * 32;
-          tc_mma(tS, sw128_desc(sQ + off, 16, 1024), sw128_desc(sK + s * kTile + off, 16, 1024), idesc_qk,
+          tc_mma(tS + 128 * b, sw128_desc(sQ + off, 16, 1024), sw128_desc(sK + s * kTile + off, 16, 1024), idesc_qk,
                  kk > 0 ? 1u : 0u);
         }
       };
@@ -366,29 +375,24 @@ __global__ void __launch_bounds__(NTHREADS, D == 64 ? 2 : 1) fwd_tc_kernel(const
                  (first && kk == 0) ? 0u : 1u);
         }
       };
+      // Q.K^T of tile j needs its K stage loaded and its S buffer released by tile j - NSB
+      auto try_qk = [&](int jq) -> bool {
+        const int s = jq % NSTAGE, b = jq % NSB;
+        if (!mbar_wait(bar_kfull(s), (jq / NSTAGE) & 1, abort_flag)) return false;
+        if (jq >= NSB && !mbar_wait(bar_sfree(b), (jq / NSB - 1) & 1, abort_flag)) return false;
+        tc_fence_after();
+        issue_qk(s, b);
+        tc_commit(bar_sfull(b));
+        tc_commit(bar_kempty(s));
+        return true;
+      };
       int j = 0;
       int t = walk.next(0);
-      if (okw && t >= 0) {
-        okw = mbar_wait(bar_kfull(0), 0, abort_flag);
-        if (okw) {
-          tc_fence_after();
-          issue_qk(0);
-          tc_commit(bar_sfull);
-          tc_commit(bar_kempty(0));
-        }
-      }
+      if (okw && t >= 0) okw = try_qk(0);
       while (okw && t >= 0) {
         const int tn = walk.next(t + 1);
         const int s = j % NSTAGE;
-        if (tn >= 0) {
-          const int jn = j + 1, sn = jn % NSTAGE;
-          if (!mbar_wait(bar_kfull(sn), (jn / NSTAGE) & 1, abort_flag)) break;
-          if (!mbar_wait(bar_sfree, j & 1, abort_flag)) break;
-          tc_fence_after();
-          issue_qk(sn);
-          tc_commit(bar_sfull);
-          tc_commit(bar_kempty(sn));
-        }
+        if (tn >= 0 && !try_qk(j + 1)) break;
         if (!mbar_wait(bar_vfull(s), (j / NSTAGE) & 1, abort_flag)) break;
         if (!mbar_wait(bar_pfull, j & 1, abort_flag)) break;
         tc_fence_after();
@@ -437,14 +441,11 @@ __global__ void __launch_bounds__(NTHREADS, D == 64 ? 2 : 1) fwd_tc_kernel(const
     float l_sum = 0.f;      // running sum of probabilities against m_ref
     int j = 0;
     for (int t = walk.next(0); ok && t >= 0; t = walk.next(t + 1), ++j) {
-      // every lane of the warp takes the same branch: the tcgen05.ld below is .sync.aligned
-      if (!__all_sync(0xffffffffu, mbar_wait(bar_sfull, j & 1, abort_flag))) { ok = false; break; }
+      const int sb = j % NSB;
+      const uint32_t tSb = tS + 128 * sb + lane_off;
+      // every lane of the warp takes the same branch: tcgen05.ld is .sync.aligned
+      if (!__all_sync(0xffffffffu, mbar_wait(bar_sfull(sb), (j / NSB) & 1, abort_flag))) { ok = false; break; }
       tc_fence_after();
-      float x[BN];
-#pragma unroll
-      for (int c = 0; c < BN / 32; ++c) tmem_ld32(tS + lane_off + c * 32, x + c * 32);
-      tc_fence_before();
-      mbar_arrive(bar_sfree);
 
       // the index rule on this tile, for row qi: window columns [lc_lo, lc_hi], skip columns bitmask
       int lc_lo, lc_hi;
@@ -453,44 +454,32 @@ __global__ void __launch_bounds__(NTHREADS, D == 64 ? 2 : 1) fwd_tc_kernel(const
         row_tile_mask(qi, (long long)t * BN, prm.S, 1, 0, 1, lc_lo, lc_hi, sk, m0);
       else
         row_tile_mask(qi, (long long)t * BN, prm.kwin, prm.pi, MODE == kFused ? prm.S : 0, m0, lc_lo, lc_hi, sk);
-      // per 32-column chunk, the cheapest exact treatment for this row (see chunk_class)
-      int cls[BN / 32];
-      int one_col[BN / 32];
-      float one_x[BN / 32];
+
+      // Pass 1 over the S row, one 32-column chunk at a time (a rolled loop: the body stays in the
+      // instruction cache): the tile max of the masked, scaled, biased logits.  A chunk of window
+      // keys only (kFull) needs the max of the raw scores, scaled afterwards (the scale is > 0 and
+      // the prior is constant); a chunk without keys (kEmpty) needs nothing.
       float mt = NEG_INF;
-#pragma unroll
+#pragma unroll 1
       for (int cb = 0; cb < BN / 32; ++cb) {
-        const int c0 = cb * 32;
-        const uint32_t skb = sk[cb];
-        cls[cb] = chunk_class(cb, lc_lo, lc_hi, skb);
-        one_col[cb] = 0;
-        one_x[cb] = NEG_INF;
-        if (cls[cb] == kFull) {
-          float mp[4] = {NEG_INF, NEG_INF, NEG_INF, NEG_INF};  // independent chains
+        float x[32];
+        tmem_ld32(tSb + cb * 32, x);
+        const uint32_t skb = cb == 0 ? sk[0] : cb == 1 ? sk[1] : cb == 2 ? sk[2] : sk[3];
+        const int cls = chunk_class(cb, lc_lo, lc_hi, skb);
+        if (cls == kFull) {
+          float mp[4] = {x[0], x[1], x[2], x[3]};
 #pragma unroll
-          for (int e = 0; e < 32; ++e) {
-            x[c0 + e] = fmaf(x[c0 + e], prm.scale_log2, bias_l);
-            mp[e & 3] = fmaxf(mp[e & 3], x[c0 + e]);
-          }
-          mt = fmaxf(mt, fmaxf(fmaxf(mp[0], mp[1]), fmaxf(mp[2], mp[3])));
-        } else if (cls[cb] == kOne) {
-          const int sc = __ffs(skb) - 1;
-          float xs = 0.f;
-#pragma unroll
-          for (int e = 0; e < 32; ++e) xs = e == sc ? x[c0 + e] : xs;
-          one_col[cb] = sc;
-          one_x[cb] = fmaf(xs, prm.scale_log2, bias_p);
-          mt = fmaxf(mt, one_x[cb]);
-        } else if (cls[cb] == kMixed) {
+          for (int e = 4; e < 32; ++e) mp[e & 3] = fmaxf(mp[e & 3], x[e]);
+          mt = fmaxf(mt, fmaf(fmaxf(fmaxf(mp[0], mp[1]), fmaxf(mp[2], mp[3])), prm.scale_log2, bias_l));
+        } else if (cls != kEmpty) {
           float mp[4] = {NEG_INF, NEG_INF, NEG_INF, NEG_INF};
 #pragma unroll
           for (int e = 0; e < 32; ++e) {
-            const int c = c0 + e;
+            const int c = cb * 32 + e;
             const bool loc = c >= lc_lo && c <= lc_hi;
             const bool skp = (skb >> e) & 1u;
             const float b = loc ? bias_l : (skp ? bias_p : NEG_INF);
-            x[c] = fmaf(x[c], prm.scale_log2, b);
-            mp[e & 3] = fmaxf(mp[e & 3], x[c]);
+            mp[e & 3] = fmaxf(mp[e & 3], fmaf(x[e], prm.scale_log2, b));
           }
           mt = fmaxf(mt, fmaxf(fmaxf(mp[0], mp[1]), fmaxf(mp[2], mp[3])));
         }
@@ -505,38 +494,8 @@ __global__ void __launch_bounds__(NTHREADS, D == 64 ? 2 : 1) fwd_tc_kernel(const
         m_ref = mt;
       }
       const float m_use = m_ref == NEG_INF ? 0.f : m_ref;
-      // probabilities, row sum, bf16 pairs
-      uint32_t pk[BN / 2];
-      float ls = 0.f;
-#pragma unroll
-      for (int cb = 0; cb < BN / 32; ++cb) {
-        const int c0 = cb * 32;
-        if (cls[cb] == kFull || cls[cb] == kMixed) {
-          float sp[4] = {0.f, 0.f, 0.f, 0.f};  // independent chains
-#pragma unroll
-          for (int e = 0; e < 32; e += 2) {
-            const float p0 = ex2(x[c0 + e] - m_use), p1 = ex2(x[c0 + e + 1] - m_use);
-            sp[(e >> 1) & 3] += p0 + p1;
-            __nv_bfloat162 b2 = __floats2bfloat162_rn(p0, p1);
-            pk[(c0 + e) / 2] = *reinterpret_cast<uint32_t*>(&b2);
-          }
-          ls += (sp[0] + sp[1]) + (sp[2] + sp[3]);
-        } else if (cls[cb] == kOne) {
-          const float p1 = ex2(one_x[cb] - m_use);
-          ls += p1;
-          __nv_bfloat162 b2 = __floats2bfloat162_rn(p1, p1);
-          const uint32_t both = *reinterpret_cast<uint32_t*>(&b2);
-          const uint32_t word = (one_col[cb] & 1) ? (both & 0xFFFF0000u) : (both & 0x0000FFFFu);
-#pragma unroll
-          for (int w = 0; w < 16; ++w) pk[c0 / 2 + w] = (one_col[cb] >> 1) == w ? word : 0u;
-        } else {
-#pragma unroll
-          for (int w = 0; w < 16; ++w) pk[c0 / 2 + w] = 0u;
-        }
-      }
-      l_sum += ls;
 
-      // P buffer and O are free once the previous P.V has completed
+      // The P buffer and O are free once the previous P.V has completed.
       if (j > 0) {
         if (!__all_sync(0xffffffffu, mbar_wait(bar_pvdone, (j - 1) & 1, abort_flag))) { ok = false; break; }
         tc_fence_after();
@@ -544,7 +503,7 @@ __global__ void __launch_bounds__(NTHREADS, D == 64 ? 2 : 1) fwd_tc_kernel(const
         // rows needs it, the others multiply by 1
         if (__any_sync(0xffffffffu, rescale)) {
           const float f = rescale ? factor : 1.f;
-#pragma unroll
+#pragma unroll 1
           for (int c = 0; c < D / 32; ++c) {
             float o[32];
             tmem_ld32(tO + lane_off + c * 32, o);
@@ -555,17 +514,66 @@ __global__ void __launch_bounds__(NTHREADS, D == 64 ? 2 : 1) fwd_tc_kernel(const
           tmem_wait_st();
         }
       }
-      // P row r -> shared memory, K-major with the 128-byte swizzle (16-byte chunk c ^ (r & 7))
+
+      // Pass 2: probabilities against the reference, the row sum, and P (bf16) into shared memory,
+      // K-major with the 128-byte swizzle (16-byte chunk cc of row r at chunk cc ^ (r & 7)).
+      const float bl_m = bias_l - m_use;
+      float ls = 0.f;
+#pragma unroll 1
+      for (int cb = 0; cb < BN / 32; ++cb) {
+        float x[32];
+        tmem_ld32(tSb + cb * 32, x);
+        const uint32_t skb = cb == 0 ? sk[0] : cb == 1 ? sk[1] : cb == 2 ? sk[2] : sk[3];
+        const int cls = chunk_class(cb, lc_lo, lc_hi, skb);
+        uint32_t pk[16];
+        if (cls == kEmpty) {
 #pragma unroll
-      for (int c = 0; c < BN / 8; ++c) {
-        const int blk = c >> 3, cc = c & 7;
-        uint4 u;
-        u.x = pk[c * 4 + 0];
-        u.y = pk[c * 4 + 1];
-        u.z = pk[c * 4 + 2];
-        u.w = pk[c * 4 + 3];
-        *reinterpret_cast<uint4*>(sbase + L::kP + blk * (BM * 128) + r * 128 + ((cc ^ (r & 7)) << 4)) = u;
+          for (int w = 0; w < 16; ++w) pk[w] = 0u;
+        } else {
+          float sp[4] = {0.f, 0.f, 0.f, 0.f};
+          if (cls == kFull) {
+#pragma unroll
+            for (int e = 0; e < 32; e += 2) {
+              const float p0 = ex2(fmaf(x[e], prm.scale_log2, bl_m));
+              const float p1 = ex2(fmaf(x[e + 1], prm.scale_log2, bl_m));
+              sp[(e >> 1) & 3] += p0 + p1;
+              __nv_bfloat162 b2 = __floats2bfloat162_rn(p0, p1);
+              pk[e >> 1] = *reinterpret_cast<uint32_t*>(&b2);
+            }
+          } else {
+#pragma unroll
+            for (int e = 0; e < 32; e += 2) {
+              float pp[2];
+#pragma unroll
+              for (int u = 0; u < 2; ++u) {
+                const int c = cb * 32 + e + u;
+                const bool loc = c >= lc_lo && c <= lc_hi;
+                const bool skp = (skb >> (e + u)) & 1u;
+                const float b = loc ? bias_l : (skp ? bias_p : NEG_INF);
+                pp[u] = ex2(fmaf(x[e + u], prm.scale_log2, b) - m_use);
+              }
+              sp[(e >> 1) & 3] += pp[0] + pp[1];
+              __nv_bfloat162 b2 = __floats2bfloat162_rn(pp[0], pp[1]);
+              pk[e >> 1] = *reinterpret_cast<uint32_t*>(&b2);
+            }
+          }
+          ls += (sp[0] + sp[1]) + (sp[2] + sp[3]);
+        }
+#pragma unroll
+        for (int g = 0; g < 4; ++g) {  // 16-byte chunks 4 cb + g of the row
+          const int c = cb * 4 + g;
+          const int blk = c >> 3, cc = c & 7;
+          uint4 u;
+          u.x = pk[g * 4 + 0];
+          u.y = pk[g * 4 + 1];
+          u.z = pk[g * 4 + 2];
+          u.w = pk[g * 4 + 3];
+          *reinterpret_cast<uint4*>(sbase + L::kP + blk * (BM * 128) + r * 128 + ((cc ^ (r & 7)) << 4)) = u;
+        }
       }
+      l_sum += ls;
+      tc_fence_before();
+      mbar_arrive(bar_sfree(sb));  // this S buffer may now take the Q.K^T of tile j + NSB
       fence_proxy_async_smem();
       tc_fence_before();
       mbar_arrive(bar_pfull);
@@ -592,7 +600,7 @@ __global__ void __launch_bounds__(NTHREADS, D == 64 ? 2 : 1) fwd_tc_kernel(const
         so = reinterpret_cast<const uint4*>(prm.skip_o + orow * D);
       }
       __nv_bfloat16* orow_ptr = (MODE == kResidue ? prm.skip_o : prm.out) + orow * D;
-#pragma unroll
+#pragma unroll 1
       for (int c = 0; c < D / 32; ++c) {
         float o[32];
         tmem_ld32(tO + lane_off + c * 32, o);
@@ -636,7 +644,7 @@ __global__ void __launch_bounds__(NTHREADS, D == 64 ? 2 : 1) fwd_tc_kernel(const
   __syncthreads();
   tc_fence_after();
   if (warp == 1) {
-    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, 256;" ::"r"(tmem) : "memory");
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "n"(L::kTmemCols) : "memory");
   }
 }
 

@@ -127,6 +127,27 @@ pi_attn_status pi_attn_fwd_ex(const void* q, const void* k, const void* v, const
   return launch_simt<__nv_bfloat16, false>(q, k, v, w_g, b_g, nullptr, out, lse, B, H, n, n, d, k_win, pi, S, s);
 }
 
+pi_attn_status pi_attn_fwd_plan(int B, int H, int n, int d, int k_win, int pi, int S, pi_attn_dtype dtype,
+                                pi_attn_path path, int* launches, long long* scratch_bytes) {
+  static const char dummy[16] __attribute__((aligned(16))) = {0};
+  if (!launches || !scratch_bytes) return fail(PI_ATTN_EINVAL, "null output pointer");
+  pi_attn_status st = check_common(dummy, dummy, dummy, (const float*)dummy, (const float*)dummy, dummy, B, H, n, d,
+                                   k_win, pi, S, dtype);
+  if (st != PI_ATTN_OK) return st;
+  if (path < PI_ATTN_PATH_AUTO || path > PI_ATTN_PATH_TC_SPLIT) return fail(PI_ATTN_EINVAL, "unknown path %d", (int)path);
+  const bool tc_ok = pia::tc_supported(dtype == PI_ATTN_BF16, d, n);
+  const bool want_tc = path == PI_ATTN_PATH_TC || path == PI_ATTN_PATH_TC_FUSED || path == PI_ATTN_PATH_TC_SPLIT;
+  if (want_tc && !tc_ok) return fail(PI_ATTN_EUNSUPPORTED, "tensor-core path does not cover this dtype / d");
+  if (path == PI_ATTN_PATH_TC_SPLIT && !pia::tc_split_applies(n, k_win, pi, S))
+    return fail(PI_ATTN_EUNSUPPORTED, "split path needs n %% pi == 0 and at least one skip outside the window");
+  bool split = false;
+  if (path != PI_ATTN_PATH_SIMT && tc_ok)
+    split = path == PI_ATTN_PATH_TC_SPLIT || (path != PI_ATTN_PATH_TC_FUSED && pia::tc_split_preferred(n, k_win, pi, S));
+  *launches = split ? 2 : 1;
+  *scratch_bytes = split ? (long long)B * H * n * (2LL * d + 4) : 0;
+  return ok();
+}
+
 pi_attn_status pi_attn_fwd(const void* q, const void* k, const void* v, const float* w_g, const float* b_g,
                            void* out, float* lse, int B, int H, int n, int d, int k_win, int pi, int S,
                            pi_attn_dtype dtype, void* stream) {

@@ -82,6 +82,15 @@ def test_decode_and_index_export_reject_bad_arguments(lib):
     assert lib.pi_attn_debug_index_sets(16, 4, 0, 2, FAKE, FAKE, 16, None) == pia.PI_ATTN_EINVAL
 
 
+def test_plan_reports_launches_and_scratch(lib):
+    assert pia.pi_attn_fwd_plan(1, 8, 4096, 64, 128, 64, 4, "bf16", "tc_fused") == (1, 0)
+    assert pia.pi_attn_fwd_plan(1, 8, 4096, 64, 128, 64, 4, "bf16", "tc_split") == (2, 8 * 4096 * (2 * 64 + 4))
+    assert pia.pi_attn_fwd_plan(1, 32, 131072, 128, 512, 1024, 16, "bf16", "auto")[0] == 2
+    assert pia.pi_attn_fwd_plan(1, 2, 256, 32, 8, 16, 2, "f32", "auto") == (1, 0)
+    with pytest.raises(pia.PiAttnError):
+        pia.pi_attn_fwd_plan(1, 8, 4000, 64, 128, 64, 4, "bf16", "tc_split")  # n % pi != 0
+
+
 def test_built_for_sm100a_only():
     cmd = pbuild.command("x.so")
     assert "arch=compute_100a,code=sm_100a" in cmd and "-lineinfo" in cmd

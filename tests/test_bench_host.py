@@ -38,14 +38,15 @@ def test_decode_work():
 
 
 def test_traffic_line_needs_the_current_source(tmp_path, monkeypatch):
-    sha = bench.source_hash()
+    files = bench.KERNEL_FILES["prefill"]
+    sha = bench.source_hash(files)
     prof = tmp_path / "profiles"
     prof.mkdir()
-    (prof / "x.md").write_text(f"bench-traffic: workload=bf16_n4k bytes_per_launch=123 source_sha={sha}\n"
-                               f"bench-traffic: workload=bf16_n32k bytes_per_launch=9 source_sha=stale\n")
+    (prof / "x.md").write_text(
+        f"bench-traffic: workload=bf16_n4k bytes_per_launch=123 files={','.join(files)} source_sha={sha}\n"
+        f"bench-traffic: workload=bf16_n32k bytes_per_launch=9 files={','.join(files)} source_sha=stale\n")
     real_root = bench.ROOT
     monkeypatch.setattr(bench, "ROOT", str(tmp_path))
-    os.symlink(os.path.join(real_root, "include"), tmp_path / "include")
     os.makedirs(tmp_path / "periodic_sparse_attention_b200")
     os.symlink(os.path.join(real_root, "periodic_sparse_attention_b200", "csrc"),
                tmp_path / "periodic_sparse_attention_b200" / "csrc")
