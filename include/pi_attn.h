@@ -97,6 +97,32 @@ pi_attn_status pi_attn_decode(const void* q, const void* kcache, const void* vca
                               const float* b_g, const int* cache_len, void* out, float* lse, int B, int H,
                               int n_cache, int d, int k_win, int pi, int S, pi_attn_dtype dtype, void* stream);
 
+/* pi_attn_decode for callers that cannot allocate device memory.  (The pages describe no such
+ * call: this is a property of the library, not of the method.)
+ *
+ * pi_attn_decode takes a small workspace from cudaMallocAsync on `stream` whenever it spreads one
+ * (b, h) over several CTAs, which it does when B*H is too small to fill the GPU.  Some callers
+ * cannot let a library allocate.  For example, a process whose device memory is reserved up front
+ * by its own allocator has no room, or no quota, for a library allocation.  A runtime with a fixed
+ * memory plan must know every byte in advance.  Such callers use this entry point: same
+ * arguments, same results, no allocation and no free.  The caller still passes every input and
+ * output.  The workspace is a fixed device array inside the library of 4 MiB (1,048,576 floats),
+ * which every GPU that loads the library holds until the process exits.
+ *   - Sizes: bf16 with d in {64, 128}.  A call whose split needs more than the 4 MiB
+ *     (B*H * splits * (d + 2) floats) returns PI_ATTN_EINVAL and enqueues nothing; with the
+ *     library's split rule this needs a B*H far above what splits at all.
+ *   - The first call on a device looks up the array's device address (cudaGetSymbolAddress), with
+ *     that device current.  Make that first call before any stream capture.
+ *   - Every call shares the one array, and it keeps the last call's contents; the kernels
+ *     overwrite every slot they read, so nothing needs clearing.  Two calls whose kernels overlap
+ *     on the GPU (different streams, no ordering between them) race on the array: order them on
+ *     one stream or with events.
+ *   - Errors as for pi_attn_decode. */
+pi_attn_status pi_attn_decode_noalloc(const void* q, const void* kcache, const void* vcache, const float* w_g,
+                                      const float* b_g, const int* cache_len, void* out, float* lse, int B, int H,
+                                      int n_cache, int d, int k_win, int pi, int S, pi_attn_dtype dtype,
+                                      void* stream);
+
 /* Index sets as the kernels see them, for exact comparison.  For query rows i = 0..n-1:
  *   counts [n, 2] int32: |L(i)|, |P(i)|
  *   idx    [n, width] int32: L(i) ascending, then P(i) in order of increasing m, then -1.

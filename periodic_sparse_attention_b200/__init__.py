@@ -31,6 +31,8 @@ SIGNATURES = {
     "pi_attn_fwd_plan": (_i32, [_i32] * 9 + [_vp, _vp]),
     # 8 pointers (q kcache vcache w_g b_g cache_len out lse), B H n_cache d k_win pi S, dtype, stream
     "pi_attn_decode": (_i32, [_vp] * 8 + [_i32] * 8 + [_vp]),
+    # as pi_attn_decode; no allocation (fixed 4 MiB device scratch inside the library)
+    "pi_attn_decode_noalloc": (_i32, [_vp] * 8 + [_i32] * 8 + [_vp]),
     "pi_attn_debug_index_sets": (_i32, [_i32, _i32, _i32, _i32, _vp, _vp, _i32, _vp]),
     "pi_attn_check": (_i32, [_vp]),
     "pi_attn_status_string": (_cstr, [_i32]),
@@ -138,6 +140,24 @@ def pi_attn_decode(q, kcache, vcache, w_g, b_g, k_win: int, pi: int, S: int, cac
         lse = torch.empty((B, H), dtype=torch.float32, device=q.device)
     st = load().pi_attn_decode(_ptr(q), _ptr(kcache), _ptr(vcache), _ptr(w_g), _ptr(b_g), _ptr(cache_len), _ptr(out),
                                _ptr(lse), B, H, n_cache, d, k_win, pi, S, _dtype_code(q), _stream(stream))
+    _raise(st)
+    return out, lse
+
+
+def pi_attn_decode_noalloc(q, kcache, vcache, w_g, b_g, k_win: int, pi: int, S: int, cache_len=None, out=None,
+                           lse=None, *, stream=None, want_lse: bool = True):
+    """pi_attn_decode without any device allocation inside the call (its workspace is a fixed
+    4 MiB array inside the library); out and lse are allocated here when not given."""
+    import torch
+    B, H, d = q.shape
+    n_cache = kcache.shape[2]
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None and want_lse:
+        lse = torch.empty((B, H), dtype=torch.float32, device=q.device)
+    st = load().pi_attn_decode_noalloc(_ptr(q), _ptr(kcache), _ptr(vcache), _ptr(w_g), _ptr(b_g), _ptr(cache_len),
+                                       _ptr(out), _ptr(lse), B, H, n_cache, d, k_win, pi, S, _dtype_code(q),
+                                       _stream(stream))
     _raise(st)
     return out, lse
 

@@ -60,6 +60,35 @@ pi_attn_status check_common(const void* q, const void* k, const void* v, const f
 
 cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s); }
 
+// ---- scratch that needs no allocation (pi_attn_decode_noalloc) ----------------------------------
+// A fixed device array, part of the library image: every GPU that loads the library holds it
+// until the process exits.  Host code must not pass its name to a kernel (on the host the name is
+// only a stand-in for the symbol); the device address comes from cudaGetSymbolAddress, once per
+// device, with that device current.
+constexpr size_t kNoAllocScratchFloats = (size_t)1 << 20;  // 4 MiB
+__device__ __align__(256) float g_noalloc_scratch[kNoAllocScratchFloats];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_noalloc_mu;
+float* g_noalloc_ptr[kMaxDevices] = {};
+
+// Device address of the scratch array on the current device (looked up on first use per device).
+cudaError_t noalloc_scratch(float** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (!g_noalloc_ptr[dev]) {
+    void* ptr = nullptr;
+    e = cudaGetSymbolAddress(&ptr, g_noalloc_scratch);
+    if (e != cudaSuccess) return e;
+    g_noalloc_ptr[dev] = static_cast<float*>(ptr);
+  }
+  *out = g_noalloc_ptr[dev];
+  return cudaSuccess;
+}
+
 int num_sms() {
   int dev = 0, sms = 148;
   if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
@@ -218,6 +247,69 @@ pi_attn_status pi_attn_decode(const void* q, const void* kcache, const void* vca
                                     S, s);
   return launch_simt<__nv_bfloat16, true>(q, kcache, vcache, w_g, b_g, cache_len, out, lse, B, H, 1, n_cache, d, k_win,
                                           pi, S, s);
+}
+
+pi_attn_status pi_attn_decode_noalloc(const void* q, const void* kcache, const void* vcache, const float* w_g,
+                                      const float* b_g, const int* cache_len, void* out, float* lse, int B, int H,
+                                      int n_cache, int d, int k_win, int pi, int S, pi_attn_dtype dtype,
+                                      void* stream) {
+  pi_attn_status st = check_common(q, kcache, vcache, w_g, b_g, out, B, H, n_cache, d, k_win, pi, S, dtype);
+  if (st != PI_ATTN_OK) return st;
+  if (dtype != PI_ATTN_BF16 || (d != 64 && d != 128))
+    return fail(PI_ATTN_EUNSUPPORTED, "pi_attn_decode_noalloc covers bf16 with d in {64, 128} (got dtype %d, d %d)",
+                (int)dtype, d);
+  const long long bh = (long long)B * H;
+  if (bh > 0x7fffffffLL) return fail(PI_ATTN_EINVAL, "B * H too large");
+  // same split rule as pi_attn_decode
+  const long long rows = (long long)k_win + 1 + S;
+  const long long slots = 14LL * num_sms();
+  int nsplit = 1;
+  if (bh * 2 < slots) {
+    long long ns = (slots + bh - 1) / bh;
+    const long long max_ns = (rows + 127) / 128;
+    if (ns > max_ns) ns = max_ns;
+    if (ns > 64) ns = 64;
+    nsplit = ns < 1 ? 1 : (int)ns;
+  }
+  const size_t need = (size_t)bh * nsplit * (d + 2);
+  if (nsplit > 1 && need > kNoAllocScratchFloats)
+    return fail(PI_ATTN_EINVAL,
+                "pi_attn_decode_noalloc: %lld (b, h) x %d splits need %zu bytes of scratch, above its fixed %zu",
+                bh, nsplit, need * sizeof(float), kNoAllocScratchFloats * sizeof(float));
+  cudaStream_t s = as_stream(stream);
+  pia::DecodeArgs a;
+  a.q = (const __nv_bfloat16*)q;
+  a.kc = (const __nv_bfloat16*)kcache;
+  a.vc = (const __nv_bfloat16*)vcache;
+  a.w_g = w_g;
+  a.b_g = b_g;
+  a.cache_len = cache_len;
+  a.out = (__nv_bfloat16*)out;
+  a.lse = lse;
+  a.part = nullptr;
+  a.H = H;
+  a.n_cache = n_cache;
+  a.kwin = k_win;
+  a.pi = pi;
+  a.S = S;
+  a.nsplit = nsplit;
+  a.scale_log2 = (float)(1.0 / std::sqrt((double)d)) * pia::kLog2e;
+  if (nsplit > 1) {
+    cudaError_t e = noalloc_scratch(&a.part);  // every split writes its whole slot: nothing to clear
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(decode scratch)");
+  }
+  dim3 grid((unsigned)bh, (unsigned)nsplit);
+  if (d == 128) pia::decode_bf16_kernel<128><<<grid, 64, 0, s>>>(a);
+  else pia::decode_bf16_kernel<64><<<grid, 64, 0, s>>>(a);
+  cudaError_t e = cudaGetLastError();
+  if (e == cudaSuccess && nsplit > 1) {
+    if (d == 128)
+      pia::decode_combine_kernel<128><<<(unsigned)bh, 128, 0, s>>>(a.part, nsplit, cache_len, H, n_cache, a.out, lse);
+    else
+      pia::decode_combine_kernel<64><<<(unsigned)bh, 64, 0, s>>>(a.part, nsplit, cache_len, H, n_cache, a.out, lse);
+    e = cudaGetLastError();
+  }
+  return e == cudaSuccess ? ok() : cuda_fail(e, "decode kernel launch");
 }
 
 pi_attn_status pi_attn_debug_index_sets(int n, int k_win, int pi, int S, int* counts, int* idx, int width,
