@@ -49,9 +49,9 @@ struct Smem {
   static constexpr int kV = kK + NSTAGE * kTileBytes;
   static constexpr int kP = kV + NSTAGE * kTileBytes;
   static constexpr int kBar = kP + BM * BN * 2;          // P: 128 x 128 bf16
-  // S buffers in TMEM: two for d = 128 (one CTA per SM: the next tile's Q.K^T overlaps this
-  // tile's softmax), one for d = 64 (two CTAs per SM overlap each other instead)
-  static constexpr int kSBufs = D == 128 ? 2 : 1;
+  // S buffers in TMEM: one suffices, the softmax reads a tile's S row with a single load and
+  // releases the buffer at once, so the next tile's Q.K^T overlaps the rest of the softmax
+  static constexpr int kSBufs = 1;
   static constexpr int kTmemCols = kSBufs == 2 ? 512 : 256;  // S buffers (128 each) + O (D)
   // barriers: q_full, k_full[2], k_empty[2], v_full[2], v_empty[2], s_full[NSB], s_free[NSB],
   // p_full, pv_done, drain
@@ -157,6 +157,28 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float* v) {
       : "memory");
 #pragma unroll
   for (int t = 0; t < 32; ++t) v[t] = __uint_as_float(r[t]);
+}
+__device__ __forceinline__ void tmem_ld64(uint32_t taddr, float* v) {
+  uint32_t r[64];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x64.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32, %33, %34, %35, %36, %37, %38, %39, %40, %41, %42, %43, %44, %45, %46, %47, %48, %49, %50, %51, %52, %53, %54, %55, %56, %57, %58, %59, %60, %61, %62, %63}, [%64];\n\t"
+      "tcgen05.wait::ld.sync.aligned;"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31]), "=r"(r[32]), "=r"(r[33]), "=r"(r[34]), "=r"(r[35]), "=r"(r[36]), "=r"(r[37]), "=r"(r[38]), "=r"(r[39]), "=r"(r[40]), "=r"(r[41]), "=r"(r[42]), "=r"(r[43]), "=r"(r[44]), "=r"(r[45]), "=r"(r[46]), "=r"(r[47]), "=r"(r[48]), "=r"(r[49]), "=r"(r[50]), "=r"(r[51]), "=r"(r[52]), "=r"(r[53]), "=r"(r[54]), "=r"(r[55]), "=r"(r[56]), "=r"(r[57]), "=r"(r[58]), "=r"(r[59]), "=r"(r[60]), "=r"(r[61]), "=r"(r[62]), "=r"(r[63])
+      : "r"(taddr)
+      : "memory");
+#pragma unroll
+  for (int t = 0; t < 64; ++t) v[t] = __uint_as_float(r[t]);
+}
+__device__ __forceinline__ void tmem_ld128(uint32_t taddr, float* v) {
+  uint32_t r[128];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x128.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32, %33, %34, %35, %36, %37, %38, %39, %40, %41, %42, %43, %44, %45, %46, %47, %48, %49, %50, %51, %52, %53, %54, %55, %56, %57, %58, %59, %60, %61, %62, %63, %64, %65, %66, %67, %68, %69, %70, %71, %72, %73, %74, %75, %76, %77, %78, %79, %80, %81, %82, %83, %84, %85, %86, %87, %88, %89, %90, %91, %92, %93, %94, %95, %96, %97, %98, %99, %100, %101, %102, %103, %104, %105, %106, %107, %108, %109, %110, %111, %112, %113, %114, %115, %116, %117, %118, %119, %120, %121, %122, %123, %124, %125, %126, %127}, [%128];\n\t"
+      "tcgen05.wait::ld.sync.aligned;"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31]), "=r"(r[32]), "=r"(r[33]), "=r"(r[34]), "=r"(r[35]), "=r"(r[36]), "=r"(r[37]), "=r"(r[38]), "=r"(r[39]), "=r"(r[40]), "=r"(r[41]), "=r"(r[42]), "=r"(r[43]), "=r"(r[44]), "=r"(r[45]), "=r"(r[46]), "=r"(r[47]), "=r"(r[48]), "=r"(r[49]), "=r"(r[50]), "=r"(r[51]), "=r"(r[52]), "=r"(r[53]), "=r"(r[54]), "=r"(r[55]), "=r"(r[56]), "=r"(r[57]), "=r"(r[58]), "=r"(r[59]), "=r"(r[60]), "=r"(r[61]), "=r"(r[62]), "=r"(r[63]), "=r"(r[64]), "=r"(r[65]), "=r"(r[66]), "=r"(r[67]), "=r"(r[68]), "=r"(r[69]), "=r"(r[70]), "=r"(r[71]), "=r"(r[72]), "=r"(r[73]), "=r"(r[74]), "=r"(r[75]), "=r"(r[76]), "=r"(r[77]), "=r"(r[78]), "=r"(r[79]), "=r"(r[80]), "=r"(r[81]), "=r"(r[82]), "=r"(r[83]), "=r"(r[84]), "=r"(r[85]), "=r"(r[86]), "=r"(r[87]), "=r"(r[88]), "=r"(r[89]), "=r"(r[90]), "=r"(r[91]), "=r"(r[92]), "=r"(r[93]), "=r"(r[94]), "=r"(r[95]), "=r"(r[96]), "=r"(r[97]), "=r"(r[98]), "=r"(r[99]), "=r"(r[100]), "=r"(r[101]), "=r"(r[102]), "=r"(r[103]), "=r"(r[104]), "=r"(r[105]), "=r"(r[106]), "=r"(r[107]), "=r"(r[108]), "=r"(r[109]), "=r"(r[110]), "=r"(r[111]), "=r"(r[112]), "=r"(r[113]), "=r"(r[114]), "=r"(r[115]), "=r"(r[116]), "=r"(r[117]), "=r"(r[118]), "=r"(r[119]), "=r"(r[120]), "=r"(r[121]), "=r"(r[122]), "=r"(r[123]), "=r"(r[124]), "=r"(r[125]), "=r"(r[126]), "=r"(r[127])
+      : "r"(taddr)
+      : "memory");
+#pragma unroll
+  for (int t = 0; t < 128; ++t) v[t] = __uint_as_float(r[t]);
 }
 __device__ __forceinline__ void tmem_st32(uint32_t taddr, const float* v) {
   asm volatile(
@@ -416,11 +438,16 @@ __global__ void __launch_bounds__(NTHREADS, D == 64 ? 2 : 1) fwd_tc_kernel(const
     const long long i = MODE == kResidue ? qi * prm.pi + res : qi;  // row in the sequence
     const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
 
-    // gate on the unscaled query row (read from the swizzled Q tile)
+    // gate on the unscaled query row.  w_g[h] is staged in shared memory with vector loads while
+    // the Q tile is still in flight; the staging area is the start of the P buffer, which is
+    // not written before both named barriers below have passed.
+    float* const wg_s = reinterpret_cast<float*>(sbase + L::kP);
+    if (threadIdx.x - 64 < D) wg_s[threadIdx.x - 64] = prm.w_g[(long long)h * D + (threadIdx.x - 64)];
+    asm volatile("bar.sync 1, 128;" ::: "memory");
     bool ok = __all_sync(0xffffffffu, mbar_wait(bar_q, 0, abort_flag));
     float z = prm.b_g[h];
     {
-      const float* wg = prm.w_g + (long long)h * D;
+      float zp[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
       for (int c = 0; c < D / 8; ++c) {
         const int blk = c >> 3, cc = c & 7;
@@ -428,10 +455,24 @@ __global__ void __launch_bounds__(NTHREADS, D == 64 ? 2 : 1) fwd_tc_kernel(const
                                                         ((cc ^ (r & 7)) << 4));
         float f[8];
         bf16x8_to_f32(u, f);
-#pragma unroll
-        for (int e = 0; e < 8; ++e) z = fmaf(f[e], wg[c * 8 + e], z);
+        const float4 w0 = reinterpret_cast<const float4*>(wg_s)[2 * c];
+        const float4 w1 = reinterpret_cast<const float4*>(wg_s)[2 * c + 1];
+        zp[0] = fmaf(f[0], w0.x, zp[0]);
+        zp[1] = fmaf(f[1], w0.y, zp[1]);
+        zp[2] = fmaf(f[2], w0.z, zp[2]);
+        zp[3] = fmaf(f[3], w0.w, zp[3]);
+        zp[0] = fmaf(f[4], w1.x, zp[0]);
+        zp[1] = fmaf(f[5], w1.y, zp[1]);
+        zp[2] = fmaf(f[6], w1.z, zp[2]);
+        zp[3] = fmaf(f[7], w1.w, zp[3]);
       }
+      z += (zp[0] + zp[1]) + (zp[2] + zp[3]);
     }
+    asm volatile("bar.sync 1, 128;" ::: "memory");  // every thread has read w_g: P may be written
+    // Beyond |z| = 40 the gate is saturated: the prior it would lower further already weighs
+    // e^-40 or less against the other one.  Clamping keeps the two priors within 40 nats of each
+    // other, which the softmax's max bound below relies on; the results change by < e^-40.
+    z = fminf(fmaxf(z, -40.f), 40.f);
     // the prior of the keys this pass unmasks as "window" columns
     const float bias_l = log_sigmoid(MODE == kResidue ? -z : z) * kLog2e;  // log2(alpha), or log2(1-alpha)
     const float bias_p = log_sigmoid(-z) * kLog2e;                         // log2(1 - alpha)
@@ -442,10 +483,20 @@ __global__ void __launch_bounds__(NTHREADS, D == 64 ? 2 : 1) fwd_tc_kernel(const
     int j = 0;
     for (int t = walk.next(0); ok && t >= 0; t = walk.next(t + 1), ++j) {
       const int sb = j % NSB;
-      const uint32_t tSb = tS + 128 * sb + lane_off;
       // every lane of the warp takes the same branch: tcgen05.ld is .sync.aligned
       if (!__all_sync(0xffffffffu, mbar_wait(bar_sfull(sb), (j / NSB) & 1, abort_flag))) { ok = false; break; }
       tc_fence_after();
+      // d = 128 (one CTA per SM): the whole S row stays in registers and the buffer is released at
+      // once, so the next Q.K^T overlaps this softmax.  d = 64 (two CTAs per SM, 168 registers):
+      // the row is read once for the max and again, in two halves, for the probabilities; the
+      // buffer is released after that, and the SM's other CTA fills the gap.
+      constexpr bool kRowInRegs = D == 128;
+      float x[BN];
+      tmem_ld128(tS + 128 * sb + lane_off, x);  // the whole S row, one load and one wait
+      if (kRowInRegs) {
+        tc_fence_before();
+        mbar_arrive(bar_sfree(sb));
+      }
 
       // the index rule on this tile, for row qi: window columns [lc_lo, lc_hi], skip columns bitmask
       int lc_lo, lc_hi;
@@ -454,36 +505,23 @@ __global__ void __launch_bounds__(NTHREADS, D == 64 ? 2 : 1) fwd_tc_kernel(const
         row_tile_mask(qi, (long long)t * BN, prm.S, 1, 0, 1, lc_lo, lc_hi, sk, m0);
       else
         row_tile_mask(qi, (long long)t * BN, prm.kwin, prm.pi, MODE == kFused ? prm.S : 0, m0, lc_lo, lc_hi, sk);
+      const bool has_win = lc_lo <= lc_hi;
+      const bool has_skip = (sk[0] | sk[1] | sk[2] | sk[3]) != 0u;
 
-      // Pass 1 over the S row, one 32-column chunk at a time (a rolled loop: the body stays in the
-      // instruction cache): the tile max of the masked, scaled, biased logits.  A chunk of window
-      // keys only (kFull) needs the max of the raw scores, scaled afterwards (the scale is > 0 and
-      // the prior is constant); a chunk without keys (kEmpty) needs nothing.
-      float mt = NEG_INF;
-#pragma unroll 1
-      for (int cb = 0; cb < BN / 32; ++cb) {
-        float x[32];
-        tmem_ld32(tSb + cb * 32, x);
-        const uint32_t skb = cb == 0 ? sk[0] : cb == 1 ? sk[1] : cb == 2 ? sk[2] : sk[3];
-        const int cls = chunk_class(cb, lc_lo, lc_hi, skb);
-        if (cls == kFull) {
-          float mp[4] = {x[0], x[1], x[2], x[3]};
+      // An upper bound of the tile max of the biased logits: the max of the raw scores of the row,
+      // scaled, plus the larger prior present in the tile.  Probabilities only need a reference
+      // at or above the true max (they stay <= 1 against it; the final division uses the same
+      // reference), so the mask is not needed here.  The bound exceeds the true max by at most the
+      // spread of the scores plus the prior gap (<= 40 nats after the clamp above).
+      float mx[8];
 #pragma unroll
-          for (int e = 4; e < 32; ++e) mp[e & 3] = fmaxf(mp[e & 3], x[e]);
-          mt = fmaxf(mt, fmaf(fmaxf(fmaxf(mp[0], mp[1]), fmaxf(mp[2], mp[3])), prm.scale_log2, bias_l));
-        } else if (cls != kEmpty) {
-          float mp[4] = {NEG_INF, NEG_INF, NEG_INF, NEG_INF};
+      for (int e = 0; e < 8; ++e) mx[e] = x[e];
 #pragma unroll
-          for (int e = 0; e < 32; ++e) {
-            const int c = cb * 32 + e;
-            const bool loc = c >= lc_lo && c <= lc_hi;
-            const bool skp = (skb >> e) & 1u;
-            const float b = loc ? bias_l : (skp ? bias_p : NEG_INF);
-            mp[e & 3] = fmaxf(mp[e & 3], fmaf(x[e], prm.scale_log2, b));
-          }
-          mt = fmaxf(mt, fmaxf(fmaxf(mp[0], mp[1]), fmaxf(mp[2], mp[3])));
-        }
-      }
+      for (int c = 8; c < BN; ++c) mx[c & 7] = fmaxf(mx[c & 7], x[c]);
+      const float mraw = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])), fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
+      const float top = has_win ? (has_skip ? fmaxf(bias_l, bias_p) : bias_l) : bias_p;
+      const float mt = (has_win || has_skip) ? fmaf(mraw, prm.scale_log2, top) : NEG_INF;
+
       // lazy reference max
       float factor = 1.f;
       bool rescale = false;
@@ -515,27 +553,34 @@ __global__ void __launch_bounds__(NTHREADS, D == 64 ? 2 : 1) fwd_tc_kernel(const
         }
       }
 
-      // Pass 2: probabilities against the reference, the row sum, and P (bf16) into shared memory,
+      // Probabilities against the reference, the row sum, and P (bf16) into shared memory,
       // K-major with the 128-byte swizzle (16-byte chunk cc of row r at chunk cc ^ (r & 7)).
-      const float bl_m = bias_l - m_use;
+      // Per 32-column chunk: no key -> zeros; window keys only -> one FMA per logit; otherwise
+      // the window bits and skip bits select each logit's prior (-inf: p = 0).
+      const float bl_m = bias_l - m_use, bp_m = bias_p - m_use;
       float ls = 0.f;
-#pragma unroll 1
+#pragma unroll
       for (int cb = 0; cb < BN / 32; ++cb) {
-        float x[32];
-        tmem_ld32(tSb + cb * 32, x);
-        const uint32_t skb = cb == 0 ? sk[0] : cb == 1 ? sk[1] : cb == 2 ? sk[2] : sk[3];
-        const int cls = chunk_class(cb, lc_lo, lc_hi, skb);
+        const int c0 = cb * 32;
+        if (!kRowInRegs && (cb & 1) == 0) tmem_ld64(tS + 128 * sb + lane_off + c0, x + c0);  // re-read half
+        const uint32_t skb = sk[cb];
+        const int lo = lc_lo - c0, hi = lc_hi - c0;  // window columns of this chunk: [lo, hi] within 0..31
+        uint32_t wm = 0u;
+        if (lo <= 31 && hi >= 0 && lo <= hi) {
+          const int a = lo < 0 ? 0 : lo, b = hi > 31 ? 31 : hi;
+          wm = (b == 31 ? 0xFFFFFFFFu : ((1u << (b + 1)) - 1u)) & ~((1u << a) - 1u);
+        }
         uint32_t pk[16];
-        if (cls == kEmpty) {
+        if ((wm | skb) == 0u) {
 #pragma unroll
           for (int w = 0; w < 16; ++w) pk[w] = 0u;
         } else {
           float sp[4] = {0.f, 0.f, 0.f, 0.f};
-          if (cls == kFull) {
+          if (wm == 0xFFFFFFFFu && skb == 0u) {
 #pragma unroll
             for (int e = 0; e < 32; e += 2) {
-              const float p0 = ex2(fmaf(x[e], prm.scale_log2, bl_m));
-              const float p1 = ex2(fmaf(x[e + 1], prm.scale_log2, bl_m));
+              const float p0 = ex2(fmaf(x[c0 + e], prm.scale_log2, bl_m));
+              const float p1 = ex2(fmaf(x[c0 + e + 1], prm.scale_log2, bl_m));
               sp[(e >> 1) & 3] += p0 + p1;
               __nv_bfloat162 b2 = __floats2bfloat162_rn(p0, p1);
               pk[e >> 1] = *reinterpret_cast<uint32_t*>(&b2);
@@ -543,17 +588,12 @@ __global__ void __launch_bounds__(NTHREADS, D == 64 ? 2 : 1) fwd_tc_kernel(const
           } else {
 #pragma unroll
             for (int e = 0; e < 32; e += 2) {
-              float pp[2];
-#pragma unroll
-              for (int u = 0; u < 2; ++u) {
-                const int c = cb * 32 + e + u;
-                const bool loc = c >= lc_lo && c <= lc_hi;
-                const bool skp = (skb >> (e + u)) & 1u;
-                const float b = loc ? bias_l : (skp ? bias_p : NEG_INF);
-                pp[u] = ex2(fmaf(x[e + u], prm.scale_log2, b) - m_use);
-              }
-              sp[(e >> 1) & 3] += pp[0] + pp[1];
-              __nv_bfloat162 b2 = __floats2bfloat162_rn(pp[0], pp[1]);
+              const float b0 = (wm >> e) & 1u ? bl_m : ((skb >> e) & 1u ? bp_m : NEG_INF);
+              const float b1 = (wm >> (e + 1)) & 1u ? bl_m : ((skb >> (e + 1)) & 1u ? bp_m : NEG_INF);
+              const float p0 = ex2(fmaf(x[c0 + e], prm.scale_log2, b0));
+              const float p1 = ex2(fmaf(x[c0 + e + 1], prm.scale_log2, b1));
+              sp[(e >> 1) & 3] += p0 + p1;
+              __nv_bfloat162 b2 = __floats2bfloat162_rn(p0, p1);
               pk[e >> 1] = *reinterpret_cast<uint32_t*>(&b2);
             }
           }
@@ -572,8 +612,10 @@ __global__ void __launch_bounds__(NTHREADS, D == 64 ? 2 : 1) fwd_tc_kernel(const
         }
       }
       l_sum += ls;
-      tc_fence_before();
-      mbar_arrive(bar_sfree(sb));  // this S buffer may now take the Q.K^T of tile j + NSB
+      if (!kRowInRegs) {
+        tc_fence_before();
+        mbar_arrive(bar_sfree(sb));
+      }
       fence_proxy_async_smem();
       tc_fence_before();
       mbar_arrive(bar_pfull);
@@ -600,10 +642,11 @@ __global__ void __launch_bounds__(NTHREADS, D == 64 ? 2 : 1) fwd_tc_kernel(const
         so = reinterpret_cast<const uint4*>(prm.skip_o + orow * D);
       }
       __nv_bfloat16* orow_ptr = (MODE == kResidue ? prm.skip_o : prm.out) + orow * D;
-#pragma unroll 1
+      float o[D];  // the whole O row, one load and one wait
+      if (D == 128) tmem_ld128(tO + lane_off, o);
+      else tmem_ld64(tO + lane_off, o);
+#pragma unroll
       for (int c = 0; c < D / 32; ++c) {
-        float o[32];
-        tmem_ld32(tO + lane_off + c * 32, o);
         if (row_ok) {
 #pragma unroll
           for (int g = 0; g < 4; ++g) {
@@ -612,8 +655,8 @@ __global__ void __launch_bounds__(NTHREADS, D == 64 ? 2 : 1) fwd_tc_kernel(const
             uint32_t w[4];
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
-              const float a0 = o[g * 8 + 2 * e] * inv * wl + sp[2 * e] * wp;
-              const float a1 = o[g * 8 + 2 * e + 1] * inv * wl + sp[2 * e + 1] * wp;
+              const float a0 = o[c * 32 + g * 8 + 2 * e] * inv * wl + sp[2 * e] * wp;
+              const float a1 = o[c * 32 + g * 8 + 2 * e + 1] * inv * wl + sp[2 * e + 1] * wp;
               __nv_bfloat162 b2 = __floats2bfloat162_rn(a0, a1);
               w[e] = *reinterpret_cast<uint32_t*>(&b2);
             }
