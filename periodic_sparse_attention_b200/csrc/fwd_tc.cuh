@@ -55,7 +55,7 @@ struct Smem {
   static constexpr int kTmemCols = kSBufs == 2 ? 512 : 256;  // S buffers (128 each) + O (D)
   // barriers: q_full, k_full[2], k_empty[2], v_full[2], v_empty[2], s_full[NSB], s_free[NSB],
   // p_full, pv_done, drain
-  static constexpr int kNumBars = 1 + 4 * NSTAGE + 2 * kSBufs + 3;
+  static constexpr int kNumBars = 1 + 4 * NSTAGE + 2 * kSBufs + 4;
   static constexpr int kMisc = kBar + kNumBars * 8;      // tmem base (4 B), abort flag (4 B)
   static constexpr int kTotal = kMisc + 16;
   static constexpr int kAlloc = kTotal + 1024 - 128;     // slack to align a (>= 128 B aligned) base to 1 KB
@@ -121,6 +121,22 @@ __device__ __forceinline__ void tma_load_4d(uint32_t dst, const CUtensorMap* map
       "%6}], [%2];" ::"r"(dst),
       "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(c0), "r"(c1), "r"(c2), "r"(c3)
       : "memory");
+}
+__device__ __forceinline__ void tma_store_3d(const CUtensorMap* map, uint32_t src, int c0, int c1, int c2) {
+  asm volatile("cp.async.bulk.tensor.3d.global.shared::cta.tile.bulk_group [%0, {%2, %3, %4}], [%1];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(src), "r"(c0), "r"(c1), "r"(c2)
+               : "memory");
+}
+__device__ __forceinline__ void tma_store_4d(const CUtensorMap* map, uint32_t src, int c0, int c1, int c2, int c3) {
+  asm volatile("cp.async.bulk.tensor.4d.global.shared::cta.tile.bulk_group [%0, {%2, %3, %4, %5}], [%1];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(src), "r"(c0), "r"(c1), "r"(c2), "r"(c3)
+               : "memory");
+}
+__device__ __forceinline__ void tma_store_commit_and_wait_read() {
+  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
 }
 __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -199,6 +215,14 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const float* v) {
 }
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
+// v[k] for a run-time k in 0..31 from a register array, by selects (no local memory).
+__device__ __forceinline__ float pick32(const float* v, int k) {
+  float r = v[0];
+#pragma unroll
+  for (int e = 1; e < 32; ++e) r = k == e ? v[e] : r;
+  return r;
+}
+
 __device__ __forceinline__ float ex2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
@@ -250,6 +274,8 @@ template <int D, int MODE>
 __global__ void __launch_bounds__(NTHREADS, D == 64 ? 2 : 1) fwd_tc_kernel(const __grid_constant__ CUtensorMap tmq,
                                                                           const __grid_constant__ CUtensorMap tmk,
                                                                           const __grid_constant__ CUtensorMap tmv,
+                                                                          const __grid_constant__ CUtensorMap tmo,
+                                                                          const __grid_constant__ CUtensorMap tms,
                                                                           Params prm) {
   using L = Smem<D>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -298,6 +324,7 @@ __global__ void __launch_bounds__(NTHREADS, D == 64 ? 2 : 1) fwd_tc_kernel(const
   const uint32_t bar_pfull = bar0 + 8u * (1 + 4 * NSTAGE + 2 * NSB);
   const uint32_t bar_pvdone = bar_pfull + 8;
   const uint32_t bar_drain = bar_pfull + 16;
+  const uint32_t bar_so = bar_pfull + 24;  // kBandMerge: the tile of skip partials has landed
   uint32_t* const tmem_slot = reinterpret_cast<uint32_t*>(sbase + L::kMisc);
   volatile int* const abort_flag = reinterpret_cast<volatile int*>(sbase + L::kMisc + 4);
 
@@ -316,6 +343,7 @@ __global__ void __launch_bounds__(NTHREADS, D == 64 ? 2 : 1) fwd_tc_kernel(const
     mbar_init(bar_pfull, BM);
     mbar_init(bar_pvdone, 1);
     mbar_init(bar_drain, 1);
+    mbar_init(bar_so, 1);
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -469,10 +497,6 @@ __global__ void __launch_bounds__(NTHREADS, D == 64 ? 2 : 1) fwd_tc_kernel(const
       z += (zp[0] + zp[1]) + (zp[2] + zp[3]);
     }
     asm volatile("bar.sync 1, 128;" ::: "memory");  // every thread has read w_g: P may be written
-    // Beyond |z| = 40 the gate is saturated: the prior it would lower further already weighs
-    // e^-40 or less against the other one.  Clamping keeps the two priors within 40 nats of each
-    // other, which the softmax's max bound below relies on; the results change by < e^-40.
-    z = fminf(fmaxf(z, -40.f), 40.f);
     // the prior of the keys this pass unmasks as "window" columns
     const float bias_l = log_sigmoid(MODE == kResidue ? -z : z) * kLog2e;  // log2(alpha), or log2(1-alpha)
     const float bias_p = log_sigmoid(-z) * kLog2e;                         // log2(1 - alpha)
@@ -505,22 +529,34 @@ __global__ void __launch_bounds__(NTHREADS, D == 64 ? 2 : 1) fwd_tc_kernel(const
         row_tile_mask(qi, (long long)t * BN, prm.S, 1, 0, 1, lc_lo, lc_hi, sk, m0);
       else
         row_tile_mask(qi, (long long)t * BN, prm.kwin, prm.pi, MODE == kFused ? prm.S : 0, m0, lc_lo, lc_hi, sk);
-      const bool has_win = lc_lo <= lc_hi;
-      const bool has_skip = (sk[0] | sk[1] | sk[2] | sk[3]) != 0u;
 
-      // An upper bound of the tile max of the biased logits: the max of the raw scores of the row,
-      // scaled, plus the larger prior present in the tile.  Probabilities only need a reference
-      // at or above the true max (they stay <= 1 against it; the final division uses the same
-      // reference), so the mask is not needed here.  The bound exceeds the true max by at most the
-      // spread of the scores plus the prior gap (<= 40 nats after the clamp above).
-      float mx[8];
+      // The tile max of the biased logits, exactly: per 32-column chunk, window-only chunks take
+      // the max of their raw scores, chunks without keys are skipped, and chunks that straddle the
+      // window edge or hold skip keys mask each column (window bits wm, skip bits skb).  The max of
+      // a kind of key is then scaled and given its prior.  (An exact reference keeps the largest
+      // probability of a row at 1, which bf16 holds exactly.)
+      float mw = NEG_INF, ms = NEG_INF;
 #pragma unroll
-      for (int e = 0; e < 8; ++e) mx[e] = x[e];
+      for (int cb = 0; cb < BN / 32; ++cb) {
+        const int c0 = cb * 32;
+        const uint32_t wm = window_bits(lc_lo - c0, lc_hi - c0), skb = sk[cb];
+        if (wm == 0xFFFFFFFFu && skb == 0u) {
+          float m4[4] = {x[c0], x[c0 + 1], x[c0 + 2], x[c0 + 3]};
 #pragma unroll
-      for (int c = 8; c < BN; ++c) mx[c & 7] = fmaxf(mx[c & 7], x[c]);
-      const float mraw = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])), fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
-      const float top = has_win ? (has_skip ? fmaxf(bias_l, bias_p) : bias_l) : bias_p;
-      const float mt = (has_win || has_skip) ? fmaf(mraw, prm.scale_log2, top) : NEG_INF;
+          for (int e = 4; e < 32; ++e) m4[e & 3] = fmaxf(m4[e & 3], x[c0 + e]);
+          mw = fmaxf(mw, fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3])));
+        } else if (wm == 0u && skb != 0u && (skb & (skb - 1u)) == 0u) {
+          ms = fmaxf(ms, pick32(x + c0, __ffs(skb) - 1));  // a single skip key
+        } else if ((wm | skb) != 0u) {
+#pragma unroll
+          for (int e = 0; e < 32; ++e) {
+            mw = fmaxf(mw, (wm >> e) & 1u ? x[c0 + e] : NEG_INF);
+            ms = fmaxf(ms, (skb >> e) & 1u ? x[c0 + e] : NEG_INF);
+          }
+        }
+      }
+      const float mt = fmaxf(mw == NEG_INF ? NEG_INF : fmaf(mw, prm.scale_log2, bias_l),
+                             ms == NEG_INF ? NEG_INF : fmaf(ms, prm.scale_log2, bias_p));
 
       // lazy reference max
       float factor = 1.f;
@@ -564,16 +600,21 @@ __global__ void __launch_bounds__(NTHREADS, D == 64 ? 2 : 1) fwd_tc_kernel(const
         const int c0 = cb * 32;
         if (!kRowInRegs && (cb & 1) == 0) tmem_ld64(tS + 128 * sb + lane_off + c0, x + c0);  // re-read half
         const uint32_t skb = sk[cb];
-        const int lo = lc_lo - c0, hi = lc_hi - c0;  // window columns of this chunk: [lo, hi] within 0..31
-        uint32_t wm = 0u;
-        if (lo <= 31 && hi >= 0 && lo <= hi) {
-          const int a = lo < 0 ? 0 : lo, b = hi > 31 ? 31 : hi;
-          wm = (b == 31 ? 0xFFFFFFFFu : ((1u << (b + 1)) - 1u)) & ~((1u << a) - 1u);
-        }
+        const uint32_t wm = window_bits(lc_lo - c0, lc_hi - c0);
         uint32_t pk[16];
         if ((wm | skb) == 0u) {
 #pragma unroll
           for (int w = 0; w < 16; ++w) pk[w] = 0u;
+        } else if (wm == 0u && (skb & (skb - 1u)) == 0u) {
+          // a single skip key: one exponential for the chunk
+          const int sc = __ffs(skb) - 1;
+          const float p1 = ex2(fmaf(pick32(x + c0, sc), prm.scale_log2, bp_m));
+          ls += p1;
+          __nv_bfloat162 b2 = __floats2bfloat162_rn(p1, p1);
+          const uint32_t both = *reinterpret_cast<uint32_t*>(&b2);
+          const uint32_t word = (sc & 1) ? (both & 0xFFFF0000u) : (both & 0x0000FFFFu);
+#pragma unroll
+          for (int w = 0; w < 16; ++w) pk[w] = (sc >> 1) == w ? word : 0u;
         } else {
           float sp[4] = {0.f, 0.f, 0.f, 0.f};
           if (wm == 0xFFFFFFFFu && skb == 0u) {
@@ -620,17 +661,30 @@ __global__ void __launch_bounds__(NTHREADS, D == 64 ? 2 : 1) fwd_tc_kernel(const
       tc_fence_before();
       mbar_arrive(bar_pfull);
     }
-    // ---- epilogue
+    // ---- epilogue: the normalised row goes to shared memory (the P buffer, free once the last
+    // P.V has completed) in the 128-byte-swizzled tile layout, then one TMA store writes the tile
+    // (rows past the end of the view are clipped by the tensor map).  kBandMerge first brings the
+    // tile of skip partials in by TMA (into the free K stage 0) and merges them row by row.
     const bool row_ok = qi < view_rows;
     const long long orow = (long long)bh * prm.n + i;  // row in [B*H, n] layouts
     const bool have_o = __all_sync(0xffffffffu, ok && j > 0 && mbar_wait(bar_pvdone, (j - 1) & 1, abort_flag));
-    if (have_o) {
-      tc_fence_after();
+    const bool no_keys = MODE == kResidue && __all_sync(0xffffffffu, ok && j == 0);  // tile with no skip at all
+    float lse_log2 = 0.f;
+    if (have_o || no_keys) {
+      if (have_o) tc_fence_after();
+      constexpr uint32_t kTile = L::kTileBytes;
+      bool so_ok = true;
+      if (MODE == kBandMerge) {
+        if (threadIdx.x == 64) {
+          mbar_expect_tx(bar_so, kTile);
+#pragma unroll
+          for (int c = 0; c < D / 64; ++c) tma_load_3d(sK + c * BM * 128, &tms, bar_so, c * 64, (int)q0, bh);
+        }
+        so_ok = __all_sync(0xffffffffu, mbar_wait(bar_so, 0, abort_flag));
+      }
       float inv = l_sum > 0.f ? 1.f / l_sum : 0.f;
       float wl = 1.f, wp = 0.f, lse2 = m_ref + log2f(l_sum);  // log2 of this pass's mass
-      const uint4* so = nullptr;
       if (MODE == kBandMerge && row_ok) {
-        // merge the skip partial of this row
         const float b2 = prm.skip_lse[orow] * kLog2e;
         const float M = fmaxf(lse2, b2);
         wl = ex2(lse2 - M);
@@ -639,48 +693,55 @@ __global__ void __launch_bounds__(NTHREADS, D == 64 ? 2 : 1) fwd_tc_kernel(const
         wl /= den;
         wp /= den;
         lse2 = M + log2f(den);
-        so = reinterpret_cast<const uint4*>(prm.skip_o + orow * D);
       }
-      __nv_bfloat16* orow_ptr = (MODE == kResidue ? prm.skip_o : prm.out) + orow * D;
-      float o[D];  // the whole O row, one load and one wait
-      if (D == 128) tmem_ld128(tO + lane_off, o);
-      else tmem_ld64(tO + lane_off, o);
+      float o[D];
+      if (have_o) {
+        if (D == 128) tmem_ld128(tO + lane_off, o);
+        else tmem_ld64(tO + lane_off, o);
+      } else {
 #pragma unroll
-      for (int c = 0; c < D / 32; ++c) {
-        if (row_ok) {
+        for (int e = 0; e < D; ++e) o[e] = 0.f;
+      }
 #pragma unroll
-          for (int g = 0; g < 4; ++g) {
-            float sp[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-            if (MODE == kBandMerge) bf16x8_to_f32(so[c * 4 + g], sp);
-            uint32_t w[4];
+      for (int c = 0; c < D / 8; ++c) {  // 16-byte chunk c of the row
+        const int blk = c >> 3, cc = c & 7;
+        const uint32_t off = blk * (BM * 128) + r * 128 + ((cc ^ (r & 7)) << 4);
+        float sp[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+        if (MODE == kBandMerge && so_ok) bf16x8_to_f32(*reinterpret_cast<const uint4*>(sbase + L::kK + off), sp);
+        uint32_t w[4];
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const float a0 = o[c * 32 + g * 8 + 2 * e] * inv * wl + sp[2 * e] * wp;
-              const float a1 = o[c * 32 + g * 8 + 2 * e + 1] * inv * wl + sp[2 * e + 1] * wp;
-              __nv_bfloat162 b2 = __floats2bfloat162_rn(a0, a1);
-              w[e] = *reinterpret_cast<uint32_t*>(&b2);
-            }
-            uint4 u;
-            u.x = w[0];
-            u.y = w[1];
-            u.z = w[2];
-            u.w = w[3];
-            *reinterpret_cast<uint4*>(orow_ptr + c * 32 + g * 8) = u;
-          }
+        for (int e = 0; e < 4; ++e) {
+          const float a0 = o[c * 8 + 2 * e] * inv * wl + sp[2 * e] * wp;
+          const float a1 = o[c * 8 + 2 * e + 1] * inv * wl + sp[2 * e + 1] * wp;
+          __nv_bfloat162 b2 = __floats2bfloat162_rn(a0, a1);
+          w[e] = *reinterpret_cast<uint32_t*>(&b2);
         }
+        *reinterpret_cast<uint4*>(sbase + L::kP + off) = make_uint4(w[0], w[1], w[2], w[3]);
+      }
+      lse_log2 = lse2;
+      fence_proxy_async_smem();
+    }
+    // Every softmax warp passes this barrier, epilogue or not (a warp that gave up on a wait must
+    // not leave the others blocked here); the tile is then staged whenever it is stored.
+    asm volatile("bar.sync 1, 128;" ::: "memory");
+    if (have_o || no_keys) {
+      if (threadIdx.x == 64) {
+#pragma unroll
+        for (int c = 0; c < D / 64; ++c) {
+          if (MODE == kResidue)
+            tma_store_4d(&tmo, sP + c * BM * 128, c * 64, res, (int)q0, bh);
+          else
+            tma_store_3d(&tmo, sP + c * BM * 128, c * 64, (int)q0, bh);
+        }
+        tma_store_commit_and_wait_read();  // shared memory must outlive the reads of the store
       }
       if (row_ok) {
         // a row with no key in this pass (only possible for kResidue) has lse -inf
+        const float lse2 = lse_log2;
         const float lse_val = l_sum > 0.f ? lse2 * kLn2 : NEG_INF;
         if (MODE == kResidue) prm.skip_lse[orow] = lse_val;
         else if (prm.lse) prm.lse[orow] = lse_val;
       }
-    } else if (MODE == kResidue && ok && j == 0 && row_ok) {
-      // no skip key for any row of this tile: empty partial
-      uint4 zero = make_uint4(0u, 0u, 0u, 0u);
-#pragma unroll
-      for (int c = 0; c < D / 8; ++c) reinterpret_cast<uint4*>(prm.skip_o + orow * D)[c] = zero;
-      prm.skip_lse[orow] = NEG_INF;
     }
     tc_fence_before();
   }
@@ -792,9 +853,14 @@ cudaError_t launch_fwd_tc_d(const void* q, const void* k, const void* v, const f
   p.scale_log2 = (float)(1.0 / std::sqrt((double)D)) * kLog2e;
   const dim3 grid((unsigned)((n + tc::BM - 1) / tc::BM), (unsigned)BH);
   cudaError_t e;
+  CUtensorMap mo;
+  if (!tc::make_map(&mo, out, BH, n, D)) {
+    *why = "cuTensorMapEncodeTiled (out) failed";
+    return cudaErrorInvalidValue;
+  }
   if (!split) {
     if ((e = tc::set_smem_attr<D, tc::kFused>()) != cudaSuccess) { *why = "cudaFuncSetAttribute"; return e; }
-    tc::fwd_tc_kernel<D, tc::kFused><<<grid, tc::NTHREADS, L::kAlloc, st>>>(mq, mk, mv, p);
+    tc::fwd_tc_kernel<D, tc::kFused><<<grid, tc::NTHREADS, L::kAlloc, st>>>(mq, mk, mv, mo, mo, p);
     *why = "tensor-core kernel launch";
     return cudaGetLastError();
   }
@@ -815,11 +881,17 @@ cudaError_t launch_fwd_tc_d(const void* q, const void* k, const void* v, const f
   }
   p.skip_o = (__nv_bfloat16*)scratch;
   p.skip_lse = (float*)((char*)scratch + rows * D * 2);
+  CUtensorMap rso, mso;  // the skip partials, in the residue view (stored) and the sequence view (loaded)
+  if (!tc::make_residue_map(&rso, p.skip_o, BH, n, D, pi) || !tc::make_map(&mso, p.skip_o, BH, n, D)) {
+    cudaFreeAsync(scratch, st);
+    *why = "cuTensorMapEncodeTiled (skip partials) failed";
+    return cudaErrorInvalidValue;
+  }
   const dim3 grid_r((unsigned)(pi * ((p.T + tc::BM - 1) / tc::BM)), (unsigned)BH);
-  tc::fwd_tc_kernel<D, tc::kResidue><<<grid_r, tc::NTHREADS, L::kAlloc, st>>>(rq, rk, rv, p);
+  tc::fwd_tc_kernel<D, tc::kResidue><<<grid_r, tc::NTHREADS, L::kAlloc, st>>>(rq, rk, rv, rso, rso, p);
   e = cudaGetLastError();
   if (e == cudaSuccess) {
-    tc::fwd_tc_kernel<D, tc::kBandMerge><<<grid, tc::NTHREADS, L::kAlloc, st>>>(mq, mk, mv, p);
+    tc::fwd_tc_kernel<D, tc::kBandMerge><<<grid, tc::NTHREADS, L::kAlloc, st>>>(mq, mk, mv, mo, mso, p);
     e = cudaGetLastError();
   }
   cudaError_t e2 = cudaFreeAsync(scratch, st);

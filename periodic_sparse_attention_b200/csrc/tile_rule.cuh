@@ -76,6 +76,13 @@ PIA_HD void row_tile_mask(long long i, long long j0, int kwin, int pi, int S, in
   }
 }
 
+// Bits of the window columns [lo, hi] (relative to a 32-column chunk) that fall in 0..31.
+PIA_HD uint32_t window_bits(int lo, int hi) {
+  if (lo > 31 || hi < 0 || lo > hi) return 0u;
+  const int a = lo < 0 ? 0 : lo, b = hi > 31 ? 31 : hi;
+  return (b == 31 ? 0xFFFFFFFFu : ((1u << (b + 1)) - 1u)) & ~((1u << a) - 1u);
+}
+
 // Cheapest exact treatment of a 32-column chunk cb of a tile for one row:
 //   kEmpty  no key of the union: p = 0, no exponential
 //   kFull   every column a window key and no skip: one FMA per logit
