@@ -49,16 +49,18 @@ struct Smem {
   static constexpr int kV = kK + NSTAGE * kTileBytes;
   static constexpr int kP = kV + NSTAGE * kTileBytes;
   static constexpr int kBar = kP + BM * BN * 2;          // P: 128 x 128 bf16
-  // S buffers in TMEM: one suffices, the softmax reads a tile's S row with a single load and
-  // releases the buffer at once, so the next tile's Q.K^T overlaps the rest of the softmax
-  static constexpr int kSBufs = 1;
+  // S buffers in TMEM: two for d = 128 (one CTA per SM: the next tile's Q.K^T overlaps this
+  // tile's softmax), one for d = 64 (two CTAs per SM overlap each other instead)
+  static constexpr int kSBufs = D == 128 ? 2 : 1;
   static constexpr int kTmemCols = kSBufs == 2 ? 512 : 256;  // S buffers (128 each) + O (D)
   // barriers: q_full, k_full[2], k_empty[2], v_full[2], v_empty[2], s_full[NSB], s_free[NSB],
   // p_full, pv_done, drain
   static constexpr int kNumBars = 1 + 4 * NSTAGE + 2 * kSBufs + 4;
   static constexpr int kMisc = kBar + kNumBars * 8;      // tmem base (4 B), abort flag (4 B)
-  static constexpr int kTotal = kMisc + 16;
+  static constexpr int kTotal = kMisc + 8;
   static constexpr int kAlloc = kTotal + 1024 - 128;     // slack to align a (>= 128 B aligned) base to 1 KB
+  // d = 64 runs two CTAs per SM: 228 KB of shared memory per SM, 1 KB of it reserved per CTA
+  static_assert(D != 64 || kAlloc <= 228 * 1024 / 2 - 1024, "d = 64 plan must fit two CTAs per SM");
 };
 
 // ---- PTX wrappers ------------------------------------------------------------------------------
@@ -74,35 +76,30 @@ __device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
 __device__ __forceinline__ void mbar_arrive(uint32_t bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
 }
+// One bounded wait step: the thread is suspended until the phase completes or the hint (1 ms)
+// passes, so a waiting warp does not take issue slots from the warps doing the work.
 __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
       "selp.u32 %0, 1, 0, p;\n\t}"
       : "=r"(ok)
-      : "r"(bar), "r"(parity)
+      : "r"(bar), "r"(parity), "r"(1000000u)
       : "memory");
   return ok != 0;
 }
-// Bounded wait: false when the limit passed or another thread of the CTA aborted.  The loop spins
-// on try_wait alone; the abort flag and the SM clock are looked at only every 64 failed tries, so
-// noticing a completed phase costs one try_wait, not a clock read.
+// Bounded wait: false when the limit passed or another thread of the CTA aborted.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag) {
   if (mbar_try_wait(bar, parity)) return true;
-  long long t0 = 0;
-  for (uint32_t it = 1;; ++it) {
+  const long long t0 = clock64();
+  while (true) {
     if (mbar_try_wait(bar, parity)) return true;
-    if ((it & 63u) == 0u) {
-      if (*abort_flag) return false;
-      const long long now = clock64();
-      if (t0 == 0) {
-        t0 = now;
-      } else if (now - t0 > kWaitLimitCycles) {
-        raise_error(kErrWaitTimeout);
-        *abort_flag = 1;
-        return false;
-      }
+    if (*abort_flag) return false;
+    if (clock64() - t0 > kWaitLimitCycles) {
+      raise_error(kErrWaitTimeout);
+      *abort_flag = 1;
+      return false;
     }
   }
 }
@@ -215,12 +212,20 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const float* v) {
 }
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
-// v[k] for a run-time k in 0..31 from a register array, by selects (no local memory).
+// v[k] for a run-time k in 0..31 from a register array: a 5-level tree of selects on the bits of
+// k (independent selects, no local memory, no long dependency chain).
 __device__ __forceinline__ float pick32(const float* v, int k) {
-  float r = v[0];
+  float a[16], b[8], c[4], d[2];
+  const bool k0 = k & 1, k1 = k & 2, k2 = k & 4, k3 = k & 8, k4 = k & 16;
 #pragma unroll
-  for (int e = 1; e < 32; ++e) r = k == e ? v[e] : r;
-  return r;
+  for (int e = 0; e < 16; ++e) a[e] = k0 ? v[2 * e + 1] : v[2 * e];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) b[e] = k1 ? a[2 * e + 1] : a[2 * e];
+#pragma unroll
+  for (int e = 0; e < 4; ++e) c[e] = k2 ? b[2 * e + 1] : b[2 * e];
+#pragma unroll
+  for (int e = 0; e < 2; ++e) d[e] = k3 ? c[2 * e + 1] : c[2 * e];
+  return k4 ? d[1] : d[0];
 }
 
 __device__ __forceinline__ float ex2(float x) {
@@ -305,6 +310,7 @@ __global__ void __launch_bounds__(NTHREADS, D == 64 ? 2 : 1) fwd_tc_kernel(const
     walk.pi = 1;
     walk.S = 0;
     walk.m0 = 1;
+    walk.rpi = 1.0;
   } else {
     q0 = (long long)blockIdx.x * BM;
     walk.init(q0, prm.n, BM, prm.kwin, prm.pi, MODE == kFused ? prm.S : 0);
@@ -503,60 +509,45 @@ __global__ void __launch_bounds__(NTHREADS, D == 64 ? 2 : 1) fwd_tc_kernel(const
     const float NEG_INF = -INFINITY;
 
     float m_ref = NEG_INF;  // reference max (log2 units)
-    float l_sum = 0.f;      // running sum of probabilities against m_ref
+    float l_sum = 0.f;      // running sum of probabilities against m_ref (fp32 values: for lse)
+    float l_rnd = 0.f;      // the same sum of their bf16 roundings (the weights in P.V: for out)
     int j = 0;
     for (int t = walk.next(0); ok && t >= 0; t = walk.next(t + 1), ++j) {
       const int sb = j % NSB;
       // every lane of the warp takes the same branch: tcgen05.ld is .sync.aligned
       if (!__all_sync(0xffffffffu, mbar_wait(bar_sfull(sb), (j / NSB) & 1, abort_flag))) { ok = false; break; }
       tc_fence_after();
-      // d = 128 (one CTA per SM): the whole S row stays in registers and the buffer is released at
-      // once, so the next Q.K^T overlaps this softmax.  d = 64 (two CTAs per SM, 168 registers):
-      // the row is read once for the max and again, in two halves, for the probabilities; the
-      // buffer is released after that, and the SM's other CTA fills the gap.
-      constexpr bool kRowInRegs = D == 128;
-      float x[BN];
-      tmem_ld128(tS + 128 * sb + lane_off, x);  // the whole S row, one load and one wait
-      if (kRowInRegs) {
-        tc_fence_before();
-        mbar_arrive(bar_sfree(sb));
-      }
-
+      const uint32_t tSb = tS + 128 * sb + lane_off;
       // the index rule on this tile, for row qi: window columns [lc_lo, lc_hi], skip columns bitmask
       int lc_lo, lc_hi;
       uint32_t sk[BN / 32];
       if (MODE == kResidue)
         row_tile_mask(qi, (long long)t * BN, prm.S, 1, 0, 1, lc_lo, lc_hi, sk, m0);
       else
-        row_tile_mask(qi, (long long)t * BN, prm.kwin, prm.pi, MODE == kFused ? prm.S : 0, m0, lc_lo, lc_hi, sk);
+        row_tile_mask(qi, (long long)t * BN, prm.kwin, prm.pi, MODE == kFused ? prm.S : 0, m0, lc_lo, lc_hi, sk, 0,
+                      walk.rpi);
+      const bool has_win = lc_lo <= lc_hi;
+      const bool has_skip = (sk[0] | sk[1] | sk[2] | sk[3]) != 0u;
 
-      // The tile max of the biased logits, exactly: per 32-column chunk, window-only chunks take
-      // the max of their raw scores, chunks without keys are skipped, and chunks that straddle the
-      // window edge or hold skip keys mask each column (window bits wm, skip bits skb).  The max of
-      // a kind of key is then scaled and given its prior.  (An exact reference keeps the largest
-      // probability of a row at 1, which bf16 holds exactly.)
-      float mw = NEG_INF, ms = NEG_INF;
+      // Pass 1: a reference for the tile, from the whole S row in one load: the max of the raw
+      // scores, scaled, plus the larger prior present.  It bounds the true max of the biased
+      // logits from above, and not by much: a key can only beat a key of higher prior by scoring
+      // at least the prior gap more, so the bound exceeds the true max by at most twice the score
+      // spread of the row.  Probabilities only need a reference at or above their max.
+      float mt;
+      {
+        float x[BN];
+        tmem_ld128(tSb, x);
+        float mx[8];
 #pragma unroll
-      for (int cb = 0; cb < BN / 32; ++cb) {
-        const int c0 = cb * 32;
-        const uint32_t wm = window_bits(lc_lo - c0, lc_hi - c0), skb = sk[cb];
-        if (wm == 0xFFFFFFFFu && skb == 0u) {
-          float m4[4] = {x[c0], x[c0 + 1], x[c0 + 2], x[c0 + 3]};
+        for (int e = 0; e < 8; ++e) mx[e] = x[e];
 #pragma unroll
-          for (int e = 4; e < 32; ++e) m4[e & 3] = fmaxf(m4[e & 3], x[c0 + e]);
-          mw = fmaxf(mw, fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3])));
-        } else if (wm == 0u && skb != 0u && (skb & (skb - 1u)) == 0u) {
-          ms = fmaxf(ms, pick32(x + c0, __ffs(skb) - 1));  // a single skip key
-        } else if ((wm | skb) != 0u) {
-#pragma unroll
-          for (int e = 0; e < 32; ++e) {
-            mw = fmaxf(mw, (wm >> e) & 1u ? x[c0 + e] : NEG_INF);
-            ms = fmaxf(ms, (skb >> e) & 1u ? x[c0 + e] : NEG_INF);
-          }
-        }
+        for (int c = 8; c < BN; ++c) mx[c & 7] = fmaxf(mx[c & 7], x[c]);
+        const float mraw =
+            fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])), fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
+        const float top = has_win ? (has_skip ? fmaxf(bias_l, bias_p) : bias_l) : bias_p;
+        mt = (has_win || has_skip) ? fmaf(mraw, prm.scale_log2, top) : NEG_INF;
       }
-      const float mt = fmaxf(mw == NEG_INF ? NEG_INF : fmaf(mw, prm.scale_log2, bias_l),
-                             ms == NEG_INF ? NEG_INF : fmaf(ms, prm.scale_log2, bias_p));
 
       // lazy reference max
       float factor = 1.f;
@@ -565,6 +556,7 @@ __global__ void __launch_bounds__(NTHREADS, D == 64 ? 2 : 1) fwd_tc_kernel(const
         factor = ex2(m_ref - mt);  // 0 when m_ref = -inf
         rescale = l_sum > 0.f;
         l_sum *= factor;
+        l_rnd *= factor;
         m_ref = mt;
       }
       const float m_use = m_ref == NEG_INF ? 0.f : m_ref;
@@ -589,74 +581,66 @@ __global__ void __launch_bounds__(NTHREADS, D == 64 ? 2 : 1) fwd_tc_kernel(const
         }
       }
 
-      // Probabilities against the reference, the row sum, and P (bf16) into shared memory,
-      // K-major with the 128-byte swizzle (16-byte chunk cc of row r at chunk cc ^ (r & 7)).
-      // Per 32-column chunk: no key -> zeros; window keys only -> one FMA per logit; otherwise
-      // the window bits and skip bits select each logit's prior (-inf: p = 0).
+      // Pass 2, one 32-column chunk at a time (a rolled loop, re-reading the chunk from TMEM):
+      // probabilities against the reference, P (bf16) into shared memory (K-major, 128-byte
+      // swizzle: 16-byte chunk cc of row r at cc ^ (r & 7)), and two row sums -- of the fp32
+      // probabilities (for lse) and of their bf16 roundings (the weights P.V actually applies; the
+      // output is normalised by this one, so a row of one key reproduces that key's value).
+      //   no key in the chunk -> zeros; window keys only -> one FMA per logit; one skip key and
+      //   no window key -> one exponential; otherwise window bits and skip bits pick each prior.
       const float bl_m = bias_l - m_use, bp_m = bias_p - m_use;
-      float ls = 0.f;
-#pragma unroll
+      float ls = 0.f, lr = 0.f;
+#pragma unroll 1
       for (int cb = 0; cb < BN / 32; ++cb) {
         const int c0 = cb * 32;
-        if (!kRowInRegs && (cb & 1) == 0) tmem_ld64(tS + 128 * sb + lane_off + c0, x + c0);  // re-read half
-        const uint32_t skb = sk[cb];
+        float x[32];
+        tmem_ld32(tSb + c0, x);
+        const uint32_t skb = cb == 0 ? sk[0] : cb == 1 ? sk[1] : cb == 2 ? sk[2] : sk[3];
         const uint32_t wm = window_bits(lc_lo - c0, lc_hi - c0);
         uint32_t pk[16];
         if ((wm | skb) == 0u) {
 #pragma unroll
           for (int w = 0; w < 16; ++w) pk[w] = 0u;
         } else if (wm == 0u && (skb & (skb - 1u)) == 0u) {
-          // a single skip key: one exponential for the chunk
           const int sc = __ffs(skb) - 1;
-          const float p1 = ex2(fmaf(pick32(x + c0, sc), prm.scale_log2, bp_m));
-          ls += p1;
+          const float p1 = ex2(fmaf(pick32(x, sc), prm.scale_log2, bp_m));
           __nv_bfloat162 b2 = __floats2bfloat162_rn(p1, p1);
           const uint32_t both = *reinterpret_cast<uint32_t*>(&b2);
+          ls += p1;
+          lr += __uint_as_float(both << 16);
           const uint32_t word = (sc & 1) ? (both & 0xFFFF0000u) : (both & 0x0000FFFFu);
 #pragma unroll
           for (int w = 0; w < 16; ++w) pk[w] = (sc >> 1) == w ? word : 0u;
         } else {
-          float sp[4] = {0.f, 0.f, 0.f, 0.f};
-          if (wm == 0xFFFFFFFFu && skb == 0u) {
+          float sp[4] = {0.f, 0.f, 0.f, 0.f}, sr[4] = {0.f, 0.f, 0.f, 0.f};
+          const bool full = wm == 0xFFFFFFFFu && skb == 0u;
 #pragma unroll
-            for (int e = 0; e < 32; e += 2) {
-              const float p0 = ex2(fmaf(x[c0 + e], prm.scale_log2, bl_m));
-              const float p1 = ex2(fmaf(x[c0 + e + 1], prm.scale_log2, bl_m));
-              sp[(e >> 1) & 3] += p0 + p1;
-              __nv_bfloat162 b2 = __floats2bfloat162_rn(p0, p1);
-              pk[e >> 1] = *reinterpret_cast<uint32_t*>(&b2);
-            }
-          } else {
-#pragma unroll
-            for (int e = 0; e < 32; e += 2) {
-              const float b0 = (wm >> e) & 1u ? bl_m : ((skb >> e) & 1u ? bp_m : NEG_INF);
-              const float b1 = (wm >> (e + 1)) & 1u ? bl_m : ((skb >> (e + 1)) & 1u ? bp_m : NEG_INF);
-              const float p0 = ex2(fmaf(x[c0 + e], prm.scale_log2, b0));
-              const float p1 = ex2(fmaf(x[c0 + e + 1], prm.scale_log2, b1));
-              sp[(e >> 1) & 3] += p0 + p1;
-              __nv_bfloat162 b2 = __floats2bfloat162_rn(p0, p1);
-              pk[e >> 1] = *reinterpret_cast<uint32_t*>(&b2);
-            }
+          for (int e = 0; e < 32; e += 2) {
+            const float b0 = full || ((wm >> e) & 1u) ? bl_m : ((skb >> e) & 1u ? bp_m : NEG_INF);
+            const float b1 = full || ((wm >> (e + 1)) & 1u) ? bl_m : ((skb >> (e + 1)) & 1u ? bp_m : NEG_INF);
+            const float p0 = ex2(fmaf(x[e], prm.scale_log2, b0));
+            const float p1 = ex2(fmaf(x[e + 1], prm.scale_log2, b1));
+            __nv_bfloat162 b2 = __floats2bfloat162_rn(p0, p1);
+            const uint32_t u = *reinterpret_cast<uint32_t*>(&b2);
+            pk[e >> 1] = u;
+            sp[(e >> 1) & 3] += p0 + p1;
+            sr[(e >> 1) & 3] += __uint_as_float(u << 16) + __uint_as_float(u & 0xFFFF0000u);
           }
           ls += (sp[0] + sp[1]) + (sp[2] + sp[3]);
+          lr += (sr[0] + sr[1]) + (sr[2] + sr[3]);
         }
 #pragma unroll
         for (int g = 0; g < 4; ++g) {  // 16-byte chunks 4 cb + g of the row
           const int c = cb * 4 + g;
           const int blk = c >> 3, cc = c & 7;
-          uint4 u;
-          u.x = pk[g * 4 + 0];
-          u.y = pk[g * 4 + 1];
-          u.z = pk[g * 4 + 2];
-          u.w = pk[g * 4 + 3];
-          *reinterpret_cast<uint4*>(sbase + L::kP + blk * (BM * 128) + r * 128 + ((cc ^ (r & 7)) << 4)) = u;
+          *reinterpret_cast<uint4*>(sbase + L::kP + blk * (BM * 128) + r * 128 + ((cc ^ (r & 7)) << 4)) =
+              make_uint4(pk[g * 4 + 0], pk[g * 4 + 1], pk[g * 4 + 2], pk[g * 4 + 3]);
         }
       }
       l_sum += ls;
-      if (!kRowInRegs) {
-        tc_fence_before();
-        mbar_arrive(bar_sfree(sb));
-      }
+      l_rnd += lr;
+      tc_fence_before();
+      mbar_arrive(bar_sfree(sb));  // the S buffer may take the Q.K^T of tile j + NSB
       fence_proxy_async_smem();
       tc_fence_before();
       mbar_arrive(bar_pfull);
@@ -682,7 +666,7 @@ __global__ void __launch_bounds__(NTHREADS, D == 64 ? 2 : 1) fwd_tc_kernel(const
         }
         so_ok = __all_sync(0xffffffffu, mbar_wait(bar_so, 0, abort_flag));
       }
-      float inv = l_sum > 0.f ? 1.f / l_sum : 0.f;
+      float inv = l_rnd > 0.f ? 1.f / l_rnd : 0.f;
       float wl = 1.f, wp = 0.f, lse2 = m_ref + log2f(l_sum);  // log2 of this pass's mass
       if (MODE == kBandMerge && row_ok) {
         const float b2 = prm.skip_lse[orow] * kLog2e;

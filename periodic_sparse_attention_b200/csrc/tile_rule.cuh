@@ -17,11 +17,21 @@ namespace pia {
 
 constexpr int kTileKeys = 128;  // keys per tile (BN)
 
+// floor(a / b) for 0 <= a < 2^52, b >= 1, through a double reciprocal of b (rb = 1.0 / b) and
+// an exact +-1 correction -- GPUs have no integer divider, and these run per row and per tile.
+PIA_HD long long div_floor(long long a, long long b, double rb) {
+  long long q = (long long)((double)a * rb);
+  if (q * b > a) --q;
+  else if ((q + 1) * b <= a) ++q;
+  return q;
+}
+
 // Walks, in increasing order, the 128-key tiles that hold at least one key of the union of L(i)
 // and P(i) over the query rows [i0, last] of one tile.
 struct TileWalk {
   long long i0, last, band_lo;  // query rows [i0, last]; the window keys of the tile start at band_lo
   int pi, S, m0;
+  double rpi;                   // 1.0 / pi
   PIA_HD void init(long long i0_, long long n, int rows, int kwin, int pi_, int S_) {
     i0 = i0_;
     last = i0_ + rows - 1 < n - 1 ? i0_ + rows - 1 : n - 1;
@@ -29,6 +39,7 @@ struct TileWalk {
     pi = pi_;
     S = S_;
     m0 = kwin / pi_ + 1;
+    rpi = 1.0 / (double)pi_;
   }
   // smallest needed key tile index >= t, or -1 when none is left
   PIA_HD int next(int t) const {
@@ -38,8 +49,8 @@ struct TileWalk {
     // the skip block of m, [i0 - m pi, last - m pi], reaches row p iff m pi <= last - p;
     // the largest such m has the leftmost block
     const long long room = last - p;
-    if (room >= 0) {
-      long long mm = room / pi;
+    if (room >= 0 && S >= m0) {
+      long long mm = div_floor(room, pi, rpi);
       if (mm > S) mm = S;
       if (mm >= m0) {
         long long st = i0 - mm * pi;
@@ -55,9 +66,9 @@ struct TileWalk {
 // lc_lo > lc_hi) and a 128-bit mask of skip columns.  Skip columns never overlap the window.
 // The window of row i is [max(0, i - kwin), i - lo_off]: lo_off = 0 for pi-attention's window;
 // the residue-class pass uses it for the skip band of a residue sequence (kwin = S, lo_off = m0,
-// no skips).
+// no skips).  rpi = 1.0 / pi.
 PIA_HD void row_tile_mask(long long i, long long j0, int kwin, int pi, int S, int m0, int& lc_lo, int& lc_hi,
-                          uint32_t sk[kTileKeys / 32], int lo_off = 0) {
+                          uint32_t sk[kTileKeys / 32], int lo_off = 0, double rpi = 0.0) {
   const long long d0 = i - j0;  // i - j at column 0
   const long long lo = (i - kwin > 0 ? i - kwin : 0) - j0;
   const long long hi = d0 - lo_off;
@@ -65,13 +76,11 @@ PIA_HD void row_tile_mask(long long i, long long j0, int kwin, int pi, int S, in
   lc_hi = hi > kTileKeys - 1 ? kTileKeys - 1 : (hi < -1 ? -1 : (int)hi);
   for (int w = 0; w < kTileKeys / 32; ++w) sk[w] = 0u;
   if (d0 > kwin && S >= m0) {
-    long long m_hi = d0 / pi;
-    if (m_hi > S) m_hi = S;
-    long long m_lo = d0 - (kTileKeys - 1) > 0 ? (d0 - (kTileKeys - 1) + pi - 1) / pi : 0;
-    if (m_lo < m0) m_lo = m0;
-    for (long long m = m_lo; m <= m_hi; ++m) {
-      const int c = (int)(d0 - m * pi);
-      sk[c >> 5] |= 1u << (c & 31);
+    // skip columns c = d0 - m pi in 0..127: from the largest m (smallest c) upwards in c
+    long long m = div_floor(d0, pi, rpi > 0.0 ? rpi : 1.0 / (double)pi);
+    if (m > S) m = S;
+    for (long long c = d0 - m * pi; m >= m0 && c < kTileKeys; --m, c += pi) {
+      if (c >= 0) sk[c >> 5] |= 1u << (c & 31);
     }
   }
 }
