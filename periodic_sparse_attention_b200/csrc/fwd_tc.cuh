@@ -212,6 +212,33 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const float* v) {
 }
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
+// log(sigmoid(x)) = min(x, 0) - log(1 + e^-|x|) from the fast exponential and logarithm: the
+// absolute error (~1e-7) is far below what the priors need, and the precise library versions are
+// on the critical path of every CTA.
+__device__ __forceinline__ float log_sigmoid_fast(float x) {
+  return fminf(x, 0.f) - __logf(1.f + __expf(-fabsf(x)));
+}
+
+// Packed fp32 pairs (Blackwell f32x2 arithmetic: two lanes of work per instruction).
+__device__ __forceinline__ unsigned long long f2pack(float a, float b) {
+  unsigned long long r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
+  return r;
+}
+__device__ __forceinline__ void f2unpack(unsigned long long r, float& a, float& b) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(r));
+}
+__device__ __forceinline__ unsigned long long f2fma(unsigned long long a, unsigned long long b, unsigned long long c) {
+  unsigned long long d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ unsigned long long f2add(unsigned long long a, unsigned long long b) {
+  unsigned long long d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+
 // v[k] for a run-time k in 0..31 from a register array: a 5-level tree of selects on the bits of
 // k (independent selects, no local memory, no long dependency chain).
 __device__ __forceinline__ float pick32(const float* v, int k) {
@@ -504,8 +531,8 @@ __global__ void __launch_bounds__(NTHREADS, D == 64 ? 2 : 1) fwd_tc_kernel(const
     }
     asm volatile("bar.sync 1, 128;" ::: "memory");  // every thread has read w_g: P may be written
     // the prior of the keys this pass unmasks as "window" columns
-    const float bias_l = log_sigmoid(MODE == kResidue ? -z : z) * kLog2e;  // log2(alpha), or log2(1-alpha)
-    const float bias_p = log_sigmoid(-z) * kLog2e;                         // log2(1 - alpha)
+    const float bias_l = log_sigmoid_fast(MODE == kResidue ? -z : z) * kLog2e;  // log2(alpha), or log2(1-alpha)
+    const float bias_p = log_sigmoid_fast(-z) * kLog2e;                         // log2(1 - alpha)
     const float NEG_INF = -INFINITY;
 
     float m_ref = NEG_INF;  // reference max (log2 units)
@@ -612,22 +639,48 @@ __global__ void __launch_bounds__(NTHREADS, D == 64 ? 2 : 1) fwd_tc_kernel(const
 #pragma unroll
           for (int w = 0; w < 16; ++w) pk[w] = (sc >> 1) == w ? word : 0u;
         } else {
-          float sp[4] = {0.f, 0.f, 0.f, 0.f}, sr[4] = {0.f, 0.f, 0.f, 0.f};
-          const bool full = wm == 0xFFFFFFFFu && skb == 0u;
+          // per pair of columns: one packed FMA (scale and prior), two exponentials, one pack to
+          // bf16x2, and packed adds into the fp32 sum and into the sum of the bf16 roundings
+          // (unpacked from the bf16x2 word by two integer ops)
+          unsigned long long sp[4], sr[4];
 #pragma unroll
-          for (int e = 0; e < 32; e += 2) {
-            const float b0 = full || ((wm >> e) & 1u) ? bl_m : ((skb >> e) & 1u ? bp_m : NEG_INF);
-            const float b1 = full || ((wm >> (e + 1)) & 1u) ? bl_m : ((skb >> (e + 1)) & 1u ? bp_m : NEG_INF);
-            const float p0 = ex2(fmaf(x[e], prm.scale_log2, b0));
-            const float p1 = ex2(fmaf(x[e + 1], prm.scale_log2, b1));
-            __nv_bfloat162 b2 = __floats2bfloat162_rn(p0, p1);
-            const uint32_t u = *reinterpret_cast<uint32_t*>(&b2);
-            pk[e >> 1] = u;
-            sp[(e >> 1) & 3] += p0 + p1;
-            sr[(e >> 1) & 3] += __uint_as_float(u << 16) + __uint_as_float(u & 0xFFFF0000u);
+          for (int a = 0; a < 4; ++a) sp[a] = sr[a] = 0ull;
+          const unsigned long long sc2 = f2pack(prm.scale_log2, prm.scale_log2);
+          if (wm == 0xFFFFFFFFu && skb == 0u) {  // window keys only
+            const unsigned long long bb = f2pack(bl_m, bl_m);
+#pragma unroll
+            for (int e = 0; e < 32; e += 2) {
+              float t0, t1;
+              f2unpack(f2fma(f2pack(x[e], x[e + 1]), sc2, bb), t0, t1);
+              const float p0 = ex2(t0), p1 = ex2(t1);
+              __nv_bfloat162 b2 = __floats2bfloat162_rn(p0, p1);
+              const uint32_t u = *reinterpret_cast<uint32_t*>(&b2);
+              pk[e >> 1] = u;
+              sp[(e >> 1) & 3] = f2add(sp[(e >> 1) & 3], f2pack(p0, p1));
+              sr[(e >> 1) & 3] = f2add(sr[(e >> 1) & 3], f2pack(__uint_as_float(u << 16), __uint_as_float(u & 0xFFFF0000u)));
+            }
+          } else {  // window edge and / or skip keys: each column's prior from its bits
+#pragma unroll
+            for (int e = 0; e < 32; e += 2) {
+              const float b0 = (wm >> e) & 1u ? bl_m : ((skb >> e) & 1u ? bp_m : NEG_INF);
+              const float b1 = (wm >> (e + 1)) & 1u ? bl_m : ((skb >> (e + 1)) & 1u ? bp_m : NEG_INF);
+              float t0, t1;
+              f2unpack(f2fma(f2pack(x[e], x[e + 1]), sc2, f2pack(b0, b1)), t0, t1);
+              const float p0 = ex2(t0), p1 = ex2(t1);
+              __nv_bfloat162 b2 = __floats2bfloat162_rn(p0, p1);
+              const uint32_t u = *reinterpret_cast<uint32_t*>(&b2);
+              pk[e >> 1] = u;
+              sp[(e >> 1) & 3] = f2add(sp[(e >> 1) & 3], f2pack(p0, p1));
+              sr[(e >> 1) & 3] = f2add(sr[(e >> 1) & 3], f2pack(__uint_as_float(u << 16), __uint_as_float(u & 0xFFFF0000u)));
+            }
           }
-          ls += (sp[0] + sp[1]) + (sp[2] + sp[3]);
-          lr += (sr[0] + sr[1]) + (sr[2] + sr[3]);
+          const unsigned long long sps = f2add(f2add(sp[0], sp[1]), f2add(sp[2], sp[3]));
+          const unsigned long long srs = f2add(f2add(sr[0], sr[1]), f2add(sr[2], sr[3]));
+          float a0, a1, r0, r1;
+          f2unpack(sps, a0, a1);
+          f2unpack(srs, r0, r1);
+          ls += a0 + a1;
+          lr += r0 + r1;
         }
 #pragma unroll
         for (int g = 0; g < 4; ++g) {  // 16-byte chunks 4 cb + g of the row
