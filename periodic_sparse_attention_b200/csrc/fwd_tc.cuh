@@ -13,15 +13,15 @@
 //                       rule as a mask and the gate as a log-prior (log(alpha) on window keys,
 //                       log(1 - alpha) on skip keys, -inf elsewhere), keeps one running max and
 //                       one running sum for the whole union (a single softmax), writes P (bf16)
-//                       to shared memory in the MMA operand layout; at the end divides O by the
-//                       sum and writes out and lse.
+//                       back into TMEM over the S columns it has read, where the P.V MMA takes
+//                       its A operand; at the end divides O by the sum and writes out and lse.
 //
 // Online softmax with a lazy reference: probabilities are taken against a reference max that is
 // only raised when a tile's max exceeds it by more than 2^8, so O (in TMEM) is rescaled rarely;
 // every probability stays <= 2^8 and the final division uses the same reference, so the result
 // is exact up to rounding.
 //
-// Every wait on an mbarrier is bounded (pia::kWaitLimitNs).  A wait that gives up sets the device
+// Every wait on an mbarrier is bounded (pia::kWaitLimitCycles).  A wait that gives up sets the device
 // error word and an abort flag in shared memory; all roles then leave their loops, drain their
 // own asynchronous work (bounded again) and the CTA frees its TMEM and exits.
 #pragma once
@@ -37,7 +37,11 @@ namespace tc {
 constexpr int BM = 128;       // query rows per CTA
 constexpr int BN = kTileKeys; // keys per tile
 constexpr int NSTAGE = 2;     // K/V ring depth
-constexpr int NTHREADS = 192; // warp 0 TMA, warp 1 MMA, warps 2-5 softmax
+// Softmax warpgroups per CTA: d = 128 runs one CTA per SM, and two warpgroups split each S row
+// by columns (a second warp per scheduler hides latency); d = 64 runs two CTAs per SM with one.
+template <int D> constexpr int kGroups = D == 128 ? 2 : 1;
+// warp 0 TMA, warp 1 MMA, warps 2 .. 2 + 4 * groups - 1 softmax
+template <int D> constexpr int kThreads = 64 + 128 * kGroups<D>;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 
 // ---- shared memory plan (offsets from a 1024-byte aligned base) ---------------------------------
@@ -47,17 +51,20 @@ struct Smem {
   static constexpr int kQ = 0;
   static constexpr int kK = kQ + kTileBytes;
   static constexpr int kV = kK + NSTAGE * kTileBytes;
-  static constexpr int kP = kV + NSTAGE * kTileBytes;
-  static constexpr int kBar = kP + BM * BN * 2;          // P: 128 x 128 bf16
+  static constexpr int kBar = kV + NSTAGE * kTileBytes;  // (P lives in TMEM, over its S columns)
   // S buffers in TMEM: two for d = 128 (one CTA per SM: the next tile's Q.K^T overlaps this
   // tile's softmax), one for d = 64 (two CTAs per SM overlap each other instead)
   static constexpr int kSBufs = D == 128 ? 2 : 1;
   static constexpr int kTmemCols = kSBufs == 2 ? 512 : 256;  // S buffers (128 each) + O (D)
   // barriers: q_full, k_full[2], k_empty[2], v_full[2], v_empty[2], s_full[NSB], s_free[NSB],
-  // p_full, pv_done, drain
-  static constexpr int kNumBars = 1 + 4 * NSTAGE + 2 * kSBufs + 4;
+  // pv_done[NSB], p_full, drain, skip partials, (two groups) max exchange
+  static constexpr int kNumBars = 1 + 4 * NSTAGE + 3 * kSBufs + 3 + (kGroups<D> > 1 ? 1 : 0);
   static constexpr int kMisc = kBar + kNumBars * 8;      // tmem base (4 B), abort flag (4 B)
-  static constexpr int kTotal = kMisc + 8;
+  // two-group exchange of per-row partials: tile maxima (double-buffered), fp32 and rounded sums
+  static constexpr int kXch = kMisc + 8;
+  static constexpr int kXchBytes = kGroups<D> > 1 ? (2 * 2 + 2) * kGroups<D> * BM * 4 : 0;
+  static constexpr int kWg = kXch + kXchBytes;          // w_g[h] staging, D floats
+  static constexpr int kTotal = kWg + D * 4;
   static constexpr int kAlloc = kTotal + 1024 - 128;     // slack to align a (>= 128 B aligned) base to 1 KB
   // d = 64 runs two CTAs per SM: 228 KB of shared memory per SM, 1 KB of it reserved per CTA
   static_assert(D != 64 || kAlloc <= 228 * 1024 / 2 - 1024, "d = 64 plan must fit two CTAs per SM");
@@ -150,6 +157,16 @@ __device__ __forceinline__ void tc_mma(uint32_t tmem_d, uint64_t adesc, uint64_t
       "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
       : "memory");
 }
+// The same with A (M x K, bf16 packed two per 32-bit column, one row per lane) read from TMEM.
+__device__ __forceinline__ void tc_mma_ts(uint32_t tmem_d, uint32_t tmem_a, uint64_t bdesc, uint32_t idesc,
+                                          uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(tmem_d),
+      "r"(tmem_a), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
 __device__ __forceinline__ void tc_commit(uint32_t bar) {
   asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar) : "memory");
 }
@@ -208,6 +225,14 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const float* v) {
       "r"(__float_as_uint(v[24])), "r"(__float_as_uint(v[25])), "r"(__float_as_uint(v[26])),
       "r"(__float_as_uint(v[27])), "r"(__float_as_uint(v[28])), "r"(__float_as_uint(v[29])),
       "r"(__float_as_uint(v[30])), "r"(__float_as_uint(v[31]))
+      : "memory");
+}
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t* v) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+      "%15, %16};" ::"r"(taddr),
+      "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]), "r"(v[8]), "r"(v[9]),
+      "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15])
       : "memory");
 }
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
@@ -303,7 +328,7 @@ struct Params {
 };
 
 template <int D, int MODE>
-__global__ void __launch_bounds__(NTHREADS, D == 64 ? 2 : 1) fwd_tc_kernel(const __grid_constant__ CUtensorMap tmq,
+__global__ void __launch_bounds__(kThreads<D>, D == 64 ? 2 : 1) fwd_tc_kernel(const __grid_constant__ CUtensorMap tmq,
                                                                           const __grid_constant__ CUtensorMap tmk,
                                                                           const __grid_constant__ CUtensorMap tmv,
                                                                           const __grid_constant__ CUtensorMap tmo,
@@ -344,7 +369,12 @@ __global__ void __launch_bounds__(NTHREADS, D == 64 ? 2 : 1) fwd_tc_kernel(const
   }
   const int view_rows = MODE == kResidue ? prm.T : prm.n;
 
-  const uint32_t sQ = base + L::kQ, sK = base + L::kK, sV = base + L::kV, sP = base + L::kP;
+  const uint32_t sQ = base + L::kQ, sK = base + L::kK, sV = base + L::kV;
+  // P of tile j sits in TMEM over the columns of S buffer j % NSB that the softmax has read:
+  // the 32-key chunk cb of P (16 packed columns) at column pcol(cb) of the buffer.  Chunks are
+  // handled by the softmax group cb / CPG, which reads its S chunks in order before writing them.
+  constexpr int CPG_K = (BN / 32) / kGroups<D>;
+  auto pcol = [](int cb) { return 64 * (cb / CPG_K) + 16 * (cb % CPG_K); };
   const uint32_t bar0 = base + L::kBar;
   const uint32_t bar_q = bar0;
   auto bar_kfull = [&](int s) { return bar0 + 8u * (1 + s); };
@@ -354,10 +384,11 @@ __global__ void __launch_bounds__(NTHREADS, D == 64 ? 2 : 1) fwd_tc_kernel(const
   constexpr int NSB = L::kSBufs;
   auto bar_sfull = [&](int b) { return bar0 + 8u * (1 + 4 * NSTAGE + b); };
   auto bar_sfree = [&](int b) { return bar0 + 8u * (1 + 4 * NSTAGE + NSB + b); };
-  const uint32_t bar_pfull = bar0 + 8u * (1 + 4 * NSTAGE + 2 * NSB);
-  const uint32_t bar_pvdone = bar_pfull + 8;
-  const uint32_t bar_drain = bar_pfull + 16;
-  const uint32_t bar_so = bar_pfull + 24;  // kBandMerge: the tile of skip partials has landed
+  auto bar_pvdone = [&](int b) { return bar0 + 8u * (1 + 4 * NSTAGE + 2 * NSB + b); };  // P.V of buffer b
+  const uint32_t bar_pfull = bar0 + 8u * (1 + 4 * NSTAGE + 3 * NSB);
+  const uint32_t bar_drain = bar_pfull + 8;
+  const uint32_t bar_so = bar_pfull + 16;  // kBandMerge: the tile of skip partials has landed
+  const uint32_t bar_xm = bar_pfull + 24;  // two groups: a tile's partial maxima are exchanged
   uint32_t* const tmem_slot = reinterpret_cast<uint32_t*>(sbase + L::kMisc);
   volatile int* const abort_flag = reinterpret_cast<volatile int*>(sbase + L::kMisc + 4);
 
@@ -371,12 +402,13 @@ __global__ void __launch_bounds__(NTHREADS, D == 64 ? 2 : 1) fwd_tc_kernel(const
     }
     for (int b = 0; b < NSB; ++b) {
       mbar_init(bar_sfull(b), 1);
-      mbar_init(bar_sfree(b), BM);
+      mbar_init(bar_sfree(b), BM * kGroups<D>);
+      mbar_init(bar_pvdone(b), 1);
     }
-    mbar_init(bar_pfull, BM);
-    mbar_init(bar_pvdone, 1);
+    mbar_init(bar_pfull, BM * kGroups<D>);
     mbar_init(bar_drain, 1);
     mbar_init(bar_so, 1);
+    if (kGroups<D> > 1) mbar_init(bar_xm, BM * kGroups<D>);
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -449,13 +481,13 @@ __global__ void __launch_bounds__(NTHREADS, D == 64 ? 2 : 1) fwd_tc_kernel(const
         }
       };
       // O += P V_j : K = 128 keys, 16 per instruction; V is N-major (d contiguous)
-      auto issue_pv = [&](int s, bool first) {
+      auto issue_pv = [&](int s, int b, bool first) {  // A = P from TMEM (S buffer b)
 #pragma unroll
         for (int kk = 0; kk < BN / 16; ++kk) {
-          const uint32_t aoff = (kk >> 2) * (BM * 128) + (kk & 3) * 32;
+          const uint32_t acol = 128 * b + pcol(kk >> 1) + 8 * (kk & 1);
           const uint32_t boff = kk * 16 * 128;
-          tc_mma(tO, sw128_desc(sP + aoff, 16, 1024), sw128_desc(sV + s * kTile + boff, BN * 128, 1024), idesc_pv,
-                 (first && kk == 0) ? 0u : 1u);
+          tc_mma_ts(tO, tS + acol, sw128_desc(sV + s * kTile + boff, BN * 128, 1024), idesc_pv,
+                    (first && kk == 0) ? 0u : 1u);
         }
       };
       // Q.K^T of tile j needs its K stage loaded and its S buffer released by tile j - NSB
@@ -472,16 +504,20 @@ __global__ void __launch_bounds__(NTHREADS, D == 64 ? 2 : 1) fwd_tc_kernel(const
       int j = 0;
       int t = walk.next(0);
       if (okw && t >= 0) okw = try_qk(0);
+      // With two S buffers the next Q.K^T goes first (it overlaps this tile's softmax); with one,
+      // P.V of this tile must read P before the next Q.K^T overwrites the buffer, so it goes first
+      // (the tensor pipe runs one thread's MMAs in issue order).
       while (okw && t >= 0) {
         const int tn = walk.next(t + 1);
         const int s = j % NSTAGE;
-        if (tn >= 0 && !try_qk(j + 1)) break;
+        if (NSB == 2 && tn >= 0 && !try_qk(j + 1)) break;
         if (!mbar_wait(bar_vfull(s), (j / NSTAGE) & 1, abort_flag)) break;
         if (!mbar_wait(bar_pfull, j & 1, abort_flag)) break;
         tc_fence_after();
-        issue_pv(s, j == 0);
-        tc_commit(bar_pvdone);
+        issue_pv(s, j % NSB, j == 0);
+        tc_commit(bar_pvdone(j % NSB));
         tc_commit(bar_vempty(s));
+        if (NSB == 1 && tn >= 0 && !try_qk(j + 1)) break;
         ++j;
         t = tn;
       }
@@ -492,9 +528,15 @@ __global__ void __launch_bounds__(NTHREADS, D == 64 ? 2 : 1) fwd_tc_kernel(const
     }
     __syncwarp();
   } else {
-    // ------------------------------------------------------------------ softmax warpgroup
+    // ------------------------------------------------------------------ softmax warpgroups
+    constexpr int NG = kGroups<D>;            // column groups: each row has one thread per group
+    constexpr int CPG = (BN / 32) / NG;       // 32-column chunks of S (and of P) per group
+    constexpr int OCG = D / NG;               // O columns per group
+    const int g = (warp - 2) >> 2;            // this thread's column group
     const int q4 = warp & 3;                  // TMEM lane quarter this warp may access
     const int r = q4 * 32 + lane;             // query row within the tile
+    float* const xmax = reinterpret_cast<float*>(sbase + L::kXch);          // [2][NG][BM]
+    float* const xsum = xmax + 2 * NG * BM;                                  // [2][NG][BM]
     const long long qi = q0 + r;              // row in the view
     const long long i = MODE == kResidue ? qi * prm.pi + res : qi;  // row in the sequence
     const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
@@ -502,9 +544,9 @@ __global__ void __launch_bounds__(NTHREADS, D == 64 ? 2 : 1) fwd_tc_kernel(const
     // gate on the unscaled query row.  w_g[h] is staged in shared memory with vector loads while
     // the Q tile is still in flight; the staging area is the start of the P buffer, which is
     // not written before both named barriers below have passed.
-    float* const wg_s = reinterpret_cast<float*>(sbase + L::kP);
+    float* const wg_s = reinterpret_cast<float*>(sbase + L::kWg);
     if (threadIdx.x - 64 < D) wg_s[threadIdx.x - 64] = prm.w_g[(long long)h * D + (threadIdx.x - 64)];
-    asm volatile("bar.sync 1, 128;" ::: "memory");
+    asm volatile("bar.sync 1, %0;" ::"n"(128 * NG) : "memory");
     bool ok = __all_sync(0xffffffffu, mbar_wait(bar_q, 0, abort_flag));
     float z = prm.b_g[h];
     {
@@ -529,7 +571,7 @@ __global__ void __launch_bounds__(NTHREADS, D == 64 ? 2 : 1) fwd_tc_kernel(const
       }
       z += (zp[0] + zp[1]) + (zp[2] + zp[3]);
     }
-    asm volatile("bar.sync 1, 128;" ::: "memory");  // every thread has read w_g: P may be written
+
     // the prior of the keys this pass unmasks as "window" columns
     const float bias_l = log_sigmoid_fast(MODE == kResidue ? -z : z) * kLog2e;  // log2(alpha), or log2(1-alpha)
     const float bias_p = log_sigmoid_fast(-z) * kLog2e;                         // log2(1 - alpha)
@@ -563,15 +605,25 @@ __global__ void __launch_bounds__(NTHREADS, D == 64 ? 2 : 1) fwd_tc_kernel(const
       // spread of the row.  Probabilities only need a reference at or above their max.
       float mt;
       {
-        float x[BN];
-        tmem_ld128(tSb, x);
+        constexpr int CW = BN / NG;  // columns of this group
+        float x[CW];
+        if (NG == 1) tmem_ld128(tSb, x);
+        else tmem_ld64(tSb + g * CW, x);
         float mx[8];
 #pragma unroll
         for (int e = 0; e < 8; ++e) mx[e] = x[e];
 #pragma unroll
-        for (int c = 8; c < BN; ++c) mx[c & 7] = fmaxf(mx[c & 7], x[c]);
-        const float mraw =
+        for (int c = 8; c < CW; ++c) mx[c & 7] = fmaxf(mx[c & 7], x[c]);
+        float mraw =
             fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])), fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
+        if (NG > 1) {  // the row's other half, through shared memory (double-buffered by tile parity)
+          float* const xm = xmax + (j & 1) * NG * BM;
+          xm[g * BM + r] = mraw;
+          mbar_arrive(bar_xm);
+          if (!__all_sync(0xffffffffu, mbar_wait(bar_xm, j & 1, abort_flag))) { ok = false; break; }
+#pragma unroll
+          for (int o = 0; o < NG; ++o) mraw = fmaxf(mraw, xm[o * BM + r]);
+        }
         const float top = has_win ? (has_skip ? fmaxf(bias_l, bias_p) : bias_l) : bias_p;
         mt = (has_win || has_skip) ? fmaf(mraw, prm.scale_log2, top) : NEG_INF;
       }
@@ -581,36 +633,44 @@ __global__ void __launch_bounds__(NTHREADS, D == 64 ? 2 : 1) fwd_tc_kernel(const
       bool rescale = false;
       if (mt > m_ref + kRescaleThreshold || (m_ref == NEG_INF && mt != NEG_INF)) {
         factor = ex2(m_ref - mt);  // 0 when m_ref = -inf
-        rescale = l_sum > 0.f;
+        rescale = m_ref != NEG_INF;  // O holds earlier tiles' sums (decided alike in every group)
         l_sum *= factor;
         l_rnd *= factor;
         m_ref = mt;
       }
       const float m_use = m_ref == NEG_INF ? 0.f : m_ref;
 
-      // The P buffer and O are free once the previous P.V has completed.
-      if (j > 0) {
-        if (!__all_sync(0xffffffffu, mbar_wait(bar_pvdone, (j - 1) & 1, abort_flag))) { ok = false; break; }
+      // P.V of tile j - NSB used this S buffer; observing its barrier phase keeps every later wait
+      // on that barrier unambiguous (its P was read before this tile's Q.K^T wrote the buffer).
+      if (j >= NSB && !__all_sync(0xffffffffu, mbar_wait(bar_pvdone(sb), (j / NSB - 1) & 1, abort_flag))) {
+        ok = false;
+        break;
+      }
+      if (__any_sync(0xffffffffu, rescale)) {
+        // O must hold every earlier tile's P.V before it is rescaled: wait for the P.V of tile j - 1
+        if (NSB == 2 && j >= 1 &&
+            !__all_sync(0xffffffffu, mbar_wait(bar_pvdone((j - 1) % NSB), ((j - 1) / NSB) & 1, abort_flag))) {
+          ok = false;
+          break;
+        }
         tc_fence_after();
         // the rescale is per row, but TMEM access is per warp: the warp rescales when any of its
         // rows needs it, the others multiply by 1
-        if (__any_sync(0xffffffffu, rescale)) {
-          const float f = rescale ? factor : 1.f;
+        const float f = rescale ? factor : 1.f;
 #pragma unroll 1
-          for (int c = 0; c < D / 32; ++c) {
-            float o[32];
-            tmem_ld32(tO + lane_off + c * 32, o);
+        for (int c = g * (OCG / 32); c < (g + 1) * (OCG / 32); ++c) {
+          float o[32];
+          tmem_ld32(tO + lane_off + c * 32, o);
 #pragma unroll
-            for (int e = 0; e < 32; ++e) o[e] *= f;
-            tmem_st32(tO + lane_off + c * 32, o);
-          }
-          tmem_wait_st();
+          for (int e = 0; e < 32; ++e) o[e] *= f;
+          tmem_st32(tO + lane_off + c * 32, o);
         }
+        tmem_wait_st();
       }
 
       // Pass 2, one 32-column chunk at a time (a rolled loop, re-reading the chunk from TMEM):
-      // probabilities against the reference, P (bf16) into shared memory (K-major, 128-byte
-      // swizzle: 16-byte chunk cc of row r at cc ^ (r & 7)), and two row sums -- of the fp32
+      // probabilities against the reference, P (bf16, two per column) back into TMEM, and two
+      // row sums -- of the fp32
       // probabilities (for lse) and of their bf16 roundings (the weights P.V actually applies; the
       // output is normalised by this one, so a row of one key reproduces that key's value).
       //   no key in the chunk -> zeros; window keys only -> one FMA per logit; one skip key and
@@ -618,7 +678,7 @@ __global__ void __launch_bounds__(NTHREADS, D == 64 ? 2 : 1) fwd_tc_kernel(const
       const float bl_m = bias_l - m_use, bp_m = bias_p - m_use;
       float ls = 0.f, lr = 0.f;
 #pragma unroll 1
-      for (int cb = 0; cb < BN / 32; ++cb) {
+      for (int cb = g * CPG; cb < (g + 1) * CPG; ++cb) {
         const int c0 = cb * 32;
         float x[32];
         tmem_ld32(tSb + c0, x);
@@ -682,30 +742,37 @@ __global__ void __launch_bounds__(NTHREADS, D == 64 ? 2 : 1) fwd_tc_kernel(const
           ls += a0 + a1;
           lr += r0 + r1;
         }
-#pragma unroll
-        for (int g = 0; g < 4; ++g) {  // 16-byte chunks 4 cb + g of the row
-          const int c = cb * 4 + g;
-          const int blk = c >> 3, cc = c & 7;
-          *reinterpret_cast<uint4*>(sbase + L::kP + blk * (BM * 128) + r * 128 + ((cc ^ (r & 7)) << 4)) =
-              make_uint4(pk[g * 4 + 0], pk[g * 4 + 1], pk[g * 4 + 2], pk[g * 4 + 3]);
-        }
+        __syncwarp();  // rows may have taken different branches; tcgen05.st is .sync.aligned
+        tmem_st16(tSb + pcol(cb), pk);  // over S columns this group has already read
       }
       l_sum += ls;
       l_rnd += lr;
+      tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(bar_sfree(sb));  // the S buffer may take the Q.K^T of tile j + NSB
-      fence_proxy_async_smem();
-      tc_fence_before();
+      mbar_arrive(bar_sfree(sb));  // the buffer may take the Q.K^T of tile j + NSB (issued after this P.V)
       mbar_arrive(bar_pfull);
     }
-    // ---- epilogue: the normalised row goes to shared memory (the P buffer, free once the last
-    // P.V has completed) in the 128-byte-swizzled tile layout, then one TMA store writes the tile
+    // ---- epilogue: the normalised row goes to shared memory (V stage 0, free once the last P.V
+    // has completed) in the 128-byte-swizzled tile layout, then one TMA store writes the tile
     // (rows past the end of the view are clipped by the tensor map).  kBandMerge first brings the
     // tile of skip partials in by TMA (into the free K stage 0) and merges them row by row.
     const bool row_ok = qi < view_rows;
     const long long orow = (long long)bh * prm.n + i;  // row in [B*H, n] layouts
-    const bool have_o = __all_sync(0xffffffffu, ok && j > 0 && mbar_wait(bar_pvdone, (j - 1) & 1, abort_flag));
+    const bool have_o = __all_sync(
+        0xffffffffu, ok && j > 0 && mbar_wait(bar_pvdone((j - 1) % NSB), ((j - 1) / NSB) & 1, abort_flag));
     const bool no_keys = MODE == kResidue && __all_sync(0xffffffffu, ok && j == 0);  // tile with no skip at all
+    if (NG > 1) {  // whole-row sums from the groups' partial sums (every softmax thread passes here)
+      xsum[g * BM + r] = l_sum;
+      xsum[NG * BM + g * BM + r] = l_rnd;
+      asm volatile("bar.sync 2, %0;" ::"n"(128 * NG) : "memory");
+      l_sum = 0.f;
+      l_rnd = 0.f;
+#pragma unroll
+      for (int o = 0; o < NG; ++o) {
+        l_sum += xsum[o * BM + r];
+        l_rnd += xsum[NG * BM + o * BM + r];
+      }
+    }
     float lse_log2 = 0.f;
     if (have_o || no_keys) {
       if (have_o) tc_fence_after();
@@ -731,16 +798,17 @@ __global__ void __launch_bounds__(NTHREADS, D == 64 ? 2 : 1) fwd_tc_kernel(const
         wp /= den;
         lse2 = M + log2f(den);
       }
-      float o[D];
+      float o[OCG];  // this group's columns of the O row, one load
       if (have_o) {
-        if (D == 128) tmem_ld128(tO + lane_off, o);
-        else tmem_ld64(tO + lane_off, o);
+        if (OCG == 128) tmem_ld128(tO + lane_off, o);
+        else tmem_ld64(tO + lane_off + g * OCG, o);
       } else {
 #pragma unroll
-        for (int e = 0; e < D; ++e) o[e] = 0.f;
+        for (int e = 0; e < OCG; ++e) o[e] = 0.f;
       }
 #pragma unroll
-      for (int c = 0; c < D / 8; ++c) {  // 16-byte chunk c of the row
+      for (int cl = 0; cl < OCG / 8; ++cl) {  // 16-byte chunk c of the row
+        const int c = g * (OCG / 8) + cl;
         const int blk = c >> 3, cc = c & 7;
         const uint32_t off = blk * (BM * 128) + r * 128 + ((cc ^ (r & 7)) << 4);
         float sp[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
@@ -748,31 +816,31 @@ __global__ void __launch_bounds__(NTHREADS, D == 64 ? 2 : 1) fwd_tc_kernel(const
         uint32_t w[4];
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-          const float a0 = o[c * 8 + 2 * e] * inv * wl + sp[2 * e] * wp;
-          const float a1 = o[c * 8 + 2 * e + 1] * inv * wl + sp[2 * e + 1] * wp;
+          const float a0 = o[cl * 8 + 2 * e] * inv * wl + sp[2 * e] * wp;
+          const float a1 = o[cl * 8 + 2 * e + 1] * inv * wl + sp[2 * e + 1] * wp;
           __nv_bfloat162 b2 = __floats2bfloat162_rn(a0, a1);
           w[e] = *reinterpret_cast<uint32_t*>(&b2);
         }
-        *reinterpret_cast<uint4*>(sbase + L::kP + off) = make_uint4(w[0], w[1], w[2], w[3]);
+        *reinterpret_cast<uint4*>(sbase + L::kV + off) = make_uint4(w[0], w[1], w[2], w[3]);
       }
       lse_log2 = lse2;
       fence_proxy_async_smem();
     }
     // Every softmax warp passes this barrier, epilogue or not (a warp that gave up on a wait must
     // not leave the others blocked here); the tile is then staged whenever it is stored.
-    asm volatile("bar.sync 1, 128;" ::: "memory");
+    asm volatile("bar.sync 1, %0;" ::"n"(128 * NG) : "memory");
     if (have_o || no_keys) {
       if (threadIdx.x == 64) {
 #pragma unroll
         for (int c = 0; c < D / 64; ++c) {
           if (MODE == kResidue)
-            tma_store_4d(&tmo, sP + c * BM * 128, c * 64, res, (int)q0, bh);
+            tma_store_4d(&tmo, sV + c * BM * 128, c * 64, res, (int)q0, bh);
           else
-            tma_store_3d(&tmo, sP + c * BM * 128, c * 64, (int)q0, bh);
+            tma_store_3d(&tmo, sV + c * BM * 128, c * 64, (int)q0, bh);
         }
         tma_store_commit_and_wait_read();  // shared memory must outlive the reads of the store
       }
-      if (row_ok) {
+      if (row_ok && g == 0) {
         // a row with no key in this pass (only possible for kResidue) has lse -inf
         const float lse2 = lse_log2;
         const float lse_val = l_sum > 0.f ? lse2 * kLn2 : NEG_INF;
@@ -897,7 +965,7 @@ cudaError_t launch_fwd_tc_d(const void* q, const void* k, const void* v, const f
   }
   if (!split) {
     if ((e = tc::set_smem_attr<D, tc::kFused>()) != cudaSuccess) { *why = "cudaFuncSetAttribute"; return e; }
-    tc::fwd_tc_kernel<D, tc::kFused><<<grid, tc::NTHREADS, L::kAlloc, st>>>(mq, mk, mv, mo, mo, p);
+    tc::fwd_tc_kernel<D, tc::kFused><<<grid, tc::kThreads<D>, L::kAlloc, st>>>(mq, mk, mv, mo, mo, p);
     *why = "tensor-core kernel launch";
     return cudaGetLastError();
   }
@@ -925,10 +993,10 @@ cudaError_t launch_fwd_tc_d(const void* q, const void* k, const void* v, const f
     return cudaErrorInvalidValue;
   }
   const dim3 grid_r((unsigned)(pi * ((p.T + tc::BM - 1) / tc::BM)), (unsigned)BH);
-  tc::fwd_tc_kernel<D, tc::kResidue><<<grid_r, tc::NTHREADS, L::kAlloc, st>>>(rq, rk, rv, rso, rso, p);
+  tc::fwd_tc_kernel<D, tc::kResidue><<<grid_r, tc::kThreads<D>, L::kAlloc, st>>>(rq, rk, rv, rso, rso, p);
   e = cudaGetLastError();
   if (e == cudaSuccess) {
-    tc::fwd_tc_kernel<D, tc::kBandMerge><<<grid, tc::NTHREADS, L::kAlloc, st>>>(mq, mk, mv, mo, mso, p);
+    tc::fwd_tc_kernel<D, tc::kBandMerge><<<grid, tc::kThreads<D>, L::kAlloc, st>>>(mq, mk, mv, mo, mso, p);
     e = cudaGetLastError();
   }
   cudaError_t e2 = cudaFreeAsync(scratch, st);
