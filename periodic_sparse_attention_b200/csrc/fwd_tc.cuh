@@ -36,10 +36,15 @@ namespace tc {
 
 constexpr int BM = 128;       // query rows per CTA
 constexpr int BN = kTileKeys; // keys per tile
-constexpr int NSTAGE = 2;     // K/V ring depth
-// Softmax warpgroups per CTA: d = 128 runs one CTA per SM, and two warpgroups split each S row
-// by columns (a second warp per scheduler hides latency); d = 64 runs two CTAs per SM with one.
-template <int D> constexpr int kGroups = D == 128 ? 2 : 1;
+// Pipeline shape.  Both head sizes run two CTAs per SM, so that one CTA's prologue (TMEM
+// allocation, Q load, gate) and epilogue overlap the other's tiles: 256 TMEM columns per CTA
+// (one S buffer of 128 columns, P written over it, and O), one softmax warpgroup.  The K/V ring
+// has two stages at d = 64 and one at d = 128 (three 32 KB tiles per CTA); with one S buffer the
+// next tile's K and V loads still have a whole softmax pass to land.
+template <int D> constexpr int kStages = D == 128 ? 1 : 2;  // K/V ring depth
+template <int D> constexpr int kGroups = 1;                 // softmax warpgroups (split S rows by columns)
+template <int D> constexpr int kSBufsT = 1;                 // S buffers in TMEM
+template <int D> constexpr int kCtasPerSm = 2;
 // warp 0 TMA, warp 1 MMA, warps 2 .. 2 + 4 * groups - 1 softmax
 template <int D> constexpr int kThreads = 64 + 128 * kGroups<D>;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
@@ -47,15 +52,15 @@ constexpr float kRescaleThreshold = 8.0f;  // log2 units
 // ---- shared memory plan (offsets from a 1024-byte aligned base) ---------------------------------
 template <int D>
 struct Smem {
+  static constexpr int NSTAGE = kStages<D>;
   static constexpr int kTileBytes = BM * D * 2;          // one 128-row bf16 tile
   static constexpr int kQ = 0;
   static constexpr int kK = kQ + kTileBytes;
   static constexpr int kV = kK + NSTAGE * kTileBytes;
   static constexpr int kBar = kV + NSTAGE * kTileBytes;  // (P lives in TMEM, over its S columns)
-  // S buffers in TMEM: two for d = 128 (one CTA per SM: the next tile's Q.K^T overlaps this
-  // tile's softmax), one for d = 64 (two CTAs per SM overlap each other instead)
-  static constexpr int kSBufs = D == 128 ? 2 : 1;
-  static constexpr int kTmemCols = kSBufs == 2 ? 512 : 256;  // S buffers (128 each) + O (D)
+  static constexpr int kSBufs = kSBufsT<D>;
+  static constexpr int kTmemCols = 128 * kSBufs + D <= 256 ? 256 : 512;  // S buffers (128 each) + O (D)
+  static_assert(kTmemCols * kCtasPerSm<D> <= 512, "TMEM columns of the CTAs on one SM");
   // barriers: q_full, k_full[2], k_empty[2], v_full[2], v_empty[2], s_full[NSB], s_free[NSB],
   // pv_done[NSB], p_full, drain, skip partials, (two groups) max exchange
   static constexpr int kNumBars = 1 + 4 * NSTAGE + 3 * kSBufs + 3 + (kGroups<D> > 1 ? 1 : 0);
@@ -66,8 +71,8 @@ struct Smem {
   static constexpr int kWg = kXch + kXchBytes;          // w_g[h] staging, D floats
   static constexpr int kTotal = kWg + D * 4;
   static constexpr int kAlloc = kTotal + 1024 - 128;     // slack to align a (>= 128 B aligned) base to 1 KB
-  // d = 64 runs two CTAs per SM: 228 KB of shared memory per SM, 1 KB of it reserved per CTA
-  static_assert(D != 64 || kAlloc <= 228 * 1024 / 2 - 1024, "d = 64 plan must fit two CTAs per SM");
+  // 228 KB of shared memory per SM, 1 KB of it reserved per CTA
+  static_assert(kAlloc <= 228 * 1024 / kCtasPerSm<D> - 1024, "shared memory of the CTAs on one SM");
 };
 
 // ---- PTX wrappers ------------------------------------------------------------------------------
@@ -328,7 +333,7 @@ struct Params {
 };
 
 template <int D, int MODE>
-__global__ void __launch_bounds__(kThreads<D>, D == 64 ? 2 : 1) fwd_tc_kernel(const __grid_constant__ CUtensorMap tmq,
+__global__ void __launch_bounds__(kThreads<D>, kCtasPerSm<D>) fwd_tc_kernel(const __grid_constant__ CUtensorMap tmq,
                                                                           const __grid_constant__ CUtensorMap tmk,
                                                                           const __grid_constant__ CUtensorMap tmv,
                                                                           const __grid_constant__ CUtensorMap tmo,
@@ -375,6 +380,7 @@ __global__ void __launch_bounds__(kThreads<D>, D == 64 ? 2 : 1) fwd_tc_kernel(co
   // handled by the softmax group cb / CPG, which reads its S chunks in order before writing them.
   constexpr int CPG_K = (BN / 32) / kGroups<D>;
   auto pcol = [](int cb) { return 64 * (cb / CPG_K) + 16 * (cb % CPG_K); };
+  constexpr int NSTAGE = L::NSTAGE;
   const uint32_t bar0 = base + L::kBar;
   const uint32_t bar_q = bar0;
   auto bar_kfull = [&](int s) { return bar0 + 8u * (1 + s); };
