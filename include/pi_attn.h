@@ -21,7 +21,8 @@
  *     (bfloat16).  Arithmetic is fp32 (bf16 products on tensor cores accumulate in fp32); out is
  *     rounded once, to nearest even, into dtype.
  *   - All pointers are DEVICE pointers owned by the caller; the library keeps no reference after
- *     the call returns and holds no allocation of its own between calls.  Tensor pointers must be
+ *     the call returns and holds no allocation of its own between calls (the decode entry point
+ *     for callers that cannot allocate uses a fixed array inside the library, see below).  Tensor pointers must be
  *     16-byte aligned and d * sizeof(dtype) a multiple of 16 bytes.
  *   - `stream` is a cudaStream_t (NULL: the legacy default stream).  Calls only enqueue work: they
  *     are asynchronous and stream-ordered.  Argument errors are returned synchronously and then
@@ -76,9 +77,23 @@ pi_attn_status pi_attn_fwd_ex(const void* q, const void* k, const void* v, const
                               void* out, float* lse, int B, int H, int n, int d, int k_win, int pi, int S,
                               pi_attn_dtype dtype, pi_attn_path path, void* stream);
 
+/* pi_attn_fwd_ex with a caller-provided device workspace for the split path's skip partials, so
+ * that the call allocates nothing (and can be captured in a CUDA graph without memory nodes).
+ *   workspace        device pointer, 16-byte aligned, owned by the caller; NULL = allocate as
+ *                    pi_attn_fwd_ex does (cudaMallocAsync on `stream`, freed stream-ordered)
+ *   workspace_bytes  its size; at least the scratch_bytes pi_attn_fwd_plan reports for the same
+ *                    arguments (0 when the call runs a single pass), else PI_ATTN_EINVAL
+ * The workspace is read and written by the call's kernels only: it may be reused by the next call
+ * on the same stream, and must not be touched by other streams while the call runs. */
+pi_attn_status pi_attn_fwd_ws(const void* q, const void* k, const void* v, const float* w_g, const float* b_g,
+                              void* out, float* lse, int B, int H, int n, int d, int k_win, int pi, int S,
+                              pi_attn_dtype dtype, pi_attn_path path, void* workspace, long long workspace_bytes,
+                              void* stream);
+
 /* What a pi_attn_fwd_ex call with these arguments would launch, without launching anything:
  * *launches = number of kernel launches (1 for a single pass, 2 for the split), *scratch_bytes =
- * device scratch it takes from cudaMallocAsync on the stream (0 for a single pass).  Returns
+ * device scratch it needs (0 for a single pass): taken from cudaMallocAsync on the stream, or the
+ * workspace given to pi_attn_fwd_ws.  Returns
  * PI_ATTN_EUNSUPPORTED / PI_ATTN_EINVAL exactly where pi_attn_fwd_ex would. */
 pi_attn_status pi_attn_fwd_plan(int B, int H, int n, int d, int k_win, int pi, int S, pi_attn_dtype dtype,
                                 pi_attn_path path, int* launches, long long* scratch_bytes);

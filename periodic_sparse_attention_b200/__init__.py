@@ -27,6 +27,8 @@ SIGNATURES = {
     "pi_attn_fwd": (_i32, [_vp] * 7 + [_i32] * 8 + [_vp]),
     # ... as above plus the path selector
     "pi_attn_fwd_ex": (_i32, [_vp] * 7 + [_i32] * 9 + [_vp]),
+    # ... plus workspace pointer and its size in bytes
+    "pi_attn_fwd_ws": (_i32, [_vp] * 7 + [_i32] * 9 + [_vp, ctypes.c_longlong, _vp]),
     # B H n d k_win pi S, dtype, path, out: launches, scratch bytes
     "pi_attn_fwd_plan": (_i32, [_i32] * 9 + [_vp, _vp]),
     # 8 pointers (q kcache vcache w_g b_g cache_len out lse), B H n_cache d k_win pi S, dtype, stream
@@ -101,18 +103,32 @@ def _ptr(t):
     return ctypes.c_void_p(t.data_ptr())
 
 
+_plans = {}
+
+
 def pi_attn_fwd(q, k, v, w_g, b_g, k_win: int, pi: int, S: int, out=None, lse=None, *, path: str = "auto",
-                stream=None, want_lse: bool = True):
+                stream=None, want_lse: bool = True, workspace=None):
     """Prefill forward on torch CUDA tensors q, k, v [B, H, n, d] (fp32 or bf16), w_g [H, d] and
-    b_g [H] (fp32).  Allocates out (q's dtype) and lse (fp32 [B, H, n]) when not given."""
+    b_g [H] (fp32).  Allocates out (q's dtype) and lse (fp32 [B, H, n]) when not given, and the
+    split path's workspace (a uint8 tensor of pi_attn_fwd_plan's scratch bytes) from torch's
+    caching allocator when not given."""
     import torch
     B, H, n, d = q.shape
     if out is None:
         out = torch.empty_like(q)
     if lse is None and want_lse:
         lse = torch.empty((B, H, n), dtype=torch.float32, device=q.device)
-    st = load().pi_attn_fwd_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(w_g), _ptr(b_g), _ptr(out), _ptr(lse), B, H, n, d,
-                               k_win, pi, S, _dtype_code(q), PATHS[path], _stream(stream))
+    dt = _dtype_code(q)
+    key = (B, H, n, d, k_win, pi, S, dt, path)
+    scratch = _plans.get(key)
+    if scratch is None:
+        scratch = pi_attn_fwd_plan(B, H, n, d, k_win, pi, S, "bf16" if dt == PI_ATTN_BF16 else "f32", path)[1]
+        _plans[key] = scratch
+    if workspace is None and scratch > 0:
+        workspace = torch.empty(scratch, dtype=torch.uint8, device=q.device)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    st = load().pi_attn_fwd_ws(_ptr(q), _ptr(k), _ptr(v), _ptr(w_g), _ptr(b_g), _ptr(out), _ptr(lse), B, H, n, d,
+                               k_win, pi, S, dt, PATHS[path], _ptr(workspace), ws_bytes, _stream(stream))
     _raise(st)
     return out, lse
 

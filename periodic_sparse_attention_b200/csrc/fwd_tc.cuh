@@ -48,6 +48,9 @@ template <int D> constexpr int kCtasPerSm = 2;
 // warp 0 TMA, warp 1 MMA, warps 2 .. 2 + 4 * groups - 1 softmax
 template <int D> constexpr int kThreads = 64 + 128 * kGroups<D>;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
+// Pairs of a 32-column window-only chunk whose exponentials run on the FMA pipe (bit e: columns
+// 2e, 2e + 1); the rest use the special-function unit.
+constexpr uint32_t kPolyPairs = 0x4924u;  // every third pair
 
 // ---- shared memory plan (offsets from a 1024-byte aligned base) ---------------------------------
 template <int D>
@@ -291,6 +294,40 @@ __device__ __forceinline__ float ex2(float x) {
   return y;
 }
 
+// 2^x for a pair on the FMA pipe, to take part of the softmax's exponentials off the special-
+// function unit (which runs a quarter of a warp per cycle).  Range reduction after Cody and
+// Waite: n = rint(x) from the low mantissa bits of x + 1.5 * 2^23, f = x - n in [-1/2, 1/2];
+// 2^f from a degree-3 polynomial, minimax in relative error and rounded to fp32 (coefficients
+// from csrc/exp2_poly.py; |relative error| < 7.5e-5, far below the bf16 rounding of P); 2^n is
+// added into the exponent field.  x is clamped at -125 so that the result stays a normal float:
+// anything below 2^-125 comes out as 2^-125, which next to the row's reference (within 2^8 of
+// its maximum) weighs nothing in fp32.
+__device__ __forceinline__ void ex2_poly2(float x0, float x1, float& y0, float& y1) {
+  const unsigned long long kRound = f2pack(12582912.f, 12582912.f);  // 1.5 * 2^23
+  const unsigned long long kNegRound = f2pack(-12582912.f, -12582912.f);
+  const unsigned long long kOne = f2pack(1.f, 1.f), kNegOne = f2pack(-1.f, -1.f);
+  const unsigned long long x = f2pack(fmaxf(x0, -125.f), fmaxf(x1, -125.f));
+  const unsigned long long t = f2add(x, kRound);        // n in the low bits
+  const unsigned long long nf = f2fma(t, kOne, kNegRound);  // n, exactly
+  const unsigned long long f = f2fma(nf, kNegOne, x);    // x - n, exactly
+  unsigned long long q = f2fma(f, f2pack(5.517166853e-02f, 5.517166853e-02f), f2pack(2.426111251e-01f, 2.426111251e-01f));
+  q = f2fma(q, f, f2pack(6.932609677e-01f, 6.932609677e-01f));
+  q = f2fma(q, f, f2pack(9.999280572e-01f, 9.999280572e-01f));
+  float q0, q1, t0, t1;
+  f2unpack(q, q0, q1);
+  f2unpack(t, t0, t1);
+  // bits(t) = bits(1.5 * 2^23) + n, and bits(1.5 * 2^23) << 23 vanishes modulo 2^32
+  y0 = __int_as_float(__float_as_int(q0) + (__float_as_int(t0) << 23));
+  y1 = __int_as_float(__float_as_int(q1) + (__float_as_int(t1) << 23));
+}
+
+// max of three (one instruction on sm_100)
+__device__ __forceinline__ float max3f(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
 // ---- UMMA descriptors ----------------------------------------------------------------------------
 // Shared-memory matrix descriptor (sm_100): start address >> 4 in bits [0,14), leading byte
 // offset >> 4 in [16,30), stride byte offset >> 4 in [32,46), version 1 in [46,48), layout type
@@ -459,9 +496,22 @@ __global__ void __launch_bounds__(kThreads<D>, kCtasPerSm<D>) fwd_tc_kernel(cons
         load_tile(sV + s * kTile, &tmv, bar_vfull(s), (long long)t * BN);
         ++nv;
       }
+      // kBandMerge: the tile of skip partials goes into K stage 0 as soon as the last Q.K^T that
+      // reads that stage has completed, so its load overlaps the last tile's softmax and P.V
+      bool so_issued = false;
+      if (MODE == kBandMerge && !*abort_flag) {
+        const int u0 = nk > 0 ? (nk - 1) / NSTAGE * NSTAGE : -1;  // last load into K stage 0
+        if (u0 < 0 || mbar_wait(bar_kempty(0), (u0 / NSTAGE) & 1, abort_flag)) {
+          mbar_expect_tx(bar_so, kTile);
+#pragma unroll
+          for (int c = 0; c < D / 64; ++c) tma_load_3d(sK + c * BM * 128, &tms, bar_so, c * 64, (int)q0, bh);
+          so_issued = true;
+        }
+      }
       if (*abort_flag) {  // let the loads already in flight land before the CTA can exit
         volatile int never = 0;
         mbar_wait(bar_q, 0, &never);
+        if (so_issued) mbar_wait(bar_so, 0, &never);
         for (int u = nk > NSTAGE ? nk - NSTAGE : 0; u < nk; ++u)
           mbar_wait(bar_kfull(u % NSTAGE), (u / NSTAGE) & 1, &never);
         for (int u = nv > NSTAGE ? nv - NSTAGE : 0; u < nv; ++u)
@@ -546,10 +596,13 @@ __global__ void __launch_bounds__(kThreads<D>, kCtasPerSm<D>) fwd_tc_kernel(cons
     const long long qi = q0 + r;              // row in the view
     const long long i = MODE == kResidue ? qi * prm.pi + res : qi;  // row in the sequence
     const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
+    // kBandMerge: this row's skip-partial lse (written by the residue pass), loaded now so that
+    // the epilogue does not wait for it
+    const float skip_lse_row =
+        MODE == kBandMerge && qi < view_rows ? prm.skip_lse[(long long)bh * prm.n + i] : 0.f;
 
-    // gate on the unscaled query row.  w_g[h] is staged in shared memory with vector loads while
-    // the Q tile is still in flight; the staging area is the start of the P buffer, which is
-    // not written before both named barriers below have passed.
+    // gate on the unscaled query row.  w_g[h] is staged in shared memory while the Q tile is
+    // still in flight.
     float* const wg_s = reinterpret_cast<float*>(sbase + L::kWg);
     if (threadIdx.x - 64 < D) wg_s[threadIdx.x - 64] = prm.w_g[(long long)h * D + (threadIdx.x - 64)];
     asm volatile("bar.sync 1, %0;" ::"n"(128 * NG) : "memory");
@@ -718,7 +771,9 @@ __global__ void __launch_bounds__(kThreads<D>, kCtasPerSm<D>) fwd_tc_kernel(cons
             for (int e = 0; e < 32; e += 2) {
               float t0, t1;
               f2unpack(f2fma(f2pack(x[e], x[e + 1]), sc2, bb), t0, t1);
-              const float p0 = ex2(t0), p1 = ex2(t1);
+              float p0, p1;
+              if ((kPolyPairs >> (e >> 1)) & 1u) ex2_poly2(t0, t1, p0, p1);
+              else p0 = ex2(t0), p1 = ex2(t1);
               __nv_bfloat162 b2 = __floats2bfloat162_rn(p0, p1);
               const uint32_t u = *reinterpret_cast<uint32_t*>(&b2);
               pk[e >> 1] = u;
@@ -782,20 +837,12 @@ __global__ void __launch_bounds__(kThreads<D>, kCtasPerSm<D>) fwd_tc_kernel(cons
     float lse_log2 = 0.f;
     if (have_o || no_keys) {
       if (have_o) tc_fence_after();
-      constexpr uint32_t kTile = L::kTileBytes;
       bool so_ok = true;
-      if (MODE == kBandMerge) {
-        if (threadIdx.x == 64) {
-          mbar_expect_tx(bar_so, kTile);
-#pragma unroll
-          for (int c = 0; c < D / 64; ++c) tma_load_3d(sK + c * BM * 128, &tms, bar_so, c * 64, (int)q0, bh);
-        }
-        so_ok = __all_sync(0xffffffffu, mbar_wait(bar_so, 0, abort_flag));
-      }
+      if (MODE == kBandMerge) so_ok = __all_sync(0xffffffffu, mbar_wait(bar_so, 0, abort_flag));
       float inv = l_rnd > 0.f ? 1.f / l_rnd : 0.f;
       float wl = 1.f, wp = 0.f, lse2 = m_ref + log2f(l_sum);  // log2 of this pass's mass
       if (MODE == kBandMerge && row_ok) {
-        const float b2 = prm.skip_lse[orow] * kLog2e;
+        const float b2 = skip_lse_row * kLog2e;
         const float M = fmaxf(lse2, b2);
         wl = ex2(lse2 - M);
         wp = ex2(b2 - M);
@@ -940,7 +987,7 @@ inline bool tc_split_preferred(int n, int kwin, int pi, int S) {
 template <int D>
 cudaError_t launch_fwd_tc_d(const void* q, const void* k, const void* v, const float* w_g, const float* b_g,
                             void* out, float* lse, int B, int H, int n, int kwin, int pi, int S, bool split,
-                            cudaStream_t st, const char** why) {
+                            void* workspace, cudaStream_t st, const char** why) {
   using L = tc::Smem<D>;
   CUtensorMap mq, mk, mv;
   const int BH = B * H;
@@ -983,10 +1030,12 @@ cudaError_t launch_fwd_tc_d(const void* q, const void* k, const void* v, const f
   }
   if ((e = tc::set_smem_attr<D, tc::kResidue>()) != cudaSuccess) { *why = "cudaFuncSetAttribute"; return e; }
   if ((e = tc::set_smem_attr<D, tc::kBandMerge>()) != cudaSuccess) { *why = "cudaFuncSetAttribute"; return e; }
-  // scratch for the skip partials: [B*H, n, D] bf16 + [B*H, n] fp32, stream-ordered
+  // scratch for the skip partials: [B*H, n, D] bf16 + [B*H, n] fp32 -- the caller's workspace,
+  // else taken from cudaMallocAsync on the stream and given back after the second launch
   const size_t rows = (size_t)BH * n;
-  void* scratch = nullptr;
-  if ((e = cudaMallocAsync(&scratch, rows * (D * 2 + 4), st)) != cudaSuccess) {
+  void* scratch = workspace;
+  const bool own = scratch == nullptr;
+  if (own && (e = cudaMallocAsync(&scratch, rows * (D * 2 + 4), st)) != cudaSuccess) {
     *why = "skip-partial scratch allocation";
     return e;
   }
@@ -994,7 +1043,7 @@ cudaError_t launch_fwd_tc_d(const void* q, const void* k, const void* v, const f
   p.skip_lse = (float*)((char*)scratch + rows * D * 2);
   CUtensorMap rso, mso;  // the skip partials, in the residue view (stored) and the sequence view (loaded)
   if (!tc::make_residue_map(&rso, p.skip_o, BH, n, D, pi) || !tc::make_map(&mso, p.skip_o, BH, n, D)) {
-    cudaFreeAsync(scratch, st);
+    if (own) cudaFreeAsync(scratch, st);
     *why = "cuTensorMapEncodeTiled (skip partials) failed";
     return cudaErrorInvalidValue;
   }
@@ -1005,7 +1054,7 @@ cudaError_t launch_fwd_tc_d(const void* q, const void* k, const void* v, const f
     tc::fwd_tc_kernel<D, tc::kBandMerge><<<grid, tc::kThreads<D>, L::kAlloc, st>>>(mq, mk, mv, mo, mso, p);
     e = cudaGetLastError();
   }
-  cudaError_t e2 = cudaFreeAsync(scratch, st);
+  cudaError_t e2 = own ? cudaFreeAsync(scratch, st) : cudaSuccess;
   *why = "tensor-core split kernels";
   return e != cudaSuccess ? e : e2;
 }
@@ -1013,10 +1062,11 @@ cudaError_t launch_fwd_tc_d(const void* q, const void* k, const void* v, const f
 // mode: 0 = choose, 1 = single pass, 2 = split (residue pass + window pass)
 inline cudaError_t launch_fwd_tc(const void* q, const void* k, const void* v, const float* w_g, const float* b_g,
                                  void* out, float* lse, int B, int H, int n, int d, int kwin, int pi, int S, int mode,
-                                 cudaStream_t st, const char** why) {
+                                 void* workspace, cudaStream_t st, const char** why) {
   const bool split = mode == 2 || (mode == 0 && tc_split_preferred(n, kwin, pi, S));
-  if (d == 128) return launch_fwd_tc_d<128>(q, k, v, w_g, b_g, out, lse, B, H, n, kwin, pi, S, split, st, why);
-  return launch_fwd_tc_d<64>(q, k, v, w_g, b_g, out, lse, B, H, n, kwin, pi, S, split, st, why);
+  if (d == 128)
+    return launch_fwd_tc_d<128>(q, k, v, w_g, b_g, out, lse, B, H, n, kwin, pi, S, split, workspace, st, why);
+  return launch_fwd_tc_d<64>(q, k, v, w_g, b_g, out, lse, B, H, n, kwin, pi, S, split, workspace, st, why);
 }
 
 }  // namespace pia

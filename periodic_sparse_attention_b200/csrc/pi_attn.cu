@@ -130,11 +130,10 @@ const char* pi_attn_last_error(void) { return g_msg; }
 
 int pi_attn_version(void) { return 100; }
 
-pi_attn_status pi_attn_fwd_ex(const void* q, const void* k, const void* v, const float* w_g, const float* b_g,
-                              void* out, float* lse, int B, int H, int n, int d, int k_win, int pi, int S,
-                              pi_attn_dtype dtype, pi_attn_path path, void* stream) {
-  pi_attn_status st = check_common(q, k, v, w_g, b_g, out, B, H, n, d, k_win, pi, S, dtype);
-  if (st != PI_ATTN_OK) return st;
+// Which kernels a forward call with these arguments runs: *tc (tensor-core path) and *split
+// (residue pass + band-merge pass), after the same checks as the call itself.
+static pi_attn_status fwd_route(int n, int d, int k_win, int pi, int S, pi_attn_dtype dtype, pi_attn_path path,
+                                bool* tc, bool* split) {
   if (path < PI_ATTN_PATH_AUTO || path > PI_ATTN_PATH_TC_SPLIT) return fail(PI_ATTN_EINVAL, "unknown path %d", (int)path);
   const bool tc_ok = pia::tc_supported(dtype == PI_ATTN_BF16, d, n);
   const bool want_tc = path == PI_ATTN_PATH_TC || path == PI_ATTN_PATH_TC_FUSED || path == PI_ATTN_PATH_TC_SPLIT;
@@ -143,17 +142,47 @@ pi_attn_status pi_attn_fwd_ex(const void* q, const void* k, const void* v, const
                 (int)dtype, d);
   if (path == PI_ATTN_PATH_TC_SPLIT && !pia::tc_split_applies(n, k_win, pi, S))
     return fail(PI_ATTN_EUNSUPPORTED, "split path needs n %% pi == 0 and at least one skip outside the window");
+  *tc = path != PI_ATTN_PATH_SIMT && tc_ok;
+  *split = *tc && (path == PI_ATTN_PATH_TC_SPLIT ||
+                   (path != PI_ATTN_PATH_TC_FUSED && pia::tc_split_preferred(n, k_win, pi, S)));
+  return ok();
+}
+
+static long long fwd_scratch_bytes(int B, int H, int n, int d, bool split) {
+  return split ? (long long)B * H * n * (2LL * d + 4) : 0;
+}
+
+pi_attn_status pi_attn_fwd_ws(const void* q, const void* k, const void* v, const float* w_g, const float* b_g,
+                              void* out, float* lse, int B, int H, int n, int d, int k_win, int pi, int S,
+                              pi_attn_dtype dtype, pi_attn_path path, void* workspace, long long workspace_bytes,
+                              void* stream) {
+  pi_attn_status st = check_common(q, k, v, w_g, b_g, out, B, H, n, d, k_win, pi, S, dtype);
+  if (st != PI_ATTN_OK) return st;
+  bool tc = false, split = false;
+  if ((st = fwd_route(n, d, k_win, pi, S, dtype, path, &tc, &split)) != PI_ATTN_OK) return st;
+  if (workspace) {
+    if (reinterpret_cast<uintptr_t>(workspace) % 16 != 0) return fail(PI_ATTN_EINVAL, "workspace not 16-byte aligned");
+    const long long need = fwd_scratch_bytes(B, H, n, d, split);
+    if (workspace_bytes < need)
+      return fail(PI_ATTN_EINVAL, "workspace of %lld bytes, this call needs %lld", workspace_bytes, need);
+  }
   cudaStream_t s = as_stream(stream);
-  if (path != PI_ATTN_PATH_SIMT && tc_ok) {
+  if (tc) {
     const char* why = nullptr;
-    const int mode = path == PI_ATTN_PATH_TC_FUSED ? 1 : path == PI_ATTN_PATH_TC_SPLIT ? 2 : 0;
-    cudaError_t e = pia::launch_fwd_tc(q, k, v, w_g, b_g, out, lse, B, H, n, d, k_win, pi, S, mode, s, &why);
+    const int mode = split ? 2 : 1;
+    cudaError_t e = pia::launch_fwd_tc(q, k, v, w_g, b_g, out, lse, B, H, n, d, k_win, pi, S, mode, workspace, s, &why);
     if (e != cudaSuccess) return cuda_fail(e, why ? why : "tensor-core kernel launch");
     return ok();
   }
   if (dtype == PI_ATTN_F32)
     return launch_simt<float, false>(q, k, v, w_g, b_g, nullptr, out, lse, B, H, n, n, d, k_win, pi, S, s);
   return launch_simt<__nv_bfloat16, false>(q, k, v, w_g, b_g, nullptr, out, lse, B, H, n, n, d, k_win, pi, S, s);
+}
+
+pi_attn_status pi_attn_fwd_ex(const void* q, const void* k, const void* v, const float* w_g, const float* b_g,
+                              void* out, float* lse, int B, int H, int n, int d, int k_win, int pi, int S,
+                              pi_attn_dtype dtype, pi_attn_path path, void* stream) {
+  return pi_attn_fwd_ws(q, k, v, w_g, b_g, out, lse, B, H, n, d, k_win, pi, S, dtype, path, nullptr, 0, stream);
 }
 
 pi_attn_status pi_attn_fwd_plan(int B, int H, int n, int d, int k_win, int pi, int S, pi_attn_dtype dtype,
@@ -163,17 +192,10 @@ pi_attn_status pi_attn_fwd_plan(int B, int H, int n, int d, int k_win, int pi, i
   pi_attn_status st = check_common(dummy, dummy, dummy, (const float*)dummy, (const float*)dummy, dummy, B, H, n, d,
                                    k_win, pi, S, dtype);
   if (st != PI_ATTN_OK) return st;
-  if (path < PI_ATTN_PATH_AUTO || path > PI_ATTN_PATH_TC_SPLIT) return fail(PI_ATTN_EINVAL, "unknown path %d", (int)path);
-  const bool tc_ok = pia::tc_supported(dtype == PI_ATTN_BF16, d, n);
-  const bool want_tc = path == PI_ATTN_PATH_TC || path == PI_ATTN_PATH_TC_FUSED || path == PI_ATTN_PATH_TC_SPLIT;
-  if (want_tc && !tc_ok) return fail(PI_ATTN_EUNSUPPORTED, "tensor-core path does not cover this dtype / d");
-  if (path == PI_ATTN_PATH_TC_SPLIT && !pia::tc_split_applies(n, k_win, pi, S))
-    return fail(PI_ATTN_EUNSUPPORTED, "split path needs n %% pi == 0 and at least one skip outside the window");
-  bool split = false;
-  if (path != PI_ATTN_PATH_SIMT && tc_ok)
-    split = path == PI_ATTN_PATH_TC_SPLIT || (path != PI_ATTN_PATH_TC_FUSED && pia::tc_split_preferred(n, k_win, pi, S));
+  bool tc = false, split = false;
+  if ((st = fwd_route(n, d, k_win, pi, S, dtype, path, &tc, &split)) != PI_ATTN_OK) return st;
   *launches = split ? 2 : 1;
-  *scratch_bytes = split ? (long long)B * H * n * (2LL * d + 4) : 0;
+  *scratch_bytes = fwd_scratch_bytes(B, H, n, d, split);
   return ok();
 }
 

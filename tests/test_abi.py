@@ -91,6 +91,17 @@ def test_plan_reports_launches_and_scratch(lib):
         pia.pi_attn_fwd_plan(1, 8, 4000, 64, 128, 64, 4, "bf16", "tc_split")  # n % pi != 0
 
 
+def test_workspace_is_checked_before_any_launch(lib):
+    # split path (n % pi == 0, skips outside the window): B*H*n*(2d+4) bytes of workspace
+    need = 2 * 4096 * (2 * 64 + 4)
+    args = [FAKE] * 7 + [1, 2, 4096, 64, 128, 64, 4, pia.PI_ATTN_BF16, pia.PATHS["tc_split"]]
+    assert lib.pi_attn_fwd_ws(*args, ctypes.c_void_p(0x10008), need, None) == pia.PI_ATTN_EINVAL  # misaligned
+    assert b"aligned" in lib.pi_attn_last_error()
+    assert lib.pi_attn_fwd_ws(*args, FAKE, need - 1, None) == pia.PI_ATTN_EINVAL  # one byte short
+    assert str(need).encode() in lib.pi_attn_last_error()
+    assert pia.pi_attn_fwd_plan(1, 2, 4096, 64, 128, 64, 4, "bf16", "tc_split") == (2, need)
+
+
 def test_built_for_sm100a_only():
     cmd = pbuild.command("x.so")
     assert "arch=compute_100a,code=sm_100a" in cmd and "-lineinfo" in cmd

@@ -193,6 +193,27 @@ def test_rows_are_normalised(path):
     assert np.max(np.abs(out - 1.0)) <= 4e-3
 
 
+def test_split_workspace_from_caller_or_library_gives_identical_results():
+    # pi_attn_fwd_ex allocates the skip partials itself; the binding passes a torch workspace to
+    # pi_attn_fwd_ws.  Same kernels, same scratch layout: the results are bit-identical.
+    import ctypes
+    inp = _inputs(2, 3, 2048, 64, "bf16", seed=9)
+    q, kk, v, wg, bg = _dev_inputs(inp, "bf16")
+    out_ws, lse_ws = pia.pi_attn_fwd(q, kk, v, wg, bg, 100, 128, 9, path="tc_split")
+    out_lib, lse_lib = torch.empty_like(q), torch.empty_like(lse_ws)
+    p = lambda t: ctypes.c_void_p(t.data_ptr())  # noqa: E731
+    st = pia.load().pi_attn_fwd_ex(p(q), p(kk), p(v), p(wg), p(bg), p(out_lib), p(lse_lib), 2, 3, 2048, 64, 100, 128, 9,
+                                   pia.PI_ATTN_BF16, pia.PATHS["tc_split"],
+                                   ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+    assert st == pia.PI_ATTN_OK
+    pia.pi_attn_check()
+    assert torch.equal(out_ws.view(torch.int16), out_lib.view(torch.int16))
+    assert torch.equal(lse_ws, lse_lib)
+    ro, rl, _ = oracle.fwd(inp["q"], inp["k"], inp["v"], inp["w_g"], inp["b_g"], 100, 128, 9)
+    assert_close(metrics(from_dev(out_ws).reshape(-1, 64), ro.reshape(-1, 64), lse_ws.cpu().numpy().reshape(-1),
+                         rl.reshape(-1)), "bf16", "split path, caller workspace")
+
+
 def test_lse_is_optional():
     inp = _inputs(1, 1, 300, 64, "bf16", seed=5)
     q, kk, v, wg, bg = _dev_inputs(inp, "bf16")
