@@ -7,7 +7,9 @@ A step is one call of the operator (the whole hot path: gate, window and skip lo
 softmax, P.V, epilogue) over one batch of the workload, inputs resident in HBM.  The default
 workload is bf16_n4k (bf16, B=1 H=8 n=4096 d=64, window 128, period 64, 4 skips); the other
 workloads of pi_synth.WORKLOADS can be timed with --workload.  The L2 is flushed (a 256 MiB
-write) before every timed step, outside the step's events.
+write, then a 256 MiB read of another buffer) before every timed step, outside the step's
+events.  Each timed step replays a CUDA graph of one public pi_attn_fwd / pi_attn_decode call
+(--eager times the plain call instead; the line reports both).
 
 Multi-GPU (torchrun, one process per GPU): every rank runs its own batch of the same workload
 (weak scaling: (b, h) problems are independent, there is no data exchange); the time is the max
@@ -329,8 +331,16 @@ def run_gpu(args):
         launches_per_step = 1  # one kernel when (b, h) fill the GPU (no split)
 
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
+    flush_rd = torch.zeros(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=device)
+
+    def flush_l2(s):
+        # write a buffer larger than L2, then read another one: the step starts with none of its
+        # inputs in L2 and without the flush's dirty lines, which it would otherwise write back
+        flush.fill_(s & 0xFF)
+        flush_rd.sum()
+
     for _ in range(args.warmup):
-        flush.fill_(1)
+        flush_l2(1)
         step()
     pia.pi_attn_check(stream)
 
@@ -350,7 +360,7 @@ def run_gpu(args):
         starts = [torch.cuda.Event(enable_timing=True) for _ in range(n)]
         ends = [torch.cuda.Event(enable_timing=True) for _ in range(n)]
         for s in range(n):
-            flush.fill_(s & 0xFF)
+            flush_l2(s)
             starts[s].record(stream)
             fn()
             ends[s].record(stream)
@@ -377,40 +387,42 @@ def run_gpu(args):
     value = tokens * world / (total_ms / 1e3 / args.steps)
 
     # end to end through the public call: pinned host inputs -> device, the call, results -> host
+    # The step's inputs come from pinned host memory and its results go back to it.  For decode
+    # the KV cache is resident state (like weights); the step's input is the new query.
     e2e = None
-    if w.kind == "prefill":
-        hq = {k: torch.from_numpy(np.ascontiguousarray(host[k]).view(np.int16) if w.dtype == "bf16"
-                                  else np.ascontiguousarray(host[k])).pin_memory() for k in ("q", "k", "v")}
-        hw = {k: torch.from_numpy(host[k]).pin_memory() for k in ("w_g", "b_g")}
-        h_out = torch.empty(out.shape, dtype=out.dtype).pin_memory()
-        h_lse = torch.empty(lse.shape, dtype=torch.float32).pin_memory()
-        dq = {k: t[k].view(torch.int16) if w.dtype == "bf16" else t[k] for k in ("q", "k", "v")}
-        e_steps = max(3, min(args.steps, 50))
-        h2d = sum(x.numel() * x.element_size() for x in hq.values()) + sum(
-            x.numel() * x.element_size() for x in hw.values())
-        d2h = h_out.numel() * h_out.element_size() + h_lse.numel() * 4
+    names = ("q", "k", "v", "w_g", "b_g") if w.kind == "prefill" else ("q", "w_g", "b_g")
+    pairs = []
+    for name in names:
+        a = np.ascontiguousarray(host[name])
+        dst = t[name]
+        if a.dtype == np.uint16:  # bf16 bits
+            a, dst = a.view(np.int16), dst.view(torch.int16)
+        pairs.append((dst, torch.from_numpy(a).pin_memory()))
+    h_out = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    h_lse = torch.empty(lse.shape, dtype=torch.float32).pin_memory()
+    e_steps = max(3, min(args.steps, 50))
+    h2d = sum(h.numel() * h.element_size() for _, h in pairs)
+    d2h = h_out.numel() * h_out.element_size() + h_lse.numel() * 4
 
-        def e2e_step():
-            for k in ("q", "k", "v"):
-                dq[k].copy_(hq[k], non_blocking=True)
-            t["w_g"].copy_(hw["w_g"], non_blocking=True)
-            t["b_g"].copy_(hw["b_g"], non_blocking=True)
-            step()
-            h_out.copy_(out, non_blocking=True)
-            h_lse.copy_(lse, non_blocking=True)
+    def e2e_step():
+        for dst, src in pairs:
+            dst.copy_(src, non_blocking=True)
+        step()
+        h_out.copy_(out, non_blocking=True)
+        h_lse.copy_(lse, non_blocking=True)
 
-        for _ in range(2):
-            e2e_step()
-        torch.cuda.synchronize(device)
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        for _ in range(e_steps):
-            e2e_step()
-        e1.record(stream)
-        torch.cuda.synchronize(device)
-        e_ms = max_over_ranks(e0.elapsed_time(e1), world, device) / e_steps
-        e2e = {"value": tokens * world / (e_ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": int(h2d),
-               "d2h_bytes_per_step": int(d2h), "ms_per_step": e_ms}
+    for _ in range(2):
+        e2e_step()
+    torch.cuda.synchronize(device)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize(device)
+    e_ms = max_over_ranks(e0.elapsed_time(e1), world, device) / e_steps
+    e2e = {"value": tokens * world / (e_ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": int(h2d),
+           "d2h_bytes_per_step": int(d2h), "ms_per_step": e_ms}
     pia.pi_attn_check(stream)
 
     peaks, peak_kind = load_peaks()
@@ -445,7 +457,7 @@ def run_gpu(args):
         "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": w.dtype, "data": "synthetic (seeded Philox normals, workload recipe)",
-        "config": dict(w.describe(), l2="flushed before every timed step (256 MiB write)",
+        "config": dict(w.describe(), l2="flushed before every timed step (256 MiB written, then another 256 MiB read)",
                        parallelism=f"replicas x{world} (independent (b, h) batches)"),
         "achieved_tflops": flops / launch_s / 1e12, "achieved_gbs": bytes_ / launch_s / 1e9,
         "roofline": roof, "cpu_baseline": cpu, "e2e": e2e,
@@ -456,7 +468,7 @@ def run_gpu(args):
     }
     if rank == 0:
         print(json.dumps(line), flush=True)
-    del t, flush, graph
+    del t, flush, flush_rd, graph
     if world > 1:
         import torch.distributed as dist
         dist.barrier()

@@ -38,9 +38,11 @@ constexpr int BM = 128;       // query rows per CTA
 constexpr int BN = kTileKeys; // keys per tile
 // Pipeline shape.  Both head sizes run two CTAs per SM, so that one CTA's prologue (TMEM
 // allocation, Q load, gate) and epilogue overlap the other's tiles: 256 TMEM columns per CTA
-// (one S buffer of 128 columns, P written over it, and O), one softmax warpgroup.  The K/V ring
-// has two stages at d = 64 and one at d = 128 (three 32 KB tiles per CTA); with one S buffer the
-// next tile's K and V loads still have a whole softmax pass to land.
+// (one S buffer of 128 columns, P written over it, and O), one softmax warpgroup.  (Two groups
+// splitting each S row by columns also fit, at 96 registers a thread, but the per-tile exchange
+// of their row maxima costs more than the halved pass over the row saves.)  The K/V ring has two
+// stages at d = 64 and one at d = 128 (three 32 KB tiles per CTA); with one S buffer the next
+// tile's K and V loads still have a whole softmax pass to land.
 template <int D> constexpr int kStages = D == 128 ? 1 : 2;  // K/V ring depth
 template <int D> constexpr int kGroups = 1;                 // softmax warpgroups (split S rows by columns)
 template <int D> constexpr int kSBufsT = 1;                 // S buffers in TMEM
@@ -69,10 +71,12 @@ struct Smem {
   static constexpr int kNumBars = 1 + 4 * NSTAGE + 3 * kSBufs + 3 + (kGroups<D> > 1 ? 1 : 0);
   static constexpr int kMisc = kBar + kNumBars * 8;      // tmem base (4 B), abort flag (4 B)
   // two-group exchange of per-row partials: tile maxima (double-buffered), fp32 and rounded sums
-  static constexpr int kXch = kMisc + 8;
+  static constexpr int kXch = (kMisc + 8 + 15) / 16 * 16;
   static constexpr int kXchBytes = kGroups<D> > 1 ? (2 * 2 + 2) * kGroups<D> * BM * 4 : 0;
-  static constexpr int kWg = kXch + kXchBytes;          // w_g[h] staging, D floats
+  static constexpr int kWg = (kXch + kXchBytes + 15) / 16 * 16;  // w_g[h] staging, D floats (read as float4)
   static constexpr int kTotal = kWg + D * 4;
+  static_assert(kQ % 1024 == 0 && kK % 1024 == 0 && kV % 1024 == 0, "128-byte-swizzled tiles sit on 1 KB");
+  static_assert(kBar % 8 == 0 && kWg % 16 == 0, "mbarriers on 8 bytes, the w_g staging on 16");
   static constexpr int kAlloc = kTotal + 1024 - 128;     // slack to align a (>= 128 B aligned) base to 1 KB
   // 228 KB of shared memory per SM, 1 KB of it reserved per CTA
   static_assert(kAlloc <= 228 * 1024 / kCtasPerSm<D> - 1024, "shared memory of the CTAs on one SM");
