@@ -34,21 +34,19 @@
 namespace pia {
 namespace tc {
 
-constexpr int BM = 128;       // query rows per CTA
-constexpr int BN = kTileKeys; // keys per tile
-// Pipeline shape.  Both head sizes run two CTAs per SM, so that one CTA's prologue (TMEM
-// allocation, Q load, gate) and epilogue overlap the other's tiles: 256 TMEM columns per CTA
-// (one S buffer of 128 columns, P written over it, and O), one softmax warpgroup.  (Two groups
-// splitting each S row by columns also fit, at 96 registers a thread, but the per-tile exchange
-// of their row maxima costs more than the halved pass over the row saves.)  The K/V ring has two
-// stages at d = 64 and one at d = 128 (three 32 KB tiles per CTA); with one S buffer the next
-// tile's K and V loads still have a whole softmax pass to land.
-template <int D> constexpr int kStages = D == 128 ? 1 : 2;  // K/V ring depth
-template <int D> constexpr int kGroups = 1;                 // softmax warpgroups (split S rows by columns)
-template <int D> constexpr int kSBufsT = 1;                 // S buffers in TMEM
+constexpr int BM = 128;        // query rows per CTA
+constexpr int BN = kTileKeys;  // keys per tile (64)
+// Pipeline shape.  Both head sizes run two CTAs per SM and one softmax warpgroup per CTA; TMEM per
+// CTA is 256 columns: two S buffers of 64 columns (the next tile's Q.K^T runs while the softmax
+// works on this one; P is written back over the S columns it has read) and O (D columns).  Shared
+// memory: the Q tile (128 rows) and a two-stage ring of 64-row K and V tiles.  The two K stages,
+// and the two V stages, are each one contiguous 128-row region, which the epilogue reuses.
+// (Two warpgroups splitting each S row by columns also fit, at 96 registers a thread, but the
+// per-tile exchange of their row maxima cost more than the halved pass over the row saved.)
+constexpr int NSTAGE = 2;      // K/V ring depth
+constexpr int NSB = 2;         // S buffers in TMEM
 template <int D> constexpr int kCtasPerSm = 2;
-// warp 0 TMA, warp 1 MMA, warps 2 .. 2 + 4 * groups - 1 softmax
-template <int D> constexpr int kThreads = 64 + 128 * kGroups<D>;
+constexpr int kThreads = 192;  // warp 0 TMA, warp 1 MMA, warps 2..5 softmax (one query row a thread)
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 // Pairs of a 32-column window-only chunk whose exponentials run on the FMA pipe (bit e: columns
 // 2e, 2e + 1); the rest use the special-function unit.
@@ -57,25 +55,23 @@ constexpr uint32_t kPolyPairs = 0x4924u;  // every third pair
 // ---- shared memory plan (offsets from a 1024-byte aligned base) ---------------------------------
 template <int D>
 struct Smem {
-  static constexpr int NSTAGE = kStages<D>;
-  static constexpr int kTileBytes = BM * D * 2;          // one 128-row bf16 tile
+  static constexpr int kQBytes = BM * D * 2;             // the Q tile (bf16)
+  static constexpr int kKVBytes = BN * D * 2;            // one K or V tile
   static constexpr int kQ = 0;
-  static constexpr int kK = kQ + kTileBytes;
-  static constexpr int kV = kK + NSTAGE * kTileBytes;
-  static constexpr int kBar = kV + NSTAGE * kTileBytes;  // (P lives in TMEM, over its S columns)
-  static constexpr int kSBufs = kSBufsT<D>;
-  static constexpr int kTmemCols = 128 * kSBufs + D <= 256 ? 256 : 512;  // S buffers (128 each) + O (D)
-  static_assert(kTmemCols * kCtasPerSm<D> <= 512, "TMEM columns of the CTAs on one SM");
-  // barriers: q_full, k_full[2], k_empty[2], v_full[2], v_empty[2], s_full[NSB], s_free[NSB],
-  // pv_done[NSB], p_full, drain, skip partials, (two groups) max exchange
-  static constexpr int kNumBars = 1 + 4 * NSTAGE + 3 * kSBufs + 3 + (kGroups<D> > 1 ? 1 : 0);
+  static constexpr int kK = kQ + kQBytes;
+  static constexpr int kV = kK + NSTAGE * kKVBytes;
+  static constexpr int kBar = kV + NSTAGE * kKVBytes;    // (P lives in TMEM, over its S columns)
+  static constexpr int kTmemCols = 256;                  // S buffers (BN each) + O (D)
+  static_assert(NSB * BN + D <= kTmemCols && kTmemCols * kCtasPerSm<D> <= 512, "TMEM columns");
+  static_assert(NSTAGE * kKVBytes == kQBytes, "the K and V regions each hold one 128-row tile");
+  // barriers: q_full, k_full[NSTAGE], k_empty[NSTAGE], v_full[NSTAGE], v_empty[NSTAGE],
+  // s_full[NSB], s_free[NSB], pv_done[NSB], p_full[NSB], drain, skip partials
+  static constexpr int kNumBars = 1 + 4 * NSTAGE + 4 * NSB + 2;
   static constexpr int kMisc = kBar + kNumBars * 8;      // tmem base (4 B), abort flag (4 B)
-  // two-group exchange of per-row partials: tile maxima (double-buffered), fp32 and rounded sums
-  static constexpr int kXch = (kMisc + 8 + 15) / 16 * 16;
-  static constexpr int kXchBytes = kGroups<D> > 1 ? (2 * 2 + 2) * kGroups<D> * BM * 4 : 0;
-  static constexpr int kWg = (kXch + kXchBytes + 15) / 16 * 16;  // w_g[h] staging, D floats (read as float4)
+  static constexpr int kWg = (kMisc + 8 + 15) / 16 * 16; // w_g[h] staging, D floats (read as float4)
   static constexpr int kTotal = kWg + D * 4;
-  static_assert(kQ % 1024 == 0 && kK % 1024 == 0 && kV % 1024 == 0, "128-byte-swizzled tiles sit on 1 KB");
+  static_assert(kQ % 1024 == 0 && kK % 1024 == 0 && kV % 1024 == 0 && kKVBytes % 1024 == 0,
+                "128-byte-swizzled tiles sit on 1 KB");
   static_assert(kBar % 8 == 0 && kWg % 16 == 0, "mbarriers on 8 bytes, the w_g staging on 16");
   static constexpr int kAlloc = kTotal + 1024 - 128;     // slack to align a (>= 128 B aligned) base to 1 KB
   // 228 KB of shared memory per SM, 1 KB of it reserved per CTA
@@ -374,7 +370,7 @@ struct Params {
 };
 
 template <int D, int MODE>
-__global__ void __launch_bounds__(kThreads<D>, kCtasPerSm<D>) fwd_tc_kernel(const __grid_constant__ CUtensorMap tmq,
+__global__ void __launch_bounds__(kThreads, kCtasPerSm<D>) fwd_tc_kernel(const __grid_constant__ CUtensorMap tmq,
                                                                           const __grid_constant__ CUtensorMap tmk,
                                                                           const __grid_constant__ CUtensorMap tmv,
                                                                           const __grid_constant__ CUtensorMap tmo,
@@ -416,26 +412,24 @@ __global__ void __launch_bounds__(kThreads<D>, kCtasPerSm<D>) fwd_tc_kernel(cons
   const int view_rows = MODE == kResidue ? prm.T : prm.n;
 
   const uint32_t sQ = base + L::kQ, sK = base + L::kK, sV = base + L::kV;
-  // P of tile j sits in TMEM over the columns of S buffer j % NSB that the softmax has read:
-  // the 32-key chunk cb of P (16 packed columns) at column pcol(cb) of the buffer.  Chunks are
-  // handled by the softmax group cb / CPG, which reads its S chunks in order before writing them.
-  constexpr int CPG_K = (BN / 32) / kGroups<D>;
-  auto pcol = [](int cb) { return 64 * (cb / CPG_K) + 16 * (cb % CPG_K); };
-  constexpr int NSTAGE = L::NSTAGE;
+  // P of tile j sits in TMEM over the columns of S buffer j % NSB that the softmax has read: the
+  // 32-key chunk cb of P (16 packed columns) at column 16 cb of the buffer, written after S chunk
+  // cb (columns 32 cb .. 32 cb + 31) has been read.
   const uint32_t bar0 = base + L::kBar;
   const uint32_t bar_q = bar0;
   auto bar_kfull = [&](int s) { return bar0 + 8u * (1 + s); };
   auto bar_kempty = [&](int s) { return bar0 + 8u * (1 + NSTAGE + s); };
   auto bar_vfull = [&](int s) { return bar0 + 8u * (1 + 2 * NSTAGE + s); };
   auto bar_vempty = [&](int s) { return bar0 + 8u * (1 + 3 * NSTAGE + s); };
-  constexpr int NSB = L::kSBufs;
   auto bar_sfull = [&](int b) { return bar0 + 8u * (1 + 4 * NSTAGE + b); };
   auto bar_sfree = [&](int b) { return bar0 + 8u * (1 + 4 * NSTAGE + NSB + b); };
   auto bar_pvdone = [&](int b) { return bar0 + 8u * (1 + 4 * NSTAGE + 2 * NSB + b); };  // P.V of buffer b
-  const uint32_t bar_pfull = bar0 + 8u * (1 + 4 * NSTAGE + 3 * NSB);
-  const uint32_t bar_drain = bar_pfull + 8;
-  const uint32_t bar_so = bar_pfull + 16;  // kBandMerge: the tile of skip partials has landed
-  const uint32_t bar_xm = bar_pfull + 24;  // two groups: a tile's partial maxima are exchanged
+  // P of buffer b written by all 128 rows.  One barrier per buffer: with two buffers a fast warp
+  // can finish the next tile before a slow one finishes this tile, and on a shared barrier its
+  // arrivals would complete this tile's phase early.
+  auto bar_pfull = [&](int b) { return bar0 + 8u * (1 + 4 * NSTAGE + 3 * NSB + b); };
+  const uint32_t bar_drain = bar0 + 8u * (1 + 4 * NSTAGE + 4 * NSB);
+  const uint32_t bar_so = bar_drain + 8;  // kBandMerge: the tile of skip partials has landed
   uint32_t* const tmem_slot = reinterpret_cast<uint32_t*>(sbase + L::kMisc);
   volatile int* const abort_flag = reinterpret_cast<volatile int*>(sbase + L::kMisc + 4);
 
@@ -449,17 +443,16 @@ __global__ void __launch_bounds__(kThreads<D>, kCtasPerSm<D>) fwd_tc_kernel(cons
     }
     for (int b = 0; b < NSB; ++b) {
       mbar_init(bar_sfull(b), 1);
-      mbar_init(bar_sfree(b), BM * kGroups<D>);
+      mbar_init(bar_sfree(b), BM);
       mbar_init(bar_pvdone(b), 1);
+      mbar_init(bar_pfull(b), BM);
     }
-    mbar_init(bar_pfull, BM * kGroups<D>);
     mbar_init(bar_drain, 1);
     mbar_init(bar_so, 1);
-    if (kGroups<D> > 1) mbar_init(bar_xm, BM * kGroups<D>);
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
-  if (warp == 1) {  // TMEM: S buffer b in columns [128 b, 128 b + 128), O in [128 NSB, 128 NSB + D)
+  if (warp == 1) {  // TMEM: S buffer b in columns [BN b, BN b + BN), O in [BN NSB, BN NSB + D)
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
                  "n"(L::kTmemCols)
                  : "memory");
@@ -469,44 +462,46 @@ __global__ void __launch_bounds__(kThreads<D>, kCtasPerSm<D>) fwd_tc_kernel(cons
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const uint32_t tS = tmem, tO = tmem + 128 * NSB;  // S buffer b at tS + 128 b
+  const uint32_t tS = tmem, tO = tmem + BN * NSB;  // S buffer b at tS + BN b
 
-  // one 128-row tile of the view (rows r0 .. r0+127) into shared memory, D/64 boxes of 64 columns
-  auto load_tile = [&](uint32_t dst, const CUtensorMap* map, uint32_t bar, long long r0) {
+  // one tile of `rows` rows of the view (r0 ..) into shared memory: D/64 boxes of 64 columns,
+  // each rows x 128 bytes (the map's box has `rows` rows: BM for Q, BN for K and V)
+  auto load_tile = [&](uint32_t dst, const CUtensorMap* map, uint32_t bar, long long r0, int rows) {
 #pragma unroll
     for (int c = 0; c < D / 64; ++c) {
       if (MODE == kResidue)
-        tma_load_4d(dst + c * BM * 128, map, bar, c * 64, res, (int)r0, bh);
+        tma_load_4d(dst + c * rows * 128, map, bar, c * 64, res, (int)r0, bh);
       else
-        tma_load_3d(dst + c * BM * 128, map, bar, c * 64, (int)r0, bh);
+        tma_load_3d(dst + c * rows * 128, map, bar, c * 64, (int)r0, bh);
     }
   };
 
   if (warp == 0) {
     // ------------------------------------------------------------------ TMA producer
     if (lane == 0) {
-      constexpr uint32_t kTile = L::kTileBytes;
-      mbar_expect_tx(bar_q, kTile);
-      load_tile(sQ, &tmq, bar_q, q0);
+      constexpr uint32_t kKV = L::kKVBytes;
+      mbar_expect_tx(bar_q, L::kQBytes);
+      load_tile(sQ, &tmq, bar_q, q0, BM);
       int nk = 0, nv = 0;  // K and V tile loads issued
       for (int t = walk.next(0); t >= 0; t = walk.next(t + 1)) {
         const int s = nk % NSTAGE, use = nk / NSTAGE;
         if (use > 0 && !mbar_wait(bar_kempty(s), (use - 1) & 1, abort_flag)) break;
-        mbar_expect_tx(bar_kfull(s), kTile);
-        load_tile(sK + s * kTile, &tmk, bar_kfull(s), (long long)t * BN);
+        mbar_expect_tx(bar_kfull(s), kKV);
+        load_tile(sK + s * kKV, &tmk, bar_kfull(s), (long long)t * BN, BN);
         ++nk;
         if (use > 0 && !mbar_wait(bar_vempty(s), (use - 1) & 1, abort_flag)) break;
-        mbar_expect_tx(bar_vfull(s), kTile);
-        load_tile(sV + s * kTile, &tmv, bar_vfull(s), (long long)t * BN);
+        mbar_expect_tx(bar_vfull(s), kKV);
+        load_tile(sV + s * kKV, &tmv, bar_vfull(s), (long long)t * BN, BN);
         ++nv;
       }
-      // kBandMerge: the tile of skip partials goes into K stage 0 as soon as the last Q.K^T that
-      // reads that stage has completed, so its load overlaps the last tile's softmax and P.V
+      // kBandMerge: the 128-row tile of skip partials goes into the K region as soon as the last
+      // Q.K^T has completed (its commit covers every earlier one), so that its load overlaps the
+      // last tile's softmax and P.V
       bool so_issued = false;
       if (MODE == kBandMerge && !*abort_flag) {
-        const int u0 = nk > 0 ? (nk - 1) / NSTAGE * NSTAGE : -1;  // last load into K stage 0
-        if (u0 < 0 || mbar_wait(bar_kempty(0), (u0 / NSTAGE) & 1, abort_flag)) {
-          mbar_expect_tx(bar_so, kTile);
+        const int u = nk - 1;  // last K load
+        if (u < 0 || mbar_wait(bar_kempty(u % NSTAGE), (u / NSTAGE) & 1, abort_flag)) {
+          mbar_expect_tx(bar_so, L::kQBytes);
 #pragma unroll
           for (int c = 0; c < D / 64; ++c) tma_load_3d(sK + c * BM * 128, &tms, bar_so, c * 64, (int)q0, bh);
           so_issued = true;
@@ -526,35 +521,40 @@ __global__ void __launch_bounds__(kThreads<D>, kCtasPerSm<D>) fwd_tc_kernel(cons
   } else if (warp == 1) {
     // ------------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      constexpr uint32_t kTile = L::kTileBytes;
+      constexpr uint32_t kKV = L::kKVBytes;
       constexpr uint32_t idesc_qk = idesc_bf16(BM, BN, 0);
       constexpr uint32_t idesc_pv = idesc_bf16(BM, D, 1);
       bool okw = mbar_wait(bar_q, 0, abort_flag);
       tc_fence_after();
-      // S_j = Q K_j^T into S buffer j % NSB : K = D, 16 per instruction; 64-column blocks of 16 KB
+      // S_j = Q K_j^T into S buffer j % NSB : K = D, 16 per instruction; the operands' 64-column
+      // blocks are BM x 128 B (Q) and BN x 128 B (K) apart
       auto issue_qk = [&](int s, int b) {
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * (BM * 128) + (kk & 3) * 32;
-          tc_mma(tS + 128 * b, sw128_desc(sQ + off, 16, 1024), sw128_desc(sK + s * kTile + off, 16, 1024), idesc_qk,
-                 kk > 0 ? 1u : 0u);
+          const uint32_t in = (kk & 3) * 32;
+          tc_mma(tS + BN * b, sw128_desc(sQ + (kk >> 2) * (BM * 128) + in, 16, 1024),
+                 sw128_desc(sK + s * kKV + (kk >> 2) * (BN * 128) + in, 16, 1024), idesc_qk, kk > 0 ? 1u : 0u);
         }
       };
-      // O += P V_j : K = 128 keys, 16 per instruction; V is N-major (d contiguous)
+      // O += P V_j : K = BN keys, 16 per instruction; V is N-major (d contiguous, 64-column
+      // blocks BN x 128 B apart)
       auto issue_pv = [&](int s, int b, bool first) {  // A = P from TMEM (S buffer b)
 #pragma unroll
         for (int kk = 0; kk < BN / 16; ++kk) {
-          const uint32_t acol = 128 * b + pcol(kk >> 1) + 8 * (kk & 1);
+          const uint32_t acol = BN * b + 16 * (kk >> 1) + 8 * (kk & 1);
           const uint32_t boff = kk * 16 * 128;
-          tc_mma_ts(tO, tS + acol, sw128_desc(sV + s * kTile + boff, BN * 128, 1024), idesc_pv,
+          tc_mma_ts(tO, tS + acol, sw128_desc(sV + s * kKV + boff, BN * 128, 1024), idesc_pv,
                     (first && kk == 0) ? 0u : 1u);
         }
       };
-      // Q.K^T of tile j needs its K stage loaded and its S buffer released by tile j - NSB
+      // Q.K^T of tile j needs its K stage loaded, its S buffer released by the softmax of tile
+      // j - NSB, and the P.V of tile j - NSB finished: that P.V reads P from the columns this
+      // Q.K^T overwrites, and MMAs into different accumulators are not ordered with each other.
       auto try_qk = [&](int jq) -> bool {
         const int s = jq % NSTAGE, b = jq % NSB;
         if (!mbar_wait(bar_kfull(s), (jq / NSTAGE) & 1, abort_flag)) return false;
         if (jq >= NSB && !mbar_wait(bar_sfree(b), (jq / NSB - 1) & 1, abort_flag)) return false;
+        if (jq >= NSB && !mbar_wait(bar_pvdone(b), (jq / NSB - 1) & 1, abort_flag)) return false;
         tc_fence_after();
         issue_qk(s, b);
         tc_commit(bar_sfull(b));
@@ -564,20 +564,17 @@ __global__ void __launch_bounds__(kThreads<D>, kCtasPerSm<D>) fwd_tc_kernel(cons
       int j = 0;
       int t = walk.next(0);
       if (okw && t >= 0) okw = try_qk(0);
-      // With two S buffers the next Q.K^T goes first (it overlaps this tile's softmax); with one,
-      // P.V of this tile must read P before the next Q.K^T overwrites the buffer, so it goes first
-      // (the tensor pipe runs one thread's MMAs in issue order).
+      // The next tile's Q.K^T goes first: it runs while the softmax works on this tile.
       while (okw && t >= 0) {
         const int tn = walk.next(t + 1);
         const int s = j % NSTAGE;
-        if (NSB == 2 && tn >= 0 && !try_qk(j + 1)) break;
+        if (tn >= 0 && !try_qk(j + 1)) break;
         if (!mbar_wait(bar_vfull(s), (j / NSTAGE) & 1, abort_flag)) break;
-        if (!mbar_wait(bar_pfull, j & 1, abort_flag)) break;
+        if (!mbar_wait(bar_pfull(j % NSB), (j / NSB) & 1, abort_flag)) break;
         tc_fence_after();
         issue_pv(s, j % NSB, j == 0);
         tc_commit(bar_pvdone(j % NSB));
         tc_commit(bar_vempty(s));
-        if (NSB == 1 && tn >= 0 && !try_qk(j + 1)) break;
         ++j;
         t = tn;
       }
@@ -588,15 +585,10 @@ __global__ void __launch_bounds__(kThreads<D>, kCtasPerSm<D>) fwd_tc_kernel(cons
     }
     __syncwarp();
   } else {
-    // ------------------------------------------------------------------ softmax warpgroups
-    constexpr int NG = kGroups<D>;            // column groups: each row has one thread per group
-    constexpr int CPG = (BN / 32) / NG;       // 32-column chunks of S (and of P) per group
-    constexpr int OCG = D / NG;               // O columns per group
-    const int g = (warp - 2) >> 2;            // this thread's column group
+    // ------------------------------------------------------------------ softmax warpgroup
+    constexpr int CPT = BN / 32;              // 32-column chunks of S (and of P) per tile
     const int q4 = warp & 3;                  // TMEM lane quarter this warp may access
     const int r = q4 * 32 + lane;             // query row within the tile
-    float* const xmax = reinterpret_cast<float*>(sbase + L::kXch);          // [2][NG][BM]
-    float* const xsum = xmax + 2 * NG * BM;                                  // [2][NG][BM]
     const long long qi = q0 + r;              // row in the view
     const long long i = MODE == kResidue ? qi * prm.pi + res : qi;  // row in the sequence
     const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
@@ -609,7 +601,7 @@ __global__ void __launch_bounds__(kThreads<D>, kCtasPerSm<D>) fwd_tc_kernel(cons
     // still in flight.
     float* const wg_s = reinterpret_cast<float*>(sbase + L::kWg);
     if (threadIdx.x - 64 < D) wg_s[threadIdx.x - 64] = prm.w_g[(long long)h * D + (threadIdx.x - 64)];
-    asm volatile("bar.sync 1, %0;" ::"n"(128 * NG) : "memory");
+    asm volatile("bar.sync 1, 128;" ::: "memory");
     bool ok = __all_sync(0xffffffffu, mbar_wait(bar_q, 0, abort_flag));
     float z = prm.b_g[h];
     {
@@ -649,7 +641,7 @@ __global__ void __launch_bounds__(kThreads<D>, kCtasPerSm<D>) fwd_tc_kernel(cons
       // every lane of the warp takes the same branch: tcgen05.ld is .sync.aligned
       if (!__all_sync(0xffffffffu, mbar_wait(bar_sfull(sb), (j / NSB) & 1, abort_flag))) { ok = false; break; }
       tc_fence_after();
-      const uint32_t tSb = tS + 128 * sb + lane_off;
+      const uint32_t tSb = tS + BN * sb + lane_off;
       // the index rule on this tile, for row qi: window columns [lc_lo, lc_hi], skip columns bitmask
       int lc_lo, lc_hi;
       uint32_t sk[BN / 32];
@@ -659,7 +651,10 @@ __global__ void __launch_bounds__(kThreads<D>, kCtasPerSm<D>) fwd_tc_kernel(cons
         row_tile_mask(qi, (long long)t * BN, prm.kwin, prm.pi, MODE == kFused ? prm.S : 0, m0, lc_lo, lc_hi, sk, 0,
                       walk.rpi);
       const bool has_win = lc_lo <= lc_hi;
-      const bool has_skip = (sk[0] | sk[1] | sk[2] | sk[3]) != 0u;
+      uint32_t sk_any = 0u;
+#pragma unroll
+      for (int w = 0; w < BN / 32; ++w) sk_any |= sk[w];
+      const bool has_skip = sk_any != 0u;
 
       // Pass 1: a reference for the tile, from the whole S row in one load: the max of the raw
       // scores, scaled, plus the larger prior present.  It bounds the true max of the biased
@@ -668,25 +663,18 @@ __global__ void __launch_bounds__(kThreads<D>, kCtasPerSm<D>) fwd_tc_kernel(cons
       // spread of the row.  Probabilities only need a reference at or above their max.
       float mt;
       {
-        constexpr int CW = BN / NG;  // columns of this group
-        float x[CW];
-        if (NG == 1) tmem_ld128(tSb, x);
-        else tmem_ld64(tSb + g * CW, x);
-        float mx[8];
+        float x[BN];
+        tmem_ld64(tSb, x);
+        static_assert(BN == 64, "pass 1 reduces eight groups of eight columns");
+        float mx[8];  // mx[e]: max over columns e, e + 8, ..., e + 56
 #pragma unroll
-        for (int e = 0; e < 8; ++e) mx[e] = x[e];
-#pragma unroll
-        for (int c = 8; c < CW; ++c) mx[c & 7] = fmaxf(mx[c & 7], x[c]);
-        float mraw =
-            fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])), fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
-        if (NG > 1) {  // the row's other half, through shared memory (double-buffered by tile parity)
-          float* const xm = xmax + (j & 1) * NG * BM;
-          xm[g * BM + r] = mraw;
-          mbar_arrive(bar_xm);
-          if (!__all_sync(0xffffffffu, mbar_wait(bar_xm, j & 1, abort_flag))) { ok = false; break; }
-#pragma unroll
-          for (int o = 0; o < NG; ++o) mraw = fmaxf(mraw, xm[o * BM + r]);
+        for (int e = 0; e < 8; ++e) {
+          float m = max3f(x[e], x[8 + e], x[16 + e]);
+          m = max3f(m, x[24 + e], x[32 + e]);
+          m = max3f(m, x[40 + e], x[48 + e]);
+          mx[e] = fmaxf(m, x[56 + e]);
         }
+        const float mraw = max3f(max3f(mx[0], mx[1], mx[2]), max3f(mx[3], mx[4], mx[5]), fmaxf(mx[6], mx[7]));
         const float top = has_win ? (has_skip ? fmaxf(bias_l, bias_p) : bias_l) : bias_p;
         mt = (has_win || has_skip) ? fmaf(mraw, prm.scale_log2, top) : NEG_INF;
       }
@@ -696,7 +684,7 @@ __global__ void __launch_bounds__(kThreads<D>, kCtasPerSm<D>) fwd_tc_kernel(cons
       bool rescale = false;
       if (mt > m_ref + kRescaleThreshold || (m_ref == NEG_INF && mt != NEG_INF)) {
         factor = ex2(m_ref - mt);  // 0 when m_ref = -inf
-        rescale = m_ref != NEG_INF;  // O holds earlier tiles' sums (decided alike in every group)
+        rescale = m_ref != NEG_INF;  // O holds earlier tiles' sums
         l_sum *= factor;
         l_rnd *= factor;
         m_ref = mt;
@@ -711,7 +699,7 @@ __global__ void __launch_bounds__(kThreads<D>, kCtasPerSm<D>) fwd_tc_kernel(cons
       }
       if (__any_sync(0xffffffffu, rescale)) {
         // O must hold every earlier tile's P.V before it is rescaled: wait for the P.V of tile j - 1
-        if (NSB == 2 && j >= 1 &&
+        if (j >= 1 &&
             !__all_sync(0xffffffffu, mbar_wait(bar_pvdone((j - 1) % NSB), ((j - 1) / NSB) & 1, abort_flag))) {
           ok = false;
           break;
@@ -721,7 +709,7 @@ __global__ void __launch_bounds__(kThreads<D>, kCtasPerSm<D>) fwd_tc_kernel(cons
         // rows needs it, the others multiply by 1
         const float f = rescale ? factor : 1.f;
 #pragma unroll 1
-        for (int c = g * (OCG / 32); c < (g + 1) * (OCG / 32); ++c) {
+        for (int c = 0; c < D / 32; ++c) {
           float o[32];
           tmem_ld32(tO + lane_off + c * 32, o);
 #pragma unroll
@@ -741,11 +729,11 @@ __global__ void __launch_bounds__(kThreads<D>, kCtasPerSm<D>) fwd_tc_kernel(cons
       const float bl_m = bias_l - m_use, bp_m = bias_p - m_use;
       float ls = 0.f, lr = 0.f;
 #pragma unroll 1
-      for (int cb = g * CPG; cb < (g + 1) * CPG; ++cb) {
+      for (int cb = 0; cb < CPT; ++cb) {
         const int c0 = cb * 32;
         float x[32];
         tmem_ld32(tSb + c0, x);
-        const uint32_t skb = cb == 0 ? sk[0] : cb == 1 ? sk[1] : cb == 2 ? sk[2] : sk[3];
+        const uint32_t skb = cb == 0 ? sk[0] : sk[CPT - 1];
         const uint32_t wm = window_bits(lc_lo - c0, lc_hi - c0);
         uint32_t pk[16];
         if ((wm | skb) == 0u) {
@@ -808,36 +796,26 @@ __global__ void __launch_bounds__(kThreads<D>, kCtasPerSm<D>) fwd_tc_kernel(cons
           lr += r0 + r1;
         }
         __syncwarp();  // rows may have taken different branches; tcgen05.st is .sync.aligned
-        tmem_st16(tSb + pcol(cb), pk);  // over S columns this group has already read
+        tmem_st16(tSb + 16 * cb, pk);  // over S columns already read
       }
       l_sum += ls;
       l_rnd += lr;
       tmem_wait_st();
       tc_fence_before();
+      // P first: once s_free completes (the Q.K^T of tile j + NSB may then start, and with it the
+      // arrivals of that tile) every thread has already arrived on this tile's p_full phase
+      mbar_arrive(bar_pfull(sb));
       mbar_arrive(bar_sfree(sb));  // the buffer may take the Q.K^T of tile j + NSB (issued after this P.V)
-      mbar_arrive(bar_pfull);
     }
-    // ---- epilogue: the normalised row goes to shared memory (V stage 0, free once the last P.V
-    // has completed) in the 128-byte-swizzled tile layout, then one TMA store writes the tile
-    // (rows past the end of the view are clipped by the tensor map).  kBandMerge first brings the
-    // tile of skip partials in by TMA (into the free K stage 0) and merges them row by row.
+    // ---- epilogue: the normalised row goes to shared memory (the V region, free once the last
+    // P.V has completed) in the 128-byte-swizzled 128-row tile layout, then one TMA store writes
+    // the tile (rows past the end of the view are clipped by the tensor map).  kBandMerge merges
+    // the tile of skip partials, which the producer has loaded into the K region.
     const bool row_ok = qi < view_rows;
     const long long orow = (long long)bh * prm.n + i;  // row in [B*H, n] layouts
     const bool have_o = __all_sync(
         0xffffffffu, ok && j > 0 && mbar_wait(bar_pvdone((j - 1) % NSB), ((j - 1) / NSB) & 1, abort_flag));
     const bool no_keys = MODE == kResidue && __all_sync(0xffffffffu, ok && j == 0);  // tile with no skip at all
-    if (NG > 1) {  // whole-row sums from the groups' partial sums (every softmax thread passes here)
-      xsum[g * BM + r] = l_sum;
-      xsum[NG * BM + g * BM + r] = l_rnd;
-      asm volatile("bar.sync 2, %0;" ::"n"(128 * NG) : "memory");
-      l_sum = 0.f;
-      l_rnd = 0.f;
-#pragma unroll
-      for (int o = 0; o < NG; ++o) {
-        l_sum += xsum[o * BM + r];
-        l_rnd += xsum[NG * BM + o * BM + r];
-      }
-    }
     float lse_log2 = 0.f;
     if (have_o || no_keys) {
       if (have_o) tc_fence_after();
@@ -855,17 +833,17 @@ __global__ void __launch_bounds__(kThreads<D>, kCtasPerSm<D>) fwd_tc_kernel(cons
         wp /= den;
         lse2 = M + log2f(den);
       }
-      float o[OCG];  // this group's columns of the O row, one load
+      float o[D];  // the O row, one load
       if (have_o) {
-        if (OCG == 128) tmem_ld128(tO + lane_off, o);
-        else tmem_ld64(tO + lane_off + g * OCG, o);
+        if (D == 128) tmem_ld128(tO + lane_off, o);
+        else tmem_ld64(tO + lane_off, o);
       } else {
 #pragma unroll
-        for (int e = 0; e < OCG; ++e) o[e] = 0.f;
+        for (int e = 0; e < D; ++e) o[e] = 0.f;
       }
 #pragma unroll
-      for (int cl = 0; cl < OCG / 8; ++cl) {  // 16-byte chunk c of the row
-        const int c = g * (OCG / 8) + cl;
+      for (int cl = 0; cl < D / 8; ++cl) {  // 16-byte chunk c of the row
+        const int c = cl;
         const int blk = c >> 3, cc = c & 7;
         const uint32_t off = blk * (BM * 128) + r * 128 + ((cc ^ (r & 7)) << 4);
         float sp[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
@@ -885,7 +863,7 @@ __global__ void __launch_bounds__(kThreads<D>, kCtasPerSm<D>) fwd_tc_kernel(cons
     }
     // Every softmax warp passes this barrier, epilogue or not (a warp that gave up on a wait must
     // not leave the others blocked here); the tile is then staged whenever it is stored.
-    asm volatile("bar.sync 1, %0;" ::"n"(128 * NG) : "memory");
+    asm volatile("bar.sync 1, 128;" ::: "memory");
     if (have_o || no_keys) {
       if (threadIdx.x == 64) {
 #pragma unroll
@@ -897,7 +875,7 @@ __global__ void __launch_bounds__(kThreads<D>, kCtasPerSm<D>) fwd_tc_kernel(cons
         }
         tma_store_commit_and_wait_read();  // shared memory must outlive the reads of the store
       }
-      if (row_ok && g == 0) {
+      if (row_ok) {
         // a row with no key in this pass (only possible for kResidue) has lse -inf
         const float lse2 = lse_log2;
         const float lse_val = l_sum > 0.f ? lse2 * kLn2 : NEG_INF;
@@ -928,12 +906,12 @@ inline PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 }
 
 // [B*H, n, d] bf16 as a 3-D tensor (d innermost); box = 64 elements x 128 rows x 1.
-inline bool make_map(CUtensorMap* m, const void* ptr, int BH, int n, int d) {
+inline bool make_map(CUtensorMap* m, const void* ptr, int BH, int n, int d, int box_rows) {
   auto fn = encode_fn();
   if (!fn) return false;
   cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)n, (cuuint64_t)BH};
   cuuint64_t strides[2] = {(cuuint64_t)d * 2, (cuuint64_t)n * d * 2};
-  cuuint32_t box[3] = {64, 128, 1};
+  cuuint32_t box[3] = {64, (cuuint32_t)box_rows, 1};
   cuuint32_t estr[3] = {1, 1, 1};
   CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides, box, estr,
                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -942,13 +920,13 @@ inline bool make_map(CUtensorMap* m, const void* ptr, int BH, int n, int d) {
 }
 
 // The residue-class view of [B*H, n, d] with n = T*pi: a 4-D tensor (d, residue, t, bh) in which
-// row t of residue r is sequence row t*pi + r; box = 64 elements x 1 residue x 128 rows x 1.
-inline bool make_residue_map(CUtensorMap* m, const void* ptr, int BH, int n, int d, int pi) {
+// row t of residue r is sequence row t*pi + r; box = 64 elements x 1 residue x box_rows rows x 1.
+inline bool make_residue_map(CUtensorMap* m, const void* ptr, int BH, int n, int d, int pi, int box_rows) {
   auto fn = encode_fn();
   if (!fn) return false;
   cuuint64_t dims[4] = {(cuuint64_t)d, (cuuint64_t)pi, (cuuint64_t)(n / pi), (cuuint64_t)BH};
   cuuint64_t strides[3] = {(cuuint64_t)d * 2, (cuuint64_t)pi * d * 2, (cuuint64_t)n * d * 2};
-  cuuint32_t box[4] = {64, 1, 128, 1};
+  cuuint32_t box[4] = {64, 1, (cuuint32_t)box_rows, 1};
   cuuint32_t estr[4] = {1, 1, 1, 1};
   CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(ptr), dims, strides, box, estr,
                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -995,7 +973,8 @@ cudaError_t launch_fwd_tc_d(const void* q, const void* k, const void* v, const f
   using L = tc::Smem<D>;
   CUtensorMap mq, mk, mv;
   const int BH = B * H;
-  if (!tc::make_map(&mq, q, BH, n, D) || !tc::make_map(&mk, k, BH, n, D) || !tc::make_map(&mv, v, BH, n, D)) {
+  if (!tc::make_map(&mq, q, BH, n, D, tc::BM) || !tc::make_map(&mk, k, BH, n, D, tc::BN) ||
+      !tc::make_map(&mv, v, BH, n, D, tc::BN)) {
     *why = "cuTensorMapEncodeTiled failed";
     return cudaErrorInvalidValue;
   }
@@ -1016,19 +995,19 @@ cudaError_t launch_fwd_tc_d(const void* q, const void* k, const void* v, const f
   const dim3 grid((unsigned)((n + tc::BM - 1) / tc::BM), (unsigned)BH);
   cudaError_t e;
   CUtensorMap mo;
-  if (!tc::make_map(&mo, out, BH, n, D)) {
+  if (!tc::make_map(&mo, out, BH, n, D, tc::BM)) {
     *why = "cuTensorMapEncodeTiled (out) failed";
     return cudaErrorInvalidValue;
   }
   if (!split) {
     if ((e = tc::set_smem_attr<D, tc::kFused>()) != cudaSuccess) { *why = "cudaFuncSetAttribute"; return e; }
-    tc::fwd_tc_kernel<D, tc::kFused><<<grid, tc::kThreads<D>, L::kAlloc, st>>>(mq, mk, mv, mo, mo, p);
+    tc::fwd_tc_kernel<D, tc::kFused><<<grid, tc::kThreads, L::kAlloc, st>>>(mq, mk, mv, mo, mo, p);
     *why = "tensor-core kernel launch";
     return cudaGetLastError();
   }
   CUtensorMap rq, rk, rv;
-  if (!tc::make_residue_map(&rq, q, BH, n, D, pi) || !tc::make_residue_map(&rk, k, BH, n, D, pi) ||
-      !tc::make_residue_map(&rv, v, BH, n, D, pi)) {
+  if (!tc::make_residue_map(&rq, q, BH, n, D, pi, tc::BM) || !tc::make_residue_map(&rk, k, BH, n, D, pi, tc::BN) ||
+      !tc::make_residue_map(&rv, v, BH, n, D, pi, tc::BN)) {
     *why = "cuTensorMapEncodeTiled (residue view) failed";
     return cudaErrorInvalidValue;
   }
@@ -1046,16 +1025,16 @@ cudaError_t launch_fwd_tc_d(const void* q, const void* k, const void* v, const f
   p.skip_o = (__nv_bfloat16*)scratch;
   p.skip_lse = (float*)((char*)scratch + rows * D * 2);
   CUtensorMap rso, mso;  // the skip partials, in the residue view (stored) and the sequence view (loaded)
-  if (!tc::make_residue_map(&rso, p.skip_o, BH, n, D, pi) || !tc::make_map(&mso, p.skip_o, BH, n, D)) {
+  if (!tc::make_residue_map(&rso, p.skip_o, BH, n, D, pi, tc::BM) || !tc::make_map(&mso, p.skip_o, BH, n, D, tc::BM)) {
     if (own) cudaFreeAsync(scratch, st);
     *why = "cuTensorMapEncodeTiled (skip partials) failed";
     return cudaErrorInvalidValue;
   }
   const dim3 grid_r((unsigned)(pi * ((p.T + tc::BM - 1) / tc::BM)), (unsigned)BH);
-  tc::fwd_tc_kernel<D, tc::kResidue><<<grid_r, tc::kThreads<D>, L::kAlloc, st>>>(rq, rk, rv, rso, rso, p);
+  tc::fwd_tc_kernel<D, tc::kResidue><<<grid_r, tc::kThreads, L::kAlloc, st>>>(rq, rk, rv, rso, rso, p);
   e = cudaGetLastError();
   if (e == cudaSuccess) {
-    tc::fwd_tc_kernel<D, tc::kBandMerge><<<grid, tc::kThreads<D>, L::kAlloc, st>>>(mq, mk, mv, mo, mso, p);
+    tc::fwd_tc_kernel<D, tc::kBandMerge><<<grid, tc::kThreads, L::kAlloc, st>>>(mq, mk, mv, mo, mso, p);
     e = cudaGetLastError();
   }
   cudaError_t e2 = own ? cudaFreeAsync(scratch, st) : cudaSuccess;

@@ -1,4 +1,4 @@
-// tile_rule.cuh -- the index rule as the tensor-core kernel applies it, in 128-key tiles.
+// tile_rule.cuh -- the index rule as the tensor-core kernel applies it, in 64-key tiles.
 //
 // Host and device code: the kernel uses it, and a CPU test compiles the same header with g++ to
 // check, for many shapes, that the keys visited and unmasked are exactly L(i) and P(i).
@@ -15,7 +15,7 @@
 
 namespace pia {
 
-constexpr int kTileKeys = 128;  // keys per tile (BN)
+constexpr int kTileKeys = 64;  // keys per tile (BN)
 
 // floor(a / b) for 0 <= a < 2^52, b >= 1, through a double reciprocal of b (rb = 1.0 / b) and
 // an exact +-1 correction -- GPUs have no integer divider, and these run per row and per tile.
@@ -26,7 +26,7 @@ PIA_HD long long div_floor(long long a, long long b, double rb) {
   return q;
 }
 
-// Walks, in increasing order, the 128-key tiles that hold at least one key of the union of L(i)
+// Walks, in increasing order, the key tiles that hold at least one key of the union of L(i)
 // and P(i) over the query rows [i0, last] of one tile.
 struct TileWalk {
   long long i0, last, band_lo;  // query rows [i0, last]; the window keys of the tile start at band_lo
@@ -63,7 +63,7 @@ struct TileWalk {
 };
 
 // For query row i and the key tile starting at j0: window columns [lc_lo, lc_hi] (empty when
-// lc_lo > lc_hi) and a 128-bit mask of skip columns.  Skip columns never overlap the window.
+// lc_lo > lc_hi) and a bitmask of skip columns (kTileKeys bits).  Skip columns never overlap the window.
 // The window of row i is [max(0, i - kwin), i - lo_off]: lo_off = 0 for pi-attention's window;
 // the residue-class pass uses it for the skip band of a residue sequence (kwin = S, lo_off = m0,
 // no skips).  rpi = 1.0 / pi.
@@ -76,7 +76,7 @@ PIA_HD void row_tile_mask(long long i, long long j0, int kwin, int pi, int S, in
   lc_hi = hi > kTileKeys - 1 ? kTileKeys - 1 : (hi < -1 ? -1 : (int)hi);
   for (int w = 0; w < kTileKeys / 32; ++w) sk[w] = 0u;
   if (d0 > kwin && S >= m0) {
-    // skip columns c = d0 - m pi in 0..127: from the largest m (smallest c) upwards in c
+    // skip columns c = d0 - m pi in 0..kTileKeys-1: from the largest m (smallest c) upwards in c
     long long m = div_floor(d0, pi, rpi > 0.0 ? rpi : 1.0 / (double)pi);
     if (m > S) m = S;
     for (long long c = d0 - m * pi; m >= m0 && c < kTileKeys; --m, c += pi) {
