@@ -48,9 +48,6 @@ constexpr int NSB = 2;         // S buffers in TMEM
 template <int D> constexpr int kCtasPerSm = 2;
 constexpr int kThreads = 192;  // warp 0 TMA, warp 1 MMA, warps 2..5 softmax (one query row a thread)
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
-// Pairs of a 32-column window-only chunk whose exponentials run on the FMA pipe (bit e: columns
-// 2e, 2e + 1); the rest use the special-function unit.
-constexpr uint32_t kPolyPairs = 0x4924u;  // every third pair
 
 // ---- shared memory plan (offsets from a 1024-byte aligned base) ---------------------------------
 template <int D>
@@ -294,33 +291,6 @@ __device__ __forceinline__ float ex2(float x) {
   return y;
 }
 
-// 2^x for a pair on the FMA pipe, to take part of the softmax's exponentials off the special-
-// function unit (which runs a quarter of a warp per cycle).  Range reduction after Cody and
-// Waite: n = rint(x) from the low mantissa bits of x + 1.5 * 2^23, f = x - n in [-1/2, 1/2];
-// 2^f from a degree-3 polynomial, minimax in relative error and rounded to fp32 (coefficients
-// from csrc/exp2_poly.py; |relative error| < 7.5e-5, far below the bf16 rounding of P); 2^n is
-// added into the exponent field.  x is clamped at -125 so that the result stays a normal float:
-// anything below 2^-125 comes out as 2^-125, which next to the row's reference (within 2^8 of
-// its maximum) weighs nothing in fp32.
-__device__ __forceinline__ void ex2_poly2(float x0, float x1, float& y0, float& y1) {
-  const unsigned long long kRound = f2pack(12582912.f, 12582912.f);  // 1.5 * 2^23
-  const unsigned long long kNegRound = f2pack(-12582912.f, -12582912.f);
-  const unsigned long long kOne = f2pack(1.f, 1.f), kNegOne = f2pack(-1.f, -1.f);
-  const unsigned long long x = f2pack(fmaxf(x0, -125.f), fmaxf(x1, -125.f));
-  const unsigned long long t = f2add(x, kRound);        // n in the low bits
-  const unsigned long long nf = f2fma(t, kOne, kNegRound);  // n, exactly
-  const unsigned long long f = f2fma(nf, kNegOne, x);    // x - n, exactly
-  unsigned long long q = f2fma(f, f2pack(5.517166853e-02f, 5.517166853e-02f), f2pack(2.426111251e-01f, 2.426111251e-01f));
-  q = f2fma(q, f, f2pack(6.932609677e-01f, 6.932609677e-01f));
-  q = f2fma(q, f, f2pack(9.999280572e-01f, 9.999280572e-01f));
-  float q0, q1, t0, t1;
-  f2unpack(q, q0, q1);
-  f2unpack(t, t0, t1);
-  // bits(t) = bits(1.5 * 2^23) + n, and bits(1.5 * 2^23) << 23 vanishes modulo 2^32
-  y0 = __int_as_float(__float_as_int(q0) + (__float_as_int(t0) << 23));
-  y1 = __int_as_float(__float_as_int(q1) + (__float_as_int(t1) << 23));
-}
-
 // max of three (one instruction on sm_100)
 __device__ __forceinline__ float max3f(float a, float b, float c) {
   float d;
@@ -433,6 +403,18 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm<D>) fwd_tc_kernel(const _
   uint32_t* const tmem_slot = reinterpret_cast<uint32_t*>(sbase + L::kMisc);
   volatile int* const abort_flag = reinterpret_cast<volatile int*>(sbase + L::kMisc + 4);
 
+  // one tile of `rows` rows of the view (r0 ..) into shared memory: D/64 boxes of 64 columns,
+  // each rows x 128 bytes (the map's box has `rows` rows: BM for Q, BN for K and V)
+  auto load_tile = [&](uint32_t dst, const CUtensorMap* map, uint32_t bar, long long r0, int rows) {
+#pragma unroll
+    for (int c = 0; c < D / 64; ++c) {
+      if (MODE == kResidue)
+        tma_load_4d(dst + c * rows * 128, map, bar, c * 64, res, (int)r0, bh);
+      else
+        tma_load_3d(dst + c * rows * 128, map, bar, c * 64, (int)r0, bh);
+    }
+  };
+
   if (threadIdx.x == 0) {
     mbar_init(bar_q, 1);
     for (int s = 0; s < NSTAGE; ++s) {
@@ -451,6 +433,17 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm<D>) fwd_tc_kernel(const _
     mbar_init(bar_so, 1);
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    // the loads that wait for nothing (Q and the first K/V tile) start now, before the TMEM
+    // allocation and the block barrier
+    mbar_expect_tx(bar_q, L::kQBytes);
+    load_tile(sQ, &tmq, bar_q, q0, BM);
+    const int t_first = walk.next(0);
+    if (t_first >= 0) {
+      mbar_expect_tx(bar_kfull(0), L::kKVBytes);
+      load_tile(sK, &tmk, bar_kfull(0), (long long)t_first * BN, BN);
+      mbar_expect_tx(bar_vfull(0), L::kKVBytes);
+      load_tile(sV, &tmv, bar_vfull(0), (long long)t_first * BN, BN);
+    }
   }
   if (warp == 1) {  // TMEM: S buffer b in columns [BN b, BN b + BN), O in [BN NSB, BN NSB + D)
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
@@ -464,26 +457,13 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm<D>) fwd_tc_kernel(const _
   const uint32_t tmem = *tmem_slot;
   const uint32_t tS = tmem, tO = tmem + BN * NSB;  // S buffer b at tS + BN b
 
-  // one tile of `rows` rows of the view (r0 ..) into shared memory: D/64 boxes of 64 columns,
-  // each rows x 128 bytes (the map's box has `rows` rows: BM for Q, BN for K and V)
-  auto load_tile = [&](uint32_t dst, const CUtensorMap* map, uint32_t bar, long long r0, int rows) {
-#pragma unroll
-    for (int c = 0; c < D / 64; ++c) {
-      if (MODE == kResidue)
-        tma_load_4d(dst + c * rows * 128, map, bar, c * 64, res, (int)r0, bh);
-      else
-        tma_load_3d(dst + c * rows * 128, map, bar, c * 64, (int)r0, bh);
-    }
-  };
-
   if (warp == 0) {
     // ------------------------------------------------------------------ TMA producer
     if (lane == 0) {
       constexpr uint32_t kKV = L::kKVBytes;
-      mbar_expect_tx(bar_q, L::kQBytes);
-      load_tile(sQ, &tmq, bar_q, q0, BM);
-      int nk = 0, nv = 0;  // K and V tile loads issued
-      for (int t = walk.next(0); t >= 0; t = walk.next(t + 1)) {
+      const int t_first = walk.next(0);
+      int nk = t_first >= 0 ? 1 : 0, nv = nk;  // K and V tile loads issued (the first one at the start)
+      for (int t = t_first >= 0 ? walk.next(t_first + 1) : -1; t >= 0; t = walk.next(t + 1)) {
         const int s = nk % NSTAGE, use = nk / NSTAGE;
         if (use > 0 && !mbar_wait(bar_kempty(s), (use - 1) & 1, abort_flag)) break;
         mbar_expect_tx(bar_kfull(s), kKV);
@@ -601,9 +581,9 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm<D>) fwd_tc_kernel(const _
     // still in flight.
     float* const wg_s = reinterpret_cast<float*>(sbase + L::kWg);
     if (threadIdx.x - 64 < D) wg_s[threadIdx.x - 64] = prm.w_g[(long long)h * D + (threadIdx.x - 64)];
+    float z = prm.b_g[h];  // in flight with the w_g staging and the Q load
     asm volatile("bar.sync 1, 128;" ::: "memory");
     bool ok = __all_sync(0xffffffffu, mbar_wait(bar_q, 0, abort_flag));
-    float z = prm.b_g[h];
     {
       float zp[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
@@ -691,12 +671,8 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm<D>) fwd_tc_kernel(const _
       }
       const float m_use = m_ref == NEG_INF ? 0.f : m_ref;
 
-      // P.V of tile j - NSB used this S buffer; observing its barrier phase keeps every later wait
-      // on that barrier unambiguous (its P was read before this tile's Q.K^T wrote the buffer).
-      if (j >= NSB && !__all_sync(0xffffffffu, mbar_wait(bar_pvdone(sb), (j / NSB - 1) & 1, abort_flag))) {
-        ok = false;
-        break;
-      }
+      // (P.V of tile j - NSB, which read this buffer's P, has completed: the MMA thread waited for
+      // it before the Q.K^T of this tile.  That also keeps the pv_done waits below unambiguous.)
       if (__any_sync(0xffffffffu, rescale)) {
         // O must hold every earlier tile's P.V before it is rescaled: wait for the P.V of tile j - 1
         if (j >= 1 &&
@@ -763,9 +739,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm<D>) fwd_tc_kernel(const _
             for (int e = 0; e < 32; e += 2) {
               float t0, t1;
               f2unpack(f2fma(f2pack(x[e], x[e + 1]), sc2, bb), t0, t1);
-              float p0, p1;
-              if ((kPolyPairs >> (e >> 1)) & 1u) ex2_poly2(t0, t1, p0, p1);
-              else p0 = ex2(t0), p1 = ex2(t1);
+              const float p0 = ex2(t0), p1 = ex2(t1);
               __nv_bfloat162 b2 = __floats2bfloat162_rn(p0, p1);
               const uint32_t u = *reinterpret_cast<uint32_t*>(&b2);
               pk[e >> 1] = u;
