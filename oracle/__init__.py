@@ -19,6 +19,10 @@ Parity status of each function (what pins it against something other than itself
                                      and skip-only attention); rows sum to 1
   decode                             pinned: equals fwd_rows on the last row of the same sequence,
                                      which is pinned as above
+  bidir=True (two-sided window and    pinned: dense brute force (masks from |i - j|), closed-form
+  skips, every function above but     totals, torch SDPA with the bias, alpha -> 1 = two-sided
+  decode)                             sliding-window attention, reversing the sequence maps the
+                                     operator onto itself
 """
 from __future__ import annotations
 
@@ -51,6 +55,15 @@ def bind(lib):
     i64, vp, i32 = ctypes.c_int64, ctypes.c_void_p, ctypes.c_int
     lib.oracle_index_set.argtypes = [i64, i64, i64, i64, vp, vp, vp, vp]
     lib.oracle_index_set.restype = i64
+    lib.oracle_index_set_ex.argtypes = [i64, i64, i64, i64, i64, i32, vp, vp, vp, vp]
+    lib.oracle_index_set_ex.restype = i64
+    lib.oracle_counts_ex.argtypes = [i64, i64, i64, i64, i32, vp, vp]
+    lib.oracle_counts_ex.restype = None
+    lib.oracle_index_table_ex.argtypes = [i64, i64, i64, i64, i32, i64, vp, vp]
+    lib.oracle_index_table_ex.restype = None
+    lib.oracle_fwd_rows_ex.argtypes = [vp, vp, vp, i32, vp, vp, i64, i64, i64, i64, i64, i64, i64, i32, vp, i64, vp, vp,
+                                       vp, i32]
+    lib.oracle_fwd_rows_ex.restype = None
     lib.oracle_counts.argtypes = [i64, i64, i64, i64, vp, vp]
     lib.oracle_counts.restype = None
     lib.oracle_index_table.argtypes = [i64, i64, i64, i64, i64, vp, vp]
@@ -83,35 +96,41 @@ def _dtype_code(a: np.ndarray) -> int:
     raise TypeError(f"oracle inputs must be float32 or bf16 bits (uint16), got {a.dtype}")
 
 
-def index_set(i: int, kwin: int, pi: int, S: int):
-    """(L(i) ascending, P(i) by increasing m) as int64 arrays."""
-    L = np.empty(kwin + 1, dtype=np.int64)
-    P = np.empty(max(S, 1), dtype=np.int64)
+def index_set(i: int, kwin: int, pi: int, S: int, n: int | None = None, bidir: bool = False):
+    """(L(i) ascending, P(i) by increasing m) as int64 arrays.  bidir: two-sided window and skips in
+    a sequence of n tokens (P lists i - m pi before i + m pi for each m)."""
+    if bidir and n is None:
+        raise ValueError("the bidirectional index rule needs the sequence length n")
+    L = np.empty(2 * kwin + 1, dtype=np.int64)
+    P = np.empty(max(2 * S, 1), dtype=np.int64)
     nL = np.zeros(1, dtype=np.int64)
     nP = np.zeros(1, dtype=np.int64)
-    _lib().oracle_index_set(i, kwin, pi, S, L.ctypes.data, nL.ctypes.data, P.ctypes.data, nP.ctypes.data)
+    _lib().oracle_index_set_ex(i, i + 1 if n is None else n, kwin, pi, S, int(bidir), L.ctypes.data, nL.ctypes.data,
+                               P.ctypes.data, nP.ctypes.data)
     return L[: nL[0]].copy(), P[: nP[0]].copy()
 
 
-def counts(n: int, kwin: int, pi: int, S: int):
+def counts(n: int, kwin: int, pi: int, S: int, bidir: bool = False):
     """(sum_i |L(i)|, sum_i |P(i)|) over i = 0..n-1."""
     a = np.zeros(1, dtype=np.int64)
     b = np.zeros(1, dtype=np.int64)
-    _lib().oracle_counts(n, kwin, pi, S, a.ctypes.data, b.ctypes.data)
+    _lib().oracle_counts_ex(n, kwin, pi, S, int(bidir), a.ctypes.data, b.ctypes.data)
     return int(a[0]), int(b[0])
 
 
-def index_table(n: int, kwin: int, pi: int, S: int, width: int | None = None):
+def index_table(n: int, kwin: int, pi: int, S: int, width: int | None = None, bidir: bool = False):
     """counts [n, 2] int32 and idx [n, width] int32 (L ascending, then P by m, then -1)."""
-    width = kwin + 1 + S if width is None else width
+    if width is None:
+        width = 2 * kwin + 1 + 2 * S if bidir else kwin + 1 + S
     c = np.zeros((n, 2), dtype=np.int32)
     idx = np.zeros((n, width), dtype=np.int32)
-    _lib().oracle_index_table(n, kwin, pi, S, width, c.ctypes.data, idx.ctypes.data)
+    _lib().oracle_index_table_ex(n, kwin, pi, S, int(bidir), width, c.ctypes.data, idx.ctypes.data)
     return c, idx
 
 
-def fwd_rows(q, k, v, w_g, b_g, kwin: int, pi: int, S: int, rows=None, nthreads: int | None = None):
-    """Oracle on selected query rows.
+def fwd_rows(q, k, v, w_g, b_g, kwin: int, pi: int, S: int, rows=None, nthreads: int | None = None,
+             bidir: bool = False):
+    """Oracle on selected query rows (bidir: two-sided window and skips).
 
     q, k, v: [B, H, n, d] float32 or bf16 bits (uint16).  w_g [H, d], b_g [H] float32.
     rows: flat indices (b*H + h)*n + i (default: all rows).
@@ -131,16 +150,16 @@ def fwd_rows(q, k, v, w_g, b_g, kwin: int, pi: int, S: int, rows=None, nthreads:
     out = np.zeros((rows.size, d), dtype=np.float64)
     lse = np.zeros(rows.size, dtype=np.float64)
     rs = np.zeros(rows.size, dtype=np.float64)
-    _lib().oracle_fwd_rows(q.ctypes.data, k.ctypes.data, v.ctypes.data, dt, w_g.ctypes.data, b_g.ctypes.data, B, H, n,
-                           d, kwin, pi, S, rows.ctypes.data, rows.size, out.ctypes.data, lse.ctypes.data, rs.ctypes.data,
-                           _threads(nthreads))
+    _lib().oracle_fwd_rows_ex(q.ctypes.data, k.ctypes.data, v.ctypes.data, dt, w_g.ctypes.data, b_g.ctypes.data, B,
+                              H, n, d, kwin, pi, S, int(bidir), rows.ctypes.data, rows.size, out.ctypes.data,
+                              lse.ctypes.data, rs.ctypes.data, _threads(nthreads))
     return out, lse, rs
 
 
-def fwd(q, k, v, w_g, b_g, kwin: int, pi: int, S: int, nthreads: int | None = None):
+def fwd(q, k, v, w_g, b_g, kwin: int, pi: int, S: int, nthreads: int | None = None, bidir: bool = False):
     """Oracle on every row: out [B, H, n, d], lse [B, H, n], rowsum [B, H, n] (float64)."""
     B, H, n, d = q.shape
-    out, lse, rs = fwd_rows(q, k, v, w_g, b_g, kwin, pi, S, None, nthreads)
+    out, lse, rs = fwd_rows(q, k, v, w_g, b_g, kwin, pi, S, None, nthreads, bidir=bidir)
     return out.reshape(B, H, n, d), lse.reshape(B, H, n), rs.reshape(B, H, n)
 
 

@@ -8,6 +8,7 @@ that idea with the pi-attention pattern and gate:
 
   window mask  W[i, j] = 0 <= i - j <= k                        (dense comparison of positions)
   skip mask    C[i, j] = (i - j) in {pi, 2 pi, ..., S pi},  skip = C and not W
+  bidirectional: W[i, j] = |i - j| <= k,  C[i, j] = |i - j| in {pi, ..., S pi}
                (set difference: a skip key inside the window stays a window key)
   bias         log(alpha_i) on W, log(1 - alpha_i) on skip, -inf elsewhere,
                alpha_i = sigmoid(q_i . w_g + b_g)  (log-sigmoid from scipy)
@@ -21,10 +22,12 @@ import numpy as np
 from scipy.special import log_expit, logsumexp
 
 
-def masks(n: int, kwin: int, pi: int, S: int):
+def masks(n: int, kwin: int, pi: int, S: int, bidir: bool = False):
     """Dense boolean window and skip masks [n, n] (query row, key column)."""
     pos = np.arange(n)
     off = pos[:, None] - pos[None, :]
+    if bidir:
+        off = np.abs(off)
     W = (off >= 0) & (off <= kwin)
     C = np.zeros((n, n), dtype=bool)
     for m in range(1, S + 1):
@@ -39,13 +42,13 @@ def widen(a: np.ndarray) -> np.ndarray:
     return a.astype(np.float64)
 
 
-def attention(q, k, v, w_g, b_g, kwin: int, pi: int, S: int):
+def attention(q, k, v, w_g, b_g, kwin: int, pi: int, S: int, bidir: bool = False):
     """q, k, v [B, H, n, d] (float32 or bf16 bits) -> out [B, H, n, d], lse [B, H, n], bias [B, H, n, n]."""
     q, k, v = widen(q), widen(k), widen(v)
     B, H, n, d = q.shape
     w_g = np.asarray(w_g, dtype=np.float64).reshape(H, d)
     b_g = np.asarray(b_g, dtype=np.float64).reshape(H)
-    W, P = masks(n, kwin, pi, S)
+    W, P = masks(n, kwin, pi, S, bidir)
     z = np.einsum("bhnd,hd->bhn", q, w_g) + b_g[None, :, None]
     log_a = log_expit(z)
     log_1ma = log_expit(-z)

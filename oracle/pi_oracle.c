@@ -13,6 +13,11 @@
  *   window  L(i) = { j : max(0, i-k) <= j <= i }              the token and the k tokens before it
  *   skips   P(i) = { i - m*pi : 1 <= m <= S, m*pi > k, i - m*pi >= 0 }
  *           (a skip that lands inside the window is dropped; its key keeps the window's prior)
+ *
+ *   bidirectional variant (same sections: the window reaches "both forward and backward", and "in
+ *   bidirectional settings" the skips also reach i + pi), for a sequence of n tokens:
+ *   window  L(i) = { j : max(0, i-k) <= j <= min(n-1, i+k) }
+ *   skips   P(i) = { i - m*pi, i + m*pi : 1 <= m <= S, m*pi > k, 0 <= j < n }
  *   gate    z = q_i . w_g[h] + b_g[h],  alpha = sigmoid(z)        (on the unscaled query)
  *           lL = log(alpha),  lP = log(1 - alpha)                  (the log-priors)
  *   logits  s_j = tau * q_i . k_j + lL   for j in L(i)
@@ -46,13 +51,19 @@ static double log_sigmoid(double x) {
     return (x < 0 ? x : 0.0) - log1p(exp(-fabs(x)));
 }
 
-/* The index sets of query row i.  L ascending; P in order of increasing m. */
-int64_t oracle_index_set(int64_t i, int64_t kwin, int64_t pi, int64_t S, int64_t* L, int64_t* nL,
-                         int64_t* P, int64_t* nP) {
+/* The index sets of query row i of a sequence of n tokens.  L ascending; P in order of
+ * increasing m, and for each m the backward key before the forward one (bidir only). */
+int64_t oracle_index_set_ex(int64_t i, int64_t n, int64_t kwin, int64_t pi, int64_t S, int bidir, int64_t* L,
+                            int64_t* nL, int64_t* P, int64_t* nP) {
     int64_t a = i - kwin;
     if (a < 0) a = 0;
+    int64_t b = i;  /* causal: the window ends at the token itself */
+    if (bidir) {
+        b = i + kwin;
+        if (b > n - 1) b = n - 1;
+    }
     int64_t c = 0;
-    for (int64_t j = a; j <= i; ++j) {
+    for (int64_t j = a; j <= b; ++j) {
         if (L) L[c] = j;
         ++c;
     }
@@ -62,20 +73,31 @@ int64_t oracle_index_set(int64_t i, int64_t kwin, int64_t pi, int64_t S, int64_t
         int64_t off = m * pi;
         if (off <= kwin) continue;  /* inside the window: already counted once, as a window key */
         int64_t j = i - off;
-        if (j < 0) break;           /* before the sequence start: no such key */
-        if (P) P[e] = j;
-        ++e;
+        if (j >= 0) {               /* before the sequence start: no such key */
+            if (P) P[e] = j;
+            ++e;
+        }
+        if (bidir && i + off <= n - 1) {  /* past the sequence end: no such key */
+            if (P) P[e] = i + off;
+            ++e;
+        }
     }
     *nP = e;
     return c + e;
 }
 
+/* The causal index sets of query row i (the default operator): L ascending, P by increasing m. */
+int64_t oracle_index_set(int64_t i, int64_t kwin, int64_t pi, int64_t S, int64_t* L, int64_t* nL,
+                         int64_t* P, int64_t* nP) {
+    return oracle_index_set_ex(i, i + 1, kwin, pi, S, 0, L, nL, P, nP);
+}
+
 /* Totals of |L(i)| and |P(i)| over i = 0..n-1, by enumeration. */
-void oracle_counts(int64_t n, int64_t kwin, int64_t pi, int64_t S, int64_t* sumL, int64_t* sumP) {
+void oracle_counts_ex(int64_t n, int64_t kwin, int64_t pi, int64_t S, int bidir, int64_t* sumL, int64_t* sumP) {
     int64_t tl = 0, tp = 0;
     for (int64_t i = 0; i < n; ++i) {
         int64_t a, b;
-        oracle_index_set(i, kwin, pi, S, 0, &a, 0, &b);
+        oracle_index_set_ex(i, n, kwin, pi, S, bidir, 0, &a, 0, &b);
         tl += a;
         tp += b;
     }
@@ -83,15 +105,19 @@ void oracle_counts(int64_t n, int64_t kwin, int64_t pi, int64_t S, int64_t* sumL
     *sumP = tp;
 }
 
+void oracle_counts(int64_t n, int64_t kwin, int64_t pi, int64_t S, int64_t* sumL, int64_t* sumP) {
+    oracle_counts_ex(n, kwin, pi, S, 0, sumL, sumP);
+}
+
 /* Per-row index table: counts[i] = {|L(i)|, |P(i)|}; idx row i holds L(i) ascending, then P(i)
  * by increasing m, then -1 up to `width` entries. */
-void oracle_index_table(int64_t n, int64_t kwin, int64_t pi, int64_t S, int64_t width, int32_t* counts,
-                        int32_t* idx) {
-    int64_t* L = (int64_t*)malloc(sizeof(int64_t) * (size_t)(kwin + 1));
-    int64_t* P = (int64_t*)malloc(sizeof(int64_t) * (size_t)(S + 1));
+void oracle_index_table_ex(int64_t n, int64_t kwin, int64_t pi, int64_t S, int bidir, int64_t width,
+                           int32_t* counts, int32_t* idx) {
+    int64_t* L = (int64_t*)malloc(sizeof(int64_t) * (size_t)(2 * kwin + 1));
+    int64_t* P = (int64_t*)malloc(sizeof(int64_t) * (size_t)(2 * S + 1));
     for (int64_t i = 0; i < n; ++i) {
         int64_t a, b;
-        oracle_index_set(i, kwin, pi, S, L, &a, P, &b);
+        oracle_index_set_ex(i, n, kwin, pi, S, bidir, L, &a, P, &b);
         counts[2 * i] = (int32_t)a;
         counts[2 * i + 1] = (int32_t)b;
         int32_t* row = idx + i * width;
@@ -104,6 +130,11 @@ void oracle_index_table(int64_t n, int64_t kwin, int64_t pi, int64_t S, int64_t 
     free(P);
 }
 
+void oracle_index_table(int64_t n, int64_t kwin, int64_t pi, int64_t S, int64_t width, int32_t* counts,
+                        int32_t* idx) {
+    oracle_index_table_ex(n, kwin, pi, S, 0, width, counts, idx);
+}
+
 /* One query row: q row at qbase (element offset qoff), keys/values of its (b, h) sequence at
  * kvoff (element offset of row 0), query position i.  Writes out[d], *lse, *rowsum. */
 typedef struct {
@@ -111,10 +142,11 @@ typedef struct {
     int dtype;
     const float *w_g, *b_g;
     int64_t H, d, kwin, pi, S;
+    int bidir;  /* 1: two-sided window and skips (prefill only) */
 } problem_t;
 
-static void attend_row(const problem_t* pr, int64_t h, int64_t qoff, int64_t kvoff, int64_t i, double* out,
-                       double* lse, double* rowsum, int64_t* L, int64_t* P, double* s, double* qd) {
+static void attend_row(const problem_t* pr, int64_t h, int64_t qoff, int64_t kvoff, int64_t n, int64_t i,
+                       double* out, double* lse, double* rowsum, int64_t* L, int64_t* P, double* s, double* qd) {
     const int64_t d = pr->d;
     for (int64_t c = 0; c < d; ++c) qd[c] = load_elem(pr->q, qoff + c, pr->dtype);
 
@@ -125,7 +157,7 @@ static void attend_row(const problem_t* pr, int64_t h, int64_t qoff, int64_t kvo
     const double lP = log_sigmoid(-z);  /* log(1 - alpha) */
 
     int64_t nL, nP;
-    oracle_index_set(i, pr->kwin, pr->pi, pr->S, L, &nL, P, &nP);
+    oracle_index_set_ex(i, n, pr->kwin, pr->pi, pr->S, pr->bidir, L, &nL, P, &nP);
     const double tau = 1.0 / sqrt((double)d);
 
     /* biased logits, window keys first, then skip keys */
@@ -166,9 +198,9 @@ typedef struct {
 static void* run_rows(void* arg) {
     rjob_t* jb = (rjob_t*)arg;
     const problem_t* pr = jb->pr;
-    int64_t* L = (int64_t*)malloc(sizeof(int64_t) * (size_t)(pr->kwin + 1));
-    int64_t* P = (int64_t*)malloc(sizeof(int64_t) * (size_t)(pr->S + 1));
-    double* s = (double*)malloc(sizeof(double) * (size_t)(pr->kwin + 1 + pr->S + 1));
+    int64_t* L = (int64_t*)malloc(sizeof(int64_t) * (size_t)(2 * pr->kwin + 1));
+    int64_t* P = (int64_t*)malloc(sizeof(int64_t) * (size_t)(2 * pr->S + 1));
+    double* s = (double*)malloc(sizeof(double) * (size_t)(2 * pr->kwin + 2 * pr->S + 2));
     double* qd = (double*)malloc(sizeof(double) * (size_t)pr->d);
     for (int64_t t = jb->begin; t < jb->end; ++t) {
         int64_t r = jb->rows[t];
@@ -184,8 +216,8 @@ static void* run_rows(void* arg) {
             qoff = r * pr->d;
         }
         int64_t h = bh % pr->H;
-        attend_row(pr, h, qoff, bh * jb->n * pr->d, i, jb->out + t * pr->d, jb->lse + t, jb->rowsum + t, L, P, s,
-                   qd);
+        attend_row(pr, h, qoff, bh * jb->n * pr->d, jb->n, i, jb->out + t * pr->d, jb->lse + t, jb->rowsum + t, L, P,
+                   s, qd);
     }
     free(L);
     free(P);
@@ -222,11 +254,11 @@ static void run_parallel(rjob_t* proto, int64_t total, int nthreads) {
 /* Prefill.  q, k, v: [B, H, n, d] (dtype 0 = fp32, 1 = bf16 bit patterns); w_g [H, d], b_g [H] fp32.
  * rows: flat query rows (b*H + h)*n + i to evaluate (nrows of them).  Outputs, per listed row:
  * out [nrows, d], lse [nrows], rowsum [nrows] (sum of the probabilities, 1 up to rounding). */
-void oracle_fwd_rows(const void* q, const void* k, const void* v, int dtype, const float* w_g, const float* b_g,
-                     int64_t B, int64_t H, int64_t n, int64_t d, int64_t kwin, int64_t pi, int64_t S,
-                     const int64_t* rows, int64_t nrows, double* out, double* lse, double* rowsum, int nthreads) {
+void oracle_fwd_rows_ex(const void* q, const void* k, const void* v, int dtype, const float* w_g, const float* b_g,
+                        int64_t B, int64_t H, int64_t n, int64_t d, int64_t kwin, int64_t pi, int64_t S, int bidir,
+                        const int64_t* rows, int64_t nrows, double* out, double* lse, double* rowsum, int nthreads) {
     (void)B;
-    problem_t pr = {q, k, v, dtype, w_g, b_g, H, d, kwin, pi, S};
+    problem_t pr = {q, k, v, dtype, w_g, b_g, H, d, kwin, pi, S, bidir};
     rjob_t jb;
     memset(&jb, 0, sizeof jb);
     jb.pr = &pr;
@@ -238,6 +270,12 @@ void oracle_fwd_rows(const void* q, const void* k, const void* v, int dtype, con
     run_parallel(&jb, nrows, nthreads);
 }
 
+void oracle_fwd_rows(const void* q, const void* k, const void* v, int dtype, const float* w_g, const float* b_g,
+                     int64_t B, int64_t H, int64_t n, int64_t d, int64_t kwin, int64_t pi, int64_t S,
+                     const int64_t* rows, int64_t nrows, double* out, double* lse, double* rowsum, int nthreads) {
+    oracle_fwd_rows_ex(q, k, v, dtype, w_g, b_g, B, H, n, d, kwin, pi, S, 0, rows, nrows, out, lse, rowsum, nthreads);
+}
+
 /* Decode.  q [B, H, d]; kc, vc [B, H, n_cache, d]; lengths: int32 [B] valid cache lengths (NULL
  * means every sequence holds n_cache tokens).  The query is the token at position length-1, and
  * it attends with the same rule as prefill.  bh: list of (b*H + h) to evaluate. */
@@ -247,7 +285,7 @@ void oracle_decode(const void* q, const void* kc, const void* vc, int dtype, con
                    int nthreads) {
     (void)B;
     /* q is read through qoff = bh*d, keys through kvoff = bh*n_cache*d */
-    problem_t pr = {q, kc, vc, dtype, w_g, b_g, H, d, kwin, pi, S};
+    problem_t pr = {q, kc, vc, dtype, w_g, b_g, H, d, kwin, pi, S, 0};
     rjob_t jb;
     memset(&jb, 0, sizeof jb);
     jb.pr = &pr;

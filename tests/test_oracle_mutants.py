@@ -30,6 +30,11 @@ MUTANTS = {
     "keys_from_values": ("dot += qd[c] * load_elem(pr->k,", "dot += qd[c] * load_elem(pr->v,"),
     "last_skip_dropped": ("for (int64_t m = 1; m <= S; ++m) {", "for (int64_t m = 1; m < S; ++m) {"),
     "unnormalised": ("double p = exp(s[t] - M) / Z;", "double p = exp(s[t] - M);"),
+    # bidirectional variant
+    "bidir_forward_window_short": ("b = i + kwin;", "b = i + kwin - 1;"),
+    "bidir_forward_skips_missing": ("if (bidir && i + off <= n - 1) {", "if (0 && i + off <= n - 1) {"),
+    "bidir_forward_skip_tied_to_backward": ("if (bidir && i + off <= n - 1) {",
+                                            "if (bidir && j >= 0 && i + off <= n - 1) {"),
 }
 
 
@@ -48,6 +53,12 @@ def _pin_calls():
     yield pins.test_gate_closed_form_zero_keys
     yield pins.test_alpha_to_one_is_causal_sliding_window
     yield pins.test_alpha_to_zero_is_skip_only
+    for args in [(256, 8, 16, 2), (100, 12, 4, 9)]:
+        yield lambda a=args: pins.test_bidir_index_totals_closed_form(*a)
+    yield lambda: pins.test_bidir_index_sets_match_dense_masks(48, 5, 7, 9)
+    yield lambda: pins.test_bidir_oracle_matches_dense_brute_force("bf16", 32, 3, 4, 5, 16)
+    yield pins.test_bidir_reversing_the_sequence_reverses_the_result
+    yield pins.test_bidir_alpha_to_one_is_two_sided_sliding_window
 
 
 def _failures(lib):

@@ -237,3 +237,93 @@ def test_decode_equals_last_prefill_row():
     out_p, lse_p, _ = oracle.fwd_rows(q, kk, v, w_g, b_g, k, pi, S, rows=rows)
     np.testing.assert_array_equal(out, out_p)
     np.testing.assert_array_equal(lse, lse_p)
+
+
+# ----------------------------------------------------------------------------------------------
+# bidirectional variant: the window reaches k tokens both ways and the skips also reach i + m pi
+# ----------------------------------------------------------------------------------------------
+
+def _closed_form_totals_bidir(n, k, pi, S):
+    # window: the token, min(i, k) before it, min(n - 1 - i, k) after it; skip m (m pi > k) lands
+    # backward on n - m pi rows and forward on n - m pi rows
+    sum_l = sum(1 + min(i, k) + min(n - 1 - i, k) for i in range(n))
+    sum_p = sum(2 * max(0, n - m * pi) for m in range(1, S + 1) if m * pi > k)
+    return sum_l, sum_p
+
+
+@pytest.mark.parametrize("n,k,pi,S", [
+    (256, 8, 16, 2), (4096, 128, 64, 4), (16, 3, 4, 5), (100, 12, 4, 9), (57, 0, 1, 60), (5, 9, 2, 3),
+    (1, 0, 1, 1), (300, 64, 32, 2),
+])
+def test_bidir_index_totals_closed_form(n, k, pi, S):
+    assert oracle.counts(n, k, pi, S, bidir=True) == _closed_form_totals_bidir(n, k, pi, S)
+
+
+@pytest.mark.parametrize("n,k,pi,S", [
+    (32, 3, 4, 5), (48, 5, 7, 9), (33, 0, 1, 40), (64, 16, 8, 4), (64, 16, 16, 3), (20, 6, 3, 10), (17, 4, 5, 0),
+])
+def test_bidir_index_sets_match_dense_masks(n, k, pi, S):
+    W, P = brute.masks(n, k, pi, S, bidir=True)
+    for i in range(n):
+        L_o, P_o = oracle.index_set(i, k, pi, S, n=n, bidir=True)
+        assert L_o.tolist() == np.nonzero(W[i])[0].tolist()
+        assert sorted(P_o.tolist()) == np.nonzero(P[i])[0].tolist()
+        assert not set(L_o.tolist()) & set(P_o.tolist())
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+@pytest.mark.parametrize("n,k,pi,S,d", [(32, 3, 4, 5, 16), (48, 5, 7, 9, 8), (64, 16, 16, 3, 12), (7, 2, 9, 3, 16)])
+def test_bidir_oracle_matches_dense_brute_force(dtype, n, k, pi, S, d):
+    q, kk, v, w_g, b_g = _inputs(2, 3, n, d, seed=n * 37 + k, dtype=dtype)
+    out, lse, rs = oracle.fwd(q, kk, v, w_g, b_g, k, pi, S, bidir=True)
+    out_b, lse_b, _ = brute.attention(q, kk, v, w_g, b_g, k, pi, S, bidir=True)
+    np.testing.assert_allclose(out, out_b, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(lse, lse_b, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(rs, 1.0, rtol=0, atol=1e-12)
+
+
+def test_bidir_oracle_matches_torch_sdpa():
+    n, k, pi, S, d = 40, 6, 5, 7, 16
+    q, kk, v, w_g, b_g = _inputs(1, 2, n, d, seed=17)
+    _, _, bias = brute.attention(q, kk, v, w_g, b_g, k, pi, S, bidir=True)
+    tq, tk, tv = (torch.from_numpy(brute.widen(x)) for x in (q, kk, v))
+    ref = torch.nn.functional.scaled_dot_product_attention(tq, tk, tv, attn_mask=torch.from_numpy(bias))
+    out, lse, _ = oracle.fwd(q, kk, v, w_g, b_g, k, pi, S, bidir=True)
+    np.testing.assert_allclose(out, ref.numpy(), rtol=0, atol=1e-12)
+    scores = torch.einsum("bhid,bhjd->bhij", tq, tk) / math.sqrt(d) + torch.from_numpy(bias)
+    np.testing.assert_allclose(lse, torch.logsumexp(scores, dim=-1).numpy(), rtol=0, atol=1e-12)
+
+
+def test_bidir_reversing_the_sequence_reverses_the_result():
+    # the two-sided rule is symmetric under i -> n - 1 - i, so reversing q, k, v along the sequence
+    # must reverse out and lse; a one-sided slip (a short forward window, a missing forward skip,
+    # an off-by-one at the sequence end) breaks the symmetry
+    n, k, pi, S, d = 61, 5, 7, 8, 16
+    q, kk, v, w_g, b_g = _inputs(1, 2, n, d, seed=21)
+    out, lse, _ = oracle.fwd(q, kk, v, w_g, b_g, k, pi, S, bidir=True)
+    rev = lambda a: np.ascontiguousarray(a[:, :, ::-1])  # noqa: E731
+    out_r, lse_r, _ = oracle.fwd(rev(q), rev(kk), rev(v), w_g, b_g, k, pi, S, bidir=True)
+    np.testing.assert_allclose(out_r[:, :, ::-1], out, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(lse_r[:, :, ::-1], lse, rtol=0, atol=1e-12)
+
+
+def test_bidir_alpha_to_one_is_two_sided_sliding_window():
+    n, k, d = 64, 6, 16
+    q, kk, v, w_g, _ = _inputs(1, 2, n, d, seed=23)
+    pos = np.arange(n)
+    two_sided = np.abs(pos[:, None] - pos[None, :]) <= k
+    o_ref, lse_ref = _sdpa_masked(q, kk, v, two_sided)
+    out, lse, _ = oracle.fwd(q, kk, v, np.zeros_like(w_g), np.full(2, 60.0, np.float32), k, 4, 9, bidir=True)
+    np.testing.assert_allclose(out, o_ref, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(lse, lse_ref, rtol=0, atol=1e-12)
+
+
+def test_bidir_last_row_equals_causal_last_row_without_forward_keys():
+    # the last row has no key after it, so its two-sided sets are its causal sets
+    n, k, pi, S, d = 50, 4, 6, 7, 8
+    q, kk, v, w_g, b_g = _inputs(1, 2, n, d, seed=29)
+    rows = np.array([n - 1, 2 * n - 1])
+    o_b, l_b, _ = oracle.fwd_rows(q, kk, v, w_g, b_g, k, pi, S, rows=rows, bidir=True)
+    o_c, l_c, _ = oracle.fwd_rows(q, kk, v, w_g, b_g, k, pi, S, rows=rows)
+    np.testing.assert_array_equal(o_b, o_c)
+    np.testing.assert_array_equal(l_b, l_c)
