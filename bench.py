@@ -47,8 +47,11 @@ L2_FLUSH_BYTES = 256 << 20
 # algorithmic work (only keys in the index sets count; no tile padding)
 # ------------------------------------------------------------------------------------------------
 
-def index_totals(n: int, k: int, pi: int, S: int):
+def index_totals(n: int, k: int, pi: int, S: int, bidir: bool = False):
     """Sum over i < n of |L(i)| and |P(i)| (closed forms of the index rule)."""
+    if bidir:  # the token, min(i, k) keys before it and min(n - 1 - i, k) after it; skips both ways
+        before = n * (n - 1) // 2 if n <= k + 1 else k * (k + 1) // 2 + (n - k - 1) * k
+        return n + 2 * before, 2 * sum(max(0, n - m * pi) for m in range(k // pi + 1, S + 1))
     sl = n * (n + 1) // 2 if n <= k + 1 else (k + 1) * (k + 2) // 2 + (n - k - 1) * (k + 1)
     sp = sum(max(0, n - m * pi) for m in range(k // pi + 1, S + 1))
     return sl, sp
@@ -58,7 +61,7 @@ def work(w):
     """(tokens, algorithmic flops, algorithmic HBM bytes) of one step of workload w."""
     es = 2 if w.dtype == "bf16" else 4
     if w.kind == "prefill":
-        sl, sp = index_totals(w.n, w.k, w.pi, w.S)
+        sl, sp = index_totals(w.n, w.k, w.pi, w.S, w.bidir)
         units = w.B * w.H
         flops = units * (4 * w.d * (sl + sp) + 2 * w.d * w.n)
         bytes_ = units * (4 * w.n * w.d * es + 4 * w.n)
@@ -210,7 +213,7 @@ def oracle_sample(w, budget_s: float, seed: int = 0):
         def run(rows):
             t0 = time.perf_counter()
             oracle.fwd_rows(inp["q"], inp["k"], inp["v"], inp["w_g"], inp["b_g"], w.k, w.pi, w.S, rows=rows,
-                            nthreads=threads)
+                            nthreads=threads, bidir=w.bidir)
             return time.perf_counter() - t0
 
         probe = np.sort(rng.choice(total, size=min(total, 4 * threads), replace=False))
@@ -323,8 +326,9 @@ def run_gpu(args):
     if w.kind == "prefill":
         def step():
             pia.pi_attn_fwd(t["q"], t["k"], t["v"], t["w_g"], t["b_g"], w.k, w.pi, w.S, out=out, lse=lse,
-                            path=args.path)  # on the current stream (the capture stream while capturing)
-        launches_per_step, _ = pia.pi_attn_fwd_plan(w.B, w.H, w.n, w.d, w.k, w.pi, w.S, w.dtype, args.path)
+                            path=args.path, bidir=w.bidir)  # on the current stream (the capture stream while capturing)
+        launches_per_step = 1 if w.bidir else pia.pi_attn_fwd_plan(w.B, w.H, w.n, w.d, w.k, w.pi, w.S, w.dtype,
+                                                                   args.path)[0]
     else:
         def step():
             pia.pi_attn_decode(t["q"], t["k"], t["v"], t["w_g"], t["b_g"], w.k, w.pi, w.S, out=out, lse=lse)

@@ -90,6 +90,19 @@ pi_attn_status pi_attn_fwd_ws(const void* q, const void* k, const void* v, const
                               pi_attn_dtype dtype, pi_attn_path path, void* workspace, long long workspace_bytes,
                               void* stream);
 
+/* Bidirectional prefill forward (the non-causal variant).  Cited passage: the Core Components of
+ * the pi-Attention method section -- the local neighbourhood reaches both forward and backward,
+ * and in bidirectional settings the skips also reach i + pi.  Row i of a sequence of n tokens
+ * attends, under one softmax, to
+ *   L(i) = { j : max(0, i - k_win) <= j <= min(n - 1, i + k_win) }        prior log(alpha)
+ *   P(i) = { i - m*pi, i + m*pi : 1 <= m <= S, m*pi > k_win, 0 <= key < n } prior log(1 - alpha)
+ * Same arguments, layouts, ownership and errors as pi_attn_fwd_ex; PI_ATTN_PATH_TC_SPLIT returns
+ * PI_ATTN_EUNSUPPORTED (the residue split covers the causal rule only) and the other paths
+ * allocate nothing. */
+pi_attn_status pi_attn_fwd_bidir(const void* q, const void* k, const void* v, const float* w_g, const float* b_g,
+                                 void* out, float* lse, int B, int H, int n, int d, int k_win, int pi, int S,
+                                 pi_attn_dtype dtype, pi_attn_path path, void* stream);
+
 /* What a pi_attn_fwd_ex call with these arguments would launch, without launching anything:
  * *launches = number of kernel launches (1 for a single pass, 2 for the split), *scratch_bytes =
  * device scratch it needs (0 for a single pass): taken from cudaMallocAsync on the stream, or the
@@ -144,6 +157,11 @@ pi_attn_status pi_attn_decode_noalloc(const void* q, const void* kcache, const v
  * width must be >= k_win + 1 + S.  Both are device pointers. */
 pi_attn_status pi_attn_debug_index_sets(int n, int k_win, int pi, int S, int* counts, int* idx, int width,
                                         void* stream);
+
+/* pi_attn_debug_index_sets for the bidirectional rule (see pi_attn_fwd_bidir): L(i) ascending, then
+ * P(i) by increasing m with i - m*pi before i + m*pi.  width must be >= 2*k_win + 1 + 2*S. */
+pi_attn_status pi_attn_debug_index_sets_bidir(int n, int k_win, int pi, int S, int* counts, int* idx, int width,
+                                              void* stream);
 
 /* Synchronises `stream`, then reads and clears the device error word of the current device.
  * Returns PI_ATTN_EDEVICE if any kernel set it since the last check (pi_attn_last_error() then

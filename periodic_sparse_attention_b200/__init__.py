@@ -27,6 +27,8 @@ SIGNATURES = {
     "pi_attn_fwd": (_i32, [_vp] * 7 + [_i32] * 8 + [_vp]),
     # ... as above plus the path selector
     "pi_attn_fwd_ex": (_i32, [_vp] * 7 + [_i32] * 9 + [_vp]),
+    # as pi_attn_fwd_ex, bidirectional index rule
+    "pi_attn_fwd_bidir": (_i32, [_vp] * 7 + [_i32] * 9 + [_vp]),
     # ... plus workspace pointer and its size in bytes
     "pi_attn_fwd_ws": (_i32, [_vp] * 7 + [_i32] * 9 + [_vp, ctypes.c_longlong, _vp]),
     # B H n d k_win pi S, dtype, path, out: launches, scratch bytes
@@ -36,6 +38,7 @@ SIGNATURES = {
     # as pi_attn_decode; no allocation (fixed 4 MiB device scratch inside the library)
     "pi_attn_decode_noalloc": (_i32, [_vp] * 8 + [_i32] * 8 + [_vp]),
     "pi_attn_debug_index_sets": (_i32, [_i32, _i32, _i32, _i32, _vp, _vp, _i32, _vp]),
+    "pi_attn_debug_index_sets_bidir": (_i32, [_i32, _i32, _i32, _i32, _vp, _vp, _i32, _vp]),
     "pi_attn_check": (_i32, [_vp]),
     "pi_attn_status_string": (_cstr, [_i32]),
     "pi_attn_last_error": (_cstr, []),
@@ -107,11 +110,11 @@ _plans = {}
 
 
 def pi_attn_fwd(q, k, v, w_g, b_g, k_win: int, pi: int, S: int, out=None, lse=None, *, path: str = "auto",
-                stream=None, want_lse: bool = True, workspace=None):
+                stream=None, want_lse: bool = True, workspace=None, bidir: bool = False):
     """Prefill forward on torch CUDA tensors q, k, v [B, H, n, d] (fp32 or bf16), w_g [H, d] and
     b_g [H] (fp32).  Allocates out (q's dtype) and lse (fp32 [B, H, n]) when not given, and the
     split path's workspace (a uint8 tensor of pi_attn_fwd_plan's scratch bytes) from torch's
-    caching allocator when not given."""
+    caching allocator when not given.  bidir: the bidirectional rule (pi_attn_fwd_bidir)."""
     import torch
     B, H, n, d = q.shape
     if out is None:
@@ -119,6 +122,11 @@ def pi_attn_fwd(q, k, v, w_g, b_g, k_win: int, pi: int, S: int, out=None, lse=No
     if lse is None and want_lse:
         lse = torch.empty((B, H, n), dtype=torch.float32, device=q.device)
     dt = _dtype_code(q)
+    if bidir:
+        st = load().pi_attn_fwd_bidir(_ptr(q), _ptr(k), _ptr(v), _ptr(w_g), _ptr(b_g), _ptr(out), _ptr(lse), B, H, n,
+                                      d, k_win, pi, S, dt, PATHS[path], _stream(stream))
+        _raise(st)
+        return out, lse
     key = (B, H, n, d, k_win, pi, S, dt, path)
     scratch = _plans.get(key)
     if scratch is None:
@@ -179,13 +187,15 @@ def pi_attn_decode_noalloc(q, kcache, vcache, w_g, b_g, k_win: int, pi: int, S: 
 
 
 def pi_attn_debug_index_sets(n: int, k_win: int, pi: int, S: int, width: int | None = None, device="cuda",
-                             stream=None):
+                             stream=None, bidir: bool = False):
     """Index sets as the kernels enumerate them: counts [n, 2] and idx [n, width] int32 tensors."""
     import torch
-    width = k_win + 1 + S if width is None else width
+    if width is None:
+        width = 2 * k_win + 1 + 2 * S if bidir else k_win + 1 + S
     counts = torch.empty((n, 2), dtype=torch.int32, device=device)
     idx = torch.empty((n, width), dtype=torch.int32, device=device)
-    st = load().pi_attn_debug_index_sets(n, k_win, pi, S, _ptr(counts), _ptr(idx), width, _stream(stream))
+    fn = load().pi_attn_debug_index_sets_bidir if bidir else load().pi_attn_debug_index_sets
+    st = fn(n, k_win, pi, S, _ptr(counts), _ptr(idx), width, _stream(stream))
     _raise(st)
     return counts, idx
 

@@ -5,6 +5,8 @@
 // cover.  Per query row it walks the window keys, then the skip keys, with an online softmax in
 // the log2 domain (scores pre-multiplied by tau*log2(e), priors by log2(e)), so the union is
 // normalised by one running max and one running sum -- a single softmax over L(i) and P(i).
+// `bidir` (prefill only) selects the bidirectional rule: the window reaches k tokens both ways
+// and each m has a forward skip i + m*pi as well, up to the sequence end.
 #pragma once
 #include "common.cuh"
 
@@ -14,7 +16,7 @@ template <typename T, bool DECODE>
 __global__ void __launch_bounds__(256) simt_attn_kernel(
     const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v, const float* __restrict__ w_g,
     const float* __restrict__ b_g, const int* __restrict__ cache_len, T* __restrict__ out, float* __restrict__ lse,
-    int B, int H, int n_q, int n_kv, int d, int kwin, int pi, int S, float scale_log2) {
+    int B, int H, int n_q, int n_kv, int d, int kwin, int pi, int S, float scale_log2, bool bidir) {
   const int lane = threadIdx.x & 31;
   const long long task = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   const long long ntask = DECODE ? (long long)B * H : (long long)B * H * n_q;
@@ -87,11 +89,13 @@ __global__ void __launch_bounds__(256) simt_attn_kernel(
     m = mn;
   };
   const long long j0 = i - kwin > 0 ? i - kwin : 0;
-  for (long long j = j0; j <= i; ++j) visit(j, bias_l);
+  const long long j1 = bidir ? (i + kwin < n_kv - 1 ? i + kwin : n_kv - 1) : i;
+  for (long long j = j0; j <= j1; ++j) visit(j, bias_l);
   for (long long mm = first_skip_m(kwin, pi); mm <= S; ++mm) {
-    const long long j = i - mm * pi;
-    if (j < 0) break;
-    visit(j, bias_p);
+    const long long jb = i - mm * pi, jf = i + mm * pi;
+    if (jb >= 0) visit(jb, bias_p);
+    if (bidir && jf < n_kv) visit(jf, bias_p);
+    if (jb < 0 && (!bidir || jf >= n_kv)) break;
   }
 
   const float inv = 1.f / l;
@@ -104,23 +108,31 @@ __global__ void __launch_bounds__(256) simt_attn_kernel(
   if (lse && lane == 0) lse[orow] = (m + log2f(l)) * kLn2;
 }
 
-// Index sets exactly as the kernels enumerate them (window ascending, then skips by m).
-__global__ void index_sets_kernel(int n, int kwin, int pi, int S, int width, int* __restrict__ counts,
+// Index sets exactly as the kernels enumerate them (window ascending, then skips by m; for each m
+// the backward key before the forward one).
+__global__ void index_sets_kernel(int n, int kwin, int pi, int S, int width, bool bidir, int* __restrict__ counts,
                                   int* __restrict__ idx) {
   const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
   if (i >= n) return;
   const long long j0 = i - kwin > 0 ? i - kwin : 0;
+  const long long j1 = bidir ? (i + kwin < n - 1 ? i + kwin : n - 1) : i;
   int w = 0;
   int* row = idx + i * width;
-  for (long long j = j0; j <= i; ++j)
+  for (long long j = j0; j <= j1; ++j)
     if (w < width) row[w++] = (int)j;
-  const int nl = (int)(i - j0 + 1);
+  const int nl = (int)(j1 - j0 + 1);
   int np = 0;
   for (long long mm = first_skip_m(kwin, pi); mm <= S; ++mm) {
-    const long long j = i - mm * pi;
-    if (j < 0) break;
-    if (w < width) row[w++] = (int)j;
-    ++np;
+    const long long jb = i - mm * pi, jf = i + mm * pi;
+    if (jb >= 0) {
+      if (w < width) row[w++] = (int)jb;
+      ++np;
+    }
+    if (bidir && jf < n) {
+      if (w < width) row[w++] = (int)jf;
+      ++np;
+    }
+    if (jb < 0 && (!bidir || jf >= n)) break;
   }
   while (w < width) row[w++] = -1;
   counts[2 * i] = nl;

@@ -337,6 +337,7 @@ struct Params {
   int H, n, kwin, pi, S;
   int T;                  // kResidue: rows per residue class (n / pi)
   float scale_log2;
+  int bidir;              // kFused: the bidirectional index rule (two-sided window, forward skips)
 };
 
 template <int D, int MODE>
@@ -371,13 +372,16 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm<D>) fwd_tc_kernel(const _
     walk.i0 = q0;
     walk.last = (q0 + BM - 1 < prm.T - 1 ? q0 + BM - 1 : prm.T - 1) - m0;
     walk.band_lo = q0 - prm.S > 0 ? q0 - prm.S : 0;
+    walk.band_hi = walk.last;
+    walk.n = prm.T;
     walk.pi = 1;
     walk.S = 0;
     walk.m0 = 1;
+    walk.bidir = false;
     walk.rpi = 1.0;
   } else {
     q0 = (long long)blockIdx.x * BM;
-    walk.init(q0, prm.n, BM, prm.kwin, prm.pi, MODE == kFused ? prm.S : 0);
+    walk.init(q0, prm.n, BM, prm.kwin, prm.pi, MODE == kFused ? prm.S : 0, MODE == kFused && prm.bidir);
   }
   const int view_rows = MODE == kResidue ? prm.T : prm.n;
 
@@ -629,7 +633,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm<D>) fwd_tc_kernel(const _
         row_tile_mask(qi, (long long)t * BN, prm.S, 1, 0, 1, lc_lo, lc_hi, sk, m0);
       else
         row_tile_mask(qi, (long long)t * BN, prm.kwin, prm.pi, MODE == kFused ? prm.S : 0, m0, lc_lo, lc_hi, sk, 0,
-                      walk.rpi);
+                      walk.rpi, MODE == kFused && prm.bidir, prm.n);
       const bool has_win = lc_lo <= lc_hi;
       uint32_t sk_any = 0u;
 #pragma unroll
@@ -943,7 +947,7 @@ inline bool tc_split_preferred(int n, int kwin, int pi, int S) {
 template <int D>
 cudaError_t launch_fwd_tc_d(const void* q, const void* k, const void* v, const float* w_g, const float* b_g,
                             void* out, float* lse, int B, int H, int n, int kwin, int pi, int S, bool split,
-                            void* workspace, cudaStream_t st, const char** why) {
+                            bool bidir, void* workspace, cudaStream_t st, const char** why) {
   using L = tc::Smem<D>;
   CUtensorMap mq, mk, mv;
   const int BH = B * H;
@@ -966,6 +970,7 @@ cudaError_t launch_fwd_tc_d(const void* q, const void* k, const void* v, const f
   p.S = S;
   p.T = n / pi;
   p.scale_log2 = (float)(1.0 / std::sqrt((double)D)) * kLog2e;
+  p.bidir = bidir ? 1 : 0;
   const dim3 grid((unsigned)((n + tc::BM - 1) / tc::BM), (unsigned)BH);
   cudaError_t e;
   CUtensorMap mo;
@@ -1019,11 +1024,11 @@ cudaError_t launch_fwd_tc_d(const void* q, const void* k, const void* v, const f
 // mode: 0 = choose, 1 = single pass, 2 = split (residue pass + window pass)
 inline cudaError_t launch_fwd_tc(const void* q, const void* k, const void* v, const float* w_g, const float* b_g,
                                  void* out, float* lse, int B, int H, int n, int d, int kwin, int pi, int S, int mode,
-                                 void* workspace, cudaStream_t st, const char** why) {
-  const bool split = mode == 2 || (mode == 0 && tc_split_preferred(n, kwin, pi, S));
+                                 bool bidir, void* workspace, cudaStream_t st, const char** why) {
+  const bool split = !bidir && (mode == 2 || (mode == 0 && tc_split_preferred(n, kwin, pi, S)));
   if (d == 128)
-    return launch_fwd_tc_d<128>(q, k, v, w_g, b_g, out, lse, B, H, n, kwin, pi, S, split, workspace, st, why);
-  return launch_fwd_tc_d<64>(q, k, v, w_g, b_g, out, lse, B, H, n, kwin, pi, S, split, workspace, st, why);
+    return launch_fwd_tc_d<128>(q, k, v, w_g, b_g, out, lse, B, H, n, kwin, pi, S, split, bidir, workspace, st, why);
+  return launch_fwd_tc_d<64>(q, k, v, w_g, b_g, out, lse, B, H, n, kwin, pi, S, split, bidir, workspace, st, why);
 }
 
 }  // namespace pia

@@ -98,7 +98,7 @@ int num_sms() {
 template <typename T, bool DECODE>
 pi_attn_status launch_simt(const void* q, const void* k, const void* v, const float* w_g, const float* b_g,
                            const int* cache_len, void* out, float* lse, int B, int H, int n_q, int n_kv, int d,
-                           int k_win, int pi, int S, cudaStream_t st) {
+                           int k_win, int pi, int S, cudaStream_t st, bool bidir = false) {
   const long long tasks = DECODE ? (long long)B * H : (long long)B * H * n_q;
   const int warps_per_block = 8;
   const long long blocks = (tasks + warps_per_block - 1) / warps_per_block;
@@ -106,7 +106,7 @@ pi_attn_status launch_simt(const void* q, const void* k, const void* v, const fl
   const float scale_log2 = (float)(1.0 / std::sqrt((double)d)) * pia::kLog2e;
   pia::simt_attn_kernel<T, DECODE><<<(unsigned)blocks, warps_per_block * 32, 0, st>>>(
       (const T*)q, (const T*)k, (const T*)v, w_g, b_g, cache_len, (T*)out, lse, B, H, n_q, n_kv, d, k_win, pi, S,
-      scale_log2);
+      scale_log2, bidir);
   cudaError_t e = cudaGetLastError();
   return e == cudaSuccess ? ok() : cuda_fail(e, "simt kernel launch");
 }
@@ -133,17 +133,19 @@ int pi_attn_version(void) { return 100; }
 // Which kernels a forward call with these arguments runs: *tc (tensor-core path) and *split
 // (residue pass + band-merge pass), after the same checks as the call itself.
 static pi_attn_status fwd_route(int n, int d, int k_win, int pi, int S, pi_attn_dtype dtype, pi_attn_path path,
-                                bool* tc, bool* split) {
+                                bool bidir, bool* tc, bool* split) {
   if (path < PI_ATTN_PATH_AUTO || path > PI_ATTN_PATH_TC_SPLIT) return fail(PI_ATTN_EINVAL, "unknown path %d", (int)path);
   const bool tc_ok = pia::tc_supported(dtype == PI_ATTN_BF16, d, n);
   const bool want_tc = path == PI_ATTN_PATH_TC || path == PI_ATTN_PATH_TC_FUSED || path == PI_ATTN_PATH_TC_SPLIT;
   if (want_tc && !tc_ok)
     return fail(PI_ATTN_EUNSUPPORTED, "tensor-core path covers bf16 with d in {64, 128} (got dtype %d, d %d)",
                 (int)dtype, d);
+  if (path == PI_ATTN_PATH_TC_SPLIT && bidir)
+    return fail(PI_ATTN_EUNSUPPORTED, "the split path covers the causal rule only");
   if (path == PI_ATTN_PATH_TC_SPLIT && !pia::tc_split_applies(n, k_win, pi, S))
     return fail(PI_ATTN_EUNSUPPORTED, "split path needs n %% pi == 0 and at least one skip outside the window");
   *tc = path != PI_ATTN_PATH_SIMT && tc_ok;
-  *split = *tc && (path == PI_ATTN_PATH_TC_SPLIT ||
+  *split = *tc && !bidir && (path == PI_ATTN_PATH_TC_SPLIT ||
                    (path != PI_ATTN_PATH_TC_FUSED && pia::tc_split_preferred(n, k_win, pi, S)));
   return ok();
 }
@@ -152,14 +154,14 @@ static long long fwd_scratch_bytes(int B, int H, int n, int d, bool split) {
   return split ? (long long)B * H * n * (2LL * d + 4) : 0;
 }
 
-pi_attn_status pi_attn_fwd_ws(const void* q, const void* k, const void* v, const float* w_g, const float* b_g,
-                              void* out, float* lse, int B, int H, int n, int d, int k_win, int pi, int S,
-                              pi_attn_dtype dtype, pi_attn_path path, void* workspace, long long workspace_bytes,
-                              void* stream) {
+static pi_attn_status fwd_impl(const void* q, const void* k, const void* v, const float* w_g, const float* b_g,
+                               void* out, float* lse, int B, int H, int n, int d, int k_win, int pi, int S,
+                               pi_attn_dtype dtype, pi_attn_path path, bool bidir, void* workspace,
+                               long long workspace_bytes, void* stream) {
   pi_attn_status st = check_common(q, k, v, w_g, b_g, out, B, H, n, d, k_win, pi, S, dtype);
   if (st != PI_ATTN_OK) return st;
   bool tc = false, split = false;
-  if ((st = fwd_route(n, d, k_win, pi, S, dtype, path, &tc, &split)) != PI_ATTN_OK) return st;
+  if ((st = fwd_route(n, d, k_win, pi, S, dtype, path, bidir, &tc, &split)) != PI_ATTN_OK) return st;
   if (workspace) {
     if (reinterpret_cast<uintptr_t>(workspace) % 16 != 0) return fail(PI_ATTN_EINVAL, "workspace not 16-byte aligned");
     const long long need = fwd_scratch_bytes(B, H, n, d, split);
@@ -170,13 +172,29 @@ pi_attn_status pi_attn_fwd_ws(const void* q, const void* k, const void* v, const
   if (tc) {
     const char* why = nullptr;
     const int mode = split ? 2 : 1;
-    cudaError_t e = pia::launch_fwd_tc(q, k, v, w_g, b_g, out, lse, B, H, n, d, k_win, pi, S, mode, workspace, s, &why);
+    cudaError_t e =
+        pia::launch_fwd_tc(q, k, v, w_g, b_g, out, lse, B, H, n, d, k_win, pi, S, mode, bidir, workspace, s, &why);
     if (e != cudaSuccess) return cuda_fail(e, why ? why : "tensor-core kernel launch");
     return ok();
   }
   if (dtype == PI_ATTN_F32)
-    return launch_simt<float, false>(q, k, v, w_g, b_g, nullptr, out, lse, B, H, n, n, d, k_win, pi, S, s);
-  return launch_simt<__nv_bfloat16, false>(q, k, v, w_g, b_g, nullptr, out, lse, B, H, n, n, d, k_win, pi, S, s);
+    return launch_simt<float, false>(q, k, v, w_g, b_g, nullptr, out, lse, B, H, n, n, d, k_win, pi, S, s, bidir);
+  return launch_simt<__nv_bfloat16, false>(q, k, v, w_g, b_g, nullptr, out, lse, B, H, n, n, d, k_win, pi, S, s,
+                                           bidir);
+}
+
+pi_attn_status pi_attn_fwd_ws(const void* q, const void* k, const void* v, const float* w_g, const float* b_g,
+                              void* out, float* lse, int B, int H, int n, int d, int k_win, int pi, int S,
+                              pi_attn_dtype dtype, pi_attn_path path, void* workspace, long long workspace_bytes,
+                              void* stream) {
+  return fwd_impl(q, k, v, w_g, b_g, out, lse, B, H, n, d, k_win, pi, S, dtype, path, false, workspace,
+                  workspace_bytes, stream);
+}
+
+pi_attn_status pi_attn_fwd_bidir(const void* q, const void* k, const void* v, const float* w_g, const float* b_g,
+                                 void* out, float* lse, int B, int H, int n, int d, int k_win, int pi, int S,
+                                 pi_attn_dtype dtype, pi_attn_path path, void* stream) {
+  return fwd_impl(q, k, v, w_g, b_g, out, lse, B, H, n, d, k_win, pi, S, dtype, path, true, nullptr, 0, stream);
 }
 
 pi_attn_status pi_attn_fwd_ex(const void* q, const void* k, const void* v, const float* w_g, const float* b_g,
@@ -193,7 +211,7 @@ pi_attn_status pi_attn_fwd_plan(int B, int H, int n, int d, int k_win, int pi, i
                                    k_win, pi, S, dtype);
   if (st != PI_ATTN_OK) return st;
   bool tc = false, split = false;
-  if ((st = fwd_route(n, d, k_win, pi, S, dtype, path, &tc, &split)) != PI_ATTN_OK) return st;
+  if ((st = fwd_route(n, d, k_win, pi, S, dtype, path, false, &tc, &split)) != PI_ATTN_OK) return st;
   *launches = split ? 2 : 1;
   *scratch_bytes = fwd_scratch_bytes(B, H, n, d, split);
   return ok();
@@ -334,16 +352,27 @@ pi_attn_status pi_attn_decode_noalloc(const void* q, const void* kcache, const v
   return e == cudaSuccess ? ok() : cuda_fail(e, "decode kernel launch");
 }
 
-pi_attn_status pi_attn_debug_index_sets(int n, int k_win, int pi, int S, int* counts, int* idx, int width,
-                                        void* stream) {
+static pi_attn_status index_sets_impl(int n, int k_win, int pi, int S, int* counts, int* idx, int width, bool bidir,
+                                      void* stream) {
   if (!counts || !idx) return fail(PI_ATTN_EINVAL, "null pointer");
   if (n < 1 || k_win < 0 || pi < 1 || S < 0) return fail(PI_ATTN_EINVAL, "need n >= 1, k_win >= 0, pi >= 1, S >= 0");
-  if ((long long)width < (long long)k_win + 1 + S) return fail(PI_ATTN_EINVAL, "width < k_win + 1 + S");
+  const long long need = bidir ? 2LL * k_win + 1 + 2LL * S : (long long)k_win + 1 + S;
+  if ((long long)width < need) return fail(PI_ATTN_EINVAL, "width %d < %lld", width, need);
   const int threads = 256;
-  pia::index_sets_kernel<<<(n + threads - 1) / threads, threads, 0, as_stream(stream)>>>(n, k_win, pi, S, width,
+  pia::index_sets_kernel<<<(n + threads - 1) / threads, threads, 0, as_stream(stream)>>>(n, k_win, pi, S, width, bidir,
                                                                                           counts, idx);
   cudaError_t e = cudaGetLastError();
   return e == cudaSuccess ? ok() : cuda_fail(e, "index-set kernel launch");
+}
+
+pi_attn_status pi_attn_debug_index_sets(int n, int k_win, int pi, int S, int* counts, int* idx, int width,
+                                        void* stream) {
+  return index_sets_impl(n, k_win, pi, S, counts, idx, width, false, stream);
+}
+
+pi_attn_status pi_attn_debug_index_sets_bidir(int n, int k_win, int pi, int S, int* counts, int* idx, int width,
+                                              void* stream) {
+  return index_sets_impl(n, k_win, pi, S, counts, idx, width, true, stream);
 }
 
 pi_attn_status pi_attn_check(void* stream) {

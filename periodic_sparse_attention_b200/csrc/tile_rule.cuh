@@ -4,6 +4,9 @@
 // check, for many shapes, that the keys visited and unmasked are exactly L(i) and P(i).
 //   window  L(i) = [max(0, i - k), i]
 //   skips   P(i) = { i - m*pi : m0 <= m <= S, i - m*pi >= 0 },  m0 = floor(k / pi) + 1
+// and its bidirectional variant (a sequence of n tokens):
+//   window  L(i) = [max(0, i - k), min(n - 1, i + k)]
+//   skips   P(i) = { i - m*pi, i + m*pi : m0 <= m <= S, 0 <= key < n }
 #pragma once
 #include <stdint.h>
 
@@ -29,23 +32,29 @@ PIA_HD long long div_floor(long long a, long long b, double rb) {
 // Walks, in increasing order, the key tiles that hold at least one key of the union of L(i)
 // and P(i) over the query rows [i0, last] of one tile.
 struct TileWalk {
-  long long i0, last, band_lo;  // query rows [i0, last]; the window keys of the tile start at band_lo
-  int pi, S, m0;
-  double rpi;                   // 1.0 / pi
-  PIA_HD void init(long long i0_, long long n, int rows, int kwin, int pi_, int S_) {
+  // every field has a value before init() (the residue pass sets them one by one)
+  long long i0 = 0, last = -1, band_lo = 0, band_hi = -1;  // query rows [i0, last]; window keys [band_lo, band_hi]
+  long long n = 0;                       // sequence length (bidirectional: forward keys stop at n - 1)
+  int pi = 1, S = 0, m0 = 1;
+  bool bidir = false;
+  double rpi = 1.0;                      // 1.0 / pi
+  PIA_HD void init(long long i0_, long long n_, int rows, int kwin, int pi_, int S_, bool bidir_ = false) {
     i0 = i0_;
-    last = i0_ + rows - 1 < n - 1 ? i0_ + rows - 1 : n - 1;
+    n = n_;
+    last = i0_ + rows - 1 < n_ - 1 ? i0_ + rows - 1 : n_ - 1;
     band_lo = i0_ - kwin > 0 ? i0_ - kwin : 0;
+    band_hi = bidir_ ? (last + kwin < n_ - 1 ? last + kwin : n_ - 1) : last;
     pi = pi_;
     S = S_;
     m0 = kwin / pi_ + 1;
+    bidir = bidir_;
     rpi = 1.0 / (double)pi_;
   }
   // smallest needed key tile index >= t, or -1 when none is left
   PIA_HD int next(int t) const {
     const long long p = (long long)t * kTileKeys;
     long long cand = -1;
-    if (p <= last) cand = p > band_lo ? p : band_lo;
+    if (p <= band_hi) cand = p > band_lo ? p : band_lo;
     // the skip block of m, [i0 - m pi, last - m pi], reaches row p iff m pi <= last - p;
     // the largest such m has the leftmost block
     const long long room = last - p;
@@ -58,6 +67,17 @@ struct TileWalk {
         if (cand < 0 || st < cand) cand = st;
       }
     }
+    // bidirectional: the forward block of m, [i0 + m pi, last + m pi], reaches row p iff
+    // last + m pi >= p; the smallest such m has the leftmost block
+    if (bidir && S >= m0) {
+      long long mf = m0;
+      if (p - last > (long long)m0 * pi) mf = div_floor(p - last + pi - 1, pi, rpi);  // ceil((p - last) / pi)
+      if (mf <= S) {
+        long long st = i0 + mf * pi;
+        if (st < p) st = p;
+        if (st <= n - 1 && (cand < 0 || st < cand)) cand = st;
+      }
+    }
     return cand < 0 ? -1 : (int)(cand / kTileKeys);
   }
 };
@@ -68,10 +88,11 @@ struct TileWalk {
 // the residue-class pass uses it for the skip band of a residue sequence (kwin = S, lo_off = m0,
 // no skips).  rpi = 1.0 / pi.
 PIA_HD void row_tile_mask(long long i, long long j0, int kwin, int pi, int S, int m0, int& lc_lo, int& lc_hi,
-                          uint32_t sk[kTileKeys / 32], int lo_off = 0, double rpi = 0.0) {
+                          uint32_t sk[kTileKeys / 32], int lo_off = 0, double rpi = 0.0, bool bidir = false,
+                          long long n = 0) {
   const long long d0 = i - j0;  // i - j at column 0
   const long long lo = (i - kwin > 0 ? i - kwin : 0) - j0;
-  const long long hi = d0 - lo_off;
+  const long long hi = bidir ? (i + kwin < n - 1 ? i + kwin : n - 1) - j0 : d0 - lo_off;
   lc_lo = lo < 0 ? 0 : (lo > kTileKeys ? kTileKeys : (int)lo);
   lc_hi = hi > kTileKeys - 1 ? kTileKeys - 1 : (hi < -1 ? -1 : (int)hi);
   for (int w = 0; w < kTileKeys / 32; ++w) sk[w] = 0u;
@@ -80,6 +101,14 @@ PIA_HD void row_tile_mask(long long i, long long j0, int kwin, int pi, int S, in
     long long m = div_floor(d0, pi, rpi > 0.0 ? rpi : 1.0 / (double)pi);
     if (m > S) m = S;
     for (long long c = d0 - m * pi; m >= m0 && c < kTileKeys; --m, c += pi) {
+      if (c >= 0) sk[c >> 5] |= 1u << (c & 31);
+    }
+  }
+  if (bidir && S >= m0) {
+    // forward skip columns c = d0 + m pi (key i + m pi < n) in 0..kTileKeys-1, from the smallest m
+    long long m = m0;
+    if (-d0 > (long long)m0 * pi) m = div_floor(-d0 + pi - 1, pi, rpi > 0.0 ? rpi : 1.0 / (double)pi);
+    for (long long c = d0 + m * pi; m <= S && c < kTileKeys && i + m * pi <= n - 1; ++m, c += pi) {
       if (c >= 0) sk[c >> 5] |= 1u << (c & 31);
     }
   }

@@ -143,14 +143,18 @@ class Workload:
     k_scale_every: int = 0
     k_scale_factor: float = 1.0
     sampled_rows: int = 0  # > 0: parity on this many sampled query rows (plus boundary rows)
+    bidir: bool = False    # the bidirectional index rule (two-sided window, skips i +- m*pi)
 
     @property
     def wg_std(self) -> float:
         return 1.0 / math.sqrt(self.d)
 
     def describe(self) -> dict:
-        return {"workload": self.name, "kind": self.kind, "dtype": self.dtype, "B": self.B, "H": self.H,
-                "n": self.n, "d": self.d, "k": self.k, "pi": self.pi, "S": self.S}
+        d = {"workload": self.name, "kind": self.kind, "dtype": self.dtype, "B": self.B, "H": self.H,
+             "n": self.n, "d": self.d, "k": self.k, "pi": self.pi, "S": self.S}
+        if self.bidir:
+            d["bidir"] = True
+        return d
 
 
 WORKLOADS = {
@@ -162,6 +166,8 @@ WORKLOADS = {
                  k_scale_factor=4.0),
         Workload("bf16_n128k", "prefill", "bf16", 1, 32, 131072, 128, 512, 1024, 16, sampled_rows=4096),
         Workload("decode_bf16", "decode", "bf16", 64, 32, 65536, 128, 1024, 2048, 31),
+        # the bf16_n4k recipe under the bidirectional rule (the pages' non-causal variant)
+        Workload("bf16_n4k_bidir", "prefill", "bf16", 1, 8, 4096, 64, 128, 64, 4, bg_std=math.sqrt(0.5), bidir=True),
     ]
 }
 

@@ -102,6 +102,12 @@ def test_workspace_is_checked_before_any_launch(lib):
     assert pia.pi_attn_fwd_plan(1, 2, 4096, 64, 128, 64, 4, "bf16", "tc_split") == (2, need)
 
 
+def test_bidir_split_is_refused_before_any_launch(lib):
+    args = [FAKE] * 7 + [1, 1, 4096, 64, 128, 64, 4, pia.PI_ATTN_BF16, pia.PATHS["tc_split"], None]
+    assert lib.pi_attn_fwd_bidir(*args) == pia.PI_ATTN_EUNSUPPORTED
+    assert lib.pi_attn_debug_index_sets_bidir(16, 4, 4, 2, FAKE, FAKE, 4 + 1 + 2, None) == pia.PI_ATTN_EINVAL  # < 2k+1+2S
+
+
 def test_built_for_sm100a_only():
     cmd = pbuild.command("x.so")
     assert "arch=compute_100a,code=sm_100a" in cmd and "-lineinfo" in cmd

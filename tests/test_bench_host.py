@@ -21,6 +21,11 @@ def test_index_totals_agree_with_oracle_enumeration():
         assert bench.index_totals(w.n, w.k, w.pi, w.S) == oracle.counts(w.n, w.k, w.pi, w.S)
 
 
+def test_index_totals_bidirectional_agree_with_oracle_enumeration():
+    for n, k, pi, S in [(4096, 128, 64, 4), (300, 400, 16, 40), (1, 0, 1, 1), (777, 0, 1, 70), (2000, 100, 300, 9)]:
+        assert bench.index_totals(n, k, pi, S, bidir=True) == oracle.counts(n, k, pi, S, bidir=True)
+
+
 def test_work_of_the_default_workload():
     w = ps.WORKLOADS["bf16_n4k"]
     tokens, flops, bytes_ = bench.work(w)

@@ -9,7 +9,7 @@
 
 using namespace pia;
 
-extern "C" int tile_rule_sets(int n, int kwin, int pi, int S, int width, int32_t* counts, int32_t* idx,
+extern "C" int tile_rule_sets(int n, int kwin, int pi, int S, int bidir, int width, int32_t* counts, int32_t* idx,
                               int64_t* stats) {
   // stats: [0] tiles visited, [1] keys counted twice, [2] chunk-class violations,
   //        [3] tiles visited out of order
@@ -17,7 +17,7 @@ extern "C" int tile_rule_sets(int n, int kwin, int pi, int S, int width, int32_t
   const int BM = 128;
   for (long long i0 = 0; i0 < n; i0 += BM) {
     TileWalk w;
-    w.init(i0, n, BM, kwin, pi, S);
+    w.init(i0, n, BM, kwin, pi, S, bidir != 0);
     int prev = -1;
     for (int t = w.next(0); t >= 0; t = w.next(t + 1)) {
       stats[0]++;
@@ -33,7 +33,7 @@ extern "C" int tile_rule_sets(int n, int kwin, int pi, int S, int width, int32_t
         const long long j0 = (long long)t * kTileKeys;
         int lo, hi;
         uint32_t sk[kTileKeys / 32];
-        row_tile_mask(i, j0, kwin, pi, S, w.m0, lo, hi, sk);
+        row_tile_mask(i, j0, kwin, pi, S, w.m0, lo, hi, sk, 0, 0.0, bidir != 0, n);
         for (int cb = 0; cb < kTileKeys / 32; ++cb) {
           const int cls = chunk_class(cb, lo, hi, sk[cb]);
           int valid = 0, loc_cnt = 0, skp_cnt = 0;
@@ -59,9 +59,13 @@ extern "C" int tile_rule_sets(int n, int kwin, int pi, int S, int width, int32_t
           if (!okc) stats[2]++;
         }
       }
-      // window keys were produced ascending; skips ascending in j -> write by increasing m
+      // window keys were produced ascending; skips ascending in j -> causal: write by increasing m
+      // (descending j); bidirectional: ascending j (the test compares the skip keys as a set)
       int wpos = nl;
-      for (int s = np - 1; s >= 0 && wpos < width; --s) row[wpos++] = skip_keys[s];
+      if (bidir)
+        for (int s = 0; s < np && wpos < width; ++s) row[wpos++] = skip_keys[s];
+      else
+        for (int s = np - 1; s >= 0 && wpos < width; --s) row[wpos++] = skip_keys[s];
       while (wpos < width) row[wpos++] = -1;
       counts[2 * i] = nl;
       counts[2 * i + 1] = np;
