@@ -19,6 +19,8 @@ Parity status of each function (what pins it against something other than itself
                                      and skip-only attention); rows sum to 1
   decode                             pinned: equals fwd_rows on the last row of the same sequence,
                                      which is pinned as above
+  bwd (gradients of a loss through    pinned: central finite differences of fwd (itself pinned);
+  out: dq, dk, dv, dw_g, db_g)        torch autograd through a dense formulation of the operator
   bidir=True (two-sided window and    pinned: dense brute force (masks from |i - j|), closed-form
   skips, every function above but     totals, torch SDPA with the bias, alpha -> 1 = two-sided
   decode)                             sliding-window attention, reversing the sequence maps the
@@ -74,6 +76,9 @@ def bind(lib):
     lib.oracle_decode.argtypes = [vp, vp, vp, i32, vp, vp, vp, i64, i64, i64, i64, i64, i64, i64, vp, i64, vp, vp, vp,
                                   i32]
     lib.oracle_decode.restype = None
+    lib.oracle_bwd.argtypes = [vp, vp, vp, i32, vp, vp, i64, i64, i64, i64, i64, i64, i64, i32, vp, vp, vp, vp, vp, vp,
+                               i32]
+    lib.oracle_bwd.restype = None
     return lib
 
 
@@ -190,3 +195,24 @@ def decode(q, kc, vc, w_g, b_g, kwin: int, pi: int, S: int, lengths=None, bh=Non
                          n_cache, d, kwin, pi, S, bh.ctypes.data, bh.size, out.ctypes.data, lse.ctypes.data,
                          rs.ctypes.data, _threads(nthreads))
     return out, lse, rs
+
+
+def bwd(q, k, v, w_g, b_g, dO, kwin: int, pi: int, S: int, bidir: bool = False, nthreads: int | None = None):
+    """Gradients of a scalar loss through out, given dO = dLoss/dout [B, H, n, d].
+    q, k, v as for fwd.  Returns dq, dk, dv [B, H, n, d], dw_g [H, d], db_g [H] (float64)."""
+    q = np.ascontiguousarray(q)
+    k = np.ascontiguousarray(k)
+    v = np.ascontiguousarray(v)
+    dt = _dtype_code(q)
+    assert _dtype_code(k) == dt and _dtype_code(v) == dt
+    B, H, n, d = q.shape
+    w_g = np.ascontiguousarray(w_g, dtype=np.float32).reshape(H, d)
+    b_g = np.ascontiguousarray(b_g, dtype=np.float32).reshape(H)
+    dO = np.ascontiguousarray(dO, dtype=np.float64).reshape(B, H, n, d)
+    dq, dk, dv = (np.zeros((B, H, n, d), dtype=np.float64) for _ in range(3))
+    dw = np.zeros((H, d), dtype=np.float64)
+    db = np.zeros(H, dtype=np.float64)
+    _lib().oracle_bwd(q.ctypes.data, k.ctypes.data, v.ctypes.data, dt, w_g.ctypes.data, b_g.ctypes.data, B, H, n, d,
+                      kwin, pi, S, int(bidir), dO.ctypes.data, dq.ctypes.data, dk.ctypes.data, dv.ctypes.data,
+                      dw.ctypes.data, db.ctypes.data, _threads(nthreads))
+    return dq, dk, dv, dw, db

@@ -14,6 +14,14 @@
  *   skips   P(i) = { i - m*pi : 1 <= m <= S, m*pi > k, i - m*pi >= 0 }
  *           (a skip that lands inside the window is dropped; its key keeps the window's prior)
  *
+ *   backward (the gradient of a scalar loss through out, given dO = dLoss/dout; not printed on the
+ *   pages -- the chain rule through the forward above, for the training the pages report):
+ *           dp_j = dO_i . v_j,  D_i = sum_j p_j dp_j,  ds_j = p_j (dp_j - D_i)
+ *           dq_i = tau sum_j ds_j k_j + dz_i w_g[h],    dk_j += tau ds_j q_i,   dv_j += p_j dO_i
+ *           dz_i = (1 - alpha) sum_{j in L} ds_j - alpha sum_{j in P} ds_j
+ *                  (d log(alpha)/dz = 1 - alpha, d log(1 - alpha)/dz = -alpha)
+ *           dw_g[h] += dz_i q_i,  db_g[h] += dz_i
+ *
  *   bidirectional variant (same sections: the window reaches "both forward and backward", and "in
  *   bidirectional settings" the skips also reach i + pi), for a sequence of n tokens:
  *   window  L(i) = { j : max(0, i-k) <= j <= min(n-1, i+k) }
@@ -297,4 +305,140 @@ void oracle_decode(const void* q, const void* kc, const void* vc, int dtype, con
     jb.lse = lse;
     jb.rowsum = rowsum;
     run_parallel(&jb, nbh, nthreads);
+}
+
+/* Backward of one (b, h) sequence, every row, in double: accumulates dq [n, d], dk [n, d],
+ * dv [n, d] (zeroed by the caller) and dw [d], db [1] of head h.  Rows in increasing order. */
+static void backward_seq(const problem_t* pr, int64_t n, int64_t h, int64_t base, const double* dO, double* dq,
+                         double* dk, double* dv, double* dw, double* db) {
+    const int64_t d = pr->d;
+    const double tau = 1.0 / sqrt((double)d);
+    int64_t* L = (int64_t*)malloc(sizeof(int64_t) * (size_t)(2 * pr->kwin + 1));
+    int64_t* P = (int64_t*)malloc(sizeof(int64_t) * (size_t)(2 * pr->S + 1));
+    const int64_t cap = 2 * pr->kwin + 2 * pr->S + 2;
+    double* s = (double*)malloc(sizeof(double) * (size_t)cap);
+    double* p = (double*)malloc(sizeof(double) * (size_t)cap);
+    double* qd = (double*)malloc(sizeof(double) * (size_t)d);
+    double* od = (double*)malloc(sizeof(double) * (size_t)d);
+    for (int64_t i = 0; i < n; ++i) {
+        const int64_t qoff = base + i * d;
+        for (int64_t c = 0; c < d; ++c) qd[c] = load_elem(pr->q, qoff + c, pr->dtype);
+        double z = (double)pr->b_g[h];
+        for (int64_t c = 0; c < d; ++c) z += qd[c] * (double)pr->w_g[h * d + c];
+        const double alpha = 1.0 / (1.0 + exp(-z));
+        const double lL = log_sigmoid(z), lP = log_sigmoid(-z);
+        int64_t nL, nP;
+        oracle_index_set_ex(i, n, pr->kwin, pr->pi, pr->S, pr->bidir, L, &nL, P, &nP);
+        const int64_t nU = nL + nP;
+        /* forward of the row: logits, probabilities, output */
+        for (int64_t t = 0; t < nU; ++t) {
+            const int64_t j = t < nL ? L[t] : P[t - nL];
+            double dot = 0.0;
+            for (int64_t c = 0; c < d; ++c) dot += qd[c] * load_elem(pr->k, base + j * d + c, pr->dtype);
+            s[t] = tau * dot + (t < nL ? lL : lP);
+        }
+        double M = -INFINITY;
+        for (int64_t t = 0; t < nU; ++t)
+            if (s[t] > M) M = s[t];
+        double Z = 0.0;
+        for (int64_t t = 0; t < nU; ++t) Z += exp(s[t] - M);
+        for (int64_t c = 0; c < d; ++c) od[c] = 0.0;
+        for (int64_t t = 0; t < nU; ++t) {
+            const int64_t j = t < nL ? L[t] : P[t - nL];
+            p[t] = exp(s[t] - M) / Z;
+            for (int64_t c = 0; c < d; ++c) od[c] += p[t] * load_elem(pr->v, base + j * d + c, pr->dtype);
+        }
+        /* backward of the row */
+        const double* g = dO + i * d;
+        double Dsum = 0.0;
+        for (int64_t c = 0; c < d; ++c) Dsum += g[c] * od[c];
+        double dz = 0.0;
+        for (int64_t t = 0; t < nU; ++t) {
+            const int64_t j = t < nL ? L[t] : P[t - nL];
+            double dpt = 0.0;
+            for (int64_t c = 0; c < d; ++c) dpt += g[c] * load_elem(pr->v, base + j * d + c, pr->dtype);
+            const double ds = p[t] * (dpt - Dsum);
+            dz += t < nL ? (1.0 - alpha) * ds : -alpha * ds;
+            for (int64_t c = 0; c < d; ++c) {
+                dq[i * d + c] += tau * ds * load_elem(pr->k, base + j * d + c, pr->dtype);
+                dk[j * d + c] += tau * ds * qd[c];
+                dv[j * d + c] += p[t] * g[c];
+            }
+        }
+        for (int64_t c = 0; c < d; ++c) {
+            dq[i * d + c] += dz * (double)pr->w_g[h * d + c];
+            dw[c] += dz * qd[c];
+        }
+        *db += dz;
+    }
+    free(L);
+    free(P);
+    free(s);
+    free(p);
+    free(qd);
+    free(od);
+}
+
+typedef struct {
+    const problem_t* pr;
+    int64_t n;
+    const double* dO;
+    double *dq, *dk, *dv, *dw_part, *db_part;  /* dw_part [B*H, d], db_part [B*H] */
+    int64_t begin, end;                        /* (b, h) range */
+} bjob_t;
+
+static void* run_backward(void* arg) {
+    bjob_t* jb = (bjob_t*)arg;
+    const problem_t* pr = jb->pr;
+    const int64_t n = jb->n, d = pr->d;
+    for (int64_t bh = jb->begin; bh < jb->end; ++bh) {
+        const int64_t off = bh * n * d;
+        backward_seq(pr, n, bh % pr->H, off, jb->dO + off, jb->dq + off, jb->dk + off, jb->dv + off,
+                     jb->dw_part + bh * d, jb->db_part + bh);
+    }
+    return 0;
+}
+
+/* Backward.  q, k, v [B, H, n, d] as for oracle_fwd_rows_ex; dO [B, H, n, d] double.  Outputs, all
+ * double and written whole: dq, dk, dv [B, H, n, d], dw_g [H, d], db_g [H] (sums over b and i,
+ * added in increasing b).  Threads split the (b, h) sequences. */
+void oracle_bwd(const void* q, const void* k, const void* v, int dtype, const float* w_g, const float* b_g, int64_t B,
+                int64_t H, int64_t n, int64_t d, int64_t kwin, int64_t pi, int64_t S, int bidir, const double* dO,
+                double* dq, double* dk, double* dv, double* dw_g, double* db_g, int nthreads) {
+    problem_t pr = {q, k, v, dtype, w_g, b_g, H, d, kwin, pi, S, bidir};
+    const int64_t BH = B * H;
+    memset(dq, 0, sizeof(double) * (size_t)(BH * n * d));
+    memset(dk, 0, sizeof(double) * (size_t)(BH * n * d));
+    memset(dv, 0, sizeof(double) * (size_t)(BH * n * d));
+    double* dw_part = (double*)calloc((size_t)(BH * d), sizeof(double));
+    double* db_part = (double*)calloc((size_t)BH, sizeof(double));
+    if (nthreads < 1) nthreads = 1;
+    if (nthreads > MAX_THREADS) nthreads = MAX_THREADS;
+    if (BH < nthreads) nthreads = (int)BH;
+    pthread_t th[MAX_THREADS];
+    int created[MAX_THREADS];
+    bjob_t jobs[MAX_THREADS];
+    const int64_t chunk = (BH + nthreads - 1) / nthreads;
+    for (int t = 0; t < nthreads; ++t) {
+        bjob_t jb = {&pr, n, dO, dq, dk, dv, dw_part, db_part, 0, 0};
+        jb.begin = (int64_t)t * chunk < BH ? (int64_t)t * chunk : BH;
+        jb.end = jb.begin + chunk < BH ? jb.begin + chunk : BH;
+        jobs[t] = jb;
+        created[t] = 0;
+        if (t > 0 && jobs[t].begin < jobs[t].end) created[t] = pthread_create(&th[t], 0, run_backward, &jobs[t]) == 0;
+    }
+    run_backward(&jobs[0]);
+    for (int t = 1; t < nthreads; ++t) {
+        if (created[t]) pthread_join(th[t], 0);
+        else if (jobs[t].begin < jobs[t].end) run_backward(&jobs[t]);
+    }
+    memset(dw_g, 0, sizeof(double) * (size_t)(H * d));
+    memset(db_g, 0, sizeof(double) * (size_t)H);
+    for (int64_t bh = 0; bh < BH; ++bh) {
+        const int64_t h = bh % H;
+        for (int64_t c = 0; c < d; ++c) dw_g[h * d + c] += dw_part[bh * d + c];
+        db_g[h] += db_part[bh];
+    }
+    free(dw_part);
+    free(db_part);
 }

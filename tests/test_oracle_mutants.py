@@ -12,6 +12,7 @@ import subprocess
 import pytest
 
 import oracle
+import tests.test_oracle_backward as bpins
 import tests.test_oracle_pins as pins
 from tests.conftest import read_golden
 
@@ -95,3 +96,46 @@ def test_planted_mistake_is_caught(name, tmp_path):
     assert src.count(old) >= 1, f"mutation site for {name} not found"
     lib = _compile(src.replace(old, new, 1), tmp_path, name)
     assert _failures(lib) >= 1, f"no pin caught the planted mistake {name!r}"
+
+
+# Mistakes planted in the backward (gradients through out); each must fail a backward pin.
+BWD_MUTANTS = {
+    "bwd_gate_term_dropped": ("dq[i * d + c] += dz * (double)pr->w_g[h * d + c];", "dq[i * d + c] += 0.0;"),
+    "bwd_prior_derivatives_swapped": ("dz += t < nL ? (1.0 - alpha) * ds : -alpha * ds;",
+                                      "dz += t < nL ? -alpha * ds : (1.0 - alpha) * ds;"),
+    "bwd_tau_dropped_in_dk": ("dk[j * d + c] += tau * ds * qd[c];", "dk[j * d + c] += ds * qd[c];"),
+    "bwd_dv_from_ds": ("dv[j * d + c] += p[t] * g[c];", "dv[j * d + c] += (p[t] * (dpt - Dsum)) * g[c];"),
+    "bwd_D_dropped": ("const double ds = p[t] * (dpt - Dsum);", "const double ds = p[t] * dpt;"),
+    "bwd_gate_bias_grad_dropped": ("*db += dz;", "*db += 0.0;"),
+}
+
+
+def _bwd_failures(lib):
+    saved = oracle._lib_handle
+    oracle._lib_handle = lib
+    failed = 0
+    calls = [lambda: bpins.test_backward_matches_torch_autograd(40, 5, 7, 4, 8, False),
+             lambda: bpins.test_backward_matches_torch_autograd(20, 30, 3, 5, 8, True),
+             lambda: bpins.test_backward_matches_finite_differences(12, 3, 4, 2, False)]
+    try:
+        for call in calls:
+            try:
+                call()
+            except AssertionError:
+                failed += 1
+    finally:
+        oracle._lib_handle = saved
+    return failed
+
+
+def test_unmodified_backward_passes_its_pins(tmp_path):
+    assert _bwd_failures(_compile(open(SRC).read(), tmp_path, "clean_bwd")) == 0
+
+
+@pytest.mark.parametrize("name", sorted(BWD_MUTANTS))
+def test_planted_backward_mistake_is_caught(name, tmp_path):
+    old, new = BWD_MUTANTS[name]
+    src = open(SRC).read()
+    assert src.count(old) >= 1, f"mutation site for {name} not found"
+    lib = _compile(src.replace(old, new, 1), tmp_path, name)
+    assert _bwd_failures(lib) >= 1, f"no backward pin caught the planted mistake {name!r}"
