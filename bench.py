@@ -41,6 +41,11 @@ import pi_synth as ps  # noqa: E402
 DEFAULT_WORKLOAD = "bf16_n4k"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 L2_FLUSH_BYTES = 256 << 20
+METRICS = {
+    "prefill": "pi-attention fwd tokens/s (and % of roofline), 1xB200",
+    "decode": "pi-attention decode tokens/s (HBM GB/s roofline), 1xB200",
+    "backward": "pi-attention bwd tokens/s (and % of roofline), 1xB200",
+}
 
 
 # ------------------------------------------------------------------------------------------------
@@ -60,6 +65,15 @@ def index_totals(n: int, k: int, pi: int, S: int, bidir: bool = False):
 def work(w):
     """(tokens, algorithmic flops, algorithmic HBM bytes) of one step of workload w."""
     es = 2 if w.dtype == "bf16" else 4
+    if w.kind == "backward":
+        # per (row, key) pair: recompute s, dp = dO.v, dv += p dO, dq += ds k, dk += ds q (2d each);
+        # per row: the gate (2d), its term in dq (2d), dw_g (2d).  Bytes: q, k, v, dO read once,
+        # dq, dk, dv written once (fp32).
+        sl, sp = index_totals(w.n, w.k, w.pi, w.S, w.bidir)
+        units = w.B * w.H
+        flops = units * (10 * w.d * (sl + sp) + 6 * w.d * w.n)
+        bytes_ = units * (4 * w.n * w.d * es + 3 * w.n * w.d * 4)
+        return w.B * w.n, flops, bytes_
     if w.kind == "prefill":
         sl, sp = index_totals(w.n, w.k, w.pi, w.S, w.bidir)
         units = w.B * w.H
@@ -86,6 +100,7 @@ def load_peaks():
 
 KERNEL_FILES = {  # sources of each timed kernel (for matching committed ncu counters to the code)
     "prefill": ["fwd_tc.cuh", "tile_rule.cuh", "common.cuh"],
+    "backward": ["bwd_simt.cuh", "common.cuh"],
     "decode": ["decode.cuh", "common.cuh"],
 }
 
@@ -205,6 +220,23 @@ def oracle_sample(w, budget_s: float, seed: int = 0):
     Returns (tokens per second, sample description, threads, seconds)."""
     import oracle
     threads = max(1, os.cpu_count() or 1)
+    if w.kind == "backward":  # whole (b, h) sequences: as many as the budget allows, at least one
+        inp = ps.backward_inputs(w, seed)
+        widen = (lambda a: (a.astype(np.uint32) << 16).view(np.float32).astype(np.float64)) if w.dtype == "bf16" \
+            else (lambda a: a.astype(np.float64))
+        t0 = time.perf_counter()
+        sub = {x: np.ascontiguousarray(inp[x][:1, :1]) for x in ("q", "k", "v", "dO")}
+        oracle.bwd(sub["q"], sub["k"], sub["v"], inp["w_g"][:1], inp["b_g"][:1], widen(sub["dO"]), w.k, w.pi, w.S,
+                   bidir=w.bidir, nthreads=1)
+        per_seq = max(time.perf_counter() - t0, 1e-6)
+        nh = int(min(w.H, max(1, budget_s * threads / per_seq)))
+        sub = {x: np.ascontiguousarray(inp[x][:1, :nh]) for x in ("q", "k", "v", "dO")}
+        t0 = time.perf_counter()
+        oracle.bwd(sub["q"], sub["k"], sub["v"], inp["w_g"][:nh], inp["b_g"][:nh], widen(sub["dO"]), w.k, w.pi, w.S,
+                   bidir=w.bidir, nthreads=threads)
+        sec = time.perf_counter() - t0
+        desc = f"{nh} of {w.B * w.H} (b, h) sequences, every row"
+        return nh * w.n / w.H / sec, desc, min(threads, nh), sec
     if w.kind == "prefill":
         inp = ps.prefill_inputs(w, seed)
         total = w.B * w.H * w.n
@@ -274,10 +306,11 @@ def device_inputs(w, seed, torch, device):
             return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).to(device).view(torch.bfloat16)
         return torch.from_numpy(np.ascontiguousarray(a)).to(device)
 
-    if w.kind == "prefill":
-        inp = ps.prefill_inputs(w, seed)
-        host = {k: inp[k] for k in ("q", "k", "v", "w_g", "b_g")}
-        t = {k: dev(inp[k], w.dtype) for k in ("q", "k", "v")}
+    if w.kind in ("prefill", "backward"):
+        inp = ps.backward_inputs(w, seed) if w.kind == "backward" else ps.prefill_inputs(w, seed)
+        names = ("q", "k", "v", "dO") if w.kind == "backward" else ("q", "k", "v")
+        host = {k: inp[k] for k in names + ("w_g", "b_g")}
+        t = {k: dev(inp[k], w.dtype) for k in names}
         t["w_g"] = torch.from_numpy(inp["w_g"]).to(device)
         t["b_g"] = torch.from_numpy(inp["b_g"]).to(device)
         return t, host
@@ -319,7 +352,7 @@ def run_gpu(args):
     tokens, flops, bytes_ = work(w)
     t, host = device_inputs(w, args.seed + rank, torch, device)
     out = torch.empty_like(t["q"])
-    lse_shape = (w.B, w.H, w.n) if w.kind == "prefill" else (w.B, w.H)
+    lse_shape = (w.B, w.H) if w.kind == "decode" else (w.B, w.H, w.n)
     lse = torch.empty(lse_shape, dtype=torch.float32, device=device)
     stream = torch.cuda.current_stream(device)
 
@@ -329,6 +362,18 @@ def run_gpu(args):
                             path=args.path, bidir=w.bidir)  # on the current stream (the capture stream while capturing)
         launches_per_step = 1 if w.bidir else pia.pi_attn_fwd_plan(w.B, w.H, w.n, w.d, w.k, w.pi, w.S, w.dtype,
                                                                    args.path)[0]
+    elif w.kind == "backward":
+        grads = (torch.empty(t["q"].shape, dtype=torch.float32, device=device),
+                 torch.empty(t["q"].shape, dtype=torch.float32, device=device),
+                 torch.empty(t["q"].shape, dtype=torch.float32, device=device),
+                 torch.empty((w.H, w.d), dtype=torch.float32, device=device),
+                 torch.empty((w.H,), dtype=torch.float32, device=device))
+        ws = torch.empty(pia.load().pi_attn_bwd_workspace_bytes(w.B, w.H, w.n, w.d), dtype=torch.uint8, device=device)
+
+        def step():
+            pia.pi_attn_bwd(t["q"], t["k"], t["v"], t["w_g"], t["b_g"], t["dO"], w.k, w.pi, w.S, bidir=w.bidir,
+                            grads=grads, workspace=ws)
+        launches_per_step = 4  # row pass, key pass, two gate reduction stages
     else:
         def step():
             pia.pi_attn_decode(t["q"], t["k"], t["v"], t["w_g"], t["b_g"], w.k, w.pi, w.S, out=out, lse=lse)
@@ -394,7 +439,8 @@ def run_gpu(args):
     # The step's inputs come from pinned host memory and its results go back to it.  For decode
     # the KV cache is resident state (like weights); the step's input is the new query.
     e2e = None
-    names = ("q", "k", "v", "w_g", "b_g") if w.kind == "prefill" else ("q", "w_g", "b_g")
+    names = {"prefill": ("q", "k", "v", "w_g", "b_g"), "backward": ("q", "k", "v", "dO", "w_g", "b_g"),
+             "decode": ("q", "w_g", "b_g")}[w.kind]
     pairs = []
     for name in names:
         a = np.ascontiguousarray(host[name])
@@ -402,18 +448,18 @@ def run_gpu(args):
         if a.dtype == np.uint16:  # bf16 bits
             a, dst = a.view(np.int16), dst.view(torch.int16)
         pairs.append((dst, torch.from_numpy(a).pin_memory()))
-    h_out = torch.empty(out.shape, dtype=out.dtype).pin_memory()
-    h_lse = torch.empty(lse.shape, dtype=torch.float32).pin_memory()
+    results = list(grads) if w.kind == "backward" else [out, lse]  # what the step hands back
+    backs = [(r, torch.empty(r.shape, dtype=r.dtype).pin_memory()) for r in results]
     e_steps = max(3, min(args.steps, 50))
     h2d = sum(h.numel() * h.element_size() for _, h in pairs)
-    d2h = h_out.numel() * h_out.element_size() + h_lse.numel() * 4
+    d2h = sum(h.numel() * h.element_size() for _, h in backs)
 
     def e2e_step():
         for dst, src in pairs:
             dst.copy_(src, non_blocking=True)
         step()
-        h_out.copy_(out, non_blocking=True)
-        h_lse.copy_(lse, non_blocking=True)
+        for src, dst in backs:
+            dst.copy_(src, non_blocking=True)
 
     for _ in range(2):
         e2e_step()
@@ -456,8 +502,7 @@ def run_gpu(args):
                "seconds": round(sec, 3)}
 
     line = {
-        "metric": "pi-attention fwd tokens/s (and % of roofline), 1xB200" if w.kind == "prefill"
-        else "pi-attention decode tokens/s (HBM GB/s roofline), 1xB200",
+        "metric": METRICS[w.kind],
         "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": w.dtype, "data": "synthetic (seeded Philox normals, workload recipe)",
@@ -496,8 +541,7 @@ def run_reference(args):
     value = statistics.mean(vals)
     line = {
         "impl": "reference",
-        "metric": "pi-attention fwd tokens/s (and % of roofline), 1xB200" if w.kind == "prefill"
-        else "pi-attention decode tokens/s (HBM GB/s roofline), 1xB200",
+        "metric": METRICS[w.kind],
         "value": value, "unit": "tokens/s", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": statistics.mean(secs) * 1e3, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded Philox normals, workload recipe)",

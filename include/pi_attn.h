@@ -151,6 +151,26 @@ pi_attn_status pi_attn_decode_noalloc(const void* q, const void* kcache, const v
                                       int n_cache, int d, int k_win, int pi, int S, pi_attn_dtype dtype,
                                       void* stream);
 
+/* Backward: the gradients of a scalar loss through out, given dout = dLoss/dout.  Not printed on
+ * the pages; it is the chain rule through the forward (prefill, causal or, with bidir = 1, the
+ * bidirectional rule) that the pages' training results rely on.  With p_ij the softmax weights:
+ *   D_i = dout_i . out_i,  ds_ij = p_ij (dout_i . v_j - D_i)
+ *   dq_i = tau sum_j ds_ij k_j + dz_i w_g[h],  dk_j = tau sum_i ds_ij q_i,  dv_j = sum_i p_ij dout_i
+ *   dz_i = (1 - alpha_i) sum_{j in L(i)} ds_ij - alpha_i sum_{j in P(i)} ds_ij
+ *   dw_g[h] = sum_{b,i} dz_i q_i,  db_g[h] = sum_{b,i} dz_i
+ *   q, k, v, dout   [B, H, n, d] in dtype (read); w_g [H, d], b_g [H] fp32 (read)
+ *   dq, dk, dv      [B, H, n, d] fp32 (written whole, 16-byte aligned)
+ *   dw_g [H, d], db_g [H] fp32 (written whole)
+ *   workspace       device scratch of pi_attn_bwd_workspace_bytes(B, H, n, d) bytes, 16-byte aligned,
+ *                   or NULL (then taken from cudaMallocAsync on the stream and released after)
+ * The forward is recomputed from the inputs; nothing of a forward call is needed.  Results do not
+ * depend on scheduling (no atomics).  Same argument rules and errors as pi_attn_fwd. */
+long long pi_attn_bwd_workspace_bytes(int B, int H, int n, int d);
+pi_attn_status pi_attn_bwd(const void* q, const void* k, const void* v, const float* w_g, const float* b_g,
+                           const void* dout, float* dq, float* dk, float* dv, float* dw_g, float* db_g, int B, int H,
+                           int n, int d, int k_win, int pi, int S, pi_attn_dtype dtype, int bidir, void* workspace,
+                           long long workspace_bytes, void* stream);
+
 /* Index sets as the kernels see them, for exact comparison.  For query rows i = 0..n-1:
  *   counts [n, 2] int32: |L(i)|, |P(i)|
  *   idx    [n, width] int32: L(i) ascending, then P(i) in order of increasing m, then -1.

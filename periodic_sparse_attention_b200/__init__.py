@@ -39,6 +39,9 @@ SIGNATURES = {
     "pi_attn_decode_noalloc": (_i32, [_vp] * 8 + [_i32] * 8 + [_vp]),
     "pi_attn_debug_index_sets": (_i32, [_i32, _i32, _i32, _i32, _vp, _vp, _i32, _vp]),
     "pi_attn_debug_index_sets_bidir": (_i32, [_i32, _i32, _i32, _i32, _vp, _vp, _i32, _vp]),
+    # q k v w_g b_g dout dq dk dv dw_g db_g, B H n d k_win pi S dtype bidir, workspace, bytes, stream
+    "pi_attn_bwd": (_i32, [_vp] * 11 + [_i32] * 9 + [_vp, ctypes.c_longlong, _vp]),
+    "pi_attn_bwd_workspace_bytes": (ctypes.c_longlong, [_i32, _i32, _i32, _i32]),
     "pi_attn_check": (_i32, [_vp]),
     "pi_attn_status_string": (_cstr, [_i32]),
     "pi_attn_last_error": (_cstr, []),
@@ -198,6 +201,32 @@ def pi_attn_debug_index_sets(n: int, k_win: int, pi: int, S: int, width: int | N
     st = fn(n, k_win, pi, S, _ptr(counts), _ptr(idx), width, _stream(stream))
     _raise(st)
     return counts, idx
+
+
+def pi_attn_bwd(q, k, v, w_g, b_g, dout, k_win: int, pi: int, S: int, *, bidir: bool = False, grads=None,
+                workspace=None, stream=None):
+    """Gradients of a loss through out: (dq, dk, dv, dw_g, db_g), fp32 tensors.  q, k, v, dout
+    [B, H, n, d] in one dtype (fp32 or bf16); w_g [H, d], b_g [H] fp32.  grads: a tuple of the five
+    output tensors to write into (allocated when None); workspace from torch's caching allocator
+    when None."""
+    import torch
+    B, H, n, d = q.shape
+    dev = q.device
+    if grads is None:
+        grads = (torch.empty((B, H, n, d), dtype=torch.float32, device=dev),
+                 torch.empty((B, H, n, d), dtype=torch.float32, device=dev),
+                 torch.empty((B, H, n, d), dtype=torch.float32, device=dev),
+                 torch.empty((H, d), dtype=torch.float32, device=dev),
+                 torch.empty((H,), dtype=torch.float32, device=dev))
+    lib = load()
+    if workspace is None:
+        workspace = torch.empty(lib.pi_attn_bwd_workspace_bytes(B, H, n, d), dtype=torch.uint8, device=dev)
+    dq, dk, dv, dw, db = grads
+    st = lib.pi_attn_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(w_g), _ptr(b_g), _ptr(dout), _ptr(dq), _ptr(dk), _ptr(dv),
+                         _ptr(dw), _ptr(db), B, H, n, d, k_win, pi, S, _dtype_code(q), int(bidir), _ptr(workspace),
+                         workspace.numel(), _stream(stream))
+    _raise(st)
+    return dq, dk, dv, dw, db
 
 
 def pi_attn_check(stream=None):

@@ -11,6 +11,7 @@
 
 #include "../../include/pi_attn.h"
 #include "common.cuh"
+#include "bwd_simt.cuh"
 #include "decode.cuh"
 #include "fwd_simt.cuh"
 #include "fwd_tc.cuh"
@@ -373,6 +374,72 @@ pi_attn_status pi_attn_debug_index_sets(int n, int k_win, int pi, int S, int* co
 pi_attn_status pi_attn_debug_index_sets_bidir(int n, int k_win, int pi, int S, int* counts, int* idx, int width,
                                               void* stream) {
   return index_sets_impl(n, k_win, pi, S, counts, idx, width, true, stream);
+}
+
+static long long gate_chunks(int B, int n) {
+  return ((long long)B * n + pia::kGateRows - 1) / pia::kGateRows;
+}
+
+long long pi_attn_bwd_workspace_bytes(int B, int H, int n, int d) {
+  if (B < 1 || H < 1 || n < 1 || d < 1) return 0;
+  // lse2, D, two log2-priors and dz per query row, then the gate's per-chunk partial sums (fp32)
+  return 4LL * (5LL * B * H * n + (long long)H * gate_chunks(B, n) * (d + 1));
+}
+
+pi_attn_status pi_attn_bwd(const void* q, const void* k, const void* v, const float* w_g, const float* b_g,
+                           const void* dout, float* dq, float* dk, float* dv, float* dw_g, float* db_g, int B, int H,
+                           int n, int d, int k_win, int pi, int S, pi_attn_dtype dtype, int bidir, void* workspace,
+                           long long workspace_bytes, void* stream) {
+  pi_attn_status st = check_common(q, k, v, w_g, b_g, dout, B, H, n, d, k_win, pi, S, dtype);
+  if (st != PI_ATTN_OK) return st;
+  if (!dq || !dk || !dv || !dw_g || !db_g) return fail(PI_ATTN_EINVAL, "null gradient pointer");
+  if (!aligned16(dq) || !aligned16(dk) || !aligned16(dv)) return fail(PI_ATTN_EINVAL, "dq, dk, dv must be 16-byte aligned");
+  const long long rows = (long long)B * H * n;
+  const long long need = pi_attn_bwd_workspace_bytes(B, H, n, d);
+  if (workspace) {
+    if (reinterpret_cast<uintptr_t>(workspace) % 16 != 0) return fail(PI_ATTN_EINVAL, "workspace not 16-byte aligned");
+    if (workspace_bytes < need)
+      return fail(PI_ATTN_EINVAL, "workspace of %lld bytes, the backward needs %lld", workspace_bytes, need);
+  }
+  const long long warps_per_block = 8;
+  const long long blocks = (rows + warps_per_block - 1) / warps_per_block;
+  if (blocks > 0x7fffffffLL) return fail(PI_ATTN_EINVAL, "too many query rows");
+  cudaStream_t s = as_stream(stream);
+  void* scratch = workspace;
+  cudaError_t e = cudaSuccess;
+  if (!scratch && (e = cudaMallocAsync(&scratch, (size_t)need, s)) != cudaSuccess)
+    return cuda_fail(e, "backward scratch allocation");
+  float* base = static_cast<float*>(scratch);
+  pia::BwdRowStats rs{base, base + rows, base + 2 * rows, base + 3 * rows, base + 4 * rows};
+  const long long nchunks = gate_chunks(B, n);
+  if (nchunks > 0x7fffffffLL || H > 65535) return fail(PI_ATTN_EINVAL, "too many rows per head for the gate sums");
+  float* part_w = base + 5 * rows;
+  float* part_b = part_w + (long long)H * nchunks * d;
+  const dim3 gg((unsigned)nchunks, (unsigned)H);
+  const float scale_log2 = (float)(1.0 / std::sqrt((double)d)) * pia::kLog2e;
+  const bool bd = bidir != 0;
+  const unsigned g = (unsigned)blocks, tb = (unsigned)(warps_per_block * 32);
+  if (dtype == PI_ATTN_F32) {
+    pia::bwd_row_kernel<float><<<g, tb, 0, s>>>((const float*)q, (const float*)k, (const float*)v, w_g, b_g,
+                                                (const float*)dout, dq, rs, B, H, n, d, k_win, pi, S, scale_log2, bd);
+    pia::bwd_key_kernel<float><<<g, tb, 0, s>>>((const float*)q, (const float*)k, (const float*)v,
+                                                (const float*)dout, rs, dk, dv, B, H, n, d, k_win, pi, S, scale_log2,
+                                                bd);
+    pia::bwd_gate_partial_kernel<float><<<gg, 256, 0, s>>>((const float*)q, rs.dz, part_w, part_b, B, H, n, d);
+  } else {
+    using bf = __nv_bfloat16;
+    pia::bwd_row_kernel<bf><<<g, tb, 0, s>>>((const bf*)q, (const bf*)k, (const bf*)v, w_g, b_g, (const bf*)dout,
+                                             dq, rs, B, H, n, d, k_win, pi, S, scale_log2, bd);
+    pia::bwd_key_kernel<bf><<<g, tb, 0, s>>>((const bf*)q, (const bf*)k, (const bf*)v, (const bf*)dout, rs, dk, dv,
+                                             B, H, n, d, k_win, pi, S, scale_log2, bd);
+    pia::bwd_gate_partial_kernel<bf><<<gg, 256, 0, s>>>((const bf*)q, rs.dz, part_w, part_b, B, H, n, d);
+  }
+  pia::bwd_gate_final_kernel<<<H, 256, 0, s>>>(part_w, part_b, dw_g, db_g, (int)nchunks, d);
+  e = cudaGetLastError();
+  cudaError_t e2 = workspace ? cudaSuccess : cudaFreeAsync(scratch, s);
+  if (e != cudaSuccess) return cuda_fail(e, "backward kernel launch");
+  if (e2 != cudaSuccess) return cuda_fail(e2, "backward scratch release");
+  return ok();
 }
 
 pi_attn_status pi_attn_check(void* stream) {

@@ -41,6 +41,7 @@ _lib_handle = None
 # stream ids: one independent Philox stream per tensor of a workload
 STREAM_Q, STREAM_K, STREAM_V, STREAM_WG, STREAM_BG = 1, 2, 3, 4, 5
 STREAM_DQ, STREAM_DK, STREAM_DV, STREAM_DWG, STREAM_DBG = 11, 12, 13, 14, 15
+STREAM_DO = 6  # the loss gradient of the backward workloads
 
 
 def build(force: bool = False) -> str:
@@ -130,7 +131,7 @@ def f32_to_bf16_bits(a: np.ndarray) -> np.ndarray:
 @dataclasses.dataclass(frozen=True)
 class Workload:
     name: str
-    kind: str            # "prefill" or "decode"
+    kind: str            # "prefill", "decode" or "backward" (gradients through a prefill)
     dtype: str           # "f32" or "bf16": storage type of q, k, v, out
     B: int
     H: int
@@ -168,6 +169,8 @@ WORKLOADS = {
         Workload("decode_bf16", "decode", "bf16", 64, 32, 65536, 128, 1024, 2048, 31),
         # the bf16_n4k recipe under the bidirectional rule (the pages' non-causal variant)
         Workload("bf16_n4k_bidir", "prefill", "bf16", 1, 8, 4096, 64, 128, 64, 4, bg_std=math.sqrt(0.5), bidir=True),
+        # the backward (gradients through out) of the bf16_n4k recipe; dO ~ N(0, 1)
+        Workload("bf16_n4k_bwd", "backward", "bf16", 1, 8, 4096, 64, 128, 64, 4, bg_std=math.sqrt(0.5)),
     ]
 }
 
@@ -192,6 +195,13 @@ def prefill_inputs(w: Workload, seed: int = 0) -> dict:
     v = normal(shp, seed=seed, stream=STREAM_V, dtype=w.dtype)
     w_g, b_g = gate_params(w, seed)
     return {"q": q, "k": k, "v": v, "w_g": w_g, "b_g": b_g}
+
+
+def backward_inputs(w: Workload, seed: int = 0) -> dict:
+    """prefill_inputs plus dO [B, H, n, d] ~ N(0, 1) in the storage dtype (the loss gradient)."""
+    inp = prefill_inputs(w, seed)
+    inp["dO"] = normal((w.B, w.H, w.n, w.d), seed=seed, stream=STREAM_DO, dtype=w.dtype)
+    return inp
 
 
 def decode_positions(n_cache: int, k: int, pi: int, S: int, length: int | None = None) -> np.ndarray:

@@ -108,6 +108,23 @@ def test_bidir_split_is_refused_before_any_launch(lib):
     assert lib.pi_attn_debug_index_sets_bidir(16, 4, 4, 2, FAKE, FAKE, 4 + 1 + 2, None) == pia.PI_ATTN_EINVAL  # < 2k+1+2S
 
 
+def test_backward_rejects_bad_arguments(lib):
+    g = [FAKE] * 5
+    # every call below is refused by the argument checks before anything is launched
+    base = [FAKE] * 6 + g + [1, 2, 64, 64, 8, 16, 2, pia.PI_ATTN_BF16, 0, None, 0, None]
+    bad = list(base)
+    bad[6] = None  # dq
+    assert lib.pi_attn_bwd(*bad) == pia.PI_ATTN_EINVAL
+    bad = list(base)
+    bad[7] = ctypes.c_void_p(0x10008)  # dk misaligned
+    assert lib.pi_attn_bwd(*bad) == pia.PI_ATTN_EINVAL
+    bad = list(base)
+    bad[-3] = FAKE  # a workspace that is too small
+    bad[-2] = 16
+    assert lib.pi_attn_bwd(*bad) == pia.PI_ATTN_EINVAL
+    assert lib.pi_attn_bwd_workspace_bytes(1, 2, 64, 64) == 4 * (5 * 2 * 64 + 2 * 2 * 65)
+
+
 def test_built_for_sm100a_only():
     cmd = pbuild.command("x.so")
     assert "arch=compute_100a,code=sm_100a" in cmd and "-lineinfo" in cmd

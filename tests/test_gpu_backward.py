@@ -1,0 +1,121 @@
+"""The backward (pi_attn_bwd) on the GPU against the fp64 backward oracle (B200 only).
+
+Every element of dq, dk, dv, dw_g and db_g is compared.  Inputs are identical bits on both sides,
+so the differences are the GPU's fp32 accumulation against the oracle's fp64; the bound, written
+here, is a relative L2 error of 1e-4 per gradient and a max-abs error of 1e-3 of the gradient's
+largest magnitude.  The gate gradients dw_g and db_g are sums over every row of dz_i, and dz_i is
+itself a sum that cancels to exactly zero when all of a row's keys carry the same prior (S = 0, or a
+window that holds every key): there the fp32 result is rounding noise around zero, bounded by
+GATE_FLOOR per summed row, and the relative bound does not apply.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import periodic_sparse_attention_b200 as pia
+import pi_synth as ps
+from periodic_sparse_attention_b200 import build as pbuild
+from tests.gpu_util import to_dev
+
+pytestmark = pytest.mark.gpu
+
+REL_L2 = 1e-4
+MAX_ABS_FRAC = 1e-3
+GATE_FLOOR = 1e-6  # per row summed into dw_g / db_g
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _library():
+    pbuild.build()
+    pia.load()
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    yield
+    torch.cuda.synchronize()
+
+
+def _problem(B, H, n, d, dtype, seed):
+    return {"q": ps.normal((B, H, n, d), seed=seed, stream=1, dtype=dtype),
+            "k": ps.normal((B, H, n, d), seed=seed, stream=2, dtype=dtype),
+            "v": ps.normal((B, H, n, d), seed=seed, stream=3, dtype=dtype),
+            "w_g": ps.normal((H, d), seed=seed, stream=4, std=1 / math.sqrt(d), dtype="f32"),
+            "b_g": ps.normal((H,), seed=seed, stream=5, std=0.7, dtype="f32"),
+            "dO": ps.normal((B, H, n, d), seed=seed, stream=6, dtype=dtype)}
+
+
+def _widen(a):
+    return (a.astype(np.uint32) << 16).view(np.float32).astype(np.float64) if a.dtype == np.uint16 else \
+        a.astype(np.float64)
+
+
+def _check(inp, dtype, k, pi, S, bidir, what):
+    dev = {x: to_dev(inp[x], dtype) for x in ("q", "k", "v", "dO")}
+    wg, bg = torch.from_numpy(inp["w_g"]).cuda(), torch.from_numpy(inp["b_g"]).cuda()
+    got = pia.pi_attn_bwd(dev["q"], dev["k"], dev["v"], wg, bg, dev["dO"], k, pi, S, bidir=bidir)
+    pia.pi_attn_check()
+    ref = oracle.bwd(inp["q"], inp["k"], inp["v"], inp["w_g"], inp["b_g"], _widen(inp["dO"]), k, pi, S, bidir=bidir)
+    B, _, n, _ = inp["q"].shape
+    for name, g, r in zip(["dq", "dk", "dv", "dw_g", "db_g"], got, ref):
+        g = g.cpu().numpy().astype(np.float64)
+        assert np.all(np.isfinite(g)), f"{what}: {name} not finite"
+        scale = max(np.max(np.abs(r)), 1e-30)
+        rel = np.linalg.norm(g - r) / max(np.linalg.norm(r), 1e-30)
+        mab = np.max(np.abs(g - r))
+        ok = rel <= REL_L2 and mab <= MAX_ABS_FRAC * scale
+        if name in ("dw_g", "db_g"):
+            ok = ok or mab <= GATE_FLOOR * B * n
+        assert ok, f"{what}: {name} rel-L2 {rel:.3g}, max-abs {mab:.3g}"
+    return got, ref
+
+
+CASES = [  # B, H, n, d, k, pi, S
+    (1, 2, 64, 32, 8, 16, 2),
+    (2, 3, 300, 64, 20, 9, 5),      # ragged, many skips
+    (1, 2, 513, 128, 128, 64, 6),   # ties m*pi == k
+    (1, 1, 1, 64, 0, 1, 1),         # a single token
+    (1, 2, 200, 64, 300, 16, 20),   # window longer than the sequence
+    (1, 1, 150, 32, 5, 1, 30),      # period 1
+    (1, 2, 128, 64, 16, 32, 0),     # no skips
+]
+
+
+@pytest.mark.parametrize("bidir", [False, True])
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+@pytest.mark.parametrize("case", CASES)
+def test_backward_every_element(case, dtype, bidir):
+    B, H, n, d, k, pi, S = case
+    _check(_problem(B, H, n, d, dtype, seed=n + 13 * k), dtype, k, pi, S, bidir, f"{case} {dtype} bidir={bidir}")
+
+
+def test_gate_gradient_cancels_when_every_key_has_one_prior():
+    # S = 0: every key is a window key, log(alpha) shifts every logit alike and cancels, so
+    # dLoss/dz = 0 for every row: the oracle's dw_g and db_g are zero up to fp64 rounding and the
+    # GPU's within the fp32 floor
+    (_, _, _, dw, db), (_, _, _, rdw, rdb) = _check(_problem(1, 2, 128, 64, "f32", seed=9), "f32", 16, 32, 0, False,
+                                                    "S = 0")
+    assert np.max(np.abs(rdw)) < 1e-12 and np.max(np.abs(rdb)) < 1e-12
+    assert float(dw.abs().max()) <= GATE_FLOOR * 128 and float(db.abs().max()) <= GATE_FLOOR * 128
+
+
+def test_backward_head_size_256_fp32():
+    _check(_problem(1, 1, 90, 256, "f32", seed=3), "f32", 12, 7, 4, False, "d = 256")
+
+
+def test_backward_bf16_n4k_workload():
+    w = ps.WORKLOADS["bf16_n4k"]
+    inp = ps.prefill_inputs(w)
+    inp["dO"] = ps.normal((w.B, w.H, w.n, w.d), seed=0, stream=6, dtype="bf16")
+    _check(inp, "bf16", w.k, w.pi, w.S, False, "bf16_n4k")
+
+
+def test_backward_is_deterministic():
+    inp = _problem(2, 2, 400, 64, "bf16", seed=5)
+    dev = {x: to_dev(inp[x], "bf16") for x in ("q", "k", "v", "dO")}
+    wg, bg = torch.from_numpy(inp["w_g"]).cuda(), torch.from_numpy(inp["b_g"]).cuda()
+    a = [t.clone() for t in pia.pi_attn_bwd(dev["q"], dev["k"], dev["v"], wg, bg, dev["dO"], 30, 11, 6)]
+    b = pia.pi_attn_bwd(dev["q"], dev["k"], dev["v"], wg, bg, dev["dO"], 30, 11, 6)
+    pia.pi_attn_check()
+    for x, y in zip(a, b):
+        assert torch.equal(x, y)

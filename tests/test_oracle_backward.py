@@ -80,3 +80,15 @@ def test_backward_matches_torch_autograd(n, kwin, pi, S, d, bidir):
     got = oracle.bwd(q, k, v, w_g, b_g, G, kwin, pi, S, bidir=bidir)
     for name, ref, g in zip(["dq", "dk", "dv", "dw_g", "db_g"], leaves, got):
         np.testing.assert_allclose(g, ref.grad.numpy(), rtol=0, atol=1e-11, err_msg=name)
+
+
+@pytest.mark.parametrize("bidir", [False, True])
+def test_gate_gradient_is_zero_when_one_prior_covers_every_key(bidir):
+    # with S = 0 every key of a row carries log(alpha): the prior shifts all logits alike and cancels
+    # in the softmax, so dLoss/dz = (1 - alpha) sum_j ds_j = (1 - alpha) (D - D) = 0
+    q, k, v, w_g, b_g, G = _problem(2, 3, 40, 8, seed=31)
+    _, _, _, dw, db = oracle.bwd(q, k, v, w_g, b_g, G, 6, 5, 0, bidir=bidir)
+    assert np.max(np.abs(dw)) < 1e-12 and np.max(np.abs(db)) < 1e-12
+    # and it does not vanish once skips are present
+    _, _, _, dw2, db2 = oracle.bwd(q, k, v, w_g, b_g, G, 6, 5, 4, bidir=bidir)
+    assert np.max(np.abs(db2)) > 1e-3
