@@ -7,15 +7,16 @@
 //   dk_j = tau sum_i ds_ij q_i,   dv_j = sum_i p_ij dO_i
 //   dz_i = (1 - alpha_i) sum_{j in L(i)} ds_ij - alpha_i sum_{j in P(i)} ds_ij
 //   dw_g[h] = sum_{b,i} dz_i q_i,   db_g[h] = sum_{b,i} dz_i
-// Three kernels, no atomics (the result does not depend on scheduling):
-//   bwd_row_kernel   one warp per query row: the row's softmax and output (online, fp32), D_i,
+// Kernels, no atomics (the result does not depend on scheduling):
+//   bwd_row_kernel   32 query rows per CTA: each row's softmax and output (online, fp32), D_i,
 //                    then dq_i and dz_i; saves lse_i, D_i, the two log2-priors and dz_i per row
-//   bwd_key_kernel   one warp per key row j: walks the rows that read key j (the index rule read
-//                    backwards) and accumulates dk_j and dv_j
+//   bwd_key_kernel   32 key rows per CTA: the rows that read them (the index rule read
+//                    backwards) accumulate dk_j and dv_j
 //   bwd_gate_*       dw_g and db_g, summed over rows in chunks and then over chunks, in a fixed order
 // Gradients are fp32 whatever the storage type of the inputs.
 #pragma once
 #include "common.cuh"
+#include "tile_rule.cuh"
 
 namespace pia {
 
@@ -28,187 +29,285 @@ struct BwdRowStats {
   float* dz;    // dLoss / dz_i
 };
 
-// Visit the keys of row i in the oracle's order: window ascending, then skips by increasing m
-// (the backward key before the forward one).  f(j, is_window).
-template <typename F>
-__device__ __forceinline__ void for_each_key(long long i, long long n, int kwin, int pi, int S, bool bidir, F&& f) {
-  const long long j0 = i - kwin > 0 ? i - kwin : 0;
-  const long long j1 = bidir ? (i + kwin < n - 1 ? i + kwin : n - 1) : i;
-  for (long long j = j0; j <= j1; ++j) f(j, true);
-  for (long long m = first_skip_m(kwin, pi); m <= S; ++m) {
-    const long long jb = i - m * pi, jf = i + m * pi;
-    if (jb >= 0) f(jb, false);
-    if (bidir && jf < n) f(jf, false);
-    if (jb < 0 && (!bidir || jf >= n)) break;
-  }
-}
+// ---- tiled kernels -------------------------------------------------------------------------------
+// A CTA of 256 threads owns 32 rows (row pass) or 32 keys (key pass); each row or key has 8
+// threads, each holding CPT = ceil(d / 8) of its columns, and dot products are reduced over those 8
+// lanes.  The other operand streams through shared memory in tiles of kTileKeys rows, chosen by the
+// forward's own tile walk (TileWalk: the key tiles a row block reads) or its transpose (ReaderWalk:
+// the row tiles that read a key block), and masked by the forward's row_tile_mask -- the same index
+// sets as the forward, by construction.  Each warp (4 rows or keys) loops over the union of its
+// members' active columns, so every lane takes part in every shuffle.
+constexpr int kBwdThreads = 256;
+constexpr int kBwdTPR = 8;                       // threads per row / key
+constexpr int kBwdRows = kBwdThreads / kBwdTPR;  // rows (or keys) per CTA
 
-// Visit the rows that read key j: row i reads j as a window key when j is in L(i), as a skip key
-// when j is in P(i).  f(i, is_window).
-template <typename F>
-__device__ __forceinline__ void for_each_reader(long long j, long long n, int kwin, int pi, int S, bool bidir, F&& f) {
-  const long long i0 = bidir ? (j - kwin > 0 ? j - kwin : 0) : j;
-  const long long i1 = j + kwin < n - 1 ? j + kwin : n - 1;
-  for (long long i = i0; i <= i1; ++i) f(i, true);
-  for (long long m = first_skip_m(kwin, pi); m <= S; ++m) {
-    const long long ia = j + m * pi, ib = j - m * pi;  // rows after j read it backward; before it, forward
-    if (ia < n) f(ia, false);
-    if (bidir && ib >= 0) f(ib, false);
-    if (ia >= n && (!bidir || ib < 0)) break;
-  }
-}
-
+// Stage rows [r0, r0 + kTileKeys) of a [n, d] matrix into shared memory (zeros past n).
 template <typename T>
-__global__ void __launch_bounds__(256) bwd_row_kernel(const T* __restrict__ q, const T* __restrict__ k,
-                                                      const T* __restrict__ v, const float* __restrict__ w_g,
-                                                      const float* __restrict__ b_g, const T* __restrict__ dout,
-                                                      float* __restrict__ dq, BwdRowStats st, int B, int H, int n,
-                                                      int d, int kwin, int pi, int S, float scale_log2, bool bidir) {
-  const int lane = threadIdx.x & 31;
-  const long long task = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
-  if (task >= (long long)B * H * n) return;
-  const long long bh = task / n, i = task % n;
+__device__ __forceinline__ void stage_tile(T* dst, const T* src, long long r0, long long n, int d) {
+  const int vec = 16 / (int)sizeof(T);  // elements per 16-byte chunk
+  const int per_row = d / vec;
+  for (int idx = threadIdx.x; idx < kTileKeys * per_row; idx += blockDim.x) {
+    const int r = idx / per_row, c = (idx % per_row) * vec;
+    uint4 u = make_uint4(0u, 0u, 0u, 0u);
+    if (r0 + r < n) u = *reinterpret_cast<const uint4*>(src + (r0 + r) * d + c);
+    *reinterpret_cast<uint4*>(dst + r * d + c) = u;
+  }
+}
+
+// The 64 columns of the key tile at j0 that row i reads, as two 32-bit words.
+__device__ __forceinline__ void row_tile_bits(long long i, long long j0, int kwin, int pi, int S, int m0, double rpi,
+                                              bool bidir, long long n, uint32_t& w0, uint32_t& w1) {
+  int lo, hi;
+  uint32_t sk[kTileKeys / 32];
+  row_tile_mask(i, j0, kwin, pi, S, m0, lo, hi, sk, 0, rpi, bidir, n);
+  w0 = window_bits(lo, hi) | sk[0];
+  w1 = window_bits(lo - 32, hi - 32) | sk[1];
+}
+
+template <typename T, int CPT>
+__device__ __forceinline__ float dot_part(const float* a, const T* b, int c0, int d) {
+  float s = 0.f;
+#pragma unroll
+  for (int e = 0; e < CPT; ++e)
+    if (c0 + e < d) s = fmaf(a[e], to_f32(b[c0 + e]), s);
+  return s;
+}
+__device__ __forceinline__ float sum8(float x) {  // over the 8 lanes of a row group (all lanes call)
+  x += __shfl_xor_sync(0xffffffffu, x, 1);
+  x += __shfl_xor_sync(0xffffffffu, x, 2);
+  x += __shfl_xor_sync(0xffffffffu, x, 4);
+  return x;
+}
+
+template <typename T, int CPT>
+__global__ void __launch_bounds__(kBwdThreads) bwd_row_kernel(const T* __restrict__ q, const T* __restrict__ k,
+                                                              const T* __restrict__ v, const float* __restrict__ w_g,
+                                                              const float* __restrict__ b_g,
+                                                              const T* __restrict__ dout, float* __restrict__ dq,
+                                                              BwdRowStats st, int H, int n, int d, int kwin, int pi,
+                                                              int S, float scale_log2, bool bidir) {
+  extern __shared__ __align__(16) uint8_t bwd_smem[];
+  T* ks = reinterpret_cast<T*>(bwd_smem);
+  T* vs = ks + kTileKeys * d;
+  const int tid = threadIdx.x, part = tid & (kBwdTPR - 1), c0 = part * CPT;
+  const long long bh = blockIdx.y;
   const int h = (int)(bh % H);
+  const long long i0 = (long long)blockIdx.x * kBwdRows, i = i0 + tid / kBwdTPR;
+  const bool valid = i < n;
+  const long long row = bh * (long long)n + (valid ? i : 0);
   const T* kb = k + bh * (long long)n * d;
   const T* vb = v + bh * (long long)n * d;
-  float qr[8], gr[8], acc[8];
+  float qr[CPT], gr[CPT], acc[CPT];
 #pragma unroll
-  for (int u = 0; u < 8; ++u) {
-    const int c = lane + 32 * u;
-    qr[u] = c < d ? to_f32(q[task * d + c]) : 0.f;
-    gr[u] = c < d ? to_f32(dout[task * d + c]) : 0.f;
-    acc[u] = 0.f;
+  for (int e = 0; e < CPT; ++e) {
+    const bool in = valid && c0 + e < d;
+    qr[e] = in ? to_f32(q[row * d + c0 + e]) : 0.f;
+    gr[e] = in ? to_f32(dout[row * d + c0 + e]) : 0.f;
+    acc[e] = 0.f;
   }
-  float z = 0.f;
+  float zp = 0.f;
 #pragma unroll
-  for (int u = 0; u < 8; ++u) {
-    const int c = lane + 32 * u;
-    if (c < d) z = fmaf(qr[u], w_g[(long long)h * d + c], z);
-  }
-  z = warp_sum(z) + b_g[h];
+  for (int e = 0; e < CPT; ++e)
+    if (c0 + e < d) zp = fmaf(qr[e], w_g[(long long)h * d + c0 + e], zp);
+  const float z = sum8(zp) + b_g[h];
   const float alpha = 1.f / (1.f + expf(-z));
   const float bl2 = log_sigmoid(z) * kLog2e, bp2 = log_sigmoid(-z) * kLog2e;
+  const int m0 = first_skip_m(kwin, pi);
+  TileWalk walk;
+  walk.init(i0, n, kBwdRows, kwin, pi, S, bidir);
 
-  auto logit = [&](long long j, bool win) {  // log2 units
-    const T* kr = kb + j * d;
-    float s = 0.f;
-#pragma unroll
-    for (int u = 0; u < 8; ++u) {
-      const int c = lane + 32 * u;
-      if (c < d) s = fmaf(qr[u], to_f32(kr[c]), s);
-    }
-    return fmaf(warp_sum(s), scale_log2, win ? bl2 : bp2);
+  // the warp walks the columns some of its rows read; each row keeps the ones it reads
+  auto tile_cols = [&](long long j0, uint32_t& w0, uint32_t& w1, uint32_t& u0, uint32_t& u1) {
+    w0 = w1 = 0u;
+    if (valid) row_tile_bits(i, j0, kwin, pi, S, m0, walk.rpi, bidir, n, w0, w1);
+    u0 = __reduce_or_sync(0xffffffffu, w0);
+    u1 = __reduce_or_sync(0xffffffffu, w1);
   };
-  // the row's forward: one online softmax over the union, out_i in acc
+  auto is_win = [&](long long j0, int c) {  // a key the row reads is a window key iff |i - j| <= k
+    const long long dj = i - (j0 + c);
+    return dj <= kwin && dj >= -kwin;
+  };
+
+  // the rows' forward: one online softmax over the union, out_i in acc
   float m = -INFINITY, l = 0.f;
-  for_each_key(i, n, kwin, pi, S, bidir, [&](long long j, bool win) {
-    const float s = logit(j, win);
-    const float mn = fmaxf(m, s);
-    const float corr = exp2f(m - mn), p = exp2f(s - mn);
-    l = fmaf(l, corr, p);
-    const T* vr = vb + j * d;
+  for (int t = walk.next(0); t >= 0; t = walk.next(t + 1)) {
+    const long long j0 = (long long)t * kTileKeys;
+    __syncthreads();
+    stage_tile(ks, kb, j0, n, d);
+    stage_tile(vs, vb, j0, n, d);
+    __syncthreads();
+    uint32_t w0, w1, u0, u1;
+    tile_cols(j0, w0, w1, u0, u1);
+    for (int half = 0; half < 2; ++half) {
+      uint32_t un = half ? u1 : u0;
+      const uint32_t mine = half ? w1 : w0;
+      while (un) {
+        const int b = __ffs(un) - 1;
+        un &= un - 1;
+        const int c = 32 * half + b;
+        const float s = fmaf(sum8(dot_part<T, CPT>(qr, ks + c * d, c0, d)), scale_log2, is_win(j0, c) ? bl2 : bp2);
+        if ((mine >> b) & 1u) {
+          const float mn = fmaxf(m, s);
+          const float corr = exp2f(m - mn), p = exp2f(s - mn);
+          l = fmaf(l, corr, p);
 #pragma unroll
-    for (int u = 0; u < 8; ++u) {
-      const int c = lane + 32 * u;
-      if (c < d) acc[u] = fmaf(acc[u], corr, p * to_f32(vr[c]));
+          for (int e = 0; e < CPT; ++e)
+            if (c0 + e < d) acc[e] = fmaf(acc[e], corr, p * to_f32(vs[c * d + c0 + e]));
+          m = mn;
+        }
+      }
     }
-    m = mn;
-  });
-  const float lse2 = m + log2f(l), inv = 1.f / l;
+  }
+  const float lse2 = valid ? m + log2f(l) : 0.f, inv = valid ? 1.f / l : 0.f;
   float Dp = 0.f;
 #pragma unroll
-  for (int u = 0; u < 8; ++u) Dp = fmaf(gr[u], acc[u] * inv, Dp);
-  const float D = warp_sum(Dp);
-  // the row's backward
-  float dqa[8];
+  for (int e = 0; e < CPT; ++e) Dp = fmaf(gr[e], acc[e] * inv, Dp);
+  const float D = sum8(Dp);
+
+  // the rows' backward
+  float dqa[CPT];
 #pragma unroll
-  for (int u = 0; u < 8; ++u) dqa[u] = 0.f;
+  for (int e = 0; e < CPT; ++e) dqa[e] = 0.f;
   float dz = 0.f;
-  for_each_key(i, n, kwin, pi, S, bidir, [&](long long j, bool win) {
-    const float p = exp2f(logit(j, win) - lse2);
-    const T* vr = vb + j * d;
-    const T* kr = kb + j * d;
-    float dp = 0.f;
+  for (int t = walk.next(0); t >= 0; t = walk.next(t + 1)) {
+    const long long j0 = (long long)t * kTileKeys;
+    __syncthreads();
+    stage_tile(ks, kb, j0, n, d);
+    stage_tile(vs, vb, j0, n, d);
+    __syncthreads();
+    uint32_t w0, w1, u0, u1;
+    tile_cols(j0, w0, w1, u0, u1);
+    for (int half = 0; half < 2; ++half) {
+      uint32_t un = half ? u1 : u0;
+      const uint32_t mine = half ? w1 : w0;
+      while (un) {
+        const int b = __ffs(un) - 1;
+        un &= un - 1;
+        const int c = 32 * half + b;
+        const bool win = is_win(j0, c);
+        const float s = fmaf(sum8(dot_part<T, CPT>(qr, ks + c * d, c0, d)), scale_log2, win ? bl2 : bp2);
+        const float dp = sum8(dot_part<T, CPT>(gr, vs + c * d, c0, d));
+        if ((mine >> b) & 1u) {
+          const float ds = exp2f(s - lse2) * (dp - D);
+          dz += win ? (1.f - alpha) * ds : -alpha * ds;
 #pragma unroll
-    for (int u = 0; u < 8; ++u) {
-      const int c = lane + 32 * u;
-      if (c < d) dp = fmaf(gr[u], to_f32(vr[c]), dp);
+          for (int e = 0; e < CPT; ++e)
+            if (c0 + e < d) dqa[e] = fmaf(ds, to_f32(ks[c * d + c0 + e]), dqa[e]);
+        }
+      }
     }
-    const float ds = p * (warp_sum(dp) - D);
-    dz += win ? (1.f - alpha) * ds : -alpha * ds;
-#pragma unroll
-    for (int u = 0; u < 8; ++u) {
-      const int c = lane + 32 * u;
-      if (c < d) dqa[u] = fmaf(ds, to_f32(kr[c]), dqa[u]);
-    }
-  });
-  const float tau = scale_log2 / kLog2e;
-#pragma unroll
-  for (int u = 0; u < 8; ++u) {
-    const int c = lane + 32 * u;
-    if (c < d) dq[task * d + c] = fmaf(tau, dqa[u], dz * w_g[(long long)h * d + c]);
   }
-  if (lane == 0) {
-    st.lse2[task] = lse2;
-    st.D[task] = D;
-    st.bl2[task] = bl2;
-    st.bp2[task] = bp2;
-    st.dz[task] = dz;
+  const float tau = scale_log2 / kLog2e;
+  if (valid) {
+#pragma unroll
+    for (int e = 0; e < CPT; ++e)
+      if (c0 + e < d) dq[row * d + c0 + e] = fmaf(tau, dqa[e], dz * w_g[(long long)h * d + c0 + e]);
+    if (part == 0) {
+      st.lse2[row] = lse2;
+      st.D[row] = D;
+      st.bl2[row] = bl2;
+      st.bp2[row] = bp2;
+      st.dz[row] = dz;
+    }
   }
 }
 
-template <typename T>
-__global__ void __launch_bounds__(256) bwd_key_kernel(const T* __restrict__ q, const T* __restrict__ k,
-                                                      const T* __restrict__ v, const T* __restrict__ dout,
-                                                      BwdRowStats st, float* __restrict__ dk, float* __restrict__ dv,
-                                                      int B, int H, int n, int d, int kwin, int pi, int S,
-                                                      float scale_log2, bool bidir) {
-  const int lane = threadIdx.x & 31;
-  const long long task = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
-  if (task >= (long long)B * H * n) return;
-  const long long bh = task / n, j = task % n;
-  const long long rbase = bh * (long long)n;  // first row of this (b, h)
-  float kr[8], vr[8], dka[8], dva[8];
+template <typename T, int CPT>
+__global__ void __launch_bounds__(kBwdThreads) bwd_key_kernel(const T* __restrict__ q, const T* __restrict__ k,
+                                                              const T* __restrict__ v, const T* __restrict__ dout,
+                                                              BwdRowStats st, float* __restrict__ dk,
+                                                              float* __restrict__ dv, int H, int n, int d, int kwin,
+                                                              int pi, int S, float scale_log2, bool bidir) {
+  extern __shared__ __align__(16) uint8_t bwd_smem[];
+  T* qs = reinterpret_cast<T*>(bwd_smem);
+  T* gs = qs + kTileKeys * d;
+  float* rstat = reinterpret_cast<float*>(gs + kTileKeys * d);  // [4][kTileKeys]: lse2, D, bl2, bp2
+  uint32_t* rbits = reinterpret_cast<uint32_t*>(rstat + 4 * kTileKeys);  // [kTileKeys]: this block's 32 keys
+  const int tid = threadIdx.x, part = tid & (kBwdTPR - 1), c0 = part * CPT;
+  const long long bh = blockIdx.y;
+  (void)H;
+  const long long j0 = (long long)blockIdx.x * kBwdRows, j = j0 + tid / kBwdTPR;
+  const bool valid = j < n;
+  const long long key = bh * (long long)n + (valid ? j : 0);
+  const long long rbase = bh * (long long)n;
+  const long long J0 = j0 / kTileKeys * kTileKeys;  // the 64-key tile holding this block's keys
+  const int off = (int)(j0 - J0);                    // 0 or 32
+  const int kc = (int)(j - j0);                       // this key's bit in the block's word
+  float kr[CPT], vr[CPT], dka[CPT], dva[CPT];
 #pragma unroll
-  for (int u = 0; u < 8; ++u) {
-    const int c = lane + 32 * u;
-    kr[u] = c < d ? to_f32(k[task * d + c]) : 0.f;
-    vr[u] = c < d ? to_f32(v[task * d + c]) : 0.f;
-    dka[u] = dva[u] = 0.f;
+  for (int e = 0; e < CPT; ++e) {
+    const bool in = valid && c0 + e < d;
+    kr[e] = in ? to_f32(k[key * d + c0 + e]) : 0.f;
+    vr[e] = in ? to_f32(v[key * d + c0 + e]) : 0.f;
+    dka[e] = dva[e] = 0.f;
   }
-  for_each_reader(j, n, kwin, pi, S, bidir, [&](long long i, bool win) {
-    const long long row = rbase + i;
-    const T* qr = q + row * d;
-    const T* gr = dout + row * d;
-    float s = 0.f, dp = 0.f;
-    float qv[8], gv[8];
-#pragma unroll
-    for (int u = 0; u < 8; ++u) {
-      const int c = lane + 32 * u;
-      qv[u] = c < d ? to_f32(qr[c]) : 0.f;
-      gv[u] = c < d ? to_f32(gr[c]) : 0.f;
-      s = fmaf(qv[u], kr[u], s);
-      dp = fmaf(gv[u], vr[u], dp);
+  const int m0 = first_skip_m(kwin, pi);
+  ReaderWalk walk;
+  walk.init(j0, n, kBwdRows, kwin, pi, S, bidir);
+  const double rpi = 1.0 / (double)pi;
+  const int wkeys = (tid >> 5) * 4;  // this warp's 4 keys: bits wkeys .. wkeys + 3 of a row's word
+  for (int t = walk.next(0); t >= 0; t = walk.next(t + 1)) {
+    const long long r0 = (long long)t * kTileKeys;
+    __syncthreads();
+    stage_tile(qs, q + rbase * d, r0, n, d);
+    stage_tile(gs, dout + rbase * d, r0, n, d);
+    if (tid < kTileKeys) {
+      const long long i = r0 + tid;
+      uint32_t w = 0u;
+      float a = 0.f, b = 0.f, c = 0.f, e = 0.f;
+      if (i < n) {
+        uint32_t w0, w1;
+        row_tile_bits(i, J0, kwin, pi, S, m0, rpi, bidir, n, w0, w1);
+        w = off ? w1 : w0;
+        a = st.lse2[rbase + i];
+        b = st.D[rbase + i];
+        c = st.bl2[rbase + i];
+        e = st.bp2[rbase + i];
+      }
+      rbits[tid] = w;
+      rstat[tid] = a;
+      rstat[kTileKeys + tid] = b;
+      rstat[2 * kTileKeys + tid] = c;
+      rstat[3 * kTileKeys + tid] = e;
     }
-    s = fmaf(warp_sum(s), scale_log2, win ? st.bl2[row] : st.bp2[row]);
-    const float p = exp2f(s - st.lse2[row]);
-    const float ds = p * (warp_sum(dp) - st.D[row]);
+    __syncthreads();
+    for (int r = 0; r < kTileKeys; ++r) {
+      const uint32_t w = rbits[r];
+      if (((w >> wkeys) & 0xFu) == 0u) continue;  // no key of this warp is read by row r (warp-uniform)
+      const long long i = r0 + r;
+      const long long dj = i - j;
+      const bool win = dj <= kwin && dj >= -kwin;
+      const float s =
+          fmaf(sum8(dot_part<T, CPT>(kr, qs + r * d, c0, d)), scale_log2, win ? rstat[2 * kTileKeys + r] : rstat[3 * kTileKeys + r]);
+      const float dp = sum8(dot_part<T, CPT>(vr, gs + r * d, c0, d));
+      if (valid && ((w >> kc) & 1u)) {
+        const float p = exp2f(s - rstat[r]);
+        const float ds = p * (dp - rstat[kTileKeys + r]);
 #pragma unroll
-    for (int u = 0; u < 8; ++u) {
-      dva[u] = fmaf(p, gv[u], dva[u]);
-      dka[u] = fmaf(ds, qv[u], dka[u]);
+        for (int e = 0; e < CPT; ++e) {
+          if (c0 + e < d) {
+            dva[e] = fmaf(p, to_f32(gs[r * d + c0 + e]), dva[e]);
+            dka[e] = fmaf(ds, to_f32(qs[r * d + c0 + e]), dka[e]);
+          }
+        }
+      }
     }
-  });
+  }
   const float tau = scale_log2 / kLog2e;
+  if (valid) {
 #pragma unroll
-  for (int u = 0; u < 8; ++u) {
-    const int c = lane + 32 * u;
-    if (c < d) {
-      dk[task * d + c] = tau * dka[u];
-      dv[task * d + c] = dva[u];
+    for (int e = 0; e < CPT; ++e) {
+      if (c0 + e < d) {
+        dk[key * d + c0 + e] = tau * dka[e];
+        dv[key * d + c0 + e] = dva[e];
+      }
     }
   }
 }
+
+// dynamic shared memory of the tiled kernels
+inline size_t bwd_row_smem(int d, size_t esz) { return 2 * (size_t)kTileKeys * d * esz; }
+inline size_t bwd_key_smem(int d, size_t esz) { return 2 * (size_t)kTileKeys * d * esz + 5 * kTileKeys * 4; }
 
 // dw_g[h][c] = sum over (b, i) of dz * q[c], db_g[h] = sum of dz, in two stages with a fixed order:
 // bwd_gate_partial_kernel sums chunks of kGateRows rows of one head (one block per (chunk, head),

@@ -112,6 +112,51 @@ pi_attn_status launch_simt(const void* q, const void* k, const void* v, const fl
   return e == cudaSuccess ? ok() : cuda_fail(e, "simt kernel launch");
 }
 
+// The tiled backward kernels for one element type: the column count per thread is a template
+// (d <= 64, 128 or 256); shared memory above 48 KB is opted into once per instantiation.
+template <typename T, int CPT>
+cudaError_t launch_bwd_cpt(const void* q, const void* k, const void* v, const float* w_g, const float* b_g,
+                           const void* dout, float* dq, float* dk, float* dv, pia::BwdRowStats rs, dim3 grid, int H,
+                           int n, int d, int kwin, int pi, int S, float scale_log2, bool bidir, cudaStream_t s) {
+  static bool attr_done = false;
+  const size_t sr = pia::bwd_row_smem(d, sizeof(T)), sk = pia::bwd_key_smem(d, sizeof(T));
+  if (!attr_done) {
+    const size_t max_r = pia::bwd_row_smem(8 * CPT, sizeof(T)), max_k = pia::bwd_key_smem(8 * CPT, sizeof(T));
+    cudaError_t e = cudaFuncSetAttribute(pia::bwd_row_kernel<T, CPT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)max_r);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(pia::bwd_key_kernel<T, CPT>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)max_k);
+    if (e != cudaSuccess) return e;
+    attr_done = true;
+  }
+  pia::bwd_row_kernel<T, CPT><<<grid, pia::kBwdThreads, sr, s>>>((const T*)q, (const T*)k, (const T*)v, w_g, b_g,
+                                                                 (const T*)dout, dq, rs, H, n, d, kwin, pi, S,
+                                                                 scale_log2, bidir);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  pia::bwd_key_kernel<T, CPT><<<grid, pia::kBwdThreads, sk, s>>>((const T*)q, (const T*)k, (const T*)v,
+                                                                 (const T*)dout, rs, dk, dv, H, n, d, kwin, pi, S,
+                                                                 scale_log2, bidir);
+  return cudaGetLastError();
+}
+
+template <typename T>
+cudaError_t launch_bwd(const void* q, const void* k, const void* v, const float* w_g, const float* b_g,
+                       const void* dout, float* dq, float* dk, float* dv, pia::BwdRowStats rs, dim3 grid, int H, int n,
+                       int d, int kwin, int pi, int S, float scale_log2, bool bidir, cudaStream_t s) {
+  if (d <= 64)
+    return launch_bwd_cpt<T, 8>(q, k, v, w_g, b_g, dout, dq, dk, dv, rs, grid, H, n, d, kwin, pi, S, scale_log2, bidir, s);
+  if (d <= 128)
+    return launch_bwd_cpt<T, 16>(q, k, v, w_g, b_g, dout, dq, dk, dv, rs, grid, H, n, d, kwin, pi, S, scale_log2, bidir,
+                                 s);
+  return launch_bwd_cpt<T, 32>(q, k, v, w_g, b_g, dout, dq, dk, dv, rs, grid, H, n, d, kwin, pi, S, scale_log2, bidir,
+                               s);
+}
+
+static long long gate_chunks(int B, int n) {
+  return ((long long)B * n + pia::kGateRows - 1) / pia::kGateRows;
+}
+
 }  // namespace
 
 extern "C" {
@@ -376,10 +421,6 @@ pi_attn_status pi_attn_debug_index_sets_bidir(int n, int k_win, int pi, int S, i
   return index_sets_impl(n, k_win, pi, S, counts, idx, width, true, stream);
 }
 
-static long long gate_chunks(int B, int n) {
-  return ((long long)B * n + pia::kGateRows - 1) / pia::kGateRows;
-}
-
 long long pi_attn_bwd_workspace_bytes(int B, int H, int n, int d) {
   if (B < 1 || H < 1 || n < 1 || d < 1) return 0;
   // lse2, D, two log2-priors and dz per query row, then the gate's per-chunk partial sums (fp32)
@@ -401,9 +442,8 @@ pi_attn_status pi_attn_bwd(const void* q, const void* k, const void* v, const fl
     if (workspace_bytes < need)
       return fail(PI_ATTN_EINVAL, "workspace of %lld bytes, the backward needs %lld", workspace_bytes, need);
   }
-  const long long warps_per_block = 8;
-  const long long blocks = (rows + warps_per_block - 1) / warps_per_block;
-  if (blocks > 0x7fffffffLL) return fail(PI_ATTN_EINVAL, "too many query rows");
+  const long long tiles = ((long long)n + pia::kBwdRows - 1) / pia::kBwdRows;
+  if (tiles > 0x7fffffffLL || (long long)B * H > 65535) return fail(PI_ATTN_EINVAL, "grid too large");
   cudaStream_t s = as_stream(stream);
   void* scratch = workspace;
   cudaError_t e = cudaSuccess;
@@ -418,23 +458,18 @@ pi_attn_status pi_attn_bwd(const void* q, const void* k, const void* v, const fl
   const dim3 gg((unsigned)nchunks, (unsigned)H);
   const float scale_log2 = (float)(1.0 / std::sqrt((double)d)) * pia::kLog2e;
   const bool bd = bidir != 0;
-  const unsigned g = (unsigned)blocks, tb = (unsigned)(warps_per_block * 32);
+  const dim3 gt((unsigned)tiles, (unsigned)(B * H));
   if (dtype == PI_ATTN_F32) {
-    pia::bwd_row_kernel<float><<<g, tb, 0, s>>>((const float*)q, (const float*)k, (const float*)v, w_g, b_g,
-                                                (const float*)dout, dq, rs, B, H, n, d, k_win, pi, S, scale_log2, bd);
-    pia::bwd_key_kernel<float><<<g, tb, 0, s>>>((const float*)q, (const float*)k, (const float*)v,
-                                                (const float*)dout, rs, dk, dv, B, H, n, d, k_win, pi, S, scale_log2,
-                                                bd);
-    pia::bwd_gate_partial_kernel<float><<<gg, 256, 0, s>>>((const float*)q, rs.dz, part_w, part_b, B, H, n, d);
+    e = launch_bwd<float>(q, k, v, w_g, b_g, dout, dq, dk, dv, rs, gt, H, n, d, k_win, pi, S, scale_log2, bd, s);
+    if (e == cudaSuccess)
+      pia::bwd_gate_partial_kernel<float><<<gg, 256, 0, s>>>((const float*)q, rs.dz, part_w, part_b, B, H, n, d);
   } else {
     using bf = __nv_bfloat16;
-    pia::bwd_row_kernel<bf><<<g, tb, 0, s>>>((const bf*)q, (const bf*)k, (const bf*)v, w_g, b_g, (const bf*)dout,
-                                             dq, rs, B, H, n, d, k_win, pi, S, scale_log2, bd);
-    pia::bwd_key_kernel<bf><<<g, tb, 0, s>>>((const bf*)q, (const bf*)k, (const bf*)v, (const bf*)dout, rs, dk, dv,
-                                             B, H, n, d, k_win, pi, S, scale_log2, bd);
-    pia::bwd_gate_partial_kernel<bf><<<gg, 256, 0, s>>>((const bf*)q, rs.dz, part_w, part_b, B, H, n, d);
+    e = launch_bwd<bf>(q, k, v, w_g, b_g, dout, dq, dk, dv, rs, gt, H, n, d, k_win, pi, S, scale_log2, bd, s);
+    if (e == cudaSuccess)
+      pia::bwd_gate_partial_kernel<bf><<<gg, 256, 0, s>>>((const bf*)q, rs.dz, part_w, part_b, B, H, n, d);
   }
-  pia::bwd_gate_final_kernel<<<H, 256, 0, s>>>(part_w, part_b, dw_g, db_g, (int)nchunks, d);
+  if (e == cudaSuccess) pia::bwd_gate_final_kernel<<<H, 256, 0, s>>>(part_w, part_b, dw_g, db_g, (int)nchunks, d);
   e = cudaGetLastError();
   cudaError_t e2 = workspace ? cudaSuccess : cudaFreeAsync(scratch, s);
   if (e != cudaSuccess) return cuda_fail(e, "backward kernel launch");

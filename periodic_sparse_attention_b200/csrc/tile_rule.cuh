@@ -82,6 +82,57 @@ struct TileWalk {
   }
 };
 
+// The transposed walk, for the backward: in increasing order, the row tiles (kTileKeys rows each)
+// holding at least one row that reads a key of the key block [j0, jl].  Row i reads key j as a
+// window key when j in L(i) -- causal: i in [j, j + k]; bidirectional: |i - j| <= k -- and as a
+// skip key when i = j + m pi (and, bidirectional, i = j - m pi) for m0 <= m <= S.
+struct ReaderWalk {
+  long long j0 = 0, jl = -1, w_lo = 0, w_hi = -1, n = 0;  // key block; rows reading it as window keys
+  int pi = 1, S = 0, m0 = 1;
+  bool bidir = false;
+  double rpi = 1.0;
+  PIA_HD void init(long long j0_, long long n_, int keys, int kwin, int pi_, int S_, bool bidir_ = false) {
+    j0 = j0_;
+    n = n_;
+    jl = j0_ + keys - 1 < n_ - 1 ? j0_ + keys - 1 : n_ - 1;
+    w_lo = bidir_ ? (j0_ - kwin > 0 ? j0_ - kwin : 0) : j0_;
+    w_hi = jl + kwin < n_ - 1 ? jl + kwin : n_ - 1;
+    pi = pi_;
+    S = S_;
+    m0 = kwin / pi_ + 1;
+    bidir = bidir_;
+    rpi = 1.0 / (double)pi_;
+  }
+  // smallest reading row tile index >= t, or -1 when none is left
+  PIA_HD int next(int t) const {
+    const long long p = (long long)t * kTileKeys;
+    long long cand = -1;
+    if (p <= w_hi) cand = p > w_lo ? p : w_lo;
+    if (S >= m0) {
+      // rows after the block, [j0 + m pi, jl + m pi]: the smallest m with jl + m pi >= p
+      long long mf = m0;
+      if (p - jl > (long long)m0 * pi) mf = div_floor(p - jl + pi - 1, pi, rpi);
+      if (mf <= S) {
+        long long st = j0 + mf * pi;
+        if (st < p) st = p;
+        if (st <= n - 1 && (cand < 0 || st < cand)) cand = st;
+      }
+      // bidirectional: rows before the block, [j0 - m pi, jl - m pi]: the largest m with
+      // jl - m pi >= p has the leftmost block
+      if (bidir && jl - p >= 0) {
+        long long mb = div_floor(jl - p, pi, rpi);
+        if (mb > S) mb = S;
+        if (mb >= m0) {
+          long long st = j0 - mb * pi;
+          if (st < p) st = p;
+          if (cand < 0 || st < cand) cand = st;
+        }
+      }
+    }
+    return cand < 0 ? -1 : (int)(cand / kTileKeys);
+  }
+};
+
 // For query row i and the key tile starting at j0: window columns [lc_lo, lc_hi] (empty when
 // lc_lo > lc_hi) and a bitmask of skip columns (kTileKeys bits).  Skip columns never overlap the window.
 // The window of row i is [max(0, i - kwin), i - lo_off]: lo_off = 0 for pi-attention's window;

@@ -69,3 +69,23 @@ def test_kernel_index_logic_matches_oracle_bidirectional(harness, n, k, pi, S):
         nl, npk = rc[i]
         assert np.array_equal(idx[i, :nl], ridx[i, :nl])  # window keys, ascending
         assert sorted(idx[i, nl:nl + npk].tolist()) == sorted(ridx[i, nl:nl + npk].tolist())
+
+
+@pytest.mark.parametrize("bidir", [False, True])
+@pytest.mark.parametrize("n,k,pi,S", [(256, 8, 16, 2), (4096, 128, 64, 4), (1000, 100, 37, 12), (333, 400, 16, 40),
+                                      (200, 64, 32, 0), (300, 8, 1, 50), (2049, 63, 65, 40), (640, 0, 128, 4),
+                                      (1, 0, 1, 1), (1500, 300, 1, 3)])
+def test_reader_walk_visits_exactly_the_reading_row_tiles(harness, n, k, pi, S, bidir):
+    harness.reader_walk_tiles.argtypes = [ctypes.c_int] * 6 + [ctypes.c_void_p, ctypes.c_void_p]
+    nb = (n + 63) // 64
+    maxper = nb
+    tiles = np.full((nb, maxper), -1, np.int32)
+    counts = np.zeros(nb, np.int32)
+    assert harness.reader_walk_tiles(n, k, pi, S, int(bidir), maxper, tiles.ctypes.data, counts.ctypes.data) == 0
+    cnt, idx = oracle.index_table(n, k, pi, S, bidir=bidir)
+    expect = [set() for _ in range(nb)]
+    for i in range(n):
+        for j in idx[i, : cnt[i].sum()]:
+            expect[j // 64].add(i // 64)
+    for b in range(nb):
+        assert set(tiles[b, : counts[b]].tolist()) == expect[b], (b, sorted(expect[b]), tiles[b, : counts[b]].tolist())

@@ -73,3 +73,24 @@ extern "C" int tile_rule_sets(int n, int kwin, int pi, int S, int bidir, int wid
   }
   return 0;
 }
+
+// The transposed walk: for each key block of kTileKeys keys, the row tiles ReaderWalk visits
+// (tiles[b * maxper + s], counts[b]); returns 1 if any block visited tiles out of order.
+extern "C" int reader_walk_tiles(int n, int kwin, int pi, int S, int bidir, int maxper, int32_t* tiles,
+                                 int32_t* counts) {
+  int bad = 0;
+  const int nb = (n + kTileKeys - 1) / kTileKeys;
+  for (int b = 0; b < nb; ++b) {
+    ReaderWalk w;
+    w.init((long long)b * kTileKeys, n, kTileKeys, kwin, pi, S, bidir != 0);
+    int c = 0, prev = -1;
+    for (int t = w.next(0); t >= 0; t = w.next(t + 1)) {
+      if (t <= prev) bad = 1;
+      prev = t;
+      if (c < maxper) tiles[b * maxper + c] = t;
+      ++c;
+    }
+    counts[b] = c;
+  }
+  return bad;
+}
