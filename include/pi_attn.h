@@ -171,6 +171,26 @@ pi_attn_status pi_attn_bwd(const void* q, const void* k, const void* v, const fl
                            int n, int d, int k_win, int pi, int S, pi_attn_dtype dtype, int bidir, void* workspace,
                            long long workspace_bytes, void* stream);
 
+/* Decode over a compact ring cache (constant memory per sequence, constant-time update).  Cited
+ * passage: "Execution & Scheduling" -- caches updated in constant time at inference.  Position j of
+ * sequence b lives in slot j mod capacity of kcache / vcache [B, H, capacity, d]; the query is the
+ * token at position cache_len[b] - 1 (any value >= 1, also beyond capacity) and reads L and P as in
+ * pi_attn_decode.  capacity must be >= max(k_win, S*pi) + 1, the farthest a step can still reach
+ * (PI_ATTN_EINVAL otherwise); cache_len is required.  bf16 with d in {64, 128}
+ * (PI_ATTN_EUNSUPPORTED otherwise).  Other arguments, errors and the device check of cache_len
+ * (>= 1) as for pi_attn_decode. */
+pi_attn_status pi_attn_decode_ring(const void* q, const void* kcache, const void* vcache, const float* w_g,
+                                   const float* b_g, const int* cache_len, void* out, float* lse, int B, int H,
+                                   int capacity, int d, int k_win, int pi, int S, pi_attn_dtype dtype, void* stream);
+
+/* One decode step's new token into the cache, then cache_len[b] += 1 for every b (stream-ordered):
+ * row cache_len[b] of every (b, h) -- slot cache_len[b] mod capacity when ring != 0 -- takes
+ * k_new / v_new [B, H, d].  kcache, vcache [B, H, capacity, d] and k_new, v_new in dtype, 16-byte
+ * aligned; cache_len device int32 [B].  A plain cache (ring = 0) that is full, or a negative
+ * cache_len, is reported through the device error word (pi_attn_check) and that b is left as is. */
+pi_attn_status pi_attn_cache_append(void* kcache, void* vcache, const void* k_new, const void* v_new, int* cache_len,
+                                    int B, int H, int capacity, int d, pi_attn_dtype dtype, int ring, void* stream);
+
 /* Index sets as the kernels see them, for exact comparison.  For query rows i = 0..n-1:
  *   counts [n, 2] int32: |L(i)|, |P(i)|
  *   idx    [n, width] int32: L(i) ascending, then P(i) in order of increasing m, then -1.

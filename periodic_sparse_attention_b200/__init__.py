@@ -42,6 +42,10 @@ SIGNATURES = {
     # q k v w_g b_g dout dq dk dv dw_g db_g, B H n d k_win pi S dtype bidir, workspace, bytes, stream
     "pi_attn_bwd": (_i32, [_vp] * 11 + [_i32] * 9 + [_vp, ctypes.c_longlong, _vp]),
     "pi_attn_bwd_workspace_bytes": (ctypes.c_longlong, [_i32, _i32, _i32, _i32]),
+    # as pi_attn_decode, capacity in place of n_cache
+    "pi_attn_decode_ring": (_i32, [_vp] * 8 + [_i32] * 8 + [_vp]),
+    # kcache vcache k_new v_new cache_len, B H capacity d dtype ring, stream
+    "pi_attn_cache_append": (_i32, [_vp] * 5 + [_i32] * 6 + [_vp]),
     "pi_attn_check": (_i32, [_vp]),
     "pi_attn_status_string": (_cstr, [_i32]),
     "pi_attn_last_error": (_cstr, []),
@@ -227,6 +231,32 @@ def pi_attn_bwd(q, k, v, w_g, b_g, dout, k_win: int, pi: int, S: int, *, bidir: 
                          workspace.numel(), _stream(stream))
     _raise(st)
     return dq, dk, dv, dw, db
+
+
+def pi_attn_decode_ring(q, kcache, vcache, w_g, b_g, cache_len, k_win: int, pi: int, S: int, out=None, lse=None, *,
+                        stream=None, want_lse: bool = True):
+    """Decode over a ring cache: q [B, H, d]; caches [B, H, capacity, d] with position j in slot
+    j mod capacity; cache_len int32 [B] (device) the sequences' lengths (query at cache_len - 1)."""
+    import torch
+    B, H, d = q.shape
+    cap = kcache.shape[2]
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None and want_lse:
+        lse = torch.empty((B, H), dtype=torch.float32, device=q.device)
+    st = load().pi_attn_decode_ring(_ptr(q), _ptr(kcache), _ptr(vcache), _ptr(w_g), _ptr(b_g), _ptr(cache_len),
+                                    _ptr(out), _ptr(lse), B, H, cap, d, k_win, pi, S, _dtype_code(q), _stream(stream))
+    _raise(st)
+    return out, lse
+
+
+def pi_attn_cache_append(kcache, vcache, k_new, v_new, cache_len, *, ring: bool = True, stream=None):
+    """Append one token per (b, h) (k_new, v_new [B, H, d]) at position cache_len[b], then advance
+    cache_len.  The caches are [B, H, capacity, d]; ring: slot = position mod capacity."""
+    B, H, cap, d = kcache.shape
+    st = load().pi_attn_cache_append(_ptr(kcache), _ptr(vcache), _ptr(k_new), _ptr(v_new), _ptr(cache_len), B, H, cap,
+                                     d, _dtype_code(kcache), int(ring), _stream(stream))
+    _raise(st)
 
 
 def pi_attn_check(stream=None):

@@ -11,6 +11,10 @@
 // which is the single softmax over the union evaluated in pieces.  With one split the CTA writes
 // out/lse directly; with several, each split writes (m, l, acc) to a workspace and a second
 // kernel merges them.
+//
+// The cache is either plain (position j in row j, len <= n_cache) or a ring of capacity
+// C = n_cache (position j in slot j mod C, any len >= 1): a ring of C >= max(k, S pi) + 1 slots
+// holds every key a decode step can still read, and a step appends one row (pi_attn_cache_append).
 #pragma once
 #include "common.cuh"
 
@@ -28,6 +32,7 @@ struct DecodeArgs {
   float* part;  // [B*H, nsplit, D + 2] when nsplit > 1: acc[D], m, l
   int H, n_cache, kwin, pi, S, nsplit;
   float scale_log2;
+  int ring;     // 1: n_cache is the capacity of a ring cache (position j in slot j mod n_cache)
 };
 
 template <int D>
@@ -56,7 +61,7 @@ __global__ void __launch_bounds__(64) decode_bf16_kernel(DecodeArgs a) {
   const int b = (int)(bh / a.H), h = (int)(bh % a.H);
 
   const int len = a.cache_len ? a.cache_len[b] : a.n_cache;
-  if (len < 1 || len > a.n_cache) {
+  if (len < 1 || (!a.ring && len > a.n_cache)) {
     if (split == 0) {
       if (threadIdx.x == 0) {
         raise_error(kErrCacheLen);
@@ -83,6 +88,10 @@ __global__ void __launch_bounds__(64) decode_bf16_kernel(DecodeArgs a) {
   if (m1 > a.S) m1 = a.S;
   const int nP = m1 >= m0 ? (int)(m1 - m0 + 1) : 0;
   const int R = nL + nP;
+  // ring: slots of the first window row and of the query row (one modulo each; window rows then
+  // step forward and skip rows step back with at most one wrap, as k + 1 <= C and S pi < C)
+  const long long C = a.n_cache;
+  const long long j0s = a.ring ? j0 % C : j0, is = a.ring ? i % C : i;
   // this split's share of the R rows
   const int per = (R + a.nsplit - 1) / a.nsplit;
   const int t_begin = split * per;
@@ -120,9 +129,11 @@ __global__ void __launch_bounds__(64) decode_bf16_kernel(DecodeArgs a) {
     for (int u = 0; u < UNR; ++u) {
       const int t = t0 + u;
       ok[u] = t < t_end;
-      long long j = t < nL ? j0 + t : i - (long long)(m0 + (t - nL)) * a.pi;
+      long long j = t < nL ? j0s + t : is - (long long)(m0 + (t - nL)) * a.pi;  // cache row (slot)
+      if (j >= C) j -= C;
+      else if (j < 0) j += C;
       bias[u] = t < nL ? bias_l : bias_p;
-      if (!ok[u]) j = i;  // a row that exists; its score is discarded below
+      if (!ok[u]) j = is;  // a row that exists; its score is discarded below
       kr[u] = __ldg(reinterpret_cast<const uint4*>(kb + j * D));
       vr[u] = __ldg(reinterpret_cast<const uint4*>(vb + j * D));
     }
@@ -209,11 +220,12 @@ __global__ void __launch_bounds__(64) decode_bf16_kernel(DecodeArgs a) {
 template <int D>
 __global__ void __launch_bounds__(D) decode_combine_kernel(const float* __restrict__ part, int nsplit,
                                                            const int* __restrict__ cache_len, int H, int n_cache,
-                                                           __nv_bfloat16* __restrict__ out, float* __restrict__ lse) {
+                                                           __nv_bfloat16* __restrict__ out, float* __restrict__ lse,
+                                                           int ring) {
   const long long bh = blockIdx.x;
   const int c = threadIdx.x;
   const int len = cache_len ? cache_len[bh / H] : n_cache;
-  if (len < 1 || len > n_cache) return;  // already reported and written as NaN
+  if (len < 1 || (!ring && len > n_cache)) return;  // already reported and written as NaN
   const float* p = part + bh * nsplit * (D + 2);
   float M = -INFINITY;
   for (int s = 0; s < nsplit; ++s) M = fmaxf(M, p[s * (D + 2) + D]);
@@ -227,6 +239,34 @@ __global__ void __launch_bounds__(D) decode_combine_kernel(const float* __restri
   }
   out[bh * D + c] = __float2bfloat16_rn(acc / L);
   if (c == 0 && lse) lse[bh] = (M + log2f(L)) * kLn2;
+}
+
+// One decode step's new token into the cache: row cache_len[b] (mod C for a ring) of every
+// (b, h) takes k_new / v_new; one CTA per (b, h), 16-byte chunks.  A cache_len below zero, or past
+// C for a plain cache, sets the error word and writes nothing.
+template <typename T>
+__global__ void cache_append_kernel(T* __restrict__ kc, T* __restrict__ vc, const T* __restrict__ k_new,
+                                    const T* __restrict__ v_new, const int* __restrict__ cache_len, int H, int C,
+                                    int d, int ring) {
+  const long long bh = blockIdx.x;
+  const int b = (int)(bh / H);
+  const int len = cache_len[b];
+  if (len < 0 || (!ring && len >= C)) {
+    if (threadIdx.x == 0) raise_error(kErrCacheLen);
+    return;
+  }
+  const long long slot = ring ? len % C : len;
+  const int vec = 16 / (int)sizeof(T);
+  for (int c = threadIdx.x * vec; c < d; c += blockDim.x * vec) {
+    *reinterpret_cast<uint4*>(kc + (bh * C + slot) * d + c) = *reinterpret_cast<const uint4*>(k_new + bh * d + c);
+    *reinterpret_cast<uint4*>(vc + (bh * C + slot) * d + c) = *reinterpret_cast<const uint4*>(v_new + bh * d + c);
+  }
+}
+
+// After every (b, h) of a step has been written: the lengths move on by one.
+__global__ void cache_len_advance_kernel(int* __restrict__ cache_len, int B, int C, int ring) {
+  const int b = blockIdx.x * blockDim.x + threadIdx.x;
+  if (b < B && cache_len[b] >= 0 && (ring || cache_len[b] < C)) cache_len[b] += 1;
 }
 
 }  // namespace pia

@@ -269,11 +269,20 @@ pi_attn_status pi_attn_fwd(const void* q, const void* k, const void* v, const fl
   return pi_attn_fwd_ex(q, k, v, w_g, b_g, out, lse, B, H, n, d, k_win, pi, S, dtype, PI_ATTN_PATH_AUTO, stream);
 }
 
-pi_attn_status pi_attn_decode(const void* q, const void* kcache, const void* vcache, const float* w_g,
-                              const float* b_g, const int* cache_len, void* out, float* lse, int B, int H,
-                              int n_cache, int d, int k_win, int pi, int S, pi_attn_dtype dtype, void* stream) {
+static pi_attn_status decode_impl(const void* q, const void* kcache, const void* vcache, const float* w_g,
+                                  const float* b_g, const int* cache_len, void* out, float* lse, int B, int H,
+                                  int n_cache, int d, int k_win, int pi, int S, pi_attn_dtype dtype, void* stream,
+                                  bool ring) {
   pi_attn_status st = check_common(q, kcache, vcache, w_g, b_g, out, B, H, n_cache, d, k_win, pi, S, dtype);
   if (st != PI_ATTN_OK) return st;
+  if (ring) {
+    if (dtype != PI_ATTN_BF16 || (d != 64 && d != 128))
+      return fail(PI_ATTN_EUNSUPPORTED, "the ring-cache decode covers bf16 with d in {64, 128}");
+    const long long reach = (long long)S * pi > k_win ? (long long)S * pi : k_win;
+    if ((long long)n_cache < reach + 1)
+      return fail(PI_ATTN_EINVAL, "ring capacity %d below max(k_win, S*pi) + 1 = %lld", n_cache, reach + 1);
+    if (!cache_len) return fail(PI_ATTN_EINVAL, "the ring-cache decode needs cache_len");
+  }
   cudaStream_t s = as_stream(stream);
   if (dtype == PI_ATTN_BF16 && (d == 64 || d == 128)) {
     const long long bh = (long long)B * H;
@@ -306,6 +315,7 @@ pi_attn_status pi_attn_decode(const void* q, const void* kcache, const void* vca
     a.S = S;
     a.nsplit = nsplit;
     a.scale_log2 = (float)(1.0 / std::sqrt((double)d)) * pia::kLog2e;
+    a.ring = ring ? 1 : 0;
     if (nsplit > 1) {
       const size_t bytes = (size_t)bh * nsplit * (d + 2) * sizeof(float);
       cudaError_t e = cudaMallocAsync((void**)&a.part, bytes, s);
@@ -317,9 +327,9 @@ pi_attn_status pi_attn_decode(const void* q, const void* kcache, const void* vca
     cudaError_t e = cudaGetLastError();
     if (e == cudaSuccess && nsplit > 1) {
       if (d == 128)
-        pia::decode_combine_kernel<128><<<(unsigned)bh, 128, 0, s>>>(a.part, nsplit, cache_len, H, n_cache, a.out, lse);
+        pia::decode_combine_kernel<128><<<(unsigned)bh, 128, 0, s>>>(a.part, nsplit, cache_len, H, n_cache, a.out, lse, a.ring);
       else
-        pia::decode_combine_kernel<64><<<(unsigned)bh, 64, 0, s>>>(a.part, nsplit, cache_len, H, n_cache, a.out, lse);
+        pia::decode_combine_kernel<64><<<(unsigned)bh, 64, 0, s>>>(a.part, nsplit, cache_len, H, n_cache, a.out, lse, a.ring);
       e = cudaGetLastError();
     }
     if (a.part) {
@@ -333,6 +343,46 @@ pi_attn_status pi_attn_decode(const void* q, const void* kcache, const void* vca
                                     S, s);
   return launch_simt<__nv_bfloat16, true>(q, kcache, vcache, w_g, b_g, cache_len, out, lse, B, H, 1, n_cache, d, k_win,
                                           pi, S, s);
+}
+
+pi_attn_status pi_attn_decode(const void* q, const void* kcache, const void* vcache, const float* w_g,
+                              const float* b_g, const int* cache_len, void* out, float* lse, int B, int H,
+                              int n_cache, int d, int k_win, int pi, int S, pi_attn_dtype dtype, void* stream) {
+  return decode_impl(q, kcache, vcache, w_g, b_g, cache_len, out, lse, B, H, n_cache, d, k_win, pi, S, dtype, stream,
+                     false);
+}
+
+pi_attn_status pi_attn_decode_ring(const void* q, const void* kcache, const void* vcache, const float* w_g,
+                                   const float* b_g, const int* cache_len, void* out, float* lse, int B, int H,
+                                   int capacity, int d, int k_win, int pi, int S, pi_attn_dtype dtype, void* stream) {
+  return decode_impl(q, kcache, vcache, w_g, b_g, cache_len, out, lse, B, H, capacity, d, k_win, pi, S, dtype, stream,
+                     true);
+}
+
+pi_attn_status pi_attn_cache_append(void* kcache, void* vcache, const void* k_new, const void* v_new, int* cache_len,
+                                    int B, int H, int capacity, int d, pi_attn_dtype dtype, int ring, void* stream) {
+  if (!kcache || !vcache || !k_new || !v_new || !cache_len) return fail(PI_ATTN_EINVAL, "null pointer");
+  if (dtype != PI_ATTN_F32 && dtype != PI_ATTN_BF16) return fail(PI_ATTN_EINVAL, "unknown dtype %d", (int)dtype);
+  if (B < 1 || H < 1 || capacity < 1 || d < 1 || d > 256) return fail(PI_ATTN_EINVAL, "bad sizes");
+  if ((d * (int)elem_size(dtype)) % 16 != 0) return fail(PI_ATTN_EINVAL, "d * sizeof(dtype) must be a multiple of 16");
+  if (!aligned16(kcache) || !aligned16(vcache) || !aligned16(k_new) || !aligned16(v_new))
+    return fail(PI_ATTN_EINVAL, "caches and new rows must be 16-byte aligned");
+  const long long bh = (long long)B * H;
+  if (bh > 0x7fffffffLL) return fail(PI_ATTN_EINVAL, "B * H too large");
+  cudaStream_t s = as_stream(stream);
+  if (dtype == PI_ATTN_BF16)
+    pia::cache_append_kernel<__nv_bfloat16><<<(unsigned)bh, 32, 0, s>>>(
+        (__nv_bfloat16*)kcache, (__nv_bfloat16*)vcache, (const __nv_bfloat16*)k_new, (const __nv_bfloat16*)v_new,
+        cache_len, H, capacity, d, ring);
+  else
+    pia::cache_append_kernel<float><<<(unsigned)bh, 32, 0, s>>>((float*)kcache, (float*)vcache, (const float*)k_new,
+                                                                (const float*)v_new, cache_len, H, capacity, d, ring);
+  cudaError_t e = cudaGetLastError();
+  if (e == cudaSuccess) {
+    pia::cache_len_advance_kernel<<<(B + 255) / 256, 256, 0, s>>>(cache_len, B, capacity, ring);
+    e = cudaGetLastError();
+  }
+  return e == cudaSuccess ? ok() : cuda_fail(e, "cache append launch");
 }
 
 pi_attn_status pi_attn_decode_noalloc(const void* q, const void* kcache, const void* vcache, const float* w_g,
@@ -373,6 +423,7 @@ pi_attn_status pi_attn_decode_noalloc(const void* q, const void* kcache, const v
   a.out = (__nv_bfloat16*)out;
   a.lse = lse;
   a.part = nullptr;
+  a.ring = 0;
   a.H = H;
   a.n_cache = n_cache;
   a.kwin = k_win;
@@ -390,9 +441,9 @@ pi_attn_status pi_attn_decode_noalloc(const void* q, const void* kcache, const v
   cudaError_t e = cudaGetLastError();
   if (e == cudaSuccess && nsplit > 1) {
     if (d == 128)
-      pia::decode_combine_kernel<128><<<(unsigned)bh, 128, 0, s>>>(a.part, nsplit, cache_len, H, n_cache, a.out, lse);
+      pia::decode_combine_kernel<128><<<(unsigned)bh, 128, 0, s>>>(a.part, nsplit, cache_len, H, n_cache, a.out, lse, a.ring);
     else
-      pia::decode_combine_kernel<64><<<(unsigned)bh, 64, 0, s>>>(a.part, nsplit, cache_len, H, n_cache, a.out, lse);
+      pia::decode_combine_kernel<64><<<(unsigned)bh, 64, 0, s>>>(a.part, nsplit, cache_len, H, n_cache, a.out, lse, a.ring);
     e = cudaGetLastError();
   }
   return e == cudaSuccess ? ok() : cuda_fail(e, "decode kernel launch");

@@ -125,6 +125,19 @@ def test_backward_rejects_bad_arguments(lib):
     assert lib.pi_attn_bwd_workspace_bytes(1, 2, 64, 64) == 4 * (5 * 2 * 64 + 2 * 2 * 65)
 
 
+def test_ring_cache_arguments_are_checked_before_any_launch(lib):
+    # capacity below max(k_win, S*pi) + 1 = 81
+    assert lib.pi_attn_decode_ring(*([FAKE] * 8), 1, 1, 80, 64, 40, 16, 5, pia.PI_ATTN_BF16, None) == pia.PI_ATTN_EINVAL
+    # no cache_len
+    args = [FAKE] * 5 + [None] + [FAKE] * 2
+    assert lib.pi_attn_decode_ring(*args, 1, 1, 81, 64, 40, 16, 5, pia.PI_ATTN_BF16, None) == pia.PI_ATTN_EINVAL
+    # fp32 is not covered
+    assert lib.pi_attn_decode_ring(*([FAKE] * 8), 1, 1, 81, 64, 40, 16, 5, pia.PI_ATTN_F32, None) == \
+        pia.PI_ATTN_EUNSUPPORTED
+    assert lib.pi_attn_cache_append(FAKE, FAKE, FAKE, FAKE, None, 1, 1, 81, 64, pia.PI_ATTN_BF16, 1, None) == \
+        pia.PI_ATTN_EINVAL
+
+
 def test_built_for_sm100a_only():
     cmd = pbuild.command("x.so")
     assert "arch=compute_100a,code=sm_100a" in cmd and "-lineinfo" in cmd
