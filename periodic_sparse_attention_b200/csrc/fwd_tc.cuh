@@ -384,6 +384,11 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm<D>) fwd_tc_kernel(const _
     walk.init(q0, prm.n, BM, prm.kwin, prm.pi, MODE == kFused ? prm.S : 0, MODE == kFused && prm.bidir);
   }
   const int view_rows = MODE == kResidue ? prm.T : prm.n;
+  // every thread walks the tiles with its own cursor (no division per step); thread 0 takes the
+  // first tile at barrier init and goes on from there as the producer
+  TileCursor cur;
+  cur.init(walk);
+  int t_first = -1;
 
   const uint32_t sQ = base + L::kQ, sK = base + L::kK, sV = base + L::kV;
   // P of tile j sits in TMEM over the columns of S buffer j % NSB that the softmax has read: the
@@ -441,7 +446,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm<D>) fwd_tc_kernel(const _
     // allocation and the block barrier
     mbar_expect_tx(bar_q, L::kQBytes);
     load_tile(sQ, &tmq, bar_q, q0, BM);
-    const int t_first = walk.next(0);
+    t_first = cur.next();
     if (t_first >= 0) {
       mbar_expect_tx(bar_kfull(0), L::kKVBytes);
       load_tile(sK, &tmk, bar_kfull(0), (long long)t_first * BN, BN);
@@ -465,9 +470,8 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm<D>) fwd_tc_kernel(const _
     // ------------------------------------------------------------------ TMA producer
     if (lane == 0) {
       constexpr uint32_t kKV = L::kKVBytes;
-      const int t_first = walk.next(0);
       int nk = t_first >= 0 ? 1 : 0, nv = nk;  // K and V tile loads issued (the first one at the start)
-      for (int t = t_first >= 0 ? walk.next(t_first + 1) : -1; t >= 0; t = walk.next(t + 1)) {
+      for (int t = cur.next(); t >= 0; t = cur.next()) {
         const int s = nk % NSTAGE, use = nk / NSTAGE;
         if (use > 0 && !mbar_wait(bar_kempty(s), (use - 1) & 1, abort_flag)) break;
         mbar_expect_tx(bar_kfull(s), kKV);
@@ -546,11 +550,11 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm<D>) fwd_tc_kernel(const _
         return true;
       };
       int j = 0;
-      int t = walk.next(0);
+      int t = cur.next();
       if (okw && t >= 0) okw = try_qk(0);
       // The next tile's Q.K^T goes first: it runs while the softmax works on this tile.
       while (okw && t >= 0) {
-        const int tn = walk.next(t + 1);
+        const int tn = cur.next();
         const int s = j % NSTAGE;
         if (tn >= 0 && !try_qk(j + 1)) break;
         if (!mbar_wait(bar_vfull(s), (j / NSTAGE) & 1, abort_flag)) break;
@@ -616,24 +620,34 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm<D>) fwd_tc_kernel(const _
     const float bias_p = log_sigmoid_fast(-z) * kLog2e;                         // log2(1 - alpha)
     const float NEG_INF = -INFINITY;
 
+    // the row's keys, tile by tile: window columns from the window's bounds, skip columns from
+    // the row's own skip keys taken in order (the residue pass: keys qi - S .. qi - m0 of its
+    // view, no skips)
+    const long long w_lo = MODE == kResidue ? (qi - prm.S > 0 ? qi - prm.S : 0) : (i - prm.kwin > 0 ? i - prm.kwin : 0);
+    const long long w_hi = MODE == kResidue ? qi - m0
+                           : (MODE == kFused && prm.bidir) ? (i + prm.kwin < prm.n - 1 ? i + prm.kwin : prm.n - 1)
+                                                           : i;
+    RowSkips rs;
+    rs.init(i, prm.pi, MODE == kFused ? prm.S : 0, m0, walk.rpi, MODE == kFused && prm.bidir, prm.n);
+
     float m_ref = NEG_INF;  // reference max (log2 units)
     float l_sum = 0.f;      // running sum of probabilities against m_ref (fp32 values: for lse)
     float l_rnd = 0.f;      // the same sum of their bf16 roundings (the weights in P.V: for out)
     int j = 0;
-    for (int t = walk.next(0); ok && t >= 0; t = walk.next(t + 1), ++j) {
+    for (int t = cur.next(); ok && t >= 0; t = cur.next(), ++j) {
       const int sb = j % NSB;
       // every lane of the warp takes the same branch: tcgen05.ld is .sync.aligned
       if (!__all_sync(0xffffffffu, mbar_wait(bar_sfull(sb), (j / NSB) & 1, abort_flag))) { ok = false; break; }
       tc_fence_after();
       const uint32_t tSb = tS + BN * sb + lane_off;
       // the index rule on this tile, for row qi: window columns [lc_lo, lc_hi], skip columns bitmask
-      int lc_lo, lc_hi;
-      uint32_t sk[BN / 32];
-      if (MODE == kResidue)
-        row_tile_mask(qi, (long long)t * BN, prm.S, 1, 0, 1, lc_lo, lc_hi, sk, m0);
-      else
-        row_tile_mask(qi, (long long)t * BN, prm.kwin, prm.pi, MODE == kFused ? prm.S : 0, m0, lc_lo, lc_hi, sk, 0,
-                      walk.rpi, MODE == kFused && prm.bidir, prm.n);
+      const long long j0 = (long long)t * BN;
+      const long long lo64 = w_lo - j0, hi64 = w_hi - j0;
+      const int lc_lo = lo64 < 0 ? 0 : (lo64 > BN ? BN : (int)lo64);
+      const int lc_hi = hi64 > BN - 1 ? BN - 1 : (hi64 < -1 ? -1 : (int)hi64);
+      static_assert(BN == 64, "one 64-bit word of skip bits per tile");
+      const uint64_t skw = rs.take(j0);
+      const uint32_t sk[2] = {(uint32_t)skw, (uint32_t)(skw >> 32)};
       const bool has_win = lc_lo <= lc_hi;
       uint32_t sk_any = 0u;
 #pragma unroll

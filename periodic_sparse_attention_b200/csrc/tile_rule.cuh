@@ -82,6 +82,139 @@ struct TileWalk {
   }
 };
 
+// The same walk as an iterator: TileWalk::next's tiles in the same order, with no division per
+// step.  The needed keys of the query tile are a union of intervals, taken here in ascending order
+// of their starts: the backward skip blocks [i0 - m pi, last - m pi] from the largest m down to m0,
+// then the window band, then (bidirectional) the forward blocks [i0 + m pi, last + m pi] from m0
+// up.  Each interval covers a contiguous run of tiles; the walk is the union of those runs, each
+// tile once, in increasing order.  One division at init (the largest backward m).
+struct TileCursor {
+  long long i0 = 0, last = -1, band_lo = 0, band_hi = -1, n = 0, pi = 1;
+  int S = 0, m0 = 1;
+  bool bidir = false;
+  int phase = 3;  // 0: backward blocks, 1: band, 2: forward blocks, 3: none left
+  int m = 0;      // next block of phase 0 or 2
+  int t = -1;     // last tile returned
+  int t_end = -1; // last tile of the interval being walked
+  PIA_HD void init(const TileWalk& w) {
+    i0 = w.i0;
+    last = w.last;
+    band_lo = w.band_lo;
+    band_hi = w.band_hi;
+    n = w.n;
+    pi = w.pi;
+    S = w.S;
+    m0 = w.m0;
+    bidir = w.bidir;
+    t = -1;
+    t_end = -1;
+    phase = 1;
+    m = 0;
+    if (S >= m0 && last >= 0) {
+      long long mm = div_floor(last, pi, w.rpi);  // blocks with last - m pi >= 0
+      if (mm > S) mm = S;
+      if (mm >= m0) {
+        m = (int)mm;
+        phase = 0;
+      }
+    }
+  }
+  // the next interval of needed keys [a, b] (0 <= a <= b); false when none is left
+  PIA_HD bool interval(long long& a, long long& b) {
+    for (;;) {
+      if (phase == 0) {
+        if (m < m0) {
+          phase = 1;
+          continue;
+        }
+        a = i0 - (long long)m * pi;
+        if (a < 0) a = 0;
+        b = last - (long long)m * pi;
+        --m;
+        return true;
+      }
+      if (phase == 1) {
+        phase = bidir && S >= m0 ? 2 : 3;
+        m = m0;
+        if (band_lo <= band_hi) {
+          a = band_lo;
+          b = band_hi;
+          return true;
+        }
+        continue;
+      }
+      if (phase == 2) {
+        a = i0 + (long long)m * pi;
+        if (m > S || a > n - 1) {
+          phase = 3;
+          continue;
+        }
+        b = last + (long long)m * pi;
+        if (b > n - 1) b = n - 1;
+        ++m;
+        return true;
+      }
+      return false;
+    }
+  }
+  // the next tile of the walk, or -1 when none is left
+  PIA_HD int next() {
+    if (t < t_end) return ++t;
+    long long a, b;
+    while (interval(a, b)) {
+      int ta = (int)(a / kTileKeys);
+      const int tb = (int)(b / kTileKeys);
+      if (ta <= t) ta = t + 1;
+      if (ta <= tb) {
+        t = ta;
+        t_end = tb;
+        return t;
+      }
+    }
+    t_end = t;
+    return -1;
+  }
+};
+
+// One query row's skip keys, in ascending order, taken tile by tile while a walk visits the key
+// tiles in increasing order: the backward skips i - m pi (m from its largest value down to m0),
+// then (bidirectional) the forward skips i + m pi (m from m0 up, keys below n).  Each key is
+// taken by the first tile at or past it, so a walk that visits every tile holding one of the row's
+// keys takes each key in its own tile.  One division per row at init, none per tile.
+struct RowSkips {
+  long long nb = 0, nf = 0, pi = 1;  // next backward / forward skip key
+  int lb = 0, lf = 0;                // backward / forward skip keys left
+  PIA_HD void init(long long i, int pi_, int S, int m0, double rpi, bool bidir, long long n) {
+    pi = pi_;
+    lb = lf = 0;
+    nb = nf = 0;
+    if (S >= m0 && i >= 0) {
+      long long mb = div_floor(i, pi_, rpi);
+      if (mb > S) mb = S;
+      if (mb >= m0) {
+        lb = (int)(mb - m0 + 1);
+        nb = i - mb * pi_;
+      }
+    }
+    if (bidir && S >= m0 && i + (long long)m0 * pi_ <= n - 1) {
+      long long mf = div_floor(n - 1 - i, pi_, rpi);
+      if (mf > S) mf = S;
+      lf = (int)(mf - m0 + 1);
+      nf = i + (long long)m0 * pi_;
+    }
+  }
+  // bit c set for each of the row's skip keys j0 + c in the tile [j0, j0 + kTileKeys)
+  PIA_HD uint64_t take(long long j0) {
+    uint64_t bits = 0;
+    const long long je = j0 + kTileKeys;
+    for (; lb > 0 && nb < je; nb += pi, --lb)
+      if (nb >= j0) bits |= 1ull << (int)(nb - j0);
+    for (; lf > 0 && nf < je; nf += pi, --lf)
+      if (nf >= j0) bits |= 1ull << (int)(nf - j0);
+    return bits;
+  }
+};
+
 // The transposed walk, for the backward: in increasing order, the row tiles (kTileKeys rows each)
 // holding at least one row that reads a key of the key block [j0, jl].  Row i reads key j as a
 // window key when j in L(i) -- causal: i in [j, j + k]; bidirectional: |i - j| <= k -- and as a
@@ -146,13 +279,14 @@ PIA_HD void row_tile_mask(long long i, long long j0, int kwin, int pi, int S, in
   const long long hi = bidir ? (i + kwin < n - 1 ? i + kwin : n - 1) - j0 : d0 - lo_off;
   lc_lo = lo < 0 ? 0 : (lo > kTileKeys ? kTileKeys : (int)lo);
   lc_hi = hi > kTileKeys - 1 ? kTileKeys - 1 : (hi < -1 ? -1 : (int)hi);
-  for (int w = 0; w < kTileKeys / 32; ++w) sk[w] = 0u;
+  static_assert(kTileKeys == 64, "one 64-bit word of skip bits per tile");
+  uint64_t bits = 0;  // a register word: an array indexed by c >> 5 would live in local memory
   if (d0 > kwin && S >= m0) {
     // skip columns c = d0 - m pi in 0..kTileKeys-1: from the largest m (smallest c) upwards in c
     long long m = div_floor(d0, pi, rpi > 0.0 ? rpi : 1.0 / (double)pi);
     if (m > S) m = S;
     for (long long c = d0 - m * pi; m >= m0 && c < kTileKeys; --m, c += pi) {
-      if (c >= 0) sk[c >> 5] |= 1u << (c & 31);
+      if (c >= 0) bits |= 1ull << (int)c;
     }
   }
   if (bidir && S >= m0) {
@@ -160,9 +294,11 @@ PIA_HD void row_tile_mask(long long i, long long j0, int kwin, int pi, int S, in
     long long m = m0;
     if (-d0 > (long long)m0 * pi) m = div_floor(-d0 + pi - 1, pi, rpi > 0.0 ? rpi : 1.0 / (double)pi);
     for (long long c = d0 + m * pi; m <= S && c < kTileKeys && i + m * pi <= n - 1; ++m, c += pi) {
-      if (c >= 0) sk[c >> 5] |= 1u << (c & 31);
+      if (c >= 0) bits |= 1ull << (int)c;
     }
   }
+  sk[0] = (uint32_t)bits;
+  sk[1] = (uint32_t)(bits >> 32);
 }
 
 // Bits of the window columns [lo, hi] (relative to a 32-column chunk) that fall in 0..31.

@@ -36,12 +36,14 @@ def test_kernel_index_logic_matches_oracle(harness, n, k, pi, S):
     width = k + 1 + S
     c = np.zeros((n, 2), np.int32)
     idx = np.zeros((n, width), np.int32)
-    st = np.zeros(4, np.int64)
+    st = np.zeros(6, np.int64)
     harness.tile_rule_sets(n, k, pi, S, 0, width, c.ctypes.data, idx.ctypes.data, st.ctypes.data)
     rc, ridx = oracle.index_table(n, k, pi, S, width)
     assert st[1] == 0, "a key was both a window key and a skip key"
     assert st[2] == 0, "a chunk class does not describe its chunk"
     assert st[3] == 0, "tiles not visited in increasing order"
+    assert st[4] == 0, "the incremental tile cursor departs from the tile walk"
+    assert st[5] == 0, "the incremental row skips depart from the row's tile mask"
     assert np.array_equal(c, rc)
     assert np.array_equal(idx, ridx)
 
@@ -58,12 +60,14 @@ def test_kernel_index_logic_matches_oracle_bidirectional(harness, n, k, pi, S):
     width = 2 * k + 1 + 2 * S
     c = np.zeros((n, 2), np.int32)
     idx = np.zeros((n, width), np.int32)
-    st = np.zeros(4, np.int64)
+    st = np.zeros(6, np.int64)
     harness.tile_rule_sets(n, k, pi, S, 1, width, c.ctypes.data, idx.ctypes.data, st.ctypes.data)
     rc, ridx = oracle.index_table(n, k, pi, S, width, bidir=True)
     assert st[1] == 0, "a key was both a window key and a skip key"
     assert st[2] == 0, "a chunk class does not describe its chunk"
     assert st[3] == 0, "tiles not visited in increasing order"
+    assert st[4] == 0, "the incremental tile cursor departs from the tile walk"
+    assert st[5] == 0, "the incremental row skips depart from the row's tile mask"
     assert np.array_equal(c, rc)
     for i in range(n):
         nl, npk = rc[i]
@@ -89,3 +93,27 @@ def test_reader_walk_visits_exactly_the_reading_row_tiles(harness, n, k, pi, S, 
             expect[j // 64].add(i // 64)
     for b in range(nb):
         assert set(tiles[b, : counts[b]].tolist()) == expect[b], (b, sorted(expect[b]), tiles[b, : counts[b]].tolist())
+
+
+def test_cursor_matches_walk_on_walks_built_by_field(harness):
+    # band-only walks as the residue-class pass builds them (rows t of a residue view read keys
+    # t - S .. t - m0: last is shifted down by m0 and may fall below i0 or below zero), and
+    # random skip walks
+    harness.cursor_vs_walk.argtypes = [ctypes.c_longlong] * 5 + [ctypes.c_int] * 4
+    rng = np.random.default_rng(5)
+    for _ in range(3000):
+        T = int(rng.integers(1, 3000))
+        q0 = int(rng.integers(0, (T + 127) // 128)) * 128
+        Sr = int(rng.integers(0, 60))
+        m0 = int(rng.integers(1, 8))
+        last = min(q0 + 127, T - 1) - m0
+        assert harness.cursor_vs_walk(q0, last, max(q0 - Sr, 0), last, T, 1, 0, 1, 0) == 0
+        n = int(rng.integers(1, 5000))
+        i0 = int(rng.integers(0, (n + 127) // 128)) * 128
+        k = int(rng.integers(0, 700))
+        pi = int(rng.integers(1, 400))
+        S = int(rng.integers(0, 40))
+        bidir = int(rng.integers(0, 2))
+        lastr = min(i0 + 127, n - 1)
+        hi = min(lastr + k, n - 1) if bidir else lastr
+        assert harness.cursor_vs_walk(i0, lastr, max(i0 - k, 0), hi, n, pi, S, k // pi + 1, bidir) == 0

@@ -12,28 +12,49 @@ using namespace pia;
 extern "C" int tile_rule_sets(int n, int kwin, int pi, int S, int bidir, int width, int32_t* counts, int32_t* idx,
                               int64_t* stats) {
   // stats: [0] tiles visited, [1] keys counted twice, [2] chunk-class violations,
-  //        [3] tiles visited out of order
-  for (int s = 0; s < 4; ++s) stats[s] = 0;
+  //        [3] tiles visited out of order, [4] TileCursor steps that differ from TileWalk::next,
+  //        [5] tiles where RowSkips and row_tile_mask give different skip bits
+  // The keys reported are the tensor-core kernel's: tiles from TileCursor, skip bits from
+  // RowSkips, window columns from the row's window bounds.
+  for (int s = 0; s < 6; ++s) stats[s] = 0;
   const int BM = 128;
   for (long long i0 = 0; i0 < n; i0 += BM) {
     TileWalk w;
     w.init(i0, n, BM, kwin, pi, S, bidir != 0);
     int prev = -1;
+    TileCursor cc;
+    cc.init(w);
     for (int t = w.next(0); t >= 0; t = w.next(t + 1)) {
       stats[0]++;
       if (t <= prev) stats[3]++;
       prev = t;
+      if (cc.next() != t) stats[4]++;
     }
+    if (cc.next() != -1 || cc.next() != -1) stats[4]++;
     for (long long i = i0; i < i0 + BM && i < n; ++i) {
       int32_t* row = idx + i * width;
       int nl = 0, np = 0;
       // window keys ascending, skip keys collected then written by increasing m (descending j)
       int32_t skip_keys[4096];
-      for (int t = w.next(0); t >= 0; t = w.next(t + 1)) {
+      TileCursor cur;
+      cur.init(w);
+      RowSkips rs;
+      rs.init(i, pi, S, w.m0, w.rpi, bidir != 0, n);
+      const long long w_lo = i - kwin > 0 ? i - kwin : 0;
+      const long long w_hi = bidir ? (i + kwin < n - 1 ? i + kwin : n - 1) : i;
+      for (int t = cur.next(); t >= 0; t = cur.next()) {
         const long long j0 = (long long)t * kTileKeys;
         int lo, hi;
         uint32_t sk[kTileKeys / 32];
         row_tile_mask(i, j0, kwin, pi, S, w.m0, lo, hi, sk, 0, 0.0, bidir != 0, n);
+        const uint64_t bits = rs.take(j0);
+        if ((uint32_t)bits != sk[0] || (uint32_t)(bits >> 32) != sk[1]) stats[5]++;
+        sk[0] = (uint32_t)bits;
+        sk[1] = (uint32_t)(bits >> 32);
+        const long long lo64 = w_lo - j0, hi64 = w_hi - j0;
+        if ((lo64 < 0 ? 0 : (lo64 > kTileKeys ? kTileKeys : lo64)) != lo ||
+            (hi64 > kTileKeys - 1 ? kTileKeys - 1 : (hi64 < -1 ? -1 : hi64)) != hi)
+          stats[5]++;
         for (int cb = 0; cb < kTileKeys / 32; ++cb) {
           const int cls = chunk_class(cb, lo, hi, sk[cb]);
           int valid = 0, loc_cnt = 0, skp_cnt = 0;
@@ -92,5 +113,29 @@ extern "C" int reader_walk_tiles(int n, int kwin, int pi, int S, int bidir, int 
     }
     counts[b] = c;
   }
+  return bad;
+}
+
+// A walk built field by field (as the residue-class pass builds its own): the number of steps at
+// which TileCursor and TileWalk::next disagree, over the whole walk.
+extern "C" int cursor_vs_walk(long long i0, long long last, long long band_lo, long long band_hi, long long n, int pi,
+                              int S, int m0, int bidir) {
+  TileWalk w;
+  w.i0 = i0;
+  w.last = last;
+  w.band_lo = band_lo;
+  w.band_hi = band_hi;
+  w.n = n;
+  w.pi = pi;
+  w.S = S;
+  w.m0 = m0;
+  w.bidir = bidir != 0;
+  w.rpi = 1.0 / (double)pi;
+  TileCursor c;
+  c.init(w);
+  int bad = 0, steps = 0;
+  for (int t = w.next(0); t >= 0 && steps < 100000; t = w.next(t + 1), ++steps)
+    if (c.next() != t) ++bad;
+  if (c.next() != -1) ++bad;
   return bad;
 }
