@@ -62,8 +62,8 @@ struct Smem {
   static_assert(NSB * BN + D <= kTmemCols && kTmemCols * kCtasPerSm<D> <= 512, "TMEM columns");
   static_assert(NSTAGE * kKVBytes == kQBytes, "the K and V regions each hold one 128-row tile");
   // barriers: q_full, k_full[NSTAGE], k_empty[NSTAGE], v_full[NSTAGE], v_empty[NSTAGE],
-  // s_full[NSB], s_free[NSB], pv_done[NSB], p_full[NSB], drain, skip partials
-  static constexpr int kNumBars = 1 + 4 * NSTAGE + 4 * NSB + 2;
+  // s_full[NSB], pv_done[NSB], p_full[NSB], drain, skip partials
+  static constexpr int kNumBars = 1 + 4 * NSTAGE + 3 * NSB + 2;
   static constexpr int kMisc = kBar + kNumBars * 8;      // tmem base (4 B), abort flag (4 B)
   static constexpr int kWg = (kMisc + 8 + 15) / 16 * 16; // w_g[h] staging, D floats (read as float4)
   static constexpr int kTotal = kWg + D * 4;
@@ -240,6 +240,16 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t* v) {
       "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15])
       : "memory");
 }
+__device__ __forceinline__ void tmem_st32u(uint32_t taddr, const uint32_t* v) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, "
+      "%14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32};" ::"r"(taddr),
+      "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]), "r"(v[8]), "r"(v[9]),
+      "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15]), "r"(v[16]), "r"(v[17]), "r"(v[18]),
+      "r"(v[19]), "r"(v[20]), "r"(v[21]), "r"(v[22]), "r"(v[23]), "r"(v[24]), "r"(v[25]), "r"(v[26]), "r"(v[27]),
+      "r"(v[28]), "r"(v[29]), "r"(v[30]), "r"(v[31])
+      : "memory");
+}
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
 // log(sigmoid(x)) = min(x, 0) - log(1 + e^-|x|) from the fast exponential and logarithm: the
@@ -401,13 +411,14 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm<D>) fwd_tc_kernel(const _
   auto bar_vfull = [&](int s) { return bar0 + 8u * (1 + 2 * NSTAGE + s); };
   auto bar_vempty = [&](int s) { return bar0 + 8u * (1 + 3 * NSTAGE + s); };
   auto bar_sfull = [&](int b) { return bar0 + 8u * (1 + 4 * NSTAGE + b); };
-  auto bar_sfree = [&](int b) { return bar0 + 8u * (1 + 4 * NSTAGE + NSB + b); };
-  auto bar_pvdone = [&](int b) { return bar0 + 8u * (1 + 4 * NSTAGE + 2 * NSB + b); };  // P.V of buffer b
+  auto bar_pvdone = [&](int b) { return bar0 + 8u * (1 + 4 * NSTAGE + NSB + b); };  // P.V of buffer b
   // P of buffer b written by all 128 rows.  One barrier per buffer: with two buffers a fast warp
   // can finish the next tile before a slow one finishes this tile, and on a shared barrier its
-  // arrivals would complete this tile's phase early.
-  auto bar_pfull = [&](int b) { return bar0 + 8u * (1 + 4 * NSTAGE + 3 * NSB + b); };
-  const uint32_t bar_drain = bar0 + 8u * (1 + 4 * NSTAGE + 4 * NSB);
+  // arrivals would complete this tile's phase early.  No phase can run two ahead of a slow warp:
+  // the tile after next in a buffer needs its Q.K^T, which waits for this tile's P.V, which waits
+  // for every row's P.
+  auto bar_pfull = [&](int b) { return bar0 + 8u * (1 + 4 * NSTAGE + 2 * NSB + b); };
+  const uint32_t bar_drain = bar0 + 8u * (1 + 4 * NSTAGE + 3 * NSB);
   const uint32_t bar_so = bar_drain + 8;  // kBandMerge: the tile of skip partials has landed
   uint32_t* const tmem_slot = reinterpret_cast<uint32_t*>(sbase + L::kMisc);
   volatile int* const abort_flag = reinterpret_cast<volatile int*>(sbase + L::kMisc + 4);
@@ -434,7 +445,6 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm<D>) fwd_tc_kernel(const _
     }
     for (int b = 0; b < NSB; ++b) {
       mbar_init(bar_sfull(b), 1);
-      mbar_init(bar_sfree(b), BM);
       mbar_init(bar_pvdone(b), 1);
       mbar_init(bar_pfull(b), BM);
     }
@@ -535,13 +545,13 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm<D>) fwd_tc_kernel(const _
                     (first && kk == 0) ? 0u : 1u);
         }
       };
-      // Q.K^T of tile j needs its K stage loaded, its S buffer released by the softmax of tile
-      // j - NSB, and the P.V of tile j - NSB finished: that P.V reads P from the columns this
-      // Q.K^T overwrites, and MMAs into different accumulators are not ordered with each other.
+      // Q.K^T of tile j needs its K stage loaded and the P.V of tile j - NSB finished: that P.V
+      // reads P from the columns this Q.K^T overwrites (MMAs into different accumulators are not
+      // ordered with each other), and it was issued only once every row had written its P, so
+      // the softmax is done with the buffer too.
       auto try_qk = [&](int jq) -> bool {
         const int s = jq % NSTAGE, b = jq % NSB;
         if (!mbar_wait(bar_kfull(s), (jq / NSTAGE) & 1, abort_flag)) return false;
-        if (jq >= NSB && !mbar_wait(bar_sfree(b), (jq / NSB - 1) & 1, abort_flag)) return false;
         if (jq >= NSB && !mbar_wait(bar_pvdone(b), (jq / NSB - 1) & 1, abort_flag)) return false;
         tc_fence_after();
         issue_qk(s, b);
@@ -660,9 +670,10 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm<D>) fwd_tc_kernel(const _
       // at least the prior gap more, so the bound exceeds the true max by at most twice the score
       // spread of the row.  Probabilities only need a reference at or above their max.
       float mt;
+      float srow[BN];  // the S row as pass 1 loads it; pass 2 reuses it when the row is all window
+      tmem_ld64(tSb, srow);
       {
-        float x[BN];
-        tmem_ld64(tSb, x);
+        const float* x = srow;
         static_assert(BN == 64, "pass 1 reduces eight groups of eight columns");
         float mx[8];  // mx[e]: max over columns e, e + 8, ..., e + 56
 #pragma unroll
@@ -688,31 +699,38 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm<D>) fwd_tc_kernel(const _
         m_ref = mt;
       }
       const float m_use = m_ref == NEG_INF ? 0.f : m_ref;
+      const float bl_m = bias_l - m_use, bp_m = bias_p - m_use;
+      float ls = 0.f, lr = 0.f;
 
-      // (P.V of tile j - NSB, which read this buffer's P, has completed: the MMA thread waited for
-      // it before the Q.K^T of this tile.  That also keeps the pv_done waits below unambiguous.)
-      if (__any_sync(0xffffffffu, rescale)) {
-        // O must hold every earlier tile's P.V before it is rescaled: wait for the P.V of tile j - 1
-        if (j >= 1 &&
-            !__all_sync(0xffffffffu, mbar_wait(bar_pvdone((j - 1) % NSB), ((j - 1) / NSB) & 1, abort_flag))) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        // the rescale is per row, but TMEM access is per warp: the warp rescales when any of its
-        // rows needs it, the others multiply by 1
-        const float f = rescale ? factor : 1.f;
-#pragma unroll 1
-        for (int c = 0; c < D / 32; ++c) {
-          float o[32];
-          tmem_ld32(tO + lane_off + c * 32, o);
+      if (__all_sync(0xffffffffu, lc_lo == 0 && lc_hi == BN - 1 && !has_skip)) {
+        // Every row of the warp reads the whole tile as window keys (the inside of the band):
+        // pass 2 from pass 1's registers, all 64 columns as one batch of independent work, and P
+        // over S columns 0..31 in one store (the whole S row has been read).  Per pair of columns:
+        // one packed FMA (scale and prior), two exponentials, one pack to bf16x2, and packed adds
+        // into the fp32 sum and into the sum of the bf16 roundings.
+        uint32_t pk[BN / 2];
+        unsigned long long sp[4], sr[4];
 #pragma unroll
-          for (int e = 0; e < 32; ++e) o[e] *= f;
-          tmem_st32(tO + lane_off + c * 32, o);
+        for (int a = 0; a < 4; ++a) sp[a] = sr[a] = 0ull;
+        const unsigned long long sc2 = f2pack(prm.scale_log2, prm.scale_log2), bb = f2pack(bl_m, bl_m);
+#pragma unroll
+        for (int e = 0; e < BN; e += 2) {
+          float t0, t1;
+          f2unpack(f2fma(f2pack(srow[e], srow[e + 1]), sc2, bb), t0, t1);
+          const float p0 = ex2(t0), p1 = ex2(t1);
+          __nv_bfloat162 b2 = __floats2bfloat162_rn(p0, p1);
+          const uint32_t u = *reinterpret_cast<uint32_t*>(&b2);
+          pk[e >> 1] = u;
+          sp[(e >> 1) & 3] = f2add(sp[(e >> 1) & 3], f2pack(p0, p1));
+          sr[(e >> 1) & 3] = f2add(sr[(e >> 1) & 3], f2pack(__uint_as_float(u << 16), __uint_as_float(u & 0xFFFF0000u)));
         }
-        tmem_wait_st();
-      }
-
+        tmem_st32u(tSb, pk);
+        float a0, a1, r0, r1;
+        f2unpack(f2add(f2add(sp[0], sp[1]), f2add(sp[2], sp[3])), a0, a1);
+        f2unpack(f2add(f2add(sr[0], sr[1]), f2add(sr[2], sr[3])), r0, r1);
+        ls = a0 + a1;
+        lr = r0 + r1;
+      } else {
       // Pass 2, one 32-column chunk at a time (a rolled loop, re-reading the chunk from TMEM):
       // probabilities against the reference, P (bf16, two per column) back into TMEM, and two
       // row sums -- of the fp32
@@ -720,8 +738,6 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm<D>) fwd_tc_kernel(const _
       // output is normalised by this one, so a row of one key reproduces that key's value).
       //   no key in the chunk -> zeros; window keys only -> one FMA per logit; one skip key and
       //   no window key -> one exponential; otherwise window bits and skip bits pick each prior.
-      const float bl_m = bias_l - m_use, bp_m = bias_p - m_use;
-      float ls = 0.f, lr = 0.f;
 #pragma unroll 1
       for (int cb = 0; cb < CPT; ++cb) {
         const int c0 = cb * 32;
@@ -790,14 +806,39 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm<D>) fwd_tc_kernel(const _
         __syncwarp();  // rows may have taken different branches; tcgen05.st is .sync.aligned
         tmem_st16(tSb + 16 * cb, pk);  // over S columns already read
       }
+      }
       l_sum += ls;
       l_rnd += lr;
+
+      // (P.V of tile j - NSB, which read this buffer's P, has completed: the MMA thread waited for
+      // it before the Q.K^T of this tile.  That also keeps the pv_done waits below unambiguous.)
+      // The rescale comes after pass 2 (which does not touch O) so that the wait for the previous
+      // P.V has had that time to complete; it must precede this tile's p_full arrival.
+      if (__any_sync(0xffffffffu, rescale)) {
+        // O must hold every earlier tile's P.V before it is rescaled: wait for the P.V of tile j - 1
+        if (j >= 1 &&
+            !__all_sync(0xffffffffu, mbar_wait(bar_pvdone((j - 1) % NSB), ((j - 1) / NSB) & 1, abort_flag))) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        // the rescale is per row, but TMEM access is per warp: the warp rescales when any of its
+        // rows needs it, the others multiply by 1
+        const float f = rescale ? factor : 1.f;
+#pragma unroll 1
+        for (int c = 0; c < D / 32; ++c) {
+          float o[32];
+          tmem_ld32(tO + lane_off + c * 32, o);
+#pragma unroll
+          for (int e = 0; e < 32; ++e) o[e] *= f;
+          tmem_st32(tO + lane_off + c * 32, o);
+        }
+      }
       tmem_wait_st();
       tc_fence_before();
-      // P first: once s_free completes (the Q.K^T of tile j + NSB may then start, and with it the
-      // arrivals of that tile) every thread has already arrived on this tile's p_full phase
+      // the P.V of this tile may start; once it has finished, the buffer may take the Q.K^T of
+      // tile j + NSB
       mbar_arrive(bar_pfull(sb));
-      mbar_arrive(bar_sfree(sb));  // the buffer may take the Q.K^T of tile j + NSB (issued after this P.V)
     }
     // ---- epilogue: the normalised row goes to shared memory (the V region, free once the last
     // P.V has completed) in the 128-byte-swizzled 128-row tile layout, then one TMA store writes
