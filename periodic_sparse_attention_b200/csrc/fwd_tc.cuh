@@ -37,14 +37,18 @@ namespace tc {
 constexpr int BM = 128;        // query rows per CTA
 constexpr int BN = kTileKeys;  // keys per tile (64)
 // Pipeline shape.  Both head sizes run two CTAs per SM and one softmax warpgroup per CTA; TMEM per
-// CTA is 256 columns: two S buffers of 64 columns (the next tile's Q.K^T runs while the softmax
-// works on this one; P is written back over the S columns it has read) and O (D columns).  Shared
+// CTA is 256 columns: S buffers of 64 columns (the next tile's Q.K^T runs while the softmax works
+// on this one; P is written back over the S columns it has read) -- three for D = 64, two for
+// D = 128 -- and O (D columns).  Shared
 // memory: the Q tile (128 rows) and a two-stage ring of 64-row K and V tiles.  The two K stages,
 // and the two V stages, are each one contiguous 128-row region, which the epilogue reuses.
 // (Two warpgroups splitting each S row by columns also fit, at 96 registers a thread, but the
 // per-tile exchange of their row maxima cost more than the halved pass over the row saved.)
 constexpr int NSTAGE = 2;      // K/V ring depth
-constexpr int NSB = 2;         // S buffers in TMEM
+// S buffers in TMEM: the Q.K^T of tile j needs the P.V of tile j - NSB finished (P sits in the
+// buffer it overwrites), so a third buffer gives that P.V a whole softmax pass of slack; it fits
+// the 256 columns of a CTA only next to a 64-column O.
+template <int D> constexpr int kNsb = D == 64 ? 3 : 2;
 template <int D> constexpr int kCtasPerSm = 2;
 constexpr int kThreads = 192;  // warp 0 TMA, warp 1 MMA, warps 2..5 softmax (one query row a thread)
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
@@ -59,6 +63,7 @@ struct Smem {
   static constexpr int kV = kK + NSTAGE * kKVBytes;
   static constexpr int kBar = kV + NSTAGE * kKVBytes;    // (P lives in TMEM, over its S columns)
   static constexpr int kTmemCols = 256;                  // S buffers (BN each) + O (D)
+  static constexpr int NSB = kNsb<D>;
   static_assert(NSB * BN + D <= kTmemCols && kTmemCols * kCtasPerSm<D> <= 512, "TMEM columns");
   static_assert(NSTAGE * kKVBytes == kQBytes, "the K and V regions each hold one 128-row tile");
   // barriers: q_full, k_full[NSTAGE], k_empty[NSTAGE], v_full[NSTAGE], v_empty[NSTAGE],
@@ -88,16 +93,16 @@ __device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
 __device__ __forceinline__ void mbar_arrive(uint32_t bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
 }
-// One bounded wait step: the thread is suspended until the phase completes or the hint (1 ms)
-// passes, so a waiting warp does not take issue slots from the warps doing the work.
+// One bounded wait step: try_wait without a suspend-time hint, so the thread waits for a short,
+// system-defined time before returning false (a hint of milliseconds measurably delayed wake-ups).
 __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
       "selp.u32 %0, 1, 0, p;\n\t}"
       : "=r"(ok)
-      : "r"(bar), "r"(parity), "r"(1000000u)
+      : "r"(bar), "r"(parity)
       : "memory");
   return ok != 0;
 }
@@ -358,6 +363,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm<D>) fwd_tc_kernel(const _
                                                                           const __grid_constant__ CUtensorMap tms,
                                                                           Params prm) {
   using L = Smem<D>;
+  constexpr int NSB = kNsb<D>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
@@ -370,6 +376,27 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm<D>) fwd_tc_kernel(const _
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int bh = blockIdx.y;
   const int h = bh % prm.H;
+  // Thread 0 starts the Q tile's load before anything else: its latency (HBM, plus the tensor
+  // map's first use) heads every CTA's critical path.  The tensor maps are prefetched meanwhile.
+  if (threadIdx.x == 0) {
+    asm volatile("prefetch.tensormap [%0];" ::"l"(&tmq) : "memory");
+    asm volatile("prefetch.tensormap [%0];" ::"l"(&tmk) : "memory");
+    asm volatile("prefetch.tensormap [%0];" ::"l"(&tmv) : "memory");
+    asm volatile("prefetch.tensormap [%0];" ::"l"(&tmo) : "memory");
+    if (MODE == kBandMerge) asm volatile("prefetch.tensormap [%0];" ::"l"(&tms) : "memory");
+    const uint32_t bq = base + L::kBar;  // bar_q
+    mbar_init(bq, 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    mbar_expect_tx(bq, L::kQBytes);
+#pragma unroll
+    for (int c = 0; c < D / 64; ++c) {
+      if (MODE == kResidue)
+        tma_load_4d(base + L::kQ + c * BM * 128, &tmq, bq, c * 64, (int)(blockIdx.x % prm.pi),
+                    (int)(blockIdx.x / prm.pi) * BM, bh);
+      else
+        tma_load_3d(base + L::kQ + c * BM * 128, &tmq, bq, c * 64, (int)blockIdx.x * BM, bh);
+    }
+  }
   const int m0 = first_skip_m(prm.kwin, prm.pi);
   // query tile: rows q0 .. q0+127 of the view (the sequence, or residue class `res`)
   int res = 0;
@@ -436,7 +463,6 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm<D>) fwd_tc_kernel(const _
   };
 
   if (threadIdx.x == 0) {
-    mbar_init(bar_q, 1);
     for (int s = 0; s < NSTAGE; ++s) {
       mbar_init(bar_kfull(s), 1);
       mbar_init(bar_kempty(s), 1);
@@ -452,10 +478,8 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm<D>) fwd_tc_kernel(const _
     mbar_init(bar_so, 1);
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-    // the loads that wait for nothing (Q and the first K/V tile) start now, before the TMEM
-    // allocation and the block barrier
-    mbar_expect_tx(bar_q, L::kQBytes);
-    load_tile(sQ, &tmq, bar_q, q0, BM);
+    // the first K/V tile waits for nothing either: it starts now, before the TMEM allocation
+    // and the block barrier
     t_first = cur.next();
     if (t_first >= 0) {
       mbar_expect_tx(bar_kfull(0), L::kKVBytes);
