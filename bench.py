@@ -100,7 +100,7 @@ def load_peaks():
 
 KERNEL_FILES = {  # sources of each timed kernel (for matching committed ncu counters to the code)
     "prefill": ["fwd_tc.cuh", "tile_rule.cuh", "common.cuh"],
-    "backward": ["bwd_simt.cuh", "common.cuh"],
+    "backward": ["bwd_simt.cuh", "tile_rule.cuh", "common.cuh"],
     "decode": ["decode.cuh", "common.cuh"],
 }
 
@@ -122,9 +122,9 @@ def source_hash(files=None) -> str:
 
 
 def profiled_traffic(workload: str):
-    """DRAM bytes per launch of the timed kernel from the committed ncu summaries, if they were
+    """DRAM bytes of one step (its launches summed) from the committed ncu summaries, if they were
     taken on the current kernel source: a line
-      bench-traffic: workload=.. bytes_per_launch=.. files=a.cuh,b.cuh source_sha=..
+      bench-traffic: workload=.. bytes_per_step=.. files=a.cuh,b.cuh source_sha=..
     in profiles/*.md whose files still hash to source_sha.  Otherwise None."""
     d = os.path.join(ROOT, "profiles")
     if not os.path.isdir(d):
@@ -140,7 +140,7 @@ def profiled_traffic(workload: str):
                         continue
                     try:
                         if kv.get("source_sha") == source_hash(kv["files"].split(",")):
-                            return int(kv["bytes_per_launch"])
+                            return int(kv.get("bytes_per_step") or kv["bytes_per_launch"])
                     except OSError:
                         continue
     return None

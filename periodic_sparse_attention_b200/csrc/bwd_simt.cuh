@@ -79,8 +79,12 @@ __device__ __forceinline__ float sum8(float x) {  // over the 8 lanes of a row g
   return x;
 }
 
+// Three 256-thread CTAs an SM for d <= 64 (at most 85 registers a thread); larger d keeps the
+// compiler's choice.
+template <int CPT> constexpr int kBwdMinBlocks = CPT <= 8 ? 3 : 1;
+
 template <typename T, int CPT>
-__global__ void __launch_bounds__(kBwdThreads) bwd_row_kernel(const T* __restrict__ q, const T* __restrict__ k,
+__global__ void __launch_bounds__(kBwdThreads, kBwdMinBlocks<CPT>) bwd_row_kernel(const T* __restrict__ q, const T* __restrict__ k,
                                                               const T* __restrict__ v, const float* __restrict__ w_g,
                                                               const float* __restrict__ b_g,
                                                               const T* __restrict__ dout, float* __restrict__ dq,
@@ -213,7 +217,7 @@ __global__ void __launch_bounds__(kBwdThreads) bwd_row_kernel(const T* __restric
 }
 
 template <typename T, int CPT>
-__global__ void __launch_bounds__(kBwdThreads) bwd_key_kernel(const T* __restrict__ q, const T* __restrict__ k,
+__global__ void __launch_bounds__(kBwdThreads, kBwdMinBlocks<CPT>) bwd_key_kernel(const T* __restrict__ q, const T* __restrict__ k,
                                                               const T* __restrict__ v, const T* __restrict__ dout,
                                                               BwdRowStats st, float* __restrict__ dk,
                                                               float* __restrict__ dv, int H, int n, int d, int kwin,
@@ -311,7 +315,7 @@ inline size_t bwd_key_smem(int d, size_t esz) { return 2 * (size_t)kTileKeys * d
 
 // dw_g[h][c] = sum over (b, i) of dz * q[c], db_g[h] = sum of dz, in two stages with a fixed order:
 // bwd_gate_partial_kernel sums chunks of kGateRows rows of one head (one block per (chunk, head),
-// one thread per column), bwd_gate_final_kernel adds the chunks in increasing order.
+// one thread per column), bwd_gate_final_kernel adds the chunks in a fixed interleaved order.
 constexpr int kGateRows = 32;
 
 template <typename T>
@@ -338,14 +342,34 @@ __global__ void __launch_bounds__(256) bwd_gate_final_kernel(const float* __rest
                                                              const float* __restrict__ part_b,
                                                              float* __restrict__ dw_g, float* __restrict__ db_g,
                                                              int nchunks, int d) {
-  const int h = blockIdx.x, c = threadIdx.x;
-  float aw = 0.f, ab = 0.f;
-  for (int k = 0; k < nchunks; ++k) {
-    if (c < d) aw += part_w[((long long)h * nchunks + k) * d + c];
-    if (c == 0) ab += part_b[(long long)h * nchunks + k];
+  // G threads a column (256 / G >= d): thread g of column c adds chunks g, g + G, ... into four
+  // interleaved sums (independent loads in flight), the G sums are then added in order -- a fixed
+  // order for a given d, so the result does not depend on scheduling.
+  __shared__ float red_w[256], red_b[256];
+  const int h = blockIdx.x;
+  const int G = d <= 32 ? 8 : d <= 64 ? 4 : d <= 128 ? 2 : 1;
+  const int c = threadIdx.x / G, g = threadIdx.x % G;
+  float aw[4] = {0.f, 0.f, 0.f, 0.f}, ab[4] = {0.f, 0.f, 0.f, 0.f};
+  const float* pw = part_w + (long long)h * nchunks * d;
+  const float* pb = part_b + (long long)h * nchunks;
+  int u = 0;
+#pragma unroll 4
+  for (int k = g; k < nchunks; k += G, u = (u + 1) & 3) {
+    if (c < d) aw[u] += pw[(long long)k * d + c];
+    if (c == 0) ab[u] += pb[k];
   }
-  if (c < d) dw_g[(long long)h * d + c] = aw;
-  if (c == 0) db_g[h] = ab;
+  red_w[threadIdx.x] = (aw[0] + aw[1]) + (aw[2] + aw[3]);
+  red_b[threadIdx.x] = (ab[0] + ab[1]) + (ab[2] + ab[3]);
+  __syncthreads();
+  if (g == 0 && c < d) {
+    float sw = 0.f, sb = 0.f;
+    for (int i = 0; i < G; ++i) {
+      sw += red_w[threadIdx.x + i];
+      sb += red_b[threadIdx.x + i];
+    }
+    dw_g[(long long)h * d + c] = sw;
+    if (c == 0) db_g[h] = sb;
+  }
 }
 
 }  // namespace pia

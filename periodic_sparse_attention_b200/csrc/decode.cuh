@@ -47,7 +47,9 @@ __device__ __forceinline__ void decode_merge(float& m, float& l, float* acc, flo
 }
 
 template <int D>
-__global__ void __launch_bounds__(64) decode_bf16_kernel(DecodeArgs a) {
+// 14 CTAs an SM (at most 72 registers a thread): one wave holds 14 x 148 = 2072 CTAs, so a step
+// of up to 2072 (b, h) runs in a single wave instead of one and a fraction.
+__global__ void __launch_bounds__(64, 14) decode_bf16_kernel(DecodeArgs a) {
   constexpr int LPR = D / 8;      // lanes per cache row
   constexpr int RPI = 32 / LPR;   // rows per warp instruction
   constexpr int NW = 2;           // warps per CTA
