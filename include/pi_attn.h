@@ -90,6 +90,24 @@ pi_attn_status pi_attn_fwd_ws(const void* q, const void* k, const void* v, const
                               pi_attn_dtype dtype, pi_attn_path path, void* workspace, long long workspace_bytes,
                               void* stream);
 
+/* One shard of a causal prefill, for a sequence split by rows across devices.  Cited passages: the
+ * gist.science summaries of "pi-Attention: Periodic Sparse Transformers for Efficient Long-Context
+ * Modeling" -- Dutch, sections 2 and 3 (the fixed strides give a communication pattern known in
+ * advance, suited to NCCL/NVLink), English, Hardware Efficiency (less inter-device traffic than
+ * random sparse patterns).  A shard owning sequence rows [row0, row0 + n_q) reads keys back to
+ * row0 - max(k_win, S*pi) (skips only where m*pi > k_win), so it needs that halo of K/V rows from
+ * the shards before it and nothing from the shards after it.
+ *   q, out  [B, H, n_q, d]   sequence rows row0 .. row0 + n_q - 1 (lse [B, H, n_q], may be NULL)
+ *   k, v    [B, H, n_kv, d]  sequence rows kv0 .. kv0 + n_kv - 1: the halo, then the shard's rows
+ * Every row is computed exactly as pi_attn_fwd computes that row of the whole sequence.
+ * PI_ATTN_EINVAL unless kv0 <= max(0, row0 - max(k_win, S*pi)) (the halo reaches every key read)
+ * and kv0 + n_kv >= row0 + n_q (the k/v rows reach the shard's last row), plus the checks of
+ * pi_attn_fwd; bf16 with d in {64, 128} (the single tensor-core pass), else PI_ATTN_EUNSUPPORTED.
+ * Allocates nothing; all pointers are device pointers owned by the caller. */
+pi_attn_status pi_attn_fwd_shard(const void* q, const void* k, const void* v, const float* w_g, const float* b_g,
+                                 void* out, float* lse, int B, int H, int n_q, int n_kv, long long row0,
+                                 long long kv0, int d, int k_win, int pi, int S, pi_attn_dtype dtype, void* stream);
+
 /* Bidirectional prefill forward (the non-causal variant).  Cited passage: the Core Components of
  * the pi-Attention method section -- the local neighbourhood reaches both forward and backward,
  * and in bidirectional settings the skips also reach i + pi.  Row i of a sequence of n tokens

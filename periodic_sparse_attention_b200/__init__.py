@@ -27,6 +27,8 @@ SIGNATURES = {
     "pi_attn_fwd": (_i32, [_vp] * 7 + [_i32] * 8 + [_vp]),
     # ... as above plus the path selector
     "pi_attn_fwd_ex": (_i32, [_vp] * 7 + [_i32] * 9 + [_vp]),
+    # 7 tensor pointers, B H n_q n_kv, row0 kv0 (int64), d k_win pi S, dtype, stream
+    "pi_attn_fwd_shard": (_i32, [_vp] * 7 + [_i32] * 4 + [ctypes.c_longlong] * 2 + [_i32] * 5 + [_vp]),
     # as pi_attn_fwd_ex, bidirectional index rule
     "pi_attn_fwd_bidir": (_i32, [_vp] * 7 + [_i32] * 9 + [_vp]),
     # ... plus workspace pointer and its size in bytes
@@ -144,6 +146,24 @@ def pi_attn_fwd(q, k, v, w_g, b_g, k_win: int, pi: int, S: int, out=None, lse=No
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     st = load().pi_attn_fwd_ws(_ptr(q), _ptr(k), _ptr(v), _ptr(w_g), _ptr(b_g), _ptr(out), _ptr(lse), B, H, n, d,
                                k_win, pi, S, dt, PATHS[path], _ptr(workspace), ws_bytes, _stream(stream))
+    _raise(st)
+    return out, lse
+
+
+def pi_attn_fwd_shard(q, k, v, w_g, b_g, k_win: int, pi: int, S: int, row0: int, kv0: int, out=None, lse=None, *,
+                      stream=None, want_lse: bool = True):
+    """One shard of a causal prefill: q [B, H, n_q, d] holds sequence rows row0 .., k and v
+    [B, H, n_kv, d] hold sequence rows kv0 .. (the halo, then the shard's rows).  bf16, d in
+    {64, 128}.  Allocates out and lse when not given."""
+    import torch
+    B, H, n_q, d = q.shape
+    n_kv = k.shape[2]
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None and want_lse:
+        lse = torch.empty((B, H, n_q), dtype=torch.float32, device=q.device)
+    st = load().pi_attn_fwd_shard(_ptr(q), _ptr(k), _ptr(v), _ptr(w_g), _ptr(b_g), _ptr(out), _ptr(lse), B, H, n_q,
+                                  n_kv, row0, kv0, d, k_win, pi, S, _dtype_code(q), _stream(stream))
     _raise(st)
     return out, lse
 

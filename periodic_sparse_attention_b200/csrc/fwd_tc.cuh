@@ -353,6 +353,9 @@ struct Params {
   int T;                  // kResidue: rows per residue class (n / pi)
   float scale_log2;
   int bidir;              // kFused: the bidirectional index rule (two-sided window, forward skips)
+  // kFused over one shard of a longer sequence: q/out/lse row r is sequence row row0 + r; k/v
+  // row r is sequence row kv0 + r (the index rule runs in sequence rows).  0 and 0 otherwise.
+  long long row0, kv0;
 };
 
 template <int D, int MODE>
@@ -418,7 +421,8 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm<D>) fwd_tc_kernel(const _
     walk.rpi = 1.0;
   } else {
     q0 = (long long)blockIdx.x * BM;
-    walk.init(q0, prm.n, BM, prm.kwin, prm.pi, MODE == kFused ? prm.S : 0, MODE == kFused && prm.bidir);
+    walk.init(prm.row0 + q0, prm.row0 + prm.n, BM, prm.kwin, prm.pi, MODE == kFused ? prm.S : 0,
+              MODE == kFused && prm.bidir);
   }
   const int view_rows = MODE == kResidue ? prm.T : prm.n;
   // every thread walks the tiles with its own cursor (no division per step); thread 0 takes the
@@ -483,9 +487,9 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm<D>) fwd_tc_kernel(const _
     t_first = cur.next();
     if (t_first >= 0) {
       mbar_expect_tx(bar_kfull(0), L::kKVBytes);
-      load_tile(sK, &tmk, bar_kfull(0), (long long)t_first * BN, BN);
+      load_tile(sK, &tmk, bar_kfull(0), (long long)t_first * BN - prm.kv0, BN);
       mbar_expect_tx(bar_vfull(0), L::kKVBytes);
-      load_tile(sV, &tmv, bar_vfull(0), (long long)t_first * BN, BN);
+      load_tile(sV, &tmv, bar_vfull(0), (long long)t_first * BN - prm.kv0, BN);
     }
   }
   if (warp == 1) {  // TMEM: S buffer b in columns [BN b, BN b + BN), O in [BN NSB, BN NSB + D)
@@ -509,11 +513,11 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm<D>) fwd_tc_kernel(const _
         const int s = nk % NSTAGE, use = nk / NSTAGE;
         if (use > 0 && !mbar_wait(bar_kempty(s), (use - 1) & 1, abort_flag)) break;
         mbar_expect_tx(bar_kfull(s), kKV);
-        load_tile(sK + s * kKV, &tmk, bar_kfull(s), (long long)t * BN, BN);
+        load_tile(sK + s * kKV, &tmk, bar_kfull(s), (long long)t * BN - prm.kv0, BN);
         ++nk;
         if (use > 0 && !mbar_wait(bar_vempty(s), (use - 1) & 1, abort_flag)) break;
         mbar_expect_tx(bar_vfull(s), kKV);
-        load_tile(sV + s * kKV, &tmv, bar_vfull(s), (long long)t * BN, BN);
+        load_tile(sV + s * kKV, &tmv, bar_vfull(s), (long long)t * BN - prm.kv0, BN);
         ++nv;
       }
       // kBandMerge: the 128-row tile of skip partials goes into the K region as soon as the last
@@ -612,7 +616,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm<D>) fwd_tc_kernel(const _
     const int q4 = warp & 3;                  // TMEM lane quarter this warp may access
     const int r = q4 * 32 + lane;             // query row within the tile
     const long long qi = q0 + r;              // row in the view
-    const long long i = MODE == kResidue ? qi * prm.pi + res : qi;  // row in the sequence
+    const long long i = MODE == kResidue ? qi * prm.pi + res : prm.row0 + qi;  // row in the sequence
     const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
     // kBandMerge: this row's skip-partial lse (written by the residue pass), loaded now so that
     // the epilogue does not wait for it
@@ -869,7 +873,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm<D>) fwd_tc_kernel(const _
     // the tile (rows past the end of the view are clipped by the tensor map).  kBandMerge merges
     // the tile of skip partials, which the producer has loaded into the K region.
     const bool row_ok = qi < view_rows;
-    const long long orow = (long long)bh * prm.n + i;  // row in [B*H, n] layouts
+    const long long orow = (long long)bh * prm.n + (MODE == kResidue ? i : qi);  // row in [B*H, n] layouts
     const bool have_o = __all_sync(
         0xffffffffu, ok && j > 0 && mbar_wait(bar_pvdone((j - 1) % NSB), ((j - 1) / NSB) & 1, abort_flag));
     const bool no_keys = MODE == kResidue && __all_sync(0xffffffffu, ok && j == 0);  // tile with no skip at all
@@ -1050,6 +1054,8 @@ cudaError_t launch_fwd_tc_d(const void* q, const void* k, const void* v, const f
   p.T = n / pi;
   p.scale_log2 = (float)(1.0 / std::sqrt((double)D)) * kLog2e;
   p.bidir = bidir ? 1 : 0;
+  p.row0 = 0;
+  p.kv0 = 0;
   const dim3 grid((unsigned)((n + tc::BM - 1) / tc::BM), (unsigned)BH);
   cudaError_t e;
   CUtensorMap mo;
@@ -1098,6 +1104,47 @@ cudaError_t launch_fwd_tc_d(const void* q, const void* k, const void* v, const f
   cudaError_t e2 = own ? cudaFreeAsync(scratch, st) : cudaSuccess;
   *why = "tensor-core split kernels";
   return e != cudaSuccess ? e : e2;
+}
+
+// One shard of a causal sequence, single pass: q, out [BH, n_q, D] are sequence rows
+// row0 .. row0 + n_q - 1; k, v [BH, n_kv, D] are sequence rows kv0 .. kv0 + n_kv - 1 (the halo
+// before row0, then the shard's own rows).  The caller has checked that the k/v rows cover every
+// key the shard's rows read.
+template <int D>
+cudaError_t launch_fwd_tc_shard_d(const void* q, const void* k, const void* v, const float* w_g, const float* b_g,
+                                  void* out, float* lse, int B, int H, int n_q, int n_kv, long long row0,
+                                  long long kv0, int kwin, int pi, int S, cudaStream_t st, const char** why) {
+  using L = tc::Smem<D>;
+  CUtensorMap mq, mk, mv, mo;
+  const int BH = B * H;
+  if (!tc::make_map(&mq, q, BH, n_q, D, tc::BM) || !tc::make_map(&mk, k, BH, n_kv, D, tc::BN) ||
+      !tc::make_map(&mv, v, BH, n_kv, D, tc::BN) || !tc::make_map(&mo, out, BH, n_q, D, tc::BM)) {
+    *why = "cuTensorMapEncodeTiled failed";
+    return cudaErrorInvalidValue;
+  }
+  tc::Params p;
+  p.w_g = w_g;
+  p.b_g = b_g;
+  p.out = (__nv_bfloat16*)out;
+  p.lse = lse;
+  p.skip_o = nullptr;
+  p.skip_lse = nullptr;
+  p.H = H;
+  p.n = n_q;
+  p.kwin = kwin;
+  p.pi = pi;
+  p.S = S;
+  p.T = 0;
+  p.scale_log2 = (float)(1.0 / std::sqrt((double)D)) * kLog2e;
+  p.bidir = 0;
+  p.row0 = row0;
+  p.kv0 = kv0;
+  cudaError_t e;
+  if ((e = tc::set_smem_attr<D, tc::kFused>()) != cudaSuccess) { *why = "cudaFuncSetAttribute"; return e; }
+  const dim3 grid((unsigned)((n_q + tc::BM - 1) / tc::BM), (unsigned)BH);
+  tc::fwd_tc_kernel<D, tc::kFused><<<grid, tc::kThreads, L::kAlloc, st>>>(mq, mk, mv, mo, mo, p);
+  *why = "tensor-core shard kernel launch";
+  return cudaGetLastError();
 }
 
 // mode: 0 = choose, 1 = single pass, 2 = split (residue pass + window pass)

@@ -243,6 +243,37 @@ pi_attn_status pi_attn_fwd_bidir(const void* q, const void* k, const void* v, co
   return fwd_impl(q, k, v, w_g, b_g, out, lse, B, H, n, d, k_win, pi, S, dtype, path, true, nullptr, 0, stream);
 }
 
+pi_attn_status pi_attn_fwd_shard(const void* q, const void* k, const void* v, const float* w_g, const float* b_g,
+                                 void* out, float* lse, int B, int H, int n_q, int n_kv, long long row0,
+                                 long long kv0, int d, int k_win, int pi, int S, pi_attn_dtype dtype, void* stream) {
+  pi_attn_status st = check_common(q, k, v, w_g, b_g, out, B, H, n_kv, d, k_win, pi, S, dtype);
+  if (st != PI_ATTN_OK) return st;
+  if (n_q < 1) return fail(PI_ATTN_EINVAL, "n_q must be >= 1 (got %d)", n_q);
+  if ((long long)B * H * n_q * d / d / n_q / H != B) return fail(PI_ATTN_EINVAL, "tensor size overflows");
+  if (dtype != PI_ATTN_BF16 || (d != 64 && d != 128))
+    return fail(PI_ATTN_EUNSUPPORTED, "the shard forward covers bf16 with d in {64, 128} (got dtype %d, d %d)",
+                (int)dtype, d);
+  if (row0 < 0 || kv0 < 0) return fail(PI_ATTN_EINVAL, "row0 and kv0 must be >= 0");
+  // every key a shard row reads: the window back to row0 - k_win and the skips back to row0 - S*pi
+  // (only those past the window exist), through the shard's last row
+  const long long m0 = k_win / pi + 1;
+  long long reach = k_win;
+  if (S >= m0 && (long long)S * pi > reach) reach = (long long)S * pi;
+  const long long need_lo = row0 - reach > 0 ? row0 - reach : 0;
+  if (kv0 > need_lo)
+    return fail(PI_ATTN_EINVAL, "k/v rows start at %lld, after the first key the shard reads (%lld)", kv0, need_lo);
+  if (kv0 + n_kv < row0 + n_q)
+    return fail(PI_ATTN_EINVAL, "k/v rows end at %lld, before the shard's last row %lld", kv0 + n_kv - 1,
+                row0 + n_q - 1);
+  if (row0 + n_q > 0x7fffffffLL) return fail(PI_ATTN_EINVAL, "sequence rows past 2^31");
+  const char* why = "";
+  cudaError_t e = d == 128 ? pia::launch_fwd_tc_shard_d<128>(q, k, v, w_g, b_g, out, lse, B, H, n_q, n_kv, row0, kv0,
+                                                             k_win, pi, S, as_stream(stream), &why)
+                           : pia::launch_fwd_tc_shard_d<64>(q, k, v, w_g, b_g, out, lse, B, H, n_q, n_kv, row0, kv0,
+                                                            k_win, pi, S, as_stream(stream), &why);
+  return e == cudaSuccess ? ok() : cuda_fail(e, why);
+}
+
 pi_attn_status pi_attn_fwd_ex(const void* q, const void* k, const void* v, const float* w_g, const float* b_g,
                               void* out, float* lse, int B, int H, int n, int d, int k_win, int pi, int S,
                               pi_attn_dtype dtype, pi_attn_path path, void* stream) {

@@ -138,6 +138,20 @@ def test_ring_cache_arguments_are_checked_before_any_launch(lib):
         pia.PI_ATTN_EINVAL
 
 
+def test_shard_arguments_are_checked_before_any_launch(lib):
+    # B H n_q n_kv row0 kv0 d k_win pi S; reach = max(40, 5 * 16) = 80
+    def call(n_q, n_kv, row0, kv0, d=64, dtype=pia.PI_ATTN_BF16):
+        return lib.pi_attn_fwd_shard(*([FAKE] * 7), 1, 2, n_q, n_kv, row0, kv0, d, 40, 16, 5, dtype, None)
+    # every call below fails its checks, so none launches (the pointers are placeholders)
+    assert call(100, 179, 200, 121) == pia.PI_ATTN_EINVAL   # halo starts at 121, after row 200 - 80
+    assert call(100, 179, 200, 120) == pia.PI_ATTN_EINVAL   # k/v rows end at 298, before row 299
+    assert call(100, 150, 200, 100) == pia.PI_ATTN_EINVAL   # ... and here at 249
+    assert call(0, 180, 200, 120) == pia.PI_ATTN_EINVAL     # empty shard
+    assert call(100, 180, -1, 0) == pia.PI_ATTN_EINVAL      # negative row
+    assert call(100, 180, 200, 120, dtype=pia.PI_ATTN_F32) == pia.PI_ATTN_EUNSUPPORTED
+    assert call(100, 180, 200, 120, d=32) == pia.PI_ATTN_EUNSUPPORTED
+
+
 def test_built_for_sm100a_only():
     cmd = pbuild.command("x.so")
     assert "arch=compute_100a,code=sm_100a" in cmd and "-lineinfo" in cmd

@@ -1,0 +1,89 @@
+"""Sequence sharding on the GPU (B200 only): pi_attn_fwd_shard over each rank's rows, the halo
+taken from the whole sequence the way the exchange delivers it, against the fp64 oracle on the
+whole sequence.  The ranks run one after another on one device (no kernel waits on another); the
+exchange itself is tested between gloo ranks in test_shard.py."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import periodic_sparse_attention_b200 as pia
+import pi_synth as ps
+from periodic_sparse_attention_b200 import build as pbuild
+from periodic_sparse_attention_b200 import shard
+from tests.gpu_util import assert_close, from_dev, metrics, to_dev
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _library():
+    pbuild.build()
+    pia.load()
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    yield
+    torch.cuda.synchronize()
+
+
+def _inputs(B, H, n, d, seed):
+    q = ps.normal((B, H, n, d), seed=seed, stream=1, dtype="bf16")
+    k = ps.normal((B, H, n, d), seed=seed, stream=2, dtype="bf16")
+    v = ps.normal((B, H, n, d), seed=seed, stream=3, dtype="bf16")
+    w_g = ps.normal((H, d), seed=seed, stream=4, std=1 / math.sqrt(d), dtype="f32")
+    b_g = ps.normal((H,), seed=seed, stream=5, std=0.7, dtype="f32")
+    return q, k, v, w_g, b_g
+
+
+def _run_shards(qt, kt, vt, wg, bg, n, world, kw, pi, S, halo_from_zero=False):
+    outs, lses = [], []
+    for r in range(world):
+        s0, s1 = shard.shard_bounds(n, world, r)
+        if s1 == s0:
+            continue
+        kv0 = 0 if halo_from_zero else max(0, s0 - shard.reach(kw, pi, S))
+        o, l = pia.pi_attn_fwd_shard(qt[:, :, s0:s1].contiguous(), kt[:, :, kv0:s1].contiguous(),
+                                     vt[:, :, kv0:s1].contiguous(), wg, bg, kw, pi, S, s0, kv0)
+        outs.append(o)
+        lses.append(l)
+    pia.pi_attn_check()
+    return torch.cat(outs, dim=2), torch.cat(lses, dim=2)
+
+
+@pytest.mark.parametrize("case", [
+    # B, H, n, d, k, pi, S, world
+    (1, 2, 1000, 64, 40, 16, 30, 4),      # halo of 480 rows: reaches two ranks back
+    (2, 2, 777, 128, 100, 7, 40, 3),      # ragged shards, rows not 128-aligned
+    (1, 3, 4096, 64, 128, 64, 4, 4),      # the bf16_n4k geometry in four shards
+    (1, 1, 2500, 128, 256, 256, 8, 2),    # the bf16_n32k geometry, shorter
+    (1, 2, 300, 64, 8, 16, 2, 5),         # short shards (60 rows)
+])
+def test_shards_match_the_oracle_on_the_whole_sequence(case):
+    B, H, n, d, kw, pi, S, world = case
+    q, k, v, w_g, b_g = _inputs(B, H, n, d, seed=n + world)
+    qt, kt, vt = to_dev(q, "bf16"), to_dev(k, "bf16"), to_dev(v, "bf16")
+    wg, bg = torch.from_numpy(w_g).cuda(), torch.from_numpy(b_g).cuda()
+    out, lse = _run_shards(qt, kt, vt, wg, bg, n, world, kw, pi, S)
+    ro, rl = oracle.fwd(q, k, v, w_g, b_g, kw, pi, S)[:2]
+    assert_close(metrics(from_dev(out).reshape(-1, d), ro.reshape(-1, d), lse.cpu().numpy().astype(np.float64).reshape(-1),
+                         rl.reshape(-1)), "bf16", str(case))
+    # a halo reaching back to row 0 holds more rows than the shard reads; the result is the same
+    # up to rounding (a tile's reference maximum also sees the masked keys, which the shorter
+    # halo zero-fills before its first row)
+    out0, lse0 = _run_shards(qt, kt, vt, wg, bg, n, world, kw, pi, S, halo_from_zero=True)
+    assert_close(metrics(from_dev(out0).reshape(-1, d), ro.reshape(-1, d),
+                         lse0.cpu().numpy().astype(np.float64).reshape(-1), rl.reshape(-1)), "bf16", f"{case} full halo")
+
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_one_shard_is_the_single_pass_forward(d):
+    B, H, n, kw, pi, S = 1, 2, 1500, 100, 32, 9
+    q, k, v, w_g, b_g = _inputs(B, H, n, d, seed=3)
+    qt, kt, vt = to_dev(q, "bf16"), to_dev(k, "bf16"), to_dev(v, "bf16")
+    wg, bg = torch.from_numpy(w_g).cuda(), torch.from_numpy(b_g).cuda()
+    o1, l1 = pia.pi_attn_fwd_shard(qt, kt, vt, wg, bg, kw, pi, S, 0, 0)
+    o2, l2 = pia.pi_attn_fwd(qt, kt, vt, wg, bg, kw, pi, S, path="tc_fused")
+    pia.pi_attn_check()
+    assert torch.equal(o1.view(torch.int16), o2.view(torch.int16))
+    assert torch.equal(l1, l2)
