@@ -39,9 +39,9 @@ constexpr int BN = kTileKeys;  // keys per tile (64)
 // Pipeline shape.  Both head sizes run two CTAs per SM and one softmax warpgroup per CTA; TMEM per
 // CTA is 256 columns: S buffers of 64 columns (the next tile's Q.K^T runs while the softmax works
 // on this one; P is written back over the S columns it has read) -- three for D = 64, two for
-// D = 128 -- and O (D columns).  Shared
-// memory: the Q tile (128 rows) and a two-stage ring of 64-row K and V tiles.  The two K stages,
-// and the two V stages, are each one contiguous 128-row region, which the epilogue reuses.
+// D = 128 -- and O (D columns).  Shared memory: the Q tile (128 rows) and a two-stage ring of
+// 64-row K and V tiles.  The two K stages, and the two V stages, are each one contiguous 128-row
+// region, which the epilogue reuses.
 // (Two warpgroups splitting each S row by columns also fit, at 96 registers a thread, but the
 // per-tile exchange of their row maxima cost more than the halved pass over the row saved.)
 constexpr int NSTAGE = 2;      // K/V ring depth
@@ -623,6 +623,16 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm<D>) fwd_tc_kernel(const _
     const float skip_lse_row =
         MODE == kBandMerge && qi < view_rows ? prm.skip_lse[(long long)bh * prm.n + i] : 0.f;
 
+    // the row's keys, tile by tile: window columns from the window's bounds, skip columns from
+    // the row's own skip keys taken in order (the residue pass: keys qi - S .. qi - m0 of its
+    // view, no skips).  Set up while the Q tile is still in flight.
+    const long long w_lo = MODE == kResidue ? (qi - prm.S > 0 ? qi - prm.S : 0) : (i - prm.kwin > 0 ? i - prm.kwin : 0);
+    const long long w_hi = MODE == kResidue ? qi - m0
+                           : (MODE == kFused && prm.bidir) ? (i + prm.kwin < prm.n - 1 ? i + prm.kwin : prm.n - 1)
+                                                           : i;
+    RowSkips rs;
+    rs.init(i, prm.pi, MODE == kFused ? prm.S : 0, m0, walk.rpi, MODE == kFused && prm.bidir, prm.n);
+
     // gate on the unscaled query row.  w_g[h] is staged in shared memory while the Q tile is
     // still in flight.
     float* const wg_s = reinterpret_cast<float*>(sbase + L::kWg);
@@ -657,16 +667,6 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm<D>) fwd_tc_kernel(const _
     const float bias_l = log_sigmoid_fast(MODE == kResidue ? -z : z) * kLog2e;  // log2(alpha), or log2(1-alpha)
     const float bias_p = log_sigmoid_fast(-z) * kLog2e;                         // log2(1 - alpha)
     const float NEG_INF = -INFINITY;
-
-    // the row's keys, tile by tile: window columns from the window's bounds, skip columns from
-    // the row's own skip keys taken in order (the residue pass: keys qi - S .. qi - m0 of its
-    // view, no skips)
-    const long long w_lo = MODE == kResidue ? (qi - prm.S > 0 ? qi - prm.S : 0) : (i - prm.kwin > 0 ? i - prm.kwin : 0);
-    const long long w_hi = MODE == kResidue ? qi - m0
-                           : (MODE == kFused && prm.bidir) ? (i + prm.kwin < prm.n - 1 ? i + prm.kwin : prm.n - 1)
-                                                           : i;
-    RowSkips rs;
-    rs.init(i, prm.pi, MODE == kFused ? prm.S : 0, m0, walk.rpi, MODE == kFused && prm.bidir, prm.n);
 
     float m_ref = NEG_INF;  // reference max (log2 units)
     float l_sum = 0.f;      // running sum of probabilities against m_ref (fp32 values: for lse)
