@@ -64,13 +64,50 @@ __device__ __forceinline__ void row_tile_bits(long long i, long long j0, int kwi
   w1 = window_bits(lo - 32, hi - 32) | sk[1];
 }
 
+// The CPT columns c0 .. c0 + CPT - 1 of a row in shared memory as fp32, zero past d: 16-byte loads
+// when the whole chunk lies in the row (row starts and c0 are 16-byte aligned: d * sizeof(T) is a
+// multiple of 16, and so is CPT * sizeof(T)).
 template <typename T, int CPT>
-__device__ __forceinline__ float dot_part(const float* a, const T* b, int c0, int d) {
-  float s = 0.f;
+__device__ __forceinline__ void load_cols(const T* rowp, int c0, int d, float* f) {
+  if (c0 + CPT <= d) {
+    if constexpr (sizeof(T) == 2) {
 #pragma unroll
-  for (int e = 0; e < CPT; ++e)
-    if (c0 + e < d) s = fmaf(a[e], to_f32(b[c0 + e]), s);
-  return s;
+      for (int u = 0; u < CPT / 8; ++u) bf16x8_to_f32(*reinterpret_cast<const uint4*>(rowp + c0 + 8 * u), f + 8 * u);
+    } else {
+#pragma unroll
+      for (int u = 0; u < CPT / 4; ++u) {
+        const float4 x = *reinterpret_cast<const float4*>(rowp + c0 + 4 * u);
+        f[4 * u] = x.x;
+        f[4 * u + 1] = x.y;
+        f[4 * u + 2] = x.z;
+        f[4 * u + 3] = x.w;
+      }
+    }
+  } else {
+#pragma unroll
+    for (int e = 0; e < CPT; ++e) f[e] = c0 + e < d ? to_f32(rowp[c0 + e]) : 0.f;
+  }
+}
+// sum of a[e] * b[e] over the chunk, in packed pairs with two independent accumulators
+template <int CPT>
+__device__ __forceinline__ float dot_cols(const float* a, const float* b) {
+  static_assert(CPT % 4 == 0, "pairs of pairs");
+  unsigned long long s0 = 0ull, s1 = 0ull;
+#pragma unroll
+  for (int e = 0; e < CPT; e += 4) {
+    s0 = f2fma(f2pack(a[e], a[e + 1]), f2pack(b[e], b[e + 1]), s0);
+    s1 = f2fma(f2pack(a[e + 2], a[e + 3]), f2pack(b[e + 2], b[e + 3]), s1);
+  }
+  float x, y;
+  f2unpack(f2add(s0, s1), x, y);
+  return x + y;
+}
+// acc[e] += s * b[e] over the chunk, in packed pairs
+template <int CPT>
+__device__ __forceinline__ void axpy_cols(float s, const float* b, float* acc) {
+  const unsigned long long s2 = f2pack(s, s);
+#pragma unroll
+  for (int e = 0; e < CPT; e += 2) f2unpack(f2fma(s2, f2pack(b[e], b[e + 1]), f2pack(acc[e], acc[e + 1])), acc[e], acc[e + 1]);
 }
 __device__ __forceinline__ float sum8(float x) {  // over the 8 lanes of a row group (all lanes call)
   x += __shfl_xor_sync(0xffffffffu, x, 1);
@@ -79,9 +116,9 @@ __device__ __forceinline__ float sum8(float x) {  // over the 8 lanes of a row g
   return x;
 }
 
-// Three 256-thread CTAs an SM for d <= 64 (at most 85 registers a thread); larger d keeps the
-// compiler's choice.
-template <int CPT> constexpr int kBwdMinBlocks = CPT <= 8 ? 3 : 1;
+// 256-thread CTAs an SM: three for d <= 64 (at most 85 registers a thread), two for d <= 128 (128
+// registers); d <= 256 keeps the compiler's choice.
+template <int CPT> constexpr int kBwdMinBlocks = CPT <= 8 ? 3 : (CPT <= 16 ? 2 : 1);
 
 template <typename T, int CPT>
 __global__ void __launch_bounds__(kBwdThreads, kBwdMinBlocks<CPT>) bwd_row_kernel(const T* __restrict__ q, const T* __restrict__ k,
@@ -149,14 +186,19 @@ __global__ void __launch_bounds__(kBwdThreads, kBwdMinBlocks<CPT>) bwd_row_kerne
         const int b = __ffs(un) - 1;
         un &= un - 1;
         const int c = 32 * half + b;
-        const float s = fmaf(sum8(dot_part<T, CPT>(qr, ks + c * d, c0, d)), scale_log2, is_win(j0, c) ? bl2 : bp2);
+        float kc[CPT];
+        load_cols<T, CPT>(ks + c * d, c0, d, kc);
+        const float s = fmaf(sum8(dot_cols<CPT>(qr, kc)), scale_log2, is_win(j0, c) ? bl2 : bp2);
         if ((mine >> b) & 1u) {
           const float mn = fmaxf(m, s);
-          const float corr = exp2f(m - mn), p = exp2f(s - mn);
+          const float corr = ex2(m - mn), p = ex2(s - mn);
           l = fmaf(l, corr, p);
+          float vc[CPT];
+          load_cols<T, CPT>(vs + c * d, c0, d, vc);
+          const unsigned long long c2 = f2pack(corr, corr), p2 = f2pack(p, p);
 #pragma unroll
-          for (int e = 0; e < CPT; ++e)
-            if (c0 + e < d) acc[e] = fmaf(acc[e], corr, p * to_f32(vs[c * d + c0 + e]));
+          for (int e = 0; e < CPT; e += 2)
+            f2unpack(f2fma(f2pack(acc[e], acc[e + 1]), c2, f2mul(p2, f2pack(vc[e], vc[e + 1]))), acc[e], acc[e + 1]);
           m = mn;
         }
       }
@@ -189,14 +231,15 @@ __global__ void __launch_bounds__(kBwdThreads, kBwdMinBlocks<CPT>) bwd_row_kerne
         un &= un - 1;
         const int c = 32 * half + b;
         const bool win = is_win(j0, c);
-        const float s = fmaf(sum8(dot_part<T, CPT>(qr, ks + c * d, c0, d)), scale_log2, win ? bl2 : bp2);
-        const float dp = sum8(dot_part<T, CPT>(gr, vs + c * d, c0, d));
+        float kc[CPT], vc[CPT];
+        load_cols<T, CPT>(ks + c * d, c0, d, kc);
+        load_cols<T, CPT>(vs + c * d, c0, d, vc);
+        const float s = fmaf(sum8(dot_cols<CPT>(qr, kc)), scale_log2, win ? bl2 : bp2);
+        const float dp = sum8(dot_cols<CPT>(gr, vc));
         if ((mine >> b) & 1u) {
-          const float ds = exp2f(s - lse2) * (dp - D);
+          const float ds = ex2(s - lse2) * (dp - D);
           dz += win ? (1.f - alpha) * ds : -alpha * ds;
-#pragma unroll
-          for (int e = 0; e < CPT; ++e)
-            if (c0 + e < d) dqa[e] = fmaf(ds, to_f32(ks[c * d + c0 + e]), dqa[e]);
+          axpy_cols<CPT>(ds, kc, dqa);
         }
       }
     }
@@ -281,19 +324,16 @@ __global__ void __launch_bounds__(kBwdThreads, kBwdMinBlocks<CPT>) bwd_key_kerne
       const long long i = r0 + r;
       const long long dj = i - j;
       const bool win = dj <= kwin && dj >= -kwin;
-      const float s =
-          fmaf(sum8(dot_part<T, CPT>(kr, qs + r * d, c0, d)), scale_log2, win ? rstat[2 * kTileKeys + r] : rstat[3 * kTileKeys + r]);
-      const float dp = sum8(dot_part<T, CPT>(vr, gs + r * d, c0, d));
+      float qc[CPT], gc[CPT];
+      load_cols<T, CPT>(qs + r * d, c0, d, qc);
+      load_cols<T, CPT>(gs + r * d, c0, d, gc);
+      const float s = fmaf(sum8(dot_cols<CPT>(kr, qc)), scale_log2, win ? rstat[2 * kTileKeys + r] : rstat[3 * kTileKeys + r]);
+      const float dp = sum8(dot_cols<CPT>(vr, gc));
       if (valid && ((w >> kc) & 1u)) {
-        const float p = exp2f(s - rstat[r]);
+        const float p = ex2(s - rstat[r]);
         const float ds = p * (dp - rstat[kTileKeys + r]);
-#pragma unroll
-        for (int e = 0; e < CPT; ++e) {
-          if (c0 + e < d) {
-            dva[e] = fmaf(p, to_f32(gs[r * d + c0 + e]), dva[e]);
-            dka[e] = fmaf(ds, to_f32(qs[r * d + c0 + e]), dka[e]);
-          }
-        }
+        axpy_cols<CPT>(p, gc, dva);
+        axpy_cols<CPT>(ds, qc, dka);
       }
     }
   }

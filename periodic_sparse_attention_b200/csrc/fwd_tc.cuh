@@ -264,25 +264,6 @@ __device__ __forceinline__ float log_sigmoid_fast(float x) {
   return fminf(x, 0.f) - __logf(1.f + __expf(-fabsf(x)));
 }
 
-// Packed fp32 pairs (Blackwell f32x2 arithmetic: two lanes of work per instruction).
-__device__ __forceinline__ unsigned long long f2pack(float a, float b) {
-  unsigned long long r;
-  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
-  return r;
-}
-__device__ __forceinline__ void f2unpack(unsigned long long r, float& a, float& b) {
-  asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(r));
-}
-__device__ __forceinline__ unsigned long long f2fma(unsigned long long a, unsigned long long b, unsigned long long c) {
-  unsigned long long d;
-  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
-  return d;
-}
-__device__ __forceinline__ unsigned long long f2add(unsigned long long a, unsigned long long b) {
-  unsigned long long d;
-  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
-  return d;
-}
 
 // v[k] for a run-time k in 0..31 from a register array: a 5-level tree of selects on the bits of
 // k (independent selects, no local memory, no long dependency chain).
@@ -300,11 +281,6 @@ __device__ __forceinline__ float pick32(const float* v, int k) {
   return k4 ? d[1] : d[0];
 }
 
-__device__ __forceinline__ float ex2(float x) {
-  float y;
-  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-  return y;
-}
 
 // max of three (one instruction on sm_100)
 __device__ __forceinline__ float max3f(float a, float b, float c) {
