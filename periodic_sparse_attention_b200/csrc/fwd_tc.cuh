@@ -878,6 +878,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm<D>) fwd_tc_kernel(const _
 #pragma unroll
         for (int e = 0; e < D; ++e) o[e] = 0.f;
       }
+      const unsigned long long ow2 = f2pack(inv * wl, inv * wl), wp2 = f2pack(wp, wp);
 #pragma unroll
       for (int cl = 0; cl < D / 8; ++cl) {  // 16-byte chunk c of the row
         const int c = cl;
@@ -887,9 +888,11 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm<D>) fwd_tc_kernel(const _
         if (MODE == kBandMerge && so_ok) bf16x8_to_f32(*reinterpret_cast<const uint4*>(sbase + L::kK + off), sp);
         uint32_t w[4];
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const float a0 = o[cl * 8 + 2 * e] * inv * wl + sp[2 * e] * wp;
-          const float a1 = o[cl * 8 + 2 * e + 1] * inv * wl + sp[2 * e + 1] * wp;
+        for (int e = 0; e < 4; ++e) {  // out = O / l_rnd * w_l + skip partial * w_p, in packed pairs
+          float a0, a1;
+          f2unpack(f2fma(f2pack(o[cl * 8 + 2 * e], o[cl * 8 + 2 * e + 1]), ow2,
+                         f2mul(f2pack(sp[2 * e], sp[2 * e + 1]), wp2)),
+                   a0, a1);
           __nv_bfloat162 b2 = __floats2bfloat162_rn(a0, a1);
           w[e] = *reinterpret_cast<uint32_t*>(&b2);
         }
