@@ -734,6 +734,37 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm<D>) fwd_tc_kernel(const _
         f2unpack(f2add(f2add(sr[0], sr[1]), f2add(sr[2], sr[3])), r0, r1);
         ls = a0 + a1;
         lr = r0 + r1;
+      } else if (__all_sync(0xffffffffu, !has_skip)) {
+        // Every row of the warp reads only window keys here, a contiguous range of columns
+        // (the band's edges and the causal diagonal): the same batch from registers, with the
+        // columns outside the row's range set to -inf before the exponential (p = 0 exactly).
+        const uint64_t wb = lc_lo > lc_hi ? 0ull : ((~0ull >> (BN - 1 - lc_hi)) & (~0ull << lc_lo));
+        const uint32_t wlo = (uint32_t)wb, whi = (uint32_t)(wb >> 32);
+        uint32_t pk[BN / 2];
+        unsigned long long sp[4], sr[4];
+#pragma unroll
+        for (int a = 0; a < 4; ++a) sp[a] = sr[a] = 0ull;
+        const unsigned long long sc2 = f2pack(prm.scale_log2, prm.scale_log2), bb = f2pack(bl_m, bl_m);
+#pragma unroll
+        for (int e = 0; e < BN; e += 2) {
+          float t0, t1;
+          f2unpack(f2fma(f2pack(srow[e], srow[e + 1]), sc2, bb), t0, t1);
+          const uint32_t wv = e < 32 ? wlo : whi;
+          if (!((wv >> (e & 31)) & 1u)) t0 = NEG_INF;
+          if (!((wv >> ((e + 1) & 31)) & 1u)) t1 = NEG_INF;
+          const float p0 = ex2(t0), p1 = ex2(t1);
+          __nv_bfloat162 b2 = __floats2bfloat162_rn(p0, p1);
+          const uint32_t u = *reinterpret_cast<uint32_t*>(&b2);
+          pk[e >> 1] = u;
+          sp[(e >> 1) & 3] = f2add(sp[(e >> 1) & 3], f2pack(p0, p1));
+          sr[(e >> 1) & 3] = f2add(sr[(e >> 1) & 3], f2pack(__uint_as_float(u << 16), __uint_as_float(u & 0xFFFF0000u)));
+        }
+        tmem_st32u(tSb, pk);
+        float a0, a1, r0, r1;
+        f2unpack(f2add(f2add(sp[0], sp[1]), f2add(sp[2], sp[3])), a0, a1);
+        f2unpack(f2add(f2add(sr[0], sr[1]), f2add(sr[2], sr[3])), r0, r1);
+        ls = a0 + a1;
+        lr = r0 + r1;
       } else {
       // Pass 2, one 32-column chunk at a time (a rolled loop, re-reading the chunk from TMEM):
       // probabilities against the reference, P (bf16, two per column) back into TMEM, and two
