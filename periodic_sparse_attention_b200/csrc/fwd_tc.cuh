@@ -734,10 +734,11 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm<D>) fwd_tc_kernel(const _
         f2unpack(f2add(f2add(sr[0], sr[1]), f2add(sr[2], sr[3])), r0, r1);
         ls = a0 + a1;
         lr = r0 + r1;
-      } else if (__all_sync(0xffffffffu, !has_skip)) {
+      } else if (__all_sync(0xffffffffu, !has_skip) && __any_sync(0xffffffffu, has_win)) {
         // Every row of the warp reads only window keys here, a contiguous range of columns
-        // (the band's edges and the causal diagonal): the same batch from registers, with the
-        // columns outside the row's range set to -inf before the exponential (p = 0 exactly).
+        // (the band's edges and the causal diagonal), and some row reads at least one: the same
+        // batch from registers, with the columns outside the row's range set to -inf before the
+        // exponential (p = 0 exactly).  A warp with no key at all takes the rolled path's zeros.
         const uint64_t wb = lc_lo > lc_hi ? 0ull : ((~0ull >> (BN - 1 - lc_hi)) & (~0ull << lc_lo));
         const uint32_t wlo = (uint32_t)wb, whi = (uint32_t)(wb >> 32);
         uint32_t pk[BN / 2];
