@@ -141,6 +141,7 @@ EDGE = [  # B, H, n, d, k, pi, S
     (2, 1, 2048, 64, 100, 128, 8),  # residue sequences of 16 rows, first skip m = 1
     (1, 1, 4096, 128, 300, 256, 12),  # first surviving skip m = 2
     (1, 1, 2112, 64, 10, 64, 40),   # 33 rows per residue, skips reach the start
+    (1, 2, 100, 64, 8, 200, 3),     # period longer than the sequence: no skip exists
 ]
 
 
