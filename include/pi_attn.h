@@ -189,6 +189,22 @@ pi_attn_status pi_attn_bwd(const void* q, const void* k, const void* v, const fl
                            int n, int d, int k_win, int pi, int S, pi_attn_dtype dtype, int bidir, void* workspace,
                            long long workspace_bytes, void* stream);
 
+/* The backward with a choice of kernels.  PI_ATTN_BWD_SIMT is pi_attn_bwd: the forward recomputed
+ * in fp32 on CUDA cores with every product in fp32.  PI_ATTN_BWD_TC runs the forward's single
+ * tensor-core pass for out and lse, D_i = dout_i . out_i from that bf16 out, the dq pass on the
+ * tensor cores (S and dP by tcgen05 in fp32, ds rounded to bf16 for dQ += dS K) and the dk/dv
+ * pass on CUDA cores; its gradients carry the bf16 roundings of out, of P and of ds (relative
+ * errors of order 2^-9), against fp32 arithmetic for the other path.  bf16 with d in {64, 128}
+ * (else PI_ATTN_EUNSUPPORTED).  PI_ATTN_BWD_AUTO: the tensor-core path where it applies, else
+ * SIMT.  The workspace is pi_attn_bwd_workspace_bytes_ex(B, H, n, d, dtype, path) bytes (the
+ * tensor-core path adds the forward's out and lse); other arguments and errors as pi_attn_bwd. */
+typedef enum { PI_ATTN_BWD_AUTO = 0, PI_ATTN_BWD_SIMT = 1, PI_ATTN_BWD_TC = 2 } pi_attn_bwd_path;
+long long pi_attn_bwd_workspace_bytes_ex(int B, int H, int n, int d, pi_attn_dtype dtype, pi_attn_bwd_path path);
+pi_attn_status pi_attn_bwd_ex(const void* q, const void* k, const void* v, const float* w_g, const float* b_g,
+                              const void* dout, float* dq, float* dk, float* dv, float* dw_g, float* db_g, int B,
+                              int H, int n, int d, int k_win, int pi, int S, pi_attn_dtype dtype, int bidir,
+                              pi_attn_bwd_path path, void* workspace, long long workspace_bytes, void* stream);
+
 /* Decode over a compact ring cache (constant memory per sequence, constant-time update).  Cited
  * passage: "Execution & Scheduling" -- caches updated in constant time at inference.  Position j of
  * sequence b lives in slot j mod capacity of kcache / vcache [B, H, capacity, d]; the query is the

@@ -44,6 +44,9 @@ SIGNATURES = {
     # q k v w_g b_g dout dq dk dv dw_g db_g, B H n d k_win pi S dtype bidir, workspace, bytes, stream
     "pi_attn_bwd": (_i32, [_vp] * 11 + [_i32] * 9 + [_vp, ctypes.c_longlong, _vp]),
     "pi_attn_bwd_workspace_bytes": (ctypes.c_longlong, [_i32, _i32, _i32, _i32]),
+    # as pi_attn_bwd plus the kernel choice before the workspace
+    "pi_attn_bwd_ex": (_i32, [_vp] * 11 + [_i32] * 10 + [_vp, ctypes.c_longlong, _vp]),
+    "pi_attn_bwd_workspace_bytes_ex": (ctypes.c_longlong, [_i32] * 6),
     # as pi_attn_decode, capacity in place of n_cache
     "pi_attn_decode_ring": (_i32, [_vp] * 8 + [_i32] * 8 + [_vp]),
     # kcache vcache k_new v_new cache_len, B H capacity d dtype ring, stream
@@ -227,12 +230,16 @@ def pi_attn_debug_index_sets(n: int, k_win: int, pi: int, S: int, width: int | N
     return counts, idx
 
 
+BWD_PATHS = {"auto": 0, "simt": 1, "tc": 2}
+
+
 def pi_attn_bwd(q, k, v, w_g, b_g, dout, k_win: int, pi: int, S: int, *, bidir: bool = False, grads=None,
-                workspace=None, stream=None):
+                workspace=None, stream=None, path: str = "simt"):
     """Gradients of a loss through out: (dq, dk, dv, dw_g, db_g), fp32 tensors.  q, k, v, dout
     [B, H, n, d] in one dtype (fp32 or bf16); w_g [H, d], b_g [H] fp32.  grads: a tuple of the five
     output tensors to write into (allocated when None); workspace from torch's caching allocator
-    when None."""
+    when None.  path: "simt" (pi_attn_bwd, fp32 throughout), "tc" (the dq pass on the tensor
+    cores, pi_attn_bwd_ex) or "auto"."""
     import torch
     B, H, n, d = q.shape
     dev = q.device
@@ -243,12 +250,13 @@ def pi_attn_bwd(q, k, v, w_g, b_g, dout, k_win: int, pi: int, S: int, *, bidir: 
                  torch.empty((H, d), dtype=torch.float32, device=dev),
                  torch.empty((H,), dtype=torch.float32, device=dev))
     lib = load()
+    dt, pc = _dtype_code(q), BWD_PATHS[path]
     if workspace is None:
-        workspace = torch.empty(lib.pi_attn_bwd_workspace_bytes(B, H, n, d), dtype=torch.uint8, device=dev)
+        workspace = torch.empty(lib.pi_attn_bwd_workspace_bytes_ex(B, H, n, d, dt, pc), dtype=torch.uint8, device=dev)
     dq, dk, dv, dw, db = grads
-    st = lib.pi_attn_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(w_g), _ptr(b_g), _ptr(dout), _ptr(dq), _ptr(dk), _ptr(dv),
-                         _ptr(dw), _ptr(db), B, H, n, d, k_win, pi, S, _dtype_code(q), int(bidir), _ptr(workspace),
-                         workspace.numel(), _stream(stream))
+    st = lib.pi_attn_bwd_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(w_g), _ptr(b_g), _ptr(dout), _ptr(dq), _ptr(dk),
+                            _ptr(dv), _ptr(dw), _ptr(db), B, H, n, d, k_win, pi, S, dt, int(bidir), pc,
+                            _ptr(workspace), workspace.numel(), _stream(stream))
     _raise(st)
     return dq, dk, dv, dw, db
 

@@ -1,0 +1,408 @@
+// bwd_tc.cuh -- the backward's dq pass on Blackwell tensor cores (tcgen05 + TMEM + TMA), bf16,
+// head size 64 or 128.
+//
+// One CTA per (query tile of 128 rows, b, h), walking the key tiles of the forward (the same
+// TileCursor over the same index rule).  Per 64-key tile:
+//   MMA warp            S = Q K^T and dP = dO V^T (fp32 in TMEM), then, once the softmax warps
+//                       have written dS, dQ += dS K (fp32 in TMEM; dS from TMEM, K N-major)
+//   softmax warpgroup   one thread per query row: p = 2^(s tau log2e + prior - lse2) on the keys
+//                       the index rule gives (0 elsewhere), ds = p (dp - D), written in bf16 over
+//                       the S columns already read; the row's dz = (1 - alpha) sum_window ds -
+//                       alpha sum_skip ds (the gate's gradient through the two log-priors)
+//   TMA producer warp   Q and dO tiles once, then K and V tiles into a 2-stage ring
+// lse and D = dO . out of every row come from the forward pass (its epilogue forms D from the
+// fp32 output rows).  The epilogue writes dq = tau dQ + dz w_g (fp32) and the row terms the dk/dv
+// pass and the gate sums read (lse2, log2-priors, dz).
+//
+// TMEM: S at columns 0..63, dP at 64..127, dQ at 128..128+D.  One S/dP pair: the next tile's
+// Q K^T waits for this tile's dS K (it reads dS over the S columns).  Every wait is bounded as in
+// the forward kernel; a wait that gives up sets the error word and the abort flag, and every role
+// leaves, drains its own asynchronous work and the CTA frees its TMEM.
+#pragma once
+#include "fwd_tc.cuh"
+
+namespace pia {
+namespace tcb {
+using tc::BM;
+using tc::BN;
+using tc::NSTAGE;
+
+template <int D>
+struct BSmem {
+  static constexpr int kCtas = D == 64 ? 2 : 1;         // shared memory: 64 KB (D = 64) or 128 KB
+  static constexpr int kTileBytes = BM * D * 2;          // the Q tile, the dO tile
+  static constexpr int kKVBytes = BN * D * 2;            // one K or V tile
+  static constexpr int kQ = 0;
+  static constexpr int kG = kQ + kTileBytes;
+  static constexpr int kK = kG + kTileBytes;
+  static constexpr int kV = kK + NSTAGE * kKVBytes;
+  static constexpr int kBar = kV + NSTAGE * kKVBytes;
+  // barriers: qg_full, k_full[NSTAGE], k_empty[NSTAGE], v_full[NSTAGE], v_empty[NSTAGE], s_full,
+  // ds_full, dq_done, drain
+  static constexpr int kNumBars = 1 + 4 * NSTAGE + 4;
+  static constexpr int kMisc = kBar + kNumBars * 8;      // tmem base (4 B), abort flag (4 B)
+  static constexpr int kWg = (kMisc + 8 + 15) / 16 * 16; // w_g[h], D floats
+  static constexpr int kTotal = kWg + D * 4;
+  static constexpr int kAlloc = kTotal + 1024 - 128;
+  static constexpr int kTmemCols = 256;
+  static_assert(2 * BN + D <= kTmemCols && kTmemCols * kCtas <= 512, "TMEM columns");
+  static_assert(kQ % 1024 == 0 && kG % 1024 == 0 && kK % 1024 == 0 && kV % 1024 == 0 && kKVBytes % 1024 == 0,
+                "128-byte-swizzled tiles sit on 1 KB");
+  static_assert(kBar % 8 == 0 && kWg % 16 == 0, "mbarriers on 8 bytes, the w_g staging on 16");
+  static_assert(kAlloc <= 228 * 1024 / kCtas - 1024, "shared memory of the CTAs on one SM");
+};
+
+struct BParams {
+  const float* w_g;
+  const float* b_g;
+  const float* lse;   // [B*H, n] the forward's lse (natural log)
+  const float* Dr;    // [B*H, n] dO . out
+  float* lse2;        // [B*H, n] lse in log2 units, for the dk/dv pass
+  float* dq;          // [B*H, n, D]
+  float* bl2;         // [B*H, n] log2(alpha), log2(1 - alpha), dz: for the dk/dv pass and the gate
+  float* bp2;
+  float* dz;
+  int H, n, kwin, pi, S;
+  float scale_log2;
+  int bidir;
+};
+
+template <int D>
+__global__ void __launch_bounds__(192, BSmem<D>::kCtas) bwd_dq_kernel(const __grid_constant__ CUtensorMap tmq,
+                                                                       const __grid_constant__ CUtensorMap tmg,
+                                                                       const __grid_constant__ CUtensorMap tmk,
+                                                                       const __grid_constant__ CUtensorMap tmv,
+                                                                       BParams prm) {
+  using namespace tc;
+  using L = BSmem<D>;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  uint8_t* const sbase = smem_raw + (base - raw);
+  if (base - raw + L::kTotal > (uint32_t)L::kAlloc) {
+    if (threadIdx.x == 0) raise_error(kErrInternal);
+    return;
+  }
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int bh = blockIdx.y;
+  const int h = bh % prm.H;
+  const long long q0 = (long long)blockIdx.x * BM;
+  const uint32_t sQ = base + L::kQ, sG = base + L::kG, sK = base + L::kK, sV = base + L::kV;
+  const uint32_t bar0 = base + L::kBar;
+  const uint32_t bar_qg = bar0;
+  auto bar_kfull = [&](int s) { return bar0 + 8u * (1 + s); };
+  auto bar_kempty = [&](int s) { return bar0 + 8u * (1 + NSTAGE + s); };
+  auto bar_vfull = [&](int s) { return bar0 + 8u * (1 + 2 * NSTAGE + s); };
+  auto bar_vempty = [&](int s) { return bar0 + 8u * (1 + 3 * NSTAGE + s); };
+  const uint32_t bar_sfull = bar0 + 8u * (1 + 4 * NSTAGE);
+  const uint32_t bar_dsfull = bar_sfull + 8;
+  const uint32_t bar_dqdone = bar_sfull + 16;
+  const uint32_t bar_drain = bar_sfull + 24;
+  uint32_t* const tmem_slot = reinterpret_cast<uint32_t*>(sbase + L::kMisc);
+  volatile int* const abort_flag = reinterpret_cast<volatile int*>(sbase + L::kMisc + 4);
+
+  // Q and dO first: their latency heads every CTA's critical path
+  if (threadIdx.x == 0) {
+    asm volatile("prefetch.tensormap [%0];" ::"l"(&tmq) : "memory");
+    asm volatile("prefetch.tensormap [%0];" ::"l"(&tmg) : "memory");
+    asm volatile("prefetch.tensormap [%0];" ::"l"(&tmk) : "memory");
+    asm volatile("prefetch.tensormap [%0];" ::"l"(&tmv) : "memory");
+    mbar_init(bar_qg, 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    mbar_expect_tx(bar_qg, 2 * L::kTileBytes);
+#pragma unroll
+    for (int c = 0; c < D / 64; ++c) {
+      tma_load_3d(sQ + c * BM * 128, &tmq, bar_qg, c * 64, (int)q0, bh);
+      tma_load_3d(sG + c * BM * 128, &tmg, bar_qg, c * 64, (int)q0, bh);
+    }
+  }
+  const int m0 = first_skip_m(prm.kwin, prm.pi);
+  TileWalk walk;
+  walk.init(q0, prm.n, BM, prm.kwin, prm.pi, prm.S, prm.bidir != 0);
+  TileCursor cur;
+  cur.init(walk);
+  int t_first = -1;
+  auto load_kv = [&](uint32_t dst, const CUtensorMap* map, uint32_t bar, long long r0) {
+#pragma unroll
+    for (int c = 0; c < D / 64; ++c) tma_load_3d(dst + c * BN * 128, map, bar, c * 64, (int)r0, bh);
+  };
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < NSTAGE; ++s) {
+      mbar_init(bar_kfull(s), 1);
+      mbar_init(bar_kempty(s), 1);
+      mbar_init(bar_vfull(s), 1);
+      mbar_init(bar_vempty(s), 1);
+    }
+    mbar_init(bar_sfull, 1);
+    mbar_init(bar_dsfull, BM);
+    mbar_init(bar_dqdone, 1);
+    mbar_init(bar_drain, 1);
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    t_first = cur.next();
+    if (t_first >= 0) {
+      mbar_expect_tx(bar_kfull(0), L::kKVBytes);
+      load_kv(sK, &tmk, bar_kfull(0), (long long)t_first * BN);
+      mbar_expect_tx(bar_vfull(0), L::kKVBytes);
+      load_kv(sV, &tmv, bar_vfull(0), (long long)t_first * BN);
+    }
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
+                 "n"(L::kTmemCols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t tS = tmem, tP = tmem + BN, tQ = tmem + 2 * BN;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      constexpr uint32_t kKV = L::kKVBytes;
+      int nk = t_first >= 0 ? 1 : 0, nv = nk;
+      for (int t = cur.next(); t >= 0; t = cur.next()) {
+        const int s = nk % NSTAGE, use = nk / NSTAGE;
+        if (use > 0 && !mbar_wait(bar_kempty(s), (use - 1) & 1, abort_flag)) break;
+        mbar_expect_tx(bar_kfull(s), kKV);
+        load_kv(sK + s * kKV, &tmk, bar_kfull(s), (long long)t * BN);
+        ++nk;
+        if (use > 0 && !mbar_wait(bar_vempty(s), (use - 1) & 1, abort_flag)) break;
+        mbar_expect_tx(bar_vfull(s), kKV);
+        load_kv(sV + s * kKV, &tmv, bar_vfull(s), (long long)t * BN);
+        ++nv;
+      }
+      if (*abort_flag) {  // let the loads already in flight land before the CTA can exit
+        volatile int never = 0;
+        mbar_wait(bar_qg, 0, &never);
+        for (int u = nk > NSTAGE ? nk - NSTAGE : 0; u < nk; ++u)
+          mbar_wait(bar_kfull(u % NSTAGE), (u / NSTAGE) & 1, &never);
+        for (int u = nv > NSTAGE ? nv - NSTAGE : 0; u < nv; ++u)
+          mbar_wait(bar_vfull(u % NSTAGE), (u / NSTAGE) & 1, &never);
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ------------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t kKV = L::kKVBytes;
+      constexpr uint32_t idesc_s = idesc_bf16(BM, BN, 0);  // S, dP: B (K, V) K-major
+      constexpr uint32_t idesc_q = idesc_bf16(BM, D, 1);   // dQ: B (K) N-major
+      bool okw = mbar_wait(bar_qg, 0, abort_flag);
+      tc_fence_after();
+      int j = 0;
+      for (int t = cur.next(); okw && t >= 0; t = cur.next(), ++j) {
+        const int s = j % NSTAGE;
+        if (!mbar_wait(bar_kfull(s), (j / NSTAGE) & 1, abort_flag)) break;
+        if (!mbar_wait(bar_vfull(s), (j / NSTAGE) & 1, abort_flag)) break;
+        // the dS K of the previous tile read dS over the S columns this Q K^T overwrites
+        if (j > 0 && !mbar_wait(bar_dqdone, (j - 1) & 1, abort_flag)) break;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t in = (kk & 3) * 32;
+          tc_mma(tS, sw128_desc(sQ + (kk >> 2) * (BM * 128) + in, 16, 1024),
+                 sw128_desc(sK + s * kKV + (kk >> 2) * (BN * 128) + in, 16, 1024), idesc_s, kk > 0 ? 1u : 0u);
+        }
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t in = (kk & 3) * 32;
+          tc_mma(tP, sw128_desc(sG + (kk >> 2) * (BM * 128) + in, 16, 1024),
+                 sw128_desc(sV + s * kKV + (kk >> 2) * (BN * 128) + in, 16, 1024), idesc_s, kk > 0 ? 1u : 0u);
+        }
+        tc_commit(bar_sfull);
+        tc_commit(bar_vempty(s));  // V was read by dO V^T only
+        if (!mbar_wait(bar_dsfull, j & 1, abort_flag)) break;
+        tc_fence_after();
+        // dQ += dS K : K = BN keys, 16 per instruction; dS packed two per column over S
+#pragma unroll
+        for (int kk = 0; kk < BN / 16; ++kk) {
+          const uint32_t acol = 16 * (kk >> 1) + 8 * (kk & 1);
+          tc_mma_ts(tQ, tS + acol, sw128_desc(sK + s * kKV + kk * 16 * 128, BN * 128, 1024), idesc_q,
+                    (j == 0 && kk == 0) ? 0u : 1u);
+        }
+        tc_commit(bar_dqdone);
+        tc_commit(bar_kempty(s));
+      }
+      tc_commit(bar_drain);
+      volatile int never = 0;
+      mbar_wait(bar_drain, 0, &never);
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------------ softmax warpgroup
+    const int q4 = warp & 3;
+    const int r = q4 * 32 + lane;
+    const long long i = q0 + r;
+    const bool row_ok = i < prm.n;
+    const long long orow = (long long)bh * prm.n + (row_ok ? i : 0);
+    const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
+    const float lse2 = row_ok ? prm.lse[orow] * kLog2e : 0.f;
+    const float Drow = row_ok ? prm.Dr[orow] : 0.f;
+    const long long w_lo = i - prm.kwin > 0 ? i - prm.kwin : 0;
+    const long long w_hi = prm.bidir ? (i + prm.kwin < prm.n - 1 ? i + prm.kwin : prm.n - 1) : i;
+    RowSkips rs;
+    rs.init(i, prm.pi, prm.S, m0, walk.rpi, prm.bidir != 0, prm.n);
+
+    float* const wg_s = reinterpret_cast<float*>(sbase + L::kWg);
+    if (threadIdx.x - 64 < D) wg_s[threadIdx.x - 64] = prm.w_g[(long long)h * D + (threadIdx.x - 64)];
+    float z = prm.b_g[h];
+    asm volatile("bar.sync 1, 128;" ::: "memory");
+    bool ok = __all_sync(0xffffffffu, mbar_wait(bar_qg, 0, abort_flag));
+    {
+      float zp[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int c = 0; c < D / 8; ++c) {
+        const int blk = c >> 3, cc = c & 7;
+        const uint4 u = *reinterpret_cast<const uint4*>(sbase + L::kQ + blk * (BM * 128) + r * 128 +
+                                                        ((cc ^ (r & 7)) << 4));
+        float f[8];
+        bf16x8_to_f32(u, f);
+        const float4 w0 = reinterpret_cast<const float4*>(wg_s)[2 * c];
+        const float4 w1 = reinterpret_cast<const float4*>(wg_s)[2 * c + 1];
+        zp[0] = fmaf(f[0], w0.x, zp[0]);
+        zp[1] = fmaf(f[1], w0.y, zp[1]);
+        zp[2] = fmaf(f[2], w0.z, zp[2]);
+        zp[3] = fmaf(f[3], w0.w, zp[3]);
+        zp[0] = fmaf(f[4], w1.x, zp[0]);
+        zp[1] = fmaf(f[5], w1.y, zp[1]);
+        zp[2] = fmaf(f[6], w1.z, zp[2]);
+        zp[3] = fmaf(f[7], w1.w, zp[3]);
+      }
+      z += (zp[0] + zp[1]) + (zp[2] + zp[3]);
+    }
+    const float ls_a = log_sigmoid_fast(z), ls_b = log_sigmoid_fast(-z);
+    const float alpha = __expf(ls_a);
+    const float bl2 = ls_a * kLog2e, bp2 = ls_b * kLog2e;
+    const float bl_m = bl2 - lse2, bp_m = bp2 - lse2;
+    const float NEG_INF = -INFINITY;
+    float dzw = 0.f, dzs = 0.f;  // sums of ds over window keys and over skip keys
+
+    int j = 0;
+    for (int t = cur.next(); ok && t >= 0; t = cur.next(), ++j) {
+      if (!__all_sync(0xffffffffu, mbar_wait(bar_sfull, j & 1, abort_flag))) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      const long long j0 = (long long)t * BN;
+      const long long lo64 = w_lo - j0, hi64 = w_hi - j0;
+      const int lc_lo = lo64 < 0 ? 0 : (lo64 > BN ? BN : (int)lo64);
+      const int lc_hi = hi64 > BN - 1 ? BN - 1 : (hi64 < -1 ? -1 : (int)hi64);
+      const uint64_t skw = rs.take(j0);
+#pragma unroll 1
+      for (int cb = 0; cb < BN / 32; ++cb) {
+        const int c0 = cb * 32;
+        float x[32], g[32];
+        tmem_ld32(tS + lane_off + c0, x);
+        tmem_ld32(tP + lane_off + c0, g);
+        const uint32_t wm = window_bits(lc_lo - c0, lc_hi - c0);
+        const uint32_t skb = (uint32_t)(skw >> c0);
+        uint32_t pk[16];
+        if ((wm | skb) == 0u) {
+#pragma unroll
+          for (int w = 0; w < 16; ++w) pk[w] = 0u;
+        } else {
+          const unsigned long long sc2 = f2pack(prm.scale_log2, prm.scale_log2);
+          const unsigned long long nd2 = f2pack(-Drow, -Drow);
+#pragma unroll
+          for (int e = 0; e < 32; e += 2) {
+            const bool w0 = (wm >> e) & 1u, w1 = (wm >> (e + 1)) & 1u;
+            const bool s0 = (skb >> e) & 1u, s1 = (skb >> (e + 1)) & 1u;
+            const float b0 = w0 ? bl_m : (s0 ? bp_m : NEG_INF);
+            const float b1 = w1 ? bl_m : (s1 ? bp_m : NEG_INF);
+            float t0, t1;
+            f2unpack(f2fma(f2pack(x[e], x[e + 1]), sc2, f2pack(b0, b1)), t0, t1);
+            float ds0, ds1;
+            f2unpack(f2mul(f2pack(ex2(t0), ex2(t1)), f2add(f2pack(g[e], g[e + 1]), nd2)), ds0, ds1);
+            dzw += (w0 ? ds0 : 0.f) + (w1 ? ds1 : 0.f);
+            dzs += (s0 ? ds0 : 0.f) + (s1 ? ds1 : 0.f);
+            __nv_bfloat162 b2 = __floats2bfloat162_rn(ds0, ds1);
+            pk[e >> 1] = *reinterpret_cast<uint32_t*>(&b2);
+          }
+        }
+        __syncwarp();
+        tmem_st16(tS + lane_off + 16 * cb, pk);  // over S columns already read
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(bar_dsfull);
+    }
+    // ---- epilogue: dq = tau dQ + dz w_g, and the row terms
+    const float dz = (1.f - alpha) * dzw - alpha * dzs;
+    const bool have_q = __all_sync(0xffffffffu, ok && j > 0 && mbar_wait(bar_dqdone, (j - 1) & 1, abort_flag));
+    if (have_q) tc_fence_after();
+    const float tau = prm.scale_log2 / kLog2e;
+    if (have_q || j == 0) {
+#pragma unroll 1
+      for (int c = 0; c < D / 32; ++c) {
+        float o[32];
+        if (have_q) {
+          tmem_ld32(tQ + lane_off + c * 32, o);
+        } else {
+#pragma unroll
+          for (int e = 0; e < 32; ++e) o[e] = 0.f;
+        }
+        if (row_ok) {
+          float4* dst = reinterpret_cast<float4*>(prm.dq + orow * D + c * 32);
+          const float4* wv = reinterpret_cast<const float4*>(wg_s + c * 32);
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            const float4 w = wv[e];
+            dst[e] = make_float4(fmaf(tau, o[4 * e], dz * w.x), fmaf(tau, o[4 * e + 1], dz * w.y),
+                                 fmaf(tau, o[4 * e + 2], dz * w.z), fmaf(tau, o[4 * e + 3], dz * w.w));
+          }
+        }
+      }
+      if (row_ok) {
+        prm.lse2[orow] = lse2;
+        prm.bl2[orow] = bl2;
+        prm.bp2[orow] = bp2;
+        prm.dz[orow] = dz;
+      }
+    }
+    tc_fence_before();
+  }
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) {
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "n"(L::kTmemCols) : "memory");
+  }
+}
+
+template <int D>
+cudaError_t set_bwd_smem_attr() {
+  static bool done = false;
+  if (done) return cudaSuccess;
+  cudaError_t e =
+      cudaFuncSetAttribute(bwd_dq_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, BSmem<D>::kAlloc);
+  if (e == cudaSuccess) done = true;
+  return e;
+}
+
+// The dq pass: q, dout [BH, n, D] bf16, k, v [BH, n, D] bf16; lse, Dr [BH, n] from the forward.
+template <int D>
+cudaError_t launch_bwd_dq(const void* q, const void* k, const void* v, const void* dout, const BParams& p, int BH,
+                          cudaStream_t st, const char** why) {
+  CUtensorMap mq, mg, mk, mv;
+  if (!tc::make_map(&mq, q, BH, p.n, D, BM) || !tc::make_map(&mg, dout, BH, p.n, D, BM) ||
+      !tc::make_map(&mk, k, BH, p.n, D, BN) || !tc::make_map(&mv, v, BH, p.n, D, BN)) {
+    *why = "cuTensorMapEncodeTiled failed";
+    return cudaErrorInvalidValue;
+  }
+  cudaError_t e = set_bwd_smem_attr<D>();
+  if (e != cudaSuccess) {
+    *why = "cudaFuncSetAttribute";
+    return e;
+  }
+  const dim3 grid((unsigned)((p.n + BM - 1) / BM), (unsigned)BH);
+  bwd_dq_kernel<D><<<grid, 192, BSmem<D>::kAlloc, st>>>(mq, mg, mk, mv, p);
+  *why = "tensor-core dq kernel launch";
+  return cudaGetLastError();
+}
+
+}  // namespace tcb
+}  // namespace pia

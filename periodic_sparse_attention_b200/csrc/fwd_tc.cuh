@@ -332,6 +332,10 @@ struct Params {
   // kFused over one shard of a longer sequence: q/out/lse row r is sequence row row0 + r; k/v
   // row r is sequence row kv0 + r (the index rule runs in sequence rows).  0 and 0 otherwise.
   long long row0, kv0;
+  // kFused for the backward: with dout given, the epilogue also writes Dout[row] = dout . out
+  // from the fp32 output row (before its rounding to bf16).  Null otherwise.
+  const __nv_bfloat16* dout;
+  float* Dout;
 };
 
 template <int D, int MODE>
@@ -930,6 +934,17 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm<D>) fwd_tc_kernel(const _
         }
         *reinterpret_cast<uint4*>(sbase + L::kV + off) = make_uint4(w[0], w[1], w[2], w[3]);
       }
+      if (MODE == kFused && prm.dout && row_ok) {
+        float dsum = 0.f;
+#pragma unroll
+        for (int cl = 0; cl < D / 8; ++cl) {
+          float g[8];
+          bf16x8_to_f32(*reinterpret_cast<const uint4*>(prm.dout + orow * D + cl * 8), g);
+#pragma unroll
+          for (int e = 0; e < 8; ++e) dsum = fmaf(o[cl * 8 + e] * inv, g[e], dsum);
+        }
+        prm.Dout[orow] = dsum;
+      }
       lse_log2 = lse2;
       fence_proxy_async_smem();
     }
@@ -1067,6 +1082,8 @@ cudaError_t launch_fwd_tc_d(const void* q, const void* k, const void* v, const f
   p.bidir = bidir ? 1 : 0;
   p.row0 = 0;
   p.kv0 = 0;
+  p.dout = nullptr;
+  p.Dout = nullptr;
   const dim3 grid((unsigned)((n + tc::BM - 1) / tc::BM), (unsigned)BH);
   cudaError_t e;
   CUtensorMap mo;
@@ -1150,11 +1167,54 @@ cudaError_t launch_fwd_tc_shard_d(const void* q, const void* k, const void* v, c
   p.bidir = 0;
   p.row0 = row0;
   p.kv0 = kv0;
+  p.dout = nullptr;
+  p.Dout = nullptr;
   cudaError_t e;
   if ((e = tc::set_smem_attr<D, tc::kFused>()) != cudaSuccess) { *why = "cudaFuncSetAttribute"; return e; }
   const dim3 grid((unsigned)((n_q + tc::BM - 1) / tc::BM), (unsigned)BH);
   tc::fwd_tc_kernel<D, tc::kFused><<<grid, tc::kThreads, L::kAlloc, st>>>(mq, mk, mv, mo, mo, p);
   *why = "tensor-core shard kernel launch";
+  return cudaGetLastError();
+}
+
+// The backward's forward: the single pass over a whole sequence, writing out, lse and, from the
+// fp32 output rows, D = dout . out of every row.
+template <int D>
+cudaError_t launch_fwd_tc_with_dot(const void* q, const void* k, const void* v, const float* w_g, const float* b_g,
+                                   const void* dout, void* out, float* lse, float* Dout, int B, int H, int n, int kwin,
+                                   int pi, int S, bool bidir, cudaStream_t st, const char** why) {
+  using L = tc::Smem<D>;
+  CUtensorMap mq, mk, mv, mo;
+  const int BH = B * H;
+  if (!tc::make_map(&mq, q, BH, n, D, tc::BM) || !tc::make_map(&mk, k, BH, n, D, tc::BN) ||
+      !tc::make_map(&mv, v, BH, n, D, tc::BN) || !tc::make_map(&mo, out, BH, n, D, tc::BM)) {
+    *why = "cuTensorMapEncodeTiled failed";
+    return cudaErrorInvalidValue;
+  }
+  tc::Params p;
+  p.w_g = w_g;
+  p.b_g = b_g;
+  p.out = (__nv_bfloat16*)out;
+  p.lse = lse;
+  p.skip_o = nullptr;
+  p.skip_lse = nullptr;
+  p.H = H;
+  p.n = n;
+  p.kwin = kwin;
+  p.pi = pi;
+  p.S = S;
+  p.T = 0;
+  p.scale_log2 = (float)(1.0 / std::sqrt((double)D)) * kLog2e;
+  p.bidir = bidir ? 1 : 0;
+  p.row0 = 0;
+  p.kv0 = 0;
+  p.dout = (const __nv_bfloat16*)dout;
+  p.Dout = Dout;
+  cudaError_t e;
+  if ((e = tc::set_smem_attr<D, tc::kFused>()) != cudaSuccess) { *why = "cudaFuncSetAttribute"; return e; }
+  const dim3 grid((unsigned)((n + tc::BM - 1) / tc::BM), (unsigned)BH);
+  tc::fwd_tc_kernel<D, tc::kFused><<<grid, tc::kThreads, L::kAlloc, st>>>(mq, mk, mv, mo, mo, p);
+  *why = "tensor-core forward (backward's) launch";
   return cudaGetLastError();
 }
 

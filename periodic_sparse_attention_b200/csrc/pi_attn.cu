@@ -15,6 +15,7 @@
 #include "decode.cuh"
 #include "fwd_simt.cuh"
 #include "fwd_tc.cuh"
+#include "bwd_tc.cuh"
 
 namespace {
 
@@ -117,7 +118,8 @@ pi_attn_status launch_simt(const void* q, const void* k, const void* v, const fl
 template <typename T, int CPT>
 cudaError_t launch_bwd_cpt(const void* q, const void* k, const void* v, const float* w_g, const float* b_g,
                            const void* dout, float* dq, float* dk, float* dv, pia::BwdRowStats rs, dim3 grid, int H,
-                           int n, int d, int kwin, int pi, int S, float scale_log2, bool bidir, cudaStream_t s) {
+                           int n, int d, int kwin, int pi, int S, float scale_log2, bool bidir, cudaStream_t s,
+                           bool row_pass) {
   static bool attr_done = false;
   const size_t sr = pia::bwd_row_smem(d, sizeof(T)), sk = pia::bwd_key_smem(d, sizeof(T));
   if (!attr_done) {
@@ -129,11 +131,13 @@ cudaError_t launch_bwd_cpt(const void* q, const void* k, const void* v, const fl
     if (e != cudaSuccess) return e;
     attr_done = true;
   }
-  pia::bwd_row_kernel<T, CPT><<<grid, pia::kBwdThreads, sr, s>>>((const T*)q, (const T*)k, (const T*)v, w_g, b_g,
-                                                                 (const T*)dout, dq, rs, H, n, d, kwin, pi, S,
-                                                                 scale_log2, bidir);
-  cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
+  if (row_pass) {  // else the rows' terms (lse2, D, priors, dz) and dq come from the tensor-core dq pass
+    pia::bwd_row_kernel<T, CPT><<<grid, pia::kBwdThreads, sr, s>>>((const T*)q, (const T*)k, (const T*)v, w_g, b_g,
+                                                                   (const T*)dout, dq, rs, H, n, d, kwin, pi, S,
+                                                                   scale_log2, bidir);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
   pia::bwd_key_kernel<T, CPT><<<grid, pia::kBwdThreads, sk, s>>>((const T*)q, (const T*)k, (const T*)v,
                                                                  (const T*)dout, rs, dk, dv, H, n, d, kwin, pi, S,
                                                                  scale_log2, bidir);
@@ -143,18 +147,31 @@ cudaError_t launch_bwd_cpt(const void* q, const void* k, const void* v, const fl
 template <typename T>
 cudaError_t launch_bwd(const void* q, const void* k, const void* v, const float* w_g, const float* b_g,
                        const void* dout, float* dq, float* dk, float* dv, pia::BwdRowStats rs, dim3 grid, int H, int n,
-                       int d, int kwin, int pi, int S, float scale_log2, bool bidir, cudaStream_t s) {
+                       int d, int kwin, int pi, int S, float scale_log2, bool bidir, cudaStream_t s,
+                       bool row_pass = true) {
   if (d <= 64)
-    return launch_bwd_cpt<T, 8>(q, k, v, w_g, b_g, dout, dq, dk, dv, rs, grid, H, n, d, kwin, pi, S, scale_log2, bidir, s);
+    return launch_bwd_cpt<T, 8>(q, k, v, w_g, b_g, dout, dq, dk, dv, rs, grid, H, n, d, kwin, pi, S, scale_log2, bidir, s,
+                                row_pass);
   if (d <= 128)
     return launch_bwd_cpt<T, 16>(q, k, v, w_g, b_g, dout, dq, dk, dv, rs, grid, H, n, d, kwin, pi, S, scale_log2, bidir,
-                                 s);
+                                 s, row_pass);
   return launch_bwd_cpt<T, 32>(q, k, v, w_g, b_g, dout, dq, dk, dv, rs, grid, H, n, d, kwin, pi, S, scale_log2, bidir,
-                               s);
+                               s, row_pass);
 }
 
 static long long gate_chunks(int B, int n) {
   return ((long long)B * n + pia::kGateRows - 1) / pia::kGateRows;
+}
+
+// Backward scratch: lse2, D, two log2-priors and dz per query row, then the gate's per-chunk
+// partial sums (fp32); the tensor-core path adds, 16-byte aligned, the forward's out (bf16) and
+// lse (fp32) of every row.
+static long long bwd_ws_bytes(int B, int H, int n, int d, bool tc) {
+  if (B < 1 || H < 1 || n < 1 || d < 1) return 0;
+  const long long base = 4LL * (5LL * B * H * n + (long long)H * gate_chunks(B, n) * (d + 1));
+  if (!tc) return base;
+  const long long rows = (long long)B * H * n;
+  return (base + 15) / 16 * 16 + rows * 2LL * d + rows * 4LL;
 }
 
 }  // namespace
@@ -503,22 +520,31 @@ pi_attn_status pi_attn_debug_index_sets_bidir(int n, int k_win, int pi, int S, i
   return index_sets_impl(n, k_win, pi, S, counts, idx, width, true, stream);
 }
 
-long long pi_attn_bwd_workspace_bytes(int B, int H, int n, int d) {
-  if (B < 1 || H < 1 || n < 1 || d < 1) return 0;
-  // lse2, D, two log2-priors and dz per query row, then the gate's per-chunk partial sums (fp32)
-  return 4LL * (5LL * B * H * n + (long long)H * gate_chunks(B, n) * (d + 1));
+long long pi_attn_bwd_workspace_bytes(int B, int H, int n, int d) { return bwd_ws_bytes(B, H, n, d, false); }
+
+long long pi_attn_bwd_workspace_bytes_ex(int B, int H, int n, int d, pi_attn_dtype dtype, pi_attn_bwd_path path) {
+  const bool tc = path == PI_ATTN_BWD_TC ||
+                  (path == PI_ATTN_BWD_AUTO && dtype == PI_ATTN_BF16 && (d == 64 || d == 128));
+  return bwd_ws_bytes(B, H, n, d, tc);
 }
 
-pi_attn_status pi_attn_bwd(const void* q, const void* k, const void* v, const float* w_g, const float* b_g,
-                           const void* dout, float* dq, float* dk, float* dv, float* dw_g, float* db_g, int B, int H,
-                           int n, int d, int k_win, int pi, int S, pi_attn_dtype dtype, int bidir, void* workspace,
-                           long long workspace_bytes, void* stream) {
+pi_attn_status pi_attn_bwd_ex(const void* q, const void* k, const void* v, const float* w_g, const float* b_g,
+                              const void* dout, float* dq, float* dk, float* dv, float* dw_g, float* db_g, int B,
+                              int H, int n, int d, int k_win, int pi, int S, pi_attn_dtype dtype, int bidir,
+                              pi_attn_bwd_path path, void* workspace, long long workspace_bytes, void* stream) {
   pi_attn_status st = check_common(q, k, v, w_g, b_g, dout, B, H, n, d, k_win, pi, S, dtype);
   if (st != PI_ATTN_OK) return st;
   if (!dq || !dk || !dv || !dw_g || !db_g) return fail(PI_ATTN_EINVAL, "null gradient pointer");
   if (!aligned16(dq) || !aligned16(dk) || !aligned16(dv)) return fail(PI_ATTN_EINVAL, "dq, dk, dv must be 16-byte aligned");
+  if (path != PI_ATTN_BWD_AUTO && path != PI_ATTN_BWD_SIMT && path != PI_ATTN_BWD_TC)
+    return fail(PI_ATTN_EINVAL, "unknown backward path %d", (int)path);
+  const bool tc_ok = dtype == PI_ATTN_BF16 && (d == 64 || d == 128);
+  if (path == PI_ATTN_BWD_TC && !tc_ok)
+    return fail(PI_ATTN_EUNSUPPORTED, "the tensor-core backward covers bf16 with d in {64, 128} (got dtype %d, d %d)",
+                (int)dtype, d);
+  const bool tc = path == PI_ATTN_BWD_TC || (path == PI_ATTN_BWD_AUTO && tc_ok);
   const long long rows = (long long)B * H * n;
-  const long long need = pi_attn_bwd_workspace_bytes(B, H, n, d);
+  const long long need = bwd_ws_bytes(B, H, n, d, tc);
   if (workspace) {
     if (reinterpret_cast<uintptr_t>(workspace) % 16 != 0) return fail(PI_ATTN_EINVAL, "workspace not 16-byte aligned");
     if (workspace_bytes < need)
@@ -526,6 +552,8 @@ pi_attn_status pi_attn_bwd(const void* q, const void* k, const void* v, const fl
   }
   const long long tiles = ((long long)n + pia::kBwdRows - 1) / pia::kBwdRows;
   if (tiles > 0x7fffffffLL || (long long)B * H > 65535) return fail(PI_ATTN_EINVAL, "grid too large");
+  const long long nchunks = gate_chunks(B, n);
+  if (nchunks > 0x7fffffffLL || H > 65535) return fail(PI_ATTN_EINVAL, "too many rows per head for the gate sums");
   cudaStream_t s = as_stream(stream);
   void* scratch = workspace;
   cudaError_t e = cudaSuccess;
@@ -533,30 +561,74 @@ pi_attn_status pi_attn_bwd(const void* q, const void* k, const void* v, const fl
     return cuda_fail(e, "backward scratch allocation");
   float* base = static_cast<float*>(scratch);
   pia::BwdRowStats rs{base, base + rows, base + 2 * rows, base + 3 * rows, base + 4 * rows};
-  const long long nchunks = gate_chunks(B, n);
-  if (nchunks > 0x7fffffffLL || H > 65535) return fail(PI_ATTN_EINVAL, "too many rows per head for the gate sums");
   float* part_w = base + 5 * rows;
   float* part_b = part_w + (long long)H * nchunks * d;
   const dim3 gg((unsigned)nchunks, (unsigned)H);
   const float scale_log2 = (float)(1.0 / std::sqrt((double)d)) * pia::kLog2e;
   const bool bd = bidir != 0;
   const dim3 gt((unsigned)tiles, (unsigned)(B * H));
-  if (dtype == PI_ATTN_F32) {
+  const char* why = "backward kernel launch";
+  using bf = __nv_bfloat16;
+  if (tc) {
+    // the forward (single tensor-core pass) for out, lse and D = dO . out (from its fp32 output
+    // rows), then the dq pass on the tensor cores, then the dk/dv pass
+    const long long off = (bwd_ws_bytes(B, H, n, d, false) + 15) / 16 * 16;
+    bf* out_ws = reinterpret_cast<bf*>(static_cast<char*>(scratch) + off);
+    float* lse_ws = reinterpret_cast<float*>(static_cast<char*>(scratch) + off + rows * 2LL * d);
+    e = d == 128 ? pia::launch_fwd_tc_with_dot<128>(q, k, v, w_g, b_g, dout, out_ws, lse_ws, rs.D, B, H, n, k_win,
+                                                    pi, S, bd, s, &why)
+                 : pia::launch_fwd_tc_with_dot<64>(q, k, v, w_g, b_g, dout, out_ws, lse_ws, rs.D, B, H, n, k_win, pi,
+                                                   S, bd, s, &why);
+    if (e == cudaSuccess) {
+      pia::tcb::BParams bp;
+      bp.w_g = w_g;
+      bp.b_g = b_g;
+      bp.lse = lse_ws;
+      bp.Dr = rs.D;
+      bp.lse2 = rs.lse2;
+      bp.dq = dq;
+      bp.bl2 = rs.bl2;
+      bp.bp2 = rs.bp2;
+      bp.dz = rs.dz;
+      bp.H = H;
+      bp.n = n;
+      bp.kwin = k_win;
+      bp.pi = pi;
+      bp.S = S;
+      bp.scale_log2 = scale_log2;
+      bp.bidir = bd ? 1 : 0;
+      e = d == 128 ? pia::tcb::launch_bwd_dq<128>(q, k, v, dout, bp, B * H, s, &why)
+                   : pia::tcb::launch_bwd_dq<64>(q, k, v, dout, bp, B * H, s, &why);
+    }
+    if (e == cudaSuccess) {
+      e = launch_bwd<bf>(q, k, v, w_g, b_g, dout, dq, dk, dv, rs, gt, H, n, d, k_win, pi, S, scale_log2, bd, s, false);
+      why = "dk/dv kernel launch";
+    }
+    if (e == cudaSuccess)
+      pia::bwd_gate_partial_kernel<bf><<<gg, 256, 0, s>>>((const bf*)q, rs.dz, part_w, part_b, B, H, n, d);
+  } else if (dtype == PI_ATTN_F32) {
     e = launch_bwd<float>(q, k, v, w_g, b_g, dout, dq, dk, dv, rs, gt, H, n, d, k_win, pi, S, scale_log2, bd, s);
     if (e == cudaSuccess)
       pia::bwd_gate_partial_kernel<float><<<gg, 256, 0, s>>>((const float*)q, rs.dz, part_w, part_b, B, H, n, d);
   } else {
-    using bf = __nv_bfloat16;
     e = launch_bwd<bf>(q, k, v, w_g, b_g, dout, dq, dk, dv, rs, gt, H, n, d, k_win, pi, S, scale_log2, bd, s);
     if (e == cudaSuccess)
       pia::bwd_gate_partial_kernel<bf><<<gg, 256, 0, s>>>((const bf*)q, rs.dz, part_w, part_b, B, H, n, d);
   }
   if (e == cudaSuccess) pia::bwd_gate_final_kernel<<<H, 256, 0, s>>>(part_w, part_b, dw_g, db_g, (int)nchunks, d);
-  e = cudaGetLastError();
+  if (e == cudaSuccess) e = cudaGetLastError();
   cudaError_t e2 = workspace ? cudaSuccess : cudaFreeAsync(scratch, s);
-  if (e != cudaSuccess) return cuda_fail(e, "backward kernel launch");
+  if (e != cudaSuccess) return cuda_fail(e, why);
   if (e2 != cudaSuccess) return cuda_fail(e2, "backward scratch release");
   return ok();
+}
+
+pi_attn_status pi_attn_bwd(const void* q, const void* k, const void* v, const float* w_g, const float* b_g,
+                           const void* dout, float* dq, float* dk, float* dv, float* dw_g, float* db_g, int B, int H,
+                           int n, int d, int k_win, int pi, int S, pi_attn_dtype dtype, int bidir, void* workspace,
+                           long long workspace_bytes, void* stream) {
+  return pi_attn_bwd_ex(q, k, v, w_g, b_g, dout, dq, dk, dv, dw_g, db_g, B, H, n, d, k_win, pi, S, dtype, bidir,
+                        PI_ATTN_BWD_SIMT, workspace, workspace_bytes, stream);
 }
 
 pi_attn_status pi_attn_check(void* stream) {

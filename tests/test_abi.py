@@ -152,6 +152,23 @@ def test_shard_arguments_are_checked_before_any_launch(lib):
     assert call(100, 180, 200, 120, d=32) == pia.PI_ATTN_EUNSUPPORTED
 
 
+def test_tensor_core_backward_arguments_are_checked_before_any_launch(lib):
+    args = [FAKE] * 11
+    # fp32 and d = 32 are not covered by the tensor-core path; an unknown path is refused
+    assert lib.pi_attn_bwd_ex(*args, 1, 2, 64, 64, 8, 16, 2, pia.PI_ATTN_F32, 0, 2, None, 0, None) == \
+        pia.PI_ATTN_EUNSUPPORTED
+    assert lib.pi_attn_bwd_ex(*args, 1, 2, 64, 32, 8, 16, 2, pia.PI_ATTN_BF16, 0, 2, None, 0, None) == \
+        pia.PI_ATTN_EUNSUPPORTED
+    assert lib.pi_attn_bwd_ex(*args, 1, 2, 64, 64, 8, 16, 2, pia.PI_ATTN_BF16, 0, 7, None, 0, None) == \
+        pia.PI_ATTN_EINVAL
+    # a workspace smaller than the path needs
+    tc = lib.pi_attn_bwd_workspace_bytes_ex(1, 2, 64, 64, pia.PI_ATTN_BF16, 2)
+    simt = lib.pi_attn_bwd_workspace_bytes_ex(1, 2, 64, 64, pia.PI_ATTN_BF16, 1)
+    assert simt == lib.pi_attn_bwd_workspace_bytes(1, 2, 64, 64) and tc >= simt + 1 * 2 * 64 * (2 * 64 + 4)
+    assert lib.pi_attn_bwd_ex(*args, 1, 2, 64, 64, 8, 16, 2, pia.PI_ATTN_BF16, 0, 2, FAKE, tc - 16, None) == \
+        pia.PI_ATTN_EINVAL
+
+
 def test_built_for_sm100a_only():
     cmd = pbuild.command("x.so")
     assert "arch=compute_100a,code=sm_100a" in cmd and "-lineinfo" in cmd
