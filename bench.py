@@ -100,7 +100,7 @@ def load_peaks():
 
 KERNEL_FILES = {  # sources of each timed kernel (for matching committed ncu counters to the code)
     "prefill": ["fwd_tc.cuh", "tile_rule.cuh", "common.cuh"],
-    "backward": ["bwd_simt.cuh", "tile_rule.cuh", "common.cuh"],
+    "backward": ["fwd_tc.cuh", "bwd_tc.cuh", "bwd_simt.cuh", "tile_rule.cuh", "common.cuh"],
     "decode": ["decode.cuh", "common.cuh"],
 }
 
@@ -368,12 +368,18 @@ def run_gpu(args):
                  torch.empty(t["q"].shape, dtype=torch.float32, device=device),
                  torch.empty((w.H, w.d), dtype=torch.float32, device=device),
                  torch.empty((w.H,), dtype=torch.float32, device=device))
-        ws = torch.empty(pia.load().pi_attn_bwd_workspace_bytes(w.B, w.H, w.n, w.d), dtype=torch.uint8, device=device)
+        bwd_tc = args.bwd_path == "tc" or (args.bwd_path == "auto" and w.dtype == "bf16" and w.d in (64, 128))
+        bwd_path = "tc" if bwd_tc else "simt"
+        ws = torch.empty(pia.load().pi_attn_bwd_workspace_bytes_ex(w.B, w.H, w.n, w.d, pia._dtype_code(t["q"]),
+                                                                    pia.BWD_PATHS[bwd_path]),
+                         dtype=torch.uint8, device=device)
 
         def step():
             pia.pi_attn_bwd(t["q"], t["k"], t["v"], t["w_g"], t["b_g"], t["dO"], w.k, w.pi, w.S, bidir=w.bidir,
-                            grads=grads, workspace=ws)
-        launches_per_step = 4  # row pass, key pass, two gate reduction stages
+                            grads=grads, workspace=ws, path=bwd_path)
+        # tc: forward (single pass, with D), dq pass, dk/dv pass, two gate reduction stages;
+        # simt: row pass, dk/dv pass, two gate reduction stages
+        launches_per_step = 5 if bwd_tc else 4
     else:
         def step():
             pia.pi_attn_decode(t["q"], t["k"], t["v"], t["w_g"], t["b_g"], w.k, w.pi, w.S, out=out, lse=lse)
@@ -510,7 +516,8 @@ def run_gpu(args):
                        parallelism=f"replicas x{world} (independent (b, h) batches)"),
         "achieved_tflops": flops / launch_s / 1e12, "achieved_gbs": bytes_ / launch_s / 1e9,
         "roofline": roof, "cpu_baseline": cpu, "e2e": e2e,
-        "gpu_launches": launches_per_step * args.steps, "clocks": clocks.summary(), "path": args.path,
+        "gpu_launches": launches_per_step * args.steps, "clocks": clocks.summary(),
+        "path": bwd_path if w.kind == "backward" else args.path,
         "timing": "CUDA graph replay of one public call per step" if graph is not None else "eager public call",
         "eager_ms_per_step": eager_ms,
         "kernel_source_sha": source_hash(KERNEL_FILES[w.kind]),
@@ -563,6 +570,8 @@ def main(argv=None):
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--path", default="auto", choices=["auto", "simt", "tc", "tc_fused", "tc_split"],
                     help="prefill kernel choice (pi_attn_fwd_ex path)")
+    ap.add_argument("--bwd-path", default="auto", choices=["auto", "simt", "tc"],
+                    help="backward kernels: the tensor-core dq pass (tc), fp32 CUDA cores (simt), or tc where it applies")
     ap.add_argument("--cpu-budget", type=float, default=10.0, help="seconds of oracle work for cpu_baseline")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--eager", action="store_true", help="time the plain call instead of a graph replay")

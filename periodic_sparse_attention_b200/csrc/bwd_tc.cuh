@@ -373,6 +373,356 @@ __global__ void __launch_bounds__(192, BSmem<D>::kCtas) bwd_dq_kernel(const __gr
   }
 }
 
+// ---- the dk/dv pass: the forward's roles swapped ---------------------------------------------
+// One CTA per (block of 128 keys, b, h), walking the 64-row tiles that read its keys
+// (ReaderWalk).  Per row tile:
+//   MMA warp            S^T = K Q^T and dP^T = V dO^T (128 keys x 64 rows, fp32 in TMEM), then,
+//                       once the softmax warps have written P^T and dS^T, dV += P^T dO and
+//                       dK += dS^T Q (fp32 in TMEM; P^T, dS^T from TMEM, dO and Q N-major)
+//   softmax warpgroup   one thread per key: for each row that reads the key (its window rows, a
+//                       range, and its skip rows, KeyReaders) p = 2^(s tau log2e + prior - lse2)
+//                       and ds = p (dp - D) from the row's terms (staged in shared memory), P^T
+//                       and dS^T in bf16 over the S^T and dP^T columns already read
+//   TMA producer warp   K and V tiles once, then Q and dO row tiles into a 2-stage ring
+// The epilogue writes dk = tau dK, dv = dV (fp32).  TMEM: S^T 0..63, dP^T 64..127, dV and dK
+// after them (256 columns for D = 64, 512 for D = 128).
+template <int D>
+struct KSmem {
+  static constexpr int kCtas = D == 64 ? 2 : 1;
+  static constexpr int kKeyBytes = BM * D * 2;           // the K tile, the V tile (128 keys)
+  static constexpr int kRowBytes = BN * D * 2;           // one Q or dO row tile (64 rows)
+  static constexpr int kK = 0;
+  static constexpr int kV = kK + kKeyBytes;
+  static constexpr int kQ = kV + kKeyBytes;
+  static constexpr int kG = kQ + NSTAGE * kRowBytes;
+  static constexpr int kStat = kG + NSTAGE * kRowBytes;  // 2 buffers x 64 rows x (lse2, D, bl2, bp2)
+  static constexpr int kBar = kStat + 2 * BN * 16;
+  // barriers: kv_full, q_full[NSTAGE], q_empty[NSTAGE], g_full[NSTAGE], g_empty[NSTAGE], s_full,
+  // p_full, kv_done, drain
+  static constexpr int kNumBars = 1 + 4 * NSTAGE + 4;
+  static constexpr int kMisc = kBar + kNumBars * 8;
+  static constexpr int kTotal = kMisc + 8;
+  static constexpr int kAlloc = kTotal + 1024 - 128;
+  static constexpr int kTmemCols = D == 64 ? 256 : 512;
+  static_assert(2 * BN + 2 * D <= kTmemCols && kTmemCols * kCtas <= 512, "TMEM columns");
+  static_assert(kK % 1024 == 0 && kV % 1024 == 0 && kQ % 1024 == 0 && kG % 1024 == 0 && kRowBytes % 1024 == 0,
+                "128-byte-swizzled tiles sit on 1 KB");
+  static_assert(kStat % 16 == 0 && kBar % 8 == 0, "row terms on 16 bytes, mbarriers on 8");
+  static_assert(kAlloc <= 228 * 1024 / kCtas - 1024, "shared memory of the CTAs on one SM");
+};
+
+struct KParams {
+  const float* lse2;  // [B*H, n] the rows' terms from the dq pass
+  const float* Dr;
+  const float* bl2;
+  const float* bp2;
+  float* dk;          // [B*H, n, D]
+  float* dv;
+  int n, kwin, pi, S;
+  float scale_log2;
+  int bidir;
+};
+
+template <int D>
+__global__ void __launch_bounds__(192, KSmem<D>::kCtas) bwd_dkv_kernel(const __grid_constant__ CUtensorMap tmk,
+                                                                        const __grid_constant__ CUtensorMap tmv,
+                                                                        const __grid_constant__ CUtensorMap tmq,
+                                                                        const __grid_constant__ CUtensorMap tmg,
+                                                                        KParams prm) {
+  using namespace tc;
+  using L = KSmem<D>;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  uint8_t* const sbase = smem_raw + (base - raw);
+  if (base - raw + L::kTotal > (uint32_t)L::kAlloc) {
+    if (threadIdx.x == 0) raise_error(kErrInternal);
+    return;
+  }
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int bh = blockIdx.y;
+  const long long j0 = (long long)blockIdx.x * BM;  // this CTA's keys j0 .. j0 + 127
+  const uint32_t sK = base + L::kK, sV = base + L::kV, sQ = base + L::kQ, sG = base + L::kG;
+  const uint32_t bar0 = base + L::kBar;
+  const uint32_t bar_kv = bar0;
+  auto bar_qfull = [&](int s) { return bar0 + 8u * (1 + s); };
+  auto bar_qempty = [&](int s) { return bar0 + 8u * (1 + NSTAGE + s); };
+  auto bar_gfull = [&](int s) { return bar0 + 8u * (1 + 2 * NSTAGE + s); };
+  auto bar_gempty = [&](int s) { return bar0 + 8u * (1 + 3 * NSTAGE + s); };
+  const uint32_t bar_sfull = bar0 + 8u * (1 + 4 * NSTAGE);
+  const uint32_t bar_pfull = bar_sfull + 8;
+  const uint32_t bar_kvdone = bar_sfull + 16;
+  const uint32_t bar_drain = bar_sfull + 24;
+  uint32_t* const tmem_slot = reinterpret_cast<uint32_t*>(sbase + L::kMisc);
+  volatile int* const abort_flag = reinterpret_cast<volatile int*>(sbase + L::kMisc + 4);
+
+  if (threadIdx.x == 0) {
+    asm volatile("prefetch.tensormap [%0];" ::"l"(&tmk) : "memory");
+    asm volatile("prefetch.tensormap [%0];" ::"l"(&tmv) : "memory");
+    asm volatile("prefetch.tensormap [%0];" ::"l"(&tmq) : "memory");
+    asm volatile("prefetch.tensormap [%0];" ::"l"(&tmg) : "memory");
+    mbar_init(bar_kv, 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    mbar_expect_tx(bar_kv, 2 * L::kKeyBytes);
+#pragma unroll
+    for (int c = 0; c < D / 64; ++c) {
+      tma_load_3d(sK + c * BM * 128, &tmk, bar_kv, c * 64, (int)j0, bh);
+      tma_load_3d(sV + c * BM * 128, &tmv, bar_kv, c * 64, (int)j0, bh);
+    }
+  }
+  const int m0 = first_skip_m(prm.kwin, prm.pi);
+  ReaderWalk walk;
+  walk.init(j0, prm.n, BM, prm.kwin, prm.pi, prm.S, prm.bidir != 0);
+  int t_first = -1;
+  auto load_rows = [&](uint32_t dst, const CUtensorMap* map, uint32_t bar, long long r0) {
+#pragma unroll
+    for (int c = 0; c < D / 64; ++c) tma_load_3d(dst + c * BN * 128, map, bar, c * 64, (int)r0, bh);
+  };
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < NSTAGE; ++s) {
+      mbar_init(bar_qfull(s), 1);
+      mbar_init(bar_qempty(s), 1);
+      mbar_init(bar_gfull(s), 1);
+      mbar_init(bar_gempty(s), 1);
+    }
+    mbar_init(bar_sfull, 1);
+    mbar_init(bar_pfull, BM);
+    mbar_init(bar_kvdone, 1);
+    mbar_init(bar_drain, 1);
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    t_first = walk.next(0);
+    if (t_first >= 0) {
+      mbar_expect_tx(bar_qfull(0), L::kRowBytes);
+      load_rows(sQ, &tmq, bar_qfull(0), (long long)t_first * BN);
+      mbar_expect_tx(bar_gfull(0), L::kRowBytes);
+      load_rows(sG, &tmg, bar_gfull(0), (long long)t_first * BN);
+    }
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
+                 "n"(L::kTmemCols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t tS = tmem, tP = tmem + BN, tdV = tmem + 2 * BN, tdK = tmem + 2 * BN + D;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      constexpr uint32_t kRow = L::kRowBytes;
+      int nq = t_first >= 0 ? 1 : 0, ng = nq;
+      for (int t = t_first >= 0 ? walk.next(t_first + 1) : -1; t >= 0; t = walk.next(t + 1)) {
+        const int s = nq % NSTAGE, use = nq / NSTAGE;
+        if (use > 0 && !mbar_wait(bar_qempty(s), (use - 1) & 1, abort_flag)) break;
+        mbar_expect_tx(bar_qfull(s), kRow);
+        load_rows(sQ + s * kRow, &tmq, bar_qfull(s), (long long)t * BN);
+        ++nq;
+        if (use > 0 && !mbar_wait(bar_gempty(s), (use - 1) & 1, abort_flag)) break;
+        mbar_expect_tx(bar_gfull(s), kRow);
+        load_rows(sG + s * kRow, &tmg, bar_gfull(s), (long long)t * BN);
+        ++ng;
+      }
+      if (*abort_flag) {
+        volatile int never = 0;
+        mbar_wait(bar_kv, 0, &never);
+        for (int u = nq > NSTAGE ? nq - NSTAGE : 0; u < nq; ++u)
+          mbar_wait(bar_qfull(u % NSTAGE), (u / NSTAGE) & 1, &never);
+        for (int u = ng > NSTAGE ? ng - NSTAGE : 0; u < ng; ++u)
+          mbar_wait(bar_gfull(u % NSTAGE), (u / NSTAGE) & 1, &never);
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ------------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t kRow = L::kRowBytes;
+      constexpr uint32_t idesc_s = idesc_bf16(BM, BN, 0);  // S^T, dP^T: B (Q, dO) K-major
+      constexpr uint32_t idesc_a = idesc_bf16(BM, D, 1);   // dV, dK: B (dO, Q) N-major
+      bool okw = mbar_wait(bar_kv, 0, abort_flag);
+      tc_fence_after();
+      int jt = 0;
+      for (int t = walk.next(0); okw && t >= 0; t = walk.next(t + 1), ++jt) {
+        const int s = jt % NSTAGE;
+        if (!mbar_wait(bar_qfull(s), (jt / NSTAGE) & 1, abort_flag)) break;
+        if (!mbar_wait(bar_gfull(s), (jt / NSTAGE) & 1, abort_flag)) break;
+        // the dV, dK MMAs of the previous tile read P^T, dS^T over the columns overwritten here
+        if (jt > 0 && !mbar_wait(bar_kvdone, (jt - 1) & 1, abort_flag)) break;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t in = (kk & 3) * 32;
+          tc_mma(tS, sw128_desc(sK + (kk >> 2) * (BM * 128) + in, 16, 1024),
+                 sw128_desc(sQ + s * kRow + (kk >> 2) * (BN * 128) + in, 16, 1024), idesc_s, kk > 0 ? 1u : 0u);
+        }
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t in = (kk & 3) * 32;
+          tc_mma(tP, sw128_desc(sV + (kk >> 2) * (BM * 128) + in, 16, 1024),
+                 sw128_desc(sG + s * kRow + (kk >> 2) * (BN * 128) + in, 16, 1024), idesc_s, kk > 0 ? 1u : 0u);
+        }
+        tc_commit(bar_sfull);
+        if (!mbar_wait(bar_pfull, jt & 1, abort_flag)) break;
+        tc_fence_after();
+        // dV += P^T dO and dK += dS^T Q : K = BN rows, 16 per instruction
+#pragma unroll
+        for (int kk = 0; kk < BN / 16; ++kk) {
+          const uint32_t acol = 16 * (kk >> 1) + 8 * (kk & 1);
+          const uint32_t acc = (jt == 0 && kk == 0) ? 0u : 1u;
+          tc_mma_ts(tdV, tS + acol, sw128_desc(sG + s * kRow + kk * 16 * 128, BN * 128, 1024), idesc_a, acc);
+          tc_mma_ts(tdK, tP + acol, sw128_desc(sQ + s * kRow + kk * 16 * 128, BN * 128, 1024), idesc_a, acc);
+        }
+        tc_commit(bar_kvdone);
+        tc_commit(bar_qempty(s));
+        tc_commit(bar_gempty(s));
+      }
+      tc_commit(bar_drain);
+      volatile int never = 0;
+      mbar_wait(bar_drain, 0, &never);
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------------ key warpgroup
+    const int q4 = warp & 3;
+    const int r = q4 * 32 + lane;
+    const long long j = j0 + r;
+    const bool key_ok = j < prm.n;
+    const long long krow = (long long)bh * prm.n + (key_ok ? j : 0);
+    const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
+    const long long w_lo = prm.bidir ? (j - prm.kwin > 0 ? j - prm.kwin : 0) : j;  // rows reading j as window key
+    const long long w_hi = j + prm.kwin < prm.n - 1 ? j + prm.kwin : prm.n - 1;
+    KeyReaders kr;
+    kr.init(j, prm.pi, prm.S, m0, walk.rpi, prm.bidir != 0, prm.n);
+    const float NEG_INF = -INFINITY;
+    const int tid = threadIdx.x - 64;  // 0..127
+    float4* const stat = reinterpret_cast<float4*>(sbase + L::kStat);
+    const long long rbase = (long long)bh * prm.n;
+    bool ok = true;
+    int jt = 0;
+    for (int t = walk.next(0); t >= 0; t = walk.next(t + 1), ++jt) {
+      const long long r0 = (long long)t * BN;
+      // the tile's row terms into this tile's buffer (the other buffer may still be read by a warp
+      // on the previous tile; a warp here has finished that one)
+      float4* const st = stat + (jt & 1) * BN;
+      if (tid < BN) {
+        const long long i = r0 + tid;
+        st[tid] = i < prm.n ? make_float4(prm.lse2[rbase + i], prm.Dr[rbase + i], prm.bl2[rbase + i], prm.bp2[rbase + i])
+                            : make_float4(0.f, 0.f, NEG_INF, NEG_INF);
+      }
+      asm volatile("bar.sync 1, 128;" ::: "memory");
+      if (!ok) continue;  // keep taking part in the barrier above while the other warps finish
+      if (!__all_sync(0xffffffffu, mbar_wait(bar_sfull, jt & 1, abort_flag))) {
+        ok = false;
+        continue;
+      }
+      tc_fence_after();
+      const long long lo64 = w_lo - r0, hi64 = w_hi - r0;
+      const int lc_lo = lo64 < 0 ? 0 : (lo64 > BN ? BN : (int)lo64);
+      const int lc_hi = hi64 > BN - 1 ? BN - 1 : (hi64 < -1 ? -1 : (int)hi64);
+      const uint64_t skw = kr.take(r0);
+      // 16 rows at a time (registers): P^T and dS^T of rows c0 .. c0 + 15 go to the 8 packed
+      // columns c0 / 2 .., which this loop has already read
+      const uint64_t wm64 = key_ok ? (uint64_t)window_bits(lc_lo, lc_hi) | ((uint64_t)window_bits(lc_lo - 32, lc_hi - 32) << 32)
+                                   : 0ull;
+      const uint64_t sk64 = key_ok ? skw : 0ull;
+#pragma unroll 1
+      for (int cb = 0; cb < BN / 16; ++cb) {
+        const int c0 = cb * 16;
+        float x[16], g[16];
+        tmem_ld16(tS + lane_off + c0, x);
+        tmem_ld16(tP + lane_off + c0, g);
+        const uint32_t wm = (uint32_t)(wm64 >> c0) & 0xFFFFu;
+        const uint32_t skb = (uint32_t)(sk64 >> c0) & 0xFFFFu;
+        uint32_t pk[8], dk2[8];
+        if (__all_sync(0xffffffffu, (wm | skb) == 0u)) {
+#pragma unroll
+          for (int w = 0; w < 8; ++w) pk[w] = dk2[w] = 0u;
+        } else {
+#pragma unroll
+          for (int e = 0; e < 16; e += 2) {
+            const float4 ra = st[c0 + e], rb = st[c0 + e + 1];
+            const float b0 = ((wm >> e) & 1u) ? ra.z : (((skb >> e) & 1u) ? ra.w : NEG_INF);
+            const float b1 = ((wm >> (e + 1)) & 1u) ? rb.z : (((skb >> (e + 1)) & 1u) ? rb.w : NEG_INF);
+            const float p0 = ex2(fmaf(x[e], prm.scale_log2, b0 - ra.x));
+            const float p1 = ex2(fmaf(x[e + 1], prm.scale_log2, b1 - rb.x));
+            const float d0 = p0 * (g[e] - ra.y), d1 = p1 * (g[e + 1] - rb.y);
+            __nv_bfloat162 pb = __floats2bfloat162_rn(p0, p1), db = __floats2bfloat162_rn(d0, d1);
+            pk[e >> 1] = *reinterpret_cast<uint32_t*>(&pb);
+            dk2[e >> 1] = *reinterpret_cast<uint32_t*>(&db);
+          }
+        }
+        __syncwarp();
+        tmem_st8(tS + lane_off + 8 * cb, pk);   // P^T over S^T columns already read
+        tmem_st8(tP + lane_off + 8 * cb, dk2);  // dS^T over dP^T columns already read
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(bar_pfull);
+    }
+    // ---- epilogue: dk = tau dK, dv = dV
+    const bool have = __all_sync(0xffffffffu, ok && jt > 0 && mbar_wait(bar_kvdone, (jt - 1) & 1, abort_flag));
+    if (have) tc_fence_after();
+    const float tau = prm.scale_log2 / kLog2e;
+    if (have || jt == 0) {
+#pragma unroll 1
+      for (int c = 0; c < D / 32; ++c) {
+        float a[32], b[32];
+        if (have) {
+          tmem_ld32(tdK + lane_off + c * 32, a);
+          tmem_ld32(tdV + lane_off + c * 32, b);
+        } else {
+#pragma unroll
+          for (int e = 0; e < 32; ++e) a[e] = b[e] = 0.f;
+        }
+        if (key_ok) {
+          float4* dkp = reinterpret_cast<float4*>(prm.dk + krow * D + c * 32);
+          float4* dvp = reinterpret_cast<float4*>(prm.dv + krow * D + c * 32);
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            dkp[e] = make_float4(tau * a[4 * e], tau * a[4 * e + 1], tau * a[4 * e + 2], tau * a[4 * e + 3]);
+            dvp[e] = make_float4(b[4 * e], b[4 * e + 1], b[4 * e + 2], b[4 * e + 3]);
+          }
+        }
+      }
+    }
+    tc_fence_before();
+  }
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) {
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "n"(L::kTmemCols) : "memory");
+  }
+}
+
+template <int D>
+cudaError_t launch_bwd_dkv(const void* q, const void* k, const void* v, const void* dout, const KParams& p, int BH,
+                           cudaStream_t st, const char** why) {
+  CUtensorMap mk, mv, mq, mg;
+  if (!tc::make_map(&mk, k, BH, p.n, D, BM) || !tc::make_map(&mv, v, BH, p.n, D, BM) ||
+      !tc::make_map(&mq, q, BH, p.n, D, BN) || !tc::make_map(&mg, dout, BH, p.n, D, BN)) {
+    *why = "cuTensorMapEncodeTiled failed";
+    return cudaErrorInvalidValue;
+  }
+  static bool attr_done = false;
+  if (!attr_done) {
+    cudaError_t e = cudaFuncSetAttribute(bwd_dkv_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         KSmem<D>::kAlloc);
+    if (e != cudaSuccess) {
+      *why = "cudaFuncSetAttribute";
+      return e;
+    }
+    attr_done = true;
+  }
+  const dim3 grid((unsigned)((p.n + BM - 1) / BM), (unsigned)BH);
+  bwd_dkv_kernel<D><<<grid, 192, KSmem<D>::kAlloc, st>>>(mk, mv, mq, mg, p);
+  *why = "tensor-core dk/dv kernel launch";
+  return cudaGetLastError();
+}
+
 template <int D>
 cudaError_t set_bwd_smem_attr() {
   static bool done = false;

@@ -571,7 +571,7 @@ pi_attn_status pi_attn_bwd_ex(const void* q, const void* k, const void* v, const
   using bf = __nv_bfloat16;
   if (tc) {
     // the forward (single tensor-core pass) for out, lse and D = dO . out (from its fp32 output
-    // rows), then the dq pass on the tensor cores, then the dk/dv pass
+    // rows), then the dq pass and the dk/dv pass on the tensor cores
     const long long off = (bwd_ws_bytes(B, H, n, d, false) + 15) / 16 * 16;
     bf* out_ws = reinterpret_cast<bf*>(static_cast<char*>(scratch) + off);
     float* lse_ws = reinterpret_cast<float*>(static_cast<char*>(scratch) + off + rows * 2LL * d);
@@ -601,8 +601,21 @@ pi_attn_status pi_attn_bwd_ex(const void* q, const void* k, const void* v, const
                    : pia::tcb::launch_bwd_dq<64>(q, k, v, dout, bp, B * H, s, &why);
     }
     if (e == cudaSuccess) {
-      e = launch_bwd<bf>(q, k, v, w_g, b_g, dout, dq, dk, dv, rs, gt, H, n, d, k_win, pi, S, scale_log2, bd, s, false);
-      why = "dk/dv kernel launch";
+      pia::tcb::KParams kp;
+      kp.lse2 = rs.lse2;
+      kp.Dr = rs.D;
+      kp.bl2 = rs.bl2;
+      kp.bp2 = rs.bp2;
+      kp.dk = dk;
+      kp.dv = dv;
+      kp.n = n;
+      kp.kwin = k_win;
+      kp.pi = pi;
+      kp.S = S;
+      kp.scale_log2 = scale_log2;
+      kp.bidir = bd ? 1 : 0;
+      e = d == 128 ? pia::tcb::launch_bwd_dkv<128>(q, k, v, dout, kp, B * H, s, &why)
+                   : pia::tcb::launch_bwd_dkv<64>(q, k, v, dout, kp, B * H, s, &why);
     }
     if (e == cudaSuccess)
       pia::bwd_gate_partial_kernel<bf><<<gg, 256, 0, s>>>((const bf*)q, rs.dz, part_w, part_b, B, H, n, d);

@@ -215,6 +215,44 @@ struct RowSkips {
   }
 };
 
+// The mirror of RowSkips, for a key: the rows that read key j as a skip key, in ascending order,
+// taken row tile by row tile while a walk visits the row tiles in increasing order: the
+// bidirectional rule's rows j - m pi (m from its largest value down to m0), then the rows j + m pi
+// (m from m0 up, rows below n).  One division per key at init, none per tile.
+struct KeyReaders {
+  long long nb = 0, nf = 0, pi = 1;  // next row before / after the key
+  int lb = 0, lf = 0;                // rows left
+  PIA_HD void init(long long j, int pi_, int S, int m0, double rpi, bool bidir, long long n) {
+    pi = pi_;
+    lb = lf = 0;
+    nb = nf = 0;
+    if (bidir && S >= m0 && j >= 0) {
+      long long mb = div_floor(j, pi_, rpi);
+      if (mb > S) mb = S;
+      if (mb >= m0) {
+        lb = (int)(mb - m0 + 1);
+        nb = j - mb * pi_;
+      }
+    }
+    if (S >= m0 && j + (long long)m0 * pi_ <= n - 1) {
+      long long mf = div_floor(n - 1 - j, pi_, rpi);
+      if (mf > S) mf = S;
+      lf = (int)(mf - m0 + 1);
+      nf = j + (long long)m0 * pi_;
+    }
+  }
+  // bit c set for each row r0 + c in [r0, r0 + kTileKeys) that reads the key as a skip key
+  PIA_HD uint64_t take(long long r0) {
+    uint64_t bits = 0;
+    const long long re = r0 + kTileKeys;
+    for (; lb > 0 && nb < re; nb += pi, --lb)
+      if (nb >= r0) bits |= 1ull << (int)(nb - r0);
+    for (; lf > 0 && nf < re; nf += pi, --lf)
+      if (nf >= r0) bits |= 1ull << (int)(nf - r0);
+    return bits;
+  }
+};
+
 // The transposed walk, for the backward: in increasing order, the row tiles (kTileKeys rows each)
 // holding at least one row that reads a key of the key block [j0, jl].  Row i reads key j as a
 // window key when j in L(i) -- causal: i in [j, j + k]; bidirectional: |i - j| <= k -- and as a

@@ -117,3 +117,21 @@ def test_cursor_matches_walk_on_walks_built_by_field(harness):
         lastr = min(i0 + 127, n - 1)
         hi = min(lastr + k, n - 1) if bidir else lastr
         assert harness.cursor_vs_walk(i0, lastr, max(i0 - k, 0), hi, n, pi, S, k // pi + 1, bidir) == 0
+
+
+@pytest.mark.parametrize("bidir", [False, True])
+@pytest.mark.parametrize("n,k,pi,S", [(256, 8, 16, 2), (700, 100, 37, 12), (333, 400, 16, 40), (200, 64, 32, 0),
+                                      (300, 8, 1, 50), (513, 128, 64, 6), (130, 5, 7, 3), (640, 0, 128, 4),
+                                      (385, 127, 129, 2), (1000, 40, 16, 30)])
+def test_key_side_walk_gives_exactly_the_reading_rows(harness, n, k, pi, S, bidir):
+    # the dk/dv pass's view: key blocks of 128 keys, 64-row reading tiles, per key its window rows
+    # (a range) and its skip rows (KeyReaders), against the oracle's index sets transposed
+    harness.key_side_mismatches.argtypes = [ctypes.c_int] * 6 + [ctypes.c_void_p]
+    width = (2 * k + 1 + 2 * S) if bidir else (k + 1 + S)
+    c, idx = oracle.index_table(n, k, pi, S, width, bidir=bidir)
+    reads = np.zeros((n, n), np.int8)
+    for i in range(n):
+        nl, npk = c[i]
+        reads[i, idx[i, :nl]] = 1
+        reads[i, idx[i, nl:nl + npk]] = 2
+    assert harness.key_side_mismatches(n, k, pi, S, int(bidir), 128, reads.ctypes.data) == 0

@@ -4,6 +4,7 @@
 // that survive, in the oracle's index-table layout, plus consistency counters.
 #include <cstdint>
 #include <cstring>
+#include <vector>
 
 #include "../periodic_sparse_attention_b200/csrc/tile_rule.cuh"
 
@@ -137,5 +138,42 @@ extern "C" int cursor_vs_walk(long long i0, long long last, long long band_lo, l
   for (int t = w.next(0); t >= 0 && steps < 100000; t = w.next(t + 1), ++steps)
     if (c.next() != t) ++bad;
   if (c.next() != -1) ++bad;
+  return bad;
+}
+
+// The backward's key-side view: for key blocks of `keys` keys, walk the reading row tiles with
+// ReaderWalk and take each key's reading rows with its window range and KeyReaders; report for
+// every (row, key) pair that the rule connects whether the walk produced it as the right kind
+// (window or skip), and count pairs produced that the rule does not connect.  reads[i * n + j]:
+// 0 none, 1 window, 2 skip, as the oracle's index sets give them (filled by the caller).
+extern "C" int key_side_mismatches(int n, int kwin, int pi, int S, int bidir, int keys, const int8_t* reads) {
+  int bad = 0;
+  const int m0 = kwin / pi + 1;
+  for (long long j0 = 0; j0 < n; j0 += keys) {
+    ReaderWalk w;
+    w.init(j0, n, keys, kwin, pi, S, bidir != 0);
+    for (long long j = j0; j < j0 + keys && j < n; ++j) {
+      KeyReaders kr;
+      kr.init(j, pi, S, m0, w.rpi, bidir != 0, n);
+      const long long wlo = bidir ? (j - kwin > 0 ? j - kwin : 0) : j;
+      const long long whi = j + kwin < n - 1 ? j + kwin : n - 1;
+      std::vector<int8_t> seen(n, 0);
+      for (int t = w.next(0); t >= 0; t = w.next(t + 1)) {
+        const long long r0 = (long long)t * kTileKeys;
+        const uint64_t sk = kr.take(r0);
+        for (int c = 0; c < kTileKeys; ++c) {
+          const long long i = r0 + c;
+          if (i >= n) break;
+          const bool win = i >= wlo && i <= whi;
+          const bool skp = (sk >> c) & 1ull;
+          if (win && skp) ++bad;
+          if (win) seen[i] = 1;
+          if (skp) seen[i] = 2;
+        }
+      }
+      for (long long i = 0; i < n; ++i)
+        if (seen[i] != reads[i * n + j]) ++bad;
+    }
+  }
   return bad;
 }
