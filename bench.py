@@ -377,9 +377,9 @@ def run_gpu(args):
         def step():
             pia.pi_attn_bwd(t["q"], t["k"], t["v"], t["w_g"], t["b_g"], t["dO"], w.k, w.pi, w.S, bidir=w.bidir,
                             grads=grads, workspace=ws, path=bwd_path)
-        # tc: forward (single pass, with D), dq pass, dk/dv pass, two gate reduction stages;
-        # simt: row pass, dk/dv pass, two gate reduction stages
-        launches_per_step = 5 if bwd_tc else 4
+        # tc: forward (single pass, with D), dq pass (with the gate's partial sums), dk/dv pass, the
+        # gate's final sum; simt: row pass, dk/dv pass, two gate reduction stages
+        launches_per_step = 4
     else:
         def step():
             pia.pi_attn_decode(t["q"], t["k"], t["v"], t["w_g"], t["b_g"], w.k, w.pi, w.S, out=out, lse=lse)

@@ -191,10 +191,10 @@ pi_attn_status pi_attn_bwd(const void* q, const void* k, const void* v, const fl
 
 /* The backward with a choice of kernels.  PI_ATTN_BWD_SIMT is pi_attn_bwd: the forward recomputed
  * in fp32 on CUDA cores with every product in fp32.  PI_ATTN_BWD_TC runs the forward's single
- * tensor-core pass for out and lse, D_i = dout_i . out_i from that bf16 out, the dq pass on the
- * tensor cores (S and dP by tcgen05 in fp32, ds rounded to bf16 for dQ += dS K) and the dk/dv
- * pass on CUDA cores; its gradients carry the bf16 roundings of out, of P and of ds (relative
- * errors of order 2^-9), against fp32 arithmetic for the other path.  bf16 with d in {64, 128}
+ * tensor-core pass for lse and D_i = dout_i . out_i (from its fp32 output rows), then a dq pass
+ * and a dk/dv pass on the tensor cores (S, dP and their transposes by tcgen05 in fp32; P and ds
+ * rounded to bf16 for dQ += dS K, dV += P^T dO, dK += dS^T Q); its gradients carry those bf16
+ * roundings (relative errors of order 2^-9), against fp32 arithmetic for the other path.  bf16 with d in {64, 128}
  * (else PI_ATTN_EUNSUPPORTED).  PI_ATTN_BWD_AUTO: the tensor-core path where it applies, else
  * SIMT.  The workspace is pi_attn_bwd_workspace_bytes_ex(B, H, n, d, dtype, path) bytes (the
  * tensor-core path adds the forward's out and lse); other arguments and errors as pi_attn_bwd. */

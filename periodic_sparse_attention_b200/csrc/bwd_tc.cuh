@@ -42,7 +42,9 @@ struct BSmem {
   static constexpr int kNumBars = 1 + 4 * NSTAGE + 4;
   static constexpr int kMisc = kBar + kNumBars * 8;      // tmem base (4 B), abort flag (4 B)
   static constexpr int kWg = (kMisc + 8 + 15) / 16 * 16; // w_g[h], D floats
-  static constexpr int kTotal = kWg + D * 4;
+  static constexpr int kDz = kWg + D * 4;                // the rows' dz, then the gate partials (BM floats each)
+  static constexpr int kRed = kDz + BM * 4;
+  static constexpr int kTotal = kRed + BM * 4;
   static constexpr int kAlloc = kTotal + 1024 - 128;
   static constexpr int kTmemCols = 256;
   static_assert(2 * BN + D <= kTmemCols && kTmemCols * kCtas <= 512, "TMEM columns");
@@ -62,6 +64,8 @@ struct BParams {
   float* bl2;         // [B*H, n] log2(alpha), log2(1 - alpha), dz: for the dk/dv pass and the gate
   float* bp2;
   float* dz;
+  float* part_w;      // [H, B * tiles, D] this CTA's sum of dz_i q_i over its rows, in chunk b * tiles + tile
+  float* part_b;      // [H, B * tiles]    and of dz_i
   int H, n, kwin, pi, S;
   float scale_log2;
   int bidir;
@@ -362,6 +366,40 @@ __global__ void __launch_bounds__(192, BSmem<D>::kCtas) bwd_dq_kernel(const __gr
         prm.bl2[orow] = bl2;
         prm.bp2[orow] = bp2;
         prm.dz[orow] = dz;
+      }
+    }
+    // The gate's partial sums over this CTA's rows, in a fixed order: dw_g[c] += sum_r dz_r q_rc
+    // and db_g += sum_r dz_r.  G = BM / D threads a column, each over BM / G rows of the Q tile
+    // (still in shared memory), then the G parts in order.
+    {
+      float* const dz_s = reinterpret_cast<float*>(sbase + L::kDz);
+      float* const red = reinterpret_cast<float*>(sbase + L::kRed);
+      dz_s[r] = (have_q || j == 0) && row_ok ? dz : 0.f;
+      asm volatile("bar.sync 1, 128;" ::: "memory");
+      constexpr int G = BM / D, RPT = BM / G;
+      const int c = r % D, g = r / D;
+      float acc = 0.f;
+#pragma unroll 4
+      for (int rr = g * RPT; rr < (g + 1) * RPT; ++rr) {
+        const int cc = c & 63;
+        const uint32_t off = (c >> 6) * (BM * 128) + rr * 128 + ((((cc >> 3) ^ (rr & 7))) << 4) + (cc & 7) * 2;
+        const float qv = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(sbase + L::kQ + off));
+        acc = fmaf(dz_s[rr], qv, acc);
+      }
+      red[r] = acc;
+      asm volatile("bar.sync 1, 128;" ::: "memory");
+      const long long chunk = (long long)(bh / prm.H) * gridDim.x + blockIdx.x;
+      const long long nchunks = (long long)(gridDim.y / prm.H) * gridDim.x;
+      if (r < D) {
+        float sw = 0.f;
+#pragma unroll
+        for (int gg = 0; gg < G; ++gg) sw += red[gg * D + r];
+        prm.part_w[((long long)h * nchunks + chunk) * D + r] = sw;
+      }
+      if (r == 0) {
+        float sb = 0.f;
+        for (int rr = 0; rr < BM; ++rr) sb += dz_s[rr];
+        prm.part_b[(long long)h * nchunks + chunk] = sb;
       }
     }
     tc_fence_before();

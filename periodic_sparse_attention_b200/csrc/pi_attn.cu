@@ -118,8 +118,7 @@ pi_attn_status launch_simt(const void* q, const void* k, const void* v, const fl
 template <typename T, int CPT>
 cudaError_t launch_bwd_cpt(const void* q, const void* k, const void* v, const float* w_g, const float* b_g,
                            const void* dout, float* dq, float* dk, float* dv, pia::BwdRowStats rs, dim3 grid, int H,
-                           int n, int d, int kwin, int pi, int S, float scale_log2, bool bidir, cudaStream_t s,
-                           bool row_pass) {
+                           int n, int d, int kwin, int pi, int S, float scale_log2, bool bidir, cudaStream_t s) {
   static bool attr_done = false;
   const size_t sr = pia::bwd_row_smem(d, sizeof(T)), sk = pia::bwd_key_smem(d, sizeof(T));
   if (!attr_done) {
@@ -131,13 +130,11 @@ cudaError_t launch_bwd_cpt(const void* q, const void* k, const void* v, const fl
     if (e != cudaSuccess) return e;
     attr_done = true;
   }
-  if (row_pass) {  // else the rows' terms (lse2, D, priors, dz) and dq come from the tensor-core dq pass
-    pia::bwd_row_kernel<T, CPT><<<grid, pia::kBwdThreads, sr, s>>>((const T*)q, (const T*)k, (const T*)v, w_g, b_g,
-                                                                   (const T*)dout, dq, rs, H, n, d, kwin, pi, S,
-                                                                   scale_log2, bidir);
-    cudaError_t e = cudaGetLastError();
-    if (e != cudaSuccess) return e;
-  }
+  pia::bwd_row_kernel<T, CPT><<<grid, pia::kBwdThreads, sr, s>>>((const T*)q, (const T*)k, (const T*)v, w_g, b_g,
+                                                                 (const T*)dout, dq, rs, H, n, d, kwin, pi, S,
+                                                                 scale_log2, bidir);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
   pia::bwd_key_kernel<T, CPT><<<grid, pia::kBwdThreads, sk, s>>>((const T*)q, (const T*)k, (const T*)v,
                                                                  (const T*)dout, rs, dk, dv, H, n, d, kwin, pi, S,
                                                                  scale_log2, bidir);
@@ -147,16 +144,14 @@ cudaError_t launch_bwd_cpt(const void* q, const void* k, const void* v, const fl
 template <typename T>
 cudaError_t launch_bwd(const void* q, const void* k, const void* v, const float* w_g, const float* b_g,
                        const void* dout, float* dq, float* dk, float* dv, pia::BwdRowStats rs, dim3 grid, int H, int n,
-                       int d, int kwin, int pi, int S, float scale_log2, bool bidir, cudaStream_t s,
-                       bool row_pass = true) {
+                       int d, int kwin, int pi, int S, float scale_log2, bool bidir, cudaStream_t s) {
   if (d <= 64)
-    return launch_bwd_cpt<T, 8>(q, k, v, w_g, b_g, dout, dq, dk, dv, rs, grid, H, n, d, kwin, pi, S, scale_log2, bidir, s,
-                                row_pass);
+    return launch_bwd_cpt<T, 8>(q, k, v, w_g, b_g, dout, dq, dk, dv, rs, grid, H, n, d, kwin, pi, S, scale_log2, bidir, s);
   if (d <= 128)
     return launch_bwd_cpt<T, 16>(q, k, v, w_g, b_g, dout, dq, dk, dv, rs, grid, H, n, d, kwin, pi, S, scale_log2, bidir,
-                                 s, row_pass);
+                                 s);
   return launch_bwd_cpt<T, 32>(q, k, v, w_g, b_g, dout, dq, dk, dv, rs, grid, H, n, d, kwin, pi, S, scale_log2, bidir,
-                               s, row_pass);
+                               s);
 }
 
 static long long gate_chunks(int B, int n) {
@@ -166,9 +161,13 @@ static long long gate_chunks(int B, int n) {
 // Backward scratch: lse2, D, two log2-priors and dz per query row, then the gate's per-chunk
 // partial sums (fp32); the tensor-core path adds, 16-byte aligned, the forward's out (bf16) and
 // lse (fp32) of every row.
+// The tensor-core dq pass writes one gate partial per (b, 128-row query tile).
+static long long tc_gate_chunks(int B, int n) { return (long long)B * ((n + pia::tc::BM - 1) / pia::tc::BM); }
+
 static long long bwd_ws_bytes(int B, int H, int n, int d, bool tc) {
   if (B < 1 || H < 1 || n < 1 || d < 1) return 0;
-  const long long base = 4LL * (5LL * B * H * n + (long long)H * gate_chunks(B, n) * (d + 1));
+  const long long chunks = tc ? tc_gate_chunks(B, n) : gate_chunks(B, n);
+  const long long base = 4LL * (5LL * B * H * n + (long long)H * chunks * (d + 1));
   if (!tc) return base;
   const long long rows = (long long)B * H * n;
   return (base + 15) / 16 * 16 + rows * 2LL * d + rows * 4LL;
@@ -552,7 +551,7 @@ pi_attn_status pi_attn_bwd_ex(const void* q, const void* k, const void* v, const
   }
   const long long tiles = ((long long)n + pia::kBwdRows - 1) / pia::kBwdRows;
   if (tiles > 0x7fffffffLL || (long long)B * H > 65535) return fail(PI_ATTN_EINVAL, "grid too large");
-  const long long nchunks = gate_chunks(B, n);
+  const long long nchunks = tc ? tc_gate_chunks(B, n) : gate_chunks(B, n);
   if (nchunks > 0x7fffffffLL || H > 65535) return fail(PI_ATTN_EINVAL, "too many rows per head for the gate sums");
   cudaStream_t s = as_stream(stream);
   void* scratch = workspace;
@@ -572,7 +571,7 @@ pi_attn_status pi_attn_bwd_ex(const void* q, const void* k, const void* v, const
   if (tc) {
     // the forward (single tensor-core pass) for out, lse and D = dO . out (from its fp32 output
     // rows), then the dq pass and the dk/dv pass on the tensor cores
-    const long long off = (bwd_ws_bytes(B, H, n, d, false) + 15) / 16 * 16;
+    const long long off = (bwd_ws_bytes(B, H, n, d, true) - rows * 2LL * d - rows * 4LL);
     bf* out_ws = reinterpret_cast<bf*>(static_cast<char*>(scratch) + off);
     float* lse_ws = reinterpret_cast<float*>(static_cast<char*>(scratch) + off + rows * 2LL * d);
     e = d == 128 ? pia::launch_fwd_tc_with_dot<128>(q, k, v, w_g, b_g, dout, out_ws, lse_ws, rs.D, B, H, n, k_win,
@@ -590,6 +589,8 @@ pi_attn_status pi_attn_bwd_ex(const void* q, const void* k, const void* v, const
       bp.bl2 = rs.bl2;
       bp.bp2 = rs.bp2;
       bp.dz = rs.dz;
+      bp.part_w = part_w;
+      bp.part_b = part_b;
       bp.H = H;
       bp.n = n;
       bp.kwin = k_win;
@@ -617,8 +618,7 @@ pi_attn_status pi_attn_bwd_ex(const void* q, const void* k, const void* v, const
       e = d == 128 ? pia::tcb::launch_bwd_dkv<128>(q, k, v, dout, kp, B * H, s, &why)
                    : pia::tcb::launch_bwd_dkv<64>(q, k, v, dout, kp, B * H, s, &why);
     }
-    if (e == cudaSuccess)
-      pia::bwd_gate_partial_kernel<bf><<<gg, 256, 0, s>>>((const bf*)q, rs.dz, part_w, part_b, B, H, n, d);
+    // (the gate's partial sums come from the dq pass, one per (b, query tile))
   } else if (dtype == PI_ATTN_F32) {
     e = launch_bwd<float>(q, k, v, w_g, b_g, dout, dq, dk, dv, rs, gt, H, n, d, k_win, pi, S, scale_log2, bd, s);
     if (e == cudaSuccess)

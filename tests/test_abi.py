@@ -164,7 +164,9 @@ def test_tensor_core_backward_arguments_are_checked_before_any_launch(lib):
     # a workspace smaller than the path needs
     tc = lib.pi_attn_bwd_workspace_bytes_ex(1, 2, 64, 64, pia.PI_ATTN_BF16, 2)
     simt = lib.pi_attn_bwd_workspace_bytes_ex(1, 2, 64, 64, pia.PI_ATTN_BF16, 1)
-    assert simt == lib.pi_attn_bwd_workspace_bytes(1, 2, 64, 64) and tc >= simt + 1 * 2 * 64 * (2 * 64 + 4)
+    rows = 1 * 2 * 64
+    # the rows' five terms and the gate partials, then the forward's out (bf16) and lse
+    assert simt == lib.pi_attn_bwd_workspace_bytes(1, 2, 64, 64) and tc >= 4 * 5 * rows + rows * (2 * 64 + 4)
     assert lib.pi_attn_bwd_ex(*args, 1, 2, 64, 64, 8, 16, 2, pia.PI_ATTN_BF16, 0, 2, FAKE, tc - 16, None) == \
         pia.PI_ATTN_EINVAL
 
