@@ -368,8 +368,12 @@ def run_gpu(args):
                  torch.empty(t["q"].shape, dtype=torch.float32, device=device),
                  torch.empty((w.H, w.d), dtype=torch.float32, device=device),
                  torch.empty((w.H,), dtype=torch.float32, device=device))
-        bwd_tc = args.bwd_path == "tc" or (args.bwd_path == "auto" and w.dtype == "bf16" and w.d in (64, 128))
-        bwd_path = "tc" if bwd_tc else "simt"
+        bwd_path = args.bwd_path
+        if bwd_path == "auto":
+            bwd_path = "tc" if w.dtype == "bf16" and w.d in (64, 128) else "simt"
+        # the tensor-core backward splits exactly where the forward with the same path name does
+        bwd_split = bwd_path != "simt" and not w.bidir and \
+            pia.pi_attn_fwd_plan(w.B, w.H, w.n, w.d, w.k, w.pi, w.S, w.dtype, bwd_path)[0] == 2
         ws = torch.empty(pia.load().pi_attn_bwd_workspace_bytes_ex(w.B, w.H, w.n, w.d, pia._dtype_code(t["q"]),
                                                                     pia.BWD_PATHS[bwd_path]),
                          dtype=torch.uint8, device=device)
@@ -378,8 +382,9 @@ def run_gpu(args):
             pia.pi_attn_bwd(t["q"], t["k"], t["v"], t["w_g"], t["b_g"], t["dO"], w.k, w.pi, w.S, bidir=w.bidir,
                             grads=grads, workspace=ws, path=bwd_path)
         # tc: forward (single pass, with D), dq pass (with the gate's partial sums), dk/dv pass, the
-        # gate's final sum; simt: row pass, dk/dv pass, two gate reduction stages
-        launches_per_step = 4
+        # gate's final sum -- split: the forward, the dq and the dk/dv passes twice each; simt: row
+        # pass, dk/dv pass, two gate reduction stages
+        launches_per_step = 7 if bwd_split else 4
     else:
         def step():
             pia.pi_attn_decode(t["q"], t["k"], t["v"], t["w_g"], t["b_g"], w.k, w.pi, w.S, out=out, lse=lse)
@@ -570,8 +575,8 @@ def main(argv=None):
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--path", default="auto", choices=["auto", "simt", "tc", "tc_fused", "tc_split"],
                     help="prefill kernel choice (pi_attn_fwd_ex path)")
-    ap.add_argument("--bwd-path", default="auto", choices=["auto", "simt", "tc"],
-                    help="backward kernels: the tensor-core dq pass (tc), fp32 CUDA cores (simt), or tc where it applies")
+    ap.add_argument("--bwd-path", default="auto", choices=["auto", "simt", "tc", "tc_fused", "tc_split"],
+                    help="backward kernels: tensor cores (tc: fused or split by shape; tc_fused; tc_split), fp32 CUDA cores (simt), or tc where it applies")
     ap.add_argument("--cpu-budget", type=float, default=10.0, help="seconds of oracle work for cpu_baseline")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--eager", action="store_true", help="time the plain call instead of a graph replay")

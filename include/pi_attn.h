@@ -190,15 +190,30 @@ pi_attn_status pi_attn_bwd(const void* q, const void* k, const void* v, const fl
                            long long workspace_bytes, void* stream);
 
 /* The backward with a choice of kernels.  PI_ATTN_BWD_SIMT is pi_attn_bwd: the forward recomputed
- * in fp32 on CUDA cores with every product in fp32.  PI_ATTN_BWD_TC runs the forward's single
- * tensor-core pass for lse and D_i = dout_i . out_i (from its fp32 output rows), then a dq pass
- * and a dk/dv pass on the tensor cores (S, dP and their transposes by tcgen05 in fp32; P and ds
- * rounded to bf16 for dQ += dS K, dV += P^T dO, dK += dS^T Q); its gradients carry those bf16
- * roundings (relative errors of order 2^-9), against fp32 arithmetic for the other path.  bf16 with d in {64, 128}
- * (else PI_ATTN_EUNSUPPORTED).  PI_ATTN_BWD_AUTO: the tensor-core path where it applies, else
- * SIMT.  The workspace is pi_attn_bwd_workspace_bytes_ex(B, H, n, d, dtype, path) bytes (the
- * tensor-core path adds the forward's out and lse); other arguments and errors as pi_attn_bwd. */
-typedef enum { PI_ATTN_BWD_AUTO = 0, PI_ATTN_BWD_SIMT = 1, PI_ATTN_BWD_TC = 2 } pi_attn_bwd_path;
+ * in fp32 on CUDA cores with every product in fp32.  The tensor-core paths run the forward on the
+ * tensor cores for lse and D_i = dout_i . out_i (from its fp32 output rows), then a dq pass and a
+ * dk/dv pass on the tensor cores (S, dP and their transposes by tcgen05 in fp32; P and ds rounded
+ * to bf16 for dQ += dS K, dV += P^T dO, dK += dS^T Q); their gradients carry those bf16 roundings
+ * (relative errors of order 2^-9), against fp32 arithmetic for the SIMT path.  bf16 with d in
+ * {64, 128} (else PI_ATTN_EUNSUPPORTED).
+ *   PI_ATTN_BWD_TC_FUSED  each pass walks the window and the skips of a row (or key) in one sweep.
+ *   PI_ATTN_BWD_TC_SPLIT  the forward's split reading for long contexts: the forward, the dq pass
+ *                         and the dk/dv pass each run once over the skips alone in the residue-class
+ *                         view (the skip keys of a row form a dense band there) and once over the
+ *                         window alone; the skip passes use dq as scratch before writing it.  The
+ *                         causal rule with n % pi == 0 and a skip outside the window (as
+ *                         PI_ATTN_PATH_TC_SPLIT), else PI_ATTN_EUNSUPPORTED.
+ *   PI_ATTN_BWD_TC        tensor cores, fused or split chosen by shape as for PI_ATTN_PATH_TC.
+ *   PI_ATTN_BWD_AUTO      PI_ATTN_BWD_TC where the tensor cores apply, else SIMT.
+ * The workspace is pi_attn_bwd_workspace_bytes_ex(B, H, n, d, dtype, path) bytes (the tensor-core
+ * paths add the forward's out and lse); other arguments and errors as pi_attn_bwd. */
+typedef enum {
+    PI_ATTN_BWD_AUTO = 0,
+    PI_ATTN_BWD_SIMT = 1,
+    PI_ATTN_BWD_TC = 2,
+    PI_ATTN_BWD_TC_FUSED = 3,
+    PI_ATTN_BWD_TC_SPLIT = 4
+} pi_attn_bwd_path;
 long long pi_attn_bwd_workspace_bytes_ex(int B, int H, int n, int d, pi_attn_dtype dtype, pi_attn_bwd_path path);
 pi_attn_status pi_attn_bwd_ex(const void* q, const void* k, const void* v, const float* w_g, const float* b_g,
                               const void* dout, float* dq, float* dk, float* dv, float* dw_g, float* db_g, int B,

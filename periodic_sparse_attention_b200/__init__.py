@@ -230,7 +230,7 @@ def pi_attn_debug_index_sets(n: int, k_win: int, pi: int, S: int, width: int | N
     return counts, idx
 
 
-BWD_PATHS = {"auto": 0, "simt": 1, "tc": 2}
+BWD_PATHS = {"auto": 0, "simt": 1, "tc": 2, "tc_fused": 3, "tc_split": 4}
 
 
 def pi_attn_bwd(q, k, v, w_g, b_g, dout, k_win: int, pi: int, S: int, *, bidir: bool = False, grads=None,
@@ -238,8 +238,9 @@ def pi_attn_bwd(q, k, v, w_g, b_g, dout, k_win: int, pi: int, S: int, *, bidir: 
     """Gradients of a loss through out: (dq, dk, dv, dw_g, db_g), fp32 tensors.  q, k, v, dout
     [B, H, n, d] in one dtype (fp32 or bf16); w_g [H, d], b_g [H] fp32.  grads: a tuple of the five
     output tensors to write into (allocated when None); workspace from torch's caching allocator
-    when None.  path: "simt" (pi_attn_bwd, fp32 throughout), "tc" (the dq pass on the tensor
-    cores, pi_attn_bwd_ex) or "auto"."""
+    when None.  path: "simt" (pi_attn_bwd, fp32 throughout), "tc_fused" or "tc_split" (the
+    tensor-core passes in one sweep, or split into a residue-class skip pass and a window pass),
+    "tc" (the tensor cores, fused or split by shape) or "auto" (pi_attn_bwd_ex)."""
     import torch
     B, H, n, d = q.shape
     dev = q.device

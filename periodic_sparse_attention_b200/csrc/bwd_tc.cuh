@@ -69,9 +69,15 @@ struct BParams {
   int H, n, kwin, pi, S;
   float scale_log2;
   int bidir;
+  int acc;            // add to the dq and dz that the residue pass wrote (the split backward)
 };
 
-template <int D>
+// RES = 0: the sequence view, the rule's window and skips (S = 0: the window alone).  RES = 1: the
+// skips alone, in the residue-class view of the forward's split path: the CTA's rows are rows
+// t*pi + res of the sequence, their skip keys the band t - S .. t - m0 of the same class (all with
+// the skip prior).  The residue pass runs first and writes its dq and dz; the window pass then
+// runs with acc set, adds to both, and takes the gate's partial sums over the whole dz.
+template <int D, int RES>
 __global__ void __launch_bounds__(192, BSmem<D>::kCtas) bwd_dq_kernel(const __grid_constant__ CUtensorMap tmq,
                                                                        const __grid_constant__ CUtensorMap tmg,
                                                                        const __grid_constant__ CUtensorMap tmk,
@@ -90,7 +96,9 @@ __global__ void __launch_bounds__(192, BSmem<D>::kCtas) bwd_dq_kernel(const __gr
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int bh = blockIdx.y;
   const int h = bh % prm.H;
-  const long long q0 = (long long)blockIdx.x * BM;
+  const int res = RES ? (int)(blockIdx.x % prm.pi) : 0;
+  const long long q0 = RES ? (long long)(blockIdx.x / prm.pi) * BM : (long long)blockIdx.x * BM;
+  const long long T = RES ? prm.n / prm.pi : prm.n;  // rows of the view
   const uint32_t sQ = base + L::kQ, sG = base + L::kG, sK = base + L::kK, sV = base + L::kV;
   const uint32_t bar0 = base + L::kBar;
   const uint32_t bar_qg = bar0;
@@ -116,19 +124,42 @@ __global__ void __launch_bounds__(192, BSmem<D>::kCtas) bwd_dq_kernel(const __gr
     mbar_expect_tx(bar_qg, 2 * L::kTileBytes);
 #pragma unroll
     for (int c = 0; c < D / 64; ++c) {
-      tma_load_3d(sQ + c * BM * 128, &tmq, bar_qg, c * 64, (int)q0, bh);
-      tma_load_3d(sG + c * BM * 128, &tmg, bar_qg, c * 64, (int)q0, bh);
+      if (RES) {
+        tma_load_4d(sQ + c * BM * 128, &tmq, bar_qg, c * 64, res, (int)q0, bh);
+        tma_load_4d(sG + c * BM * 128, &tmg, bar_qg, c * 64, res, (int)q0, bh);
+      } else {
+        tma_load_3d(sQ + c * BM * 128, &tmq, bar_qg, c * 64, (int)q0, bh);
+        tma_load_3d(sG + c * BM * 128, &tmg, bar_qg, c * 64, (int)q0, bh);
+      }
     }
   }
   const int m0 = first_skip_m(prm.kwin, prm.pi);
   TileWalk walk;
-  walk.init(q0, prm.n, BM, prm.kwin, prm.pi, prm.S, prm.bidir != 0);
+  if (RES) {  // keys of view row t: t - S .. t - m0
+    walk.i0 = q0;
+    walk.last = (q0 + BM - 1 < T - 1 ? q0 + BM - 1 : T - 1) - m0;
+    walk.band_lo = q0 - prm.S > 0 ? q0 - prm.S : 0;
+    walk.band_hi = walk.last;
+    walk.n = T;
+    walk.pi = 1;
+    walk.S = 0;
+    walk.m0 = 1;
+    walk.bidir = false;
+    walk.rpi = 1.0;
+  } else {
+    walk.init(q0, prm.n, BM, prm.kwin, prm.pi, prm.S, prm.bidir != 0);
+  }
   TileCursor cur;
   cur.init(walk);
   int t_first = -1;
   auto load_kv = [&](uint32_t dst, const CUtensorMap* map, uint32_t bar, long long r0) {
 #pragma unroll
-    for (int c = 0; c < D / 64; ++c) tma_load_3d(dst + c * BN * 128, map, bar, c * 64, (int)r0, bh);
+    for (int c = 0; c < D / 64; ++c) {
+      if (RES)
+        tma_load_4d(dst + c * BN * 128, map, bar, c * 64, res, (int)r0, bh);
+      else
+        tma_load_3d(dst + c * BN * 128, map, bar, c * 64, (int)r0, bh);
+    }
   };
   if (threadIdx.x == 0) {
     for (int s = 0; s < NSTAGE; ++s) {
@@ -240,16 +271,18 @@ __global__ void __launch_bounds__(192, BSmem<D>::kCtas) bwd_dq_kernel(const __gr
     // ------------------------------------------------------------------ softmax warpgroup
     const int q4 = warp & 3;
     const int r = q4 * 32 + lane;
-    const long long i = q0 + r;
-    const bool row_ok = i < prm.n;
+    const long long qi = q0 + r;                       // row of the view
+    const long long i = RES ? qi * prm.pi + res : qi;  // row of the sequence
+    const bool row_ok = qi < T;
     const long long orow = (long long)bh * prm.n + (row_ok ? i : 0);
     const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
     const float lse2 = row_ok ? prm.lse[orow] * kLog2e : 0.f;
     const float Drow = row_ok ? prm.Dr[orow] : 0.f;
-    const long long w_lo = i - prm.kwin > 0 ? i - prm.kwin : 0;
-    const long long w_hi = prm.bidir ? (i + prm.kwin < prm.n - 1 ? i + prm.kwin : prm.n - 1) : i;
+    // RES: the band of view columns qi - S .. qi - m0 (every one a skip key)
+    const long long w_lo = RES ? (qi - prm.S > 0 ? qi - prm.S : 0) : (i - prm.kwin > 0 ? i - prm.kwin : 0);
+    const long long w_hi = RES ? qi - m0 : (prm.bidir ? (i + prm.kwin < prm.n - 1 ? i + prm.kwin : prm.n - 1) : i);
     RowSkips rs;
-    rs.init(i, prm.pi, prm.S, m0, walk.rpi, prm.bidir != 0, prm.n);
+    rs.init(i, prm.pi, RES ? 0 : prm.S, m0, walk.rpi, prm.bidir != 0, prm.n);
 
     float* const wg_s = reinterpret_cast<float*>(sbase + L::kWg);
     if (threadIdx.x - 64 < D) wg_s[threadIdx.x - 64] = prm.w_g[(long long)h * D + (threadIdx.x - 64)];
@@ -281,7 +314,7 @@ __global__ void __launch_bounds__(192, BSmem<D>::kCtas) bwd_dq_kernel(const __gr
     const float ls_a = log_sigmoid_fast(z), ls_b = log_sigmoid_fast(-z);
     const float alpha = __expf(ls_a);
     const float bl2 = ls_a * kLog2e, bp2 = ls_b * kLog2e;
-    const float bl_m = bl2 - lse2, bp_m = bp2 - lse2;
+    const float bl_m = (RES ? bp2 : bl2) - lse2, bp_m = bp2 - lse2;  // RES: the band is skip keys
     const float NEG_INF = -INFINITY;
     float dzw = 0.f, dzs = 0.f;  // sums of ds over window keys and over skip keys
 
@@ -336,7 +369,14 @@ __global__ void __launch_bounds__(192, BSmem<D>::kCtas) bwd_dq_kernel(const __gr
       mbar_arrive(bar_dsfull);
     }
     // ---- epilogue: dq = tau dQ + dz w_g, and the row terms
-    const float dz = (1.f - alpha) * dzw - alpha * dzs;
+    if (RES) {  // the band columns were skip keys
+      dzs += dzw;
+      dzw = 0.f;
+    }
+    // this pass's dz goes into its dq; the row's whole dz (with the residue pass's part, whose dq
+    // already holds its own) into the gate's sums
+    const float dz_own = (1.f - alpha) * dzw - alpha * dzs;
+    const float dz = !RES && prm.acc && row_ok ? dz_own + prm.dz[orow] : dz_own;
     const bool have_q = __all_sync(0xffffffffu, ok && j > 0 && mbar_wait(bar_dqdone, (j - 1) & 1, abort_flag));
     if (have_q) tc_fence_after();
     const float tau = prm.scale_log2 / kLog2e;
@@ -356,22 +396,29 @@ __global__ void __launch_bounds__(192, BSmem<D>::kCtas) bwd_dq_kernel(const __gr
 #pragma unroll
           for (int e = 0; e < 8; ++e) {
             const float4 w = wv[e];
-            dst[e] = make_float4(fmaf(tau, o[4 * e], dz * w.x), fmaf(tau, o[4 * e + 1], dz * w.y),
-                                 fmaf(tau, o[4 * e + 2], dz * w.z), fmaf(tau, o[4 * e + 3], dz * w.w));
+            float4 v = make_float4(fmaf(tau, o[4 * e], dz_own * w.x), fmaf(tau, o[4 * e + 1], dz_own * w.y),
+                                   fmaf(tau, o[4 * e + 2], dz_own * w.z), fmaf(tau, o[4 * e + 3], dz_own * w.w));
+            if (!RES && prm.acc) {  // add to the residue pass's dq
+              const float4 a = dst[e];
+              v = make_float4(a.x + v.x, a.y + v.y, a.z + v.z, a.w + v.w);
+            }
+            dst[e] = v;
           }
         }
       }
       if (row_ok) {
-        prm.lse2[orow] = lse2;
-        prm.bl2[orow] = bl2;
-        prm.bp2[orow] = bp2;
+        if (!RES) {
+          prm.lse2[orow] = lse2;
+          prm.bl2[orow] = bl2;
+          prm.bp2[orow] = bp2;
+        }
         prm.dz[orow] = dz;
       }
     }
     // The gate's partial sums over this CTA's rows, in a fixed order: dw_g[c] += sum_r dz_r q_rc
     // and db_g += sum_r dz_r.  G = BM / D threads a column, each over BM / G rows of the Q tile
     // (still in shared memory), then the G parts in order.
-    {
+    if (!RES) {
       float* const dz_s = reinterpret_cast<float*>(sbase + L::kDz);
       float* const red = reinterpret_cast<float*>(sbase + L::kRed);
       dz_s[r] = (have_q || j == 0) && row_ok ? dz : 0.f;
@@ -459,9 +506,13 @@ struct KParams {
   int n, kwin, pi, S;
   float scale_log2;
   int bidir;
+  int acc;            // add to the dk and dv that the residue pass wrote (the split backward)
 };
 
-template <int D>
+// RES as for the dq pass: RES = 1 takes the skips alone in the residue-class view (the CTA's keys
+// are keys u*pi + res of the sequence, read by the rows u + m0 .. u + S of the same class, all with
+// the skip prior) and writes dk, dv; the window pass (S = 0) then adds to them.
+template <int D, int RES>
 __global__ void __launch_bounds__(192, KSmem<D>::kCtas) bwd_dkv_kernel(const __grid_constant__ CUtensorMap tmk,
                                                                         const __grid_constant__ CUtensorMap tmv,
                                                                         const __grid_constant__ CUtensorMap tmq,
@@ -479,7 +530,10 @@ __global__ void __launch_bounds__(192, KSmem<D>::kCtas) bwd_dkv_kernel(const __g
   }
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int bh = blockIdx.y;
-  const long long j0 = (long long)blockIdx.x * BM;  // this CTA's keys j0 .. j0 + 127
+  const int res = RES ? (int)(blockIdx.x % prm.pi) : 0;
+  // this CTA's keys j0 .. j0 + 127 of the view (the sequence, or residue class res)
+  const long long j0 = RES ? (long long)(blockIdx.x / prm.pi) * BM : (long long)blockIdx.x * BM;
+  const long long T = RES ? prm.n / prm.pi : prm.n;  // rows of the view
   const uint32_t sK = base + L::kK, sV = base + L::kV, sQ = base + L::kQ, sG = base + L::kG;
   const uint32_t bar0 = base + L::kBar;
   const uint32_t bar_kv = bar0;
@@ -504,17 +558,41 @@ __global__ void __launch_bounds__(192, KSmem<D>::kCtas) bwd_dkv_kernel(const __g
     mbar_expect_tx(bar_kv, 2 * L::kKeyBytes);
 #pragma unroll
     for (int c = 0; c < D / 64; ++c) {
-      tma_load_3d(sK + c * BM * 128, &tmk, bar_kv, c * 64, (int)j0, bh);
-      tma_load_3d(sV + c * BM * 128, &tmv, bar_kv, c * 64, (int)j0, bh);
+      if (RES) {
+        tma_load_4d(sK + c * BM * 128, &tmk, bar_kv, c * 64, res, (int)j0, bh);
+        tma_load_4d(sV + c * BM * 128, &tmv, bar_kv, c * 64, res, (int)j0, bh);
+      } else {
+        tma_load_3d(sK + c * BM * 128, &tmk, bar_kv, c * 64, (int)j0, bh);
+        tma_load_3d(sV + c * BM * 128, &tmv, bar_kv, c * 64, (int)j0, bh);
+      }
     }
   }
   const int m0 = first_skip_m(prm.kwin, prm.pi);
   ReaderWalk walk;
-  walk.init(j0, prm.n, BM, prm.kwin, prm.pi, prm.S, prm.bidir != 0);
+  if (RES) {  // readers of view key u: rows u + m0 .. u + S
+    walk.j0 = j0;
+    walk.n = T;
+    walk.jl = j0 + BM - 1 < T - 1 ? j0 + BM - 1 : T - 1;
+    walk.w_lo = j0 + m0;
+    walk.w_hi = walk.jl + prm.S < T - 1 ? walk.jl + prm.S : T - 1;
+    if (walk.w_lo > walk.w_hi) walk.w_hi = -1;  // no reader at all
+    walk.pi = 1;
+    walk.S = 0;
+    walk.m0 = 1;
+    walk.bidir = false;
+    walk.rpi = 1.0;
+  } else {
+    walk.init(j0, prm.n, BM, prm.kwin, prm.pi, prm.S, prm.bidir != 0);
+  }
   int t_first = -1;
   auto load_rows = [&](uint32_t dst, const CUtensorMap* map, uint32_t bar, long long r0) {
 #pragma unroll
-    for (int c = 0; c < D / 64; ++c) tma_load_3d(dst + c * BN * 128, map, bar, c * 64, (int)r0, bh);
+    for (int c = 0; c < D / 64; ++c) {
+      if (RES)
+        tma_load_4d(dst + c * BN * 128, map, bar, c * 64, res, (int)r0, bh);
+      else
+        tma_load_3d(dst + c * BN * 128, map, bar, c * 64, (int)r0, bh);
+    }
   };
   if (threadIdx.x == 0) {
     for (int s = 0; s < NSTAGE; ++s) {
@@ -627,14 +705,16 @@ __global__ void __launch_bounds__(192, KSmem<D>::kCtas) bwd_dkv_kernel(const __g
     // ------------------------------------------------------------------ key warpgroup
     const int q4 = warp & 3;
     const int r = q4 * 32 + lane;
-    const long long j = j0 + r;
-    const bool key_ok = j < prm.n;
-    const long long krow = (long long)bh * prm.n + (key_ok ? j : 0);
+    const long long j = j0 + r;  // key of the view
+    const bool key_ok = j < T;
+    const long long krow = (long long)bh * prm.n + (key_ok ? (RES ? j * prm.pi + res : j) : 0);
     const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
-    const long long w_lo = prm.bidir ? (j - prm.kwin > 0 ? j - prm.kwin : 0) : j;  // rows reading j as window key
-    const long long w_hi = j + prm.kwin < prm.n - 1 ? j + prm.kwin : prm.n - 1;
+    // rows reading j as window key (RES: the band of view rows j + m0 .. j + S, all skip readers)
+    const long long w_lo = RES ? j + m0 : (prm.bidir ? (j - prm.kwin > 0 ? j - prm.kwin : 0) : j);
+    const long long w_hi = RES ? (j + prm.S < T - 1 ? j + prm.S : T - 1)
+                               : (j + prm.kwin < prm.n - 1 ? j + prm.kwin : prm.n - 1);
     KeyReaders kr;
-    kr.init(j, prm.pi, prm.S, m0, walk.rpi, prm.bidir != 0, prm.n);
+    kr.init(j, prm.pi, RES ? 0 : prm.S, m0, walk.rpi, prm.bidir != 0, prm.n);
     const float NEG_INF = -INFINITY;
     const int tid = threadIdx.x - 64;  // 0..127
     float4* const stat = reinterpret_cast<float4*>(sbase + L::kStat);
@@ -647,9 +727,11 @@ __global__ void __launch_bounds__(192, KSmem<D>::kCtas) bwd_dkv_kernel(const __g
       // on the previous tile; a warp here has finished that one)
       float4* const st = stat + (jt & 1) * BN;
       if (tid < BN) {
-        const long long i = r0 + tid;
-        st[tid] = i < prm.n ? make_float4(prm.lse2[rbase + i], prm.Dr[rbase + i], prm.bl2[rbase + i], prm.bp2[rbase + i])
-                            : make_float4(0.f, 0.f, NEG_INF, NEG_INF);
+        const long long i = r0 + tid;  // row of the view
+        const long long ri = rbase + (RES ? i * prm.pi + res : i);
+        // (lse2, D, the band's prior, the skip prior): RES's band is skip keys
+        st[tid] = i < T ? make_float4(prm.lse2[ri], prm.Dr[ri], RES ? prm.bp2[ri] : prm.bl2[ri], prm.bp2[ri])
+                        : make_float4(0.f, 0.f, NEG_INF, NEG_INF);
       }
       asm volatile("bar.sync 1, 128;" ::: "memory");
       if (!ok) continue;  // keep taking part in the barrier above while the other warps finish
@@ -721,8 +803,15 @@ __global__ void __launch_bounds__(192, KSmem<D>::kCtas) bwd_dkv_kernel(const __g
           float4* dvp = reinterpret_cast<float4*>(prm.dv + krow * D + c * 32);
 #pragma unroll
           for (int e = 0; e < 8; ++e) {
-            dkp[e] = make_float4(tau * a[4 * e], tau * a[4 * e + 1], tau * a[4 * e + 2], tau * a[4 * e + 3]);
-            dvp[e] = make_float4(b[4 * e], b[4 * e + 1], b[4 * e + 2], b[4 * e + 3]);
+            float4 kv = make_float4(tau * a[4 * e], tau * a[4 * e + 1], tau * a[4 * e + 2], tau * a[4 * e + 3]);
+            float4 vv = make_float4(b[4 * e], b[4 * e + 1], b[4 * e + 2], b[4 * e + 3]);
+            if (!RES && prm.acc) {  // add to the residue pass's dk, dv
+              const float4 ka = dkp[e], va = dvp[e];
+              kv = make_float4(ka.x + kv.x, ka.y + kv.y, ka.z + kv.z, ka.w + kv.w);
+              vv = make_float4(va.x + vv.x, va.y + vv.y, va.z + vv.z, va.w + vv.w);
+            }
+            dkp[e] = kv;
+            dvp[e] = vv;
           }
         }
       }
@@ -736,18 +825,30 @@ __global__ void __launch_bounds__(192, KSmem<D>::kCtas) bwd_dkv_kernel(const __g
   }
 }
 
-template <int D>
+// The row-side tensor maps: the sequence view, or (RES) the residue-class view, box_rows rows a box.
+template <int RES>
+inline bool bwd_map(CUtensorMap* m, const void* p, int BH, int n, int d, int pi, int box_rows) {
+  return RES ? tc::make_residue_map(m, p, BH, n, d, pi, box_rows) : tc::make_map(m, p, BH, n, d, box_rows);
+}
+
+// Grid columns: the 128-row (or key) tiles of the view; RES: pi classes of n / pi rows each.
+template <int RES>
+inline unsigned bwd_tiles(int n, int pi) {
+  return RES ? (unsigned)(pi * ((n / pi + BM - 1) / BM)) : (unsigned)((n + BM - 1) / BM);
+}
+
+template <int D, int RES>
 cudaError_t launch_bwd_dkv(const void* q, const void* k, const void* v, const void* dout, const KParams& p, int BH,
                            cudaStream_t st, const char** why) {
   CUtensorMap mk, mv, mq, mg;
-  if (!tc::make_map(&mk, k, BH, p.n, D, BM) || !tc::make_map(&mv, v, BH, p.n, D, BM) ||
-      !tc::make_map(&mq, q, BH, p.n, D, BN) || !tc::make_map(&mg, dout, BH, p.n, D, BN)) {
+  if (!bwd_map<RES>(&mk, k, BH, p.n, D, p.pi, BM) || !bwd_map<RES>(&mv, v, BH, p.n, D, p.pi, BM) ||
+      !bwd_map<RES>(&mq, q, BH, p.n, D, p.pi, BN) || !bwd_map<RES>(&mg, dout, BH, p.n, D, p.pi, BN)) {
     *why = "cuTensorMapEncodeTiled failed";
     return cudaErrorInvalidValue;
   }
   static bool attr_done = false;
   if (!attr_done) {
-    cudaError_t e = cudaFuncSetAttribute(bwd_dkv_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaError_t e = cudaFuncSetAttribute(bwd_dkv_kernel<D, RES>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          KSmem<D>::kAlloc);
     if (e != cudaSuccess) {
       *why = "cudaFuncSetAttribute";
@@ -755,39 +856,39 @@ cudaError_t launch_bwd_dkv(const void* q, const void* k, const void* v, const vo
     }
     attr_done = true;
   }
-  const dim3 grid((unsigned)((p.n + BM - 1) / BM), (unsigned)BH);
-  bwd_dkv_kernel<D><<<grid, 192, KSmem<D>::kAlloc, st>>>(mk, mv, mq, mg, p);
+  const dim3 grid(bwd_tiles<RES>(p.n, p.pi), (unsigned)BH);
+  bwd_dkv_kernel<D, RES><<<grid, 192, KSmem<D>::kAlloc, st>>>(mk, mv, mq, mg, p);
   *why = "tensor-core dk/dv kernel launch";
   return cudaGetLastError();
 }
 
-template <int D>
+template <int D, int RES>
 cudaError_t set_bwd_smem_attr() {
   static bool done = false;
   if (done) return cudaSuccess;
   cudaError_t e =
-      cudaFuncSetAttribute(bwd_dq_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, BSmem<D>::kAlloc);
+      cudaFuncSetAttribute(bwd_dq_kernel<D, RES>, cudaFuncAttributeMaxDynamicSharedMemorySize, BSmem<D>::kAlloc);
   if (e == cudaSuccess) done = true;
   return e;
 }
 
 // The dq pass: q, dout [BH, n, D] bf16, k, v [BH, n, D] bf16; lse, Dr [BH, n] from the forward.
-template <int D>
+template <int D, int RES>
 cudaError_t launch_bwd_dq(const void* q, const void* k, const void* v, const void* dout, const BParams& p, int BH,
                           cudaStream_t st, const char** why) {
   CUtensorMap mq, mg, mk, mv;
-  if (!tc::make_map(&mq, q, BH, p.n, D, BM) || !tc::make_map(&mg, dout, BH, p.n, D, BM) ||
-      !tc::make_map(&mk, k, BH, p.n, D, BN) || !tc::make_map(&mv, v, BH, p.n, D, BN)) {
+  if (!bwd_map<RES>(&mq, q, BH, p.n, D, p.pi, BM) || !bwd_map<RES>(&mg, dout, BH, p.n, D, p.pi, BM) ||
+      !bwd_map<RES>(&mk, k, BH, p.n, D, p.pi, BN) || !bwd_map<RES>(&mv, v, BH, p.n, D, p.pi, BN)) {
     *why = "cuTensorMapEncodeTiled failed";
     return cudaErrorInvalidValue;
   }
-  cudaError_t e = set_bwd_smem_attr<D>();
+  cudaError_t e = set_bwd_smem_attr<D, RES>();
   if (e != cudaSuccess) {
     *why = "cudaFuncSetAttribute";
     return e;
   }
-  const dim3 grid((unsigned)((p.n + BM - 1) / BM), (unsigned)BH);
-  bwd_dq_kernel<D><<<grid, 192, BSmem<D>::kAlloc, st>>>(mq, mg, mk, mv, p);
+  const dim3 grid(bwd_tiles<RES>(p.n, p.pi), (unsigned)BH);
+  bwd_dq_kernel<D, RES><<<grid, 192, BSmem<D>::kAlloc, st>>>(mq, mg, mk, mv, p);
   *why = "tensor-core dq kernel launch";
   return cudaGetLastError();
 }

@@ -952,14 +952,20 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm<D>) fwd_tc_kernel(const _
         }
         *reinterpret_cast<uint4*>(sbase + L::kV + off) = make_uint4(w[0], w[1], w[2], w[3]);
       }
-      if (MODE == kFused && prm.dout && row_ok) {
+      // for the backward: D = dout . out over the fp32 output row (the values rounded to bf16 above)
+      if (MODE != kResidue && prm.dout && row_ok) {
+        const float ow = inv * wl;
         float dsum = 0.f;
 #pragma unroll
         for (int cl = 0; cl < D / 8; ++cl) {
-          float g[8];
+          float g[8], sp[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
           bf16x8_to_f32(*reinterpret_cast<const uint4*>(prm.dout + orow * D + cl * 8), g);
+          if (MODE == kBandMerge && so_ok) {
+            const uint32_t off = (cl >> 3) * (BM * 128) + r * 128 + (((cl & 7) ^ (r & 7)) << 4);
+            bf16x8_to_f32(*reinterpret_cast<const uint4*>(sbase + L::kK + off), sp);
+          }
 #pragma unroll
-          for (int e = 0; e < 8; ++e) dsum = fmaf(o[cl * 8 + e] * inv, g[e], dsum);
+          for (int e = 0; e < 8; ++e) dsum = fmaf(fmaf(o[cl * 8 + e], ow, sp[e] * wp), g[e], dsum);
         }
         prm.Dout[orow] = dsum;
       }
@@ -1074,7 +1080,8 @@ inline bool tc_split_preferred(int n, int kwin, int pi, int S) {
 template <int D>
 cudaError_t launch_fwd_tc_d(const void* q, const void* k, const void* v, const float* w_g, const float* b_g,
                             void* out, float* lse, int B, int H, int n, int kwin, int pi, int S, bool split,
-                            bool bidir, void* workspace, cudaStream_t st, const char** why) {
+                            bool bidir, void* workspace, cudaStream_t st, const char** why,
+                            const void* dout = nullptr, float* Dout = nullptr) {
   using L = tc::Smem<D>;
   CUtensorMap mq, mk, mv;
   const int BH = B * H;
@@ -1100,8 +1107,8 @@ cudaError_t launch_fwd_tc_d(const void* q, const void* k, const void* v, const f
   p.bidir = bidir ? 1 : 0;
   p.row0 = 0;
   p.kv0 = 0;
-  p.dout = nullptr;
-  p.Dout = nullptr;
+  p.dout = (const __nv_bfloat16*)dout;
+  p.Dout = Dout;
   const dim3 grid((unsigned)((n + tc::BM - 1) / tc::BM), (unsigned)BH);
   cudaError_t e;
   CUtensorMap mo;
@@ -1195,45 +1202,16 @@ cudaError_t launch_fwd_tc_shard_d(const void* q, const void* k, const void* v, c
   return cudaGetLastError();
 }
 
-// The backward's forward: the single pass over a whole sequence, writing out, lse and, from the
-// fp32 output rows, D = dout . out of every row.
+// The backward's forward over a whole sequence, writing out, lse and, from the fp32 output rows,
+// D = dout . out of every row: the single pass, or (split) the residue pass and the window pass,
+// whose skip partials take rows * (2 D + 4) bytes of `workspace` (16-byte aligned).
 template <int D>
 cudaError_t launch_fwd_tc_with_dot(const void* q, const void* k, const void* v, const float* w_g, const float* b_g,
                                    const void* dout, void* out, float* lse, float* Dout, int B, int H, int n, int kwin,
-                                   int pi, int S, bool bidir, cudaStream_t st, const char** why) {
-  using L = tc::Smem<D>;
-  CUtensorMap mq, mk, mv, mo;
-  const int BH = B * H;
-  if (!tc::make_map(&mq, q, BH, n, D, tc::BM) || !tc::make_map(&mk, k, BH, n, D, tc::BN) ||
-      !tc::make_map(&mv, v, BH, n, D, tc::BN) || !tc::make_map(&mo, out, BH, n, D, tc::BM)) {
-    *why = "cuTensorMapEncodeTiled failed";
-    return cudaErrorInvalidValue;
-  }
-  tc::Params p;
-  p.w_g = w_g;
-  p.b_g = b_g;
-  p.out = (__nv_bfloat16*)out;
-  p.lse = lse;
-  p.skip_o = nullptr;
-  p.skip_lse = nullptr;
-  p.H = H;
-  p.n = n;
-  p.kwin = kwin;
-  p.pi = pi;
-  p.S = S;
-  p.T = 0;
-  p.scale_log2 = (float)(1.0 / std::sqrt((double)D)) * kLog2e;
-  p.bidir = bidir ? 1 : 0;
-  p.row0 = 0;
-  p.kv0 = 0;
-  p.dout = (const __nv_bfloat16*)dout;
-  p.Dout = Dout;
-  cudaError_t e;
-  if ((e = tc::set_smem_attr<D, tc::kFused>()) != cudaSuccess) { *why = "cudaFuncSetAttribute"; return e; }
-  const dim3 grid((unsigned)((n + tc::BM - 1) / tc::BM), (unsigned)BH);
-  tc::fwd_tc_kernel<D, tc::kFused><<<grid, tc::kThreads, L::kAlloc, st>>>(mq, mk, mv, mo, mo, p);
-  *why = "tensor-core forward (backward's) launch";
-  return cudaGetLastError();
+                                   int pi, int S, bool bidir, bool split, void* workspace, cudaStream_t st,
+                                   const char** why) {
+  return launch_fwd_tc_d<D>(q, k, v, w_g, b_g, out, lse, B, H, n, kwin, pi, S, split, bidir, workspace, st, why, dout,
+                            Dout);
 }
 
 // mode: 0 = choose, 1 = single pass, 2 = split (residue pass + window pass)

@@ -522,7 +522,7 @@ pi_attn_status pi_attn_debug_index_sets_bidir(int n, int k_win, int pi, int S, i
 long long pi_attn_bwd_workspace_bytes(int B, int H, int n, int d) { return bwd_ws_bytes(B, H, n, d, false); }
 
 long long pi_attn_bwd_workspace_bytes_ex(int B, int H, int n, int d, pi_attn_dtype dtype, pi_attn_bwd_path path) {
-  const bool tc = path == PI_ATTN_BWD_TC ||
+  const bool tc = path == PI_ATTN_BWD_TC || path == PI_ATTN_BWD_TC_FUSED || path == PI_ATTN_BWD_TC_SPLIT ||
                   (path == PI_ATTN_BWD_AUTO && dtype == PI_ATTN_BF16 && (d == 64 || d == 128));
   return bwd_ws_bytes(B, H, n, d, tc);
 }
@@ -535,13 +535,20 @@ pi_attn_status pi_attn_bwd_ex(const void* q, const void* k, const void* v, const
   if (st != PI_ATTN_OK) return st;
   if (!dq || !dk || !dv || !dw_g || !db_g) return fail(PI_ATTN_EINVAL, "null gradient pointer");
   if (!aligned16(dq) || !aligned16(dk) || !aligned16(dv)) return fail(PI_ATTN_EINVAL, "dq, dk, dv must be 16-byte aligned");
-  if (path != PI_ATTN_BWD_AUTO && path != PI_ATTN_BWD_SIMT && path != PI_ATTN_BWD_TC)
+  if (path < PI_ATTN_BWD_AUTO || path > PI_ATTN_BWD_TC_SPLIT)
     return fail(PI_ATTN_EINVAL, "unknown backward path %d", (int)path);
   const bool tc_ok = dtype == PI_ATTN_BF16 && (d == 64 || d == 128);
-  if (path == PI_ATTN_BWD_TC && !tc_ok)
+  const bool want_tc = path == PI_ATTN_BWD_TC || path == PI_ATTN_BWD_TC_FUSED || path == PI_ATTN_BWD_TC_SPLIT;
+  if (want_tc && !tc_ok)
     return fail(PI_ATTN_EUNSUPPORTED, "the tensor-core backward covers bf16 with d in {64, 128} (got dtype %d, d %d)",
                 (int)dtype, d);
-  const bool tc = path == PI_ATTN_BWD_TC || (path == PI_ATTN_BWD_AUTO && tc_ok);
+  if (path == PI_ATTN_BWD_TC_SPLIT && bidir)
+    return fail(PI_ATTN_EUNSUPPORTED, "the split backward covers the causal rule only");
+  if (path == PI_ATTN_BWD_TC_SPLIT && !pia::tc_split_applies(n, k_win, pi, S))
+    return fail(PI_ATTN_EUNSUPPORTED, "split backward needs n %% pi == 0 and at least one skip outside the window");
+  const bool tc = want_tc || (path == PI_ATTN_BWD_AUTO && tc_ok);
+  const bool split = tc && !bidir && (path == PI_ATTN_BWD_TC_SPLIT ||
+                                      (path != PI_ATTN_BWD_TC_FUSED && pia::tc_split_preferred(n, k_win, pi, S)));
   const long long rows = (long long)B * H * n;
   const long long need = bwd_ws_bytes(B, H, n, d, tc);
   if (workspace) {
@@ -569,56 +576,74 @@ pi_attn_status pi_attn_bwd_ex(const void* q, const void* k, const void* v, const
   const char* why = "backward kernel launch";
   using bf = __nv_bfloat16;
   if (tc) {
-    // the forward (single tensor-core pass) for out, lse and D = dO . out (from its fp32 output
-    // rows), then the dq pass and the dk/dv pass on the tensor cores
+    // the forward on the tensor cores for out, lse and D = dO . out (from its fp32 output rows),
+    // then the dq pass and the dk/dv pass on the tensor cores.  Split: the forward's skip partials
+    // go to dq (rows * (2d + 4) <= rows * 4d bytes, written over by the dq passes after it), and
+    // each pass runs over the skips in the residue view first, then over the window (S = 0),
+    // adding to what the first wrote.
     const long long off = (bwd_ws_bytes(B, H, n, d, true) - rows * 2LL * d - rows * 4LL);
     bf* out_ws = reinterpret_cast<bf*>(static_cast<char*>(scratch) + off);
     float* lse_ws = reinterpret_cast<float*>(static_cast<char*>(scratch) + off + rows * 2LL * d);
     e = d == 128 ? pia::launch_fwd_tc_with_dot<128>(q, k, v, w_g, b_g, dout, out_ws, lse_ws, rs.D, B, H, n, k_win,
-                                                    pi, S, bd, s, &why)
+                                                    pi, S, bd, split, dq, s, &why)
                  : pia::launch_fwd_tc_with_dot<64>(q, k, v, w_g, b_g, dout, out_ws, lse_ws, rs.D, B, H, n, k_win, pi,
-                                                   S, bd, s, &why);
-    if (e == cudaSuccess) {
-      pia::tcb::BParams bp;
-      bp.w_g = w_g;
-      bp.b_g = b_g;
-      bp.lse = lse_ws;
-      bp.Dr = rs.D;
-      bp.lse2 = rs.lse2;
-      bp.dq = dq;
-      bp.bl2 = rs.bl2;
-      bp.bp2 = rs.bp2;
-      bp.dz = rs.dz;
-      bp.part_w = part_w;
-      bp.part_b = part_b;
-      bp.H = H;
-      bp.n = n;
-      bp.kwin = k_win;
-      bp.pi = pi;
-      bp.S = S;
-      bp.scale_log2 = scale_log2;
-      bp.bidir = bd ? 1 : 0;
-      e = d == 128 ? pia::tcb::launch_bwd_dq<128>(q, k, v, dout, bp, B * H, s, &why)
-                   : pia::tcb::launch_bwd_dq<64>(q, k, v, dout, bp, B * H, s, &why);
+                                                   S, bd, split, dq, s, &why);
+    pia::tcb::BParams bp;
+    bp.w_g = w_g;
+    bp.b_g = b_g;
+    bp.lse = lse_ws;
+    bp.Dr = rs.D;
+    bp.lse2 = rs.lse2;
+    bp.dq = dq;
+    bp.bl2 = rs.bl2;
+    bp.bp2 = rs.bp2;
+    bp.dz = rs.dz;
+    bp.part_w = part_w;
+    bp.part_b = part_b;
+    bp.H = H;
+    bp.n = n;
+    bp.kwin = k_win;
+    bp.pi = pi;
+    bp.S = S;
+    bp.scale_log2 = scale_log2;
+    bp.bidir = bd ? 1 : 0;
+    bp.acc = 0;
+    pia::tcb::KParams kp;
+    kp.lse2 = rs.lse2;
+    kp.Dr = rs.D;
+    kp.bl2 = rs.bl2;
+    kp.bp2 = rs.bp2;
+    kp.dk = dk;
+    kp.dv = dv;
+    kp.n = n;
+    kp.kwin = k_win;
+    kp.pi = pi;
+    kp.S = S;
+    kp.scale_log2 = scale_log2;
+    kp.bidir = bd ? 1 : 0;
+    kp.acc = 0;
+    using namespace pia::tcb;
+    if (split) {
+      if (e == cudaSuccess)
+        e = d == 128 ? launch_bwd_dq<128, 1>(q, k, v, dout, bp, B * H, s, &why)
+                     : launch_bwd_dq<64, 1>(q, k, v, dout, bp, B * H, s, &why);
+      bp.S = 0;  // the window pass
+      bp.acc = 1;
     }
-    if (e == cudaSuccess) {
-      pia::tcb::KParams kp;
-      kp.lse2 = rs.lse2;
-      kp.Dr = rs.D;
-      kp.bl2 = rs.bl2;
-      kp.bp2 = rs.bp2;
-      kp.dk = dk;
-      kp.dv = dv;
-      kp.n = n;
-      kp.kwin = k_win;
-      kp.pi = pi;
-      kp.S = S;
-      kp.scale_log2 = scale_log2;
-      kp.bidir = bd ? 1 : 0;
-      e = d == 128 ? pia::tcb::launch_bwd_dkv<128>(q, k, v, dout, kp, B * H, s, &why)
-                   : pia::tcb::launch_bwd_dkv<64>(q, k, v, dout, kp, B * H, s, &why);
+    if (e == cudaSuccess)
+      e = d == 128 ? launch_bwd_dq<128, 0>(q, k, v, dout, bp, B * H, s, &why)
+                   : launch_bwd_dq<64, 0>(q, k, v, dout, bp, B * H, s, &why);
+    if (split) {
+      if (e == cudaSuccess)
+        e = d == 128 ? launch_bwd_dkv<128, 1>(q, k, v, dout, kp, B * H, s, &why)
+                     : launch_bwd_dkv<64, 1>(q, k, v, dout, kp, B * H, s, &why);
+      kp.S = 0;
+      kp.acc = 1;
     }
-    // (the gate's partial sums come from the dq pass, one per (b, query tile))
+    if (e == cudaSuccess)
+      e = d == 128 ? launch_bwd_dkv<128, 0>(q, k, v, dout, kp, B * H, s, &why)
+                   : launch_bwd_dkv<64, 0>(q, k, v, dout, kp, B * H, s, &why);
+    // (the gate's partial sums come from the window dq pass, one per (b, query tile))
   } else if (dtype == PI_ATTN_F32) {
     e = launch_bwd<float>(q, k, v, w_g, b_g, dout, dq, dk, dv, rs, gt, H, n, d, k_win, pi, S, scale_log2, bd, s);
     if (e == cudaSuccess)

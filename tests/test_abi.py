@@ -169,6 +169,19 @@ def test_tensor_core_backward_arguments_are_checked_before_any_launch(lib):
     assert simt == lib.pi_attn_bwd_workspace_bytes(1, 2, 64, 64) and tc >= 4 * 5 * rows + rows * (2 * 64 + 4)
     assert lib.pi_attn_bwd_ex(*args, 1, 2, 64, 64, 8, 16, 2, pia.PI_ATTN_BF16, 0, 2, FAKE, tc - 16, None) == \
         pia.PI_ATTN_EINVAL
+    # the fused and split tensor-core paths take the same workspace (the split's skip partials
+    # live in dq until the dq passes write it)
+    assert lib.pi_attn_bwd_workspace_bytes_ex(1, 2, 64, 64, pia.PI_ATTN_BF16, 3) == tc
+    assert lib.pi_attn_bwd_workspace_bytes_ex(1, 2, 64, 64, pia.PI_ATTN_BF16, 4) == tc
+    split = pia.BWD_PATHS["tc_split"]
+    assert lib.pi_attn_bwd_ex(*args, 1, 2, 64, 64, 8, 16, 2, pia.PI_ATTN_BF16, 1, split, None, 0, None) == \
+        pia.PI_ATTN_EUNSUPPORTED  # bidirectional
+    assert lib.pi_attn_bwd_ex(*args, 1, 2, 60, 64, 8, 16, 2, pia.PI_ATTN_BF16, 0, split, None, 0, None) == \
+        pia.PI_ATTN_EUNSUPPORTED  # n not a whole number of periods
+    assert lib.pi_attn_bwd_ex(*args, 1, 2, 64, 64, 40, 16, 2, pia.PI_ATTN_BF16, 0, split, None, 0, None) == \
+        pia.PI_ATTN_EUNSUPPORTED  # no skip outside the window (m0 = 3 > S)
+    assert lib.pi_attn_bwd_ex(*args, 1, 2, 64, 64, 8, 16, 2, pia.PI_ATTN_BF16, 0, 5, None, 0, None) == \
+        pia.PI_ATTN_EINVAL
 
 
 def test_built_for_sm100a_only():

@@ -65,7 +65,7 @@ def _check(inp, dtype, k, pi, S, bidir, what, path="simt"):
     dev = {x: to_dev(inp[x], dtype) for x in ("q", "k", "v", "dO")}
     wg, bg = torch.from_numpy(inp["w_g"]).cuda(), torch.from_numpy(inp["b_g"]).cuda()
     got = pia.pi_attn_bwd(dev["q"], dev["k"], dev["v"], wg, bg, dev["dO"], k, pi, S, bidir=bidir, path=path)
-    rel_l2, max_abs, floor = (REL_L2_TC, MAX_ABS_FRAC_TC, GATE_FLOOR_TC) if path == "tc" else \
+    rel_l2, max_abs, floor = (REL_L2_TC, MAX_ABS_FRAC_TC, GATE_FLOOR_TC) if path != "simt" else \
         (REL_L2, MAX_ABS_FRAC, GATE_FLOOR)
     pia.pi_attn_check()
     ref = oracle.bwd(inp["q"], inp["k"], inp["v"], inp["w_g"], inp["b_g"], _widen(inp["dO"]), k, pi, S, bidir=bidir)
@@ -108,6 +108,42 @@ def test_backward_tensor_core_path(case, bidir):
     B, H, n, d, k, pi, S = case
     _check(_problem(B, H, n, d, "bf16", seed=n + 13 * k), "bf16", k, pi, S, bidir, f"{case} tc bidir={bidir}",
            path="tc")
+
+
+# The split backward: causal, n a whole number of periods, skips outside the window.  The residue
+# view has T = n / pi rows per class: fewer than a 128-row tile, one tile, several with a ragged
+# last one; pi = 1 (the view is the sequence); a skip band wider than a key tile.
+SPLIT_CASES = [  # B, H, n, d, k, pi, S
+    (1, 1, 64, 64, 8, 16, 3),          # T = 4
+    (1, 2, 1024, 64, 40, 16, 30),      # T = 64, 28 skips
+    (2, 2, 2048, 128, 100, 64, 12),    # T = 32, m0 = 2
+    (1, 1, 8192, 128, 256, 32, 40),    # T = 256: two row tiles per class, m0 = 9
+    (1, 2, 3000, 64, 10, 1, 90),       # pi = 1: the band of 80 skips is the sequence's
+    (1, 2, 2560, 64, 50, 10, 20),      # T = 256, m0 = 6
+    (1, 1, 4480, 128, 200, 35, 7),     # T = 128, m0 = 6: two skips
+    (1, 1, 2048, 64, 64, 32, 6),       # tie: 2 * pi == k is a window key, m0 = 3
+]
+
+
+@pytest.mark.parametrize("case", SPLIT_CASES)
+@pytest.mark.parametrize("path", ["tc_split", "tc_fused"])
+def test_backward_tensor_core_split_and_fused(case, path):
+    B, H, n, d, k, pi, S = case
+    _check(_problem(B, H, n, d, "bf16", seed=n + 7 * S), "bf16", k, pi, S, False, f"{case} {path}", path=path)
+
+
+def test_backward_split_n4k_geometry_and_determinism():
+    # the bf16_n4k shape (pi = 64, T = 64) through the split passes, twice: the same bits
+    w = ps.WORKLOADS["bf16_n4k"]
+    inp = ps.prefill_inputs(w)
+    inp["dO"] = ps.normal((w.B, w.H, w.n, w.d), seed=0, stream=6, dtype="bf16")
+    a = [t.clone() for t in _check(inp, "bf16", w.k, w.pi, w.S, False, "bf16_n4k tc_split", path="tc_split")[0]]
+    dev = {x: to_dev(inp[x], "bf16") for x in ("q", "k", "v", "dO")}
+    wg, bg = torch.from_numpy(inp["w_g"]).cuda(), torch.from_numpy(inp["b_g"]).cuda()
+    b = pia.pi_attn_bwd(dev["q"], dev["k"], dev["v"], wg, bg, dev["dO"], w.k, w.pi, w.S, path="tc_split")
+    pia.pi_attn_check()
+    for x, y in zip(a, b):
+        assert torch.equal(x, y)
 
 
 def test_backward_tensor_core_path_bf16_n4k_workload():
