@@ -355,7 +355,7 @@ inline size_t bwd_key_smem(int d, size_t esz) { return 2 * (size_t)kTileKeys * d
 
 // dw_g[h][c] = sum over (b, i) of dz * q[c], db_g[h] = sum of dz, in two stages with a fixed order:
 // bwd_gate_partial_kernel sums chunks of kGateRows rows of one head (one block per (chunk, head),
-// one thread per column), bwd_gate_final_kernel adds the chunks in a fixed interleaved order.
+// one thread per column), bwd_gate_final_kernel adds the chunks in a fixed order.
 constexpr int kGateRows = 32;
 
 template <typename T>
@@ -378,37 +378,56 @@ __global__ void __launch_bounds__(256) bwd_gate_partial_kernel(const T* __restri
   if (c == 0) part_b[(long long)h * nchunks + chunk] = ab;
 }
 
-__global__ void __launch_bounds__(256) bwd_gate_final_kernel(const float* __restrict__ part_w,
-                                                             const float* __restrict__ part_b,
-                                                             float* __restrict__ dw_g, float* __restrict__ db_g,
-                                                             int nchunks, int d) {
-  // G threads a column (256 / G >= d): thread g of column c adds chunks g, g + G, ... into four
-  // interleaved sums (independent loads in flight), the G sums are then added in order -- a fixed
-  // order for a given d, so the result does not depend on scheduling.
-  __shared__ float red_w[256], red_b[256];
-  const int h = blockIdx.x;
-  const int G = d <= 32 ? 8 : d <= 64 ? 4 : d <= 128 ? 2 : 1;
-  const int c = threadIdx.x / G, g = threadIdx.x % G;
-  float aw[4] = {0.f, 0.f, 0.f, 0.f}, ab[4] = {0.f, 0.f, 0.f, 0.f};
-  const float* pw = part_w + (long long)h * nchunks * d;
-  const float* pb = part_b + (long long)h * nchunks;
-  int u = 0;
-#pragma unroll 4
-  for (int k = g; k < nchunks; k += G, u = (u + 1) & 3) {
-    if (c < d) aw[u] += pw[(long long)k * d + c];
-    if (c == 0) ab[u] += pb[k];
-  }
-  red_w[threadIdx.x] = (aw[0] + aw[1]) + (aw[2] + aw[3]);
-  red_b[threadIdx.x] = (ab[0] + ab[1]) + (ab[2] + ab[3]);
-  __syncthreads();
-  if (g == 0 && c < d) {
-    float sw = 0.f, sb = 0.f;
-    for (int i = 0; i < G; ++i) {
-      sw += red_w[threadIdx.x + i];
-      sb += red_b[threadIdx.x + i];
+// Grid (H, ceil(d / 32)), 1024 threads: 32 columns x 32 chunk groups.  Thread (g, c) adds the
+// chunks g, g + 32, ... of column c into four interleaved sums (independent loads in flight), and a
+// fixed tree then adds the 32 group sums; the blocks of column group 0 also add part_b the same way
+// over all 1024 threads.  The order is fixed for a given nchunks: the result does not depend on
+// scheduling.
+__global__ void __launch_bounds__(1024) bwd_gate_final_kernel(const float* __restrict__ part_w,
+                                                              const float* __restrict__ part_b,
+                                                              float* __restrict__ dw_g, float* __restrict__ db_g,
+                                                              int nchunks, int d) {
+  __shared__ float red[32][33];
+  __shared__ float red_b[1024];
+  const int h = blockIdx.x, tx = threadIdx.x & 31, ty = threadIdx.x >> 5;
+  const int c = blockIdx.y * 32 + tx;
+  float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+  if (c < d) {
+    const float* pw = part_w + (long long)h * nchunks * d + c;
+    int k = ty;
+    for (; k + 96 < nchunks; k += 128) {
+      a0 += pw[(long long)k * d];
+      a1 += pw[(long long)(k + 32) * d];
+      a2 += pw[(long long)(k + 64) * d];
+      a3 += pw[(long long)(k + 96) * d];
     }
-    dw_g[(long long)h * d + c] = sw;
-    if (c == 0) db_g[h] = sb;
+    for (; k < nchunks; k += 32) a0 += pw[(long long)k * d];
+  }
+  red[ty][tx] = (a0 + a1) + (a2 + a3);
+  const bool do_b = blockIdx.y == 0;
+  if (do_b) {
+    const float* pb = part_b + (long long)h * nchunks;
+    float b0 = 0.f, b1 = 0.f;
+    int k = threadIdx.x;
+    for (; k + 1024 < nchunks; k += 2048) {
+      b0 += pb[k];
+      b1 += pb[k + 1024];
+    }
+    if (k < nchunks) b0 += pb[k];
+    red_b[threadIdx.x] = b0 + b1;
+  }
+  __syncthreads();
+  for (int st = 16; st > 0; st >>= 1) {
+    if (ty < st) red[ty][tx] += red[ty + st][tx];
+    __syncthreads();
+  }
+  if (ty == 0 && c < d) dw_g[(long long)h * d + c] = red[0][tx];
+  if (do_b) {  // uniform over the block
+    for (int st = 512; st > 0; st >>= 1) {
+      if ((int)threadIdx.x < st) red_b[threadIdx.x] += red_b[threadIdx.x + st];
+      __syncthreads();
+    }
+    if (threadIdx.x == 0) db_g[h] = red_b[0];
   }
 }
 

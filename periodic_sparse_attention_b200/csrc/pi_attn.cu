@@ -653,7 +653,8 @@ pi_attn_status pi_attn_bwd_ex(const void* q, const void* k, const void* v, const
     if (e == cudaSuccess)
       pia::bwd_gate_partial_kernel<bf><<<gg, 256, 0, s>>>((const bf*)q, rs.dz, part_w, part_b, B, H, n, d);
   }
-  if (e == cudaSuccess) pia::bwd_gate_final_kernel<<<H, 256, 0, s>>>(part_w, part_b, dw_g, db_g, (int)nchunks, d);
+  if (e == cudaSuccess) pia::bwd_gate_final_kernel<<<dim3((unsigned)H, (unsigned)((d + 31) / 32)), 1024, 0, s>>>(
+        part_w, part_b, dw_g, db_g, (int)nchunks, d);
   if (e == cudaSuccess) e = cudaGetLastError();
   cudaError_t e2 = workspace ? cudaSuccess : cudaFreeAsync(scratch, s);
   if (e != cudaSuccess) return cuda_fail(e, why);
