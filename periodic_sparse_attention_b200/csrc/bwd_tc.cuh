@@ -9,13 +9,17 @@
 //                       the index rule gives (0 elsewhere), ds = p (dp - D), written in bf16 over
 //                       the S columns already read; the row's dz = (1 - alpha) sum_window ds -
 //                       alpha sum_skip ds (the gate's gradient through the two log-priors)
-//   TMA producer warp   Q and dO tiles once, then K and V tiles into a 2-stage ring
+//   TMA producer warp   Q and dO tiles once, then K and V tiles into a ring of NSTAGE stages
 // lse and D = dO . out of every row come from the forward pass (its epilogue forms D from the
 // fp32 output rows).  The epilogue writes dq = tau dQ + dz w_g (fp32) and the row terms the dk/dv
 // pass and the gate sums read (lse2, log2-priors, dz).
 //
-// TMEM: S at columns 0..63, dP at 64..127, dQ at 128..128+D.  One S/dP pair: the next tile's
-// Q K^T waits for this tile's dS K (it reads dS over the S columns).  Every wait is bounded as in
+// TMEM: NBUF pairs of S (64 columns) and dP (64), then dQ (D columns).  D = 64 (two CTAs an SM):
+// one pair and one softmax warpgroup, the next tile's Q K^T waits for this tile's dS K (it reads
+// dS over the S columns).  D = 128 (one CTA an SM): two pairs and two softmax warpgroups taking
+// the tiles in turn (even tiles pair 0, odd tiles pair 1), the MMA warp issuing tile j + 1's
+// Q K^T before tile j's dS K, so one group's softmax runs while the other's MMAs do; the groups
+// add their rows' dz sums in a fixed order at the end.  Every wait is bounded as in
 // the forward kernel; a wait that gives up sets the error word and the abort flag, and every role
 // leaves, drains its own asynchronous work and the CTA frees its TMEM.
 #pragma once
@@ -25,11 +29,16 @@ namespace pia {
 namespace tcb {
 using tc::BM;
 using tc::BN;
-using tc::NSTAGE;
+// Depth of the ring of streamed tiles (K and V in the dq pass, Q and dO in the dk/dv pass): a
+// stage is held until the tile's last MMA has completed, and the load into it must land before
+// the tile NSTAGE later is needed.
+constexpr int NSTAGE = 4;
 
 template <int D>
 struct BSmem {
-  static constexpr int kCtas = D == 64 ? 2 : 1;         // shared memory: 64 KB (D = 64) or 128 KB
+  static constexpr int kCtas = D == 64 ? 2 : 1;         // shared memory: 97 KB (D = 64) or 194 KB
+  static constexpr int kNbuf = D == 64 ? 1 : 2;         // S/dP pairs in TMEM = softmax warpgroups
+  static constexpr int kThreads = 64 + 128 * kNbuf;
   static constexpr int kTileBytes = BM * D * 2;          // the Q tile, the dO tile
   static constexpr int kKVBytes = BN * D * 2;            // one K or V tile
   static constexpr int kQ = 0;
@@ -37,17 +46,18 @@ struct BSmem {
   static constexpr int kK = kG + kTileBytes;
   static constexpr int kV = kK + NSTAGE * kKVBytes;
   static constexpr int kBar = kV + NSTAGE * kKVBytes;
-  // barriers: qg_full, k_full[NSTAGE], k_empty[NSTAGE], v_full[NSTAGE], v_empty[NSTAGE], s_full,
-  // ds_full, dq_done, drain
-  static constexpr int kNumBars = 1 + 4 * NSTAGE + 4;
+  // barriers: qg_full, k_full[NSTAGE], k_empty[NSTAGE], v_full[NSTAGE], v_empty[NSTAGE],
+  // s_full[kNbuf], ds_full[kNbuf], dq_done[kNbuf], drain
+  static constexpr int kNumBars = 1 + 4 * NSTAGE + 3 * kNbuf + 1;
   static constexpr int kMisc = kBar + kNumBars * 8;      // tmem base (4 B), abort flag (4 B)
   static constexpr int kWg = (kMisc + 8 + 15) / 16 * 16; // w_g[h], D floats
   static constexpr int kDz = kWg + D * 4;                // the rows' dz, then the gate partials (BM floats each)
   static constexpr int kRed = kDz + BM * 4;
-  static constexpr int kTotal = kRed + BM * 4;
+  static constexpr int kComb = kRed + BM * 4;            // warpgroup 1's dz sums (window, skip) per row
+  static constexpr int kTotal = kComb + 2 * BM * 4;
   static constexpr int kAlloc = kTotal + 1024 - 128;
-  static constexpr int kTmemCols = 256;
-  static_assert(2 * BN + D <= kTmemCols && kTmemCols * kCtas <= 512, "TMEM columns");
+  static constexpr int kTmemCols = kNbuf == 1 ? 256 : 512;
+  static_assert(2 * BN * kNbuf + D <= kTmemCols && kTmemCols * kCtas <= 512, "TMEM columns");
   static_assert(kQ % 1024 == 0 && kG % 1024 == 0 && kK % 1024 == 0 && kV % 1024 == 0 && kKVBytes % 1024 == 0,
                 "128-byte-swizzled tiles sit on 1 KB");
   static_assert(kBar % 8 == 0 && kWg % 16 == 0, "mbarriers on 8 bytes, the w_g staging on 16");
@@ -78,7 +88,7 @@ struct BParams {
 // the skip prior).  The residue pass runs first and writes its dq and dz; the window pass then
 // runs with acc set, adds to both, and takes the gate's partial sums over the whole dz.
 template <int D, int RES>
-__global__ void __launch_bounds__(192, BSmem<D>::kCtas) bwd_dq_kernel(const __grid_constant__ CUtensorMap tmq,
+__global__ void __launch_bounds__(BSmem<D>::kThreads, BSmem<D>::kCtas) bwd_dq_kernel(const __grid_constant__ CUtensorMap tmq,
                                                                        const __grid_constant__ CUtensorMap tmg,
                                                                        const __grid_constant__ CUtensorMap tmk,
                                                                        const __grid_constant__ CUtensorMap tmv,
@@ -106,10 +116,11 @@ __global__ void __launch_bounds__(192, BSmem<D>::kCtas) bwd_dq_kernel(const __gr
   auto bar_kempty = [&](int s) { return bar0 + 8u * (1 + NSTAGE + s); };
   auto bar_vfull = [&](int s) { return bar0 + 8u * (1 + 2 * NSTAGE + s); };
   auto bar_vempty = [&](int s) { return bar0 + 8u * (1 + 3 * NSTAGE + s); };
-  const uint32_t bar_sfull = bar0 + 8u * (1 + 4 * NSTAGE);
-  const uint32_t bar_dsfull = bar_sfull + 8;
-  const uint32_t bar_dqdone = bar_sfull + 16;
-  const uint32_t bar_drain = bar_sfull + 24;
+  constexpr int NBUF = L::kNbuf;
+  auto bar_sfull = [&](int b) { return bar0 + 8u * (1 + 4 * NSTAGE + b); };
+  auto bar_dsfull = [&](int b) { return bar0 + 8u * (1 + 4 * NSTAGE + NBUF + b); };
+  auto bar_dqdone = [&](int b) { return bar0 + 8u * (1 + 4 * NSTAGE + 2 * NBUF + b); };
+  const uint32_t bar_drain = bar0 + 8u * (1 + 4 * NSTAGE + 3 * NBUF);
   uint32_t* const tmem_slot = reinterpret_cast<uint32_t*>(sbase + L::kMisc);
   volatile int* const abort_flag = reinterpret_cast<volatile int*>(sbase + L::kMisc + 4);
 
@@ -168,9 +179,11 @@ __global__ void __launch_bounds__(192, BSmem<D>::kCtas) bwd_dq_kernel(const __gr
       mbar_init(bar_vfull(s), 1);
       mbar_init(bar_vempty(s), 1);
     }
-    mbar_init(bar_sfull, 1);
-    mbar_init(bar_dsfull, BM);
-    mbar_init(bar_dqdone, 1);
+    for (int b = 0; b < NBUF; ++b) {
+      mbar_init(bar_sfull(b), 1);
+      mbar_init(bar_dsfull(b), BM);
+      mbar_init(bar_dqdone(b), 1);
+    }
     mbar_init(bar_drain, 1);
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -192,7 +205,8 @@ __global__ void __launch_bounds__(192, BSmem<D>::kCtas) bwd_dq_kernel(const __gr
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const uint32_t tS = tmem, tP = tmem + BN, tQ = tmem + 2 * BN;
+  // pair b: S at b * 128, dP at b * 128 + 64; dQ after the pairs
+  const uint32_t tQ = tmem + 2 * BN * NBUF;
 
   if (warp == 0) {
     // ------------------------------------------------------------------ TMA producer
@@ -228,14 +242,15 @@ __global__ void __launch_bounds__(192, BSmem<D>::kCtas) bwd_dq_kernel(const __gr
       constexpr uint32_t idesc_q = idesc_bf16(BM, D, 1);   // dQ: B (K) N-major
       bool okw = mbar_wait(bar_qg, 0, abort_flag);
       tc_fence_after();
-      int j = 0;
-      for (int t = cur.next(); okw && t >= 0; t = cur.next(), ++j) {
-        const int s = j % NSTAGE;
-        if (!mbar_wait(bar_kfull(s), (j / NSTAGE) & 1, abort_flag)) break;
-        if (!mbar_wait(bar_vfull(s), (j / NSTAGE) & 1, abort_flag)) break;
-        // the dS K of the previous tile read dS over the S columns this Q K^T overwrites
-        if (j > 0 && !mbar_wait(bar_dqdone, (j - 1) & 1, abort_flag)) break;
+      // S = Q K^T, dP = dO V^T of tile j into pair j % NBUF
+      auto issue_s = [&](int j) -> bool {
+        const int s = j % NSTAGE, b = j % NBUF;
+        if (!mbar_wait(bar_kfull(s), (j / NSTAGE) & 1, abort_flag)) return false;
+        if (!mbar_wait(bar_vfull(s), (j / NSTAGE) & 1, abort_flag)) return false;
+        // the dS K of tile j - NBUF read dS over the S columns this Q K^T overwrites
+        if (j >= NBUF && !mbar_wait(bar_dqdone(b), ((j - NBUF) / NBUF) & 1, abort_flag)) return false;
         tc_fence_after();
+        const uint32_t tS = tmem + b * 2 * BN, tP = tS + BN;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t in = (kk & 3) * 32;
@@ -248,19 +263,34 @@ __global__ void __launch_bounds__(192, BSmem<D>::kCtas) bwd_dq_kernel(const __gr
           tc_mma(tP, sw128_desc(sG + (kk >> 2) * (BM * 128) + in, 16, 1024),
                  sw128_desc(sV + s * kKV + (kk >> 2) * (BN * 128) + in, 16, 1024), idesc_s, kk > 0 ? 1u : 0u);
         }
-        tc_commit(bar_sfull);
+        tc_commit(bar_sfull(b));
         tc_commit(bar_vempty(s));  // V was read by dO V^T only
-        if (!mbar_wait(bar_dsfull, j & 1, abort_flag)) break;
+        return true;
+      };
+      // dQ += dS K of tile j: K = BN keys, 16 per instruction; dS packed two per column over S
+      auto issue_dq = [&](int j) -> bool {
+        const int s = j % NSTAGE, b = j % NBUF;
+        if (!mbar_wait(bar_dsfull(b), (j / NBUF) & 1, abort_flag)) return false;
         tc_fence_after();
-        // dQ += dS K : K = BN keys, 16 per instruction; dS packed two per column over S
+        const uint32_t tS = tmem + b * 2 * BN;
 #pragma unroll
         for (int kk = 0; kk < BN / 16; ++kk) {
           const uint32_t acol = 16 * (kk >> 1) + 8 * (kk & 1);
           tc_mma_ts(tQ, tS + acol, sw128_desc(sK + s * kKV + kk * 16 * 128, BN * 128, 1024), idesc_q,
                     (j == 0 && kk == 0) ? 0u : 1u);
         }
-        tc_commit(bar_dqdone);
+        tc_commit(bar_dqdone(b));
         tc_commit(bar_kempty(s));
+        return true;
+      };
+      // one pair: dS K of tile j - 1, then Q K^T of tile j; two pairs: Q K^T of tile j first
+      int j = 0;
+      for (int t = cur.next(); okw; t = cur.next(), ++j) {
+        const bool have = t >= 0;
+        if (NBUF == 1 && j > 0 && !issue_dq(j - 1)) break;
+        if (have && !issue_s(j)) break;
+        if (NBUF == 2 && j > 0 && !issue_dq(j - 1)) break;
+        if (!have) break;
       }
       tc_commit(bar_drain);
       volatile int never = 0;
@@ -268,7 +298,8 @@ __global__ void __launch_bounds__(192, BSmem<D>::kCtas) bwd_dq_kernel(const __gr
     }
     __syncwarp();
   } else {
-    // ------------------------------------------------------------------ softmax warpgroup
+    // ------------------------------------------------------------------ softmax warpgroups
+    const int wg = (warp - 2) >> 2;  // takes the tiles j with j % NBUF == wg, in pair wg
     const int q4 = warp & 3;
     const int r = q4 * 32 + lane;
     const long long qi = q0 + r;                       // row of the view
@@ -287,7 +318,7 @@ __global__ void __launch_bounds__(192, BSmem<D>::kCtas) bwd_dq_kernel(const __gr
     float* const wg_s = reinterpret_cast<float*>(sbase + L::kWg);
     if (threadIdx.x - 64 < D) wg_s[threadIdx.x - 64] = prm.w_g[(long long)h * D + (threadIdx.x - 64)];
     float z = prm.b_g[h];
-    asm volatile("bar.sync 1, 128;" ::: "memory");
+    asm volatile("bar.sync 2, %0;" ::"r"(128 * NBUF) : "memory");
     bool ok = __all_sync(0xffffffffu, mbar_wait(bar_qg, 0, abort_flag));
     {
       float zp[4] = {0.f, 0.f, 0.f, 0.f};
@@ -318,9 +349,11 @@ __global__ void __launch_bounds__(192, BSmem<D>::kCtas) bwd_dq_kernel(const __gr
     const float NEG_INF = -INFINITY;
     float dzw = 0.f, dzs = 0.f;  // sums of ds over window keys and over skip keys
 
+    const uint32_t tS = tmem + wg * 2 * BN, tP = tS + BN;
     int j = 0;
     for (int t = cur.next(); ok && t >= 0; t = cur.next(), ++j) {
-      if (!__all_sync(0xffffffffu, mbar_wait(bar_sfull, j & 1, abort_flag))) {
+      if (j % NBUF != wg) continue;
+      if (!__all_sync(0xffffffffu, mbar_wait(bar_sfull(wg), (j / NBUF) & 1, abort_flag))) {
         ok = false;
         break;
       }
@@ -366,87 +399,103 @@ __global__ void __launch_bounds__(192, BSmem<D>::kCtas) bwd_dq_kernel(const __gr
       }
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(bar_dsfull);
+      mbar_arrive(bar_dsfull(wg));
     }
-    // ---- epilogue: dq = tau dQ + dz w_g, and the row terms
-    if (RES) {  // the band columns were skip keys
-      dzs += dzw;
-      dzw = 0.f;
+    if (NBUF == 2) {  // warpgroup 1's sums to warpgroup 0, added in that order
+      float* const comb = reinterpret_cast<float*>(sbase + L::kComb);
+      if (wg == 1) {
+        comb[r] = dzw;
+        comb[BM + r] = dzs;
+      }
+      asm volatile("bar.sync 3, %0;" ::"r"(128 * NBUF) : "memory");
+      if (wg == 0) {
+        dzw += comb[r];
+        dzs += comb[BM + r];
+      }
     }
-    // this pass's dz goes into its dq; the row's whole dz (with the residue pass's part, whose dq
-    // already holds its own) into the gate's sums
-    const float dz_own = (1.f - alpha) * dzw - alpha * dzs;
-    const float dz = !RES && prm.acc && row_ok ? dz_own + prm.dz[orow] : dz_own;
-    const bool have_q = __all_sync(0xffffffffu, ok && j > 0 && mbar_wait(bar_dqdone, (j - 1) & 1, abort_flag));
-    if (have_q) tc_fence_after();
-    const float tau = prm.scale_log2 / kLog2e;
-    if (have_q || j == 0) {
+    if (wg == 0) {
+      // ---- epilogue: dq = tau dQ + dz w_g, and the row terms
+      if (RES) {  // the band columns were skip keys
+        dzs += dzw;
+        dzw = 0.f;
+      }
+      // this pass's dz goes into its dq; the row's whole dz (with the residue pass's part, whose dq
+      // already holds its own) into the gate's sums
+      const float dz_own = (1.f - alpha) * dzw - alpha * dzs;
+      const float dz = !RES && prm.acc && row_ok ? dz_own + prm.dz[orow] : dz_own;
+      // every MMA done: the drain barrier, committed once after the MMA warp's last issue (a
+      // pair's own barrier could alias: its parity says nothing to a group that skipped phases)
+      const bool have_q = __all_sync(0xffffffffu, ok && j > 0 && mbar_wait(bar_drain, 0, abort_flag));
+      if (have_q) tc_fence_after();
+      const float tau = prm.scale_log2 / kLog2e;
+      if (have_q || j == 0) {
 #pragma unroll 1
-      for (int c = 0; c < D / 32; ++c) {
-        float o[32];
-        if (have_q) {
-          tmem_ld32(tQ + lane_off + c * 32, o);
-        } else {
+        for (int c = 0; c < D / 32; ++c) {
+          float o[32];
+          if (have_q) {
+            tmem_ld32(tQ + lane_off + c * 32, o);
+          } else {
 #pragma unroll
-          for (int e = 0; e < 32; ++e) o[e] = 0.f;
-        }
-        if (row_ok) {
-          float4* dst = reinterpret_cast<float4*>(prm.dq + orow * D + c * 32);
-          const float4* wv = reinterpret_cast<const float4*>(wg_s + c * 32);
+            for (int e = 0; e < 32; ++e) o[e] = 0.f;
+          }
+          if (row_ok) {
+            float4* dst = reinterpret_cast<float4*>(prm.dq + orow * D + c * 32);
+            const float4* wv = reinterpret_cast<const float4*>(wg_s + c * 32);
 #pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            const float4 w = wv[e];
-            float4 v = make_float4(fmaf(tau, o[4 * e], dz_own * w.x), fmaf(tau, o[4 * e + 1], dz_own * w.y),
-                                   fmaf(tau, o[4 * e + 2], dz_own * w.z), fmaf(tau, o[4 * e + 3], dz_own * w.w));
-            if (!RES && prm.acc) {  // add to the residue pass's dq
-              const float4 a = dst[e];
-              v = make_float4(a.x + v.x, a.y + v.y, a.z + v.z, a.w + v.w);
+            for (int e = 0; e < 8; ++e) {
+              const float4 w = wv[e];
+              float4 v = make_float4(fmaf(tau, o[4 * e], dz_own * w.x), fmaf(tau, o[4 * e + 1], dz_own * w.y),
+                                     fmaf(tau, o[4 * e + 2], dz_own * w.z), fmaf(tau, o[4 * e + 3], dz_own * w.w));
+              if (!RES && prm.acc) {  // add to the residue pass's dq
+                const float4 a = dst[e];
+                v = make_float4(a.x + v.x, a.y + v.y, a.z + v.z, a.w + v.w);
+              }
+              dst[e] = v;
             }
-            dst[e] = v;
           }
         }
-      }
-      if (row_ok) {
-        if (!RES) {
-          prm.lse2[orow] = lse2;
-          prm.bl2[orow] = bl2;
-          prm.bp2[orow] = bp2;
+        if (row_ok) {
+          if (!RES) {
+            prm.lse2[orow] = lse2;
+            prm.bl2[orow] = bl2;
+            prm.bp2[orow] = bp2;
+          }
+          prm.dz[orow] = dz;
         }
-        prm.dz[orow] = dz;
       }
-    }
-    // The gate's partial sums over this CTA's rows, in a fixed order: dw_g[c] += sum_r dz_r q_rc
-    // and db_g += sum_r dz_r.  G = BM / D threads a column, each over BM / G rows of the Q tile
-    // (still in shared memory), then the G parts in order.
-    if (!RES) {
-      float* const dz_s = reinterpret_cast<float*>(sbase + L::kDz);
-      float* const red = reinterpret_cast<float*>(sbase + L::kRed);
-      dz_s[r] = (have_q || j == 0) && row_ok ? dz : 0.f;
-      asm volatile("bar.sync 1, 128;" ::: "memory");
-      constexpr int G = BM / D, RPT = BM / G;
-      const int c = r % D, g = r / D;
-      float acc = 0.f;
+      // The gate's partial sums over this CTA's rows, in a fixed order: dw_g[c] += sum_r dz_r q_rc
+      // and db_g += sum_r dz_r.  G = BM / D threads a column, each over BM / G rows of the Q tile
+      // (still in shared memory), then the G parts in order.
+      if (!RES) {
+        float* const dz_s = reinterpret_cast<float*>(sbase + L::kDz);
+        float* const red = reinterpret_cast<float*>(sbase + L::kRed);
+        dz_s[r] = (have_q || j == 0) && row_ok ? dz : 0.f;
+        asm volatile("bar.sync 1, 128;" ::: "memory");
+        constexpr int G = BM / D, RPT = BM / G;
+        const int c = r % D, g = r / D;
+        float acc = 0.f;
 #pragma unroll 4
-      for (int rr = g * RPT; rr < (g + 1) * RPT; ++rr) {
-        const int cc = c & 63;
-        const uint32_t off = (c >> 6) * (BM * 128) + rr * 128 + ((((cc >> 3) ^ (rr & 7))) << 4) + (cc & 7) * 2;
-        const float qv = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(sbase + L::kQ + off));
-        acc = fmaf(dz_s[rr], qv, acc);
-      }
-      red[r] = acc;
-      asm volatile("bar.sync 1, 128;" ::: "memory");
-      const long long chunk = (long long)(bh / prm.H) * gridDim.x + blockIdx.x;
-      const long long nchunks = (long long)(gridDim.y / prm.H) * gridDim.x;
-      if (r < D) {
-        float sw = 0.f;
+        for (int rr = g * RPT; rr < (g + 1) * RPT; ++rr) {
+          const int cc = c & 63;
+          const uint32_t off = (c >> 6) * (BM * 128) + rr * 128 + ((((cc >> 3) ^ (rr & 7))) << 4) + (cc & 7) * 2;
+          const float qv = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(sbase + L::kQ + off));
+          acc = fmaf(dz_s[rr], qv, acc);
+        }
+        red[r] = acc;
+        asm volatile("bar.sync 1, 128;" ::: "memory");
+        const long long chunk = (long long)(bh / prm.H) * gridDim.x + blockIdx.x;
+        const long long nchunks = (long long)(gridDim.y / prm.H) * gridDim.x;
+        if (r < D) {
+          float sw = 0.f;
 #pragma unroll
-        for (int gg = 0; gg < G; ++gg) sw += red[gg * D + r];
-        prm.part_w[((long long)h * nchunks + chunk) * D + r] = sw;
-      }
-      if (r == 0) {
-        float sb = 0.f;
-        for (int rr = 0; rr < BM; ++rr) sb += dz_s[rr];
-        prm.part_b[(long long)h * nchunks + chunk] = sb;
+          for (int gg = 0; gg < G; ++gg) sw += red[gg * D + r];
+          prm.part_w[((long long)h * nchunks + chunk) * D + r] = sw;
+        }
+        if (r == 0) {
+          float sb = 0.f;
+          for (int rr = 0; rr < BM; ++rr) sb += dz_s[rr];
+          prm.part_b[(long long)h * nchunks + chunk] = sb;
+        }
       }
     }
     tc_fence_before();
@@ -468,28 +517,34 @@ __global__ void __launch_bounds__(192, BSmem<D>::kCtas) bwd_dq_kernel(const __gr
 //                       range, and its skip rows, KeyReaders) p = 2^(s tau log2e + prior - lse2)
 //                       and ds = p (dp - D) from the row's terms (staged in shared memory), P^T
 //                       and dS^T in bf16 over the S^T and dP^T columns already read
-//   TMA producer warp   K and V tiles once, then Q and dO row tiles into a 2-stage ring
-// The epilogue writes dk = tau dK, dv = dV (fp32).  TMEM: S^T 0..63, dP^T 64..127, dV and dK
-// after them (256 columns for D = 64, 512 for D = 128).
+//   TMA producer warp   K and V tiles once, then Q and dO row tiles into a ring of NSTAGE stages
+// The epilogue writes dk = tau dK, dv = dV (fp32).  TMEM: NBUF pairs of S^T (64 columns) and dP^T
+// (64), dV and dK after them: D = 64 one pair and one key warpgroup (256 columns, two CTAs an
+// SM); D = 128 two pairs and two key warpgroups taking the row tiles in turn, the MMA warp issuing
+// tile j + 1's S^T, dP^T before tile j's dV, dK MMAs (512 columns, one CTA an SM); in the
+// epilogue warpgroup 0 writes dk and warpgroup 1 dv.
 template <int D>
 struct KSmem {
   static constexpr int kCtas = D == 64 ? 2 : 1;
+  static constexpr int kNbuf = D == 64 ? 1 : 2;          // S^T/dP^T pairs in TMEM = key warpgroups
+  static constexpr int kThreads = 64 + 128 * kNbuf;
   static constexpr int kKeyBytes = BM * D * 2;           // the K tile, the V tile (128 keys)
   static constexpr int kRowBytes = BN * D * 2;           // one Q or dO row tile (64 rows)
   static constexpr int kK = 0;
   static constexpr int kV = kK + kKeyBytes;
   static constexpr int kQ = kV + kKeyBytes;
   static constexpr int kG = kQ + NSTAGE * kRowBytes;
-  static constexpr int kStat = kG + NSTAGE * kRowBytes;  // 2 buffers x 64 rows x (lse2, D, bl2, bp2)
-  static constexpr int kBar = kStat + 2 * BN * 16;
-  // barriers: kv_full, q_full[NSTAGE], q_empty[NSTAGE], g_full[NSTAGE], g_empty[NSTAGE], s_full,
-  // p_full, kv_done, drain
-  static constexpr int kNumBars = 1 + 4 * NSTAGE + 4;
+  // 2 buffers a key warpgroup x 64 rows x (lse2, D, bl2, bp2)
+  static constexpr int kStat = kG + NSTAGE * kRowBytes;
+  static constexpr int kBar = kStat + 2 * kNbuf * BN * 16;
+  // barriers: kv_full, q_full[NSTAGE], q_empty[NSTAGE], g_full[NSTAGE], g_empty[NSTAGE],
+  // s_full[kNbuf], p_full[kNbuf], kv_done[kNbuf], drain
+  static constexpr int kNumBars = 1 + 4 * NSTAGE + 3 * kNbuf + 1;
   static constexpr int kMisc = kBar + kNumBars * 8;
   static constexpr int kTotal = kMisc + 8;
   static constexpr int kAlloc = kTotal + 1024 - 128;
   static constexpr int kTmemCols = D == 64 ? 256 : 512;
-  static_assert(2 * BN + 2 * D <= kTmemCols && kTmemCols * kCtas <= 512, "TMEM columns");
+  static_assert(2 * BN * kNbuf + 2 * D <= kTmemCols && kTmemCols * kCtas <= 512, "TMEM columns");
   static_assert(kK % 1024 == 0 && kV % 1024 == 0 && kQ % 1024 == 0 && kG % 1024 == 0 && kRowBytes % 1024 == 0,
                 "128-byte-swizzled tiles sit on 1 KB");
   static_assert(kStat % 16 == 0 && kBar % 8 == 0, "row terms on 16 bytes, mbarriers on 8");
@@ -513,7 +568,7 @@ struct KParams {
 // are keys u*pi + res of the sequence, read by the rows u + m0 .. u + S of the same class, all with
 // the skip prior) and writes dk, dv; the window pass (S = 0) then adds to them.
 template <int D, int RES>
-__global__ void __launch_bounds__(192, KSmem<D>::kCtas) bwd_dkv_kernel(const __grid_constant__ CUtensorMap tmk,
+__global__ void __launch_bounds__(KSmem<D>::kThreads, KSmem<D>::kCtas) bwd_dkv_kernel(const __grid_constant__ CUtensorMap tmk,
                                                                         const __grid_constant__ CUtensorMap tmv,
                                                                         const __grid_constant__ CUtensorMap tmq,
                                                                         const __grid_constant__ CUtensorMap tmg,
@@ -541,10 +596,11 @@ __global__ void __launch_bounds__(192, KSmem<D>::kCtas) bwd_dkv_kernel(const __g
   auto bar_qempty = [&](int s) { return bar0 + 8u * (1 + NSTAGE + s); };
   auto bar_gfull = [&](int s) { return bar0 + 8u * (1 + 2 * NSTAGE + s); };
   auto bar_gempty = [&](int s) { return bar0 + 8u * (1 + 3 * NSTAGE + s); };
-  const uint32_t bar_sfull = bar0 + 8u * (1 + 4 * NSTAGE);
-  const uint32_t bar_pfull = bar_sfull + 8;
-  const uint32_t bar_kvdone = bar_sfull + 16;
-  const uint32_t bar_drain = bar_sfull + 24;
+  constexpr int NBUF = L::kNbuf;
+  auto bar_sfull = [&](int b) { return bar0 + 8u * (1 + 4 * NSTAGE + b); };
+  auto bar_pfull = [&](int b) { return bar0 + 8u * (1 + 4 * NSTAGE + NBUF + b); };
+  auto bar_kvdone = [&](int b) { return bar0 + 8u * (1 + 4 * NSTAGE + 2 * NBUF + b); };
+  const uint32_t bar_drain = bar0 + 8u * (1 + 4 * NSTAGE + 3 * NBUF);
   uint32_t* const tmem_slot = reinterpret_cast<uint32_t*>(sbase + L::kMisc);
   volatile int* const abort_flag = reinterpret_cast<volatile int*>(sbase + L::kMisc + 4);
 
@@ -601,9 +657,11 @@ __global__ void __launch_bounds__(192, KSmem<D>::kCtas) bwd_dkv_kernel(const __g
       mbar_init(bar_gfull(s), 1);
       mbar_init(bar_gempty(s), 1);
     }
-    mbar_init(bar_sfull, 1);
-    mbar_init(bar_pfull, BM);
-    mbar_init(bar_kvdone, 1);
+    for (int b = 0; b < NBUF; ++b) {
+      mbar_init(bar_sfull(b), 1);
+      mbar_init(bar_pfull(b), BM);
+      mbar_init(bar_kvdone(b), 1);
+    }
     mbar_init(bar_drain, 1);
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -625,7 +683,8 @@ __global__ void __launch_bounds__(192, KSmem<D>::kCtas) bwd_dkv_kernel(const __g
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const uint32_t tS = tmem, tP = tmem + BN, tdV = tmem + 2 * BN, tdK = tmem + 2 * BN + D;
+  // pair b: S^T at b * 128, dP^T at b * 128 + 64; dV, dK after the pairs
+  const uint32_t tdV = tmem + 2 * BN * NBUF, tdK = tdV + D;
 
   if (warp == 0) {
     // ------------------------------------------------------------------ TMA producer
@@ -661,14 +720,15 @@ __global__ void __launch_bounds__(192, KSmem<D>::kCtas) bwd_dkv_kernel(const __g
       constexpr uint32_t idesc_a = idesc_bf16(BM, D, 1);   // dV, dK: B (dO, Q) N-major
       bool okw = mbar_wait(bar_kv, 0, abort_flag);
       tc_fence_after();
-      int jt = 0;
-      for (int t = walk.next(0); okw && t >= 0; t = walk.next(t + 1), ++jt) {
-        const int s = jt % NSTAGE;
-        if (!mbar_wait(bar_qfull(s), (jt / NSTAGE) & 1, abort_flag)) break;
-        if (!mbar_wait(bar_gfull(s), (jt / NSTAGE) & 1, abort_flag)) break;
-        // the dV, dK MMAs of the previous tile read P^T, dS^T over the columns overwritten here
-        if (jt > 0 && !mbar_wait(bar_kvdone, (jt - 1) & 1, abort_flag)) break;
+      // S^T = K Q^T, dP^T = V dO^T of row tile j into pair j % NBUF
+      auto issue_s = [&](int j) -> bool {
+        const int s = j % NSTAGE, b = j % NBUF;
+        if (!mbar_wait(bar_qfull(s), (j / NSTAGE) & 1, abort_flag)) return false;
+        if (!mbar_wait(bar_gfull(s), (j / NSTAGE) & 1, abort_flag)) return false;
+        // the dV, dK MMAs of tile j - NBUF read P^T, dS^T over the columns overwritten here
+        if (j >= NBUF && !mbar_wait(bar_kvdone(b), ((j - NBUF) / NBUF) & 1, abort_flag)) return false;
         tc_fence_after();
+        const uint32_t tS = tmem + b * 2 * BN, tP = tS + BN;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t in = (kk & 3) * 32;
@@ -681,20 +741,35 @@ __global__ void __launch_bounds__(192, KSmem<D>::kCtas) bwd_dkv_kernel(const __g
           tc_mma(tP, sw128_desc(sV + (kk >> 2) * (BM * 128) + in, 16, 1024),
                  sw128_desc(sG + s * kRow + (kk >> 2) * (BN * 128) + in, 16, 1024), idesc_s, kk > 0 ? 1u : 0u);
         }
-        tc_commit(bar_sfull);
-        if (!mbar_wait(bar_pfull, jt & 1, abort_flag)) break;
+        tc_commit(bar_sfull(b));
+        return true;
+      };
+      // dV += P^T dO and dK += dS^T Q of tile j: K = BN rows, 16 per instruction
+      auto issue_kv = [&](int j) -> bool {
+        const int s = j % NSTAGE, b = j % NBUF;
+        if (!mbar_wait(bar_pfull(b), (j / NBUF) & 1, abort_flag)) return false;
         tc_fence_after();
-        // dV += P^T dO and dK += dS^T Q : K = BN rows, 16 per instruction
+        const uint32_t tS = tmem + b * 2 * BN, tP = tS + BN;
 #pragma unroll
         for (int kk = 0; kk < BN / 16; ++kk) {
           const uint32_t acol = 16 * (kk >> 1) + 8 * (kk & 1);
-          const uint32_t acc = (jt == 0 && kk == 0) ? 0u : 1u;
+          const uint32_t acc = (j == 0 && kk == 0) ? 0u : 1u;
           tc_mma_ts(tdV, tS + acol, sw128_desc(sG + s * kRow + kk * 16 * 128, BN * 128, 1024), idesc_a, acc);
           tc_mma_ts(tdK, tP + acol, sw128_desc(sQ + s * kRow + kk * 16 * 128, BN * 128, 1024), idesc_a, acc);
         }
-        tc_commit(bar_kvdone);
+        tc_commit(bar_kvdone(b));
         tc_commit(bar_qempty(s));
         tc_commit(bar_gempty(s));
+        return true;
+      };
+      // one pair: dV, dK of tile j - 1, then S^T of tile j; two pairs: S^T of tile j first
+      int jt = 0;
+      for (int t = walk.next(0); okw; t = walk.next(t + 1), ++jt) {
+        const bool have = t >= 0;
+        if (NBUF == 1 && jt > 0 && !issue_kv(jt - 1)) break;
+        if (have && !issue_s(jt)) break;
+        if (NBUF == 2 && jt > 0 && !issue_kv(jt - 1)) break;
+        if (!have) break;
       }
       tc_commit(bar_drain);
       volatile int never = 0;
@@ -702,7 +777,8 @@ __global__ void __launch_bounds__(192, KSmem<D>::kCtas) bwd_dkv_kernel(const __g
     }
     __syncwarp();
   } else {
-    // ------------------------------------------------------------------ key warpgroup
+    // ------------------------------------------------------------------ key warpgroups
+    const int wg = (warp - 2) >> 2;  // takes the row tiles j with j % NBUF == wg, in pair wg
     const int q4 = warp & 3;
     const int r = q4 * 32 + lane;
     const long long j = j0 + r;  // key of the view
@@ -716,16 +792,18 @@ __global__ void __launch_bounds__(192, KSmem<D>::kCtas) bwd_dkv_kernel(const __g
     KeyReaders kr;
     kr.init(j, prm.pi, RES ? 0 : prm.S, m0, walk.rpi, prm.bidir != 0, prm.n);
     const float NEG_INF = -INFINITY;
-    const int tid = threadIdx.x - 64;  // 0..127
-    float4* const stat = reinterpret_cast<float4*>(sbase + L::kStat);
+    const int tid = (threadIdx.x - 64) & 127;  // within the warpgroup
+    float4* const stat = reinterpret_cast<float4*>(sbase + L::kStat) + wg * 2 * BN;
     const long long rbase = (long long)bh * prm.n;
+    const uint32_t tS = tmem + wg * 2 * BN, tP = tS + BN;
     bool ok = true;
     int jt = 0;
     for (int t = walk.next(0); t >= 0; t = walk.next(t + 1), ++jt) {
+      if (jt % NBUF != wg) continue;
       const long long r0 = (long long)t * BN;
-      // the tile's row terms into this tile's buffer (the other buffer may still be read by a warp
-      // on the previous tile; a warp here has finished that one)
-      float4* const st = stat + (jt & 1) * BN;
+      // the tile's row terms into this tile's buffer of the warpgroup (the other buffer may still
+      // be read by a warp on the group's previous tile; a warp here has finished that one)
+      float4* const st = stat + ((jt / NBUF) & 1) * BN;
       if (tid < BN) {
         const long long i = r0 + tid;  // row of the view
         const long long ri = rbase + (RES ? i * prm.pi + res : i);
@@ -733,9 +811,9 @@ __global__ void __launch_bounds__(192, KSmem<D>::kCtas) bwd_dkv_kernel(const __g
         st[tid] = i < T ? make_float4(prm.lse2[ri], prm.Dr[ri], RES ? prm.bp2[ri] : prm.bl2[ri], prm.bp2[ri])
                         : make_float4(0.f, 0.f, NEG_INF, NEG_INF);
       }
-      asm volatile("bar.sync 1, 128;" ::: "memory");
+      asm volatile("bar.sync %0, 128;" ::"r"(1 + wg) : "memory");
       if (!ok) continue;  // keep taking part in the barrier above while the other warps finish
-      if (!__all_sync(0xffffffffu, mbar_wait(bar_sfull, jt & 1, abort_flag))) {
+      if (!__all_sync(0xffffffffu, mbar_wait(bar_sfull(wg), (jt / NBUF) & 1, abort_flag))) {
         ok = false;
         continue;
       }
@@ -781,40 +859,42 @@ __global__ void __launch_bounds__(192, KSmem<D>::kCtas) bwd_dkv_kernel(const __g
       }
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(bar_pfull);
+      mbar_arrive(bar_pfull(wg));
     }
-    // ---- epilogue: dk = tau dK, dv = dV
-    const bool have = __all_sync(0xffffffffu, ok && jt > 0 && mbar_wait(bar_kvdone, (jt - 1) & 1, abort_flag));
+    // ---- epilogue: dk = tau dK, dv = dV (two warpgroups: dk from group 0, dv from group 1)
+    // every MMA done: the drain barrier, committed once after the MMA warp's last issue (a pair's
+    // own barrier could alias: a group that took none of the pair's last tiles cannot tell its
+    // phases apart by parity)
+    const bool have = __all_sync(0xffffffffu, ok && jt > 0 && mbar_wait(bar_drain, 0, abort_flag));
     if (have) tc_fence_after();
     const float tau = prm.scale_log2 / kLog2e;
-    if (have || jt == 0) {
+    auto write_rows = [&](uint32_t tacc, float* dst, float scale) {
 #pragma unroll 1
       for (int c = 0; c < D / 32; ++c) {
-        float a[32], b[32];
+        float a[32];
         if (have) {
-          tmem_ld32(tdK + lane_off + c * 32, a);
-          tmem_ld32(tdV + lane_off + c * 32, b);
+          tmem_ld32(tacc + lane_off + c * 32, a);
         } else {
 #pragma unroll
-          for (int e = 0; e < 32; ++e) a[e] = b[e] = 0.f;
+          for (int e = 0; e < 32; ++e) a[e] = 0.f;
         }
         if (key_ok) {
-          float4* dkp = reinterpret_cast<float4*>(prm.dk + krow * D + c * 32);
-          float4* dvp = reinterpret_cast<float4*>(prm.dv + krow * D + c * 32);
+          float4* p = reinterpret_cast<float4*>(dst + krow * D + c * 32);
 #pragma unroll
           for (int e = 0; e < 8; ++e) {
-            float4 kv = make_float4(tau * a[4 * e], tau * a[4 * e + 1], tau * a[4 * e + 2], tau * a[4 * e + 3]);
-            float4 vv = make_float4(b[4 * e], b[4 * e + 1], b[4 * e + 2], b[4 * e + 3]);
+            float4 v = make_float4(scale * a[4 * e], scale * a[4 * e + 1], scale * a[4 * e + 2], scale * a[4 * e + 3]);
             if (!RES && prm.acc) {  // add to the residue pass's dk, dv
-              const float4 ka = dkp[e], va = dvp[e];
-              kv = make_float4(ka.x + kv.x, ka.y + kv.y, ka.z + kv.z, ka.w + kv.w);
-              vv = make_float4(va.x + vv.x, va.y + vv.y, va.z + vv.z, va.w + vv.w);
+              const float4 u = p[e];
+              v = make_float4(u.x + v.x, u.y + v.y, u.z + v.z, u.w + v.w);
             }
-            dkp[e] = kv;
-            dvp[e] = vv;
+            p[e] = v;
           }
         }
       }
+    };
+    if (have || jt == 0) {
+      if (NBUF == 1 || wg == 0) write_rows(tdK, prm.dk, tau);
+      if (NBUF == 1 || wg == 1) write_rows(tdV, prm.dv, 1.f);
     }
     tc_fence_before();
   }
@@ -857,7 +937,7 @@ cudaError_t launch_bwd_dkv(const void* q, const void* k, const void* v, const vo
     attr_done = true;
   }
   const dim3 grid(bwd_tiles<RES>(p.n, p.pi), (unsigned)BH);
-  bwd_dkv_kernel<D, RES><<<grid, 192, KSmem<D>::kAlloc, st>>>(mk, mv, mq, mg, p);
+  bwd_dkv_kernel<D, RES><<<grid, KSmem<D>::kThreads, KSmem<D>::kAlloc, st>>>(mk, mv, mq, mg, p);
   *why = "tensor-core dk/dv kernel launch";
   return cudaGetLastError();
 }
@@ -888,7 +968,7 @@ cudaError_t launch_bwd_dq(const void* q, const void* k, const void* v, const voi
     return e;
   }
   const dim3 grid(bwd_tiles<RES>(p.n, p.pi), (unsigned)BH);
-  bwd_dq_kernel<D, RES><<<grid, 192, BSmem<D>::kAlloc, st>>>(mq, mg, mk, mv, p);
+  bwd_dq_kernel<D, RES><<<grid, BSmem<D>::kThreads, BSmem<D>::kAlloc, st>>>(mq, mg, mk, mv, p);
   *why = "tensor-core dq kernel launch";
   return cudaGetLastError();
 }
