@@ -53,8 +53,8 @@ struct BSmem {
   static constexpr int kWg = (kMisc + 8 + 15) / 16 * 16; // w_g[h], D floats
   static constexpr int kDz = kWg + D * 4;                // the rows' dz, then the gate partials (BM floats each)
   static constexpr int kRed = kDz + BM * 4;
-  static constexpr int kComb = kRed + BM * 4;            // warpgroup 1's dz sums (window, skip) per row
-  static constexpr int kTotal = kComb + 2 * BM * 4;
+  static constexpr int kComb = kRed + BM * 4;            // each warpgroup's dz sums (window, skip) per row
+  static constexpr int kTotal = kComb + kNbuf * 2 * BM * 4;
   static constexpr int kAlloc = kTotal + 1024 - 128;
   static constexpr int kTmemCols = kNbuf == 1 ? 256 : 512;
   static_assert(2 * BN * kNbuf + D <= kTmemCols && kTmemCols * kCtas <= 512, "TMEM columns");
@@ -401,20 +401,17 @@ __global__ void __launch_bounds__(BSmem<D>::kThreads, BSmem<D>::kCtas) bwd_dq_ke
       tc_fence_before();
       mbar_arrive(bar_dsfull(wg));
     }
-    if (NBUF == 2) {  // warpgroup 1's sums to warpgroup 0, added in that order
+    if (NBUF == 2) {  // both groups' sums, added in group order by each group
       float* const comb = reinterpret_cast<float*>(sbase + L::kComb);
-      if (wg == 1) {
-        comb[r] = dzw;
-        comb[BM + r] = dzs;
-      }
+      comb[wg * 2 * BM + r] = dzw;
+      comb[wg * 2 * BM + BM + r] = dzs;
       asm volatile("bar.sync 3, %0;" ::"r"(128 * NBUF) : "memory");
-      if (wg == 0) {
-        dzw += comb[r];
-        dzs += comb[BM + r];
-      }
+      dzw = comb[r] + comb[2 * BM + r];
+      dzs = comb[BM + r] + comb[3 * BM + r];
     }
-    if (wg == 0) {
-      // ---- epilogue: dq = tau dQ + dz w_g, and the row terms
+    {
+      // ---- epilogue: dq = tau dQ + dz w_g (each group its share of the columns), and (group 0)
+      // the row terms
       if (RES) {  // the band columns were skip keys
         dzs += dzw;
         dzw = 0.f;
@@ -429,8 +426,18 @@ __global__ void __launch_bounds__(BSmem<D>::kThreads, BSmem<D>::kCtas) bwd_dq_ke
       if (have_q) tc_fence_after();
       const float tau = prm.scale_log2 / kLog2e;
       if (have_q || j == 0) {
+        constexpr int kChunks = D / 32 / NBUF;  // 32-column chunks a group
 #pragma unroll 1
-        for (int c = 0; c < D / 32; ++c) {
+        for (int c = wg * kChunks; c < (wg + 1) * kChunks; ++c) {
+          float4* dst = reinterpret_cast<float4*>(prm.dq + orow * D + c * 32);
+          float4 prev[8];  // the residue pass's dq, loaded before the TMEM read to overlap it
+          if (!RES && prm.acc && row_ok) {
+#pragma unroll
+            for (int e = 0; e < 8; ++e) prev[e] = dst[e];
+          } else {
+#pragma unroll
+            for (int e = 0; e < 8; ++e) prev[e] = make_float4(0.f, 0.f, 0.f, 0.f);
+          }
           float o[32];
           if (have_q) {
             tmem_ld32(tQ + lane_off + c * 32, o);
@@ -439,21 +446,18 @@ __global__ void __launch_bounds__(BSmem<D>::kThreads, BSmem<D>::kCtas) bwd_dq_ke
             for (int e = 0; e < 32; ++e) o[e] = 0.f;
           }
           if (row_ok) {
-            float4* dst = reinterpret_cast<float4*>(prm.dq + orow * D + c * 32);
             const float4* wv = reinterpret_cast<const float4*>(wg_s + c * 32);
 #pragma unroll
             for (int e = 0; e < 8; ++e) {
-              const float4 w = wv[e];
-              float4 v = make_float4(fmaf(tau, o[4 * e], dz_own * w.x), fmaf(tau, o[4 * e + 1], dz_own * w.y),
-                                     fmaf(tau, o[4 * e + 2], dz_own * w.z), fmaf(tau, o[4 * e + 3], dz_own * w.w));
-              if (!RES && prm.acc) {  // add to the residue pass's dq
-                const float4 a = dst[e];
-                v = make_float4(a.x + v.x, a.y + v.y, a.z + v.z, a.w + v.w);
-              }
-              dst[e] = v;
+              const float4 w = wv[e], a = prev[e];
+              dst[e] = make_float4(a.x + fmaf(tau, o[4 * e], dz_own * w.x), a.y + fmaf(tau, o[4 * e + 1], dz_own * w.y),
+                                   a.z + fmaf(tau, o[4 * e + 2], dz_own * w.z),
+                                   a.w + fmaf(tau, o[4 * e + 3], dz_own * w.w));
             }
           }
         }
+      }
+      if (wg == 0 && (have_q || j == 0)) {
         if (row_ok) {
           if (!RES) {
             prm.lse2[orow] = lse2;
@@ -465,8 +469,8 @@ __global__ void __launch_bounds__(BSmem<D>::kThreads, BSmem<D>::kCtas) bwd_dq_ke
       }
       // The gate's partial sums over this CTA's rows, in a fixed order: dw_g[c] += sum_r dz_r q_rc
       // and db_g += sum_r dz_r.  G = BM / D threads a column, each over BM / G rows of the Q tile
-      // (still in shared memory), then the G parts in order.
-      if (!RES) {
+      // (still in shared memory), then the G parts in order.  Group 0 alone.
+      if (!RES && wg == 0) {
         float* const dz_s = reinterpret_cast<float*>(sbase + L::kDz);
         float* const red = reinterpret_cast<float*>(sbase + L::kRed);
         dz_s[r] = (have_q || j == 0) && row_ok ? dz : 0.f;
@@ -796,20 +800,36 @@ __global__ void __launch_bounds__(KSmem<D>::kThreads, KSmem<D>::kCtas) bwd_dkv_k
     float4* const stat = reinterpret_cast<float4*>(sbase + L::kStat) + wg * 2 * BN;
     const long long rbase = (long long)bh * prm.n;
     const uint32_t tS = tmem + wg * 2 * BN, tP = tS + BN;
+    // (lse2, D, the band's prior, the skip prior) of row tid of the tile at r0: RES's band is skip
+    // keys
+    auto row_terms = [&](long long r0) -> float4 {
+      const long long i = r0 + tid;  // row of the view
+      const long long ri = rbase + (RES ? i * prm.pi + res : i);
+      return i < T ? make_float4(prm.lse2[ri], prm.Dr[ri], RES ? prm.bp2[ri] : prm.bl2[ri], prm.bp2[ri])
+                   : make_float4(0.f, 0.f, NEG_INF, NEG_INF);
+    };
+    // the group's next tile after t (the walk's next, or the one after it with two groups)
+    auto next_own = [&](int t) -> int {
+      int u = walk.next(t + 1);
+      if (NBUF == 2 && u >= 0) u = walk.next(u + 1);
+      return u;
+    };
     bool ok = true;
     int jt = 0;
+    float4 pre = make_float4(0.f, 0.f, NEG_INF, NEG_INF);  // the row terms of the group's next tile
+    bool have_pre = false;
     for (int t = walk.next(0); t >= 0; t = walk.next(t + 1), ++jt) {
       if (jt % NBUF != wg) continue;
       const long long r0 = (long long)t * BN;
       // the tile's row terms into this tile's buffer of the warpgroup (the other buffer may still
-      // be read by a warp on the group's previous tile; a warp here has finished that one)
+      // be read by a warp on the group's previous tile; a warp here has finished that one); the
+      // next tile's are loaded now, to land while this tile is processed
       float4* const st = stat + ((jt / NBUF) & 1) * BN;
       if (tid < BN) {
-        const long long i = r0 + tid;  // row of the view
-        const long long ri = rbase + (RES ? i * prm.pi + res : i);
-        // (lse2, D, the band's prior, the skip prior): RES's band is skip keys
-        st[tid] = i < T ? make_float4(prm.lse2[ri], prm.Dr[ri], RES ? prm.bp2[ri] : prm.bl2[ri], prm.bp2[ri])
-                        : make_float4(0.f, 0.f, NEG_INF, NEG_INF);
+        st[tid] = have_pre ? pre : row_terms(r0);
+        const int tn = next_own(t);
+        if (tn >= 0) pre = row_terms((long long)tn * BN);
+        have_pre = true;
       }
       asm volatile("bar.sync %0, 128;" ::"r"(1 + wg) : "memory");
       if (!ok) continue;  // keep taking part in the barrier above while the other warps finish
@@ -871,6 +891,15 @@ __global__ void __launch_bounds__(KSmem<D>::kThreads, KSmem<D>::kCtas) bwd_dkv_k
     auto write_rows = [&](uint32_t tacc, float* dst, float scale) {
 #pragma unroll 1
       for (int c = 0; c < D / 32; ++c) {
+        float4* p = reinterpret_cast<float4*>(dst + krow * D + c * 32);
+        float4 prev[8];  // the residue pass's dk or dv, loaded before the TMEM read to overlap it
+        if (!RES && prm.acc && key_ok) {
+#pragma unroll
+          for (int e = 0; e < 8; ++e) prev[e] = p[e];
+        } else {
+#pragma unroll
+          for (int e = 0; e < 8; ++e) prev[e] = make_float4(0.f, 0.f, 0.f, 0.f);
+        }
         float a[32];
         if (have) {
           tmem_ld32(tacc + lane_off + c * 32, a);
@@ -879,15 +908,11 @@ __global__ void __launch_bounds__(KSmem<D>::kThreads, KSmem<D>::kCtas) bwd_dkv_k
           for (int e = 0; e < 32; ++e) a[e] = 0.f;
         }
         if (key_ok) {
-          float4* p = reinterpret_cast<float4*>(dst + krow * D + c * 32);
 #pragma unroll
           for (int e = 0; e < 8; ++e) {
-            float4 v = make_float4(scale * a[4 * e], scale * a[4 * e + 1], scale * a[4 * e + 2], scale * a[4 * e + 3]);
-            if (!RES && prm.acc) {  // add to the residue pass's dk, dv
-              const float4 u = p[e];
-              v = make_float4(u.x + v.x, u.y + v.y, u.z + v.z, u.w + v.w);
-            }
-            p[e] = v;
+            const float4 u = prev[e];
+            p[e] = make_float4(u.x + scale * a[4 * e], u.y + scale * a[4 * e + 1], u.z + scale * a[4 * e + 2],
+                               u.w + scale * a[4 * e + 3]);
           }
         }
       }
