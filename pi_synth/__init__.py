@@ -171,6 +171,10 @@ WORKLOADS = {
         Workload("bf16_n4k_bidir", "prefill", "bf16", 1, 8, 4096, 64, 128, 64, 4, bg_std=math.sqrt(0.5), bidir=True),
         # the backward (gradients through out) of the bf16_n4k recipe; dO ~ N(0, 1)
         Workload("bf16_n4k_bwd", "backward", "bf16", 1, 8, 4096, 64, 128, 64, 4, bg_std=math.sqrt(0.5)),
+        # the backward of the bf16_n32k recipe: a long context, where the tensor-core backward takes
+        # the split (residue-class) passes
+        Workload("bf16_n32k_bwd", "backward", "bf16", 2, 16, 32768, 128, 256, 256, 8, k_scale_every=256,
+                 k_scale_factor=4.0),
         # the decode step's launch shape (64 x 32 (b, h), one CTA each, k = 1024, S = 31) over a
         # 4096-row cache (pi = 128: skips m = 9..31 lie in the cache): a case small enough for
         # Nsight Compute

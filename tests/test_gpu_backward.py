@@ -146,6 +146,16 @@ def test_backward_split_n4k_geometry_and_determinism():
         assert torch.equal(x, y)
 
 
+def test_backward_split_bf16_n32k_workload_one_sequence():
+    # one (b, h) sequence of the bf16_n32k_bwd workload at its full length, through the split path
+    # the bench's tc path takes there, every element against the oracle
+    w = ps.WORKLOADS["bf16_n32k_bwd"]
+    inp = ps.backward_inputs(w)
+    one = {x: np.ascontiguousarray(inp[x][:1, :1]) for x in ("q", "k", "v", "dO")}
+    one["w_g"], one["b_g"] = inp["w_g"][:1], inp["b_g"][:1]
+    _check(one, "bf16", w.k, w.pi, w.S, False, "bf16_n32k_bwd (0, 0) tc_split", path="tc_split")
+
+
 def test_backward_tensor_core_path_bf16_n4k_workload():
     w = ps.WORKLOADS["bf16_n4k"]
     inp = ps.prefill_inputs(w)
