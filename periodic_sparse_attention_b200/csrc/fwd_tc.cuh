@@ -39,12 +39,14 @@ constexpr int BN = kTileKeys;  // keys per tile (64)
 // Pipeline shape.  Both head sizes run two CTAs per SM and one softmax warpgroup per CTA; TMEM per
 // CTA is 256 columns: S buffers of 64 columns (the next tile's Q.K^T runs while the softmax works
 // on this one; P is written back over the S columns it has read) -- three for D = 64, two for
-// D = 128 -- and O (D columns).  Shared memory: the Q tile (128 rows) and a two-stage ring of
-// 64-row K and V tiles.  The two K stages, and the two V stages, are each one contiguous 128-row
-// region, which the epilogue reuses.
+// D = 128 -- and O (D columns).  Shared memory: the Q tile (128 rows) and a ring of 64-row K and
+// V tiles, four stages at D = 64 (the loads of the tiles after next are in flight while this one
+// is worked on) and two at D = 128 (where two CTAs an SM leave room for no more).  The K stages,
+// and the V stages, are each one contiguous region of at least 128 rows, which the epilogue
+// reuses.
 // (Two warpgroups splitting each S row by columns also fit, at 96 registers a thread, but the
 // per-tile exchange of their row maxima cost more than the halved pass over the row saved.)
-constexpr int NSTAGE = 2;      // K/V ring depth
+template <int D> constexpr int kNstage = D == 64 ? 4 : 2;  // K/V ring depth
 // S buffers in TMEM: the Q.K^T of tile j needs the P.V of tile j - NSB finished (P sits in the
 // buffer it overwrites), so a third buffer gives that P.V a whole softmax pass of slack; it fits
 // the 256 columns of a CTA only next to a 64-column O.
@@ -56,6 +58,7 @@ constexpr float kRescaleThreshold = 8.0f;  // log2 units
 // ---- shared memory plan (offsets from a 1024-byte aligned base) ---------------------------------
 template <int D>
 struct Smem {
+  static constexpr int NSTAGE = kNstage<D>;
   static constexpr int kQBytes = BM * D * 2;             // the Q tile (bf16)
   static constexpr int kKVBytes = BN * D * 2;            // one K or V tile
   static constexpr int kQ = 0;
@@ -65,7 +68,7 @@ struct Smem {
   static constexpr int kTmemCols = 256;                  // S buffers (BN each) + O (D)
   static constexpr int NSB = kNsb<D>;
   static_assert(NSB * BN + D <= kTmemCols && kTmemCols * kCtasPerSm<D> <= 512, "TMEM columns");
-  static_assert(NSTAGE * kKVBytes == kQBytes, "the K and V regions each hold one 128-row tile");
+  static_assert(NSTAGE * kKVBytes >= kQBytes, "the K and V regions each hold one 128-row tile");
   // barriers: q_full, k_full[NSTAGE], k_empty[NSTAGE], v_full[NSTAGE], v_empty[NSTAGE],
   // s_full[NSB], pv_done[NSB], p_full[NSB], drain, skip partials
   static constexpr int kNumBars = 1 + 4 * NSTAGE + 3 * NSB + 2;
@@ -365,6 +368,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm<D>) fwd_tc_kernel(const _
                                                                           Params prm) {
   using L = Smem<D>;
   constexpr int NSB = kNsb<D>;
+  constexpr int NSTAGE = L::NSTAGE;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
