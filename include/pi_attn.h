@@ -40,7 +40,7 @@ extern "C" {
 typedef enum {
     PI_ATTN_OK = 0,
     PI_ATTN_EINVAL = 1,        /* invalid argument: null pointer, size out of range, misalignment */
-    PI_ATTN_EUNSUPPORTED = 2,  /* valid request this build does not implement (e.g. head size) */
+    PI_ATTN_EUNSUPPORTED = 2,  /* valid request the library does not implement (e.g. head size) */
     PI_ATTN_ECUDA = 3,         /* a CUDA runtime call or kernel launch failed */
     PI_ATTN_EDEVICE = 4        /* a kernel reported an error through the device error word */
 } pi_attn_status;

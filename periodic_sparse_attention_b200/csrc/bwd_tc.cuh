@@ -147,16 +147,7 @@ __global__ void __launch_bounds__(BSmem<D>::kThreads, BSmem<D>::kCtas) bwd_dq_ke
   const int m0 = first_skip_m(prm.kwin, prm.pi);
   TileWalk walk;
   if (RES) {  // keys of view row t: t - S .. t - m0
-    walk.i0 = q0;
-    walk.last = (q0 + BM - 1 < T - 1 ? q0 + BM - 1 : T - 1) - m0;
-    walk.band_lo = q0 - prm.S > 0 ? q0 - prm.S : 0;
-    walk.band_hi = walk.last;
-    walk.n = T;
-    walk.pi = 1;
-    walk.S = 0;
-    walk.m0 = 1;
-    walk.bidir = false;
-    walk.rpi = 1.0;
+    walk.init_residue(q0, T, BM, prm.S, m0);
   } else {
     walk.init(q0, prm.n, BM, prm.kwin, prm.pi, prm.S, prm.bidir != 0);
   }
@@ -630,17 +621,7 @@ __global__ void __launch_bounds__(KSmem<D>::kThreads, KSmem<D>::kCtas) bwd_dkv_k
   const int m0 = first_skip_m(prm.kwin, prm.pi);
   ReaderWalk walk;
   if (RES) {  // readers of view key u: rows u + m0 .. u + S
-    walk.j0 = j0;
-    walk.n = T;
-    walk.jl = j0 + BM - 1 < T - 1 ? j0 + BM - 1 : T - 1;
-    walk.w_lo = j0 + m0;
-    walk.w_hi = walk.jl + prm.S < T - 1 ? walk.jl + prm.S : T - 1;
-    if (walk.w_lo > walk.w_hi) walk.w_hi = -1;  // no reader at all
-    walk.pi = 1;
-    walk.S = 0;
-    walk.m0 = 1;
-    walk.bidir = false;
-    walk.rpi = 1.0;
+    walk.init_residue(j0, T, BM, prm.S, m0);
   } else {
     walk.init(j0, prm.n, BM, prm.kwin, prm.pi, prm.S, prm.bidir != 0);
   }

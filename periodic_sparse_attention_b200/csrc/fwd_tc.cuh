@@ -411,16 +411,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm<D>) fwd_tc_kernel(const _
     res = blockIdx.x % prm.pi;
     q0 = (long long)(blockIdx.x / prm.pi) * BM;
     // keys of row t: t - S .. t - m0 (the skips of sequence row t*pi + res)
-    walk.i0 = q0;
-    walk.last = (q0 + BM - 1 < prm.T - 1 ? q0 + BM - 1 : prm.T - 1) - m0;
-    walk.band_lo = q0 - prm.S > 0 ? q0 - prm.S : 0;
-    walk.band_hi = walk.last;
-    walk.n = prm.T;
-    walk.pi = 1;
-    walk.S = 0;
-    walk.m0 = 1;
-    walk.bidir = false;
-    walk.rpi = 1.0;
+    walk.init_residue(q0, prm.T, BM, prm.S, m0);
   } else {
     q0 = (long long)blockIdx.x * BM;
     walk.init(prm.row0 + q0, prm.row0 + prm.n, BM, prm.kwin, prm.pi, MODE == kFused ? prm.S : 0,

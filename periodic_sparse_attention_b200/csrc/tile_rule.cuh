@@ -50,6 +50,20 @@ struct TileWalk {
     bidir = bidir_;
     rpi = 1.0 / (double)pi_;
   }
+  // The residue-class view of the split path: rows q0 .. q0 + rows - 1 of a class of T rows,
+  // row t reading the band of keys t - S .. t - m0 of the same class (its skips, as a dense band)
+  PIA_HD void init_residue(long long q0, long long T, int rows, int S_, int m0_) {
+    i0 = q0;
+    last = (q0 + rows - 1 < T - 1 ? q0 + rows - 1 : T - 1) - m0_;
+    band_lo = q0 - S_ > 0 ? q0 - S_ : 0;
+    band_hi = S_ >= m0_ ? last : -1;  // S < m0: no row has a key
+    n = T;
+    pi = 1;
+    S = 0;
+    m0 = 1;
+    bidir = false;
+    rpi = 1.0;
+  }
   // smallest needed key tile index >= t, or -1 when none is left
   PIA_HD int next(int t) const {
     const long long p = (long long)t * kTileKeys;
@@ -273,6 +287,21 @@ struct ReaderWalk {
     m0 = kwin / pi_ + 1;
     bidir = bidir_;
     rpi = 1.0 / (double)pi_;
+  }
+  // The residue-class view: keys j0 .. j0 + keys - 1 of a class of T rows, key u read (as a skip
+  // key) by the rows u + m0 .. u + S of the same class
+  PIA_HD void init_residue(long long j0_, long long T, int keys, int S_, int m0_) {
+    j0 = j0_;
+    n = T;
+    jl = j0_ + keys - 1 < T - 1 ? j0_ + keys - 1 : T - 1;
+    w_lo = j0_ + m0_;
+    w_hi = jl + S_ < T - 1 ? jl + S_ : T - 1;
+    if (w_lo > w_hi || S_ < m0_) w_hi = -1;  // no reader at all
+    pi = 1;
+    S = 0;
+    m0 = 1;
+    bidir = false;
+    rpi = 1.0;
   }
   // smallest reading row tile index >= t, or -1 when none is left
   PIA_HD int next(int t) const {

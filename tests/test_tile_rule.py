@@ -95,6 +95,21 @@ def test_reader_walk_visits_exactly_the_reading_row_tiles(harness, n, k, pi, S, 
         assert set(tiles[b, : counts[b]].tolist()) == expect[b], (b, sorted(expect[b]), tiles[b, : counts[b]].tolist())
 
 
+def test_residue_view_walks_give_exactly_the_needed_tiles(harness):
+    # the split path's query walk (the dq and residue forward passes) and reader walk (the dk/dv
+    # skip pass) over one residue class, against brute force: T rows a class, blocks of 128
+    harness.residue_walk_mismatches.argtypes = [ctypes.c_longlong, ctypes.c_int, ctypes.c_int, ctypes.c_int]
+    for T, S, m0 in [(1, 1, 1), (4, 3, 1), (64, 30, 3), (128, 8, 2), (256, 40, 9), (3000, 90, 11), (200, 5, 6),
+                     (129, 200, 1), (700, 64, 64)]:
+        assert harness.residue_walk_mismatches(T, S, m0, 128) == 0, (T, S, m0)
+    rng = np.random.default_rng(11)
+    for _ in range(300):
+        T = int(rng.integers(1, 1500))
+        m0 = int(rng.integers(1, 12))
+        S = int(rng.integers(0, 150))
+        assert harness.residue_walk_mismatches(T, S, m0, 128) == 0, (T, S, m0)
+
+
 def test_cursor_matches_walk_on_walks_built_by_field(harness):
     # band-only walks as the residue-class pass builds them (rows t of a residue view read keys
     # t - S .. t - m0: last is shifted down by m0 and may fall below i0 or below zero), and

@@ -3,6 +3,7 @@
 // tile, unmask window columns and skip bits, classify 32-column chunks -- and reports the keys
 // that survive, in the oracle's index-table layout, plus consistency counters.
 #include <cstdint>
+#include <algorithm>
 #include <cstring>
 #include <vector>
 
@@ -174,6 +175,50 @@ extern "C" int key_side_mismatches(int n, int kwin, int pi, int S, int bidir, in
       for (long long i = 0; i < n; ++i)
         if (seen[i] != reads[i * n + j]) ++bad;
     }
+  }
+  return bad;
+}
+
+// The residue-class view's walks, against brute force over one class of T rows: the query walk of
+// the rows [q0, q0 + rows) (row t reads keys t - S .. t - m0, clipped at 0) and the reader walk of
+// the keys [j0, j0 + rows) (key u read by rows u + m0 .. u + S, clipped below T).  Returns the
+// number of tiles produced or missed wrongly, over every block of the class.
+extern "C" int residue_walk_mismatches(long long T, int S, int m0, int rows) {
+  int bad = 0;
+  const long long ntiles = (T + kTileKeys - 1) / kTileKeys;
+  std::vector<char> want(ntiles), got(ntiles);
+  for (long long b0 = 0; b0 < T; b0 += rows) {
+    const long long b1 = b0 + rows < T ? b0 + rows : T;  // block [b0, b1)
+    // query side
+    std::fill(want.begin(), want.end(), 0);
+    std::fill(got.begin(), got.end(), 0);
+    for (long long t = b0; t < b1; ++t)
+      for (long long key = t - S; key <= t - m0; ++key)
+        if (key >= 0) want[key / kTileKeys] = 1;
+    TileWalk w;
+    w.init_residue(b0, T, rows, S, m0);
+    TileCursor c;
+    c.init(w);
+    int steps = 0;
+    for (int t = c.next(); t >= 0 && steps < 100000; t = c.next(), ++steps) {
+      if (t >= ntiles || got[t]) ++bad;
+      else got[t] = 1;
+    }
+    for (long long t = 0; t < ntiles; ++t) bad += want[t] != got[t];
+    // key side
+    std::fill(want.begin(), want.end(), 0);
+    std::fill(got.begin(), got.end(), 0);
+    for (long long u = b0; u < b1; ++u)
+      for (long long r = u + m0; r <= u + S; ++r)
+        if (r < T) want[r / kTileKeys] = 1;
+    ReaderWalk rw;
+    rw.init_residue(b0, T, rows, S, m0);
+    steps = 0;
+    for (int t = rw.next(0); t >= 0 && steps < 100000; t = rw.next(t + 1), ++steps) {
+      if (t >= ntiles || got[t]) ++bad;
+      else got[t] = 1;
+    }
+    for (long long t = 0; t < ntiles; ++t) bad += want[t] != got[t];
   }
   return bad;
 }
