@@ -1,6 +1,8 @@
-// bwd_tc.cuh -- the backward's dq pass on Blackwell tensor cores (tcgen05 + TMEM + TMA), bf16,
-// head size 64 or 128.
+// bwd_tc.cuh -- the backward's dq pass and dk/dv pass on Blackwell tensor cores (tcgen05 + TMEM +
+// TMA), bf16, head size 64 or 128.  Each runs in the sequence view (window and skips in one
+// sweep, or the window alone) or in the residue-class view of the split path (the skips alone).
 //
+// The dq pass:
 // One CTA per (query tile of 128 rows, b, h), walking the key tiles of the forward (the same
 // TileCursor over the same index rule).  Per 64-key tile:
 //   MMA warp            S = Q K^T and dP = dO V^T (fp32 in TMEM), then, once the softmax warps
@@ -19,9 +21,10 @@
 // dS over the S columns).  D = 128 (one CTA an SM): two pairs and two softmax warpgroups taking
 // the tiles in turn (even tiles pair 0, odd tiles pair 1), the MMA warp issuing tile j + 1's
 // Q K^T before tile j's dS K, so one group's softmax runs while the other's MMAs do; the groups
-// add their rows' dz sums in a fixed order at the end.  Every wait is bounded as in
-// the forward kernel; a wait that gives up sets the error word and the abort flag, and every role
-// leaves, drains its own asynchronous work and the CTA frees its TMEM.
+// add their rows' dz sums in a fixed order at the end and share the epilogue's columns.  The
+// epilogues wait on the drain barrier, committed after the MMA warp's last issue.  Every wait is
+// bounded as in the forward kernel; a wait that gives up sets the error word and the abort flag,
+// and every role leaves, drains its own asynchronous work and the CTA frees its TMEM.
 #pragma once
 #include "fwd_tc.cuh"
 

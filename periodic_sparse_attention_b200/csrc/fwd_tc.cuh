@@ -3,12 +3,13 @@
 //
 // Work unit: one CTA per (query tile of 128 rows, b, h).  The keys a tile needs are the union of
 // its window band [i0 - k, i0 + 127] and, for every surviving skip m, the block
-// [i0 - m*pi, i0 + 127 - m*pi]; the CTA walks the 128-key tiles that intersect this union in
+// [i0 - m*pi, i0 + 127 - m*pi]; the CTA walks the 64-key tiles that intersect this union in
 // increasing order ("local sweep" and "periodic gather" of the method's execution schedule, both
 // as tile loads) and evaluates every tile with the tensor cores:
 //
-//   TMA producer warp   Q tile once, then K and V tiles into a 2-stage ring (128B swizzle)
-//   MMA warp            S = Q K^T (128 x 128, fp32 in TMEM), then O += P V (128 x d, fp32 in TMEM)
+//   TMA producer warp   Q tile once, then K and V tiles into a ring (four stages at d = 64, two at
+//                       d = 128; 128B swizzle)
+//   MMA warp            S = Q K^T (128 x 64, fp32 in TMEM), then O += P V (128 x d, fp32 in TMEM)
 //   softmax warpgroup   one thread per query row: reads its S row from TMEM, applies the index
 //                       rule as a mask and the gate as a log-prior (log(alpha) on window keys,
 //                       log(1 - alpha) on skip keys, -inf elsewhere), keeps one running max and
@@ -353,8 +354,8 @@ struct Params {
   // kFused over one shard of a longer sequence: q/out/lse row r is sequence row row0 + r; k/v
   // row r is sequence row kv0 + r (the index rule runs in sequence rows).  0 and 0 otherwise.
   long long row0, kv0;
-  // kFused for the backward: with dout given, the epilogue also writes Dout[row] = dout . out
-  // from the fp32 output row (before its rounding to bf16).  Null otherwise.
+  // For the backward (kFused, kBandMerge): with dout given, the epilogue also writes
+  // Dout[row] = dout . out from the fp32 output row (before its rounding to bf16).  Null otherwise.
   const __nv_bfloat16* dout;
   float* Dout;
 };
