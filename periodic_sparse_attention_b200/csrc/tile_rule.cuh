@@ -32,7 +32,7 @@ PIA_HD long long div_floor(long long a, long long b, double rb) {
 // Walks, in increasing order, the key tiles that hold at least one key of the union of L(i)
 // and P(i) over the query rows [i0, last] of one tile.
 struct TileWalk {
-  // every field has a value before init() (the residue pass sets them one by one)
+  // every field has a value before init() or init_residue()
   long long i0 = 0, last = -1, band_lo = 0, band_hi = -1;  // query rows [i0, last]; window keys [band_lo, band_hi]
   long long n = 0;                       // sequence length (bidirectional: forward keys stop at n - 1)
   int pi = 1, S = 0, m0 = 1;
