@@ -156,6 +156,28 @@ def test_backward_split_bf16_n32k_workload_one_sequence():
     _check(one, "bf16", w.k, w.pi, w.S, False, "bf16_n32k_bwd (0, 0) tc_split", path="tc_split")
 
 
+@pytest.mark.parametrize("workload", ["bf16_n32k_bwd", "bf16_n4k_bwd"])
+def test_backward_full_workload_gradient_sums(workload):
+    # The whole workload in the bench's launch configuration (path tc: the split passes on
+    # bf16_n32k_bwd), every (b, h) and column, against two closed forms of the method: a row's
+    # weights sum to one, so sum_j dv_j = sum_i dO_i, and a row's ds sum to zero, so sum_j dk_j = 0.
+    # The bounds allow the bf16 roundings of P and ds (relative 2^-9 each, summed with random
+    # signs): 4e-3 of the column norm of dO, and 1e-2 of the column norm of dk.
+    w = ps.WORKLOADS[workload]
+    inp = ps.backward_inputs(w)
+    dev = {x: to_dev(inp[x], "bf16") for x in ("q", "k", "v", "dO")}
+    wg, bg = torch.from_numpy(inp["w_g"]).cuda(), torch.from_numpy(inp["b_g"]).cuda()
+    _, dk, dv, dw, db = pia.pi_attn_bwd(dev["q"], dev["k"], dev["v"], wg, bg, dev["dO"], w.k, w.pi, w.S, path="tc")
+    pia.pi_attn_check()
+    assert bool(torch.isfinite(dw).all()) and bool(torch.isfinite(db).all())
+    dO = dev["dO"].double()
+    ev = (dv.double().sum(dim=2) - dO.sum(dim=2)).abs() / dO.norm(dim=2)
+    assert float(ev.max()) <= 4e-3, float(ev.max())
+    dk = dk.double()
+    ek = dk.sum(dim=2).abs() / dk.norm(dim=2).clamp_min(1e-30)
+    assert float(ek.max()) <= 1e-2, float(ek.max())
+
+
 def test_backward_tensor_core_path_bf16_n4k_workload():
     w = ps.WORKLOADS["bf16_n4k"]
     inp = ps.prefill_inputs(w)

@@ -92,3 +92,18 @@ def test_gate_gradient_is_zero_when_one_prior_covers_every_key(bidir):
     # and it does not vanish once skips are present
     _, _, _, dw2, db2 = oracle.bwd(q, k, v, w_g, b_g, G, 6, 5, 4, bidir=bidir)
     assert np.max(np.abs(db2)) > 1e-3
+
+
+@pytest.mark.parametrize("bidir", [False, True])
+@pytest.mark.parametrize("n,kwin,pi,S,d", [(64, 8, 16, 3, 8), (300, 20, 9, 5, 16), (129, 0, 1, 40, 4)])
+def test_key_and_value_gradients_sum_to_their_closed_forms(n, kwin, pi, S, d, bidir):
+    # Each row's weights p_ij sum to one over its keys, so sum_j dv_j = sum_j sum_i p_ij dO_i =
+    # sum_i dO_i; and each row's ds_ij = p_ij (dp_ij - D_i) sums to D_i - D_i = 0 whatever the gate's
+    # priors, so sum_j dk_j = tau sum_i q_i sum_j ds_ij = 0.  Both hold per (b, h) and column; a
+    # dropped key, a weight counted twice or a wrong D breaks them.
+    q, k, v, w_g, b_g, G = _problem(2, 2, n, d, seed=n + S)
+    _, dk, dv, _, _ = oracle.bwd(q, k, v, w_g, b_g, G, kwin, pi, S, bidir=bidir)
+    scale_v = np.linalg.norm(G, axis=2)
+    np.testing.assert_allclose(dv.sum(axis=2), G.sum(axis=2), rtol=0, atol=1e-12 * scale_v.max())
+    scale_k = np.linalg.norm(dk, axis=2)
+    assert np.max(np.abs(dk.sum(axis=2)) / scale_k) < 1e-12
