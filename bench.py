@@ -5,7 +5,8 @@
 
 A step is one call of the operator (the whole hot path: gate, window and skip logits, single
 softmax, P.V, epilogue) over one batch of the workload, inputs resident in HBM.  The default
-workload is bf16_n4k (bf16, B=1 H=8 n=4096 d=64, window 128, period 64, 4 skips); the other
+workload is bf16_n128k, the largest prefill that fits one GPU (bf16, B=1 H=32 n=131072 d=128,
+window 512, period 1024, 16 skips; its inputs and output are 4.3 GB, far above the L2); the other
 workloads of pi_synth.WORKLOADS can be timed with --workload.  The L2 is flushed (a 256 MiB
 write, then a 256 MiB read of another buffer) before every timed step, outside the step's
 events.  Each timed step replays a CUDA graph of one public pi_attn_fwd / pi_attn_decode call
@@ -38,7 +39,7 @@ import numpy as np  # noqa: E402
 
 import pi_synth as ps  # noqa: E402
 
-DEFAULT_WORKLOAD = "bf16_n4k"
+DEFAULT_WORKLOAD = "bf16_n128k"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 L2_FLUSH_BYTES = 256 << 20
 METRICS = {
@@ -122,27 +123,22 @@ def source_hash(files=None) -> str:
 
 
 def profiled_traffic(workload: str):
-    """DRAM bytes of one step (its launches summed) from the committed ncu summaries, if they were
-    taken on the current kernel source: a line
-      bench-traffic: workload=.. bytes_per_step=.. files=a.cuh,b.cuh source_sha=..
-    in profiles/*.md whose files still hash to source_sha.  Otherwise None."""
-    d = os.path.join(ROOT, "profiles")
-    if not os.path.isdir(d):
+    """DRAM bytes of one step (its launches summed) from the committed ncu record
+    profiles/traffic.json, if it was taken on the current kernel source: a record for the workload
+    whose listed files still hash to its source_sha.  Otherwise None."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(path):
         return None
-    for fn in sorted(os.listdir(d)):
-        if not fn.endswith((".md", ".txt")):
+    with open(path) as f:
+        records = json.load(f).get("records", [])
+    for r in records:
+        if r.get("workload") != workload:
             continue
-        with open(os.path.join(d, fn)) as f:
-            for line in f:
-                if line.startswith("bench-traffic:"):
-                    kv = dict(x.split("=", 1) for x in line.split()[1:] if "=" in x)
-                    if kv.get("workload") != workload or "files" not in kv:
-                        continue
-                    try:
-                        if kv.get("source_sha") == source_hash(kv["files"].split(",")):
-                            return int(kv.get("bytes_per_step") or kv["bytes_per_launch"])
-                    except OSError:
-                        continue
+        try:
+            if r.get("source_sha") == source_hash(r["files"]):
+                return int(r["bytes_per_step"])
+        except (OSError, KeyError):
+            continue
     return None
 
 
@@ -215,8 +211,9 @@ class ClockSampler:
 # the oracle on the host (reference arm and cpu_baseline)
 # ------------------------------------------------------------------------------------------------
 
-def oracle_sample(w, budget_s: float, seed: int = 0):
+def oracle_sample(w, budget_s: float, seed: int = 0, inputs=None):
     """Time the fp64 oracle on a bounded sample of workload w's query rows, using all host cores.
+    `inputs`: the workload's host inputs when the caller has them already (prefill).
     Returns (tokens per second, sample description, threads, seconds)."""
     import oracle
     threads = max(1, os.cpu_count() or 1)
@@ -238,7 +235,7 @@ def oracle_sample(w, budget_s: float, seed: int = 0):
         desc = f"{nh} of {w.B * w.H} (b, h) sequences, every row"
         return nh * w.n / w.H / sec, desc, min(threads, nh), sec
     if w.kind == "prefill":
-        inp = ps.prefill_inputs(w, seed)
+        inp = inputs if inputs is not None else ps.prefill_inputs(w, seed)
         total = w.B * w.H * w.n
         rng = np.random.default_rng(seed)
 
@@ -508,7 +505,8 @@ def run_gpu(args):
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        v, desc, threads, sec = oracle_sample(w, args.cpu_budget)
+        v, desc, threads, sec = oracle_sample(w, args.cpu_budget, args.seed,
+                                              inputs=host if w.kind == "prefill" else None)
         cpu = {"value": v, "unit": "tokens/s", "cores": threads, "kind": "oracle", "sample": desc,
                "seconds": round(sec, 3)}
 
@@ -543,11 +541,12 @@ def run_reference(args):
     w = ps.WORKLOADS[args.workload]
     tokens, flops, bytes_ = work(w)
     budget = max(0.2, min(args.cpu_budget, 120.0 / max(1, args.steps + args.warmup)))
+    inputs = ps.prefill_inputs(w, args.seed) if w.kind == "prefill" else None  # generated once, outside the steps
     for _ in range(args.warmup):
-        oracle_sample(w, budget)
+        oracle_sample(w, budget, args.seed, inputs=inputs)
     vals, secs, desc, threads = [], [], "", 0
     for _ in range(args.steps):
-        v, desc, threads, sec = oracle_sample(w, budget)
+        v, desc, threads, sec = oracle_sample(w, budget, args.seed, inputs=inputs)
         vals.append(v)
         secs.append(sec)
     value = statistics.mean(vals)

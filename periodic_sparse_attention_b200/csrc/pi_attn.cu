@@ -173,6 +173,66 @@ static long long bwd_ws_bytes(int B, int H, int n, int d, bool tc) {
   return (base + 15) / 16 * 16 + rows * 2LL * d + rows * 4LL;
 }
 
+// Decode: how many CTAs share one (b, h).  Split only when there are too few (b, h) to fill the
+// GPU (two-warp CTAs, ~14 resident per SM), keeping >= 128 cache rows per split, at most 64.
+int decode_splits(long long bh, int k_win, int S) {
+  const long long rows = (long long)k_win + 1 + S;
+  const long long slots = 14LL * num_sms();
+  if (bh * 2 >= slots) return 1;
+  long long ns = (slots + bh - 1) / bh;
+  const long long max_ns = (rows + 127) / 128;
+  if (ns > max_ns) ns = max_ns;
+  if (ns > 64) ns = 64;
+  return ns < 1 ? 1 : (int)ns;
+}
+
+// Floats of split workspace a decode with these sizes needs (0 without a split).
+size_t decode_part_floats(long long bh, int nsplit, int d) { return nsplit > 1 ? (size_t)bh * nsplit * (d + 2) : 0; }
+
+// The decode kernel (and, with a split, the combine kernel) on a filled DecodeArgs whose `part`
+// points at decode_part_floats(...) floats of workspace when nsplit > 1.
+cudaError_t launch_decode(const pia::DecodeArgs& a, int d, long long bh, cudaStream_t s) {
+  dim3 grid((unsigned)bh, (unsigned)a.nsplit);
+  if (d == 128) pia::decode_bf16_kernel<128><<<grid, 64, 0, s>>>(a);
+  else pia::decode_bf16_kernel<64><<<grid, 64, 0, s>>>(a);
+  cudaError_t e = cudaGetLastError();
+  if (e == cudaSuccess && a.nsplit > 1) {
+    if (d == 128)
+      pia::decode_combine_kernel<128><<<(unsigned)bh, 128, 0, s>>>(a.part, a.nsplit, a.cache_len, a.H, a.n_cache,
+                                                                  a.out, a.lse, a.ring);
+    else
+      pia::decode_combine_kernel<64><<<(unsigned)bh, 64, 0, s>>>(a.part, a.nsplit, a.cache_len, a.H, a.n_cache,
+                                                                a.out, a.lse, a.ring);
+    e = cudaGetLastError();
+  }
+  return e;
+}
+
+// DecodeArgs for a bf16 decode call (no workspace yet).
+pia::DecodeArgs decode_args(const void* q, const void* kcache, const void* vcache, const float* w_g, const float* b_g,
+                            const int* cache_len, void* out, float* lse, int H, int n_cache, int d, int k_win, int pi,
+                            int S, int nsplit, bool ring) {
+  pia::DecodeArgs a;
+  a.q = (const __nv_bfloat16*)q;
+  a.kc = (const __nv_bfloat16*)kcache;
+  a.vc = (const __nv_bfloat16*)vcache;
+  a.w_g = w_g;
+  a.b_g = b_g;
+  a.cache_len = cache_len;
+  a.out = (__nv_bfloat16*)out;
+  a.lse = lse;
+  a.part = nullptr;
+  a.H = H;
+  a.n_cache = n_cache;
+  a.kwin = k_win;
+  a.pi = pi;
+  a.S = S;
+  a.nsplit = nsplit;
+  a.scale_log2 = (float)(1.0 / std::sqrt((double)d)) * pia::kLog2e;
+  a.ring = ring ? 1 : 0;
+  return a;
+}
+
 }  // namespace
 
 extern "C" {
@@ -334,51 +394,14 @@ static pi_attn_status decode_impl(const void* q, const void* kcache, const void*
   if (dtype == PI_ATTN_BF16 && (d == 64 || d == 128)) {
     const long long bh = (long long)B * H;
     if (bh > 0x7fffffffLL) return fail(PI_ATTN_EINVAL, "B * H too large");
-    // Split each (b, h) across CTAs only when there are too few (b, h) to fill the GPU.
-    const long long rows = (long long)k_win + 1 + S;
-    const long long slots = 14LL * num_sms();  // two-warp CTAs resident at once (~14 per SM)
-    int nsplit = 1;
-    if (bh * 2 < slots) {
-      long long ns = (slots + bh - 1) / bh;
-      const long long max_ns = (rows + 127) / 128;  // keep >= 128 rows per split
-      if (ns > max_ns) ns = max_ns;
-      if (ns > 64) ns = 64;
-      nsplit = ns < 1 ? 1 : (int)ns;
-    }
-    pia::DecodeArgs a;
-    a.q = (const __nv_bfloat16*)q;
-    a.kc = (const __nv_bfloat16*)kcache;
-    a.vc = (const __nv_bfloat16*)vcache;
-    a.w_g = w_g;
-    a.b_g = b_g;
-    a.cache_len = cache_len;
-    a.out = (__nv_bfloat16*)out;
-    a.lse = lse;
-    a.part = nullptr;
-    a.H = H;
-    a.n_cache = n_cache;
-    a.kwin = k_win;
-    a.pi = pi;
-    a.S = S;
-    a.nsplit = nsplit;
-    a.scale_log2 = (float)(1.0 / std::sqrt((double)d)) * pia::kLog2e;
-    a.ring = ring ? 1 : 0;
-    if (nsplit > 1) {
-      const size_t bytes = (size_t)bh * nsplit * (d + 2) * sizeof(float);
-      cudaError_t e = cudaMallocAsync((void**)&a.part, bytes, s);
+    pia::DecodeArgs a = decode_args(q, kcache, vcache, w_g, b_g, cache_len, out, lse, H, n_cache, d, k_win, pi, S,
+                                    decode_splits(bh, k_win, S), ring);
+    const size_t part = decode_part_floats(bh, a.nsplit, d);
+    if (part) {
+      cudaError_t e = cudaMallocAsync((void**)&a.part, part * sizeof(float), s);
       if (e != cudaSuccess) return cuda_fail(e, "decode workspace allocation");
     }
-    dim3 grid((unsigned)bh, (unsigned)nsplit);
-    if (d == 128) pia::decode_bf16_kernel<128><<<grid, 64, 0, s>>>(a);
-    else pia::decode_bf16_kernel<64><<<grid, 64, 0, s>>>(a);
-    cudaError_t e = cudaGetLastError();
-    if (e == cudaSuccess && nsplit > 1) {
-      if (d == 128)
-        pia::decode_combine_kernel<128><<<(unsigned)bh, 128, 0, s>>>(a.part, nsplit, cache_len, H, n_cache, a.out, lse, a.ring);
-      else
-        pia::decode_combine_kernel<64><<<(unsigned)bh, 64, 0, s>>>(a.part, nsplit, cache_len, H, n_cache, a.out, lse, a.ring);
-      e = cudaGetLastError();
-    }
+    cudaError_t e = launch_decode(a, d, bh, s);
     if (a.part) {
       cudaError_t e2 = cudaFreeAsync(a.part, s);
       if (e == cudaSuccess) e = e2;
@@ -443,56 +466,19 @@ pi_attn_status pi_attn_decode_noalloc(const void* q, const void* kcache, const v
                 (int)dtype, d);
   const long long bh = (long long)B * H;
   if (bh > 0x7fffffffLL) return fail(PI_ATTN_EINVAL, "B * H too large");
-  // same split rule as pi_attn_decode
-  const long long rows = (long long)k_win + 1 + S;
-  const long long slots = 14LL * num_sms();
-  int nsplit = 1;
-  if (bh * 2 < slots) {
-    long long ns = (slots + bh - 1) / bh;
-    const long long max_ns = (rows + 127) / 128;
-    if (ns > max_ns) ns = max_ns;
-    if (ns > 64) ns = 64;
-    nsplit = ns < 1 ? 1 : (int)ns;
-  }
-  const size_t need = (size_t)bh * nsplit * (d + 2);
-  if (nsplit > 1 && need > kNoAllocScratchFloats)
+  // the same split and the same kernels as pi_attn_decode; only the workspace differs
+  pia::DecodeArgs a = decode_args(q, kcache, vcache, w_g, b_g, cache_len, out, lse, H, n_cache, d, k_win, pi, S,
+                                  decode_splits(bh, k_win, S), false);
+  const size_t need = decode_part_floats(bh, a.nsplit, d);
+  if (need > kNoAllocScratchFloats)
     return fail(PI_ATTN_EINVAL,
                 "pi_attn_decode_noalloc: %lld (b, h) x %d splits need %zu bytes of scratch, above its fixed %zu",
-                bh, nsplit, need * sizeof(float), kNoAllocScratchFloats * sizeof(float));
-  cudaStream_t s = as_stream(stream);
-  pia::DecodeArgs a;
-  a.q = (const __nv_bfloat16*)q;
-  a.kc = (const __nv_bfloat16*)kcache;
-  a.vc = (const __nv_bfloat16*)vcache;
-  a.w_g = w_g;
-  a.b_g = b_g;
-  a.cache_len = cache_len;
-  a.out = (__nv_bfloat16*)out;
-  a.lse = lse;
-  a.part = nullptr;
-  a.ring = 0;
-  a.H = H;
-  a.n_cache = n_cache;
-  a.kwin = k_win;
-  a.pi = pi;
-  a.S = S;
-  a.nsplit = nsplit;
-  a.scale_log2 = (float)(1.0 / std::sqrt((double)d)) * pia::kLog2e;
-  if (nsplit > 1) {
+                bh, a.nsplit, need * sizeof(float), kNoAllocScratchFloats * sizeof(float));
+  if (need) {
     cudaError_t e = noalloc_scratch(&a.part);  // every split writes its whole slot: nothing to clear
     if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(decode scratch)");
   }
-  dim3 grid((unsigned)bh, (unsigned)nsplit);
-  if (d == 128) pia::decode_bf16_kernel<128><<<grid, 64, 0, s>>>(a);
-  else pia::decode_bf16_kernel<64><<<grid, 64, 0, s>>>(a);
-  cudaError_t e = cudaGetLastError();
-  if (e == cudaSuccess && nsplit > 1) {
-    if (d == 128)
-      pia::decode_combine_kernel<128><<<(unsigned)bh, 128, 0, s>>>(a.part, nsplit, cache_len, H, n_cache, a.out, lse, a.ring);
-    else
-      pia::decode_combine_kernel<64><<<(unsigned)bh, 64, 0, s>>>(a.part, nsplit, cache_len, H, n_cache, a.out, lse, a.ring);
-    e = cudaGetLastError();
-  }
+  cudaError_t e = launch_decode(a, d, bh, as_stream(stream));
   return e == cudaSuccess ? ok() : cuda_fail(e, "decode kernel launch");
 }
 

@@ -179,6 +179,9 @@ WORKLOADS = {
         # 4096-row cache (pi = 128: skips m = 9..31 lie in the cache): a case small enough for
         # Nsight Compute
         Workload("decode_bf16_c4k", "decode", "bf16", 64, 32, 4096, 128, 1024, 128, 31),
+        # the bf16_n128k recipe with 4 heads instead of 32: the same per-(b, h) geometry and launch
+        # shape per head (inputs 384 MB, above the L2), small enough for Nsight Compute
+        Workload("bf16_n128k_h4", "prefill", "bf16", 1, 4, 131072, 128, 512, 1024, 16, sampled_rows=512),
     ]
 }
 

@@ -53,6 +53,47 @@ def assert_close(m: dict, dtype: str, what: str = ""):
         assert m["lse_abs"] <= tol["lse_abs"], f"{what}: lse max-abs {m['lse_abs']:.3g} > {tol['lse_abs']} {m}"
 
 
+# Backward tolerances, per gradient: relative L2 error, and max-abs error as a fraction of the
+# gradient's largest magnitude.
+#   simt: fp32 arithmetic against fp64 on the same bits.
+#   tc:   the tensor-core path rounds on purpose -- the forward's P to bf16 (so its out, and the
+#         D = dO . out taken from the fp32 output rows, carry a relative error of order 2^-9 per
+#         weight) and dS to bf16 for dQ += dS K (2^-9 per element); each gradient carries a few
+#         such roundings: 1e-2 (about 5 * 2^-9) for both measures.
+# gate_floor applies only where the true gate gradients are zero (no row of the problem has a skip
+# key, so every row's dz cancels exactly): a row's dz is then the rounding of D times the row's
+# window mass, and the rows summed into dw_g and db_g add such noise with random signs, so the
+# floor is gate_floor * 4 * sqrt(rows summed).
+GRAD_TOL = {
+    "simt": dict(rel_l2=1e-4, max_abs_frac=1e-3, gate_floor=1e-6),
+    "tc": dict(rel_l2=1e-2, max_abs_frac=1e-2, gate_floor=5e-3),
+}
+
+
+def no_skip_anywhere(n: int, k: int, pi: int, S: int) -> bool:
+    """True when no row of a length-n sequence has a skip key (causal or bidirectional rule): the
+    first surviving skip m0 = k // pi + 1 is past S, or m0 * pi reaches past the sequence."""
+    m0 = k // pi + 1
+    return S < m0 or m0 * pi > n - 1
+
+
+def grad_close(name: str, got: np.ndarray, ref: np.ndarray, rows_summed: int, cancels: bool, path: str):
+    """(ok, message) for one gradient of the backward against the oracle's."""
+    tol = GRAD_TOL[path]
+    got = np.asarray(got, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    if not np.all(np.isfinite(got)):
+        return False, f"{name} not finite"
+    mab = float(np.max(np.abs(got - ref))) if got.size else 0.0
+    if name in ("dw_g", "db_g") and cancels:
+        floor = tol["gate_floor"] * 4.0 * math.sqrt(rows_summed)
+        return mab <= floor, f"{name} (true value zero) max-abs {mab:.3g} > floor {floor:.3g}"
+    scale = max(float(np.max(np.abs(ref))) if ref.size else 0.0, 1e-30)
+    rel = float(np.linalg.norm(got - ref) / max(np.linalg.norm(ref), 1e-30))
+    ok = rel <= tol["rel_l2"] and mab <= tol["max_abs_frac"] * scale
+    return ok, f"{name} rel-L2 {rel:.3g} (bound {tol['rel_l2']}), max-abs {mab:.3g} (bound {tol['max_abs_frac'] * scale:.3g})"
+
+
 def sampled_rows(w, count: int, seed: int = 0) -> np.ndarray:
     """`count` flat query rows drawn without replacement, plus for every (b, h) the boundary rows
     i in {0, k-1, k, k+1, pi, m0*pi, S*pi - 1, S*pi, n-1} (m0 = first skip outside the window)."""

@@ -47,9 +47,9 @@ def test_traffic_line_needs_the_current_source(tmp_path, monkeypatch):
     sha = bench.source_hash(files)
     prof = tmp_path / "profiles"
     prof.mkdir()
-    (prof / "x.md").write_text(
-        f"bench-traffic: workload=bf16_n4k bytes_per_launch=123 files={','.join(files)} source_sha={sha}\n"
-        f"bench-traffic: workload=bf16_n32k bytes_per_launch=9 files={','.join(files)} source_sha=stale\n")
+    (prof / "traffic.json").write_text(json.dumps({"records": [
+        {"workload": "bf16_n4k", "bytes_per_step": 123, "files": files, "source_sha": sha},
+        {"workload": "bf16_n32k", "bytes_per_step": 9, "files": files, "source_sha": "stale"}]}))
     real_root = bench.ROOT
     monkeypatch.setattr(bench, "ROOT", str(tmp_path))
     os.makedirs(tmp_path / "periodic_sparse_attention_b200")
@@ -57,6 +57,22 @@ def test_traffic_line_needs_the_current_source(tmp_path, monkeypatch):
                tmp_path / "periodic_sparse_attention_b200" / "csrc")
     assert bench.profiled_traffic("bf16_n4k") == 123
     assert bench.profiled_traffic("bf16_n32k") is None
+    assert bench.profiled_traffic("bf16_n128k") is None
+
+
+def test_default_workload_is_the_largest_single_gpu_prefill():
+    w = ps.WORKLOADS[bench.DEFAULT_WORKLOAD]
+    prefills = [x for x in ps.WORKLOADS.values() if x.kind == "prefill"]
+    assert w.kind == "prefill" and w.B * w.H * w.n == max(x.B * x.H * x.n for x in prefills)
+    assert (w.B, w.H, w.n, w.d, w.k, w.pi, w.S) == (1, 32, 131072, 128, 512, 1024, 16)
+
+
+def test_committed_traffic_records_are_well_formed():
+    with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
+        recs = json.load(f)["records"]
+    for r in recs:
+        assert r["workload"] in ps.WORKLOADS and r["bytes_per_step"] > 0
+        assert os.path.exists(os.path.join(ROOT, "profiles", r["profile"]))
 
 
 def _free_port():
