@@ -76,7 +76,7 @@ def bind(lib):
     lib.oracle_decode.argtypes = [vp, vp, vp, i32, vp, vp, vp, i64, i64, i64, i64, i64, i64, i64, vp, i64, vp, vp, vp,
                                   i32]
     lib.oracle_decode.restype = None
-    lib.oracle_bwd.argtypes = [vp, vp, vp, i32, vp, vp, i64, i64, i64, i64, i64, i64, i64, i32, vp, vp, vp, vp, vp, vp,
+    lib.oracle_bwd.argtypes = [vp, vp, vp, i32, vp, vp, i64, i64, i64, i64, i64, i64, i64, i32, vp, vp, vp, vp, vp, vp, vp,
                                i32]
     lib.oracle_bwd.restype = None
     return lib
@@ -197,9 +197,11 @@ def decode(q, kc, vc, w_g, b_g, kwin: int, pi: int, S: int, lengths=None, bh=Non
     return out, lse, rs
 
 
-def bwd(q, k, v, w_g, b_g, dO, kwin: int, pi: int, S: int, bidir: bool = False, nthreads: int | None = None):
+def bwd(q, k, v, w_g, b_g, dO, kwin: int, pi: int, S: int, bidir: bool = False, nthreads: int | None = None,
+        return_terms: bool = False):
     """Gradients of a scalar loss through out, given dO = dLoss/dout [B, H, n, d].
-    q, k, v as for fwd.  Returns dq, dk, dv [B, H, n, d], dw_g [H, d], db_g [H] (float64)."""
+    q, k, v as for fwd.  Returns dq, dk, dv [B, H, n, d], dw_g [H, d], db_g [H] (float64); with
+    return_terms also terms [B, H, n, 2]: per row dz_i (its term in db_g) and D_i = dO_i . out_i."""
     q = np.ascontiguousarray(q)
     k = np.ascontiguousarray(k)
     v = np.ascontiguousarray(v)
@@ -212,7 +214,10 @@ def bwd(q, k, v, w_g, b_g, dO, kwin: int, pi: int, S: int, bidir: bool = False, 
     dq, dk, dv = (np.zeros((B, H, n, d), dtype=np.float64) for _ in range(3))
     dw = np.zeros((H, d), dtype=np.float64)
     db = np.zeros(H, dtype=np.float64)
+    terms = np.zeros((B, H, n, 2), dtype=np.float64) if return_terms else None
     _lib().oracle_bwd(q.ctypes.data, k.ctypes.data, v.ctypes.data, dt, w_g.ctypes.data, b_g.ctypes.data, B, H, n, d,
                       kwin, pi, S, int(bidir), dO.ctypes.data, dq.ctypes.data, dk.ctypes.data, dv.ctypes.data,
-                      dw.ctypes.data, db.ctypes.data, _threads(nthreads))
+                      dw.ctypes.data, db.ctypes.data, None if terms is None else terms.ctypes.data, _threads(nthreads))
+    if return_terms:
+        return dq, dk, dv, dw, db, terms
     return dq, dk, dv, dw, db

@@ -310,7 +310,7 @@ void oracle_decode(const void* q, const void* kc, const void* vc, int dtype, con
 /* Backward of one (b, h) sequence, every row, in double: accumulates dq [n, d], dk [n, d],
  * dv [n, d] (zeroed by the caller) and dw [d], db [1] of head h.  Rows in increasing order. */
 static void backward_seq(const problem_t* pr, int64_t n, int64_t h, int64_t base, const double* dO, double* dq,
-                         double* dk, double* dv, double* dw, double* db) {
+                         double* dk, double* dv, double* dw, double* db, double* terms) {
     const int64_t d = pr->d;
     const double tau = 1.0 / sqrt((double)d);
     int64_t* L = (int64_t*)malloc(sizeof(int64_t) * (size_t)(2 * pr->kwin + 1));
@@ -370,6 +370,10 @@ static void backward_seq(const problem_t* pr, int64_t n, int64_t h, int64_t base
             dw[c] += dz * qd[c];
         }
         *db += dz;
+        if (terms) {
+            terms[2 * i] = dz;
+            terms[2 * i + 1] = Dsum;
+        }
     }
     free(L);
     free(P);
@@ -384,6 +388,7 @@ typedef struct {
     int64_t n;
     const double* dO;
     double *dq, *dk, *dv, *dw_part, *db_part;  /* dw_part [B*H, d], db_part [B*H] */
+    double* terms;                             /* [B*H, n, 2] or NULL */
     int64_t begin, end;                        /* (b, h) range */
 } bjob_t;
 
@@ -394,17 +399,18 @@ static void* run_backward(void* arg) {
     for (int64_t bh = jb->begin; bh < jb->end; ++bh) {
         const int64_t off = bh * n * d;
         backward_seq(pr, n, bh % pr->H, off, jb->dO + off, jb->dq + off, jb->dk + off, jb->dv + off,
-                     jb->dw_part + bh * d, jb->db_part + bh);
+                     jb->dw_part + bh * d, jb->db_part + bh, jb->terms ? jb->terms + bh * n * 2 : 0);
     }
     return 0;
 }
 
 /* Backward.  q, k, v [B, H, n, d] as for oracle_fwd_rows_ex; dO [B, H, n, d] double.  Outputs, all
  * double and written whole: dq, dk, dv [B, H, n, d], dw_g [H, d], db_g [H] (sums over b and i,
- * added in increasing b).  Threads split the (b, h) sequences. */
+ * added in increasing b); with terms non-NULL also, per row, [B, H, n, 2]: the row's dz_i (its
+ * term in db_g) and D_i = dO_i . out_i.  Threads split the (b, h) sequences. */
 void oracle_bwd(const void* q, const void* k, const void* v, int dtype, const float* w_g, const float* b_g, int64_t B,
                 int64_t H, int64_t n, int64_t d, int64_t kwin, int64_t pi, int64_t S, int bidir, const double* dO,
-                double* dq, double* dk, double* dv, double* dw_g, double* db_g, int nthreads) {
+                double* dq, double* dk, double* dv, double* dw_g, double* db_g, double* terms, int nthreads) {
     problem_t pr = {q, k, v, dtype, w_g, b_g, H, d, kwin, pi, S, bidir};
     const int64_t BH = B * H;
     memset(dq, 0, sizeof(double) * (size_t)(BH * n * d));
@@ -420,7 +426,7 @@ void oracle_bwd(const void* q, const void* k, const void* v, int dtype, const fl
     bjob_t jobs[MAX_THREADS];
     const int64_t chunk = (BH + nthreads - 1) / nthreads;
     for (int t = 0; t < nthreads; ++t) {
-        bjob_t jb = {&pr, n, dO, dq, dk, dv, dw_part, db_part, 0, 0};
+        bjob_t jb = {&pr, n, dO, dq, dk, dv, dw_part, db_part, terms, 0, 0};
         jb.begin = (int64_t)t * chunk < BH ? (int64_t)t * chunk : BH;
         jb.end = jb.begin + chunk < BH ? jb.begin + chunk : BH;
         jobs[t] = jb;

@@ -9,7 +9,7 @@ import pytest
 
 import oracle
 import pi_synth as ps
-from tests.gpu_util import grad_close, no_skip_anywhere
+from tests.gpu_util import gate_scales, grad_close, no_skip_anywhere
 
 NAMES = ("dq", "dk", "dv", "dw_g", "db_g")
 
@@ -21,34 +21,42 @@ def _ref(B, H, n, d, k, pi, S, seed):
     dO = ps.normal((B, H, n, d), seed=seed, stream=6)
     w_g = ps.normal((H, d), seed=seed, stream=4, std=1 / math.sqrt(d), dtype="f32")
     b_g = ps.normal((H,), seed=seed, stream=5, std=0.7, dtype="f32")
-    return oracle.bwd(q, kk, v, w_g, b_g, ps.bf16_bits_to_f32(dO).astype(np.float64), k, pi, S)
+    *ref, terms = oracle.bwd(q, kk, v, w_g, b_g, ps.bf16_bits_to_f32(dO).astype(np.float64), k, pi, S,
+                             return_terms=True)
+    return ref, gate_scales(q, terms)
 
 
 SHAPES = [(1, 2, 512, 64, 32, 16, 8, 3),     # the smoke test's backward
-          (1, 1, 4096, 64, 128, 64, 4, 0)]   # one sequence of bf16_n4k_bwd
+          (1, 1, 4096, 64, 128, 64, 4, 0),   # one sequence of bf16_n4k_bwd
+          (1, 1, 64, 64, 8, 16, 3, 85)]      # the smallest split case of the GPU tests
 
 
-@pytest.fixture(scope="module", params=SHAPES, ids=["smoke", "n4k"])
+@pytest.fixture(scope="module", params=SHAPES, ids=["smoke", "n4k", "split64"])
 def case(request):
     B, H, n, d, k, pi, S, seed = request.param
     assert not no_skip_anywhere(n, k, pi, S)
-    return B * n, _ref(B, H, n, d, k, pi, S, seed)
+    return _ref(B, H, n, d, k, pi, S, seed)
+
+
+def _close(name, g, r, scales):
+    rss_dw, rss_db = scales
+    return grad_close(name, g, r, "tc", rss_dw if name == "dw_g" else rss_db if name == "db_g" else None)
 
 
 def test_exact_and_rounded_gradients_pass(case):
-    rows, ref = case
+    ref, scales = case
     rng = np.random.default_rng(1)
     for name, r in zip(NAMES, ref):
-        assert grad_close(name, r, r, rows, False, "tc")[0]
+        assert _close(name, r, r, scales)[0]
         # a relative perturbation of 2^-9 per element, random signs: a bf16 rounding
         noisy = r * (1 + rng.choice([-1.0, 1.0], size=r.shape) * 2.0 ** -9)
-        ok, msg = grad_close(name, noisy, r, rows, False, "tc")
+        ok, msg = _close(name, noisy, r, scales)
         assert ok, msg
 
 
 @pytest.mark.parametrize("mutant", ["db_g zero", "dw_g half", "db_g sign", "dw_g transposed head", "dq zero row"])
 def test_planted_mistakes_fail(case, mutant):
-    rows, ref = case
+    ref, scales = case
     got = [np.array(r, copy=True) for r in ref]
     if mutant == "db_g zero":
         got[4][:] = 0.0
@@ -62,15 +70,20 @@ def test_planted_mistakes_fail(case, mutant):
         got[0][0, 0, 7] = 0.0
         if not np.any(ref[0][0, 0, 7]):
             pytest.skip("row already zero")
-    bad = [name for name, g, r in zip(NAMES, got, ref) if not grad_close(name, g, r, rows, False, "tc")[0]]
+    bad = [name for name, g, r in zip(NAMES, got, ref) if not _close(name, g, r, scales)[0]]
     assert bad, f"{mutant} passed the check"
 
 
-def test_floor_only_where_the_gate_gradients_vanish():
-    # with no skip anywhere the gate gradients are zero and a floor ~ sqrt(rows) applies; a gate
-    # gradient of the size a problem with skips has is far above it
+def test_no_skip_anywhere():
     assert no_skip_anywhere(128, 16, 32, 0) and no_skip_anywhere(200, 300, 16, 20) and no_skip_anywhere(1, 0, 1, 1)
     assert not no_skip_anywhere(300, 20, 9, 5)
-    zero = np.zeros(4)
-    assert grad_close("db_g", zero + 1e-3, zero, 512, True, "tc")[0]
-    assert not grad_close("db_g", zero + 1.0, zero, 512, True, "tc")[0]
+
+
+def test_zero_gate_gradients_get_a_noise_bound_not_a_free_pass():
+    # S = 0: every row's dz cancels and the true gate gradients are zero; the bound is the rounding
+    # of D_i summed over rows, far below a gate gradient of the size a problem with skips has
+    (ref, scales) = _ref(1, 2, 256, 64, 16, 32, 0, 5)
+    assert np.max(np.abs(ref[4])) < 1e-12
+    rss_dw, rss_db = scales
+    assert grad_close("db_g", ref[4] + 0.5 * 2.0 ** -9 * rss_db, ref[4], "tc", rss_db)[0]
+    assert not grad_close("db_g", ref[4] + 3 * 2.0 ** -9 * rss_db, ref[4], "tc", rss_db)[0]
