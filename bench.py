@@ -14,7 +14,9 @@ events.  Each timed step replays a CUDA graph of one public pi_attn_fwd / pi_att
 
 Multi-GPU (torchrun, one process per GPU): every rank runs its own batch of the same workload
 (weak scaling: (b, h) problems are independent, there is no data exchange); the time is the max
-over ranks and the throughput counts the tokens of all ranks.
+over ranks and the throughput counts the tokens of all ranks.  --shard seq instead splits every
+sequence of the workload across the ranks (strong scaling): a step is one halo exchange of K/V
+rows between the ranks (point-to-point, NCCL) and the shard kernel on each rank.
 
 --impl reference times the fp64 CPU oracle on the host cores on a bounded sample of the same
 workload (the comparison arm).  bench.py is the only product-side file that runs the oracle, and
@@ -534,6 +536,170 @@ def run_gpu(args):
         dist.destroy_process_group()
 
 
+def shard_plan(w, world: int, rank: int):
+    """The sequence-sharded step's bookkeeping for one rank: its rows [s0, s1) of every (b, h), the
+    first key row kv0 it reads (the halo from the ranks before it starts there), and the halo
+    pieces it receives and sends, (src, dst, g0, g1) as shard.halo_plan lists them."""
+    from periodic_sparse_attention_b200 import shard
+    s0, s1 = shard.shard_bounds(w.n, world, rank)
+    kv0 = max(0, s0 - shard.reach(w.k, w.pi, w.S)) if s1 > s0 else s0
+    plan = shard.halo_plan(w.n, world, w.k, w.pi, w.S)
+    recv = [p for p in plan if p[1] == rank]
+    send = [p for p in plan if p[0] == rank]
+    return {"s0": s0, "s1": s1, "kv0": kv0, "recv": recv, "send": send,
+            "halo_rows": sum(g1 - g0 for _, _, g0, g1 in recv)}
+
+
+def run_shard(args):
+    """--shard seq: every rank owns a contiguous block of rows of every (b, h) sequence of the
+    workload (strong scaling: the whole sequence is split across the ranks).  A step is the halo
+    exchange (point-to-point sends of the K/V rows the rank's windows and skips reach back to) and
+    the shard kernel over the halo and the rank's own rows."""
+    import torch
+    import periodic_sparse_attention_b200 as pia
+    from periodic_sparse_attention_b200 import build as pbuild
+    from periodic_sparse_attention_b200 import shard
+
+    rank, world, local = dist_env()
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=device)
+    if rank == 0 or world == 1:
+        pbuild.build()
+    if world > 1:
+        dist.barrier()
+    pia.load()
+    w = ps.WORKLOADS[args.workload]
+    if w.kind != "prefill" or w.bidir or w.dtype != "bf16" or w.d not in (64, 128):
+        raise SystemExit(f"--shard seq covers causal bf16 prefill workloads with d in (64, 128), not {w.name}")
+    plan = shard_plan(w, world, rank)
+    s0, s1, kv0 = plan["s0"], plan["s1"], plan["kv0"]
+    host = ps.prefill_rows(w, s0, s1, args.seed)
+
+    def dev(a):
+        return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).to(device).view(torch.bfloat16)
+
+    t = {x: dev(host[x]) for x in ("q", "k", "v")}
+    t["w_g"] = torch.from_numpy(host["w_g"]).to(device)
+    t["b_g"] = torch.from_numpy(host["b_g"]).to(device)
+    out = torch.empty_like(t["q"])
+    lse = torch.empty((w.B, w.H, s1 - s0), dtype=torch.float32, device=device)
+    stream = torch.cuda.current_stream(device)
+
+    def step():
+        if world > 1:
+            k_ext, v_ext, kv = shard.exchange_halo(t["k"], t["v"], w.n, w.k, w.pi, w.S)
+        else:
+            k_ext, v_ext, kv = t["k"], t["v"], 0
+        pia.pi_attn_fwd_shard(t["q"], k_ext.contiguous(), v_ext.contiguous(), t["w_g"], t["b_g"], w.k, w.pi, w.S, s0,
+                              kv, out=out, lse=lse)
+
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
+    flush_rd = torch.zeros(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=device)
+
+    def flush_l2(i):
+        flush.fill_(i & 0xFF)
+        flush_rd.sum()
+
+    for i in range(args.warmup):
+        flush_l2(i)
+        step()
+    pia.pi_attn_check(stream)
+
+    def timed(n_steps):
+        starts = [torch.cuda.Event(enable_timing=True) for _ in range(n_steps)]
+        ends = [torch.cuda.Event(enable_timing=True) for _ in range(n_steps)]
+        for i in range(n_steps):
+            flush_l2(i)
+            if world > 1:
+                dist.barrier()
+            starts[i].record(stream)
+            step()
+            ends[i].record(stream)
+        torch.cuda.synchronize(device)
+        return [a.elapsed_time(b) for a, b in zip(starts, ends)]
+
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(device)
+    with ClockSampler(local) as clocks:
+        per_step = timed(args.steps)
+    pia.pi_attn_check(stream)
+    total_ms = max_over_ranks(sum(per_step), world, device)
+    ms_per_step = total_ms / args.steps
+    tokens, flops, bytes_ = work(w)
+    value = tokens / (ms_per_step / 1e3)  # the whole sequence's tokens, over all ranks
+
+    # end to end: this rank's input rows from pinned host memory, its output rows back
+    pairs = [(t[x].view(torch.int16), torch.from_numpy(np.ascontiguousarray(host[x]).view(np.int16)).pin_memory())
+             for x in ("q", "k", "v")]
+    backs = [(r, torch.empty(r.shape, dtype=r.dtype).pin_memory()) for r in (out, lse)]
+    h2d = sum(h.numel() * h.element_size() for _, h in pairs)
+    d2h = sum(h.numel() * h.element_size() for _, h in backs)
+
+    def e2e_step():
+        for dst, src in pairs:
+            dst.copy_(src, non_blocking=True)
+        step()
+        for src, dst in backs:
+            dst.copy_(src, non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize(device)
+    e_steps = max(3, min(args.steps, 20))
+    if world > 1:
+        dist.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize(device)
+    e_ms = max_over_ranks(e0.elapsed_time(e1), world, device) / e_steps
+    h2d_all = max_over_ranks(float(h2d), world, device) * world
+    d2h_all = max_over_ranks(float(d2h), world, device) * world
+    pia.pi_attn_check(stream)
+
+    peaks, peak_kind = load_peaks()
+    # one GPU's share of the algorithmic work over the step time, against one GPU's peak
+    per_gpu_flops, per_gpu_bytes = flops / world, bytes_ / world
+    ridge = peaks["bf16_tflops"] * 1e12 / (peaks["hbm_gbs"] * 1e9)
+    sec = ms_per_step / 1e3
+    if flops / bytes_ < ridge:
+        roof = {"bound": "hbm", "achieved": per_gpu_bytes / sec / 1e9, "peak": peaks["hbm_gbs"], "unit": "GB/s"}
+    else:
+        roof = {"bound": "tensor", "achieved": per_gpu_flops / sec / 1e12, "peak": peaks["bf16_tflops"],
+                "unit": "TFLOP/s"}
+    roof["frac"] = roof["achieved"] / roof["peak"]
+    roof["traffic"] = None
+    roof["peak_source"] = f"{peak_kind} ({'MEASURED_PEAKS.json' if peak_kind == 'measured' else 'recipe fallback'})"
+    halo = max_over_ranks(float(plan["halo_rows"]), world, device)
+    line = {
+        "metric": METRICS["prefill"],
+        "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "strong", "vs_baseline": None,
+        "dtype": w.dtype, "data": "synthetic (seeded Philox normals, workload recipe)",
+        "config": dict(w.describe(), l2="flushed before every timed step (256 MiB written, then another 256 MiB read)",
+                       parallelism=f"sequence sharded x{world} (one halo exchange a step)"),
+        "roofline": roof, "cpu_baseline": None,
+        "e2e": {"value": tokens / (e_ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": int(h2d_all),
+                "d2h_bytes_per_step": int(d2h_all), "ms_per_step": e_ms},
+        "gpu_launches": args.steps,  # one shard kernel a step per rank (the exchange is NCCL's)
+        "clocks": clocks.summary(), "path": "shard (single pass over halo + own rows)",
+        "timing": "eager step: halo exchange + shard kernel, CUDA events, max over ranks",
+        "halo_rows_max": int(halo), "kernel_source_sha": source_hash(KERNEL_FILES["prefill"]),
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    del t, flush, flush_rd
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
 def run_reference(args):
     rank, world, _ = dist_env()
     if rank != 0:
@@ -579,10 +745,14 @@ def main(argv=None):
     ap.add_argument("--cpu-budget", type=float, default=10.0, help="seconds of oracle work for cpu_baseline")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--eager", action="store_true", help="time the plain call instead of a graph replay")
+    ap.add_argument("--shard", default="none", choices=["none", "seq"],
+                    help="seq: split every sequence across the ranks (one halo exchange a step) instead of replicas")
     args = ap.parse_args(argv)
     args.warmup = max(3, args.warmup)  # at least 3 untimed warm-up steps
     if args.impl == "reference":
         run_reference(args)
+    elif args.shard == "seq":
+        run_shard(args)
     else:
         run_gpu(args)
 

@@ -201,7 +201,8 @@ def bwd(q, k, v, w_g, b_g, dO, kwin: int, pi: int, S: int, bidir: bool = False, 
         return_terms: bool = False):
     """Gradients of a scalar loss through out, given dO = dLoss/dout [B, H, n, d].
     q, k, v as for fwd.  Returns dq, dk, dv [B, H, n, d], dw_g [H, d], db_g [H] (float64); with
-    return_terms also terms [B, H, n, 2]: per row dz_i (its term in db_g) and D_i = dO_i . out_i."""
+    return_terms also terms [B, H, n, 3]: per row dz_i (its term in db_g), D_i = dO_i . out_i and
+    sum_j p_j^2 (dO_i . v_j)^2."""
     q = np.ascontiguousarray(q)
     k = np.ascontiguousarray(k)
     v = np.ascontiguousarray(v)
@@ -214,7 +215,7 @@ def bwd(q, k, v, w_g, b_g, dO, kwin: int, pi: int, S: int, bidir: bool = False, 
     dq, dk, dv = (np.zeros((B, H, n, d), dtype=np.float64) for _ in range(3))
     dw = np.zeros((H, d), dtype=np.float64)
     db = np.zeros(H, dtype=np.float64)
-    terms = np.zeros((B, H, n, 2), dtype=np.float64) if return_terms else None
+    terms = np.zeros((B, H, n, 3), dtype=np.float64) if return_terms else None
     _lib().oracle_bwd(q.ctypes.data, k.ctypes.data, v.ctypes.data, dt, w_g.ctypes.data, b_g.ctypes.data, B, H, n, d,
                       kwin, pi, S, int(bidir), dO.ctypes.data, dq.ctypes.data, dk.ctypes.data, dv.ctypes.data,
                       dw.ctypes.data, db.ctypes.data, None if terms is None else terms.ctypes.data, _threads(nthreads))

@@ -352,13 +352,14 @@ static void backward_seq(const problem_t* pr, int64_t n, int64_t h, int64_t base
         const double* g = dO + i * d;
         double Dsum = 0.0;
         for (int64_t c = 0; c < d; ++c) Dsum += g[c] * od[c];
-        double dz = 0.0;
+        double dz = 0.0, sig2 = 0.0;
         for (int64_t t = 0; t < nU; ++t) {
             const int64_t j = t < nL ? L[t] : P[t - nL];
             double dpt = 0.0;
             for (int64_t c = 0; c < d; ++c) dpt += g[c] * load_elem(pr->v, base + j * d + c, pr->dtype);
             const double ds = p[t] * (dpt - Dsum);
             dz += t < nL ? (1.0 - alpha) * ds : -alpha * ds;
+            sig2 += p[t] * p[t] * dpt * dpt;
             for (int64_t c = 0; c < d; ++c) {
                 dq[i * d + c] += tau * ds * load_elem(pr->k, base + j * d + c, pr->dtype);
                 dk[j * d + c] += tau * ds * qd[c];
@@ -371,8 +372,9 @@ static void backward_seq(const problem_t* pr, int64_t n, int64_t h, int64_t base
         }
         *db += dz;
         if (terms) {
-            terms[2 * i] = dz;
-            terms[2 * i + 1] = Dsum;
+            terms[3 * i] = dz;
+            terms[3 * i + 1] = Dsum;
+            terms[3 * i + 2] = sig2;
         }
     }
     free(L);
@@ -388,7 +390,7 @@ typedef struct {
     int64_t n;
     const double* dO;
     double *dq, *dk, *dv, *dw_part, *db_part;  /* dw_part [B*H, d], db_part [B*H] */
-    double* terms;                             /* [B*H, n, 2] or NULL */
+    double* terms;                             /* [B*H, n, 3] or NULL */
     int64_t begin, end;                        /* (b, h) range */
 } bjob_t;
 
@@ -399,15 +401,16 @@ static void* run_backward(void* arg) {
     for (int64_t bh = jb->begin; bh < jb->end; ++bh) {
         const int64_t off = bh * n * d;
         backward_seq(pr, n, bh % pr->H, off, jb->dO + off, jb->dq + off, jb->dk + off, jb->dv + off,
-                     jb->dw_part + bh * d, jb->db_part + bh, jb->terms ? jb->terms + bh * n * 2 : 0);
+                     jb->dw_part + bh * d, jb->db_part + bh, jb->terms ? jb->terms + bh * n * 3 : 0);
     }
     return 0;
 }
 
 /* Backward.  q, k, v [B, H, n, d] as for oracle_fwd_rows_ex; dO [B, H, n, d] double.  Outputs, all
  * double and written whole: dq, dk, dv [B, H, n, d], dw_g [H, d], db_g [H] (sums over b and i,
- * added in increasing b); with terms non-NULL also, per row, [B, H, n, 2]: the row's dz_i (its
- * term in db_g) and D_i = dO_i . out_i.  Threads split the (b, h) sequences. */
+ * added in increasing b); with terms non-NULL also, per row, [B, H, n, 3]: the row's dz_i (its
+ * term in db_g), D_i = dO_i . out_i and sum_j p_j^2 (dO_i . v_j)^2 (the spread of the terms D_i is
+ * summed from).  Threads split the (b, h) sequences. */
 void oracle_bwd(const void* q, const void* k, const void* v, int dtype, const float* w_g, const float* b_g, int64_t B,
                 int64_t H, int64_t n, int64_t d, int64_t kwin, int64_t pi, int64_t S, int bidir, const double* dO,
                 double* dq, double* dk, double* dv, double* dw_g, double* db_g, double* terms, int nthreads) {

@@ -208,6 +208,20 @@ def prefill_inputs(w: Workload, seed: int = 0) -> dict:
     return {"q": q, "k": k, "v": v, "w_g": w_g, "b_g": b_g}
 
 
+def prefill_rows(w: Workload, s0: int, s1: int, seed: int = 0) -> dict:
+    """Rows [s0, s1) of every (b, h) sequence of prefill_inputs(w, seed): q, k, v [B, H, s1 - s0, d]
+    holding the identical values (each row regenerated alone), and the full w_g, b_g."""
+    s0, s1 = max(0, int(s0)), min(w.n, int(s1))
+    shp = (w.B, w.H, w.n, w.d)
+    rows_ = (np.arange(w.B * w.H, dtype=np.int64)[:, None] * w.n + np.arange(s0, s1, dtype=np.int64)[None, :]).reshape(-1)
+    out = {}
+    for name, stream in (("q", STREAM_Q), ("k", STREAM_K), ("v", STREAM_V)):
+        extra = dict(scale_every=w.k_scale_every, scale_factor=w.k_scale_factor) if name == "k" else {}
+        out[name] = rows(shp, rows_, seed=seed, stream=stream, dtype=w.dtype, **extra).reshape(w.B, w.H, s1 - s0, w.d)
+    out["w_g"], out["b_g"] = gate_params(w, seed)
+    return out
+
+
 def backward_inputs(w: Workload, seed: int = 0) -> dict:
     """prefill_inputs plus dO [B, H, n, d] ~ N(0, 1) in the storage dtype (the loss gradient)."""
     inp = prefill_inputs(w, seed)

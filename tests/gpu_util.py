@@ -60,16 +60,21 @@ def assert_close(m: dict, dtype: str, what: str = ""):
 #         D = dO . out taken from the fp32 output rows, carry a relative error of order 2^-9 per
 #         weight) and dS to bf16 for dQ += dS K (2^-9 per element); each gradient carries a few
 #         such roundings: 1e-2 (about 5 * 2^-9) for both measures.
-# dw_g and db_g are sums over every row of dz_i q_i and dz_i.  A row's dz_i carries a rounding of
-# the size of the unit roundoff (2^-9 for the tensor-core path's bf16 P and dS, fp32's for the simt
-# path) times |dz_i| and times |D_i| (dz_i takes D_i as an input, and when every key of the row
-# carries one prior dz_i is exactly zero while D_i's rounding still shows); summed with random
-# signs, the error of a gate gradient is of the order of gate_tol times the root-sum-square of
-# those per-row scales, (|dz_i| + |D_i|) |q_ic| for dw_g[h, c] and (|dz_i| + |D_i|) for db_g[h].
+# dw_g and db_g are sums over every row of dz_i q_i and dz_i, and a row's dz_i carries roundings:
+#   - of D_i = dO_i . out_i, which the tensor-core path takes from an output computed with P rounded
+#     to bf16: D_i - sum_j p_j dO_i . v_j = sum_j (p~_j - p_j) dO_i . v_j, each |p~_j - p_j| within
+#     2^-9 p_j with an independent sign, so its spread is 2^-9 sqrt(sum_j p_j^2 (dO_i . v_j)^2); dz_i
+#     takes it times (1 - alpha_i - sum_P p_j), and when every key of the row carries one prior the
+#     true dz_i is exactly zero while this rounding remains;
+#   - of dz_i's own sum, of the order of the unit roundoff times |dz_i|.
+# Summed over rows with independent signs, a gate gradient's error has a spread of the unit
+# roundoff times the root-sum-square of the rows' scales, sqrt(sum_j p_j^2 (dO_i . v_j)^2 + dz_i^2)
+# (times |q_ic| for dw_g[h, c]).  gate_tol is 3 unit roundoffs (about 5 standard deviations of a
+# uniform rounding) for the tensor-core path; the simt path, fp32 throughout, is held to 2^-16.
 # This one rule also covers the problems whose true gate gradients are zero (no row has a skip).
 GRAD_TOL = {
     "simt": dict(rel_l2=1e-4, max_abs_frac=1e-3, gate_tol=2.0 ** -16),
-    "tc": dict(rel_l2=1e-2, max_abs_frac=1e-2, gate_tol=2.0 ** -9),
+    "tc": dict(rel_l2=1e-2, max_abs_frac=1e-2, gate_tol=3 * 2.0 ** -9),
 }
 
 
@@ -83,11 +88,11 @@ def no_skip_anywhere(n: int, k: int, pi: int, S: int) -> bool:
 def gate_scales(q_bits: np.ndarray, terms: np.ndarray):
     """Root-sum-square scales of the gate gradients' rounding: (for dw_g [H, d], for db_g [H]).
     q_bits: q [B, H, n, d] as stored (bf16 bits or fp32); terms: oracle.bwd(..., return_terms=True)'s
-    per-row (dz_i, D_i) [B, H, n, 2]."""
+    per-row (dz_i, D_i, sum_j p_j^2 (dO_i . v_j)^2) [B, H, n, 3]."""
     q = ps.bf16_bits_to_f32(q_bits).astype(np.float64) if q_bits.dtype == np.uint16 else q_bits.astype(np.float64)
-    s = np.abs(terms[..., 0]) + np.abs(terms[..., 1])                     # [B, H, n]
-    rss_dw = np.sqrt(np.einsum("bhn,bhnc->hc", s * s, q * q))
-    rss_db = np.sqrt((s * s).sum(axis=(0, 2)))
+    s2 = terms[..., 2] + terms[..., 0] ** 2                                # [B, H, n]
+    rss_dw = np.sqrt(np.einsum("bhn,bhnc->hc", s2, q * q))
+    rss_db = np.sqrt(s2.sum(axis=(0, 2)))
     return rss_dw, rss_db
 
 

@@ -113,3 +113,39 @@ def test_reference_arm_prints_one_line():
     d = json.loads(lines[0])
     assert d["impl"] == "reference" and d["value"] > 0 and d["cpu_baseline"]["cores"] >= 1
     assert d["e2e"]["h2d_bytes_per_step"] == 0
+
+
+def _shard_rank_main(rank, world, port, out_dir):
+    import dataclasses
+
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+
+    from periodic_sparse_attention_b200 import shard
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank), WORLD_SIZE=str(world))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    # the bf16_n128k recipe's index rule on a short sequence: the halo spans several periods
+    w = dataclasses.replace(ps.WORKLOADS["bf16_n128k"], name="n128k_short", H=2, n=6000, k=100, pi=64, S=16)
+    plan = bench.shard_plan(w, world, rank)
+    host = ps.prefill_rows(w, plan["s0"], plan["s1"], 0)
+    k_loc = torch.from_numpy(host["k"].view(np.int16))
+    v_loc = torch.from_numpy(host["v"].view(np.int16))
+    k_ext, v_ext, kv0 = shard.exchange_halo(k_loc, v_loc, w.n, w.k, w.pi, w.S)
+    full = ps.prefill_inputs(w, 0)
+    ok = (kv0 == plan["kv0"] and k_ext.shape[2] == plan["s1"] - kv0 and plan["halo_rows"] == plan["s0"] - kv0
+          and np.array_equal(k_ext.numpy().view(np.uint16), full["k"][:, :, kv0:plan["s1"]])
+          and np.array_equal(v_ext.numpy().view(np.uint16), full["v"][:, :, kv0:plan["s1"]]))
+    with open(os.path.join(out_dir, f"s{rank}.json"), "w") as f:
+        json.dump({"ok": bool(ok), "plan": {k: v for k, v in plan.items() if k in ("s0", "s1", "kv0", "halo_rows")}}, f)
+    dist.barrier()
+    dist.destroy_process_group()
+
+
+def test_shard_step_plan_and_halo_two_gloo_ranks(tmp_path):
+    port = _free_port()
+    mp.start_processes(_shard_rank_main, args=(2, port, str(tmp_path)), nprocs=2, start_method="spawn")
+    res = [json.load(open(tmp_path / f"s{i}.json")) for i in range(2)]
+    assert all(r["ok"] for r in res), res
+    assert res[0]["plan"] == {"s0": 0, "s1": 3000, "kv0": 0, "halo_rows": 0}
+    assert res[1]["plan"] == {"s0": 3000, "s1": 6000, "kv0": 3000 - 16 * 64, "halo_rows": 16 * 64}

@@ -142,6 +142,8 @@ EDGE = [  # B, H, n, d, k, pi, S
     (1, 1, 4096, 128, 300, 256, 12),  # first surviving skip m = 2
     (1, 1, 2112, 64, 10, 64, 40),   # 33 rows per residue, skips reach the start
     (1, 2, 100, 64, 8, 200, 3),     # period longer than the sequence: no skip exists
+    (1, 1, 2100, 128, 513, 300, 7),  # window not a multiple of a key tile; last 256-row block ragged
+    (3, 5, 768, 128, 1000, 128, 9),  # window longer than the sequence: the skips of m >= 8 lie before it
 ]
 
 

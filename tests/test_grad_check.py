@@ -27,11 +27,10 @@ def _ref(B, H, n, d, k, pi, S, seed):
 
 
 SHAPES = [(1, 2, 512, 64, 32, 16, 8, 3),     # the smoke test's backward
-          (1, 1, 4096, 64, 128, 64, 4, 0),   # one sequence of bf16_n4k_bwd
-          (1, 1, 64, 64, 8, 16, 3, 85)]      # the smallest split case of the GPU tests
+          (1, 1, 4096, 64, 128, 64, 4, 0)]   # one sequence of bf16_n4k_bwd
 
 
-@pytest.fixture(scope="module", params=SHAPES, ids=["smoke", "n4k", "split64"])
+@pytest.fixture(scope="module", params=SHAPES, ids=["smoke", "n4k"])
 def case(request):
     B, H, n, d, k, pi, S, seed = request.param
     assert not no_skip_anywhere(n, k, pi, S)
@@ -85,5 +84,6 @@ def test_zero_gate_gradients_get_a_noise_bound_not_a_free_pass():
     (ref, scales) = _ref(1, 2, 256, 64, 16, 32, 0, 5)
     assert np.max(np.abs(ref[4])) < 1e-12
     rss_dw, rss_db = scales
-    assert grad_close("db_g", ref[4] + 0.5 * 2.0 ** -9 * rss_db, ref[4], "tc", rss_db)[0]
-    assert not grad_close("db_g", ref[4] + 3 * 2.0 ** -9 * rss_db, ref[4], "tc", rss_db)[0]
+    assert grad_close("db_g", ref[4] + 2 * 2.0 ** -9 * rss_db, ref[4], "tc", rss_db)[0]
+    assert not grad_close("db_g", ref[4] + 4 * 2.0 ** -9 * rss_db, ref[4], "tc", rss_db)[0]
+

@@ -1,5 +1,6 @@
 """The seeded input generator (CPU only)."""
 import numpy as np
+import pytest
 
 import pi_synth as ps
 
@@ -61,3 +62,15 @@ def test_decode_storage_plan_covers_window_and_skips():
     pos = ps.decode_positions(65536, 1024, 2048, 31)
     assert pos.size == 1025 + 31
     assert pos.max() == 65535 and pos.min() == 65535 - 31 * 2048
+
+
+@pytest.mark.parametrize("s0,s1", [(0, 4096), (1000, 2300), (4000, 4096), (17, 18)])
+def test_prefill_rows_are_slices_of_the_full_inputs(s0, s1):
+    # the sequence-sharded bench generates only its own rows; they must be the same values
+    import dataclasses
+    w = dataclasses.replace(ps.WORKLOADS["bf16_n32k"], name="n32k_small", H=2, n=4096)
+    full = ps.prefill_inputs(w, 3)
+    part = ps.prefill_rows(w, s0, s1, 3)
+    for name in ("q", "k", "v"):
+        assert np.array_equal(full[name][:, :, s0:s1], part[name]), name
+    assert np.array_equal(full["w_g"], part["w_g"]) and np.array_equal(full["b_g"], part["b_g"])
