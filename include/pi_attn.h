@@ -54,9 +54,11 @@ typedef enum {
     PI_ATTN_PATH_TC = 2,        /* tcgen05/TMEM kernels only (single pass or split, chosen by shape);
                                    PI_ATTN_EUNSUPPORTED where they do not apply */
     PI_ATTN_PATH_TC_FUSED = 3,  /* tensor cores, window and skips in one pass */
-    PI_ATTN_PATH_TC_SPLIT = 4   /* tensor cores, skips in a residue-class pass (scratch of
-                                   B*H*n*(2d + 4) bytes from cudaMallocAsync on `stream`), then the
-                                   window pass merging them; needs n % pi == 0 */
+    PI_ATTN_PATH_TC_SPLIT = 4   /* tensor cores, skips in a residue-class pass over the whole periods,
+                                   rows [0, (n / pi) pi) (scratch of B*H*n*(2d + 4) bytes from
+                                   cudaMallocAsync on `stream`), then the window pass merging them;
+                                   query tiles reaching past the whole periods take the single pass.
+                                   Causal; needs n >= pi and a skip outside the window */
 } pi_attn_path;
 
 /* Prefill forward.  Cited passage: the Core Components (window, skips, gate as log-prior, one
@@ -122,7 +124,9 @@ pi_attn_status pi_attn_fwd_bidir(const void* q, const void* k, const void* v, co
                                  pi_attn_dtype dtype, pi_attn_path path, void* stream);
 
 /* What a pi_attn_fwd_ex call with these arguments would launch, without launching anything:
- * *launches = number of kernel launches (1 for a single pass, 2 for the split), *scratch_bytes =
+ * *launches = number of kernel launches (1 for a single pass; 2 or 3 for the split: the residue pass,
+ * then the band-merge pass and / or the single pass over the tiles past the whole periods),
+ * *scratch_bytes =
  * device scratch it needs (0 for a single pass): taken from cudaMallocAsync on the stream, or the
  * workspace given to pi_attn_fwd_ws.  Returns
  * PI_ATTN_EUNSUPPORTED / PI_ATTN_EINVAL exactly where pi_attn_fwd_ex would. */
@@ -201,8 +205,8 @@ pi_attn_status pi_attn_bwd(const void* q, const void* k, const void* v, const fl
  *                         and the dk/dv pass each run once over the skips alone in the residue-class
  *                         view (the skip keys of a row form a dense band there) and once over the
  *                         window alone; the skip passes use dq as scratch before writing it.  The
- *                         causal rule with n % pi == 0 and a skip outside the window (as
- *                         PI_ATTN_PATH_TC_SPLIT), else PI_ATTN_EUNSUPPORTED.
+ *                         causal rule with n % pi == 0 (the backward's residue view holds every
+ *                         row) and a skip outside the window, else PI_ATTN_EUNSUPPORTED.
  *   PI_ATTN_BWD_TC        tensor cores, fused or split chosen by shape as for PI_ATTN_PATH_TC.
  *   PI_ATTN_BWD_AUTO      PI_ATTN_BWD_TC where the tensor cores apply, else SIMT.
  * The workspace is pi_attn_bwd_workspace_bytes_ex(B, H, n, d, dtype, path) bytes (the tensor-core

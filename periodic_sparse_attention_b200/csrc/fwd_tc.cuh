@@ -350,7 +350,8 @@ struct Params {
   int H, n, kwin, pi, S;
   int T;                  // kResidue: rows per residue class (n / pi)
   float scale_log2;
-  int bidir;              // kFused: the bidirectional index rule (two-sided window, forward skips)
+  int bidir;              // the bidirectional index rule (two-sided window, forward skips; kResidue: both bands)
+  int tile0;              // kFused, kBandMerge: query tile of the grid's first CTA
   // kFused over one shard of a longer sequence: q/out/lse row r is sequence row row0 + r; k/v
   // row r is sequence row kv0 + r (the index rule runs in sequence rows).  0 and 0 otherwise.
   long long row0, kv0;
@@ -400,7 +401,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm<D>) fwd_tc_kernel(const _
         tma_load_4d(base + L::kQ + c * BM * 128, &tmq, bq, c * 64, (int)(blockIdx.x % prm.pi),
                     (int)(blockIdx.x / prm.pi) * BM, bh);
       else
-        tma_load_3d(base + L::kQ + c * BM * 128, &tmq, bq, c * 64, (int)blockIdx.x * BM, bh);
+        tma_load_3d(base + L::kQ + c * BM * 128, &tmq, bq, c * 64, (prm.tile0 + (int)blockIdx.x) * BM, bh);
     }
   }
   const int m0 = first_skip_m(prm.kwin, prm.pi);
@@ -412,11 +413,10 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm<D>) fwd_tc_kernel(const _
     res = blockIdx.x % prm.pi;
     q0 = (long long)(blockIdx.x / prm.pi) * BM;
     // keys of row t: t - S .. t - m0 (the skips of sequence row t*pi + res)
-    walk.init_residue(q0, prm.T, BM, prm.S, m0);
+    walk.init_residue(q0, prm.T, BM, prm.S, m0, prm.bidir != 0);
   } else {
-    q0 = (long long)blockIdx.x * BM;
-    walk.init(prm.row0 + q0, prm.row0 + prm.n, BM, prm.kwin, prm.pi, MODE == kFused ? prm.S : 0,
-              MODE == kFused && prm.bidir);
+    q0 = (long long)(prm.tile0 + (int)blockIdx.x) * BM;
+    walk.init(prm.row0 + q0, prm.row0 + prm.n, BM, prm.kwin, prm.pi, MODE == kFused ? prm.S : 0, prm.bidir != 0);
   }
   const int view_rows = MODE == kResidue ? prm.T : prm.n;
   // every thread walks the tiles with its own cursor (no division per step); thread 0 takes the
@@ -622,8 +622,12 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm<D>) fwd_tc_kernel(const _
     // view, no skips).  Set up while the Q tile is still in flight.
     const long long w_lo = MODE == kResidue ? (qi - prm.S > 0 ? qi - prm.S : 0) : (i - prm.kwin > 0 ? i - prm.kwin : 0);
     const long long w_hi = MODE == kResidue ? qi - m0
-                           : (MODE == kFused && prm.bidir) ? (i + prm.kwin < prm.n - 1 ? i + prm.kwin : prm.n - 1)
-                                                           : i;
+                           : prm.bidir ? (i + prm.kwin < prm.n - 1 ? i + prm.kwin : prm.n - 1)
+                                       : i;
+    // kResidue, bidirectional: the forward band qi + m0 .. qi + S of the view, carried as skip bits
+    // (in this pass every key takes the skip prior, so the bits and the window columns weigh alike)
+    const long long f_lo = qi + m0, f_hi = qi + prm.S < view_rows - 1 ? qi + prm.S : view_rows - 1;
+    const bool fwd_band = MODE == kResidue && prm.bidir && prm.S >= m0;
     RowSkips rs;
     rs.init(i, prm.pi, MODE == kFused ? prm.S : 0, m0, walk.rpi, MODE == kFused && prm.bidir, prm.n);
 
@@ -678,7 +682,14 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm<D>) fwd_tc_kernel(const _
       const int lc_lo = lo64 < 0 ? 0 : (lo64 > BN ? BN : (int)lo64);
       const int lc_hi = hi64 > BN - 1 ? BN - 1 : (hi64 < -1 ? -1 : (int)hi64);
       static_assert(BN == 64, "one 64-bit word of skip bits per tile");
-      const uint64_t skw = rs.take(j0);
+      uint64_t skw = rs.take(j0);
+      if (fwd_band) {  // columns of the forward band [f_lo, f_hi] in this tile
+        const long long a = f_lo - j0, b = f_hi - j0;
+        if (a <= BN - 1 && b >= 0 && a <= b) {
+          const int lo = a < 0 ? 0 : (int)a, hi = b > BN - 1 ? BN - 1 : (int)b;
+          skw = (hi == BN - 1 ? ~0ull : ((1ull << (hi + 1)) - 1ull)) & ~((1ull << lo) - 1ull);
+        }
+      }
       const uint32_t sk[2] = {(uint32_t)skw, (uint32_t)(skw >> 32)};
       const bool has_win = lc_lo <= lc_hi;
       uint32_t sk_any = 0u;
@@ -1055,18 +1066,40 @@ cudaError_t set_smem_attr() {
 
 inline bool tc_supported(bool bf16, int d, int n) { return bf16 && (d == 64 || d == 128) && n >= 1; }
 
-// The split (residue pass + window pass) applies when the sequence is a whole number of periods
-// (the residue view is a plain 4-D tensor) and the residue sequences fit the int coordinates.
+// The backward's split (residue passes + window passes) applies when the sequence is a whole number
+// of periods (the residue view is a plain 4-D tensor) and the residue sequences fit the int
+// coordinates.
 inline bool tc_split_applies(int n, int kwin, int pi, int S) {
   const int m0 = first_skip_m(kwin, pi);
   return S >= m0 && n % pi == 0 && (long long)pi * ((n / pi + tc::BM - 1) / tc::BM) < 0x7fffffffLL;
 }
 
+// The forward's split applies from one whole period on: the residue view covers the whole
+// periods, rows [0, (n / pi) pi), and the query tiles that reach past them run the single pass.
+inline bool tc_split_applies_fwd(int n, int kwin, int pi, int S) {
+  const int m0 = first_skip_m(kwin, pi);
+  return S >= m0 && n >= pi && (long long)pi * ((n / pi + tc::BM - 1) / tc::BM) < 0x7fffffffLL;
+}
+
+// Query tiles of the forward's split path: [0, tiles_merge) take the band-merge pass (every one of
+// their rows has a skip partial from the residue pass), the rest the single pass.
+inline int split_merge_tiles(int n, int pi) {
+  const long long whole = (long long)(n / pi) * pi;  // rows covered by the residue view
+  const int tiles = (n + tc::BM - 1) / tc::BM;
+  return whole == n ? tiles : (int)(whole / tc::BM);
+}
+
 // Pick the split when the skips would cost more tensor work as diagonal tiles than the extra
 // HBM traffic of the split costs: diagonal skip tiles ~ S' per query tile vs ~(k + 128)/128 window
 // tiles; the split adds ~1.3 KB of traffic per row.
-inline bool tc_split_preferred(int n, int kwin, int pi, int S) {
-  if (!tc_split_applies(n, kwin, pi, S)) return false;
+// The bidirectional forward's split: the forward skips of a row may reach past the whole periods,
+// so the residue view must hold every row (n a whole number of periods, as the backward's).
+inline bool tc_split_applies_bidir(int n, int kwin, int pi, int S) { return tc_split_applies(n, kwin, pi, S); }
+
+inline bool tc_split_preferred(int n, int kwin, int pi, int S, bool fwd = false, bool bidir = false) {
+  if (!(bidir ? tc_split_applies_bidir(n, kwin, pi, S)
+              : fwd ? tc_split_applies_fwd(n, kwin, pi, S) : tc_split_applies(n, kwin, pi, S)))
+    return false;
   const int m0 = first_skip_m(kwin, pi);
   const int nskip = S - m0 + 1;
   const int band_tiles = (kwin + 127) / 128 + 1;
@@ -1101,6 +1134,7 @@ cudaError_t launch_fwd_tc_d(const void* q, const void* k, const void* v, const f
   p.T = n / pi;
   p.scale_log2 = (float)(1.0 / std::sqrt((double)D)) * kLog2e;
   p.bidir = bidir ? 1 : 0;
+  p.tile0 = 0;
   p.row0 = 0;
   p.kv0 = 0;
   p.dout = (const __nv_bfloat16*)dout;
@@ -1146,9 +1180,22 @@ cudaError_t launch_fwd_tc_d(const void* q, const void* k, const void* v, const f
   const dim3 grid_r((unsigned)(pi * ((p.T + tc::BM - 1) / tc::BM)), (unsigned)BH);
   tc::fwd_tc_kernel<D, tc::kResidue><<<grid_r, tc::kThreads, L::kAlloc, st>>>(rq, rk, rv, rso, rso, p);
   e = cudaGetLastError();
-  if (e == cudaSuccess) {
-    tc::fwd_tc_kernel<D, tc::kBandMerge><<<grid, tc::kThreads, L::kAlloc, st>>>(mq, mk, mv, mo, mso, p);
+  // the band-merge pass over the query tiles inside the whole periods; the single pass over the
+  // tiles that reach the rows past them (their skips as key tiles, as the fused path takes them)
+  const int ntiles = (n + tc::BM - 1) / tc::BM, nmerge = split_merge_tiles(n, pi);
+  if (e == cudaSuccess && nmerge > 0) {
+    tc::fwd_tc_kernel<D, tc::kBandMerge><<<dim3((unsigned)nmerge, (unsigned)BH), tc::kThreads, L::kAlloc, st>>>(
+        mq, mk, mv, mo, mso, p);
     e = cudaGetLastError();
+  }
+  if (e == cudaSuccess && nmerge < ntiles) {
+    if ((e = tc::set_smem_attr<D, tc::kFused>()) == cudaSuccess) {
+      tc::Params pt = p;
+      pt.tile0 = nmerge;
+      tc::fwd_tc_kernel<D, tc::kFused><<<dim3((unsigned)(ntiles - nmerge), (unsigned)BH), tc::kThreads, L::kAlloc,
+                                         st>>>(mq, mk, mv, mo, mo, pt);
+      e = cudaGetLastError();
+    }
   }
   cudaError_t e2 = own ? cudaFreeAsync(scratch, st) : cudaSuccess;
   *why = "tensor-core split kernels";
@@ -1186,6 +1233,7 @@ cudaError_t launch_fwd_tc_shard_d(const void* q, const void* k, const void* v, c
   p.T = 0;
   p.scale_log2 = (float)(1.0 / std::sqrt((double)D)) * kLog2e;
   p.bidir = 0;
+  p.tile0 = 0;
   p.row0 = row0;
   p.kv0 = kv0;
   p.dout = nullptr;
@@ -1214,7 +1262,7 @@ cudaError_t launch_fwd_tc_with_dot(const void* q, const void* k, const void* v, 
 inline cudaError_t launch_fwd_tc(const void* q, const void* k, const void* v, const float* w_g, const float* b_g,
                                  void* out, float* lse, int B, int H, int n, int d, int kwin, int pi, int S, int mode,
                                  bool bidir, void* workspace, cudaStream_t st, const char** why) {
-  const bool split = !bidir && (mode == 2 || (mode == 0 && tc_split_preferred(n, kwin, pi, S)));
+  const bool split = mode == 2 || (mode == 0 && tc_split_preferred(n, kwin, pi, S, true, bidir));
   if (d == 128)
     return launch_fwd_tc_d<128>(q, k, v, w_g, b_g, out, lse, B, H, n, kwin, pi, S, split, bidir, workspace, st, why);
   return launch_fwd_tc_d<64>(q, k, v, w_g, b_g, out, lse, B, H, n, kwin, pi, S, split, bidir, workspace, st, why);

@@ -262,13 +262,14 @@ static pi_attn_status fwd_route(int n, int d, int k_win, int pi, int S, pi_attn_
   if (want_tc && !tc_ok)
     return fail(PI_ATTN_EUNSUPPORTED, "tensor-core path covers bf16 with d in {64, 128} (got dtype %d, d %d)",
                 (int)dtype, d);
-  if (path == PI_ATTN_PATH_TC_SPLIT && bidir)
-    return fail(PI_ATTN_EUNSUPPORTED, "the split path covers the causal rule only");
-  if (path == PI_ATTN_PATH_TC_SPLIT && !pia::tc_split_applies(n, k_win, pi, S))
-    return fail(PI_ATTN_EUNSUPPORTED, "split path needs n %% pi == 0 and at least one skip outside the window");
+  if (path == PI_ATTN_PATH_TC_SPLIT && bidir && !pia::tc_split_applies_bidir(n, k_win, pi, S))
+    return fail(PI_ATTN_EUNSUPPORTED,
+                "the bidirectional split path needs n %% pi == 0 and at least one skip outside the window");
+  if (path == PI_ATTN_PATH_TC_SPLIT && !bidir && !pia::tc_split_applies_fwd(n, k_win, pi, S))
+    return fail(PI_ATTN_EUNSUPPORTED, "split path needs n >= pi and at least one skip outside the window");
   *tc = path != PI_ATTN_PATH_SIMT && tc_ok;
-  *split = *tc && !bidir && (path == PI_ATTN_PATH_TC_SPLIT ||
-                   (path != PI_ATTN_PATH_TC_FUSED && pia::tc_split_preferred(n, k_win, pi, S)));
+  *split = *tc && (path == PI_ATTN_PATH_TC_SPLIT ||
+                   (path != PI_ATTN_PATH_TC_FUSED && pia::tc_split_preferred(n, k_win, pi, S, true, bidir)));
   return ok();
 }
 
@@ -365,7 +366,12 @@ pi_attn_status pi_attn_fwd_plan(int B, int H, int n, int d, int k_win, int pi, i
   if (st != PI_ATTN_OK) return st;
   bool tc = false, split = false;
   if ((st = fwd_route(n, d, k_win, pi, S, dtype, path, false, &tc, &split)) != PI_ATTN_OK) return st;
-  *launches = split ? 2 : 1;
+  if (split) {  // the residue pass; the band-merge pass and / or the single pass over the ragged tail
+    const int ntiles = (n + pia::tc::BM - 1) / pia::tc::BM, nmerge = pia::split_merge_tiles(n, pi);
+    *launches = 1 + (nmerge > 0 ? 1 : 0) + (nmerge < ntiles ? 1 : 0);
+  } else {
+    *launches = 1;
+  }
   *scratch_bytes = fwd_scratch_bytes(B, H, n, d, split);
   return ok();
 }

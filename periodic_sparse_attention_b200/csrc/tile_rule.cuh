@@ -51,12 +51,14 @@ struct TileWalk {
     rpi = 1.0 / (double)pi_;
   }
   // The residue-class view of the split path: rows q0 .. q0 + rows - 1 of a class of T rows,
-  // row t reading the band of keys t - S .. t - m0 of the same class (its skips, as a dense band)
-  PIA_HD void init_residue(long long q0, long long T, int rows, int S_, int m0_) {
+  // row t reading the band of keys t - S .. t - m0 of the same class (its skips, as a dense band);
+  // bidirectional, also the band t + m0 .. t + S (the forward skips).  The walk covers the union.
+  PIA_HD void init_residue(long long q0, long long T, int rows, int S_, int m0_, bool bidir_ = false) {
     i0 = q0;
-    last = (q0 + rows - 1 < T - 1 ? q0 + rows - 1 : T - 1) - m0_;
+    const long long qlast = q0 + rows - 1 < T - 1 ? q0 + rows - 1 : T - 1;
+    last = qlast - m0_;
     band_lo = q0 - S_ > 0 ? q0 - S_ : 0;
-    band_hi = S_ >= m0_ ? last : -1;  // S < m0: no row has a key
+    band_hi = S_ < m0_ ? -1 : (bidir_ ? (qlast + S_ < T - 1 ? qlast + S_ : T - 1) : last);  // S < m0: no key
     n = T;
     pi = 1;
     S = 0;

@@ -87,8 +87,14 @@ def test_plan_reports_launches_and_scratch(lib):
     assert pia.pi_attn_fwd_plan(1, 8, 4096, 64, 128, 64, 4, "bf16", "tc_split") == (2, 8 * 4096 * (2 * 64 + 4))
     assert pia.pi_attn_fwd_plan(1, 32, 131072, 128, 512, 1024, 16, "bf16", "auto")[0] == 2
     assert pia.pi_attn_fwd_plan(1, 2, 256, 32, 8, 16, 2, "f32", "auto") == (1, 0)
+    # n % pi != 0: the residue view covers rows [0, 62 * 64); the tiles from row 3968 on (tile 31,
+    # which reaches past the whole periods) run the single pass -- three launches
+    assert pia.pi_attn_fwd_plan(1, 8, 4000, 64, 128, 64, 4, "bf16", "tc_split")[0] == 3
+    # n % pi != 0 with the whole periods ending on a tile boundary: 2 * 128 rows, then a tail
+    assert pia.pi_attn_fwd_plan(1, 1, 300, 64, 10, 128, 3, "bf16", "tc_split")[0] == 3
+    # fewer rows than one period: no residue view
     with pytest.raises(pia.PiAttnError):
-        pia.pi_attn_fwd_plan(1, 8, 4000, 64, 128, 64, 4, "bf16", "tc_split")  # n % pi != 0
+        pia.pi_attn_fwd_plan(1, 8, 100, 64, 16, 128, 4, "bf16", "tc_split")
 
 
 def test_workspace_is_checked_before_any_launch(lib):
@@ -103,8 +109,10 @@ def test_workspace_is_checked_before_any_launch(lib):
 
 
 def test_bidir_split_is_refused_before_any_launch(lib):
-    args = [FAKE] * 7 + [1, 1, 4096, 64, 128, 64, 4, pia.PI_ATTN_BF16, pia.PATHS["tc_split"], None]
+    # the bidirectional split needs whole periods (a forward skip may reach past the last one)
+    args = [FAKE] * 7 + [1, 1, 4000, 64, 128, 64, 4, pia.PI_ATTN_BF16, pia.PATHS["tc_split"], None]
     assert lib.pi_attn_fwd_bidir(*args) == pia.PI_ATTN_EUNSUPPORTED
+    assert b"n % pi == 0" in lib.pi_attn_last_error()
     assert lib.pi_attn_debug_index_sets_bidir(16, 4, 4, 2, FAKE, FAKE, 4 + 1 + 2, None) == pia.PI_ATTN_EINVAL  # < 2k+1+2S
 
 

@@ -5,7 +5,6 @@ surviving m adds a forward skip i + m*pi next to the backward one (pi_attn_fwd_b
 cases compare every row; the long case compares sampled rows plus the rows at both ends of every
 (b, h), where the two directions are cut by the sequence bounds.
 """
-import ctypes
 import math
 
 import numpy as np
@@ -60,10 +59,17 @@ CASES = [  # B, H, n, d, k, pi, S
 ]
 
 
-@pytest.mark.parametrize("path", ["auto", "simt", "tc_fused"])
+def _bidir_split_applies(n, k, pi, S, d):
+    # the bidirectional split: n a whole number of periods, a skip outside the window
+    return d in (64, 128) and n % pi == 0 and S >= k // pi + 1
+
+
+@pytest.mark.parametrize("path", ["auto", "simt", "tc_fused", "tc_split"])
 @pytest.mark.parametrize("case", CASES)
 def test_bidir_bf16_every_row(case, path):
     B, H, n, d, k, pi, S = case
+    if path == "tc_split" and not _bidir_split_applies(n, k, pi, S, d):
+        pytest.skip("the bidirectional split needs n % pi == 0 and a skip outside the window")
     inp = _inputs(B, H, n, d, "bf16", seed=3 * n + k)
     out, lse = _run(inp, "bf16", k, pi, S, path)
     ro, rl, _ = oracle.fwd(inp["q"], inp["k"], inp["v"], inp["w_g"], inp["b_g"], k, pi, S, bidir=True)
@@ -80,17 +86,20 @@ def test_bidir_f32_every_row(case):
     assert_close(metrics(out, ro, lse, rl), "f32", f"bidir {case}")
 
 
-def test_bidir_long_sequence_sampled_rows():
-    # the bf16_n32k shape under the bidirectional rule, single pass
+@pytest.mark.parametrize("path", ["auto", "tc_fused", "tc_split"])
+def test_bidir_long_sequence_sampled_rows(path):
+    # the bf16_n32k shape under the bidirectional rule; auto takes the split (both skip bands in the
+    # residue-class pass, the two-sided window in the band-merge pass)
     B, H, n, d, k, pi, S = 2, 16, 32768, 128, 256, 256, 8
+    assert pia.pi_attn_fwd_plan(B, H, n, d, k, pi, S, "bf16", "auto")[0] == 2  # the causal rule splits this shape too
     inp = _inputs(B, H, n, d, "bf16", seed=41)
-    out, lse = _run(inp, "bf16", k, pi, S, "auto")
+    out, lse = _run(inp, "bf16", k, pi, S, path)
     rng = np.random.default_rng(0)
     rows = rng.choice(B * H * n, 2048, replace=False)
     ends = [bh * n + i for bh in range(B * H) for i in (0, k, pi, n - 1 - pi, n - 1 - k, n - 1)]
     rows = np.unique(np.concatenate([rows, np.array(ends)]))
     ro, rl, _ = oracle.fwd_rows(inp["q"], inp["k"], inp["v"], inp["w_g"], inp["b_g"], k, pi, S, rows=rows, bidir=True)
-    assert_close(metrics(out.reshape(-1, d)[rows], ro, lse.reshape(-1)[rows], rl), "bf16", "bidir n32k")
+    assert_close(metrics(out.reshape(-1, d)[rows], ro, lse.reshape(-1)[rows], rl), "bf16", f"bidir n32k/{path}")
     assert np.all(np.isfinite(out)) and np.all(np.isfinite(lse))
 
 
@@ -116,18 +125,17 @@ def test_bidir_index_sets_bit_exact(n, k, pi, S):
     assert np.array_equal(idx.cpu().numpy(), ridx)
 
 
-def test_bidir_split_path_is_unsupported():
-    inp = _inputs(1, 1, 256, 64, "bf16", seed=1)
+def test_bidir_split_path_needs_whole_periods():
+    # a forward skip may reach past the last whole period, outside the residue view: refused before
+    # any launch; on a whole number of periods the split runs and matches the oracle
+    inp = _inputs(1, 1, 250, 64, "bf16", seed=1)
     q, kk, v = (to_dev(inp[x], "bf16") for x in ("q", "k", "v"))
     wg, bg = torch.from_numpy(inp["w_g"]).cuda(), torch.from_numpy(inp["b_g"]).cuda()
     with pytest.raises(pia.PiAttnError) as e:
         pia.pi_attn_fwd(q, kk, v, wg, bg, 8, 64, 3, path="tc_split", bidir=True)
     assert e.value.status == pia.PI_ATTN_EUNSUPPORTED
-    # nothing was launched: the stream is still clean
-    pia.pi_attn_check()
-    out = torch.empty_like(q)
-    p = lambda t: ctypes.c_void_p(t.data_ptr())  # noqa: E731
-    assert pia.load().pi_attn_fwd_bidir(p(q), p(kk), p(v), p(wg), p(bg), p(out), None, 1, 1, 256, 64, 8, 64, 3,
-                                        pia.PI_ATTN_BF16, pia.PATHS["tc"],
-                                        ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)) == pia.PI_ATTN_OK
-    pia.pi_attn_check()
+    pia.pi_attn_check()  # nothing was launched: the stream is still clean
+    inp = _inputs(1, 2, 256, 64, "bf16", seed=1)
+    out, lse = _run(inp, "bf16", 8, 64, 3, "tc_split")
+    ro, rl, _ = oracle.fwd(inp["q"], inp["k"], inp["v"], inp["w_g"], inp["b_g"], 8, 64, 3, bidir=True)
+    assert_close(metrics(out, ro, lse, rl), "bf16", "bidir split n256")

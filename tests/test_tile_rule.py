@@ -110,6 +110,21 @@ def test_residue_view_walks_give_exactly_the_needed_tiles(harness):
         assert harness.residue_walk_mismatches(T, S, m0, 128) == 0, (T, S, m0)
 
 
+def test_bidirectional_residue_walk_covers_both_bands(harness):
+    # the bidirectional split's residue pass: every tile holding a key of some row's backward or
+    # forward band is walked once, and nothing outside the block's reach
+    harness.residue_walk_bidir_errors.argtypes = [ctypes.c_longlong, ctypes.c_int, ctypes.c_int, ctypes.c_int]
+    for T, S, m0 in [(1, 1, 1), (4, 3, 1), (64, 30, 3), (128, 8, 2), (256, 40, 9), (300, 90, 11), (200, 5, 6),
+                     (129, 200, 1), (700, 64, 64)]:
+        assert harness.residue_walk_bidir_errors(T, S, m0, 128) == 0, (T, S, m0)
+    rng = np.random.default_rng(12)
+    for _ in range(200):
+        T = int(rng.integers(1, 1500))
+        m0 = int(rng.integers(1, 12))
+        S = int(rng.integers(0, 150))
+        assert harness.residue_walk_bidir_errors(T, S, m0, 128) == 0, (T, S, m0)
+
+
 def test_cursor_matches_walk_on_walks_built_by_field(harness):
     # band-only walks as the residue-class pass builds them (rows t of a residue view read keys
     # t - S .. t - m0: last is shifted down by m0 and may fall below i0 or below zero), and

@@ -222,3 +222,37 @@ extern "C" int residue_walk_mismatches(long long T, int S, int m0, int rows) {
   }
   return bad;
 }
+
+// The bidirectional residue-class walk (the forward's split of the two-sided rule): rows [q0,
+// q0 + rows) of a class of T rows, row t reading keys t - S .. t - m0 and t + m0 .. t + S within
+// [0, T).  The walk covers the union of the rows' key ranges as one band; it may also walk the few
+// tiles between the two bands of a short block (every row masks them out).  Returns the number of
+// needed tiles missed, tiles walked twice, and tiles walked outside [q0 - S, last row + S].
+extern "C" int residue_walk_bidir_errors(long long T, int S, int m0, int rows) {
+  int bad = 0;
+  const long long ntiles = (T + kTileKeys - 1) / kTileKeys;
+  std::vector<char> want(ntiles), got(ntiles);
+  for (long long b0 = 0; b0 < T; b0 += rows) {
+    const long long b1 = b0 + rows < T ? b0 + rows : T;
+    std::fill(want.begin(), want.end(), 0);
+    std::fill(got.begin(), got.end(), 0);
+    for (long long t = b0; t < b1; ++t)
+      for (long long m = m0; m <= S; ++m) {
+        if (t - m >= 0) want[(t - m) / kTileKeys] = 1;
+        if (t + m < T) want[(t + m) / kTileKeys] = 1;
+      }
+    TileWalk w;
+    w.init_residue(b0, T, rows, S, m0, true);
+    TileCursor c;
+    c.init(w);
+    const long long lo = b0 - S < 0 ? 0 : b0 - S, hi = b1 - 1 + S < T - 1 ? b1 - 1 + S : T - 1;
+    int steps = 0;
+    for (int t = c.next(); t >= 0 && steps < 100000; t = c.next(), ++steps) {
+      if (t >= ntiles || got[t]) ++bad;
+      else got[t] = 1;
+      if ((long long)(t + 1) * kTileKeys - 1 < lo || (long long)t * kTileKeys > hi) ++bad;
+    }
+    for (long long t = 0; t < ntiles; ++t) bad += want[t] && !got[t];
+  }
+  return bad;
+}
