@@ -124,17 +124,18 @@ def source_hash(files=None) -> str:
     return h.hexdigest()[:16]
 
 
-def profiled_traffic(workload: str):
+def profiled_traffic(workload: str, path: str = "auto"):
     """DRAM bytes of one step (its launches summed) from the committed ncu record
-    profiles/traffic.json, if it was taken on the current kernel source: a record for the workload
-    whose listed files still hash to its source_sha.  Otherwise None."""
-    path = os.path.join(ROOT, "profiles", "traffic.json")
-    if not os.path.exists(path):
+    profiles/traffic.json, if it was taken on the current kernel source and the same path: a record
+    for the workload and path (the bench line's "path") whose listed files still hash to its
+    source_sha.  Otherwise None."""
+    fn = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(fn):
         return None
-    with open(path) as f:
+    with open(fn) as f:
         records = json.load(f).get("records", [])
     for r in records:
-        if r.get("workload") != workload:
+        if r.get("workload") != workload or r.get("path", "auto") != path:
             continue
         try:
             if r.get("source_sha") == source_hash(r["files"]):
@@ -498,7 +499,7 @@ def run_gpu(args):
         achieved = flops / launch_s / 1e12
         roof = {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s"}
     roof["frac"] = roof["achieved"] / roof["peak"]
-    roof["traffic"] = profiled_traffic(w.name)
+    roof["traffic"] = profiled_traffic(w.name, bwd_path if w.kind == "backward" else args.path)
     roof["peak_source"] = f"{peak_kind} ({'MEASURED_PEAKS.json' if peak_kind == 'measured' else 'recipe fallback'})"
     roof["algorithmic_bytes"] = bytes_
     roof["algorithmic_flops"] = flops

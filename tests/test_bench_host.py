@@ -48,7 +48,8 @@ def test_traffic_line_needs_the_current_source(tmp_path, monkeypatch):
     prof = tmp_path / "profiles"
     prof.mkdir()
     (prof / "traffic.json").write_text(json.dumps({"records": [
-        {"workload": "bf16_n4k", "bytes_per_step": 123, "files": files, "source_sha": sha},
+        {"workload": "bf16_n4k", "bytes_per_step": 123, "files": files, "source_sha": sha, "path": "auto"},
+        {"workload": "bf16_n4k", "bytes_per_step": 77, "files": files, "source_sha": sha, "path": "tc_fused"},
         {"workload": "bf16_n32k", "bytes_per_step": 9, "files": files, "source_sha": "stale"}]}))
     real_root = bench.ROOT
     monkeypatch.setattr(bench, "ROOT", str(tmp_path))
@@ -56,6 +57,8 @@ def test_traffic_line_needs_the_current_source(tmp_path, monkeypatch):
     os.symlink(os.path.join(real_root, "periodic_sparse_attention_b200", "csrc"),
                tmp_path / "periodic_sparse_attention_b200" / "csrc")
     assert bench.profiled_traffic("bf16_n4k") == 123
+    assert bench.profiled_traffic("bf16_n4k", "tc_fused") == 77
+    assert bench.profiled_traffic("bf16_n4k", "simt") is None  # a record of another path does not apply
     assert bench.profiled_traffic("bf16_n32k") is None
     assert bench.profiled_traffic("bf16_n128k") is None
 
@@ -71,7 +74,7 @@ def test_committed_traffic_records_are_well_formed():
     with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
         recs = json.load(f)["records"]
     for r in recs:
-        assert r["workload"] in ps.WORKLOADS and r["bytes_per_step"] > 0
+        assert r["workload"] in ps.WORKLOADS and r["bytes_per_step"] > 0 and "path" in r
         assert os.path.exists(os.path.join(ROOT, "profiles", r["profile"]))
 
 
