@@ -210,7 +210,12 @@ pi_attn_status pi_attn_bwd(const void* q, const void* k, const void* v, const fl
  *   PI_ATTN_BWD_TC        tensor cores, fused or split chosen by shape as for PI_ATTN_PATH_TC.
  *   PI_ATTN_BWD_AUTO      PI_ATTN_BWD_TC where the tensor cores apply, else SIMT.
  * The workspace is pi_attn_bwd_workspace_bytes_ex(B, H, n, d, dtype, path) bytes (the tensor-core
- * paths add the forward's out and lse); other arguments and errors as pi_attn_bwd. */
+ * paths add the forward's out and lse); other arguments and errors as pi_attn_bwd.
+ * Streams (tensor-core paths): the dk/dv pass runs on a second stream that the library creates
+ * once per device, forked from `stream` after the forward and joined back into it before the call
+ * returns, so all work of the call is ordered before whatever the caller enqueues on `stream`
+ * next; a graph capture of `stream` captures both branches.  The first tensor-core backward on a
+ * device creates that stream and two events, so make it before any graph capture. */
 typedef enum {
     PI_ATTN_BWD_AUTO = 0,
     PI_ATTN_BWD_SIMT = 1,

@@ -13,8 +13,8 @@
 //                       alpha sum_skip ds (the gate's gradient through the two log-priors)
 //   TMA producer warp   Q and dO tiles once, then K and V tiles into a ring of NSTAGE stages
 // lse and D = dO . out of every row come from the forward pass (its epilogue forms D from the
-// fp32 output rows).  The epilogue writes dq = tau dQ + dz w_g (fp32) and the row terms the dk/dv
-// pass and the gate sums read (lse2, log2-priors, dz).
+// fp32 output rows).  The epilogue writes dq = tau dQ + dz w_g (fp32) and the rows' dz, which the
+// gate sums read.
 //
 // TMEM: NBUF pairs of S (64 columns) and dP (64), then dQ (D columns).  D = 64 (two CTAs an SM):
 // one pair and one softmax warpgroup, the next tile's Q K^T waits for this tile's dS K (it reads
@@ -72,11 +72,8 @@ struct BParams {
   const float* b_g;
   const float* lse;   // [B*H, n] the forward's lse (natural log)
   const float* Dr;    // [B*H, n] dO . out
-  float* lse2;        // [B*H, n] lse in log2 units, for the dk/dv pass
   float* dq;          // [B*H, n, D]
-  float* bl2;         // [B*H, n] log2(alpha), log2(1 - alpha), dz: for the dk/dv pass and the gate
-  float* bp2;
-  float* dz;
+  float* dz;          // [B*H, n] dLoss / dz_i, for the gate
   float* part_w;      // [H, B * tiles, D] this CTA's sum of dz_i q_i over its rows, in chunk b * tiles + tile
   float* part_b;      // [H, B * tiles]    and of dz_i
   int H, n, kwin, pi, S;
@@ -405,7 +402,7 @@ __global__ void __launch_bounds__(BSmem<D>::kThreads, BSmem<D>::kCtas) bwd_dq_ke
     }
     {
       // ---- epilogue: dq = tau dQ + dz w_g (each group its share of the columns), and (group 0)
-      // the row terms
+      // the rows' dz
       if (RES) {  // the band columns were skip keys
         dzs += dzw;
         dzw = 0.f;
@@ -452,14 +449,7 @@ __global__ void __launch_bounds__(BSmem<D>::kThreads, BSmem<D>::kCtas) bwd_dq_ke
         }
       }
       if (wg == 0 && (have_q || j == 0)) {
-        if (row_ok) {
-          if (!RES) {
-            prm.lse2[orow] = lse2;
-            prm.bl2[orow] = bl2;
-            prm.bp2[orow] = bp2;
-          }
-          prm.dz[orow] = dz;
-        }
+        if (row_ok) prm.dz[orow] = dz;
       }
       // The gate's partial sums over this CTA's rows, in a fixed order: dw_g[c] += sum_r dz_r q_rc
       // and db_g += sum_r dz_r.  G = BM / D threads a column, each over BM / G rows of the Q tile
@@ -550,7 +540,7 @@ struct KSmem {
 };
 
 struct KParams {
-  const float* lse2;  // [B*H, n] the rows' terms from the dq pass
+  const float* lse2;  // [B*H, n] the rows' terms, written by the forward that precedes the backward
   const float* Dr;
   const float* bl2;
   const float* bp2;

@@ -359,6 +359,12 @@ struct Params {
   // Dout[row] = dout . out from the fp32 output row (before its rounding to bf16).  Null otherwise.
   const __nv_bfloat16* dout;
   float* Dout;
+  // For the backward too (kFused, kBandMerge; null otherwise): the row terms its dk/dv pass reads,
+  // lse in log2 units (from the stored natural-log value) and the log2 priors log2(alpha) and
+  // log2(1 - alpha).
+  float* lse2;
+  float* bl2;
+  float* bp2;
 };
 
 template <int D, int MODE>
@@ -999,6 +1005,11 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm<D>) fwd_tc_kernel(const _
         const float lse_val = l_sum > 0.f ? lse2 * kLn2 : NEG_INF;
         if (MODE == kResidue) prm.skip_lse[orow] = lse_val;
         else if (prm.lse) prm.lse[orow] = lse_val;
+        if (MODE != kResidue && prm.lse2) {
+          prm.lse2[orow] = lse_val * kLog2e;
+          prm.bl2[orow] = bias_l;
+          prm.bp2[orow] = bias_p;
+        }
       }
     }
     tc_fence_before();
@@ -1110,7 +1121,8 @@ template <int D>
 cudaError_t launch_fwd_tc_d(const void* q, const void* k, const void* v, const float* w_g, const float* b_g,
                             void* out, float* lse, int B, int H, int n, int kwin, int pi, int S, bool split,
                             bool bidir, void* workspace, cudaStream_t st, const char** why,
-                            const void* dout = nullptr, float* Dout = nullptr) {
+                            const void* dout = nullptr, float* Dout = nullptr, float* lse2 = nullptr,
+                            float* bl2 = nullptr, float* bp2 = nullptr) {
   using L = tc::Smem<D>;
   CUtensorMap mq, mk, mv;
   const int BH = B * H;
@@ -1139,6 +1151,9 @@ cudaError_t launch_fwd_tc_d(const void* q, const void* k, const void* v, const f
   p.kv0 = 0;
   p.dout = (const __nv_bfloat16*)dout;
   p.Dout = Dout;
+  p.lse2 = lse2;
+  p.bl2 = bl2;
+  p.bp2 = bp2;
   const dim3 grid((unsigned)((n + tc::BM - 1) / tc::BM), (unsigned)BH);
   cudaError_t e;
   CUtensorMap mo;
@@ -1238,6 +1253,7 @@ cudaError_t launch_fwd_tc_shard_d(const void* q, const void* k, const void* v, c
   p.kv0 = kv0;
   p.dout = nullptr;
   p.Dout = nullptr;
+  p.lse2 = p.bl2 = p.bp2 = nullptr;
   cudaError_t e;
   if ((e = tc::set_smem_attr<D, tc::kFused>()) != cudaSuccess) { *why = "cudaFuncSetAttribute"; return e; }
   const dim3 grid((unsigned)((n_q + tc::BM - 1) / tc::BM), (unsigned)BH);
@@ -1251,11 +1267,11 @@ cudaError_t launch_fwd_tc_shard_d(const void* q, const void* k, const void* v, c
 // whose skip partials take rows * (2 D + 4) bytes of `workspace` (16-byte aligned).
 template <int D>
 cudaError_t launch_fwd_tc_with_dot(const void* q, const void* k, const void* v, const float* w_g, const float* b_g,
-                                   const void* dout, void* out, float* lse, float* Dout, int B, int H, int n, int kwin,
-                                   int pi, int S, bool bidir, bool split, void* workspace, cudaStream_t st,
-                                   const char** why) {
+                                   const void* dout, void* out, float* lse, float* Dout, float* lse2, float* bl2,
+                                   float* bp2, int B, int H, int n, int kwin, int pi, int S, bool bidir, bool split,
+                                   void* workspace, cudaStream_t st, const char** why) {
   return launch_fwd_tc_d<D>(q, k, v, w_g, b_g, out, lse, B, H, n, kwin, pi, S, split, bidir, workspace, st, why, dout,
-                            Dout);
+                            Dout, lse2, bl2, bp2);
 }
 
 // mode: 0 = choose, 1 = single pass, 2 = split (residue pass + window pass)

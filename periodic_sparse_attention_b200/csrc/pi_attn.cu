@@ -91,6 +91,56 @@ cudaError_t noalloc_scratch(float** out) {
   return cudaSuccess;
 }
 
+// ---- a second stream per device (the tensor-core backward's dk/dv passes beside its dq passes) ---
+// Created on first use per device: a non-blocking stream and two events without timing.  A call
+// forks onto it and joins back with the lock held, so that calls from several host threads do not
+// record over each other's events between a record and its wait; the kernels themselves run
+// outside the lock.
+struct SideStream {
+  cudaStream_t stream = nullptr;
+  cudaEvent_t fork = nullptr, join = nullptr;
+};
+std::mutex g_side_mu;
+SideStream g_side[kMaxDevices];
+
+cudaError_t side_stream(SideStream** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lock(g_side_mu);
+  SideStream& ss = g_side[dev];
+  if (!ss.stream) {
+    cudaStream_t st = nullptr;
+    cudaEvent_t f = nullptr, j = nullptr;
+    if ((e = cudaStreamCreateWithFlags(&st, cudaStreamNonBlocking)) != cudaSuccess) return e;
+    if ((e = cudaEventCreateWithFlags(&f, cudaEventDisableTiming)) != cudaSuccess ||
+        (e = cudaEventCreateWithFlags(&j, cudaEventDisableTiming)) != cudaSuccess) {
+      if (f) cudaEventDestroy(f);
+      cudaStreamDestroy(st);
+      return e;
+    }
+    ss.stream = st;
+    ss.fork = f;
+    ss.join = j;
+  }
+  *out = &ss;
+  return cudaSuccess;
+}
+
+// Work on `side` after everything enqueued on `s` so far.
+cudaError_t side_fork(SideStream& ss, cudaStream_t s) {
+  std::lock_guard<std::mutex> lock(g_side_mu);
+  cudaError_t e = cudaEventRecord(ss.fork, s);
+  return e == cudaSuccess ? cudaStreamWaitEvent(ss.stream, ss.fork, 0) : e;
+}
+// Work on `s` after everything enqueued on `side` so far.
+cudaError_t side_join(SideStream& ss, cudaStream_t s) {
+  std::lock_guard<std::mutex> lock(g_side_mu);
+  cudaError_t e = cudaEventRecord(ss.join, ss.stream);
+  return e == cudaSuccess ? cudaStreamWaitEvent(s, ss.join, 0) : e;
+}
+
 int num_sms() {
   int dev = 0, sms = 148;
   if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
@@ -576,19 +626,16 @@ pi_attn_status pi_attn_bwd_ex(const void* q, const void* k, const void* v, const
     const long long off = (bwd_ws_bytes(B, H, n, d, true) - rows * 2LL * d - rows * 4LL);
     bf* out_ws = reinterpret_cast<bf*>(static_cast<char*>(scratch) + off);
     float* lse_ws = reinterpret_cast<float*>(static_cast<char*>(scratch) + off + rows * 2LL * d);
-    e = d == 128 ? pia::launch_fwd_tc_with_dot<128>(q, k, v, w_g, b_g, dout, out_ws, lse_ws, rs.D, B, H, n, k_win,
-                                                    pi, S, bd, split, dq, s, &why)
-                 : pia::launch_fwd_tc_with_dot<64>(q, k, v, w_g, b_g, dout, out_ws, lse_ws, rs.D, B, H, n, k_win, pi,
-                                                   S, bd, split, dq, s, &why);
+    e = d == 128 ? pia::launch_fwd_tc_with_dot<128>(q, k, v, w_g, b_g, dout, out_ws, lse_ws, rs.D, rs.lse2, rs.bl2,
+                                                    rs.bp2, B, H, n, k_win, pi, S, bd, split, dq, s, &why)
+                 : pia::launch_fwd_tc_with_dot<64>(q, k, v, w_g, b_g, dout, out_ws, lse_ws, rs.D, rs.lse2, rs.bl2,
+                                                   rs.bp2, B, H, n, k_win, pi, S, bd, split, dq, s, &why);
     pia::tcb::BParams bp;
     bp.w_g = w_g;
     bp.b_g = b_g;
     bp.lse = lse_ws;
     bp.Dr = rs.D;
-    bp.lse2 = rs.lse2;
     bp.dq = dq;
-    bp.bl2 = rs.bl2;
-    bp.bp2 = rs.bp2;
     bp.dz = rs.dz;
     bp.part_w = part_w;
     bp.part_b = part_b;
@@ -615,6 +662,27 @@ pi_attn_status pi_attn_bwd_ex(const void* q, const void* k, const void* v, const
     kp.bidir = bd ? 1 : 0;
     kp.acc = 0;
     using namespace pia::tcb;
+    // The forward wrote every row term the two passes read (lse, D, the log2 priors), so the
+    // dk/dv passes run on the side stream beside the dq passes: they read what the forward wrote
+    // and write only dk and dv.  The side stream joins back before anything after them on `s`
+    // (the gate's final sums wait for the dq passes alone; the scratch release for both).
+    SideStream* side = nullptr;
+    bool forked = false;
+    if (e == cudaSuccess && (e = side_stream(&side)) == cudaSuccess && (e = side_fork(*side, s)) == cudaSuccess)
+      forked = true;
+    if (e != cudaSuccess) why = "backward side stream";
+    if (forked) {
+      const cudaStream_t s2 = side->stream;
+      if (split) {
+        e = d == 128 ? launch_bwd_dkv<128, 1>(q, k, v, dout, kp, B * H, s2, &why)
+                     : launch_bwd_dkv<64, 1>(q, k, v, dout, kp, B * H, s2, &why);
+        kp.S = 0;
+        kp.acc = 1;
+      }
+      if (e == cudaSuccess)
+        e = d == 128 ? launch_bwd_dkv<128, 0>(q, k, v, dout, kp, B * H, s2, &why)
+                     : launch_bwd_dkv<64, 0>(q, k, v, dout, kp, B * H, s2, &why);
+    }
     if (split) {
       if (e == cudaSuccess)
         e = d == 128 ? launch_bwd_dq<128, 1>(q, k, v, dout, bp, B * H, s, &why)
@@ -625,17 +693,17 @@ pi_attn_status pi_attn_bwd_ex(const void* q, const void* k, const void* v, const
     if (e == cudaSuccess)
       e = d == 128 ? launch_bwd_dq<128, 0>(q, k, v, dout, bp, B * H, s, &why)
                    : launch_bwd_dq<64, 0>(q, k, v, dout, bp, B * H, s, &why);
-    if (split) {
-      if (e == cudaSuccess)
-        e = d == 128 ? launch_bwd_dkv<128, 1>(q, k, v, dout, kp, B * H, s, &why)
-                     : launch_bwd_dkv<64, 1>(q, k, v, dout, kp, B * H, s, &why);
-      kp.S = 0;
-      kp.acc = 1;
+    // the gate's partial sums come from the window dq pass, one per (b, query tile); their final
+    // sums run while the side stream may still be busy
+    if (e == cudaSuccess) pia::bwd_gate_final_kernel<<<dim3((unsigned)H, (unsigned)((d + 31) / 32)), 1024, 0, s>>>(
+          part_w, part_b, dw_g, db_g, (int)nchunks, d);
+    if (forked) {  // always, whatever failed above: `s` must not run ahead of the side stream's work
+      const cudaError_t ej = side_join(*side, s);
+      if (e == cudaSuccess && ej != cudaSuccess) {
+        e = ej;
+        why = "backward side stream join";
+      }
     }
-    if (e == cudaSuccess)
-      e = d == 128 ? launch_bwd_dkv<128, 0>(q, k, v, dout, kp, B * H, s, &why)
-                   : launch_bwd_dkv<64, 0>(q, k, v, dout, kp, B * H, s, &why);
-    // (the gate's partial sums come from the window dq pass, one per (b, query tile))
   } else if (dtype == PI_ATTN_F32) {
     e = launch_bwd<float>(q, k, v, w_g, b_g, dout, dq, dk, dv, rs, gt, H, n, d, k_win, pi, S, scale_log2, bd, s);
     if (e == cudaSuccess)
@@ -645,7 +713,7 @@ pi_attn_status pi_attn_bwd_ex(const void* q, const void* k, const void* v, const
     if (e == cudaSuccess)
       pia::bwd_gate_partial_kernel<bf><<<gg, 256, 0, s>>>((const bf*)q, rs.dz, part_w, part_b, B, H, n, d);
   }
-  if (e == cudaSuccess) pia::bwd_gate_final_kernel<<<dim3((unsigned)H, (unsigned)((d + 31) / 32)), 1024, 0, s>>>(
+  if (e == cudaSuccess && !tc) pia::bwd_gate_final_kernel<<<dim3((unsigned)H, (unsigned)((d + 31) / 32)), 1024, 0, s>>>(
         part_w, part_b, dw_g, db_g, (int)nchunks, d);
   if (e == cudaSuccess) e = cudaGetLastError();
   cudaError_t e2 = workspace ? cudaSuccess : cudaFreeAsync(scratch, s);
