@@ -116,12 +116,40 @@ pi_attn_status pi_attn_fwd_shard(const void* q, const void* k, const void* v, co
  * attends, under one softmax, to
  *   L(i) = { j : max(0, i - k_win) <= j <= min(n - 1, i + k_win) }        prior log(alpha)
  *   P(i) = { i - m*pi, i + m*pi : 1 <= m <= S, m*pi > k_win, 0 <= key < n } prior log(1 - alpha)
- * Same arguments, layouts, ownership and errors as pi_attn_fwd_ex; PI_ATTN_PATH_TC_SPLIT returns
- * PI_ATTN_EUNSUPPORTED (the residue split covers the causal rule only) and the other paths
- * allocate nothing. */
+ * Same arguments, layouts, ownership and errors as pi_attn_fwd_ex.  PI_ATTN_PATH_TC_SPLIT (and the
+ * automatic choice of it for long contexts) needs n % pi == 0 and a skip outside the window, else
+ * PI_ATTN_EUNSUPPORTED: its residue-class pass takes both skip bands of a class, and its scratch
+ * comes from cudaMallocAsync on `stream` as for pi_attn_fwd_ex; the other paths allocate nothing. */
 pi_attn_status pi_attn_fwd_bidir(const void* q, const void* k, const void* v, const float* w_g, const float* b_g,
                                  void* out, float* lse, int B, int H, int n, int d, int k_win, int pi, int S,
                                  pi_attn_dtype dtype, pi_attn_path path, void* stream);
+
+/* pi_attn_fwd_ex over inputs and outputs in HOST memory, as a pipeline of chunks.  Cited
+ * passage: "Execution & Scheduling" (the operator streams a long context through the device).
+ * The (b, h) heads are taken chunk_heads at a time (within one b; 0 = about an eighth of H): the
+ * copy of the next chunk's q, k and v to the device, the computation of this chunk (the same
+ * kernels and bits as pi_attn_fwd_ex on device copies of the same inputs) and the copy of the
+ * previous chunk's out and lse back overlap, on two copy streams the library creates once per
+ * device and on `stream` for the computation.
+ *   q, k, v   HOST [B, H, n, d] in dtype, read only; page-locked (cudaHostAlloc or pinned) for the
+ *             copies to overlap -- pageable memory works, but each copy then blocks the host
+ *   out       HOST [B, H, n, d] in dtype; lse HOST fp32 [B, H, n] or NULL
+ *   w_g, b_g  DEVICE, as for pi_attn_fwd (the gate parameters stay resident)
+ *   workspace DEVICE, 256-byte aligned, pi_attn_fwd_host_workspace_bytes(B, H, n, d, dtype,
+ *             chunk_heads) bytes, owned by the caller (three rotating chunk buffers and the split
+ *             path's scratch)
+ * Ordering: the copies start after the work already enqueued on `stream`, and `stream` waits for
+ * all of the call's copies before anything enqueued on it after the call; out and lse are
+ * complete on the host once `stream` has been synchronized.  The host buffers must stay valid
+ * and untouched until then.  Errors as pi_attn_fwd_ex, plus PI_ATTN_EINVAL for a NULL host
+ * pointer, a negative chunk_heads or a workspace that is missing, misaligned or too small.
+ * Causal rule only; not for graph capture with pageable host memory. */
+pi_attn_status pi_attn_fwd_host(const void* q, const void* k, const void* v, const float* w_g, const float* b_g,
+                                void* out, float* lse, int B, int H, int n, int d, int k_win, int pi, int S,
+                                pi_attn_dtype dtype, pi_attn_path path, int chunk_heads, void* workspace,
+                                long long workspace_bytes, void* stream);
+/* Device workspace bytes pi_attn_fwd_host needs for these sizes; -1 for invalid sizes. */
+long long pi_attn_fwd_host_workspace_bytes(int B, int H, int n, int d, pi_attn_dtype dtype, int chunk_heads);
 
 /* What a pi_attn_fwd_ex call with these arguments would launch, without launching anything:
  * *launches = number of kernel launches (1 for a single pass; 2 or 3 for the split: the residue pass,

@@ -33,6 +33,10 @@ SIGNATURES = {
     "pi_attn_fwd_bidir": (_i32, [_vp] * 7 + [_i32] * 9 + [_vp]),
     # ... plus workspace pointer and its size in bytes
     "pi_attn_fwd_ws": (_i32, [_vp] * 7 + [_i32] * 9 + [_vp, ctypes.c_longlong, _vp]),
+    # 7 pointers (q k v host, w_g b_g device, out lse host), B H n d k_win pi S, dtype, path, chunk_heads,
+    # device workspace, its bytes, stream
+    "pi_attn_fwd_host": (_i32, [_vp] * 7 + [_i32] * 10 + [_vp, ctypes.c_longlong, _vp]),
+    "pi_attn_fwd_host_workspace_bytes": (ctypes.c_longlong, [_i32] * 6),
     # B H n d k_win pi S, dtype, path, out: launches, scratch bytes
     "pi_attn_fwd_plan": (_i32, [_i32] * 9 + [_vp, _vp]),
     # 8 pointers (q kcache vcache w_g b_g cache_len out lse), B H n_cache d k_win pi S, dtype, stream
@@ -167,6 +171,48 @@ def pi_attn_fwd_shard(q, k, v, w_g, b_g, k_win: int, pi: int, S: int, row0: int,
         lse = torch.empty((B, H, n_q), dtype=torch.float32, device=q.device)
     st = load().pi_attn_fwd_shard(_ptr(q), _ptr(k), _ptr(v), _ptr(w_g), _ptr(b_g), _ptr(out), _ptr(lse), B, H, n_q,
                                   n_kv, row0, kv0, d, k_win, pi, S, _dtype_code(q), _stream(stream))
+    _raise(st)
+    return out, lse
+
+
+def _hptr(t):
+    if t is None:
+        return None
+    if t.is_cuda:
+        raise ValueError("pi_attn_fwd_host takes q, k, v, out and lse in host memory")
+    if not t.is_contiguous():
+        raise ValueError("pi-attention tensors must be contiguous")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def pi_attn_fwd_host_workspace_bytes(B: int, H: int, n: int, d: int, dtype: str = "bf16", chunk_heads: int = 0):
+    return load().pi_attn_fwd_host_workspace_bytes(B, H, n, d, PI_ATTN_BF16 if dtype == "bf16" else PI_ATTN_F32,
+                                                   chunk_heads)
+
+
+def pi_attn_fwd_host(q, k, v, w_g, b_g, k_win: int, pi: int, S: int, out=None, lse=None, *, path: str = "auto",
+                     chunk_heads: int = 0, workspace=None, stream=None, want_lse: bool = True):
+    """Prefill forward with q, k, v, out and lse in host memory (torch CPU tensors; pinned for the
+    copies to overlap), w_g and b_g on the device: pi_attn_fwd_host, a pipeline of chunks of
+    chunk_heads heads.  Allocates out and lse (pinned) when not given and the device workspace
+    from torch's caching allocator when not given.  The results are on the host once the stream
+    has been synchronized (this function does not synchronize)."""
+    import torch
+    B, H, n, d = q.shape
+    if out is None:
+        out = torch.empty(q.shape, dtype=q.dtype).pin_memory()
+    if lse is None and want_lse:
+        lse = torch.empty((B, H, n), dtype=torch.float32).pin_memory()
+    dt = _dtype_code(q)
+    if workspace is None:
+        nbytes = pi_attn_fwd_host_workspace_bytes(B, H, n, d, "bf16" if dt == PI_ATTN_BF16 else "f32", chunk_heads)
+        if nbytes < 0:
+            raise ValueError(f"invalid sizes for pi_attn_fwd_host: {tuple(q.shape)}, chunk_heads={chunk_heads}")
+        workspace = torch.empty(nbytes, dtype=torch.uint8, device=w_g.device)
+    ws_bytes = workspace.numel() * workspace.element_size()
+    st = load().pi_attn_fwd_host(_hptr(q), _hptr(k), _hptr(v), _ptr(w_g), _ptr(b_g), _hptr(out), _hptr(lse), B, H, n,
+                                 d, k_win, pi, S, dt, PATHS[path], chunk_heads, _ptr(workspace), ws_bytes,
+                                 _stream(stream))
     _raise(st)
     return out, lse
 

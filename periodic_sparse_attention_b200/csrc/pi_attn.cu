@@ -141,6 +141,59 @@ cudaError_t side_join(SideStream& ss, cudaStream_t s) {
   return e == cudaSuccess ? cudaStreamWaitEvent(s, ss.join, 0) : e;
 }
 
+// ---- the host-buffer prefill's copy streams (pi_attn_fwd_host) ----------------------------------
+// Per device: a stream for the copies in, one for the copies out, and events for the three
+// rotating chunk buffers of the workspace (loaded, computed, free again) plus two for the joins.
+// A call holds the lock for its whole enqueue sequence: its events are recorded and waited on in
+// one order, whatever other host threads do.
+constexpr int kHostSets = 3;
+struct HostPipe {
+  cudaStream_t in = nullptr, out = nullptr;
+  cudaEvent_t start = nullptr, join_in = nullptr, join_out = nullptr;
+  cudaEvent_t loaded[kHostSets] = {}, computed[kHostSets] = {}, freed[kHostSets] = {};
+};
+std::mutex g_pipe_mu;
+HostPipe g_pipe[kMaxDevices];
+
+// The current device's pipe, created on first use; call with g_pipe_mu held.
+cudaError_t host_pipe(HostPipe** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  HostPipe& hp = g_pipe[dev];
+  if (!hp.in) {
+    HostPipe t;
+    e = cudaStreamCreateWithFlags(&t.in, cudaStreamNonBlocking);
+    if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&t.out, cudaStreamNonBlocking);
+    cudaEvent_t* evs[] = {&t.start, &t.join_in, &t.join_out, &t.loaded[0], &t.loaded[1], &t.loaded[2],
+                          &t.computed[0], &t.computed[1], &t.computed[2], &t.freed[0], &t.freed[1], &t.freed[2]};
+    for (cudaEvent_t* ev : evs)
+      if (e == cudaSuccess) e = cudaEventCreateWithFlags(ev, cudaEventDisableTiming);
+    if (e != cudaSuccess) {
+      for (cudaEvent_t* ev : evs)
+        if (*ev) cudaEventDestroy(*ev);
+      if (t.in) cudaStreamDestroy(t.in);
+      if (t.out) cudaStreamDestroy(t.out);
+      return e;
+    }
+    hp = t;
+  }
+  *out = &hp;
+  return cudaSuccess;
+}
+
+long long round256(long long x) { return (x + 255) / 256 * 256; }
+// (b, h) heads per chunk of pi_attn_fwd_host: the caller's choice, or about an eighth of H
+int host_chunk_heads(int H, int chunk_heads) {
+  if (chunk_heads > 0) return chunk_heads < H ? chunk_heads : H;
+  return (H + 7) / 8;
+}
+// One rotating buffer set: q, k, v and out of a chunk, then its lse.
+long long host_set_bytes(int hc, int n, int d, int elem) {
+  return 4 * round256((long long)hc * n * d * elem) + round256((long long)hc * n * 4);
+}
+
 int num_sms() {
   int dev = 0, sms = 148;
   if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
@@ -405,6 +458,91 @@ pi_attn_status pi_attn_fwd_ex(const void* q, const void* k, const void* v, const
                               void* out, float* lse, int B, int H, int n, int d, int k_win, int pi, int S,
                               pi_attn_dtype dtype, pi_attn_path path, void* stream) {
   return pi_attn_fwd_ws(q, k, v, w_g, b_g, out, lse, B, H, n, d, k_win, pi, S, dtype, path, nullptr, 0, stream);
+}
+
+long long pi_attn_fwd_host_workspace_bytes(int B, int H, int n, int d, pi_attn_dtype dtype, int chunk_heads) {
+  if (B < 1 || H < 1 || n < 1 || d < 1 || chunk_heads < 0 || (dtype != PI_ATTN_F32 && dtype != PI_ATTN_BF16))
+    return -1;
+  const int hc = host_chunk_heads(H, chunk_heads);
+  return kHostSets * host_set_bytes(hc, n, d, (int)elem_size(dtype)) + round256((long long)hc * n * (2LL * d + 4));
+}
+
+pi_attn_status pi_attn_fwd_host(const void* q, const void* k, const void* v, const float* w_g, const float* b_g,
+                                void* out, float* lse, int B, int H, int n, int d, int k_win, int pi, int S,
+                                pi_attn_dtype dtype, pi_attn_path path, int chunk_heads, void* workspace,
+                                long long workspace_bytes, void* stream) {
+  if (!q || !k || !v || !out) return fail(PI_ATTN_EINVAL, "null host tensor pointer");
+  if (!w_g || !b_g) return fail(PI_ATTN_EINVAL, "null gate parameter pointer");
+  if (chunk_heads < 0) return fail(PI_ATTN_EINVAL, "chunk_heads must be >= 0 (got %d)", chunk_heads);
+  // the checks every chunk's call makes, once for the whole problem before anything is enqueued
+  static const char dummy[16] __attribute__((aligned(16))) = {0};
+  pi_attn_status st = check_common(dummy, dummy, dummy, w_g, b_g, dummy, B, H, n, d, k_win, pi, S, dtype);
+  if (st != PI_ATTN_OK) return st;
+  bool tc = false, split = false;
+  if ((st = fwd_route(n, d, k_win, pi, S, dtype, path, false, &tc, &split)) != PI_ATTN_OK) return st;
+  const long long need = pi_attn_fwd_host_workspace_bytes(B, H, n, d, dtype, chunk_heads);
+  if (!workspace || reinterpret_cast<uintptr_t>(workspace) % 256 != 0)
+    return fail(PI_ATTN_EINVAL, "workspace must be a 256-byte aligned device pointer");
+  if (workspace_bytes < need)
+    return fail(PI_ATTN_EINVAL, "workspace of %lld bytes, the call needs %lld", workspace_bytes, need);
+  const int hc = host_chunk_heads(H, chunk_heads);
+  const int elem = (int)elem_size(dtype);
+  const long long tile = round256((long long)hc * n * d * elem), set_bytes = host_set_bytes(hc, n, d, elem);
+  char* const ws = static_cast<char*>(workspace);
+  void* const scratch = ws + kHostSets * set_bytes;
+  const long long scratch_bytes = round256((long long)hc * n * (2LL * d + 4));
+  cudaStream_t s = as_stream(stream);
+
+  std::lock_guard<std::mutex> lock(g_pipe_mu);
+  HostPipe* hp = nullptr;
+  cudaError_t e = host_pipe(&hp);
+  if (e != cudaSuccess) return cuda_fail(e, "copy streams");
+  // the copies start after the work already on `stream` (an earlier call may still use the workspace)
+  if ((e = cudaEventRecord(hp->start, s)) != cudaSuccess || (e = cudaStreamWaitEvent(hp->in, hp->start, 0)) != cudaSuccess ||
+      (e = cudaStreamWaitEvent(hp->out, hp->start, 0)) != cudaSuccess)
+    return cuda_fail(e, "copy streams");
+  const char* why = "host-buffer chunk copies";
+  int c = 0;
+  for (int b = 0; b < B && st == PI_ATTN_OK && e == cudaSuccess; ++b) {
+    for (int h0 = 0; h0 < H && st == PI_ATTN_OK && e == cudaSuccess; h0 += hc, ++c) {
+      const int h = hc < H - h0 ? hc : H - h0, set = c % kHostSets;
+      char* const base = ws + set * set_bytes;
+      void *dq = base, *dk = base + tile, *dv = base + 2 * tile, *dout = base + 3 * tile;
+      float* const dlse = reinterpret_cast<float*>(base + 4 * tile);
+      const long long row0 = (long long)b * H + h0;  // first (b, h) of the chunk
+      const size_t bytes = (size_t)h * n * d * elem, off = (size_t)row0 * n * d * elem;
+      // in: the set's buffers are free once the copies out of the chunk three before have run
+      if (c >= kHostSets && (e = cudaStreamWaitEvent(hp->in, hp->freed[set], 0)) != cudaSuccess) break;
+      if ((e = cudaMemcpyAsync(dq, static_cast<const char*>(q) + off, bytes, cudaMemcpyHostToDevice, hp->in)) != cudaSuccess ||
+          (e = cudaMemcpyAsync(dk, static_cast<const char*>(k) + off, bytes, cudaMemcpyHostToDevice, hp->in)) != cudaSuccess ||
+          (e = cudaMemcpyAsync(dv, static_cast<const char*>(v) + off, bytes, cudaMemcpyHostToDevice, hp->in)) != cudaSuccess ||
+          (e = cudaEventRecord(hp->loaded[set], hp->in)) != cudaSuccess ||
+          (e = cudaStreamWaitEvent(s, hp->loaded[set], 0)) != cudaSuccess)
+        break;
+      // compute on `stream`: the chunk as a [1, h, n, d] problem with its heads' gate parameters
+      st = fwd_impl(dq, dk, dv, w_g + (long long)h0 * d, b_g + h0, dout, lse ? dlse : nullptr, 1, h, n, d, k_win, pi,
+                    S, dtype, path, false, scratch, scratch_bytes, stream);
+      if (st != PI_ATTN_OK) break;
+      // out
+      if ((e = cudaEventRecord(hp->computed[set], s)) != cudaSuccess ||
+          (e = cudaStreamWaitEvent(hp->out, hp->computed[set], 0)) != cudaSuccess ||
+          (e = cudaMemcpyAsync(static_cast<char*>(out) + off, dout, bytes, cudaMemcpyDeviceToHost, hp->out)) != cudaSuccess)
+        break;
+      if (lse && (e = cudaMemcpyAsync(lse + row0 * n, dlse, (size_t)h * n * 4, cudaMemcpyDeviceToHost, hp->out)) != cudaSuccess)
+        break;
+      if ((e = cudaEventRecord(hp->freed[set], hp->out)) != cudaSuccess) break;
+    }
+  }
+  // join both copy streams back into `stream`, whatever failed above: the caller's next work on
+  // `stream` (and the workspace's next user) must come after every copy this call enqueued
+  cudaError_t ej = cudaEventRecord(hp->join_in, hp->in);
+  if (ej == cudaSuccess) ej = cudaStreamWaitEvent(s, hp->join_in, 0);
+  if (ej == cudaSuccess) ej = cudaEventRecord(hp->join_out, hp->out);
+  if (ej == cudaSuccess) ej = cudaStreamWaitEvent(s, hp->join_out, 0);
+  if (st != PI_ATTN_OK) return st;
+  if (e != cudaSuccess) return cuda_fail(e, why);
+  if (ej != cudaSuccess) return cuda_fail(ej, "joining the copy streams");
+  return ok();
 }
 
 pi_attn_status pi_attn_fwd_plan(int B, int H, int n, int d, int k_win, int pi, int S, pi_attn_dtype dtype,

@@ -209,3 +209,33 @@ def test_product_path_never_touches_the_oracle():
 def test_binding_fails_loudly_without_the_library(tmp_path):
     with pytest.raises(ImportError):
         pia.load(str(tmp_path / "missing.so"))
+
+
+def test_host_entry_workspace_size_and_argument_checks(lib):
+    # three rotating chunk buffers (q, k, v, out and lse of chunk_heads heads, 256-byte rounded)
+    # and the split path's scratch for one chunk
+    r = lambda x: (x + 255) // 256 * 256  # noqa: E731
+    B, H, n, d = 1, 32, 131072, 128
+    for chunk, hc in ((4, 4), (0, 4), (100, 32), (1, 1)):
+        want = 3 * (4 * r(hc * n * d * 2) + r(hc * n * 4)) + r(hc * n * (2 * d + 4))
+        assert lib.pi_attn_fwd_host_workspace_bytes(B, H, n, d, pia.PI_ATTN_BF16, chunk) == want
+    assert lib.pi_attn_fwd_host_workspace_bytes(1, 5, 300, 32, pia.PI_ATTN_F32, 0) == \
+        3 * (4 * r(300 * 32 * 4) + r(300 * 4)) + r(300 * 68)
+    for bad in ((0, 1, 1, 64, 1, 0), (1, 1, 1, 64, 1, -1), (1, 1, 1, 64, 7, 0)):
+        assert lib.pi_attn_fwd_host_workspace_bytes(*bad) == -1
+    # rejected before any CUDA call: no device is needed for these
+    h = ctypes.c_void_p(0x1000)  # stand-in pointers, never dereferenced
+    ws = ctypes.c_void_p(0x10000)
+    need = lib.pi_attn_fwd_host_workspace_bytes(1, 2, 256, 64, pia.PI_ATTN_BF16, 1)
+
+    def call(q=h, wg=h, chunk=1, w=ws, nbytes=need, n=256, pi=16, path=0):
+        return lib.pi_attn_fwd_host(q, h, h, wg, h, h, None, 1, 2, n, 64, 16, pi, 3, pia.PI_ATTN_BF16, path, chunk, w,
+                                    nbytes, None)
+    assert call(q=None) == pia.PI_ATTN_EINVAL
+    assert call(wg=None) == pia.PI_ATTN_EINVAL
+    assert call(chunk=-1) == pia.PI_ATTN_EINVAL
+    assert call(w=None) == pia.PI_ATTN_EINVAL
+    assert call(w=ctypes.c_void_p(0x10010)) == pia.PI_ATTN_EINVAL  # not 256-byte aligned
+    assert call(nbytes=need - 1) == pia.PI_ATTN_EINVAL
+    assert call(pi=0) == pia.PI_ATTN_EINVAL
+    assert call(n=100, path=pia.PATHS["tc_split"], pi=128) == pia.PI_ATTN_EUNSUPPORTED  # n < pi
