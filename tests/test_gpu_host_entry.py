@@ -89,3 +89,50 @@ def test_host_entry_against_the_oracle_and_back_to_back_calls():
         got = ps.bf16_bits_to_f32(out.view(torch.int16).numpy().view(np.uint16)).astype(np.float64)
         m = metrics(got.reshape(-1, d), ro.reshape(-1, d), lse.numpy().astype(np.float64).reshape(-1), rl.reshape(-1))
         assert_close(m, "bf16", f"pi_attn_fwd_host, call with seed {seed}")
+
+
+def test_two_host_threads_share_the_library_streams():
+    # the host-buffer prefill and the tensor-core backward use streams and events the library
+    # keeps per device; two host threads, each on its own stream with its own problem, call both
+    # at once, several times, and each must get its own problem's bits
+    import threading
+    B, H, n, d, k, pi, S = 1, 4, 2048, 64, 60, 40, 6
+    probs = [_problem(B, H, n, d, "bf16", seed) for seed in (21, 22)]
+    refs, dev = [], []
+    for inp in probs:
+        dq = {x: _host(inp[x], "bf16", False).cuda() for x in ("q", "k", "v")}
+        wg, bg = torch.from_numpy(inp["w_g"]).cuda(), torch.from_numpy(inp["b_g"]).cuda()
+        go = torch.from_numpy(ps.normal((B, H, n, d), seed=7, stream=6, dtype="bf16").view(np.int16)).view(
+            torch.bfloat16).cuda()
+        o, l = pia.pi_attn_fwd(dq["q"], dq["k"], dq["v"], wg, bg, k, pi, S)
+        g = pia.pi_attn_bwd(dq["q"], dq["k"], dq["v"], wg, bg, go, k, pi, S, path="tc")
+        refs.append((o.cpu(), l.cpu(), [t.cpu() for t in g]))
+        dev.append((dq, wg, bg, go, {x: _host(inp[x], "bf16", True) for x in ("q", "k", "v")}))
+    torch.cuda.synchronize()
+    errors = []
+
+    def work(i):
+        try:
+            dq, wg, bg, go, host = dev[i]
+            s = torch.cuda.Stream()
+            with torch.cuda.stream(s):
+                for _ in range(4):
+                    out, lse = pia.pi_attn_fwd_host(host["q"], host["k"], host["v"], wg, bg, k, pi, S, chunk_heads=1)
+                    g = pia.pi_attn_bwd(dq["q"], dq["k"], dq["v"], wg, bg, go, k, pi, S, path="tc")
+                    s.synchronize()
+                    ro, rl, rg = refs[i]
+                    if not (torch.equal(out.view(torch.int16), ro.view(torch.int16)) and torch.equal(lse, rl)):
+                        errors.append(f"thread {i}: host-buffer prefill differs")
+                    if not all(torch.equal(a.cpu(), b) for a, b in zip(g, rg)):
+                        errors.append(f"thread {i}: backward differs")
+        except Exception as e:  # reported below, on the test's thread
+            errors.append(f"thread {i}: {e!r}")
+
+    threads = [threading.Thread(target=work, args=(i,)) for i in range(2)]
+    for t in threads:
+        t.start()
+    for t in threads:
+        t.join(timeout=300)
+    assert not any(t.is_alive() for t in threads), "a thread did not finish"
+    pia.pi_attn_check()
+    assert not errors, errors
