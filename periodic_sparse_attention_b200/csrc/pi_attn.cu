@@ -806,9 +806,12 @@ pi_attn_status pi_attn_bwd_ex(const void* q, const void* k, const void* v, const
     // (the gate's final sums wait for the dq passes alone; the scratch release for both).
     SideStream* side = nullptr;
     bool forked = false;
-    if (e == cudaSuccess && (e = side_stream(&side)) == cudaSuccess && (e = side_fork(*side, s)) == cudaSuccess)
-      forked = true;
-    if (e != cudaSuccess) why = "backward side stream";
+    if (e == cudaSuccess) {
+      if ((e = side_stream(&side)) == cudaSuccess && (e = side_fork(*side, s)) == cudaSuccess)
+        forked = true;
+      else
+        why = "backward side stream";
+    }
     if (forked) {
       const cudaStream_t s2 = side->stream;
       if (split) {
