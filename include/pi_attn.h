@@ -20,10 +20,13 @@
  *   - dtype names the storage type of q, k, v, caches and out: PI_ATTN_F32 (fp32) or PI_ATTN_BF16
  *     (bfloat16).  Arithmetic is fp32 (bf16 products on tensor cores accumulate in fp32); out is
  *     rounded once, to nearest even, into dtype.
- *   - All pointers are DEVICE pointers owned by the caller; the library keeps no reference after
- *     the call returns and holds no allocation of its own between calls (the decode entry point
- *     for callers that cannot allocate uses a fixed array inside the library, see below).  Tensor pointers must be
- *     16-byte aligned and d * sizeof(dtype) a multiple of 16 bytes.
+ *   - All pointers are DEVICE pointers owned by the caller (pi_attn_fwd_host takes host buffers
+ *     instead); the library keeps no reference after the call returns and holds no memory
+ *     allocation of its own between calls, with two exceptions stated at their entry points: the
+ *     fixed device array of the decode for callers that cannot allocate, and the streams and
+ *     events it creates once per device, on first use, for the tensor-core backward and the
+ *     host-buffer prefill (kept until the process exits).  Tensor pointers must be 16-byte aligned
+ *     and d * sizeof(dtype) a multiple of 16 bytes.
  *   - `stream` is a cudaStream_t (NULL: the legacy default stream).  Calls only enqueue work: they
  *     are asynchronous and stream-ordered.  Argument errors are returned synchronously and then
  *     nothing is enqueued.  Errors that only a kernel can see (a cache length out of range, an
