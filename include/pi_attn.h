@@ -129,7 +129,7 @@ pi_attn_status pi_attn_fwd_bidir(const void* q, const void* k, const void* v, co
 
 /* pi_attn_fwd_ex over inputs and outputs in HOST memory, as a pipeline of chunks.  Cited
  * passage: "Execution & Scheduling" (the operator streams a long context through the device).
- * The (b, h) heads are taken chunk_heads at a time (within one b; 0 = about an eighth of H): the
+ * The (b, h) heads are taken chunk_heads at a time (within one b; 0 = about a thirty-second of H): the
  * copy of the next chunk's q, k and v to the device, the computation of this chunk (the same
  * kernels and bits as pi_attn_fwd_ex on device copies of the same inputs) and the copy of the
  * previous chunk's out and lse back overlap, on two copy streams the library creates once per

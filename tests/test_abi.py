@@ -216,7 +216,7 @@ def test_host_entry_workspace_size_and_argument_checks(lib):
     # and the split path's scratch for one chunk
     r = lambda x: (x + 255) // 256 * 256  # noqa: E731
     B, H, n, d = 1, 32, 131072, 128
-    for chunk, hc in ((4, 4), (0, 4), (100, 32), (1, 1)):
+    for chunk, hc in ((4, 4), (0, 1), (100, 32), (1, 1)):
         want = 3 * (4 * r(hc * n * d * 2) + r(hc * n * 4)) + r(hc * n * (2 * d + 4))
         assert lib.pi_attn_fwd_host_workspace_bytes(B, H, n, d, pia.PI_ATTN_BF16, chunk) == want
     assert lib.pi_attn_fwd_host_workspace_bytes(1, 5, 300, 32, pia.PI_ATTN_F32, 0) == \
