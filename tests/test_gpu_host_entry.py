@@ -136,3 +136,34 @@ def test_two_host_threads_share_the_library_streams():
     assert not any(t.is_alive() for t in threads), "a thread did not finish"
     pia.pi_attn_check()
     assert not errors, errors
+
+
+def test_host_entry_replays_as_a_cuda_graph_with_pinned_buffers():
+    # captured on a side stream with pinned host buffers (the copy streams join the capture
+    # through the call's events) and replayed: the eager call's bits, on the host
+    B, H, n, d, k, pi, S = 1, 3, 2048, 64, 60, 40, 6
+    inp = _problem(B, H, n, d, "bf16", seed=31)
+    wg, bg = torch.from_numpy(inp["w_g"]).cuda(), torch.from_numpy(inp["b_g"]).cuda()
+    host = {x: _host(inp[x], "bf16", True) for x in ("q", "k", "v")}
+    ws = torch.empty(pia.pi_attn_fwd_host_workspace_bytes(B, H, n, d, "bf16", 1), dtype=torch.uint8, device="cuda")
+    ref_out, ref_lse = pia.pi_attn_fwd_host(host["q"], host["k"], host["v"], wg, bg, k, pi, S, chunk_heads=1,
+                                            workspace=ws)
+    torch.cuda.synchronize()
+    ref_out, ref_lse = ref_out.clone(), ref_lse.clone()
+    out = torch.empty_like(ref_out).pin_memory()
+    lse = torch.empty_like(ref_lse).pin_memory()
+    g = torch.cuda.CUDAGraph()
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side), torch.cuda.graph(g, stream=side):
+        pia.pi_attn_fwd_host(host["q"], host["k"], host["v"], wg, bg, k, pi, S, out=out, lse=lse, chunk_heads=1,
+                             workspace=ws)
+    for _ in range(2):
+        out.view(torch.int16).fill_(-1)
+        lse.fill_(float("nan"))
+        g.replay()
+        torch.cuda.synchronize()
+        pia.pi_attn_check()
+        assert torch.equal(out.view(torch.int16), ref_out.view(torch.int16)), "out differs after a graph replay"
+        assert torch.equal(lse, ref_lse), "lse differs after a graph replay"
+    del g
