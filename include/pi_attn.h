@@ -52,7 +52,8 @@ typedef enum { PI_ATTN_F32 = 0, PI_ATTN_BF16 = 1 } pi_attn_dtype;
 
 /* Kernel choice for pi_attn_fwd_ex. */
 typedef enum {
-    PI_ATTN_PATH_AUTO = 0,      /* tensor-core kernel where it applies (bf16, d in {64, 128}), else SIMT */
+    PI_ATTN_PATH_AUTO = 0,      /* tensor-core kernel where it applies (bf16, d in {64, 128}, B*H <= 65535),
+                                   else SIMT */
     PI_ATTN_PATH_SIMT = 1,      /* CUDA-core kernel: every dtype, d <= 256 */
     PI_ATTN_PATH_TC = 2,        /* tcgen05/TMEM kernels only (single pass or split, chosen by shape);
                                    PI_ATTN_EUNSUPPORTED where they do not apply */

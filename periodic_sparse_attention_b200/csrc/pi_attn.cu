@@ -359,11 +359,17 @@ int pi_attn_version(void) { return 100; }
 
 // Which kernels a forward call with these arguments runs: *tc (tensor-core path) and *split
 // (residue pass + band-merge pass), after the same checks as the call itself.
-static pi_attn_status fwd_route(int n, int d, int k_win, int pi, int S, pi_attn_dtype dtype, pi_attn_path path,
-                                bool bidir, bool* tc, bool* split) {
+// The tensor-core kernels take the (b, h) pairs as their grid's y dimension.
+constexpr long long kMaxGridY = 65535;
+
+static pi_attn_status fwd_route(long long bh, int n, int d, int k_win, int pi, int S, pi_attn_dtype dtype,
+                                pi_attn_path path, bool bidir, bool* tc, bool* split) {
   if (path < PI_ATTN_PATH_AUTO || path > PI_ATTN_PATH_TC_SPLIT) return fail(PI_ATTN_EINVAL, "unknown path %d", (int)path);
-  const bool tc_ok = pia::tc_supported(dtype == PI_ATTN_BF16, d, n);
+  const bool tc_ok = pia::tc_supported(dtype == PI_ATTN_BF16, d, n) && bh <= kMaxGridY;
   const bool want_tc = path == PI_ATTN_PATH_TC || path == PI_ATTN_PATH_TC_FUSED || path == PI_ATTN_PATH_TC_SPLIT;
+  if (want_tc && bh > kMaxGridY)
+    return fail(PI_ATTN_EUNSUPPORTED, "tensor-core path takes at most %lld (b, h) pairs a call (got %lld)", kMaxGridY,
+                bh);
   if (want_tc && !tc_ok)
     return fail(PI_ATTN_EUNSUPPORTED, "tensor-core path covers bf16 with d in {64, 128} (got dtype %d, d %d)",
                 (int)dtype, d);
@@ -389,7 +395,7 @@ static pi_attn_status fwd_impl(const void* q, const void* k, const void* v, cons
   pi_attn_status st = check_common(q, k, v, w_g, b_g, out, B, H, n, d, k_win, pi, S, dtype);
   if (st != PI_ATTN_OK) return st;
   bool tc = false, split = false;
-  if ((st = fwd_route(n, d, k_win, pi, S, dtype, path, bidir, &tc, &split)) != PI_ATTN_OK) return st;
+  if ((st = fwd_route((long long)B * H, n, d, k_win, pi, S, dtype, path, bidir, &tc, &split)) != PI_ATTN_OK) return st;
   if (workspace) {
     if (reinterpret_cast<uintptr_t>(workspace) % 16 != 0) return fail(PI_ATTN_EINVAL, "workspace not 16-byte aligned");
     const long long need = fwd_scratch_bytes(B, H, n, d, split);
@@ -448,6 +454,9 @@ pi_attn_status pi_attn_fwd_shard(const void* q, const void* k, const void* v, co
     return fail(PI_ATTN_EINVAL, "k/v rows end at %lld, before the shard's last row %lld", kv0 + n_kv - 1,
                 row0 + n_q - 1);
   if (row0 + n_q > 0x7fffffffLL) return fail(PI_ATTN_EINVAL, "sequence rows past 2^31");
+  if ((long long)B * H > kMaxGridY)
+    return fail(PI_ATTN_EUNSUPPORTED, "the shard forward takes at most %lld (b, h) pairs a call (got %lld)", kMaxGridY,
+                (long long)B * H);
   const char* why = "";
   cudaError_t e = d == 128 ? pia::launch_fwd_tc_shard_d<128>(q, k, v, w_g, b_g, out, lse, B, H, n_q, n_kv, row0, kv0,
                                                              k_win, pi, S, as_stream(stream), &why)
@@ -480,8 +489,10 @@ pi_attn_status pi_attn_fwd_host(const void* q, const void* k, const void* v, con
   static const char dummy[16] __attribute__((aligned(16))) = {0};
   pi_attn_status st = check_common(dummy, dummy, dummy, w_g, b_g, dummy, B, H, n, d, k_win, pi, S, dtype);
   if (st != PI_ATTN_OK) return st;
-  bool tc = false, split = false;
-  if ((st = fwd_route(n, d, k_win, pi, S, dtype, path, false, &tc, &split)) != PI_ATTN_OK) return st;
+  bool tc = false, split = false;  // (each chunk is a [1, chunk_heads, n, d] problem)
+  if ((st = fwd_route(host_chunk_heads(H, chunk_heads), n, d, k_win, pi, S, dtype, path, false, &tc, &split)) !=
+      PI_ATTN_OK)
+    return st;
   const long long need = pi_attn_fwd_host_workspace_bytes(B, H, n, d, dtype, chunk_heads);
   if (!workspace || reinterpret_cast<uintptr_t>(workspace) % 256 != 0)
     return fail(PI_ATTN_EINVAL, "workspace must be a 256-byte aligned device pointer");
@@ -555,7 +566,7 @@ pi_attn_status pi_attn_fwd_plan(int B, int H, int n, int d, int k_win, int pi, i
                                    k_win, pi, S, dtype);
   if (st != PI_ATTN_OK) return st;
   bool tc = false, split = false;
-  if ((st = fwd_route(n, d, k_win, pi, S, dtype, path, false, &tc, &split)) != PI_ATTN_OK) return st;
+  if ((st = fwd_route((long long)B * H, n, d, k_win, pi, S, dtype, path, false, &tc, &split)) != PI_ATTN_OK) return st;
   if (split) {  // the residue pass; the band-merge pass and / or the single pass over the ragged tail
     const int ntiles = (n + pia::tc::BM - 1) / pia::tc::BM, nmerge = pia::split_merge_tiles(n, pi);
     *launches = 1 + (nmerge > 0 ? 1 : 0) + (nmerge < ntiles ? 1 : 0);

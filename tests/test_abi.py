@@ -239,3 +239,15 @@ def test_host_entry_workspace_size_and_argument_checks(lib):
     assert call(nbytes=need - 1) == pia.PI_ATTN_EINVAL
     assert call(pi=0) == pia.PI_ATTN_EINVAL
     assert call(n=100, path=pia.PATHS["tc_split"], pi=128) == pia.PI_ATTN_EUNSUPPORTED  # n < pi
+
+
+def test_tensor_core_paths_refuse_more_than_65535_heads_before_any_launch(lib):
+    # the tensor-core grids take (b, h) as their y dimension: an explicit tensor-core path refuses
+    # B*H > 65535 up front; the automatic choice takes the CUDA-core kernel (the plan shows it)
+    args = [FAKE] * 7 + [2, 40000, 256, 64, 16, 32, 2, pia.PI_ATTN_BF16]
+    for path in ("tc", "tc_fused", "tc_split"):
+        assert lib.pi_attn_fwd_ex(*args, pia.PATHS[path], None) == pia.PI_ATTN_EUNSUPPORTED
+        assert b"65535" in lib.pi_attn_last_error()
+    assert pia.pi_attn_fwd_plan(2, 40000, 256, 64, 16, 32, 2, "bf16", "auto") == (1, 0)
+    assert lib.pi_attn_fwd_shard(*([FAKE] * 7), 2, 40000, 128, 256, 128, 0, 64, 16, 32, 2, pia.PI_ATTN_BF16,
+                                 None) == pia.PI_ATTN_EUNSUPPORTED
