@@ -492,6 +492,26 @@ def run_gpu(args):
 
         e2e_how = ("pi_attn_fwd_host: pinned host q, k, v in, out and lse back, in chunks of heads whose copies "
                    "overlap the kernels")
+    elif w.kind == "backward":
+        # the host-buffer backward: q, k, v, dO in and dq, dk, dv back in chunks of heads whose copies
+        # overlap the kernels; the gate parameters in first, their gradients back last
+        src = {name: h for name, (_, h) in zip(names, pairs)}
+        hin = {x: src[x].view(torch.bfloat16) if w.dtype == "bf16" else src[x] for x in ("q", "k", "v", "dO")}
+        params = [(t[x], src[x]) for x in ("w_g", "b_g")]
+        host_grads = (backs[0][1], backs[1][1], backs[2][1], grads[3], grads[4])
+        ws_host = torch.empty(pia.load().pi_attn_bwd_host_workspace_bytes(
+            w.B, w.H, w.n, w.d, pia._dtype_code(t["q"]), pia.BWD_PATHS[bwd_path], 0), dtype=torch.uint8, device=device)
+
+        def e2e_step():  # noqa: F811
+            for dst, src_ in params:
+                dst.copy_(src_, non_blocking=True)
+            pia.pi_attn_bwd_host(hin["q"], hin["k"], hin["v"], t["w_g"], t["b_g"], hin["dO"], w.k, w.pi, w.S,
+                                 bidir=w.bidir, grads=host_grads, path=bwd_path, workspace=ws_host)
+            for src_, dst in backs[3:]:
+                dst.copy_(src_, non_blocking=True)
+
+        e2e_how = ("pi_attn_bwd_host: pinned host q, k, v, dO in, dq, dk, dv back, in chunks of heads whose copies "
+                   "overlap the kernels")
 
     for _ in range(2):
         e2e_step()

@@ -20,12 +20,12 @@
  *   - dtype names the storage type of q, k, v, caches and out: PI_ATTN_F32 (fp32) or PI_ATTN_BF16
  *     (bfloat16).  Arithmetic is fp32 (bf16 products on tensor cores accumulate in fp32); out is
  *     rounded once, to nearest even, into dtype.
- *   - All pointers are DEVICE pointers owned by the caller (pi_attn_fwd_host takes host buffers
- *     instead); the library keeps no reference after the call returns and holds no memory
+ *   - All pointers are DEVICE pointers owned by the caller (pi_attn_fwd_host and pi_attn_bwd_host
+ *     take host buffers instead); the library keeps no reference after the call returns and holds no memory
  *     allocation of its own between calls, with two exceptions stated at their entry points: the
  *     fixed device array of the decode for callers that cannot allocate, and the streams and
  *     events it creates once per device, on first use, for the tensor-core backward and the
- *     host-buffer prefill (kept until the process exits).  Tensor pointers must be 16-byte aligned
+ *     host-buffer entry points (kept until the process exits).  Tensor pointers must be 16-byte aligned
  *     and d * sizeof(dtype) a multiple of 16 bytes.
  *   - `stream` is a cudaStream_t (NULL: the legacy default stream).  Calls only enqueue work: they
  *     are asynchronous and stream-ordered.  Argument errors are returned synchronously and then
@@ -260,6 +260,30 @@ pi_attn_status pi_attn_bwd_ex(const void* q, const void* k, const void* v, const
                               const void* dout, float* dq, float* dk, float* dv, float* dw_g, float* db_g, int B,
                               int H, int n, int d, int k_win, int pi, int S, pi_attn_dtype dtype, int bidir,
                               pi_attn_bwd_path path, void* workspace, long long workspace_bytes, void* stream);
+
+/* pi_attn_bwd_ex over inputs and gradients in HOST memory, as a pipeline of chunks of heads (as
+ * pi_attn_fwd_host does for the prefill).  A chunk is chunk_heads heads of every b (0 = about a
+ * thirty-second of H), so the gate gradients of its heads are complete within it; its q, k, v and
+ * dout are copied in, its gradients computed by pi_attn_bwd_ex on `stream` (the same kernels and
+ * bits as a pi_attn_bwd_ex call on device copies of the same inputs) and dq, dk, dv copied out,
+ * the copies of neighbouring chunks overlapping each chunk's kernels on the library's two copy
+ * streams.
+ *   q, k, v, dout  HOST [B, H, n, d] in dtype, read only (page-locked for the copies to overlap)
+ *   dq, dk, dv     HOST fp32 [B, H, n, d]
+ *   w_g, b_g       DEVICE, as for pi_attn_bwd; dw_g, db_g DEVICE fp32 [H, d] and [H]
+ *   workspace      DEVICE, 256-byte aligned, pi_attn_bwd_host_workspace_bytes(B, H, n, d, dtype,
+ *                  path, chunk_heads) bytes, owned by the caller
+ * Ordering as for pi_attn_fwd_host: the gradients are on the host once `stream` has been
+ * synchronized.  Errors as pi_attn_bwd_ex, plus PI_ATTN_EINVAL for a NULL host pointer, a negative
+ * chunk_heads or a workspace that is missing, misaligned or too small. */
+pi_attn_status pi_attn_bwd_host(const void* q, const void* k, const void* v, const float* w_g, const float* b_g,
+                                const void* dout, float* dq, float* dk, float* dv, float* dw_g, float* db_g, int B,
+                                int H, int n, int d, int k_win, int pi, int S, pi_attn_dtype dtype, int bidir,
+                                pi_attn_bwd_path path, int chunk_heads, void* workspace, long long workspace_bytes,
+                                void* stream);
+/* Device workspace bytes pi_attn_bwd_host needs; -1 for invalid arguments. */
+long long pi_attn_bwd_host_workspace_bytes(int B, int H, int n, int d, pi_attn_dtype dtype, pi_attn_bwd_path path,
+                                           int chunk_heads);
 
 /* Decode over a compact ring cache (constant memory per sequence, constant-time update).  Cited
  * passage: "Execution & Scheduling" -- caches updated in constant time at inference.  Position j of

@@ -51,6 +51,9 @@ SIGNATURES = {
     # as pi_attn_bwd plus the kernel choice before the workspace
     "pi_attn_bwd_ex": (_i32, [_vp] * 11 + [_i32] * 10 + [_vp, ctypes.c_longlong, _vp]),
     "pi_attn_bwd_workspace_bytes_ex": (ctypes.c_longlong, [_i32] * 6),
+    # as pi_attn_bwd_ex (q k v dout dq dk dv on the host) plus chunk_heads before the workspace
+    "pi_attn_bwd_host": (_i32, [_vp] * 11 + [_i32] * 11 + [_vp, ctypes.c_longlong, _vp]),
+    "pi_attn_bwd_host_workspace_bytes": (ctypes.c_longlong, [_i32] * 7),
     # as pi_attn_decode, capacity in place of n_cache
     "pi_attn_decode_ring": (_i32, [_vp] * 8 + [_i32] * 8 + [_vp]),
     # kcache vcache k_new v_new cache_len, B H capacity d dtype ring, stream
@@ -215,6 +218,33 @@ def pi_attn_fwd_host(q, k, v, w_g, b_g, k_win: int, pi: int, S: int, out=None, l
                                  _stream(stream))
     _raise(st)
     return out, lse
+
+
+def pi_attn_bwd_host(q, k, v, w_g, b_g, dout, k_win: int, pi: int, S: int, *, bidir: bool = False, grads=None,
+                     path: str = "auto", chunk_heads: int = 0, workspace=None, stream=None):
+    """Gradients with q, k, v, dout (torch CPU tensors; pinned for the copies to overlap) and dq, dk,
+    dv (fp32, pinned, allocated when grads is None) in host memory; w_g, b_g and dw_g, db_g on the
+    device: pi_attn_bwd_host, a pipeline of chunks of chunk_heads heads.  Returns (dq, dk, dv, dw_g,
+    db_g); the host gradients are complete once the stream has been synchronized."""
+    import torch
+    B, H, n, d = q.shape
+    if grads is None:
+        grads = tuple(torch.empty((B, H, n, d), dtype=torch.float32).pin_memory() for _ in range(3)) + (
+            torch.empty((H, d), dtype=torch.float32, device=w_g.device),
+            torch.empty((H,), dtype=torch.float32, device=w_g.device))
+    dq, dk, dv, dw, db = grads
+    dt = _dtype_code(q)
+    if workspace is None:
+        nbytes = load().pi_attn_bwd_host_workspace_bytes(B, H, n, d, dt, BWD_PATHS[path], chunk_heads)
+        if nbytes < 0:
+            raise ValueError(f"invalid sizes for pi_attn_bwd_host: {tuple(q.shape)}, chunk_heads={chunk_heads}")
+        workspace = torch.empty(nbytes, dtype=torch.uint8, device=w_g.device)
+    st = load().pi_attn_bwd_host(_hptr(q), _hptr(k), _hptr(v), _ptr(w_g), _ptr(b_g), _hptr(dout), _hptr(dq),
+                                 _hptr(dk), _hptr(dv), _ptr(dw), _ptr(db), B, H, n, d, k_win, pi, S, dt, int(bidir),
+                                 BWD_PATHS[path], chunk_heads, _ptr(workspace),
+                                 workspace.numel() * workspace.element_size(), _stream(stream))
+    _raise(st)
+    return dq, dk, dv, dw, db
 
 
 def pi_attn_fwd_plan(B: int, H: int, n: int, d: int, k_win: int, pi: int, S: int, dtype: str = "bf16",

@@ -720,14 +720,9 @@ long long pi_attn_bwd_workspace_bytes_ex(int B, int H, int n, int d, pi_attn_dty
   return bwd_ws_bytes(B, H, n, d, tc);
 }
 
-pi_attn_status pi_attn_bwd_ex(const void* q, const void* k, const void* v, const float* w_g, const float* b_g,
-                              const void* dout, float* dq, float* dk, float* dv, float* dw_g, float* db_g, int B,
-                              int H, int n, int d, int k_win, int pi, int S, pi_attn_dtype dtype, int bidir,
-                              pi_attn_bwd_path path, void* workspace, long long workspace_bytes, void* stream) {
-  pi_attn_status st = check_common(q, k, v, w_g, b_g, dout, B, H, n, d, k_win, pi, S, dtype);
-  if (st != PI_ATTN_OK) return st;
-  if (!dq || !dk || !dv || !dw_g || !db_g) return fail(PI_ATTN_EINVAL, "null gradient pointer");
-  if (!aligned16(dq) || !aligned16(dk) || !aligned16(dv)) return fail(PI_ATTN_EINVAL, "dq, dk, dv must be 16-byte aligned");
+// The backward's kernel choice and the checks it implies, before anything is enqueued.
+static pi_attn_status bwd_route(int B, int H, int n, int d, int k_win, int pi, int S, pi_attn_dtype dtype, int bidir,
+                                pi_attn_bwd_path path, bool* tc, bool* split) {
   if (path < PI_ATTN_BWD_AUTO || path > PI_ATTN_BWD_TC_SPLIT)
     return fail(PI_ATTN_EINVAL, "unknown backward path %d", (int)path);
   const bool tc_ok = dtype == PI_ATTN_BF16 && (d == 64 || d == 128);
@@ -739,9 +734,26 @@ pi_attn_status pi_attn_bwd_ex(const void* q, const void* k, const void* v, const
     return fail(PI_ATTN_EUNSUPPORTED, "the split backward covers the causal rule only");
   if (path == PI_ATTN_BWD_TC_SPLIT && !pia::tc_split_applies(n, k_win, pi, S))
     return fail(PI_ATTN_EUNSUPPORTED, "split backward needs n %% pi == 0 and at least one skip outside the window");
-  const bool tc = want_tc || (path == PI_ATTN_BWD_AUTO && tc_ok);
-  const bool split = tc && !bidir && (path == PI_ATTN_BWD_TC_SPLIT ||
-                                      (path != PI_ATTN_BWD_TC_FUSED && pia::tc_split_preferred(n, k_win, pi, S)));
+  *tc = want_tc || (path == PI_ATTN_BWD_AUTO && tc_ok);
+  *split = *tc && !bidir && (path == PI_ATTN_BWD_TC_SPLIT ||
+                             (path != PI_ATTN_BWD_TC_FUSED && pia::tc_split_preferred(n, k_win, pi, S)));
+  const long long tiles = ((long long)n + pia::kBwdRows - 1) / pia::kBwdRows;
+  if (tiles > 0x7fffffffLL || (long long)B * H > 65535) return fail(PI_ATTN_EINVAL, "grid too large");
+  const long long nchunks = *tc ? tc_gate_chunks(B, n) : gate_chunks(B, n);
+  if (nchunks > 0x7fffffffLL || H > 65535) return fail(PI_ATTN_EINVAL, "too many rows per head for the gate sums");
+  return ok();
+}
+
+pi_attn_status pi_attn_bwd_ex(const void* q, const void* k, const void* v, const float* w_g, const float* b_g,
+                              const void* dout, float* dq, float* dk, float* dv, float* dw_g, float* db_g, int B,
+                              int H, int n, int d, int k_win, int pi, int S, pi_attn_dtype dtype, int bidir,
+                              pi_attn_bwd_path path, void* workspace, long long workspace_bytes, void* stream) {
+  pi_attn_status st = check_common(q, k, v, w_g, b_g, dout, B, H, n, d, k_win, pi, S, dtype);
+  if (st != PI_ATTN_OK) return st;
+  if (!dq || !dk || !dv || !dw_g || !db_g) return fail(PI_ATTN_EINVAL, "null gradient pointer");
+  if (!aligned16(dq) || !aligned16(dk) || !aligned16(dv)) return fail(PI_ATTN_EINVAL, "dq, dk, dv must be 16-byte aligned");
+  bool tc = false, split = false;
+  if ((st = bwd_route(B, H, n, d, k_win, pi, S, dtype, bidir, path, &tc, &split)) != PI_ATTN_OK) return st;
   const long long rows = (long long)B * H * n;
   const long long need = bwd_ws_bytes(B, H, n, d, tc);
   if (workspace) {
@@ -750,9 +762,7 @@ pi_attn_status pi_attn_bwd_ex(const void* q, const void* k, const void* v, const
       return fail(PI_ATTN_EINVAL, "workspace of %lld bytes, the backward needs %lld", workspace_bytes, need);
   }
   const long long tiles = ((long long)n + pia::kBwdRows - 1) / pia::kBwdRows;
-  if (tiles > 0x7fffffffLL || (long long)B * H > 65535) return fail(PI_ATTN_EINVAL, "grid too large");
   const long long nchunks = tc ? tc_gate_chunks(B, n) : gate_chunks(B, n);
-  if (nchunks > 0x7fffffffLL || H > 65535) return fail(PI_ATTN_EINVAL, "too many rows per head for the gate sums");
   cudaStream_t s = as_stream(stream);
   void* scratch = workspace;
   cudaError_t e = cudaSuccess;
@@ -873,6 +883,93 @@ pi_attn_status pi_attn_bwd_ex(const void* q, const void* k, const void* v, const
   cudaError_t e2 = workspace ? cudaSuccess : cudaFreeAsync(scratch, s);
   if (e != cudaSuccess) return cuda_fail(e, why);
   if (e2 != cudaSuccess) return cuda_fail(e2, "backward scratch release");
+  return ok();
+}
+
+long long pi_attn_bwd_host_workspace_bytes(int B, int H, int n, int d, pi_attn_dtype dtype, pi_attn_bwd_path path,
+                                           int chunk_heads) {
+  if (B < 1 || H < 1 || n < 1 || d < 1 || chunk_heads < 0 || (dtype != PI_ATTN_F32 && dtype != PI_ATTN_BF16) ||
+      path < PI_ATTN_BWD_AUTO || path > PI_ATTN_BWD_TC_SPLIT)
+    return -1;
+  const int hc = host_chunk_heads(H, chunk_heads);
+  const long long per = (long long)B * hc * n * d;
+  const long long set = 4 * round256(per * (long long)elem_size(dtype)) + 3 * round256(per * 4);
+  return kHostSets * set + round256(pi_attn_bwd_workspace_bytes_ex(B, hc, n, d, dtype, path));
+}
+
+pi_attn_status pi_attn_bwd_host(const void* q, const void* k, const void* v, const float* w_g, const float* b_g,
+                                const void* dout, float* dq, float* dk, float* dv, float* dw_g, float* db_g, int B,
+                                int H, int n, int d, int k_win, int pi, int S, pi_attn_dtype dtype, int bidir,
+                                pi_attn_bwd_path path, int chunk_heads, void* workspace, long long workspace_bytes,
+                                void* stream) {
+  if (!q || !k || !v || !dout || !dq || !dk || !dv) return fail(PI_ATTN_EINVAL, "null host tensor pointer");
+  if (!w_g || !b_g || !dw_g || !db_g) return fail(PI_ATTN_EINVAL, "null gate parameter or gradient pointer");
+  if (chunk_heads < 0) return fail(PI_ATTN_EINVAL, "chunk_heads must be >= 0 (got %d)", chunk_heads);
+  static const char dummy[16] __attribute__((aligned(16))) = {0};
+  pi_attn_status st = check_common(dummy, dummy, dummy, w_g, b_g, dummy, B, H, n, d, k_win, pi, S, dtype);
+  if (st != PI_ATTN_OK) return st;
+  const int hc = host_chunk_heads(H, chunk_heads);
+  bool tc = false, split = false;  // (each chunk is a [B, chunk_heads, n, d] problem)
+  if ((st = bwd_route(B, hc, n, d, k_win, pi, S, dtype, bidir, path, &tc, &split)) != PI_ATTN_OK) return st;
+  const long long need = pi_attn_bwd_host_workspace_bytes(B, H, n, d, dtype, path, chunk_heads);
+  if (!workspace || reinterpret_cast<uintptr_t>(workspace) % 256 != 0)
+    return fail(PI_ATTN_EINVAL, "workspace must be a 256-byte aligned device pointer");
+  if (workspace_bytes < need)
+    return fail(PI_ATTN_EINVAL, "workspace of %lld bytes, the call needs %lld", workspace_bytes, need);
+  const size_t elem = elem_size(dtype);
+  const long long per = (long long)B * hc * n * d;
+  const long long ti = round256(per * (long long)elem), to = round256(per * 4), set_bytes = 4 * ti + 3 * to;
+  char* const ws = static_cast<char*>(workspace);
+  void* const bwd_ws = ws + kHostSets * set_bytes;
+  const long long bwd_ws_bytes_chunk = round256(pi_attn_bwd_workspace_bytes_ex(B, hc, n, d, dtype, path));
+  cudaStream_t s = as_stream(stream);
+
+  std::lock_guard<std::mutex> lock(g_pipe_mu);
+  HostPipe* hp = nullptr;
+  cudaError_t e = host_pipe(&hp);
+  if (e != cudaSuccess) return cuda_fail(e, "copy streams");
+  if ((e = cudaEventRecord(hp->start, s)) != cudaSuccess || (e = cudaStreamWaitEvent(hp->in, hp->start, 0)) != cudaSuccess ||
+      (e = cudaStreamWaitEvent(hp->out, hp->start, 0)) != cudaSuccess)
+    return cuda_fail(e, "copy streams");
+  // a chunk holds heads [h0, h0 + h) of every b: in host memory B slabs of h heads, H heads apart
+  const size_t head_in = (size_t)n * d * elem, head_out = (size_t)n * d * 4;
+  int c = 0;
+  for (int h0 = 0; h0 < H && st == PI_ATTN_OK && e == cudaSuccess; h0 += hc, ++c) {
+    const int h = hc < H - h0 ? hc : H - h0, set = c % kHostSets;
+    char* const base = ws + set * set_bytes;
+    void* din[4] = {base, base + ti, base + 2 * ti, base + 3 * ti};  // q, k, v, dout
+    float* dgr[3] = {reinterpret_cast<float*>(base + 4 * ti), reinterpret_cast<float*>(base + 4 * ti + to),
+                     reinterpret_cast<float*>(base + 4 * ti + 2 * to)};  // dq, dk, dv
+    const void* hin[4] = {q, k, v, dout};
+    float* hgr[3] = {dq, dk, dv};
+    if (c >= kHostSets && (e = cudaStreamWaitEvent(hp->in, hp->freed[set], 0)) != cudaSuccess) break;
+    for (int x = 0; x < 4 && e == cudaSuccess; ++x)
+      e = cudaMemcpy2DAsync(din[x], h * head_in, static_cast<const char*>(hin[x]) + h0 * head_in, (size_t)H * head_in,
+                            h * head_in, B, cudaMemcpyHostToDevice, hp->in);
+    if (e != cudaSuccess || (e = cudaEventRecord(hp->loaded[set], hp->in)) != cudaSuccess ||
+        (e = cudaStreamWaitEvent(s, hp->loaded[set], 0)) != cudaSuccess)
+      break;
+    // the chunk as a [B, h, n, d] problem: its heads' gate parameters, and their gradients (every b
+    // is in the chunk, so the gate gradients of these heads are complete) straight into dw_g, db_g
+    st = pi_attn_bwd_ex(din[0], din[1], din[2], w_g + (long long)h0 * d, b_g + h0, din[3], dgr[0], dgr[1], dgr[2],
+                        dw_g + (long long)h0 * d, db_g + h0, B, h, n, d, k_win, pi, S, dtype, bidir, path, bwd_ws,
+                        bwd_ws_bytes_chunk, stream);
+    if (st != PI_ATTN_OK) break;
+    if ((e = cudaEventRecord(hp->computed[set], s)) != cudaSuccess ||
+        (e = cudaStreamWaitEvent(hp->out, hp->computed[set], 0)) != cudaSuccess)
+      break;
+    for (int x = 0; x < 3 && e == cudaSuccess; ++x)
+      e = cudaMemcpy2DAsync(reinterpret_cast<char*>(hgr[x]) + h0 * head_out, (size_t)H * head_out, dgr[x],
+                            h * head_out, h * head_out, B, cudaMemcpyDeviceToHost, hp->out);
+    if (e != cudaSuccess || (e = cudaEventRecord(hp->freed[set], hp->out)) != cudaSuccess) break;
+  }
+  cudaError_t ej = cudaEventRecord(hp->join_in, hp->in);
+  if (ej == cudaSuccess) ej = cudaStreamWaitEvent(s, hp->join_in, 0);
+  if (ej == cudaSuccess) ej = cudaEventRecord(hp->join_out, hp->out);
+  if (ej == cudaSuccess) ej = cudaStreamWaitEvent(s, hp->join_out, 0);
+  if (st != PI_ATTN_OK) return st;
+  if (e != cudaSuccess) return cuda_fail(e, "host-buffer chunk copies");
+  if (ej != cudaSuccess) return cuda_fail(ej, "joining the copy streams");
   return ok();
 }
 

@@ -251,3 +251,29 @@ def test_tensor_core_paths_refuse_more_than_65535_heads_before_any_launch(lib):
     assert pia.pi_attn_fwd_plan(2, 40000, 256, 64, 16, 32, 2, "bf16", "auto") == (1, 0)
     assert lib.pi_attn_fwd_shard(*([FAKE] * 7), 2, 40000, 128, 256, 128, 0, 64, 16, 32, 2, pia.PI_ATTN_BF16,
                                  None) == pia.PI_ATTN_EUNSUPPORTED
+
+
+def test_backward_host_entry_workspace_size_and_argument_checks(lib):
+    r = lambda x: (x + 255) // 256 * 256  # noqa: E731
+    B, H, n, d = 2, 16, 32768, 128
+    for chunk, hc in ((0, 1), (4, 4), (64, 16)):
+        per = B * hc * n * d
+        want = 3 * (4 * r(per * 2) + 3 * r(per * 4)) + \
+            r(lib.pi_attn_bwd_workspace_bytes_ex(B, hc, n, d, pia.PI_ATTN_BF16, pia.BWD_PATHS["tc"]))
+        assert lib.pi_attn_bwd_host_workspace_bytes(B, H, n, d, pia.PI_ATTN_BF16, pia.BWD_PATHS["tc"], chunk) == want
+    assert lib.pi_attn_bwd_host_workspace_bytes(1, 1, 1, 64, pia.PI_ATTN_BF16, 9, 0) == -1  # unknown path
+    assert lib.pi_attn_bwd_host_workspace_bytes(1, 1, 1, 64, pia.PI_ATTN_BF16, 0, -2) == -1
+    h = ctypes.c_void_p(0x1000)
+    ws = ctypes.c_void_p(0x10000)
+    need = lib.pi_attn_bwd_host_workspace_bytes(1, 2, 256, 64, pia.PI_ATTN_BF16, 0, 1)
+
+    def call(q=h, dw=h, chunk=1, w=ws, nbytes=need, path=0, bidir=0, n=256, pi=16):
+        return lib.pi_attn_bwd_host(q, h, h, h, h, h, h, h, h, dw, h, 1, 2, n, 64, 16, pi, 3, pia.PI_ATTN_BF16, bidir,
+                                    path, chunk, w, nbytes, None)
+    assert call(q=None) == pia.PI_ATTN_EINVAL
+    assert call(dw=None) == pia.PI_ATTN_EINVAL
+    assert call(chunk=-1) == pia.PI_ATTN_EINVAL
+    assert call(w=ctypes.c_void_p(0x10010)) == pia.PI_ATTN_EINVAL
+    assert call(nbytes=need - 1) == pia.PI_ATTN_EINVAL
+    assert call(path=pia.BWD_PATHS["tc_split"], bidir=1) == pia.PI_ATTN_EUNSUPPORTED
+    assert call(path=pia.BWD_PATHS["tc_split"], n=250) == pia.PI_ATTN_EUNSUPPORTED  # n % pi != 0

@@ -167,3 +167,29 @@ def test_host_entry_replays_as_a_cuda_graph_with_pinned_buffers():
         assert torch.equal(out.view(torch.int16), ref_out.view(torch.int16)), "out differs after a graph replay"
         assert torch.equal(lse, ref_lse), "lse differs after a graph replay"
     del g
+
+
+BWD_CASES = [  # B, H, n, d, k, pi, S, dtype, path, bidir, chunk_heads, pinned
+    (2, 3, 2048, 64, 100, 64, 12, "bf16", "tc_split", False, 2, True),   # chunks of 2 + 1 heads of both b
+    (1, 8, 4096, 64, 128, 64, 4, "bf16", "tc", False, 0, True),          # the bf16_n4k_bwd shape, 8 chunks
+    (1, 4, 1024, 64, 40, 32, 6, "bf16", "tc_fused", True, 3, False),     # bidirectional, pageable, ragged
+    (2, 2, 300, 32, 20, 9, 5, "f32", "simt", False, 0, True),            # the fp32 CUDA-core backward
+]
+
+
+@pytest.mark.parametrize("case", BWD_CASES, ids=[f"{c[7]}-{c[8]}-bidir{int(c[9])}-chunk{c[10]}" for c in BWD_CASES])
+def test_backward_host_entry_gives_the_device_entrys_bits(case):
+    B, H, n, d, k, pi, S, dtype, path, bidir, chunk, pinned = case
+    inp = _problem(B, H, n, d, dtype, seed=7 * H + n)
+    inp["dO"] = ps.normal((B, H, n, d), seed=5, stream=6, dtype=dtype)
+    dev = {x: _host(inp[x], dtype, False).cuda() for x in ("q", "k", "v", "dO")}
+    wg, bg = torch.from_numpy(inp["w_g"]).cuda(), torch.from_numpy(inp["b_g"]).cuda()
+    ref = [t.cpu() for t in pia.pi_attn_bwd(dev["q"], dev["k"], dev["v"], wg, bg, dev["dO"], k, pi, S, bidir=bidir,
+                                             path=path)]
+    host = {x: _host(inp[x], dtype, pinned) for x in ("q", "k", "v", "dO")}
+    got = pia.pi_attn_bwd_host(host["q"], host["k"], host["v"], wg, bg, host["dO"], k, pi, S, bidir=bidir, path=path,
+                               chunk_heads=chunk)
+    torch.cuda.synchronize()
+    pia.pi_attn_check()
+    for name, x, y in zip(("dq", "dk", "dv", "dw_g", "db_g"), got, ref):
+        assert torch.equal(x.cpu(), y), f"{name} differs from pi_attn_bwd_ex"
