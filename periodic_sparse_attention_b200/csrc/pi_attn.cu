@@ -141,7 +141,7 @@ cudaError_t side_join(SideStream& ss, cudaStream_t s) {
   return e == cudaSuccess ? cudaStreamWaitEvent(s, ss.join, 0) : e;
 }
 
-// ---- the host-buffer prefill's copy streams (pi_attn_fwd_host) ----------------------------------
+// ---- the host-buffer entry points' copy streams (pi_attn_fwd_host, pi_attn_bwd_host) ------------------
 // Per device: a stream for the copies in, one for the copies out, and events for the three
 // rotating chunk buffers of the workspace (loaded, computed, free again) plus two for the joins.
 // A call holds the lock for its whole enqueue sequence: its events are recorded and waited on in
