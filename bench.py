@@ -730,7 +730,8 @@ def run_shard(args):
         "e2e": {"value": tokens / (e_ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": int(h2d_all),
                 "d2h_bytes_per_step": int(d2h_all), "ms_per_step": e_ms},
         "gpu_launches": args.steps,  # one shard kernel a step per rank (the exchange is NCCL's)
-        "clocks": clocks.summary(), "path": "shard (single pass over halo + own rows)",
+        "clocks": clocks.summary(),
+        "path": "shard (the split path where the shard's rows and halo start on whole periods, else the single pass)",
         "timing": "eager step: halo exchange + shard kernel, CUDA events, max over ranks",
         "halo_rows_max": int(halo), "kernel_source_sha": source_hash(KERNEL_FILES["prefill"]),
     }

@@ -105,11 +105,16 @@ pi_attn_status pi_attn_fwd_ws(const void* q, const void* k, const void* v, const
  * the shards before it and nothing from the shards after it.
  *   q, out  [B, H, n_q, d]   sequence rows row0 .. row0 + n_q - 1 (lse [B, H, n_q], may be NULL)
  *   k, v    [B, H, n_kv, d]  sequence rows kv0 .. kv0 + n_kv - 1: the halo, then the shard's rows
- * Every row is computed exactly as pi_attn_fwd computes that row of the whole sequence.
+ * Where row0 and kv0 are whole periods (multiples of pi) and a sequence of n_q rows would take the
+ * split path, the shard takes it too (the residue-class pass over its whole periods, with its
+ * scratch of B*H*n_q*(2d + 4) bytes from cudaMallocAsync on `stream`, then the window pass);
+ * otherwise the single tensor-core pass, which allocates nothing.  Either way every row is computed
+ * by the same kernels as the whole sequence's call on that path; the single pass gives it the same
+ * bits, the split path up to the rounding of the tiles it groups the row with.
  * PI_ATTN_EINVAL unless kv0 <= max(0, row0 - max(k_win, S*pi)) (the halo reaches every key read)
  * and kv0 + n_kv >= row0 + n_q (the k/v rows reach the shard's last row), plus the checks of
- * pi_attn_fwd; bf16 with d in {64, 128} (the single tensor-core pass), else PI_ATTN_EUNSUPPORTED.
- * Allocates nothing; all pointers are device pointers owned by the caller. */
+ * pi_attn_fwd; bf16 with d in {64, 128}, else PI_ATTN_EUNSUPPORTED.  All pointers are device
+ * pointers owned by the caller. */
 pi_attn_status pi_attn_fwd_shard(const void* q, const void* k, const void* v, const float* w_g, const float* b_g,
                                  void* out, float* lse, int B, int H, int n_q, int n_kv, long long row0,
                                  long long kv0, int d, int k_win, int pi, int S, pi_attn_dtype dtype, void* stream);

@@ -418,13 +418,16 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm<D>) fwd_tc_kernel(const _
   if (MODE == kResidue) {
     res = blockIdx.x % prm.pi;
     q0 = (long long)(blockIdx.x / prm.pi) * BM;
-    // keys of row t: t - S .. t - m0 (the skips of sequence row t*pi + res)
-    walk.init_residue(q0, prm.T, BM, prm.S, m0, prm.bidir != 0);
+    // keys of row t: t - S .. t - m0 (the skips of sequence row t*pi + res).  The walk runs in
+    // periods of the whole sequence: a shard's rows start at period row0 / pi (whole periods)
+    walk.init_residue(q0 + prm.row0 / prm.pi, prm.T + prm.row0 / prm.pi, BM, prm.S, m0, prm.bidir != 0);
   } else {
     q0 = (long long)(prm.tile0 + (int)blockIdx.x) * BM;
     walk.init(prm.row0 + q0, prm.row0 + prm.n, BM, prm.kwin, prm.pi, MODE == kFused ? prm.S : 0, prm.bidir != 0);
   }
   const int view_rows = MODE == kResidue ? prm.T : prm.n;
+  // the k/v buffer's first row, in the walk's units (sequence rows; kResidue: periods)
+  const long long kv_off = MODE == kResidue ? prm.kv0 / prm.pi : prm.kv0;
   // every thread walks the tiles with its own cursor (no division per step); thread 0 takes the
   // first tile at barrier init and goes on from there as the producer
   TileCursor cur;
@@ -487,9 +490,9 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm<D>) fwd_tc_kernel(const _
     t_first = cur.next();
     if (t_first >= 0) {
       mbar_expect_tx(bar_kfull(0), L::kKVBytes);
-      load_tile(sK, &tmk, bar_kfull(0), (long long)t_first * BN - prm.kv0, BN);
+      load_tile(sK, &tmk, bar_kfull(0), (long long)t_first * BN - kv_off, BN);
       mbar_expect_tx(bar_vfull(0), L::kKVBytes);
-      load_tile(sV, &tmv, bar_vfull(0), (long long)t_first * BN - prm.kv0, BN);
+      load_tile(sV, &tmv, bar_vfull(0), (long long)t_first * BN - kv_off, BN);
     }
   }
   if (warp == 1) {  // TMEM: S buffer b in columns [BN b, BN b + BN), O in [BN NSB, BN NSB + D)
@@ -513,11 +516,11 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm<D>) fwd_tc_kernel(const _
         const int s = nk % NSTAGE, use = nk / NSTAGE;
         if (use > 0 && !mbar_wait(bar_kempty(s), (use - 1) & 1, abort_flag)) break;
         mbar_expect_tx(bar_kfull(s), kKV);
-        load_tile(sK + s * kKV, &tmk, bar_kfull(s), (long long)t * BN - prm.kv0, BN);
+        load_tile(sK + s * kKV, &tmk, bar_kfull(s), (long long)t * BN - kv_off, BN);
         ++nk;
         if (use > 0 && !mbar_wait(bar_vempty(s), (use - 1) & 1, abort_flag)) break;
         mbar_expect_tx(bar_vfull(s), kKV);
-        load_tile(sV + s * kKV, &tmv, bar_vfull(s), (long long)t * BN - prm.kv0, BN);
+        load_tile(sV + s * kKV, &tmv, bar_vfull(s), (long long)t * BN - kv_off, BN);
         ++nv;
       }
       // kBandMerge: the 128-row tile of skip partials goes into the K region as soon as the last
@@ -616,18 +619,20 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm<D>) fwd_tc_kernel(const _
     const int q4 = warp & 3;                  // TMEM lane quarter this warp may access
     const int r = q4 * 32 + lane;             // query row within the tile
     const long long qi = q0 + r;              // row in the view
-    const long long i = MODE == kResidue ? qi * prm.pi + res : prm.row0 + qi;  // row in the sequence
+    const long long i = MODE == kResidue ? qi * prm.pi + res : prm.row0 + qi;  // row in the sequence (kResidue:
+                                                                               // in the q buffer)
+    const long long qg = MODE == kResidue ? qi + prm.row0 / prm.pi : qi;      // kResidue: period of the row
     const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
     // kBandMerge: this row's skip-partial lse (written by the residue pass), loaded now so that
     // the epilogue does not wait for it
     const float skip_lse_row =
-        MODE == kBandMerge && qi < view_rows ? prm.skip_lse[(long long)bh * prm.n + i] : 0.f;
+        MODE == kBandMerge && qi < view_rows ? prm.skip_lse[(long long)bh * prm.n + qi] : 0.f;
 
     // the row's keys, tile by tile: window columns from the window's bounds, skip columns from
     // the row's own skip keys taken in order (the residue pass: keys qi - S .. qi - m0 of its
     // view, no skips).  Set up while the Q tile is still in flight.
-    const long long w_lo = MODE == kResidue ? (qi - prm.S > 0 ? qi - prm.S : 0) : (i - prm.kwin > 0 ? i - prm.kwin : 0);
-    const long long w_hi = MODE == kResidue ? qi - m0
+    const long long w_lo = MODE == kResidue ? (qg - prm.S > 0 ? qg - prm.S : 0) : (i - prm.kwin > 0 ? i - prm.kwin : 0);
+    const long long w_hi = MODE == kResidue ? qg - m0
                            : prm.bidir ? (i + prm.kwin < prm.n - 1 ? i + prm.kwin : prm.n - 1)
                                        : i;
     // kResidue, bidirectional: the forward band qi + m0 .. qi + S of the view, carried as skip bits
@@ -1117,17 +1122,28 @@ inline bool tc_split_preferred(int n, int kwin, int pi, int S, bool fwd = false,
   return pi >= tc::BN && nskip > 2 * band_tiles;
 }
 
+// A shard takes the split path where a whole sequence of its length would, and its rows and its
+// k/v rows start on whole periods (the residue views of its buffers align with the sequence's).
+inline bool shard_split_applies(int n_q, long long row0, long long kv0, int kwin, int pi, int S) {
+  return row0 % pi == 0 && kv0 % pi == 0 && tc_split_preferred(n_q, kwin, pi, S, true, false);
+}
+
 template <int D>
 cudaError_t launch_fwd_tc_d(const void* q, const void* k, const void* v, const float* w_g, const float* b_g,
                             void* out, float* lse, int B, int H, int n, int kwin, int pi, int S, bool split,
                             bool bidir, void* workspace, cudaStream_t st, const char** why,
                             const void* dout = nullptr, float* Dout = nullptr, float* lse2 = nullptr,
-                            float* bl2 = nullptr, float* bp2 = nullptr) {
+                            float* bl2 = nullptr, float* bp2 = nullptr, long long row0 = 0, long long kv0 = 0,
+                            int n_kv = 0) {
+  // A shard (row0, kv0, n_kv given): q and out hold sequence rows row0 .., k and v the n_kv
+  // sequence rows kv0 ..; the split needs row0 and kv0 on whole periods (the residue views of the
+  // two buffers then align).  Otherwise k and v hold the same n rows as q.
   using L = tc::Smem<D>;
   CUtensorMap mq, mk, mv;
   const int BH = B * H;
-  if (!tc::make_map(&mq, q, BH, n, D, tc::BM) || !tc::make_map(&mk, k, BH, n, D, tc::BN) ||
-      !tc::make_map(&mv, v, BH, n, D, tc::BN)) {
+  if (n_kv <= 0) n_kv = n;
+  if (!tc::make_map(&mq, q, BH, n, D, tc::BM) || !tc::make_map(&mk, k, BH, n_kv, D, tc::BN) ||
+      !tc::make_map(&mv, v, BH, n_kv, D, tc::BN)) {
     *why = "cuTensorMapEncodeTiled failed";
     return cudaErrorInvalidValue;
   }
@@ -1147,8 +1163,8 @@ cudaError_t launch_fwd_tc_d(const void* q, const void* k, const void* v, const f
   p.scale_log2 = (float)(1.0 / std::sqrt((double)D)) * kLog2e;
   p.bidir = bidir ? 1 : 0;
   p.tile0 = 0;
-  p.row0 = 0;
-  p.kv0 = 0;
+  p.row0 = row0;
+  p.kv0 = kv0;
   p.dout = (const __nv_bfloat16*)dout;
   p.Dout = Dout;
   p.lse2 = lse2;
@@ -1168,8 +1184,8 @@ cudaError_t launch_fwd_tc_d(const void* q, const void* k, const void* v, const f
     return cudaGetLastError();
   }
   CUtensorMap rq, rk, rv;
-  if (!tc::make_residue_map(&rq, q, BH, n, D, pi, tc::BM) || !tc::make_residue_map(&rk, k, BH, n, D, pi, tc::BN) ||
-      !tc::make_residue_map(&rv, v, BH, n, D, pi, tc::BN)) {
+  if (!tc::make_residue_map(&rq, q, BH, n, D, pi, tc::BM) || !tc::make_residue_map(&rk, k, BH, n_kv, D, pi, tc::BN) ||
+      !tc::make_residue_map(&rv, v, BH, n_kv, D, pi, tc::BN)) {
     *why = "cuTensorMapEncodeTiled (residue view) failed";
     return cudaErrorInvalidValue;
   }
@@ -1255,6 +1271,9 @@ cudaError_t launch_fwd_tc_shard_d(const void* q, const void* k, const void* v, c
   p.Dout = nullptr;
   p.lse2 = p.bl2 = p.bp2 = nullptr;
   cudaError_t e;
+  if (shard_split_applies(n_q, row0, kv0, kwin, pi, S))  // the residue pass and the window pass, as the whole
+    return launch_fwd_tc_d<D>(q, k, v, w_g, b_g, out, lse, B, H, n_q, kwin, pi, S, true, false, nullptr, st, why,
+                              nullptr, nullptr, nullptr, nullptr, nullptr, row0, kv0, n_kv);
   if ((e = tc::set_smem_attr<D, tc::kFused>()) != cudaSuccess) { *why = "cudaFuncSetAttribute"; return e; }
   const dim3 grid((unsigned)((n_q + tc::BM - 1) / tc::BM), (unsigned)BH);
   tc::fwd_tc_kernel<D, tc::kFused><<<grid, tc::kThreads, L::kAlloc, st>>>(mq, mk, mv, mo, mo, p);

@@ -58,6 +58,10 @@ def _run_shards(qt, kt, vt, wg, bg, n, world, kw, pi, S, halo_from_zero=False):
     (1, 3, 4096, 64, 128, 64, 4, 4),      # the bf16_n4k geometry in four shards
     (1, 1, 2500, 128, 256, 256, 8, 2),    # the bf16_n32k geometry, shorter
     (1, 2, 300, 64, 8, 16, 2, 5),         # short shards (60 rows)
+    # shards of whole periods with halos of whole periods: every rank takes the split path (the
+    # residue pass and the window pass with the shard's offsets)
+    (1, 2, 8192, 64, 128, 256, 16, 4),    # halos of 4096 rows, reaching two ranks back
+    (2, 2, 6144, 128, 256, 512, 8, 3),    # d = 128, halo to row 0
 ])
 def test_shards_match_the_oracle_on_the_whole_sequence(case):
     B, H, n, d, kw, pi, S, world = case
@@ -84,6 +88,22 @@ def test_one_shard_is_the_single_pass_forward(d):
     wg, bg = torch.from_numpy(w_g).cuda(), torch.from_numpy(b_g).cuda()
     o1, l1 = pia.pi_attn_fwd_shard(qt, kt, vt, wg, bg, kw, pi, S, 0, 0)
     o2, l2 = pia.pi_attn_fwd(qt, kt, vt, wg, bg, kw, pi, S, path="tc_fused")
+    pia.pi_attn_check()
+    assert torch.equal(o1.view(torch.int16), o2.view(torch.int16))
+    assert torch.equal(l1, l2)
+
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_a_whole_sequence_shard_takes_the_split_path(d):
+    # a shard that is the whole sequence, on a shape that takes the split path, runs the same
+    # launches as the whole-sequence forward: the same bits
+    B, H, n, kw, pi, S = 1, 2, 4096, 128, 256, 12
+    assert pia.pi_attn_fwd_plan(B, H, n, d, kw, pi, S, "bf16", "auto")[0] >= 2  # the split path
+    q, k, v, w_g, b_g = _inputs(B, H, n, d, seed=11)
+    qt, kt, vt = to_dev(q, "bf16"), to_dev(k, "bf16"), to_dev(v, "bf16")
+    wg, bg = torch.from_numpy(w_g).cuda(), torch.from_numpy(b_g).cuda()
+    o1, l1 = pia.pi_attn_fwd_shard(qt, kt, vt, wg, bg, kw, pi, S, 0, 0)
+    o2, l2 = pia.pi_attn_fwd(qt, kt, vt, wg, bg, kw, pi, S)
     pia.pi_attn_check()
     assert torch.equal(o1.view(torch.int16), o2.view(torch.int16))
     assert torch.equal(l1, l2)
