@@ -581,11 +581,12 @@ def run_gpu(args):
 def shard_plan(w, world: int, rank: int):
     """The sequence-sharded step's bookkeeping for one rank: its rows [s0, s1) of every (b, h), the
     first key row kv0 it reads (the halo from the ranks before it starts there), and the halo
-    pieces it receives and sends, (src, dst, g0, g1) as shard.halo_plan lists them."""
+    pieces it receives and sends, (src, dst, g0, g1) as shard.halo_plan lists them.  The blocks and
+    the halos start on whole periods (align = pi), so that every shard can take the split path."""
     from periodic_sparse_attention_b200 import shard
-    s0, s1 = shard.shard_bounds(w.n, world, rank)
-    kv0 = max(0, s0 - shard.reach(w.k, w.pi, w.S)) if s1 > s0 else s0
-    plan = shard.halo_plan(w.n, world, w.k, w.pi, w.S)
+    s0, s1 = shard.shard_bounds(w.n, world, rank, w.pi)
+    kv0 = shard.halo_start(s0, s1, w.k, w.pi, w.S, w.pi)
+    plan = shard.halo_plan(w.n, world, w.k, w.pi, w.S, w.pi)
     recv = [p for p in plan if p[1] == rank]
     send = [p for p in plan if p[0] == rank]
     return {"s0": s0, "s1": s1, "kv0": kv0, "recv": recv, "send": send,
@@ -633,7 +634,7 @@ def run_shard(args):
 
     def step():
         if world > 1:
-            k_ext, v_ext, kv = shard.exchange_halo(t["k"], t["v"], w.n, w.k, w.pi, w.S)
+            k_ext, v_ext, kv = shard.exchange_halo(t["k"], t["v"], w.n, w.k, w.pi, w.S, align=w.pi)
         else:
             k_ext, v_ext, kv = t["k"], t["v"], 0
         pia.pi_attn_fwd_shard(t["q"], k_ext.contiguous(), v_ext.contiguous(), t["w_g"], t["b_g"], w.k, w.pi, w.S, s0,

@@ -134,7 +134,7 @@ def _shard_rank_main(rank, world, port, out_dir):
     host = ps.prefill_rows(w, plan["s0"], plan["s1"], 0)
     k_loc = torch.from_numpy(host["k"].view(np.int16))
     v_loc = torch.from_numpy(host["v"].view(np.int16))
-    k_ext, v_ext, kv0 = shard.exchange_halo(k_loc, v_loc, w.n, w.k, w.pi, w.S)
+    k_ext, v_ext, kv0 = shard.exchange_halo(k_loc, v_loc, w.n, w.k, w.pi, w.S, align=w.pi)
     full = ps.prefill_inputs(w, 0)
     ok = (kv0 == plan["kv0"] and k_ext.shape[2] == plan["s1"] - kv0 and plan["halo_rows"] == plan["s0"] - kv0
           and np.array_equal(k_ext.numpy().view(np.uint16), full["k"][:, :, kv0:plan["s1"]])
@@ -150,5 +150,6 @@ def test_shard_step_plan_and_halo_two_gloo_ranks(tmp_path):
     mp.start_processes(_shard_rank_main, args=(2, port, str(tmp_path)), nprocs=2, start_method="spawn")
     res = [json.load(open(tmp_path / f"s{i}.json")) for i in range(2)]
     assert all(r["ok"] for r in res), res
-    assert res[0]["plan"] == {"s0": 0, "s1": 3000, "kv0": 0, "halo_rows": 0}
-    assert res[1]["plan"] == {"s0": 3000, "s1": 6000, "kv0": 3000 - 16 * 64, "halo_rows": 16 * 64}
+    # blocks of whole periods (pi = 64): 47 and 46 periods, the second taking the 48 rows past the last
+    assert res[0]["plan"] == {"s0": 0, "s1": 47 * 64, "kv0": 0, "halo_rows": 0}
+    assert res[1]["plan"] == {"s0": 47 * 64, "s1": 6000, "kv0": 47 * 64 - 16 * 64, "halo_rows": 16 * 64}

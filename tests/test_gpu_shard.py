@@ -36,13 +36,13 @@ def _inputs(B, H, n, d, seed):
     return q, k, v, w_g, b_g
 
 
-def _run_shards(qt, kt, vt, wg, bg, n, world, kw, pi, S, halo_from_zero=False):
+def _run_shards(qt, kt, vt, wg, bg, n, world, kw, pi, S, halo_from_zero=False, align=1):
     outs, lses = [], []
     for r in range(world):
-        s0, s1 = shard.shard_bounds(n, world, r)
+        s0, s1 = shard.shard_bounds(n, world, r, align)
         if s1 == s0:
             continue
-        kv0 = 0 if halo_from_zero else max(0, s0 - shard.reach(kw, pi, S))
+        kv0 = 0 if halo_from_zero else shard.halo_start(s0, s1, kw, pi, S, align)
         o, l = pia.pi_attn_fwd_shard(qt[:, :, s0:s1].contiguous(), kt[:, :, kv0:s1].contiguous(),
                                      vt[:, :, kv0:s1].contiguous(), wg, bg, kw, pi, S, s0, kv0)
         outs.append(o)
@@ -107,3 +107,17 @@ def test_a_whole_sequence_shard_takes_the_split_path(d):
     pia.pi_attn_check()
     assert torch.equal(o1.view(torch.int16), o2.view(torch.int16))
     assert torch.equal(l1, l2)
+
+
+def test_shards_on_whole_periods_take_the_split_path_and_match_the_oracle():
+    # three ranks on a sequence that is not a whole number of periods: blocks and halos aligned to
+    # whole periods (the layout bench.py --shard seq uses), so every rank takes the split path and
+    # the last rank's tail its single pass
+    B, H, n, d, kw, pi, S, world = 1, 2, 20 * 1024 + 300, 128, 512, 1024, 12, 3  # the last halo from row 2048
+    q, k, v, w_g, b_g = _inputs(B, H, n, d, seed=17)
+    qt, kt, vt = to_dev(q, "bf16"), to_dev(k, "bf16"), to_dev(v, "bf16")
+    wg, bg = torch.from_numpy(w_g).cuda(), torch.from_numpy(b_g).cuda()
+    out, lse = _run_shards(qt, kt, vt, wg, bg, n, world, kw, pi, S, align=pi)
+    ro, rl = oracle.fwd(q, k, v, w_g, b_g, kw, pi, S)[:2]
+    assert_close(metrics(from_dev(out).reshape(-1, d), ro.reshape(-1, d), lse.cpu().numpy().astype(np.float64).reshape(-1),
+                         rl.reshape(-1)), "bf16", "aligned shards")

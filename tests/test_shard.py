@@ -21,6 +21,31 @@ def test_shard_bounds_tile_the_sequence(n, world):
     assert max(sizes) - min(sizes) <= 1
 
 
+@pytest.mark.parametrize("n,world,align", [(131072, 3, 1024), (131072, 8, 1024), (6000, 4, 64), (100, 8, 16),
+                                           (5000, 3, 2048)])
+def test_aligned_shard_bounds_start_on_whole_units(n, world, align):
+    blocks = [shard.shard_bounds(n, world, r, align) for r in range(world)]
+    assert blocks[0][0] == 0 and blocks[-1][1] == n
+    for (a0, a1), (b0, b1) in zip(blocks, blocks[1:]):
+        assert a1 == b0
+    assert all(a % align == 0 for a, b in blocks)
+    units = [(b - a) // align for a, b in blocks[:-1]] + [(blocks[-1][1] - blocks[-1][0]) // align]
+    assert max(units) - min(units) <= 1  # whole units spread evenly; the last block adds the rest
+    assert shard.shard_bounds(n, world, 0, 1) == shard.shard_bounds(n, world, 0)  # align 1: the plain split
+
+
+@pytest.mark.parametrize("n,world,k,pi,S", [(131072, 3, 512, 1024, 16), (6000, 4, 100, 64, 16),
+                                             (5000, 3, 300, 256, 1)])
+def test_aligned_halo_plan_covers_the_rows_from_a_whole_period(n, world, k, pi, S):
+    plan = shard.halo_plan(n, world, k, pi, S, align=pi)
+    for dst in range(world):
+        s0, s1 = shard.shard_bounds(n, world, dst, pi)
+        kv0 = shard.halo_start(s0, s1, k, pi, S, pi)
+        assert kv0 % pi == 0 and kv0 <= max(0, s0 - shard.reach(k, pi, S))
+        rows = [r for src, d, g0, g1 in plan if d == dst for r in range(g0, g1)]
+        assert rows == (list(range(kv0, s0)) if s1 > s0 else [])
+
+
 def test_reach_counts_skips_only_outside_the_window():
     assert shard.reach(128, 64, 4) == 256        # skips m = 3, 4 exist: back to 4 * 64
     assert shard.reach(128, 64, 2) == 128        # m0 = 3 > S: no skip, the window only
