@@ -632,13 +632,17 @@ def run_shard(args):
     lse = torch.empty((w.B, w.H, s1 - s0), dtype=torch.float32, device=device)
     stream = torch.cuda.current_stream(device)
 
+    # the split path's skip partials: one workspace for every step (nothing allocated inside a step)
+    need = pia.load().pi_attn_fwd_shard_scratch_bytes(w.B, w.H, s1 - s0, s0, kv0, w.d, w.k, w.pi, w.S)
+    ws = torch.empty(max(need, 16), dtype=torch.uint8, device=device)
+
     def step():
         if world > 1:
             k_ext, v_ext, kv = shard.exchange_halo(t["k"], t["v"], w.n, w.k, w.pi, w.S, align=w.pi)
         else:
             k_ext, v_ext, kv = t["k"], t["v"], 0
         pia.pi_attn_fwd_shard(t["q"], k_ext.contiguous(), v_ext.contiguous(), t["w_g"], t["b_g"], w.k, w.pi, w.S, s0,
-                              kv, out=out, lse=lse)
+                              kv, out=out, lse=lse, workspace=ws)
 
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
     flush_rd = torch.zeros(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=device)

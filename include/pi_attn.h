@@ -119,6 +119,19 @@ pi_attn_status pi_attn_fwd_shard(const void* q, const void* k, const void* v, co
                                  void* out, float* lse, int B, int H, int n_q, int n_kv, long long row0,
                                  long long kv0, int d, int k_win, int pi, int S, pi_attn_dtype dtype, void* stream);
 
+/* pi_attn_fwd_shard with a caller-provided device workspace for the split path's skip partials
+ * (16-byte aligned, owned by the caller; at least pi_attn_fwd_shard_scratch_bytes bytes; NULL =
+ * allocate as pi_attn_fwd_shard does), so that the call allocates nothing.  Errors as
+ * pi_attn_fwd_shard, plus PI_ATTN_EINVAL for a misaligned or too small workspace. */
+pi_attn_status pi_attn_fwd_shard_ws(const void* q, const void* k, const void* v, const float* w_g, const float* b_g,
+                                    void* out, float* lse, int B, int H, int n_q, int n_kv, long long row0,
+                                    long long kv0, int d, int k_win, int pi, int S, pi_attn_dtype dtype,
+                                    void* workspace, long long workspace_bytes, void* stream);
+/* Scratch bytes a shard call with these arguments takes: B*H*n_q*(2d + 4) where it runs the split
+ * path, 0 where it runs the single pass; -1 for invalid sizes. */
+long long pi_attn_fwd_shard_scratch_bytes(int B, int H, int n_q, long long row0, long long kv0, int d, int k_win,
+                                          int pi, int S);
+
 /* Bidirectional prefill forward (the non-causal variant).  Cited passage: the Core Components of
  * the pi-Attention method section -- the local neighbourhood reaches both forward and backward,
  * and in bidirectional settings the skips also reach i + pi.  Row i of a sequence of n tokens

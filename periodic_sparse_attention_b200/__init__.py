@@ -29,6 +29,11 @@ SIGNATURES = {
     "pi_attn_fwd_ex": (_i32, [_vp] * 7 + [_i32] * 9 + [_vp]),
     # 7 tensor pointers, B H n_q n_kv, row0 kv0 (int64), d k_win pi S, dtype, stream
     "pi_attn_fwd_shard": (_i32, [_vp] * 7 + [_i32] * 4 + [ctypes.c_longlong] * 2 + [_i32] * 5 + [_vp]),
+    # ... plus workspace pointer and bytes before the stream
+    "pi_attn_fwd_shard_ws": (_i32, [_vp] * 7 + [_i32] * 4 + [ctypes.c_longlong] * 2 + [_i32] * 5 +
+                             [_vp, ctypes.c_longlong, _vp]),
+    # B H n_q, row0 kv0 (int64), d k_win pi S
+    "pi_attn_fwd_shard_scratch_bytes": (ctypes.c_longlong, [_i32] * 3 + [ctypes.c_longlong] * 2 + [_i32] * 4),
     # as pi_attn_fwd_ex, bidirectional index rule
     "pi_attn_fwd_bidir": (_i32, [_vp] * 7 + [_i32] * 9 + [_vp]),
     # ... plus workspace pointer and its size in bytes
@@ -161,10 +166,11 @@ def pi_attn_fwd(q, k, v, w_g, b_g, k_win: int, pi: int, S: int, out=None, lse=No
 
 
 def pi_attn_fwd_shard(q, k, v, w_g, b_g, k_win: int, pi: int, S: int, row0: int, kv0: int, out=None, lse=None, *,
-                      stream=None, want_lse: bool = True):
+                      stream=None, want_lse: bool = True, workspace=None):
     """One shard of a causal prefill: q [B, H, n_q, d] holds sequence rows row0 .., k and v
     [B, H, n_kv, d] hold sequence rows kv0 .. (the halo, then the shard's rows).  bf16, d in
-    {64, 128}.  Allocates out and lse when not given."""
+    {64, 128}.  Allocates out and lse when not given, and the split path's workspace (a uint8
+    tensor of pi_attn_fwd_shard_scratch_bytes) from torch's caching allocator when not given."""
     import torch
     B, H, n_q, d = q.shape
     n_kv = k.shape[2]
@@ -172,8 +178,14 @@ def pi_attn_fwd_shard(q, k, v, w_g, b_g, k_win: int, pi: int, S: int, row0: int,
         out = torch.empty_like(q)
     if lse is None and want_lse:
         lse = torch.empty((B, H, n_q), dtype=torch.float32, device=q.device)
-    st = load().pi_attn_fwd_shard(_ptr(q), _ptr(k), _ptr(v), _ptr(w_g), _ptr(b_g), _ptr(out), _ptr(lse), B, H, n_q,
-                                  n_kv, row0, kv0, d, k_win, pi, S, _dtype_code(q), _stream(stream))
+    if workspace is None:
+        need = load().pi_attn_fwd_shard_scratch_bytes(B, H, n_q, row0, kv0, d, k_win, pi, S)
+        if need > 0:
+            workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    st = load().pi_attn_fwd_shard_ws(_ptr(q), _ptr(k), _ptr(v), _ptr(w_g), _ptr(b_g), _ptr(out), _ptr(lse), B, H, n_q,
+                                     n_kv, row0, kv0, d, k_win, pi, S, _dtype_code(q), _ptr(workspace), ws_bytes,
+                                     _stream(stream))
     _raise(st)
     return out, lse
 

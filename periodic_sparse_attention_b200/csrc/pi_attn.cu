@@ -431,9 +431,16 @@ pi_attn_status pi_attn_fwd_bidir(const void* q, const void* k, const void* v, co
   return fwd_impl(q, k, v, w_g, b_g, out, lse, B, H, n, d, k_win, pi, S, dtype, path, true, nullptr, 0, stream);
 }
 
-pi_attn_status pi_attn_fwd_shard(const void* q, const void* k, const void* v, const float* w_g, const float* b_g,
-                                 void* out, float* lse, int B, int H, int n_q, int n_kv, long long row0,
-                                 long long kv0, int d, int k_win, int pi, int S, pi_attn_dtype dtype, void* stream) {
+long long pi_attn_fwd_shard_scratch_bytes(int B, int H, int n_q, long long row0, long long kv0, int d, int k_win,
+                                          int pi, int S) {
+  if (B < 1 || H < 1 || n_q < 1 || d < 1 || row0 < 0 || kv0 < 0 || k_win < 0 || pi < 1 || S < 0) return -1;
+  return pia::shard_split_applies(n_q, row0, kv0, k_win, pi, S) ? (long long)B * H * n_q * (2LL * d + 4) : 0;
+}
+
+pi_attn_status pi_attn_fwd_shard_ws(const void* q, const void* k, const void* v, const float* w_g, const float* b_g,
+                                    void* out, float* lse, int B, int H, int n_q, int n_kv, long long row0,
+                                    long long kv0, int d, int k_win, int pi, int S, pi_attn_dtype dtype,
+                                    void* workspace, long long workspace_bytes, void* stream) {
   pi_attn_status st = check_common(q, k, v, w_g, b_g, out, B, H, n_kv, d, k_win, pi, S, dtype);
   if (st != PI_ATTN_OK) return st;
   if (n_q < 1) return fail(PI_ATTN_EINVAL, "n_q must be >= 1 (got %d)", n_q);
@@ -457,12 +464,38 @@ pi_attn_status pi_attn_fwd_shard(const void* q, const void* k, const void* v, co
   if ((long long)B * H > kMaxGridY)
     return fail(PI_ATTN_EUNSUPPORTED, "the shard forward takes at most %lld (b, h) pairs a call (got %lld)", kMaxGridY,
                 (long long)B * H);
+  // the split path (residue pass, band-merge pass, tail) where the shard's rows and halo start on
+  // whole periods, its skip partials in the caller's workspace (else cudaMallocAsync on `stream`)
+  const bool split = pia::shard_split_applies(n_q, row0, kv0, k_win, pi, S);
+  if (workspace) {
+    if (reinterpret_cast<uintptr_t>(workspace) % 16 != 0) return fail(PI_ATTN_EINVAL, "workspace not 16-byte aligned");
+    const long long need = split ? (long long)B * H * n_q * (2LL * d + 4) : 0;
+    if (workspace_bytes < need)
+      return fail(PI_ATTN_EINVAL, "workspace of %lld bytes, the shard needs %lld", workspace_bytes, need);
+  }
   const char* why = "";
-  cudaError_t e = d == 128 ? pia::launch_fwd_tc_shard_d<128>(q, k, v, w_g, b_g, out, lse, B, H, n_q, n_kv, row0, kv0,
-                                                             k_win, pi, S, as_stream(stream), &why)
-                           : pia::launch_fwd_tc_shard_d<64>(q, k, v, w_g, b_g, out, lse, B, H, n_q, n_kv, row0, kv0,
-                                                            k_win, pi, S, as_stream(stream), &why);
+  const cudaStream_t s = as_stream(stream);
+  cudaError_t e;
+  if (split)
+    e = d == 128 ? pia::launch_fwd_tc_d<128>(q, k, v, w_g, b_g, out, lse, B, H, n_q, k_win, pi, S, true, false,
+                                             workspace, s, &why, nullptr, nullptr, nullptr, nullptr, nullptr, row0,
+                                             kv0, n_kv)
+                 : pia::launch_fwd_tc_d<64>(q, k, v, w_g, b_g, out, lse, B, H, n_q, k_win, pi, S, true, false,
+                                            workspace, s, &why, nullptr, nullptr, nullptr, nullptr, nullptr, row0,
+                                            kv0, n_kv);
+  else
+    e = d == 128 ? pia::launch_fwd_tc_shard_d<128>(q, k, v, w_g, b_g, out, lse, B, H, n_q, n_kv, row0, kv0, k_win,
+                                                   pi, S, s, &why)
+                 : pia::launch_fwd_tc_shard_d<64>(q, k, v, w_g, b_g, out, lse, B, H, n_q, n_kv, row0, kv0, k_win, pi,
+                                                  S, s, &why);
   return e == cudaSuccess ? ok() : cuda_fail(e, why);
+}
+
+pi_attn_status pi_attn_fwd_shard(const void* q, const void* k, const void* v, const float* w_g, const float* b_g,
+                                 void* out, float* lse, int B, int H, int n_q, int n_kv, long long row0,
+                                 long long kv0, int d, int k_win, int pi, int S, pi_attn_dtype dtype, void* stream) {
+  return pi_attn_fwd_shard_ws(q, k, v, w_g, b_g, out, lse, B, H, n_q, n_kv, row0, kv0, d, k_win, pi, S, dtype, nullptr,
+                              0, stream);
 }
 
 pi_attn_status pi_attn_fwd_ex(const void* q, const void* k, const void* v, const float* w_g, const float* b_g,

@@ -277,3 +277,18 @@ def test_backward_host_entry_workspace_size_and_argument_checks(lib):
     assert call(nbytes=need - 1) == pia.PI_ATTN_EINVAL
     assert call(path=pia.BWD_PATHS["tc_split"], bidir=1) == pia.PI_ATTN_EUNSUPPORTED
     assert call(path=pia.BWD_PATHS["tc_split"], n=250) == pia.PI_ATTN_EUNSUPPORTED  # n % pi != 0
+
+
+def test_shard_scratch_and_workspace_checks_before_any_launch(lib):
+    # the split path's scratch where the shard's rows and halo start on whole periods; none otherwise
+    B, H, d = 1, 32, 128
+    assert lib.pi_attn_fwd_shard_scratch_bytes(B, H, 16384, 16384, 0, d, 512, 1024, 16) == B * H * 16384 * (2 * d + 4)
+    assert lib.pi_attn_fwd_shard_scratch_bytes(B, H, 16384, 16000, 0, d, 512, 1024, 16) == 0     # row0 off a period
+    assert lib.pi_attn_fwd_shard_scratch_bytes(B, H, 16384, 16384, 100, d, 512, 1024, 16) == 0   # halo off a period
+    assert lib.pi_attn_fwd_shard_scratch_bytes(B, H, 4096, 0, 0, 64, 128, 64, 4) == 0            # single pass shape
+    assert lib.pi_attn_fwd_shard_scratch_bytes(0, H, 16, 0, 0, d, 1, 1, 1) == -1
+    need = lib.pi_attn_fwd_shard_scratch_bytes(1, 2, 2048, 2048, 0, 64, 128, 256, 16)
+    assert need > 0
+    args = [FAKE] * 7 + [1, 2, 2048, 4096, 2048, 0, 64, 128, 256, 16, pia.PI_ATTN_BF16]
+    assert lib.pi_attn_fwd_shard_ws(*args, ctypes.c_void_p(0x10008), need, None) == pia.PI_ATTN_EINVAL  # misaligned
+    assert lib.pi_attn_fwd_shard_ws(*args, FAKE, need - 1, None) == pia.PI_ATTN_EINVAL  # one byte short

@@ -121,3 +121,27 @@ def test_shards_on_whole_periods_take_the_split_path_and_match_the_oracle():
     ro, rl = oracle.fwd(q, k, v, w_g, b_g, kw, pi, S)[:2]
     assert_close(metrics(from_dev(out).reshape(-1, d), ro.reshape(-1, d), lse.cpu().numpy().astype(np.float64).reshape(-1),
                          rl.reshape(-1)), "bf16", "aligned shards")
+
+
+def test_shard_with_a_workspace_gives_the_same_bits():
+    # pi_attn_fwd_shard_ws with the caller's workspace and pi_attn_fwd_shard with its own scratch:
+    # the same launches, the same bits (a shard of whole periods with a halo: the split path)
+    import ctypes
+    B, H, n, d, kw, pi, S = 1, 2, 8192, 64, 128, 256, 16
+    q, k, v, w_g, b_g = _inputs(B, H, n, d, seed=23)
+    qt, kt, vt = to_dev(q, "bf16"), to_dev(k, "bf16"), to_dev(v, "bf16")
+    wg, bg = torch.from_numpy(w_g).cuda(), torch.from_numpy(b_g).cuda()
+    s0, s1, kv0 = 4096, 8192, 0
+    need = pia.load().pi_attn_fwd_shard_scratch_bytes(B, H, s1 - s0, s0, kv0, d, kw, pi, S)
+    assert need > 0
+    qs, ks, vs = qt[:, :, s0:s1].contiguous(), kt[:, :, kv0:s1].contiguous(), vt[:, :, kv0:s1].contiguous()
+    o1, l1 = pia.pi_attn_fwd_shard(qs, ks, vs, wg, bg, kw, pi, S, s0, kv0)  # the binding's workspace
+    o2, l2 = torch.empty_like(o1), torch.empty_like(l1)
+    P = lambda t: ctypes.c_void_p(t.data_ptr())  # noqa: E731
+    st = pia.load().pi_attn_fwd_shard(P(qs), P(ks), P(vs), P(wg), P(bg), P(o2), P(l2), B, H, s1 - s0, s1 - kv0, s0,
+                                      kv0, d, kw, pi, S, pia.PI_ATTN_BF16,
+                                      ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))  # its own scratch
+    assert st == pia.PI_ATTN_OK, pia.load().pi_attn_last_error()
+    pia.pi_attn_check()
+    assert torch.equal(o1.view(torch.int16), o2.view(torch.int16))
+    assert torch.equal(l1, l2)
