@@ -781,8 +781,8 @@ def run_reference(args):
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
-    # 50 timed steps: short enough that the GPU stays at its full clock (the burst figures of the
-    # measured peaks are the denominators); a 200-step run settles under the power cap
+    # 50 timed steps: closer to the full clock that the burst figures of the measured peaks assume
+    # (a 200-step run of the long-context prefill settles deeper under the power cap)
     ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(ps.WORKLOADS))
